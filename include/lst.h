@@ -1,0 +1,165 @@
+/*
+ * lst.h -- layer-streamed LoRA fine-tuning on one GPU: the C ABI of liblst.so.
+ *
+ * What it computes (sources by page title and section):
+ *  - "Soup: Fine-Tuning an 8B Model on a 4 GB Laptop GPU, One Layer at a Time" (toknow.ai),
+ *    first paragraph: the frozen base stays in CPU RAM and is copied to the GPU one layer at a
+ *    time, double-buffered so the next layer loads while the current one computes; the base can
+ *    be 4-bit (NF4) or unquantised 16-bit; second paragraph: the forward pass is bit-exact
+ *    against a resident run.
+ *  - Tutorial "Fine-tune Llama 3.1 8B on a 4GB GPU with Soup" (lachieslifestyle.com), section
+ *    "What Soup layer streaming changes": a two-buffer VRAM pool; each decoder layer is read in
+ *    the forward pass and read again for backward recomputation; LoRA adapters stay on the GPU.
+ *  - "Soup CLI fine-tunes Llama-3.1-8B on a 4 GB laptop GPU, ..." (thetesserapress.com),
+ *    second paragraph: copies run on a dedicated CUDA stream; logits stay resident.
+ *  - "Fine-Tuning an 8B Parameter Model on a 4 GB Laptop GPU" (codeinktechnologies.com),
+ *    sections "Quantization" (NF4 with nested quantisation of the constants) and "LoRA and
+ *    QLoRA" (frozen quantised base, full-precision adapters).
+ *
+ * One step = embedding -> L pre-norm decoder layers (RMSNorm, q/k/v with RoPE, causal GQA
+ * attention, o, RMSNorm, SwiGLU MLP; every projection y = x W^T + (alpha/r) (x A^T) B^T) ->
+ * final RMSNorm -> LM head -> mean cross-entropy, then the analytic backward with each layer
+ * recomputed from its saved input. Outputs: the loss and dL/dA, dL/dB of every adapter.
+ *
+ * Conventions
+ *  - Every call returns an lst_status; no exception or abort crosses the ABI. After a non-OK
+ *    status, lst_last_error(ctx) describes it (valid until the next call on ctx).
+ *  - Matrices are row-major; a projection's W is [out, in], its A is [r, in], its B is [out, r].
+ *  - Projection order everywhere: q, k, v, o, gate, up, down (LST_PROJ_*).
+ *  - Pointer arguments may be host or device memory unless stated; the library detects which.
+ *    The library copies what it needs before returning; the caller keeps ownership.
+ *  - A context is bound to the device current at lst_create and is not thread-safe.
+ *  - Device faults are never used for error reporting: device code records an error word that
+ *    the host turns into LST_ERR_DEVICE, and waits are bounded (LST_ERR_TIMEOUT).
+ */
+#ifndef LST_H_
+#define LST_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct lst_ctx lst_ctx;
+
+typedef enum {
+  LST_OK = 0,
+  LST_ERR_ARG = 1,      /* bad argument: null pointer, shape beyond the config, bad index */
+  LST_ERR_STATE = 2,    /* call out of order: e.g. a step before every layer is registered */
+  LST_ERR_OOM = 3,      /* device or pinned host allocation failed */
+  LST_ERR_CUDA = 4,     /* a CUDA runtime call failed */
+  LST_ERR_TIMEOUT = 5,  /* the step did not complete within timeout_ms */
+  LST_ERR_DEVICE = 6    /* device code reported an error (bad token id, a bounded wait ran out) */
+} lst_status;
+
+enum { LST_BASE_NF4 = 0, LST_BASE_BF16 = 1 };
+enum {
+  LST_PROJ_Q = 0, LST_PROJ_K = 1, LST_PROJ_V = 2, LST_PROJ_O = 3,
+  LST_PROJ_GATE = 4, LST_PROJ_UP = 5, LST_PROJ_DOWN = 6, LST_NUM_PROJ = 7
+};
+
+typedef struct {
+  int32_t n_layers;     /* L >= 1 */
+  int32_t d_model;      /* d, multiple of 8 */
+  int32_t n_heads;      /* hq */
+  int32_t n_kv_heads;   /* hkv, divides hq */
+  int32_t head_dim;     /* 64 or 128 */
+  int32_t ffn;          /* F, multiple of 8 */
+  int32_t vocab;        /* V; 0 = headless stack (use lst_step_hidden) */
+  float rms_eps;
+  float rope_theta;     /* rotate-half RoPE, angle pos * theta^(-2j/hd) */
+  int32_t qkv_bias;     /* 1: q, k, v projections carry a frozen bias */
+  int32_t lora_rank;    /* r; 3*r <= 64 */
+  float lora_alpha;     /* LoRA scale s = alpha / r */
+  int32_t base_format;  /* LST_BASE_NF4: 4-bit NF4, blocks of 64, absmax double-quantised to
+                           int8 in groups of 256; LST_BASE_BF16: unquantised bf16 */
+  int32_t max_batch;
+  int32_t max_seq;
+  int32_t streamed;     /* 1: base in pinned host RAM, copied per layer read into a two-buffer
+                           device pool on a dedicated copy stream; 0: all layers resident on the
+                           device (same kernels, same results) */
+  int32_t timeout_ms;   /* host-side wait limit of one step; <= 0 means 600000 */
+} lst_config;
+
+typedef struct {
+  const float* w[LST_NUM_PROJ];       /* frozen base W [out, in] fp32 */
+  const float* bias[3];               /* q, k, v bias [out] fp32; required iff qkv_bias */
+  const float* attn_norm;             /* RMSNorm gains before attention [d] fp32 */
+  const float* mlp_norm;              /* RMSNorm gains before the MLP [d] fp32 */
+  const float* lora_a[LST_NUM_PROJ];  /* A [r, in] fp32 */
+  const float* lora_b[LST_NUM_PROJ];  /* B [out, r] fp32 */
+} lst_layer_weights;
+
+typedef struct {
+  int64_t steps;               /* completed steps */
+  int64_t launches_last_step;  /* kernels launched by the last step */
+  int64_t layer_reads_last_step; /* layer blobs copied host -> device by the last step (2L) */
+  int64_t h2d_bytes_last_step; /* bytes of layer copies of the last step */
+  int64_t blob_bytes;          /* bytes of one layer's frozen base as stored */
+  int64_t arena_bytes;         /* pinned host bytes (streamed) or device bytes (resident) of the base */
+  int64_t device_bytes;        /* device bytes allocated by the context */
+  /* filled when profiling is on (lst_set_profiling): device time of the last step by class */
+  double gemm_ms, attention_ms, dequant_ms, other_ms, copy_ms, step_ms;
+  int64_t gemm_launches, attention_launches, dequant_launches, copy_count;
+  double gemm_flops;           /* algorithmic FLOPs of the GEMM launches of the last step */
+} lst_stats;
+
+/* Create a context. embed [V, d], final_norm [d], lm_head [V, d] are fp32 (host or device; the
+ * library rounds E and H to bf16 and keeps them resident); all three must be NULL iff vocab == 0.
+ * cuda_stream: cudaStream_t the steps run on, or NULL for a stream owned by the context.
+ * Errors: LST_ERR_ARG (bad config), LST_ERR_OOM, LST_ERR_CUDA. On error *out is NULL. */
+lst_status lst_create(const lst_config* cfg, const float* embed, const float* final_norm,
+                      const float* lm_head, void* cuda_stream, lst_ctx** out);
+
+/* Register layer `layer` (0 <= layer < L): quantise (NF4) or round (bf16) the base on the device,
+ * lay it out as one contiguous blob, store it in the pinned arena (streamed) or on the device
+ * (resident), and copy the LoRA A, B into resident device memory. May be called again to replace
+ * a layer. Synchronous. Errors: LST_ERR_ARG, LST_ERR_OOM, LST_ERR_CUDA. */
+lst_status lst_register_layer(lst_ctx* ctx, int32_t layer, const lst_layer_weights* w);
+
+/* Replace the adapters of one projection (A [r, in], B [out, r] fp32). */
+lst_status lst_set_lora(lst_ctx* ctx, int32_t layer, int32_t proj, const float* a, const float* b);
+
+/* Number of fp32 values in the gradient (and parameter) layout: for each layer, for each
+ * projection in LST_PROJ order, dA [r, in] then dB [out, r]. */
+int64_t lst_lora_numel(const lst_ctx* ctx);
+
+/* One forward + backward step of the model with a head: tokens and targets are int32
+ * [batch * seq] (host or device), the loss is the mean cross-entropy over all tokens (written to
+ * *loss, host memory). grads (host or device, may be NULL) receives lst_lora_numel() fp32 values.
+ * Requires vocab > 0, every layer registered (else LST_ERR_STATE), batch <= max_batch,
+ * seq <= max_seq. Blocks until the step is done or timeout_ms passed (LST_ERR_TIMEOUT). */
+lst_status lst_step(lst_ctx* ctx, const int32_t* tokens, const int32_t* targets, int32_t batch,
+                    int32_t seq, float* loss, float* grads);
+
+/* Headless step of the decoder stack: x and g are bf16 bit patterns [batch * seq, d] (host or
+ * device); the loss is sum(x_L * g) over all elements, so dL/dx_L = g. Same outputs and rules as
+ * lst_step; requires vocab == 0. */
+lst_status lst_step_hidden(lst_ctx* ctx, const uint16_t* x, const uint16_t* g, int32_t batch,
+                           int32_t seq, float* loss, float* grads);
+
+/* Copy the last step's logits [batch * seq, V] fp32 to dst (host or device). */
+lst_status lst_get_logits(lst_ctx* ctx, float* dst);
+
+/* Record per-class device times of every step (CUDA events around each launch) when on != 0. */
+lst_status lst_set_profiling(lst_ctx* ctx, int32_t on);
+lst_status lst_get_stats(const lst_ctx* ctx, lst_stats* out);
+
+const char* lst_last_error(const lst_ctx* ctx);
+
+/* Free everything the context owns. NULL-safe. */
+void lst_destroy(lst_ctx* ctx);
+
+/* The 16 NF4 values (fp32, ascending) the library quantises with: 8 positive and 7 negative
+ * standard-normal quantiles and an exact 0, scaled to [-1, 1]. Needs no GPU. */
+lst_status lst_nf4_codebook(float out[16]);
+
+/* Bytes of one layer blob for a config (needs no GPU). */
+int64_t lst_blob_bytes(const lst_config* cfg);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LST_H_ */

@@ -1,0 +1,95 @@
+/*
+ * lst_kernels.h -- the individual device kernels of liblst.so behind a C ABI, so each can be
+ * checked on its own against the CPU oracle. All pointers are DEVICE pointers unless stated;
+ * `stream` is a cudaStream_t (NULL = legacy default stream). Calls enqueue work and return
+ * without synchronising; errors in the arguments return LST_ERR_ARG before anything is
+ * launched, a failed launch returns LST_ERR_CUDA. bf16 buffers are passed as uint16_t bits.
+ */
+#ifndef LST_KERNELS_H_
+#define LST_KERNELS_H_
+
+#include <stdint.h>
+
+#include "lst.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* NF4 quantisation of w [n] fp32 (n a multiple of 64), as defined in "Fine-Tuning an 8B Parameter
+ * Model on a 4 GB Laptop GPU", section "Quantization" (NF4 + nested quantisation; construction
+ * after QLoRA): packed [n/2] (element 2i in the high nibble), qabs [n/64] int8,
+ * gscale [ceil(n/64/256)] fp32, mean [1] fp32. Allocates and frees its own scratch. */
+lst_status lst_k_nf4_quantize(const float* w, int64_t n, uint8_t* packed, int8_t* qabs,
+                              float* gscale, float* mean, void* stream);
+
+/* Dequantise one NF4 tensor into bf16 [n]: a^ = (q * s) / 127 + mean, w^ = bf16(code * a^),
+ * each operation one fp32 rounding; bit-exact by construction. */
+lst_status lst_k_nf4_dequant(const uint8_t* packed, const int8_t* qabs, const float* gscale,
+                             const float* mean, int64_t n, uint16_t* out, void* stream);
+
+/* C = alpha * (A B' + A2 B2') + bias + R on the tcgen05 tensor cores (fp32 accumulate).
+ * A [M, K] row stride lda; B' = B^T with B [N, K] (b_mn = 0) or B' = B with B [K, N] (b_mn = 1),
+ * row stride ldb; (A2 [M, K2], B2) optional second pair of the same major-ness (NULL to skip);
+ * C [M, N] fp32 (c_f32 = 1) or bf16; bias [N] fp32 or NULL; R [M, N] bf16 or NULL.
+ * Leading dimensions must be multiples of 8 and A/B/A2/B2 16-byte aligned. */
+lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda,
+                      const uint16_t* B, int64_t ldb, int32_t b_mn, const uint16_t* A2,
+                      int64_t lda2, const uint16_t* B2, int64_t ldb2, int32_t K2, void* C,
+                      int64_t ldc, int32_t c_f32, float alpha, const float* bias,
+                      const uint16_t* R, int64_t ldr, void* stream);
+
+/* Causal GQA attention forward over T = batch*S tokens: q [T, ldq], k [T, ldk], v [T, ldv]
+ * (head h at column h*hd), o [T, ldo] bf16, lse [T, hq] fp32. hd in {64, 128}. */
+lst_status lst_k_attention_fwd(const uint16_t* q, int64_t ldq, const uint16_t* k, int64_t ldk,
+                               const uint16_t* v, int64_t ldv, uint16_t* o, int64_t ldo,
+                               float* lse, int64_t T, int32_t S, int32_t hq, int32_t hkv,
+                               int32_t hd, void* stream);
+
+/* Attention backward: dq [T, lddq], dk [T, lddk], dv [T, lddv] bf16 from dout [T, lddo] and the
+ * forward's o and lse; D is scratch [T, hq] fp32. Deterministic (no atomics). */
+lst_status lst_k_attention_bwd(const uint16_t* q, int64_t ldq, const uint16_t* k, int64_t ldk,
+                               const uint16_t* v, int64_t ldv, const uint16_t* o, int64_t ldo,
+                               const uint16_t* dout, int64_t lddo, const float* lse, float* D,
+                               uint16_t* dq, int64_t lddq, uint16_t* dk, int64_t lddk,
+                               uint16_t* dv, int64_t lddv, int64_t T, int32_t S, int32_t hq,
+                               int32_t hkv, int32_t hd, void* stream);
+
+/* RMSNorm forward: y = bf16(x * rstd * g), rstd [T]. */
+lst_status lst_k_rmsnorm_fwd(const uint16_t* x, const float* g, int64_t T, int32_t d, float eps,
+                             uint16_t* y, float* rstd, void* stream);
+/* RMSNorm backward: dx = dres + rstd (dy g - xhat mean(dy g xhat)); dres and dx_bf16 may be NULL. */
+lst_status lst_k_rmsnorm_bwd(const float* dy, const uint16_t* x, const float* g,
+                             const float* rstd, const float* dres, int64_t T, int32_t d,
+                             float* dx, uint16_t* dx_bf16, void* stream);
+
+/* RoPE in place on nh heads starting at column col0 of buf [T, ld]; cos/sin tables [S, hd/2]
+ * from lst_k_rope_tables; inverse != 0 applies the transpose (backward). */
+lst_status lst_k_rope_tables(int32_t S, int32_t hd, double theta, float* cos_t, float* sin_t,
+                             void* stream);
+lst_status lst_k_rope(uint16_t* buf, int64_t ld, int64_t T, int32_t S, int32_t col0, int32_t nh,
+                      int32_t hd, const float* cos_t, const float* sin_t, int32_t inverse,
+                      void* stream);
+
+/* SwiGLU: m = silu(g) * u with gu = [g | u] [T, 2F]; backward gives dgu [T, 2F] from dm fp32. */
+lst_status lst_k_swiglu_fwd(const uint16_t* gu, int64_t T, int32_t F, uint16_t* m, void* stream);
+lst_status lst_k_swiglu_bwd(const float* dm, const uint16_t* gu, int64_t T, int32_t F,
+                            uint16_t* dgu, void* stream);
+
+/* Cross-entropy rows over fp32 logits [T, V]: loss_rows [T], dlogits bf16 [T, V] scaled by inv_T. */
+lst_status lst_k_cross_entropy(const float* logits, int64_t T, int32_t V, const int32_t* targets,
+                               float inv_T, float* loss_rows, uint16_t* dlogits, void* stream);
+
+/* LoRA down-projection U = X A^T (A fp32 [R, in]); U fp32 [T, R], Us = bf16(s U) [T, ldus]. */
+lst_status lst_k_lora_project(const uint16_t* X, int64_t ldx, int64_t T, int32_t in,
+                              const float* A, int32_t R, float s, float* U, uint16_t* Us,
+                              int64_t ldus, void* stream);
+
+/* Kernel launches made by this library so far in this process (all contexts). Needs no GPU. */
+int64_t lst_k_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LST_KERNELS_H_ */

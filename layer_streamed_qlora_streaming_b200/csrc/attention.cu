@@ -1,0 +1,499 @@
+// Causal grouped-query attention, forward and deterministic backward, on the warp-level tensor-core
+// path (mma.sync m16n8k16 bf16 -> fp32) with online softmax, never materialising the S x S scores.
+//
+//   o = softmax(q k^T / sqrt(hd) + causal mask) v ; query head h reads kv head h / (hq / hkv)
+//
+// Layouts: q/k/v/o are rows of token-major matrices (token t = b * S + s); head h of a row starts
+// at column h * hd; row strides are arguments so q, k, v can live side by side in one fused qkv
+// buffer. lse and D are [T, hq] fp32. The backward is split in two kernels so that nothing is
+// accumulated with atomics: dK/dV (one CTA per kv block, summing the query heads of its group in
+// order) and dQ (one CTA per query block).
+#include "attention.cuh"
+#include "common.cuh"
+
+namespace lst {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Shared tile of `rows` x HD bf16 with a 16-byte row pad (conflict-free ldmatrix).
+template <int HD>
+struct Tile {
+  static constexpr int LD = HD + 8;
+};
+
+// Cooperative load of rows [r0, r0+nrows) of one head into a shared tile; rows outside [0, S)
+// of the sequence are zero.
+template <int HD>
+__device__ __forceinline__ void load_tile(__nv_bfloat16* sm, const __nv_bfloat16* g, int64_t ld, int64_t tok0,
+                                          int r0, int nrows, int S, int col) {
+  constexpr int V = HD / 8;  // 16-byte vectors per row
+  for (int i = threadIdx.x; i < nrows * V; i += blockDim.x) {
+    const int r = i / V, c = (i % V) * 8;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (r0 + r < S) val = *reinterpret_cast<const uint4*>(g + (tok0 + r0 + r) * ld + col + c);
+    *reinterpret_cast<uint4*>(sm + r * Tile<HD>::LD + c) = val;
+  }
+}
+
+// A fragment (16 rows x 16 k) at (row0, k0) of a shared tile.
+template <int HD>
+__device__ __forceinline__ void lda_frag(uint32_t (&a)[4], const __nv_bfloat16* sm, int row0, int k0) {
+  const int l = threadIdx.x & 31;
+  const int r = row0 + (l & 7) + ((l >> 3) & 1) * 8;
+  const int c = k0 + (l >> 4) * 8;
+  ldsm4(a, smem_u32(sm + r * Tile<HD>::LD + c));
+}
+// B fragments for two n-tiles (n0, n0+8) x k-step k0 where B(k, n) = tile[n][k] (rows are n).
+template <int HD>
+__device__ __forceinline__ void ldb_rows(uint32_t (&b)[4], const __nv_bfloat16* sm, int n0, int k0) {
+  const int l = threadIdx.x & 31;
+  const int r = n0 + (l & 7) + (l >> 4) * 8;
+  const int c = k0 + ((l >> 3) & 1) * 8;
+  ldsm4(b, smem_u32(sm + r * Tile<HD>::LD + c));
+}
+// B fragments for two n-tiles (n0, n0+8) x k-step k0 where B(k, n) = tile[k][n] (rows are k).
+template <int HD>
+__device__ __forceinline__ void ldb_trans(uint32_t (&b)[4], const __nv_bfloat16* sm, int k0, int n0) {
+  const int l = threadIdx.x & 31;
+  const int r = k0 + (l & 7) + ((l >> 3) & 1) * 8;
+  const int c = n0 + (l >> 4) * 8;
+  ldsm4t(b, smem_u32(sm + r * Tile<HD>::LD + c));
+}
+
+// ------------------------------------------------------------------------------------ forward
+// grid (ceil(S/64), hq, B), 128 threads; warp w owns query rows 16w..16w+15 of the block.
+template <int HD>
+__global__ void __launch_bounds__(128) k_attn_fwd(AttnArgs p) {
+  extern __shared__ __align__(16) uint8_t sm_raw[];
+  __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(sm_raw);
+  __nv_bfloat16* Ks = Qs + 64 * Tile<HD>::LD;
+  __nv_bfloat16* Vs = Ks + 64 * Tile<HD>::LD;
+  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / (p.hq / p.hkv);
+  const int64_t tok0 = (int64_t)b * p.S;
+  const int q0 = qb * 64;
+  const int warp = threadIdx.x >> 5, l = threadIdx.x & 31, g = l >> 2, t4 = l & 3;
+  const float sl2 = p.scale * kLog2e;
+
+  load_tile<HD>(Qs, p.q, p.ldq, tok0, q0, 64, p.S, h * HD);
+
+  float o[HD / 8][4];
+#pragma unroll
+  for (int i = 0; i < HD / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+  const int qr0 = q0 + warp * 16 + g, qr1 = qr0 + 8;  // this thread's two query rows
+  const int nkb = min(qb, (p.S - 1) / 64) + 1;
+
+  for (int kb = 0; kb < nkb; ++kb) {
+    __syncthreads();
+    load_tile<HD>(Ks, p.k, p.ldk, tok0, kb * 64, 64, p.S, kvh * HD);
+    load_tile<HD>(Vs, p.v, p.ldv, tok0, kb * 64, 64, p.S, kvh * HD);
+    __syncthreads();
+    float s[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < HD; kk += 16) {
+      uint32_t a[4];
+      lda_frag<HD>(a, Qs, warp * 16, kk);
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) {
+        uint32_t bb[4];
+        ldb_rows<HD>(bb, Ks, j * 8, kk);
+        mma16816(s[j], a, bb[0], bb[1]);
+        mma16816(s[j + 1], a, bb[2], bb[3]);
+      }
+    }
+    // mask + online softmax (base-2 domain of the scaled scores)
+    float mx[2] = {mrow[0], mrow[1]};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = kb * 64 + j * 8 + 2 * t4 + (e & 1);
+        const int qr = (e < 2) ? qr0 : qr1;
+        float v = s[j][e] * sl2;
+        if (key > qr || key >= p.S) v = -INFINITY;
+        s[j][e] = v;
+        mx[e >> 1] = fmaxf(mx[e >> 1], v);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+    }
+    float corr[2], rs[2] = {0.f, 0.f};
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float mref = mx[r] == -INFINITY ? 0.f : mx[r];
+      corr[r] = exp2f(mrow[r] - mref);
+      mrow[r] = mx[r];
+      mx[r] = mref;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float pv = exp2f(s[j][e] - mx[e >> 1]);
+        s[j][e] = pv;
+        rs[e >> 1] += pv;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 1);
+      rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 2);
+      lrow[r] = lrow[r] * corr[r] + rs[r];
+    }
+#pragma unroll
+    for (int i = 0; i < HD / 8; ++i) {
+      o[i][0] *= corr[0];
+      o[i][1] *= corr[0];
+      o[i][2] *= corr[1];
+      o[i][3] *= corr[1];
+    }
+    // o += P v
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {  // 16 keys per k-step
+      uint32_t a[4];
+      a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+      a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+      a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+      for (int i = 0; i < HD / 8; i += 2) {
+        uint32_t bb[4];
+        ldb_trans<HD>(bb, Vs, kk * 16, i * 8);
+        mma16816(o[i], a, bb[0], bb[1]);
+        mma16816(o[i + 1], a, bb[2], bb[3]);
+      }
+    }
+  }
+  // normalise and write o, lse
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int qr = r ? qr1 : qr0;
+    if (qr >= p.S) continue;
+    const float inv = 1.0f / lrow[r];
+    __nv_bfloat16* op = p.o + (tok0 + qr) * p.ldo + h * HD;
+#pragma unroll
+    for (int i = 0; i < HD / 8; ++i) {
+      const int c = i * 8 + 2 * t4;
+      *reinterpret_cast<__nv_bfloat162*>(op + c) = __floats2bfloat162_rn(o[i][2 * r] * inv, o[i][2 * r + 1] * inv);
+    }
+    if (t4 == 0) p.lse[(tok0 + qr) * p.hq + h] = (mrow[r] + log2f(lrow[r])) / kLog2e;
+  }
+}
+
+// --------------------------------------------------------------------------- backward: D = rowsum(dO o)
+__global__ void k_attn_D(AttnBwdArgs p) {
+  const int64_t idx = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // (t, h)
+  const int l = threadIdx.x & 31;
+  if (idx >= p.T * (int64_t)p.hq) return;
+  const int64_t t = idx / p.hq;
+  const int h = (int)(idx % p.hq);
+  const __nv_bfloat16* a = p.dout + t * p.lddo + (int64_t)h * p.hd;
+  const __nv_bfloat16* o = p.o + t * p.ldo + (int64_t)h * p.hd;
+  float s = 0.f;
+  for (int c = l; c < p.hd; c += 32) s += __bfloat162float(a[c]) * __bfloat162float(o[c]);
+  s = warp_sum(s);
+  if (l == 0) p.D[idx] = s;
+}
+
+// --------------------------------------------------------------------------- backward: dK, dV
+// grid (ceil(S/64), hkv, B), 128 threads; warp w owns keys 16w..16w+15 of the block; query blocks
+// of 32 rows; the query heads of the group are visited in increasing order.
+template <int HD>
+__global__ void __launch_bounds__(128) k_attn_dkdv(AttnBwdArgs p) {
+  extern __shared__ __align__(16) uint8_t sm_raw[];
+  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(sm_raw);
+  __nv_bfloat16* Vs = Ks + 64 * Tile<HD>::LD;
+  __nv_bfloat16* Qs = Vs + 64 * Tile<HD>::LD;
+  __nv_bfloat16* Os = Qs + 32 * Tile<HD>::LD;  // dO tile
+  float* Ls = reinterpret_cast<float*>(Os + 32 * Tile<HD>::LD);
+  float* Ds = Ls + 32;
+  const int kb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int grp = p.hq / p.hkv;
+  const int64_t tok0 = (int64_t)b * p.S;
+  const int k0 = kb * 64;
+  const int warp = threadIdx.x >> 5, l = threadIdx.x & 31, g = l >> 2, t4 = l & 3;
+  const float sl2 = p.scale * kLog2e;
+
+  load_tile<HD>(Ks, p.k, p.ldk, tok0, k0, 64, p.S, kvh * HD);
+  load_tile<HD>(Vs, p.v, p.ldv, tok0, k0, 64, p.S, kvh * HD);
+
+  float dk[HD / 8][4], dv[HD / 8][4];
+#pragma unroll
+  for (int i = 0; i < HD / 8; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dk[i][e] = dv[i][e] = 0.f;
+  const int kr0 = k0 + warp * 16 + g, kr1 = kr0 + 8;  // this thread's key rows
+
+  for (int hh = 0; hh < grp; ++hh) {
+    const int h = kvh * grp + hh;
+    for (int qs0 = k0; qs0 < p.S; qs0 += 32) {
+      __syncthreads();
+      load_tile<HD>(Qs, p.q, p.ldq, tok0, qs0, 32, p.S, h * HD);
+      load_tile<HD>(Os, p.dout, p.lddo, tok0, qs0, 32, p.S, h * HD);
+      if (threadIdx.x < 32) {
+        const int qr = qs0 + threadIdx.x;
+        Ls[threadIdx.x] = qr < p.S ? p.lse[(tok0 + qr) * p.hq + h] * kLog2e : 0.f;
+        Ds[threadIdx.x] = qr < p.S ? p.D[(tok0 + qr) * p.hq + h] : 0.f;
+      }
+      __syncthreads();
+      // S^T (16 keys x 32 queries) and dP^T
+      float st[4][4], dp[4][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st[j][e] = dp[j][e] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < HD; kk += 16) {
+        uint32_t ak[4], av[4];
+        lda_frag<HD>(ak, Ks, warp * 16, kk);
+        lda_frag<HD>(av, Vs, warp * 16, kk);
+#pragma unroll
+        for (int j = 0; j < 4; j += 2) {
+          uint32_t bq[4], bo[4];
+          ldb_rows<HD>(bq, Qs, j * 8, kk);
+          ldb_rows<HD>(bo, Os, j * 8, kk);
+          mma16816(st[j], ak, bq[0], bq[1]);
+          mma16816(st[j + 1], ak, bq[2], bq[3]);
+          mma16816(dp[j], av, bo[0], bo[1]);
+          mma16816(dp[j + 1], av, bo[2], bo[3]);
+        }
+      }
+      // P^T and dS^T
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int qi = j * 8 + 2 * t4 + (e & 1);
+          const int qr = qs0 + qi;
+          const int kr = (e < 2) ? kr0 : kr1;
+          float pv = exp2f(st[j][e] * sl2 - Ls[qi]);
+          if (qr < kr || qr >= p.S || kr >= p.S) pv = 0.f;
+          st[j][e] = pv;
+          dp[j][e] = pv * (dp[j][e] - Ds[qi]);
+        }
+      }
+      // dV += P^T dO ; dK += dS^T Q
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) {
+        uint32_t ap[4], as[4];
+        ap[0] = pack_bf16(st[2 * kk][0], st[2 * kk][1]);
+        ap[1] = pack_bf16(st[2 * kk][2], st[2 * kk][3]);
+        ap[2] = pack_bf16(st[2 * kk + 1][0], st[2 * kk + 1][1]);
+        ap[3] = pack_bf16(st[2 * kk + 1][2], st[2 * kk + 1][3]);
+        as[0] = pack_bf16(dp[2 * kk][0], dp[2 * kk][1]);
+        as[1] = pack_bf16(dp[2 * kk][2], dp[2 * kk][3]);
+        as[2] = pack_bf16(dp[2 * kk + 1][0], dp[2 * kk + 1][1]);
+        as[3] = pack_bf16(dp[2 * kk + 1][2], dp[2 * kk + 1][3]);
+#pragma unroll
+        for (int i = 0; i < HD / 8; i += 2) {
+          uint32_t bo[4], bq[4];
+          ldb_trans<HD>(bo, Os, kk * 16, i * 8);
+          ldb_trans<HD>(bq, Qs, kk * 16, i * 8);
+          mma16816(dv[i], ap, bo[0], bo[1]);
+          mma16816(dv[i + 1], ap, bo[2], bo[3]);
+          mma16816(dk[i], as, bq[0], bq[1]);
+          mma16816(dk[i + 1], as, bq[2], bq[3]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int kr = r ? kr1 : kr0;
+    if (kr >= p.S) continue;
+    __nv_bfloat16* kp = p.dk + (tok0 + kr) * p.lddk + kvh * HD;
+    __nv_bfloat16* vp = p.dv + (tok0 + kr) * p.lddv + kvh * HD;
+#pragma unroll
+    for (int i = 0; i < HD / 8; ++i) {
+      const int c = i * 8 + 2 * t4;
+      *reinterpret_cast<__nv_bfloat162*>(kp + c) =
+          __floats2bfloat162_rn(dk[i][2 * r] * p.scale, dk[i][2 * r + 1] * p.scale);
+      *reinterpret_cast<__nv_bfloat162*>(vp + c) = __floats2bfloat162_rn(dv[i][2 * r], dv[i][2 * r + 1]);
+    }
+  }
+}
+
+// --------------------------------------------------------------------------- backward: dQ
+// grid (ceil(S/64), hq, B), 128 threads; warp w owns queries 16w..16w+15; key blocks of 32.
+template <int HD>
+__global__ void __launch_bounds__(128) k_attn_dq(AttnBwdArgs p) {
+  extern __shared__ __align__(16) uint8_t sm_raw[];
+  __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(sm_raw);
+  __nv_bfloat16* Os = Qs + 64 * Tile<HD>::LD;  // dO
+  __nv_bfloat16* Ks = Os + 64 * Tile<HD>::LD;
+  __nv_bfloat16* Vs = Ks + 32 * Tile<HD>::LD;
+  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / (p.hq / p.hkv);
+  const int64_t tok0 = (int64_t)b * p.S;
+  const int q0 = qb * 64;
+  const int warp = threadIdx.x >> 5, l = threadIdx.x & 31, g = l >> 2, t4 = l & 3;
+  const float sl2 = p.scale * kLog2e;
+
+  load_tile<HD>(Qs, p.q, p.ldq, tok0, q0, 64, p.S, h * HD);
+  load_tile<HD>(Os, p.dout, p.lddo, tok0, q0, 64, p.S, h * HD);
+  const int qr0 = q0 + warp * 16 + g, qr1 = qr0 + 8;
+  float lse2[2], dd[2];
+  lse2[0] = qr0 < p.S ? p.lse[(tok0 + qr0) * p.hq + h] * kLog2e : 0.f;
+  lse2[1] = qr1 < p.S ? p.lse[(tok0 + qr1) * p.hq + h] * kLog2e : 0.f;
+  dd[0] = qr0 < p.S ? p.D[(tok0 + qr0) * p.hq + h] : 0.f;
+  dd[1] = qr1 < p.S ? p.D[(tok0 + qr1) * p.hq + h] : 0.f;
+
+  float dq[HD / 8][4];
+#pragma unroll
+  for (int i = 0; i < HD / 8; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
+  const int kend = min(q0 + 64, p.S);
+  for (int ks0 = 0; ks0 < kend; ks0 += 32) {
+    __syncthreads();
+    load_tile<HD>(Ks, p.k, p.ldk, tok0, ks0, 32, p.S, kvh * HD);
+    load_tile<HD>(Vs, p.v, p.ldv, tok0, ks0, 32, p.S, kvh * HD);
+    __syncthreads();
+    float s[4][4], dp[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[j][e] = dp[j][e] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < HD; kk += 16) {
+      uint32_t aq[4], ao[4];
+      lda_frag<HD>(aq, Qs, warp * 16, kk);
+      lda_frag<HD>(ao, Os, warp * 16, kk);
+#pragma unroll
+      for (int j = 0; j < 4; j += 2) {
+        uint32_t bk[4], bv[4];
+        ldb_rows<HD>(bk, Ks, j * 8, kk);
+        ldb_rows<HD>(bv, Vs, j * 8, kk);
+        mma16816(s[j], aq, bk[0], bk[1]);
+        mma16816(s[j + 1], aq, bk[2], bk[3]);
+        mma16816(dp[j], ao, bv[0], bv[1]);
+        mma16816(dp[j + 1], ao, bv[2], bv[3]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = ks0 + j * 8 + 2 * t4 + (e & 1);
+        const int r = e >> 1;
+        const int qr = r ? qr1 : qr0;
+        float pv = exp2f(s[j][e] * sl2 - lse2[r]);
+        if (key > qr || key >= p.S || qr >= p.S) pv = 0.f;
+        s[j][e] = pv * (dp[j][e] - dd[r]);  // dS
+      }
+    }
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      uint32_t a[4];
+      a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+      a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+      a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+      for (int i = 0; i < HD / 8; i += 2) {
+        uint32_t bk[4];
+        ldb_trans<HD>(bk, Ks, kk * 16, i * 8);
+        mma16816(dq[i], a, bk[0], bk[1]);
+        mma16816(dq[i + 1], a, bk[2], bk[3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int qr = r ? qr1 : qr0;
+    if (qr >= p.S) continue;
+    __nv_bfloat16* qp = p.dq + (tok0 + qr) * p.lddq + h * HD;
+#pragma unroll
+    for (int i = 0; i < HD / 8; ++i) {
+      const int c = i * 8 + 2 * t4;
+      *reinterpret_cast<__nv_bfloat162*>(qp + c) =
+          __floats2bfloat162_rn(dq[i][2 * r] * p.scale, dq[i][2 * r + 1] * p.scale);
+    }
+  }
+}
+
+template <typename K>
+cudaError_t set_smem(K kern, int bytes) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+bool check_common(int hd, int hq, int hkv, int S, int64_t T) {
+  if (hd != 64 && hd != 128) return false;
+  if (hq <= 0 || hkv <= 0 || hq % hkv) return false;
+  if (S <= 0 || T <= 0 || T % S) return false;
+  return true;
+}
+
+}  // namespace
+
+cudaError_t attention_fwd(const AttnArgs& a, cudaStream_t s) {
+  if (!check_common(a.hd, a.hq, a.hkv, a.S, a.T)) return cudaErrorInvalidValue;
+  const int B = (int)(a.T / a.S);
+  dim3 grid((a.S + 63) / 64, a.hq, B);
+  if (a.hd == 128) {
+    const int sm = 3 * 64 * Tile<128>::LD * 2;
+    cudaError_t e = set_smem(k_attn_fwd<128>, sm);
+    if (e != cudaSuccess) return e;
+    k_attn_fwd<128><<<grid, 128, sm, s>>>(a);
+  } else {
+    const int sm = 3 * 64 * Tile<64>::LD * 2;
+    k_attn_fwd<64><<<grid, 128, sm, s>>>(a);
+  }
+  note_launch(1);
+  return cudaGetLastError();
+}
+
+cudaError_t attention_bwd(const AttnBwdArgs& a, cudaStream_t s) {
+  if (!check_common(a.hd, a.hq, a.hkv, a.S, a.T)) return cudaErrorInvalidValue;
+  const int B = (int)(a.T / a.S);
+  {
+    const int64_t n = a.T * (int64_t)a.hq;
+    k_attn_D<<<(unsigned)((n + 7) / 8), 256, 0, s>>>(a);
+  }
+  dim3 gk((a.S + 63) / 64, a.hkv, B), gq((a.S + 63) / 64, a.hq, B);
+  if (a.hd == 128) {
+    const int smk = (64 + 64 + 32 + 32) * Tile<128>::LD * 2 + 64 * 4;
+    const int smq = (64 + 64 + 32 + 32) * Tile<128>::LD * 2;
+    cudaError_t e = set_smem(k_attn_dkdv<128>, smk);
+    if (e == cudaSuccess) e = set_smem(k_attn_dq<128>, smq);
+    if (e != cudaSuccess) return e;
+    k_attn_dkdv<128><<<gk, 128, smk, s>>>(a);
+    k_attn_dq<128><<<gq, 128, smq, s>>>(a);
+  } else {
+    const int smk = (64 + 64 + 32 + 32) * Tile<64>::LD * 2 + 64 * 4;
+    const int smq = (64 + 64 + 32 + 32) * Tile<64>::LD * 2;
+    k_attn_dkdv<64><<<gk, 128, smk, s>>>(a);
+    k_attn_dq<64><<<gq, 128, smq, s>>>(a);
+  }
+  note_launch(3);
+  return cudaGetLastError();
+}
+
+}  // namespace lst

@@ -1,0 +1,1173 @@
+// Streaming engine and the C ABI of include/lst.h.
+//
+// The frozen base of every decoder layer is one contiguous blob. In streamed mode the blobs live in
+// one pinned host arena; each step makes 2L layer reads n = 0..2L-1 (layer n for n < L, layer
+// 2L-1-n after), copied with cudaMemcpyAsync on a dedicated copy stream into a two-buffer device
+// pool (read n uses buffer n % 2). Events fence the two streams: compute of read n waits for
+// "loaded[n]"; the copy of read n+2 into the same buffer waits for "free[n]", recorded when the
+// compute of read n is done with the buffer. So layer n+1 streams in while layer n computes
+// ("Soup: Fine-Tuning an 8B Model on a 4 GB Laptop GPU, One Layer at a Time", first paragraph:
+// double buffering; tutorial "Fine-tune Llama 3.1 8B on a 4GB GPU with Soup", section "What Soup
+// layer streaming changes": two-buffer pool, forward read plus backward-recomputation read;
+// "Soup CLI fine-tunes Llama-3.1-8B on a 4 GB laptop GPU", second paragraph: a dedicated CUDA
+// stream for the copies).
+//
+// The forward keeps only each layer's input; the backward reads the layer again, recomputes its
+// forward (keeping the intermediates) and runs its backward. Resident mode runs the same launches
+// on blobs that stay on the device, so both modes give the same bytes.
+#include "../../include/lst.h"
+#include "../../include/lst_kernels.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "nf4.cuh"
+#include "ops.cuh"
+
+#include <atomic>
+#include <chrono>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <thread>
+#include <vector>
+
+namespace lst {
+__device__ int g_lst_dev_error = 0;
+std::atomic<long long> g_launch_count{0};
+}  // namespace lst
+
+using namespace lst;
+
+namespace {
+
+constexpr int NPROJ = 7;
+enum { G_QKV = 0, G_O = 1, G_GU = 2, G_DOWN = 3, NGROUP = 4 };
+
+inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+// ------------------------------------------------------------------------- host fault injection
+// LST_FAULT=pinned_alloc:N | device_alloc:N | memcpy:N | timeout  -- fail the N-th (1-based)
+// pinned allocation / device allocation / layer-copy enqueue, or report a step timeout.
+struct Faults {
+  long pinned_at = 0, device_at = 0, memcpy_at = 0;
+  bool timeout = false;
+  long pinned_n = 0, device_n = 0, memcpy_n = 0;
+  Faults() {
+    const char* e = std::getenv("LST_FAULT");
+    if (!e) return;
+    std::string s(e);
+    auto num = [&](const char* key) -> long {
+      auto p = s.find(key);
+      if (p == std::string::npos) return 0;
+      return std::atol(s.c_str() + p + std::strlen(key));
+    };
+    pinned_at = num("pinned_alloc:");
+    device_at = num("device_alloc:");
+    memcpy_at = num("memcpy:");
+    timeout = s.find("timeout") != std::string::npos;
+  }
+  bool fail_pinned() { return pinned_at && ++pinned_n == pinned_at; }
+  bool fail_device() { return device_at && ++device_n == device_at; }
+  bool fail_memcpy() { return memcpy_at && ++memcpy_n == memcpy_at; }
+};
+
+struct Group {
+  int nseg = 0;
+  int proj[3] = {0, 0, 0};
+  int in = 0, out = 0;
+  int bounds[4] = {0, 0, 0, 0};
+  int R = 0, KP = 0;
+  int64_t woff = 0;  // element offset of the group's W in the concatenated bf16 weights
+};
+
+struct Layout {
+  int64_t n[NPROJ], outd[NPROJ], ind[NPROJ], woff[NPROJ];
+  int64_t P = 0;
+  int64_t packed[NPROJ], qabs[NPROJ], gscale[NPROJ], means = 0, w16 = 0, norms = 0, bias = 0, total = 0;
+};
+
+bool valid_config(const lst_config* c, std::string* why) {
+  auto bad = [&](const char* m) {
+    if (why) *why = m;
+    return false;
+  };
+  if (!c) return bad("null config");
+  if (c->n_layers < 1) return bad("n_layers must be >= 1");
+  if (c->d_model <= 0 || c->d_model % 8) return bad("d_model must be a positive multiple of 8");
+  if (c->n_heads <= 0 || c->n_kv_heads <= 0 || c->n_heads % c->n_kv_heads) return bad("bad head counts");
+  if (c->head_dim != 64 && c->head_dim != 128) return bad("head_dim must be 64 or 128");
+  if (c->ffn <= 0 || c->ffn % 8) return bad("ffn must be a positive multiple of 8");
+  if (c->vocab < 0) return bad("vocab must be >= 0");
+  if (c->lora_rank <= 0 || 3 * c->lora_rank > 64) return bad("lora_rank must be in [1, 21]");
+  if (!(c->lora_alpha == c->lora_alpha)) return bad("lora_alpha is NaN");
+  if (c->base_format != LST_BASE_NF4 && c->base_format != LST_BASE_BF16) return bad("bad base_format");
+  if (c->max_batch <= 0 || c->max_seq <= 0) return bad("max_batch and max_seq must be positive");
+  if (!(c->rms_eps > 0.f) || !(c->rope_theta > 0.f)) return bad("rms_eps and rope_theta must be positive");
+  const int64_t dq = (int64_t)c->n_heads * c->head_dim, dkv = (int64_t)c->n_kv_heads * c->head_dim;
+  if ((dq * c->d_model) % 64 || (dkv * c->d_model) % 64 || ((int64_t)c->ffn * c->d_model) % 64)
+    return bad("every projection must have a multiple of 64 elements");
+  return true;
+}
+
+Layout make_layout(const lst_config& c) {
+  Layout L{};
+  const int64_t d = c.d_model, dq = (int64_t)c.n_heads * c.head_dim, dkv = (int64_t)c.n_kv_heads * c.head_dim,
+                F = c.ffn;
+  const int64_t outs[NPROJ] = {dq, dkv, dkv, d, F, F, d};
+  const int64_t ins[NPROJ] = {d, d, d, dq, d, d, F};
+  int64_t acc = 0;
+  for (int p = 0; p < NPROJ; ++p) {
+    L.outd[p] = outs[p];
+    L.ind[p] = ins[p];
+    L.n[p] = outs[p] * ins[p];
+    L.woff[p] = acc;
+    acc += L.n[p];
+  }
+  L.P = acc;
+  int64_t off = 0;
+  if (c.base_format == LST_BASE_NF4) {
+    for (int p = 0; p < NPROJ; ++p) { L.packed[p] = off; off = align256(off + L.n[p] / 2); }
+    for (int p = 0; p < NPROJ; ++p) { L.qabs[p] = off; off = align256(off + L.n[p] / 64); }
+    for (int p = 0; p < NPROJ; ++p) {
+      L.gscale[p] = off;
+      off = align256(off + ((L.n[p] / 64 + 255) / 256) * 4);
+    }
+    L.means = off;
+    off = align256(off + NPROJ * 4);
+  } else {
+    L.w16 = 0;
+    off = align256(L.P * 2);
+  }
+  L.norms = off;
+  off = align256(off + 2 * d * 4);
+  L.bias = off;
+  if (c.qkv_bias) off = align256(off + (dq + 2 * dkv) * 4);
+  L.total = off;
+  return L;
+}
+
+bool is_device_ptr(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+// Profiling classes
+enum { PC_GEMM = 0, PC_ATTN = 1, PC_DEQ = 2, PC_OTHER = 3, PC_COPY = 4, PC_N = 5 };
+
+}  // namespace
+
+struct lst_ctx {
+  lst_config cfg{};
+  int dev = 0;
+  cudaStream_t stream = nullptr, copy_stream = nullptr;
+  bool own_stream = false;
+  std::string err;
+  Faults faults;
+
+  int d = 0, hq = 0, hkv = 0, hd = 0, F = 0, V = 0, L = 0, r = 0;
+  int64_t dq = 0, dkv = 0, dqkv = 0, Tmax = 0;
+  float s = 1.f;
+  Layout lay{};
+  Group grp[NGROUP];
+
+  uint8_t* arena = nullptr;     // pinned host, L blobs (streamed)
+  uint8_t* resident = nullptr;  // device, L blobs (resident)
+  uint8_t* pool[2] = {nullptr, nullptr};
+  std::vector<char> registered;
+
+  __nv_bfloat16 *E = nullptr, *H = nullptr;
+  float* gf = nullptr;
+
+  float* lora = nullptr;
+  int64_t lora_numel = 0;
+  std::vector<int64_t> offA, offB;
+  struct Derived {
+    float* Acat32 = nullptr;
+    __nv_bfloat16* Acat16 = nullptr;
+    float* BexpT32 = nullptr;
+    __nv_bfloat16* Bexp16 = nullptr;
+  };
+  std::vector<Derived> der;  // L * NGROUP
+  float* grads = nullptr;
+
+  __nv_bfloat16* xs = nullptr;
+  __nv_bfloat16 *n1 = nullptr, *qkv = nullptr, *o = nullptr, *h = nullptr, *n2 = nullptr, *gu = nullptr,
+                *m = nullptr, *wscr = nullptr;
+  float *rstd1 = nullptr, *rstd2 = nullptr, *lse = nullptr, *Dbuf = nullptr;
+  float* U[NGROUP] = {};
+  __nv_bfloat16* Us[NGROUP] = {};
+  float* Vv[NGROUP] = {};
+  __nv_bfloat16* Vs[NGROUP] = {};
+  float *ga = nullptr, *gb = nullptr, *dn = nullptr, *dm = nullptr, *part = nullptr;
+  __nv_bfloat16 *dout_b = nullptr, *dh_b = nullptr, *do_b = nullptr, *dqkvb = nullptr, *dgu = nullptr;
+  __nv_bfloat16* nf = nullptr;
+  float *rstdf = nullptr, *logits = nullptr, *loss_rows = nullptr, *loss_dev = nullptr, *dot_part = nullptr;
+  __nv_bfloat16* dlog = nullptr;
+  __nv_bfloat16* gbuf = nullptr;
+  int32_t *tok = nullptr, *tgt = nullptr;
+  float *cos_t = nullptr, *sin_t = nullptr;
+  float* host_loss = nullptr;
+
+  std::vector<cudaEvent_t> ev_loaded, ev_free;
+  cudaEvent_t ev_done = nullptr;
+
+  float* stage_w = nullptr;
+  uint8_t* stage_blob = nullptr;
+  float* stage_absmax = nullptr;
+  double* stage_gsum = nullptr;
+
+  std::vector<void*> dev_allocs;
+  int64_t dev_bytes = 0;
+  int64_t curT = 0, curB = 0, curS = 0;
+  bool have_logits = false;
+
+  lst_stats st{};
+  // profiling
+  bool profiling = false;
+  struct ProfRec {
+    cudaEvent_t a, b;
+    int cls;
+    double flops;
+  };
+  std::vector<cudaEvent_t> prof_pool;
+  size_t prof_used = 0;
+  std::vector<ProfRec> prof_recs;
+  cudaEvent_t prof_step0 = nullptr, prof_step1 = nullptr;
+  int64_t launches_at_step_start = 0;
+};
+
+namespace {
+
+lst_status fail(lst_ctx* c, lst_status s, const std::string& m) {
+  if (c) c->err = m;
+  return s;
+}
+lst_status cuda_fail(lst_ctx* c, cudaError_t e, const char* where) {
+  cudaGetLastError();
+  return fail(c, e == cudaErrorMemoryAllocation ? LST_ERR_OOM : LST_ERR_CUDA,
+              std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+#define CK(call)                                           \
+  do {                                                     \
+    cudaError_t e__ = (call);                              \
+    if (e__ != cudaSuccess) return cuda_fail(c, e__, #call); \
+  } while (0)
+
+template <class T>
+lst_status dalloc(lst_ctx* c, T** p, int64_t n, bool zero = false) {
+  *p = nullptr;
+  if (n <= 0) n = 1;
+  if (c->faults.fail_device()) return fail(c, LST_ERR_OOM, "device allocation failed (injected)");
+  void* q = nullptr;
+  cudaError_t e = cudaMalloc(&q, (size_t)n * sizeof(T));
+  if (e != cudaSuccess) return cuda_fail(c, e, "cudaMalloc");
+  c->dev_allocs.push_back(q);
+  c->dev_bytes += n * (int64_t)sizeof(T);
+  if (zero) {
+    e = cudaMemset(q, 0, (size_t)n * sizeof(T));
+    if (e != cudaSuccess) return cuda_fail(c, e, "cudaMemset");
+  }
+  *p = static_cast<T*>(q);
+  return LST_OK;
+}
+
+#define TRY(x)                        \
+  do {                                \
+    lst_status s__ = (x);             \
+    if (s__ != LST_OK) return s__;    \
+  } while (0)
+
+// ------------------------------------------------------------------------- profiling helpers
+cudaEvent_t prof_event(lst_ctx* c) {
+  if (c->prof_used == c->prof_pool.size()) {
+    cudaEvent_t e;
+    cudaEventCreate(&e);
+    c->prof_pool.push_back(e);
+  }
+  return c->prof_pool[c->prof_used++];
+}
+struct ProfScope {
+  lst_ctx* c;
+  cudaStream_t s;
+  int cls;
+  double flops;
+  cudaEvent_t a = nullptr;
+  ProfScope(lst_ctx* c_, cudaStream_t s_, int cls_, double flops_ = 0) : c(c_), s(s_), cls(cls_), flops(flops_) {
+    if (c->profiling) {
+      a = prof_event(c);
+      cudaEventRecord(a, s);
+    }
+  }
+  ~ProfScope() {
+    if (c->profiling) {
+      cudaEvent_t b = prof_event(c);
+      cudaEventRecord(b, s);
+      c->prof_recs.push_back({a, b, cls, flops});
+    }
+  }
+};
+
+// ------------------------------------------------------------------------- LoRA operands
+lst_status prep_lora(lst_ctx* c, int layer) {
+  for (int g = 0; g < NGROUP; ++g) {
+    const Group& G = c->grp[g];
+    const auto& D = c->der[layer * NGROUP + g];
+    LoraPrepArgs a{};
+    for (int k = 0; k < G.nseg; ++k) {
+      a.A[k] = c->lora + c->offA[layer * NPROJ + G.proj[k]];
+      a.B[k] = c->lora + c->offB[layer * NPROJ + G.proj[k]];
+    }
+    a.nseg = G.nseg;
+    a.r = c->r;
+    a.in = G.in;
+    for (int k = 0; k <= G.nseg; ++k) a.bounds[k] = G.bounds[k];
+    a.KP = G.KP;
+    a.Acat32 = D.Acat32;
+    a.Acat16 = D.Acat16;
+    a.BexpT32 = D.BexpT32;
+    a.Bexp16 = D.Bexp16;
+    CK(lora_prep(a, c->stream));
+  }
+  return LST_OK;
+}
+
+// ------------------------------------------------------------------------- layer compute
+const __nv_bfloat16* group_w(lst_ctx* c, const __nv_bfloat16* W, int g) { return W + c->grp[g].woff; }
+
+lst_status group_fwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const __nv_bfloat16* X, int64_t ldx,
+                     __nv_bfloat16* Y, int64_t ldy, const float* bias, const __nv_bfloat16* resid, bool gemm) {
+  const Group& G = c->grp[g];
+  const auto& D = c->der[layer * NGROUP + g];
+  const int64_t T = c->curT;
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(lora_project(X, ldx, T, G.in, D.Acat32, G.in, G.R, c->s, c->U[g], c->Us[g], G.KP, c->stream));
+  }
+  if (!gemm) return LST_OK;
+  GemmArgs a;
+  a.M = (int)T;
+  a.N = G.out;
+  a.K = G.in;
+  a.A = X;
+  a.lda = ldx;
+  a.B = group_w(c, W, g);
+  a.ldb = G.in;
+  a.b_mn = 0;
+  a.A2 = c->Us[g];
+  a.lda2 = G.KP;
+  a.B2 = D.Bexp16;
+  a.ldb2 = G.KP;
+  a.K2 = G.KP;
+  a.C = Y;
+  a.ldc = ldy;
+  a.c_f32 = 0;
+  a.bias = bias;
+  a.R = resid;
+  a.ldr = c->d;
+  ProfScope ps(c, c->stream, PC_GEMM, 2.0 * T * G.out * (double)(G.in + G.KP));
+  CK(gemm_bf16(a, c->stream));
+  return LST_OK;
+}
+
+lst_status group_bwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const __nv_bfloat16* dY, int64_t ldy,
+                     const __nv_bfloat16* X, int64_t ldx, void* dX, int dx_f32) {
+  const Group& G = c->grp[g];
+  const auto& D = c->der[layer * NGROUP + g];
+  const int64_t T = c->curT;
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(lora_project(dY, ldy, T, G.out, D.BexpT32, G.out, G.R, c->s, c->Vv[g], c->Vs[g], G.KP, c->stream));
+  }
+  {
+    GemmArgs a;
+    a.M = (int)T;
+    a.N = G.in;
+    a.K = G.out;
+    a.A = dY;
+    a.lda = ldy;
+    a.B = group_w(c, W, g);
+    a.ldb = G.in;
+    a.b_mn = 1;
+    a.A2 = c->Vs[g];
+    a.lda2 = G.KP;
+    a.B2 = D.Acat16;
+    a.ldb2 = G.in;
+    a.K2 = G.KP;
+    a.C = dX;
+    a.ldc = G.in;
+    a.c_f32 = dx_f32;
+    ProfScope ps(c, c->stream, PC_GEMM, 2.0 * T * G.in * (double)(G.out + G.KP));
+    CK(gemm_bf16(a, c->stream));
+  }
+  ProfScope ps(c, c->stream, PC_OTHER);
+  LoraGradArgs ga{};
+  ga.P = c->Vv[g];
+  ga.R = G.R;
+  ga.Q = X;
+  ga.ldq = ldx;
+  ga.C = G.in;
+  ga.T = T;
+  ga.s = c->s;
+  ga.seg_r = 0;
+  ga.nseg = G.nseg;
+  ga.rows_per_dst = c->r;
+  for (int k = 0; k < G.nseg; ++k) ga.dst[k] = c->grads + c->offA[layer * NPROJ + G.proj[k]];
+  ga.partial = c->part;
+  CK(lora_grad(ga, c->stream));
+  LoraGradArgs gb{};
+  gb.P = c->U[g];
+  gb.R = G.R;
+  gb.Q = dY;
+  gb.ldq = ldy;
+  gb.C = G.out;
+  gb.T = T;
+  gb.s = c->s;
+  gb.seg_r = c->r;
+  gb.nseg = G.nseg;
+  for (int k = 0; k <= G.nseg; ++k) gb.bounds[k] = G.bounds[k];
+  for (int k = 0; k < G.nseg; ++k) gb.dst[k] = c->grads + c->offB[layer * NPROJ + G.proj[k]];
+  gb.partial = c->part;
+  CK(lora_grad(gb, c->stream));
+  return LST_OK;
+}
+
+// Weights of a layer read: the bf16 [P] matrix the GEMMs consume.
+lst_status layer_weights(lst_ctx* c, const uint8_t* blob, const __nv_bfloat16** W) {
+  if (c->cfg.base_format == LST_BASE_BF16) {
+    *W = reinterpret_cast<const __nv_bfloat16*>(blob + c->lay.w16);
+    return LST_OK;
+  }
+  Nf4Seg segs[NPROJ];
+  for (int p = 0; p < NPROJ; ++p) {
+    segs[p].packed = blob + c->lay.packed[p];
+    segs[p].qabs = reinterpret_cast<const int8_t*>(blob + c->lay.qabs[p]);
+    segs[p].gscale = reinterpret_cast<const float*>(blob + c->lay.gscale[p]);
+    segs[p].mean = reinterpret_cast<const float*>(blob + c->lay.means) + p;
+    segs[p].n = c->lay.n[p];
+    segs[p].out_offset = c->lay.woff[p];
+  }
+  ProfScope ps(c, c->stream, PC_DEQ);
+  CK(nf4_dequant(segs, NPROJ, c->wscr, c->stream));
+  *W = c->wscr;
+  return LST_OK;
+}
+
+lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16* W, bool recompute) {
+  const int64_t T = c->curT;
+  const int S = (int)c->curS;
+  const float* g1 = reinterpret_cast<const float*>(blob + c->lay.norms);
+  const float* g2 = g1 + c->d;
+  const float* bias = c->cfg.qkv_bias ? reinterpret_cast<const float*>(blob + c->lay.bias) : nullptr;
+  const __nv_bfloat16* x = c->xs + (int64_t)i * c->Tmax * c->d;
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(rmsnorm_fwd(x, g1, T, c->d, c->cfg.rms_eps, c->n1, c->rstd1, c->stream));
+  }
+  TRY(group_fwd(c, i, G_QKV, W, c->n1, c->d, c->qkv, c->dqkv, bias, nullptr, true));
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(rope(c->qkv, c->dqkv, T, S, 0, c->hq, c->hd, c->cos_t, c->sin_t, 0, c->stream));
+    CK(rope(c->qkv, c->dqkv, T, S, (int)c->dq, c->hkv, c->hd, c->cos_t, c->sin_t, 0, c->stream));
+  }
+  {
+    AttnArgs a;
+    a.q = c->qkv;
+    a.k = c->qkv + c->dq;
+    a.v = c->qkv + c->dq + c->dkv;
+    a.o = c->o;
+    a.lse = c->lse;
+    a.ldq = a.ldk = a.ldv = c->dqkv;
+    a.ldo = c->dq;
+    a.T = T;
+    a.S = S;
+    a.hq = c->hq;
+    a.hkv = c->hkv;
+    a.hd = c->hd;
+    a.scale = 1.0f / std::sqrt((float)c->hd);
+    ProfScope ps(c, c->stream, PC_ATTN);
+    CK(attention_fwd(a, c->stream));
+  }
+  TRY(group_fwd(c, i, G_O, W, c->o, c->dq, c->h, c->d, nullptr, x, true));
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(rmsnorm_fwd(c->h, g2, T, c->d, c->cfg.rms_eps, c->n2, c->rstd2, c->stream));
+  }
+  TRY(group_fwd(c, i, G_GU, W, c->n2, c->d, c->gu, 2 * c->F, nullptr, nullptr, true));
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(swiglu_fwd(c->gu, T, c->F, c->m, c->stream));
+  }
+  // the recompute pass needs only the LoRA projection of m (for dB of down), not the output
+  TRY(group_fwd(c, i, G_DOWN, W, c->m, c->F, c->xs + (int64_t)(i + 1) * c->Tmax * c->d, c->d, nullptr, c->h,
+                !recompute));
+  return LST_OK;
+}
+
+// dL/dx_{i+1} is in c->ga (fp32) and c->dout_b (bf16); leaves dL/dx_i there.
+lst_status layer_bwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16* W) {
+  const int64_t T = c->curT;
+  const int S = (int)c->curS;
+  const float* g1 = reinterpret_cast<const float*>(blob + c->lay.norms);
+  const float* g2 = g1 + c->d;
+  const __nv_bfloat16* x = c->xs + (int64_t)i * c->Tmax * c->d;
+  TRY(group_bwd(c, i, G_DOWN, W, c->dout_b, c->d, c->m, c->F, c->dm, 1));
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(swiglu_bwd(c->dm, c->gu, T, c->F, c->dgu, c->stream));
+  }
+  TRY(group_bwd(c, i, G_GU, W, c->dgu, 2 * c->F, c->n2, c->d, c->dn, 1));
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(rmsnorm_bwd(c->dn, c->h, g2, c->rstd2, c->ga, T, c->d, c->gb, c->dh_b, c->stream));
+  }
+  TRY(group_bwd(c, i, G_O, W, c->dh_b, c->d, c->o, c->dq, c->do_b, 0));
+  {
+    AttnBwdArgs a;
+    a.q = c->qkv;
+    a.k = c->qkv + c->dq;
+    a.v = c->qkv + c->dq + c->dkv;
+    a.o = c->o;
+    a.dout = c->do_b;
+    a.lse = c->lse;
+    a.D = c->Dbuf;
+    a.dq = c->dqkvb;
+    a.dk = c->dqkvb + c->dq;
+    a.dv = c->dqkvb + c->dq + c->dkv;
+    a.ldq = a.ldk = a.ldv = c->dqkv;
+    a.ldo = c->dq;
+    a.lddo = c->dq;
+    a.lddq = a.lddk = a.lddv = c->dqkv;
+    a.T = T;
+    a.S = S;
+    a.hq = c->hq;
+    a.hkv = c->hkv;
+    a.hd = c->hd;
+    a.scale = 1.0f / std::sqrt((float)c->hd);
+    ProfScope ps(c, c->stream, PC_ATTN);
+    CK(attention_bwd(a, c->stream));
+  }
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(rope(c->dqkvb, c->dqkv, T, S, 0, c->hq, c->hd, c->cos_t, c->sin_t, 1, c->stream));
+    CK(rope(c->dqkvb, c->dqkv, T, S, (int)c->dq, c->hkv, c->hd, c->cos_t, c->sin_t, 1, c->stream));
+  }
+  TRY(group_bwd(c, i, G_QKV, W, c->dqkvb, c->dqkv, c->n1, c->d, c->dn, 1));
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(rmsnorm_bwd(c->dn, x, g1, c->rstd1, c->gb, T, c->d, c->ga, c->dout_b, c->stream));
+  }
+  return LST_OK;
+}
+
+lst_status head_fwd_bwd(lst_ctx* c) {
+  const int64_t T = c->curT;
+  const __nv_bfloat16* xL = c->xs + (int64_t)c->L * c->Tmax * c->d;
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(rmsnorm_fwd(xL, c->gf, T, c->d, c->cfg.rms_eps, c->nf, c->rstdf, c->stream));
+  }
+  {
+    GemmArgs a;
+    a.M = (int)T;
+    a.N = c->V;
+    a.K = c->d;
+    a.A = c->nf;
+    a.lda = c->d;
+    a.B = c->H;
+    a.ldb = c->d;
+    a.b_mn = 0;
+    a.C = c->logits;
+    a.ldc = c->V;
+    a.c_f32 = 1;
+    ProfScope ps(c, c->stream, PC_GEMM, 2.0 * T * c->V * (double)c->d);
+    CK(gemm_bf16(a, c->stream));
+  }
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(cross_entropy(c->logits, T, c->V, c->tgt, 1.0f / (float)T, c->loss_rows, c->dlog, c->stream));
+    CK(mean_fixed(c->loss_rows, T, c->loss_dev, c->stream));
+  }
+  {
+    GemmArgs a;
+    a.M = (int)T;
+    a.N = c->d;
+    a.K = c->V;
+    a.A = c->dlog;
+    a.lda = c->V;
+    a.B = c->H;
+    a.ldb = c->d;
+    a.b_mn = 1;
+    a.C = c->dn;
+    a.ldc = c->d;
+    a.c_f32 = 1;
+    ProfScope ps(c, c->stream, PC_GEMM, 2.0 * T * c->V * (double)c->d);
+    CK(gemm_bf16(a, c->stream));
+  }
+  ProfScope ps(c, c->stream, PC_OTHER);
+  CK(rmsnorm_bwd(c->dn, xL, c->gf, c->rstdf, nullptr, T, c->d, c->ga, c->dout_b, c->stream));
+  return LST_OK;
+}
+
+lst_status enqueue_copy(lst_ctx* c, int n) {
+  const int L = c->L;
+  const int j = n < L ? n : 2 * L - 1 - n;
+  const int b = n & 1;
+  if (c->faults.fail_memcpy()) return fail(c, LST_ERR_CUDA, "layer copy enqueue failed (injected)");
+  if (n >= 2) CK(cudaStreamWaitEvent(c->copy_stream, c->ev_free[n - 2], 0));
+  ProfScope ps(c, c->copy_stream, PC_COPY);
+  CK(cudaMemcpyAsync(c->pool[b], c->arena + (int64_t)j * c->lay.total, c->lay.total, cudaMemcpyHostToDevice,
+                     c->copy_stream));
+  CK(cudaEventRecord(c->ev_loaded[n], c->copy_stream));
+  c->st.layer_reads_last_step += 1;
+  c->st.h2d_bytes_last_step += c->lay.total;
+  return LST_OK;
+}
+
+__global__ void k_bf16_to_f32(const __nv_bfloat16* x, int64_t n, float* y) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = __bfloat162float(x[i]);
+}
+
+lst_status run_layers(lst_ctx* c, bool head) {
+  const int L = c->L;
+  const bool streamed = c->cfg.streamed != 0;
+  if (streamed) {
+    TRY(enqueue_copy(c, 0));
+    if (2 * L > 1) TRY(enqueue_copy(c, 1));
+  }
+  for (int n = 0; n < 2 * L; ++n) {
+    const int j = n < L ? n : 2 * L - 1 - n;
+    const uint8_t* blob = streamed ? c->pool[n & 1] : c->resident + (int64_t)j * c->lay.total;
+    if (streamed) CK(cudaStreamWaitEvent(c->stream, c->ev_loaded[n], 0));
+    const __nv_bfloat16* W = nullptr;
+    TRY(layer_weights(c, blob, &W));
+    if (n < L) {
+      TRY(layer_fwd(c, j, blob, W, false));
+    } else {
+      TRY(layer_fwd(c, j, blob, W, true));
+      TRY(layer_bwd(c, j, blob, W));
+    }
+    if (streamed) CK(cudaEventRecord(c->ev_free[n], c->stream));
+    if (n == L - 1) {
+      if (head) {
+        TRY(head_fwd_bwd(c));
+      } else {
+        const int64_t T = c->curT;
+        const __nv_bfloat16* xL = c->xs + (int64_t)L * c->Tmax * c->d;
+        ProfScope ps(c, c->stream, PC_OTHER);
+        CK(dot_fixed(xL, c->gbuf, T * c->d, c->dot_part, c->loss_dev, c->stream));
+        CK(cudaMemcpyAsync(c->dout_b, c->gbuf, T * c->d * 2, cudaMemcpyDeviceToDevice, c->stream));
+        k_bf16_to_f32<<<(unsigned)((T * c->d + 255) / 256), 256, 0, c->stream>>>(c->gbuf, T * c->d, c->ga);
+        note_launch(1);
+        CK(cudaGetLastError());
+      }
+    }
+    if (streamed && n + 2 < 2 * L) TRY(enqueue_copy(c, n + 2));
+  }
+  return LST_OK;
+}
+
+lst_status finish_step(lst_ctx* c, float* loss, float* grads_out) {
+  if (grads_out) {
+    const bool dev = is_device_ptr(grads_out);
+    CK(cudaMemcpyAsync(grads_out, c->grads, c->lora_numel * 4, dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
+                       c->stream));
+  }
+  CK(cudaMemcpyAsync(c->host_loss, c->loss_dev, 4, cudaMemcpyDeviceToHost, c->stream));
+  if (c->profiling) CK(cudaEventRecord(c->prof_step1, c->stream));
+  CK(cudaEventRecord(c->ev_done, c->stream));
+  const int tmo = c->cfg.timeout_ms > 0 ? c->cfg.timeout_ms : 600000;
+  const auto t0 = std::chrono::steady_clock::now();
+  while (true) {
+    cudaError_t q = cudaEventQuery(c->ev_done);
+    if (q == cudaSuccess) break;
+    if (q != cudaErrorNotReady) return cuda_fail(c, q, "step");
+    if (c->faults.timeout ||
+        std::chrono::duration_cast<std::chrono::milliseconds>(std::chrono::steady_clock::now() - t0).count() > tmo)
+      return fail(c, LST_ERR_TIMEOUT, "step did not finish within timeout_ms");
+    std::this_thread::sleep_for(std::chrono::microseconds(20));
+  }
+  if (c->faults.timeout) return fail(c, LST_ERR_TIMEOUT, "step did not finish within timeout_ms (injected)");
+  int derr = 0;
+  CK(cudaMemcpyFromSymbol(&derr, g_lst_dev_error, sizeof(int)));
+  if (derr) {
+    int zero = 0;
+    cudaMemcpyToSymbol(g_lst_dev_error, &zero, sizeof(int));
+    return fail(c, LST_ERR_DEVICE, "device code reported error " + std::to_string(derr));
+  }
+  *loss = *c->host_loss;
+  c->st.steps += 1;
+  c->st.launches_last_step = g_launch_count.load() - c->launches_at_step_start;
+  if (c->profiling) {
+    double ms[PC_N] = {0, 0, 0, 0, 0};
+    int64_t cnt[PC_N] = {0, 0, 0, 0, 0};
+    double flops = 0;
+    for (auto& r : c->prof_recs) {
+      float t = 0.f;
+      cudaEventElapsedTime(&t, r.a, r.b);
+      ms[r.cls] += t;
+      cnt[r.cls] += 1;
+      if (r.cls == PC_GEMM) flops += r.flops;
+    }
+    float step = 0.f;
+    cudaEventElapsedTime(&step, c->prof_step0, c->prof_step1);
+    c->st.gemm_ms = ms[PC_GEMM];
+    c->st.attention_ms = ms[PC_ATTN];
+    c->st.dequant_ms = ms[PC_DEQ];
+    c->st.other_ms = ms[PC_OTHER];
+    c->st.copy_ms = ms[PC_COPY];
+    c->st.gemm_launches = cnt[PC_GEMM];
+    c->st.attention_launches = cnt[PC_ATTN];
+    c->st.dequant_launches = cnt[PC_DEQ];
+    c->st.copy_count = cnt[PC_COPY];
+    c->st.gemm_flops = flops;
+    c->st.step_ms = step;
+  }
+  return LST_OK;
+}
+
+lst_status begin_step(lst_ctx* c, int32_t batch, int32_t seq) {
+  for (int i = 0; i < c->L; ++i)
+    if (!c->registered[i]) return fail(c, LST_ERR_STATE, "layer " + std::to_string(i) + " is not registered");
+  if (batch <= 0 || seq <= 0 || batch > c->cfg.max_batch || seq > c->cfg.max_seq)
+    return fail(c, LST_ERR_ARG, "batch/seq outside (0, max]");
+  c->curB = batch;
+  c->curS = seq;
+  c->curT = (int64_t)batch * seq;
+  c->st.layer_reads_last_step = 0;
+  c->st.h2d_bytes_last_step = 0;
+  c->prof_used = 0;
+  c->prof_recs.clear();
+  c->launches_at_step_start = g_launch_count.load();
+  if (c->profiling) CK(cudaEventRecord(c->prof_step0, c->stream));
+  return LST_OK;
+}
+
+lst_status copy_in(lst_ctx* c, void* dst, const void* src, int64_t bytes) {
+  CK(cudaMemcpyAsync(dst, src, bytes, is_device_ptr(src) ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice,
+                     c->stream));
+  return LST_OK;
+}
+
+// fp32 host/device tensor -> bf16 device buffer
+lst_status upload_bf16(lst_ctx* c, __nv_bfloat16* dst, const float* src, int64_t n) {
+  if (is_device_ptr(src)) {
+    CK(f32_to_bf16(src, n, dst, c->stream));
+    return LST_OK;
+  }
+  const int64_t chunk = 1 << 24;
+  float* tmp = nullptr;
+  CK(cudaMalloc(&tmp, chunk * 4));
+  for (int64_t i = 0; i < n; i += chunk) {
+    const int64_t k = std::min(chunk, n - i);
+    cudaError_t e = cudaMemcpyAsync(tmp, src + i, k * 4, cudaMemcpyHostToDevice, c->stream);
+    if (e == cudaSuccess) e = f32_to_bf16(tmp, k, dst + i, c->stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(c->stream);
+    if (e != cudaSuccess) {
+      cudaFree(tmp);
+      return cuda_fail(c, e, "upload_bf16");
+    }
+  }
+  cudaFree(tmp);
+  return LST_OK;
+}
+
+lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, const float* lm_head,
+                       void* stream) {
+  const lst_config& k = c->cfg;
+  CK(cudaGetDevice(&c->dev));
+  c->d = k.d_model;
+  c->hq = k.n_heads;
+  c->hkv = k.n_kv_heads;
+  c->hd = k.head_dim;
+  c->F = k.ffn;
+  c->V = k.vocab;
+  c->L = k.n_layers;
+  c->r = k.lora_rank;
+  c->s = k.lora_alpha / (float)k.lora_rank;
+  c->dq = (int64_t)c->hq * c->hd;
+  c->dkv = (int64_t)c->hkv * c->hd;
+  c->dqkv = c->dq + 2 * c->dkv;
+  c->Tmax = (int64_t)k.max_batch * k.max_seq;
+  c->lay = make_layout(k);
+  const int R3 = 3 * c->r;
+  const int KP = ((R3 + 63) / 64) * 64;
+  auto setg = [&](int g, int nseg, std::initializer_list<int> pr, int in, std::initializer_list<int> bnd) {
+    Group& G = c->grp[g];
+    G.nseg = nseg;
+    int i = 0;
+    for (int p : pr) G.proj[i++] = p;
+    G.in = in;
+    i = 0;
+    for (int b : bnd) G.bounds[i++] = b;
+    G.out = G.bounds[nseg];
+    G.R = nseg * c->r;
+    G.KP = KP;
+    G.woff = c->lay.woff[G.proj[0]];
+  };
+  setg(G_QKV, 3, {0, 1, 2}, c->d, {0, (int)c->dq, (int)(c->dq + c->dkv), (int)c->dqkv});
+  setg(G_O, 1, {3}, (int)c->dq, {0, c->d});
+  setg(G_GU, 2, {4, 5}, c->d, {0, c->F, 2 * c->F});
+  setg(G_DOWN, 1, {6}, c->F, {0, c->d});
+
+  if (stream) {
+    c->stream = static_cast<cudaStream_t>(stream);
+  } else {
+    CK(cudaStreamCreateWithFlags(&c->stream, cudaStreamNonBlocking));
+    c->own_stream = true;
+  }
+  CK(cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking));
+
+  // LoRA parameter / gradient layout
+  c->offA.resize(c->L * NPROJ);
+  c->offB.resize(c->L * NPROJ);
+  int64_t off = 0;
+  for (int l = 0; l < c->L; ++l)
+    for (int p = 0; p < NPROJ; ++p) {
+      c->offA[l * NPROJ + p] = off;
+      off += (int64_t)c->r * c->lay.ind[p];
+      c->offB[l * NPROJ + p] = off;
+      off += c->lay.outd[p] * c->r;
+    }
+  c->lora_numel = off;
+  TRY(dalloc(c, &c->lora, off, true));
+  TRY(dalloc(c, &c->grads, off, true));
+  c->der.resize(c->L * NGROUP);
+  for (int l = 0; l < c->L; ++l)
+    for (int g = 0; g < NGROUP; ++g) {
+      auto& D = c->der[l * NGROUP + g];
+      const Group& G = c->grp[g];
+      TRY(dalloc(c, &D.Acat32, (int64_t)G.R * G.in, true));
+      TRY(dalloc(c, &D.Acat16, (int64_t)G.KP * G.in, true));
+      TRY(dalloc(c, &D.BexpT32, (int64_t)G.R * G.out, true));
+      TRY(dalloc(c, &D.Bexp16, (int64_t)G.out * G.KP, true));
+    }
+
+  // base storage
+  const int64_t blob = c->lay.total;
+  if (k.streamed) {
+    if (c->faults.fail_pinned()) return fail(c, LST_ERR_OOM, "pinned host allocation failed (injected)");
+    void* a = nullptr;
+    cudaError_t e = cudaHostAlloc(&a, (size_t)blob * c->L, cudaHostAllocDefault);
+    if (e != cudaSuccess) return cuda_fail(c, e, "cudaHostAlloc(arena)");
+    c->arena = static_cast<uint8_t*>(a);
+    TRY(dalloc(c, &c->pool[0], blob));
+    TRY(dalloc(c, &c->pool[1], blob));
+    c->st.arena_bytes = blob * c->L;
+  } else {
+    TRY(dalloc(c, &c->resident, blob * c->L));
+    c->st.arena_bytes = blob * c->L;
+  }
+  c->st.blob_bytes = blob;
+  c->registered.assign(c->L, 0);
+  if (k.base_format == LST_BASE_NF4) TRY(dalloc(c, &c->wscr, c->lay.P));
+
+  // activations
+  const int64_t T = c->Tmax, d = c->d;
+  TRY(dalloc(c, &c->xs, (int64_t)(c->L + 1) * T * d));
+  TRY(dalloc(c, &c->n1, T * d));
+  TRY(dalloc(c, &c->qkv, T * c->dqkv));
+  TRY(dalloc(c, &c->o, T * c->dq));
+  TRY(dalloc(c, &c->h, T * d));
+  TRY(dalloc(c, &c->n2, T * d));
+  TRY(dalloc(c, &c->gu, T * 2 * c->F));
+  TRY(dalloc(c, &c->m, T * c->F));
+  TRY(dalloc(c, &c->rstd1, T));
+  TRY(dalloc(c, &c->rstd2, T));
+  TRY(dalloc(c, &c->lse, T * c->hq));
+  TRY(dalloc(c, &c->Dbuf, T * c->hq));
+  int64_t part = 0;
+  for (int g = 0; g < NGROUP; ++g) {
+    const Group& G = c->grp[g];
+    TRY(dalloc(c, &c->U[g], T * G.R));
+    TRY(dalloc(c, &c->Us[g], T * G.KP, true));
+    TRY(dalloc(c, &c->Vv[g], T * G.R));
+    TRY(dalloc(c, &c->Vs[g], T * G.KP, true));
+    part = std::max(part, (int64_t)G.R * G.in);
+    part = std::max(part, (int64_t)c->r * G.out);
+  }
+  TRY(dalloc(c, &c->part, part * ((T + 127) / 128)));
+  TRY(dalloc(c, &c->ga, T * d));
+  TRY(dalloc(c, &c->gb, T * d));
+  TRY(dalloc(c, &c->dn, T * d));
+  TRY(dalloc(c, &c->dm, T * c->F));
+  TRY(dalloc(c, &c->dout_b, T * d));
+  TRY(dalloc(c, &c->dh_b, T * d));
+  TRY(dalloc(c, &c->do_b, T * c->dq));
+  TRY(dalloc(c, &c->dqkvb, T * c->dqkv));
+  TRY(dalloc(c, &c->dgu, T * 2 * c->F));
+  TRY(dalloc(c, &c->loss_dev, 1, true));
+  TRY(dalloc(c, &c->dot_part, 1024));
+  TRY(dalloc(c, &c->cos_t, (int64_t)k.max_seq * c->hd / 2));
+  TRY(dalloc(c, &c->sin_t, (int64_t)k.max_seq * c->hd / 2));
+  CK(rope_tables(k.max_seq, c->hd, (double)k.rope_theta, c->cos_t, c->sin_t, c->stream));
+  {
+    void* hl = nullptr;
+    CK(cudaHostAlloc(&hl, 64, cudaHostAllocDefault));
+    c->host_loss = static_cast<float*>(hl);
+  }
+  if (c->V > 0) {
+    const int64_t Vd = (int64_t)c->V * d;
+    TRY(dalloc(c, &c->E, Vd));
+    TRY(dalloc(c, &c->H, Vd));
+    TRY(dalloc(c, &c->gf, d));
+    TRY(upload_bf16(c, c->E, embed, Vd));
+    TRY(upload_bf16(c, c->H, lm_head, Vd));
+    TRY(copy_in(c, c->gf, final_norm, d * 4));
+    TRY(dalloc(c, &c->nf, T * d));
+    TRY(dalloc(c, &c->rstdf, T));
+    TRY(dalloc(c, &c->logits, T * c->V));
+    TRY(dalloc(c, &c->dlog, T * c->V));
+    TRY(dalloc(c, &c->loss_rows, T));
+    TRY(dalloc(c, &c->tok, T));
+    TRY(dalloc(c, &c->tgt, T));
+  } else {
+    TRY(dalloc(c, &c->gbuf, T * d));
+  }
+  c->ev_loaded.resize(2 * c->L);
+  c->ev_free.resize(2 * c->L);
+  for (int i = 0; i < 2 * c->L; ++i) {
+    CK(cudaEventCreateWithFlags(&c->ev_loaded[i], cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&c->ev_free[i], cudaEventDisableTiming));
+  }
+  CK(cudaEventCreateWithFlags(&c->ev_done, cudaEventDisableTiming));
+  CK(cudaEventCreate(&c->prof_step0));
+  CK(cudaEventCreate(&c->prof_step1));
+  CK(cudaStreamSynchronize(c->stream));
+  c->st.device_bytes = c->dev_bytes;
+  return LST_OK;
+}
+
+void free_all(lst_ctx* c) {
+  if (c->stream) cudaStreamSynchronize(c->stream);
+  if (c->copy_stream) cudaStreamSynchronize(c->copy_stream);
+  for (void* p : c->dev_allocs) cudaFree(p);
+  c->dev_allocs.clear();
+  if (c->stage_w) cudaFree(c->stage_w);
+  if (c->stage_blob) cudaFree(c->stage_blob);
+  if (c->stage_absmax) cudaFree(c->stage_absmax);
+  if (c->stage_gsum) cudaFree(c->stage_gsum);
+  if (c->arena) cudaFreeHost(c->arena);
+  if (c->host_loss) cudaFreeHost(c->host_loss);
+  for (auto e : c->ev_loaded) cudaEventDestroy(e);
+  for (auto e : c->ev_free) cudaEventDestroy(e);
+  for (auto e : c->prof_pool) cudaEventDestroy(e);
+  if (c->ev_done) cudaEventDestroy(c->ev_done);
+  if (c->prof_step0) cudaEventDestroy(c->prof_step0);
+  if (c->prof_step1) cudaEventDestroy(c->prof_step1);
+  if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
+  if (c->own_stream && c->stream) cudaStreamDestroy(c->stream);
+  cudaGetLastError();
+}
+
+lst_status ensure_staging(lst_ctx* c) {
+  if (c->stage_blob) return LST_OK;
+  int64_t maxn = 0;
+  for (int p = 0; p < NPROJ; ++p) maxn = std::max(maxn, c->lay.n[p]);
+  CK(cudaMalloc(&c->stage_w, maxn * 4));
+  CK(cudaMalloc(&c->stage_blob, c->lay.total));
+  CK(cudaMalloc(&c->stage_absmax, (maxn / 64) * 4));
+  CK(cudaMalloc(&c->stage_gsum, ((maxn / 64 + 255) / 256) * 8));
+  return LST_OK;
+}
+
+void release_staging(lst_ctx* c) {
+  cudaStreamSynchronize(c->stream);
+  cudaFree(c->stage_w);
+  cudaFree(c->stage_blob);
+  cudaFree(c->stage_absmax);
+  cudaFree(c->stage_gsum);
+  c->stage_w = nullptr;
+  c->stage_blob = nullptr;
+  c->stage_absmax = nullptr;
+  c->stage_gsum = nullptr;
+}
+
+lst_status register_impl(lst_ctx* c, int layer, const lst_layer_weights* w) {
+  const lst_config& k = c->cfg;
+  for (int p = 0; p < NPROJ; ++p)
+    if (!w->w[p] || !w->lora_a[p] || !w->lora_b[p]) return fail(c, LST_ERR_ARG, "null weight pointer");
+  if (!w->attn_norm || !w->mlp_norm) return fail(c, LST_ERR_ARG, "null norm pointer");
+  if (k.qkv_bias && (!w->bias[0] || !w->bias[1] || !w->bias[2])) return fail(c, LST_ERR_ARG, "qkv_bias needs 3 biases");
+  TRY(ensure_staging(c));
+  CK(cudaMemsetAsync(c->stage_blob, 0, c->lay.total, c->stream));
+  for (int p = 0; p < NPROJ; ++p) {
+    const int64_t n = c->lay.n[p];
+    const float* src = w->w[p];
+    if (!is_device_ptr(src)) {
+      CK(cudaMemcpyAsync(c->stage_w, src, n * 4, cudaMemcpyHostToDevice, c->stream));
+      src = c->stage_w;
+    }
+    if (k.base_format == LST_BASE_NF4) {
+      Nf4Out o;
+      o.packed = c->stage_blob + c->lay.packed[p];
+      o.qabs = reinterpret_cast<int8_t*>(c->stage_blob + c->lay.qabs[p]);
+      o.gscale = reinterpret_cast<float*>(c->stage_blob + c->lay.gscale[p]);
+      o.mean = reinterpret_cast<float*>(c->stage_blob + c->lay.means) + p;
+      CK(nf4_quantize(src, n, o, c->stage_absmax, c->stage_gsum, c->stream));
+    } else {
+      CK(f32_to_bf16(src, n, reinterpret_cast<__nv_bfloat16*>(c->stage_blob + c->lay.w16) + c->lay.woff[p],
+                     c->stream));
+    }
+    CK(cudaStreamSynchronize(c->stream));  // stage_w is reused by the next projection
+  }
+  TRY(copy_in(c, c->stage_blob + c->lay.norms, w->attn_norm, c->d * 4));
+  TRY(copy_in(c, c->stage_blob + c->lay.norms + c->d * 4, w->mlp_norm, c->d * 4));
+  if (k.qkv_bias) {
+    float* b = reinterpret_cast<float*>(c->stage_blob + c->lay.bias);
+    TRY(copy_in(c, b, w->bias[0], c->dq * 4));
+    TRY(copy_in(c, b + c->dq, w->bias[1], c->dkv * 4));
+    TRY(copy_in(c, b + c->dq + c->dkv, w->bias[2], c->dkv * 4));
+  }
+  if (k.streamed) {
+    CK(cudaMemcpyAsync(c->arena + (int64_t)layer * c->lay.total, c->stage_blob, c->lay.total,
+                       cudaMemcpyDeviceToHost, c->stream));
+  } else {
+    CK(cudaMemcpyAsync(c->resident + (int64_t)layer * c->lay.total, c->stage_blob, c->lay.total,
+                       cudaMemcpyDeviceToDevice, c->stream));
+  }
+  for (int p = 0; p < NPROJ; ++p) {
+    TRY(copy_in(c, c->lora + c->offA[layer * NPROJ + p], w->lora_a[p], (int64_t)c->r * c->lay.ind[p] * 4));
+    TRY(copy_in(c, c->lora + c->offB[layer * NPROJ + p], w->lora_b[p], c->lay.outd[p] * c->r * 4));
+  }
+  TRY(prep_lora(c, layer));
+  CK(cudaStreamSynchronize(c->stream));
+  int derr = 0;
+  CK(cudaMemcpyFromSymbol(&derr, g_lst_dev_error, sizeof(int)));
+  if (derr) return fail(c, LST_ERR_DEVICE, "device error during registration");
+  c->registered[layer] = 1;
+  bool all = true;
+  for (int i = 0; i < c->L; ++i) all = all && c->registered[i];
+  if (all) release_staging(c);
+  return LST_OK;
+}
+
+}  // namespace
+
+namespace lst {
+void note_launch(int n) { g_launch_count.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace lst
+
+// =========================================================================== C ABI
+extern "C" {
+
+lst_status lst_create(const lst_config* cfg, const float* embed, const float* final_norm, const float* lm_head,
+                      void* cuda_stream, lst_ctx** out) {
+  if (!out) return LST_ERR_ARG;
+  *out = nullptr;
+  std::string why;
+  if (!valid_config(cfg, &why)) return LST_ERR_ARG;
+  if ((cfg->vocab > 0) != (embed && final_norm && lm_head)) return LST_ERR_ARG;
+  if (cfg->vocab == 0 && (embed || final_norm || lm_head)) return LST_ERR_ARG;
+  lst_ctx* c = new lst_ctx();
+  c->cfg = *cfg;
+  lst_status s = create_impl(c, embed, final_norm, lm_head, cuda_stream);
+  if (s != LST_OK) {
+    free_all(c);
+    delete c;
+    return s;
+  }
+  *out = c;
+  return LST_OK;
+}
+
+lst_status lst_register_layer(lst_ctx* c, int32_t layer, const lst_layer_weights* w) {
+  if (!c) return LST_ERR_ARG;
+  if (!w || layer < 0 || layer >= c->L) return fail(c, LST_ERR_ARG, "bad layer index or null weights");
+  return register_impl(c, layer, w);
+}
+
+lst_status lst_set_lora(lst_ctx* c, int32_t layer, int32_t proj, const float* a, const float* b) {
+  if (!c) return LST_ERR_ARG;
+  if (layer < 0 || layer >= c->L || proj < 0 || proj >= NPROJ || !a || !b)
+    return fail(c, LST_ERR_ARG, "bad layer/projection or null pointer");
+  TRY(copy_in(c, c->lora + c->offA[layer * NPROJ + proj], a, (int64_t)c->r * c->lay.ind[proj] * 4));
+  TRY(copy_in(c, c->lora + c->offB[layer * NPROJ + proj], b, c->lay.outd[proj] * c->r * 4));
+  TRY(prep_lora(c, layer));
+  CK(cudaStreamSynchronize(c->stream));
+  return LST_OK;
+}
+
+int64_t lst_lora_numel(const lst_ctx* c) { return c ? c->lora_numel : 0; }
+
+lst_status lst_step(lst_ctx* c, const int32_t* tokens, const int32_t* targets, int32_t batch, int32_t seq,
+                    float* loss, float* grads) {
+  if (!c) return LST_ERR_ARG;
+  if (!tokens || !targets || !loss) return fail(c, LST_ERR_ARG, "null tokens/targets/loss");
+  if (c->V <= 0) return fail(c, LST_ERR_STATE, "lst_step needs a head (vocab > 0); use lst_step_hidden");
+  TRY(begin_step(c, batch, seq));
+  TRY(copy_in(c, c->tok, tokens, c->curT * 4));
+  TRY(copy_in(c, c->tgt, targets, c->curT * 4));
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(embed(c->tok, c->E, c->curT, c->d, c->V, c->xs, c->stream));
+  }
+  TRY(run_layers(c, true));
+  c->have_logits = true;
+  return finish_step(c, loss, grads);
+}
+
+lst_status lst_step_hidden(lst_ctx* c, const uint16_t* x, const uint16_t* g, int32_t batch, int32_t seq,
+                           float* loss, float* grads) {
+  if (!c) return LST_ERR_ARG;
+  if (!x || !g || !loss) return fail(c, LST_ERR_ARG, "null x/g/loss");
+  if (c->V != 0) return fail(c, LST_ERR_STATE, "lst_step_hidden needs a headless config (vocab == 0)");
+  TRY(begin_step(c, batch, seq));
+  TRY(copy_in(c, c->xs, x, c->curT * c->d * 2));
+  TRY(copy_in(c, c->gbuf, g, c->curT * c->d * 2));
+  TRY(run_layers(c, false));
+  c->have_logits = false;
+  return finish_step(c, loss, grads);
+}
+
+lst_status lst_get_logits(lst_ctx* c, float* dst) {
+  if (!c) return LST_ERR_ARG;
+  if (!dst) return fail(c, LST_ERR_ARG, "null dst");
+  if (!c->have_logits) return fail(c, LST_ERR_STATE, "no logits: run lst_step first");
+  const bool dev = is_device_ptr(dst);
+  CK(cudaMemcpyAsync(dst, c->logits, c->curT * c->V * 4, dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
+                     c->stream));
+  CK(cudaStreamSynchronize(c->stream));
+  return LST_OK;
+}
+
+lst_status lst_set_profiling(lst_ctx* c, int32_t on) {
+  if (!c) return LST_ERR_ARG;
+  c->profiling = on != 0;
+  return LST_OK;
+}
+
+lst_status lst_get_stats(const lst_ctx* c, lst_stats* out) {
+  if (!c || !out) return LST_ERR_ARG;
+  *out = c->st;
+  out->device_bytes = c->dev_bytes;
+  return LST_OK;
+}
+
+const char* lst_last_error(const lst_ctx* c) { return c ? c->err.c_str() : "null context"; }
+
+void lst_destroy(lst_ctx* c) {
+  if (!c) return;
+  free_all(c);
+  delete c;
+}
+
+lst_status lst_nf4_codebook(float out[16]) {
+  if (!out) return LST_ERR_ARG;
+  nf4_codebook(out);
+  return LST_OK;
+}
+
+int64_t lst_blob_bytes(const lst_config* cfg) {
+  std::string why;
+  if (!valid_config(cfg, &why)) return -1;
+  return make_layout(*cfg).total;
+}
+
+}  // extern "C"

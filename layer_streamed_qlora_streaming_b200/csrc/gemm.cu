@@ -1,0 +1,296 @@
+// bf16 GEMM on the 5th-generation tensor cores (tcgen05.mma kind::f16, fp32 accumulate in TMEM).
+//
+// One CTA computes a 128 x BN tile (BN = 64, 128 or 256) with three warp roles:
+//   warp 0  : TMA producer (one thread) -- A and B tiles, 64 K-elements per stage, 128-byte
+//             swizzle, into a ring of shared-memory stages guarded by full/empty mbarriers;
+//   warp 1  : TMEM allocator and MMA issuer (one thread) -- 4 x tcgen05.mma (K = 16) per stage,
+//             tcgen05.commit frees the stage when the tensor core has read it;
+//   warps 2-5: epilogue -- tcgen05.ld of 32 fp32 columns per thread (one accumulator row per
+//             thread), scale / bias / residual, store bf16 or fp32.
+// The optional second operand pair (A2, B2) is streamed as extra K-blocks after the main ones.
+#include "common.cuh"
+#include "gemm.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace lst {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+
+struct Epi {
+  void* C;
+  int64_t ldc;
+  const float* bias;
+  const __nv_bfloat16* R;
+  int64_t ldr;
+  float alpha;
+  int c_f32;
+  int M, N;
+};
+
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t SMEM = STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*bars*/;
+  static constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;
+};
+
+__device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const uint32_t (&r)[32]) {
+  if (row >= e.M || col0 >= e.N) return;
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * e.alpha;
+  const bool full = col0 + 32 <= e.N;
+  if (e.bias) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (full || col0 + i < e.N) v[i] += e.bias[col0 + i];
+  }
+  if (e.R) {
+    const __nv_bfloat16* rp = e.R + (int64_t)row * e.ldr + col0;
+    if (full && ((reinterpret_cast<uintptr_t>(rp) & 15) == 0)) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 u = *reinterpret_cast<const uint4*>(rp + q * 8);
+        const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[q * 8 + i] += __bfloat162float(b[i]);
+      }
+    } else {
+      for (int i = 0; i < 32; ++i)
+        if (col0 + i < e.N) v[i] += __bfloat162float(rp[i]);
+    }
+  }
+  if (e.c_f32) {
+    float* cp = reinterpret_cast<float*>(e.C) + (int64_t)row * e.ldc + col0;
+    if (full && ((reinterpret_cast<uintptr_t>(cp) & 15) == 0)) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<float4*>(cp + q * 4) = make_float4(v[q * 4], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
+    } else {
+      for (int i = 0; i < 32; ++i)
+        if (col0 + i < e.N) cp[i] = v[i];
+    }
+  } else {
+    __nv_bfloat16* cp = reinterpret_cast<__nv_bfloat16*>(e.C) + (int64_t)row * e.ldc + col0;
+    if (full && ((reinterpret_cast<uintptr_t>(cp) & 15) == 0)) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 u;
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+        *reinterpret_cast<uint4*>(cp + q * 8) = u;
+      }
+    } else {
+      for (int i = 0; i < 32; ++i)
+        if (col0 + i < e.N) cp[i] = __float2bfloat16_rn(v[i]);
+    }
+  }
+}
+
+template <int BN, int BMN>
+__global__ void __launch_bounds__(192, 1)
+k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+       const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+       const Epi ep, const int nk1, const int nk2) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* accf = empty + C::STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * BM;
+  const int n0 = blockIdx.x * BN;
+  const int nk = nk1 + nk2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (nk2) {
+      tma_prefetch_desc(&tmA2);
+      tma_prefetch_desc(&tmB2);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % C::STAGES;
+        const uint32_t ph = (kb / C::STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1)) break;
+        mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
+        const bool second = kb >= nk1;
+        const CUtensorMap* ma = second ? &tmA2 : &tmA;
+        const CUtensorMap* mb = second ? &tmB2 : &tmB;
+        const int kk = (second ? kb - nk1 : kb) * BK;
+        tma_load_2d(sA + s * C::A_BYTES, ma, &full[s], kk, m0);
+        if (BMN == 0) {
+          tma_load_2d(sB + s * C::B_BYTES, mb, &full[s], kk, n0);
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN / 64; ++c)
+            tma_load_2d(sB + s * C::B_BYTES + c * (64 * BK * 2), mb, &full[s], n0 + c * 64, kk);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(BM, BN, BMN);
+      bool ok = true;
+      for (int kb = 0; kb < nk && ok; ++kb) {
+        const int s = kb % C::STAGES;
+        const uint32_t ph = (kb / C::STAGES) & 1;
+        ok = mbar_wait(&full[s], ph);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s * C::A_BYTES);
+        const uint32_t b0 = smem_u32(sB + s * C::B_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          const uint64_t da = umma_desc(a0 + k * 32, 16, 1024);
+          const uint64_t db = BMN ? umma_desc(b0 + k * 16 * 128, 64 * BK * 2, 1024)
+                                  : umma_desc(b0 + k * 32, 16, 1024);
+          umma_bf16(tmem, da, db, idesc, (kb | k) != 0);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accf);
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    mbar_wait(accf, 0);
+    tc_fence_after();
+    const int row = m0 + q * 32 + lane;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + c, r);
+      tmem_ld_wait();
+      epi_store(ep, row, n0 + c, r);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 tensor map over a row-major [rows, cols] matrix with row stride ld (elements),
+// box = [box_rows, 64 columns], 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int BMN>
+cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
+  using C = Cfg<BN>;
+  CUtensorMap tA, tB, tA2, tB2;
+  const int box_b = BMN ? BK : BN;  // K-major B: box [BN rows, 64 k]; MN-major: [64 k rows, 64 n]
+  if (!make_map(&tA, a.A, a.M, a.K, a.lda, BM)) return cudaErrorInvalidValue;
+  if (BMN) {
+    if (!make_map(&tB, a.B, a.K, a.N, a.ldb, box_b)) return cudaErrorInvalidValue;
+  } else {
+    if (!make_map(&tB, a.B, a.N, a.K, a.ldb, box_b)) return cudaErrorInvalidValue;
+  }
+  int nk2 = 0;
+  if (a.A2 && a.B2 && a.K2 > 0) {
+    if (!make_map(&tA2, a.A2, a.M, a.K2, a.lda2, BM)) return cudaErrorInvalidValue;
+    if (BMN) {
+      if (!make_map(&tB2, a.B2, a.K2, a.N, a.ldb2, box_b)) return cudaErrorInvalidValue;
+    } else {
+      if (!make_map(&tB2, a.B2, a.N, a.K2, a.ldb2, box_b)) return cudaErrorInvalidValue;
+    }
+    nk2 = (a.K2 + BK - 1) / BK;
+  } else {
+    tA2 = tA;
+    tB2 = tB;
+  }
+  Epi e{a.C, a.ldc, a.bias, a.R, a.ldr, a.alpha, a.c_f32, a.M, a.N};
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t err = cudaFuncSetAttribute(k_gemm<BN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (err != cudaSuccess) return err;
+    attr_set = true;
+  }
+  dim3 grid((a.N + BN - 1) / BN, (a.M + BM - 1) / BM);
+  const int nk1 = (a.K + BK - 1) / BK;
+  k_gemm<BN, BMN><<<grid, 192, C::SMEM, s>>>(tA, tB, tA2, tB2, e, nk1, nk2);
+  note_launch(1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t gemm_bf16(const GemmArgs& a, cudaStream_t s) {
+  if (a.M <= 0 || a.N <= 0 || a.K <= 0 || !a.A || !a.B || !a.C) return cudaErrorInvalidValue;
+  // TMA: 16-byte aligned bases and row strides
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  if (!al16(a.A) || !al16(a.B) || (a.lda % 8) || (a.ldb % 8)) return cudaErrorInvalidValue;
+  if (a.A2 && (!al16(a.A2) || !al16(a.B2) || (a.lda2 % 8) || (a.ldb2 % 8))) return cudaErrorInvalidValue;
+  const int64_t tiles256 = (int64_t)((a.M + BM - 1) / BM) * ((a.N + 255) / 256);
+  int bn;
+  if (a.N <= 64) bn = 64;
+  else if (a.N <= 128 || tiles256 < 120) bn = 128;
+  else bn = 256;
+  if (a.b_mn) {
+    if (bn == 64) return launch<64, 1>(a, s);
+    if (bn == 128) return launch<128, 1>(a, s);
+    return launch<256, 1>(a, s);
+  }
+  if (bn == 64) return launch<64, 0>(a, s);
+  if (bn == 128) return launch<128, 0>(a, s);
+  return launch<256, 0>(a, s);
+}
+
+}  // namespace lst

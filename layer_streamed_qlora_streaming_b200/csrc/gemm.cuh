@@ -1,0 +1,41 @@
+// bf16 tensor-core GEMM for sm_100a (tcgen05 + TMEM + TMA), host interface.
+//
+//   C[m, n] = alpha * ( sum_k A[m, k] B(n, k)  +  sum_j A2[m, j] B2(n, j) ) + bias[n] + R[m, n]
+//
+// A, A2 are row-major [M, K] / [M, K2] (K-major). B is either row-major [N, K] (K-major,
+// b_mn = 0, "x W^T") or row-major [K, N] (MN-major, b_mn = 1, "x W"); B2 has the same major-ness.
+// The optional (A2, B2) pair is a second contraction appended along K; the LoRA path uses it
+// to fold s (x A^T) B^T into the same accumulator as the frozen base.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace lst {
+
+struct GemmArgs {
+  int M = 0, N = 0, K = 0;
+  const __nv_bfloat16* A = nullptr;   // [M, K], row stride lda
+  int64_t lda = 0;
+  const __nv_bfloat16* B = nullptr;   // b_mn=0: [N, K]; b_mn=1: [K, N]; row stride ldb
+  int64_t ldb = 0;
+  int b_mn = 0;
+  const __nv_bfloat16* A2 = nullptr;  // optional [M, K2]
+  int64_t lda2 = 0;
+  const __nv_bfloat16* B2 = nullptr;  // optional b_mn=0: [N, K2]; b_mn=1: [K2, N]
+  int64_t ldb2 = 0;
+  int K2 = 0;
+  void* C = nullptr;                  // [M, N] row stride ldc; fp32 if c_f32 else bf16
+  int64_t ldc = 0;
+  int c_f32 = 0;
+  float alpha = 1.0f;
+  const float* bias = nullptr;        // [N] or null
+  const __nv_bfloat16* R = nullptr;   // residual [M, N] row stride ldr, or null
+  int64_t ldr = 0;
+};
+
+// Returns cudaSuccess or the launch / argument error. Deterministic: no split-K, no atomics.
+cudaError_t gemm_bf16(const GemmArgs& a, cudaStream_t s);
+
+}  // namespace lst

@@ -1,0 +1,176 @@
+// C ABI of the individual kernels (include/lst_kernels.h): argument checks and marshalling only.
+#include "../../include/lst_kernels.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "nf4.cuh"
+#include "ops.cuh"
+
+#include <atomic>
+
+namespace lst {
+extern std::atomic<long long> g_launch_count;
+}
+
+using namespace lst;
+
+namespace {
+inline cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
+inline const bf16* B16(const uint16_t* p) { return reinterpret_cast<const bf16*>(p); }
+inline bf16* B16(uint16_t* p) { return reinterpret_cast<bf16*>(p); }
+inline lst_status st(cudaError_t e) {
+  if (e == cudaSuccess) return LST_OK;
+  cudaGetLastError();
+  return e == cudaErrorInvalidValue ? LST_ERR_ARG : LST_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" {
+
+lst_status lst_k_nf4_quantize(const float* w, int64_t n, uint8_t* packed, int8_t* qabs, float* gscale, float* mean,
+                              void* stream) {
+  if (!w || !packed || !qabs || !gscale || !mean || n <= 0 || n % 64) return LST_ERR_ARG;
+  const int64_t nb = n / 64, ng = (nb + 255) / 256;
+  float* absmax = nullptr;
+  double* gsum = nullptr;
+  if (cudaMalloc(&absmax, nb * 4) != cudaSuccess) return LST_ERR_OOM;
+  if (cudaMalloc(&gsum, ng * 8) != cudaSuccess) {
+    cudaFree(absmax);
+    return LST_ERR_OOM;
+  }
+  Nf4Out o{packed, qabs, gscale, mean};
+  cudaError_t e = nf4_quantize(w, n, o, absmax, gsum, S(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(S(stream));
+  cudaFree(absmax);
+  cudaFree(gsum);
+  return st(e);
+}
+
+lst_status lst_k_nf4_dequant(const uint8_t* packed, const int8_t* qabs, const float* gscale, const float* mean,
+                             int64_t n, uint16_t* out, void* stream) {
+  if (!packed || !qabs || !gscale || !mean || !out || n <= 0 || n % 64) return LST_ERR_ARG;
+  Nf4Seg s{packed, qabs, gscale, mean, n, 0};
+  return st(nf4_dequant(&s, 1, B16(out), S(stream)));
+}
+
+lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb,
+                      int32_t b_mn, const uint16_t* A2, int64_t lda2, const uint16_t* B2, int64_t ldb2, int32_t K2,
+                      void* C, int64_t ldc, int32_t c_f32, float alpha, const float* bias, const uint16_t* R,
+                      int64_t ldr, void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0 || !A || !B || !C) return LST_ERR_ARG;
+  if ((A2 == nullptr) != (B2 == nullptr)) return LST_ERR_ARG;
+  GemmArgs a;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.A = B16(A);
+  a.lda = lda;
+  a.B = B16(B);
+  a.ldb = ldb;
+  a.b_mn = b_mn ? 1 : 0;
+  a.A2 = B16(A2);
+  a.lda2 = lda2;
+  a.B2 = B16(B2);
+  a.ldb2 = ldb2;
+  a.K2 = A2 ? K2 : 0;
+  a.C = C;
+  a.ldc = ldc;
+  a.c_f32 = c_f32 ? 1 : 0;
+  a.alpha = alpha;
+  a.bias = bias;
+  a.R = B16(R);
+  a.ldr = ldr;
+  return st(gemm_bf16(a, S(stream)));
+}
+
+lst_status lst_k_attention_fwd(const uint16_t* q, int64_t ldq, const uint16_t* k, int64_t ldk, const uint16_t* v,
+                               int64_t ldv, uint16_t* o, int64_t ldo, float* lse, int64_t T, int32_t Sq, int32_t hq,
+                               int32_t hkv, int32_t hd, void* stream) {
+  if (!q || !k || !v || !o || !lse) return LST_ERR_ARG;
+  AttnArgs a{B16(q), B16(k), B16(v), B16(o), lse, ldq, ldk, ldv, ldo, T, Sq, hq, hkv, hd, 0.f};
+  a.scale = 1.0f / sqrtf((float)hd);
+  return st(attention_fwd(a, S(stream)));
+}
+
+lst_status lst_k_attention_bwd(const uint16_t* q, int64_t ldq, const uint16_t* k, int64_t ldk, const uint16_t* v,
+                               int64_t ldv, const uint16_t* o, int64_t ldo, const uint16_t* dout, int64_t lddo,
+                               const float* lse, float* D, uint16_t* dq, int64_t lddq, uint16_t* dk, int64_t lddk,
+                               uint16_t* dv, int64_t lddv, int64_t T, int32_t Sq, int32_t hq, int32_t hkv, int32_t hd,
+                               void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !D || !dq || !dk || !dv) return LST_ERR_ARG;
+  AttnBwdArgs a;
+  a.q = B16(q);
+  a.k = B16(k);
+  a.v = B16(v);
+  a.o = B16(o);
+  a.dout = B16(dout);
+  a.lse = lse;
+  a.D = D;
+  a.dq = B16(dq);
+  a.dk = B16(dk);
+  a.dv = B16(dv);
+  a.ldq = ldq;
+  a.ldk = ldk;
+  a.ldv = ldv;
+  a.ldo = ldo;
+  a.lddo = lddo;
+  a.lddq = lddq;
+  a.lddk = lddk;
+  a.lddv = lddv;
+  a.T = T;
+  a.S = Sq;
+  a.hq = hq;
+  a.hkv = hkv;
+  a.hd = hd;
+  a.scale = 1.0f / sqrtf((float)hd);
+  return st(attention_bwd(a, S(stream)));
+}
+
+lst_status lst_k_rmsnorm_fwd(const uint16_t* x, const float* g, int64_t T, int32_t d, float eps, uint16_t* y,
+                             float* rstd, void* stream) {
+  if (!x || !g || !y || !rstd || T <= 0 || d <= 0) return LST_ERR_ARG;
+  return st(rmsnorm_fwd(B16(x), g, T, d, eps, B16(y), rstd, S(stream)));
+}
+
+lst_status lst_k_rmsnorm_bwd(const float* dy, const uint16_t* x, const float* g, const float* rstd, const float* dres,
+                             int64_t T, int32_t d, float* dx, uint16_t* dxb, void* stream) {
+  if (!dy || !x || !g || !rstd || !dx || T <= 0 || d <= 0) return LST_ERR_ARG;
+  return st(rmsnorm_bwd(dy, B16(x), g, rstd, dres, T, d, dx, B16(dxb), S(stream)));
+}
+
+lst_status lst_k_rope_tables(int32_t Sq, int32_t hd, double theta, float* ct, float* sn, void* stream) {
+  if (!ct || !sn || Sq <= 0 || hd <= 0 || hd % 2) return LST_ERR_ARG;
+  return st(rope_tables(Sq, hd, theta, ct, sn, S(stream)));
+}
+
+lst_status lst_k_rope(uint16_t* buf, int64_t ld, int64_t T, int32_t Sq, int32_t col0, int32_t nh, int32_t hd,
+                      const float* ct, const float* sn, int32_t inverse, void* stream) {
+  if (!buf || !ct || !sn || T <= 0 || Sq <= 0) return LST_ERR_ARG;
+  return st(rope(B16(buf), ld, T, Sq, col0, nh, hd, ct, sn, inverse, S(stream)));
+}
+
+lst_status lst_k_swiglu_fwd(const uint16_t* gu, int64_t T, int32_t F, uint16_t* m, void* stream) {
+  if (!gu || !m || T <= 0 || F <= 0) return LST_ERR_ARG;
+  return st(swiglu_fwd(B16(gu), T, F, B16(m), S(stream)));
+}
+
+lst_status lst_k_swiglu_bwd(const float* dm, const uint16_t* gu, int64_t T, int32_t F, uint16_t* dgu, void* stream) {
+  if (!dm || !gu || !dgu || T <= 0 || F <= 0) return LST_ERR_ARG;
+  return st(swiglu_bwd(dm, B16(gu), T, F, B16(dgu), S(stream)));
+}
+
+lst_status lst_k_cross_entropy(const float* logits, int64_t T, int32_t V, const int32_t* targets, float inv_T,
+                               float* loss_rows, uint16_t* dlogits, void* stream) {
+  if (!logits || !targets || !loss_rows || !dlogits || T <= 0 || V <= 0) return LST_ERR_ARG;
+  return st(cross_entropy(logits, T, V, targets, inv_T, loss_rows, B16(dlogits), S(stream)));
+}
+
+lst_status lst_k_lora_project(const uint16_t* X, int64_t ldx, int64_t T, int32_t in, const float* A, int32_t R, float s,
+                              float* U, uint16_t* Us, int64_t ldus, void* stream) {
+  if (!X || !A || !U || !Us || T <= 0 || in <= 0 || R <= 0 || R > 64) return LST_ERR_ARG;
+  return st(lora_project(B16(X), ldx, T, in, A, in, R, s, U, B16(Us), ldus, S(stream)));
+}
+
+int64_t lst_k_launch_count(void) { return g_launch_count.load(); }
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+// Memory-bound kernels of the decoder layer and the LoRA side path (host interface). See ops.cu.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace lst {
+
+using bf16 = __nv_bfloat16;
+
+// y = bf16(x * rstd * g), rstd = 1/sqrt(mean(x^2) + eps) per row; rstd saved [T].
+cudaError_t rmsnorm_fwd(const bf16* x, const float* g, int64_t T, int d, float eps, bf16* y, float* rstd,
+                        cudaStream_t s);
+// dx = dres + rstd * (dy*g - xhat * mean(dy*g*xhat)); writes fp32 dx and (optional) bf16 copy.
+cudaError_t rmsnorm_bwd(const float* dy, const bf16* x, const float* g, const float* rstd, const float* dres,
+                        int64_t T, int d, float* dx, bf16* dx_bf16, cudaStream_t s);
+
+// Rotate pairs (j, j + hd/2) of the first nh heads of each row of buf (row stride ld) by the
+// angle of position (t mod S): cos/sin tables [S_max, hd/2]. inverse = 1 rotates backwards.
+cudaError_t rope(bf16* buf, int64_t ld, int64_t T, int S, int col0, int nh, int hd, const float* cos_t,
+                 const float* sin_t, int inverse, cudaStream_t s);
+// cos/sin of pos * theta^(-2j/hd) computed in fp64, stored fp32 [S, hd/2].
+cudaError_t rope_tables(int S, int hd, double theta, float* cos_t, float* sin_t, cudaStream_t s);
+
+// m = bf16(silu(g) * u) where gu = [g | u] along columns ([T, 2F]).
+cudaError_t swiglu_fwd(const bf16* gu, int64_t T, int F, bf16* m, cudaStream_t s);
+// dgu = [dm * u * silu'(g) | dm * silu(g)] (bf16), dm fp32 [T, F].
+cudaError_t swiglu_bwd(const float* dm, const bf16* gu, int64_t T, int F, bf16* dgu, cudaStream_t s);
+
+cudaError_t embed(const int32_t* tok, const bf16* E, int64_t T, int d, int vocab, bf16* x, cudaStream_t s);
+
+// Cross-entropy rows: loss_t = lse_t - logit[t, y_t]; dlogits = (softmax - onehot) * inv_T (bf16).
+cudaError_t cross_entropy(const float* logits, int64_t T, int V, const int32_t* targets, float inv_T,
+                          float* loss_rows, bf16* dlogits, cudaStream_t s);
+// out = mean of v[0..n) with a fixed summation order.
+cudaError_t mean_fixed(const float* v, int64_t n, float* out, cudaStream_t s);
+// out = sum_i a[i] * b[i] (bf16 inputs) with a fixed order; partials: scratch of 1024 floats.
+cudaError_t dot_fixed(const bf16* a, const bf16* b, int64_t n, float* partials, float* out, cudaStream_t s);
+
+cudaError_t f32_to_bf16(const float* x, int64_t n, bf16* y, cudaStream_t s);
+
+// ------------------------------------------------------------------------ LoRA side path
+// U[t, j] = sum_i X[t, i] * A[j, i] for j < R (A fp32 [R, in] row stride lda); writes U fp32
+// [T, R] (row stride R) and Us = bf16(s * U) [T, ldus].
+cudaError_t lora_project(const bf16* X, int64_t ldx, int64_t T, int in, const float* A, int64_t lda, int R,
+                         float s, float* U, bf16* Us, int64_t ldus, cudaStream_t st);
+
+// Fixed-order reduction over tokens of out[j, c] = s * sum_t P[t, j] * Q[t, c].
+// P fp32 [T, R] (row stride R), Q bf16 [T, ldq] with C columns. If seg_r > 0 the columns are
+// split in up to 3 segments by bounds[0..nseg]; column c of segment p only pairs with
+// j in [p*seg_r, p*seg_r + seg_r) and the result goes to dst[p] + (c - bounds[p]) * seg_r + j
+// ("dB" layout [out_p, r]). If seg_r == 0, row j goes to dst[j / rows_per_dst] +
+// (j % rows_per_dst) * C + c ("dA" layout [r, in]). partial: scratch of
+// ceil(T/128) * (seg_r ? seg_r : R) * C floats.
+struct LoraGradArgs {
+  const float* P;
+  int R;
+  const bf16* Q;
+  int64_t ldq;
+  int C;
+  int64_t T;
+  float s;
+  int seg_r;
+  int nseg;
+  int bounds[4];
+  float* dst[4];
+  int rows_per_dst;
+  float* partial;
+};
+cudaError_t lora_grad(const LoraGradArgs& a, cudaStream_t st);
+
+// Build the derived LoRA operands of one fused projection group (nseg segments with own A_p
+// [r, in], B_p [out_p, r] fp32):
+//   Acat32 [R, in], Acat16 [KP, in] (rows >= R zero), BexpT32 [R, out] (segment-masked),
+//   Bexp16 [out, KP] (segment-masked, columns >= R zero), R = nseg * r.
+struct LoraPrepArgs {
+  const float* A[3];
+  const float* B[3];
+  int nseg, r, in;
+  int bounds[4];  // out-row bounds of the segments
+  int KP;
+  float* Acat32;
+  bf16* Acat16;
+  float* BexpT32;
+  bf16* Bexp16;
+};
+cudaError_t lora_prep(const LoraPrepArgs& a, cudaStream_t st);
+
+}  // namespace lst

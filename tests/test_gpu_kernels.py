@@ -1,0 +1,261 @@
+"""Kernel-level parity of the CUDA library against the oracle (GPU). Every call goes through the
+C ABI (include/lst_kernels.h)."""
+import numpy as np
+import pytest
+
+import synthetic as syn
+from oracle import model as M
+from oracle import nf4
+from helpers import cosine, maxrel, to_np, torch_bf16, torch_f32
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+lst = pytest.importorskip("layer_streamed_qlora_streaming_b200")
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _bf(x):
+    return syn.round_bf16(np.asarray(x, dtype=np.float32))
+
+
+# ------------------------------------------------------------------------------------ NF4
+@pytest.mark.parametrize("shape", [(256, 256), (688, 256), (256, 688), (1024, 4096), (14336, 4096),
+                                   (27648, 5120)])
+def test_nf4_quantize_and_dequant_bit_exact(shape):
+    n = shape[0] * shape[1]
+    w = syn.normal(11, shape[0], n, 0.02).astype(np.float32).reshape(shape)
+    if shape == (256, 256):
+        w[3, :64] = 0.0                      # an all-zero block
+        w[5, 64:128] = 1e-3                  # a constant block
+    ref = nf4.quantize(w)
+    wd = torch_f32(w)
+    packed = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
+    qabs = torch.empty(n // 64, dtype=torch.int8, device="cuda")
+    gsc = torch.empty(ref.gscale.size, dtype=torch.float32, device="cuda")
+    mean = torch.empty(1, dtype=torch.float32, device="cuda")
+    lst.k_nf4_quantize(wd, packed, qabs, gsc, mean)
+    torch.cuda.synchronize()
+    assert np.array_equal(packed.cpu().numpy(), ref.packed)
+    assert np.array_equal(qabs.cpu().numpy(), ref.qabs)
+    assert np.array_equal(gsc.cpu().numpy().view(np.uint32), ref.gscale.view(np.uint32))
+    assert mean.cpu().numpy().view(np.uint32)[0] == np.float32(ref.mean).view(np.uint32)
+    out = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    lst.k_nf4_dequant(packed, qabs, gsc, mean, n, out)
+    torch.cuda.synchronize()
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, nf4.dequantize_bits(ref).reshape(-1))
+
+
+# ------------------------------------------------------------------------------------ GEMM
+GEMM_CASES = [
+    # M, N, K, b_mn, ext, out_f32, bias, resid
+    (128, 256, 64, 0, False, True, False, False),
+    (300, 520, 200, 0, False, True, False, False),      # ragged M / N / K tails
+    (256, 1000, 688, 1, False, True, False, False),     # MN-major B, ragged
+    (128, 64, 128, 0, False, True, False, False),       # BN = 64
+    (384, 768, 256, 0, True, False, True, True),        # LoRA extension + bias + residual, bf16 out
+    (256, 1536, 512, 1, True, True, False, False),      # MN-major with extension
+    (2048, 6144, 4096, 0, True, False, False, False),   # fused q/k/v of an 8B layer
+    (2048, 4096, 14336, 1, True, True, False, False),   # dX of the 8B down projection
+]
+
+
+@pytest.mark.parametrize("M,N,K,b_mn,ext,f32,bias,resid", GEMM_CASES)
+def test_gemm(M, N, K, b_mn, ext, f32, bias, resid):
+    r = _rng(M + N + K)
+    A = _bf(r.normal(size=(M, K)))
+    B = _bf(r.normal(size=(K, N) if b_mn else (N, K)) * 0.05)
+    ref = A.astype(np.float64) @ (B if b_mn else B.T).astype(np.float64)
+    kw = {}
+    if ext:
+        A2 = np.zeros((M, 64), np.float32)
+        A2[:, :48] = _bf(r.normal(size=(M, 48)))
+        B2 = np.zeros((64, N) if b_mn else (N, 64), np.float32)
+        if b_mn:
+            B2[:48] = _bf(r.normal(size=(48, N)) * 0.1)
+        else:
+            B2[:, :48] = _bf(r.normal(size=(N, 48)) * 0.1)
+        ref = ref + A2.astype(np.float64) @ (B2 if b_mn else B2.T).astype(np.float64)
+        kw.update(A2=torch_bf16(A2), lda2=64, B2=torch_bf16(B2), ldb2=N if b_mn else 64, K2=64)
+    if bias:
+        bv = r.normal(size=N).astype(np.float32)
+        ref = ref + bv
+        kw["bias"] = torch_f32(bv)
+    if resid:
+        Rv = _bf(r.normal(size=(M, N)))
+        ref = ref + Rv
+        kw.update(R=torch_bf16(Rv), ldr=N)
+    C = torch.zeros(M, N, dtype=torch.float32 if f32 else torch.bfloat16, device="cuda")
+    lst.k_gemm(M, N, K, torch_bf16(A), K, torch_bf16(B), N if b_mn else K, b_mn, C, N, int(f32), **kw)
+    torch.cuda.synchronize()
+    got = to_np(C)
+    tol = 1e-4 if f32 else 8e-3
+    assert maxrel(got, ref) < tol, maxrel(got, ref)
+
+
+def test_gemm_rejects_misaligned_stride():
+    A = torch.zeros(128, 100, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lst.LstError):
+        lst.k_gemm(128, 128, 100, A, 100, A, 100, 0, torch.zeros(128, 128, device="cuda"), 128, 1)
+
+
+# ------------------------------------------------------------------------------------ attention
+@pytest.mark.parametrize("B,S,hq,hkv,hd", [(2, 64, 4, 4, 64), (2, 100, 4, 2, 64), (1, 200, 4, 1, 128),
+                                           (2, 128, 8, 2, 128)])
+def test_attention_fwd_bwd(B, S, hq, hkv, hd):
+    r = _rng(S * hq + hd)
+    T = B * S
+    ldq = (hq + 2 * hkv) * hd
+    qkv = _bf(r.normal(size=(T, ldq)))
+    q = qkv[:, :hq * hd].reshape(T, hq, hd)
+    k = qkv[:, hq * hd:(hq + hkv) * hd].reshape(T, hkv, hd)
+    v = qkv[:, (hq + hkv) * hd:].reshape(T, hkv, hd)
+    o_ref, P = M.attention(q.astype(np.float64), k.astype(np.float64), v.astype(np.float64), B, S)
+    tq = torch_bf16(qkv)
+    o = torch.empty(T, hq * hd, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(T, hq, dtype=torch.float32, device="cuda")
+    lst.k_attention_fwd(tq, ldq, tq[:, hq * hd:], ldq, tq[:, (hq + hkv) * hd:], ldq, o, hq * hd, lse,
+                        T, S, hq, hkv, hd)
+    torch.cuda.synchronize()
+    og = to_np(o).reshape(T, hq, hd)
+    assert maxrel(og, o_ref) < 1e-2
+    assert cosine(og, o_ref) > 0.9999
+    # backward, upstream gradient dO ~ N(0,1)
+    do = _bf(r.normal(size=(T, hq * hd)))
+    dq_r, dk_r, dv_r = M.attention_bwd(do.reshape(T, hq, hd).astype(np.float64), q.astype(np.float64),
+                                       k.astype(np.float64), v.astype(np.float64), P, B, S)
+    dqkv = torch.zeros(T, ldq, dtype=torch.bfloat16, device="cuda")
+    Dscr = torch.empty(T, hq, dtype=torch.float32, device="cuda")
+    lst.k_attention_bwd(tq, ldq, tq[:, hq * hd:], ldq, tq[:, (hq + hkv) * hd:], ldq, o, hq * hd,
+                        torch_bf16(do), hq * hd, lse, Dscr, dqkv, ldq, dqkv[:, hq * hd:], ldq,
+                        dqkv[:, (hq + hkv) * hd:], ldq, T, S, hq, hkv, hd)
+    torch.cuda.synchronize()
+    g = to_np(dqkv)
+    for got, ref in ((g[:, :hq * hd], dq_r), (g[:, hq * hd:(hq + hkv) * hd], dk_r), (g[:, (hq + hkv) * hd:], dv_r)):
+        ref = ref.reshape(T, -1)
+        assert cosine(got, ref) > 0.999, cosine(got, ref)
+        assert maxrel(got, ref) < 2e-2, maxrel(got, ref)
+
+
+def test_attention_deterministic():
+    r = _rng(5)
+    B, S, hq, hkv, hd = 2, 256, 8, 2, 128
+    T, ldq = B * S, (hq + 2 * hkv) * hd
+    tq = torch_bf16(_bf(r.normal(size=(T, ldq))))
+    outs = []
+    for _ in range(2):
+        o = torch.empty(T, hq * hd, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(T, hq, dtype=torch.float32, device="cuda")
+        lst.k_attention_fwd(tq, ldq, tq[:, hq * hd:], ldq, tq[:, (hq + hkv) * hd:], ldq, o, hq * hd, lse,
+                            T, S, hq, hkv, hd)
+        dqkv = torch.zeros(T, ldq, dtype=torch.bfloat16, device="cuda")
+        Dscr = torch.empty(T, hq, dtype=torch.float32, device="cuda")
+        lst.k_attention_bwd(tq, ldq, tq[:, hq * hd:], ldq, tq[:, (hq + hkv) * hd:], ldq, o, hq * hd,
+                            o, hq * hd, lse, Dscr, dqkv, ldq, dqkv[:, hq * hd:], ldq,
+                            dqkv[:, (hq + hkv) * hd:], ldq, T, S, hq, hkv, hd)
+        torch.cuda.synchronize()
+        outs.append(dqkv.view(torch.int16).cpu().numpy())
+    assert np.array_equal(outs[0], outs[1])
+
+
+# ------------------------------------------------------------------------------------ small ops
+def test_rmsnorm_fwd_bwd():
+    r = _rng(6)
+    T, d = 37, 4096
+    x = _bf(r.normal(size=(T, d)))
+    g = r.uniform(0.5, 1.5, size=d).astype(np.float32)
+    y_ref, rs = M.rmsnorm(x.astype(np.float64), g.astype(np.float64), 1e-5)
+    y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    rstd = torch.empty(T, dtype=torch.float32, device="cuda")
+    lst.k_rmsnorm_fwd(torch_bf16(x), torch_f32(g), T, d, 1e-5, y, rstd)
+    dy = r.normal(size=(T, d)).astype(np.float32)
+    dres = r.normal(size=(T, d)).astype(np.float32)
+    dx = torch.empty(T, d, dtype=torch.float32, device="cuda")
+    lst.k_rmsnorm_bwd(torch_f32(dy), torch_bf16(x), torch_f32(g), rstd, torch_f32(dres), T, d, dx)
+    torch.cuda.synchronize()
+    assert maxrel(to_np(y), y_ref) < 8e-3
+    dx_ref = dres + M.rmsnorm_bwd(dy.astype(np.float64), x.astype(np.float64), g.astype(np.float64), rs)
+    assert maxrel(to_np(dx), dx_ref) < 1e-5
+
+
+def test_rope_fwd_inverse():
+    r = _rng(7)
+    B, S, nh, hd = 2, 48, 3, 128
+    T = B * S
+    x = _bf(r.normal(size=(T, nh * hd)))
+    cos_t = torch.empty(S, hd // 2, device="cuda")
+    sin_t = torch.empty(S, hd // 2, device="cuda")
+    lst.k_rope_tables(S, hd, 5e5, cos_t, sin_t)
+    buf = torch_bf16(x)
+    lst.k_rope(buf, nh * hd, T, S, 0, nh, hd, cos_t, sin_t, 0)
+    torch.cuda.synchronize()
+    c, s = M.rope_tables(S, hd, 5e5)
+    ref = M.rope(x.reshape(T, nh, hd).astype(np.float64), c, s, B, S).reshape(T, -1)
+    assert maxrel(to_np(buf), ref) < 8e-3
+    dy = r.normal(size=(T, nh * hd)).astype(np.float32)
+    dbuf = torch_bf16(_bf(dy))
+    lst.k_rope(dbuf, nh * hd, T, S, 0, nh, hd, cos_t, sin_t, 1)
+    torch.cuda.synchronize()
+    ref_b = M.rope_bwd(_bf(dy).reshape(T, nh, hd).astype(np.float64), c, s, B, S).reshape(T, -1)
+    assert maxrel(to_np(dbuf), ref_b) < 8e-3
+
+
+def test_swiglu_fwd_bwd():
+    r = _rng(8)
+    T, F = 64, 688
+    gu = _bf(r.normal(size=(T, 2 * F)) * 2)
+    m = torch.empty(T, F, dtype=torch.bfloat16, device="cuda")
+    lst.k_swiglu_fwd(torch_bf16(gu), T, F, m)
+    g, u = gu[:, :F].astype(np.float64), gu[:, F:].astype(np.float64)
+    dm = r.normal(size=(T, F)).astype(np.float32)
+    dgu = torch.empty(T, 2 * F, dtype=torch.bfloat16, device="cuda")
+    lst.k_swiglu_bwd(torch_f32(dm), torch_bf16(gu), T, F, dgu)
+    torch.cuda.synchronize()
+    assert maxrel(to_np(m), M.silu(g) * u) < 8e-3
+    sg = 1 / (1 + np.exp(-g))
+    ref = np.concatenate([dm * u * sg * (1 + g * (1 - sg)), dm * g * sg], axis=1)
+    assert maxrel(to_np(dgu), ref) < 8e-3
+
+
+def test_cross_entropy_rows():
+    r = _rng(9)
+    T, V = 40, 50000
+    logits = r.normal(size=(T, V)).astype(np.float32) * 2
+    y = r.integers(0, V, size=T).astype(np.int32)
+    loss = torch.empty(T, device="cuda")
+    dl = torch.empty(T, V, dtype=torch.bfloat16, device="cuda")
+    lst.k_cross_entropy(torch_f32(logits), T, V, torch.from_numpy(y).cuda(), 1.0 / T, loss, dl)
+    torch.cuda.synchronize()
+    L = logits.astype(np.float64)
+    mx = L.max(1, keepdims=True)
+    lse = (mx + np.log(np.exp(L - mx).sum(1, keepdims=True)))[:, 0]
+    ref = lse - L[np.arange(T), y]
+    assert maxrel(to_np(loss), ref) < 1e-5
+    p = np.exp(L - lse[:, None])
+    p[np.arange(T), y] -= 1
+    assert maxrel(to_np(dl), p / T) < 8e-3
+
+
+def test_lora_project():
+    r = _rng(10)
+    T, din, R = 300, 688, 24
+    X = _bf(r.normal(size=(T, din)))
+    A = r.uniform(-0.05, 0.05, size=(R, din)).astype(np.float32)
+    U = torch.empty(T, R, device="cuda")
+    Us = torch.zeros(T, 64, dtype=torch.bfloat16, device="cuda")
+    lst.k_lora_project(torch_bf16(X), din, T, din, torch_f32(A), R, 2.0, U, Us, 64)
+    torch.cuda.synchronize()
+    ref = X.astype(np.float64) @ A.T.astype(np.float64)
+    assert maxrel(to_np(U), ref) < 1e-5
+    assert maxrel(to_np(Us)[:, :R], 2 * ref) < 8e-3
+    assert np.all(to_np(Us)[:, R:] == 0)

@@ -1,0 +1,135 @@
+"""Step-level parity (GPU): loss, logits and every LoRA gradient of the library against the oracle,
+streamed == resident byte for byte, and determinism. All calls go through the C ABI (lst.h)."""
+import numpy as np
+import pytest
+
+import synthetic as syn
+from helpers import (GRAD_COS, GRAD_MAXREL, LOGITS_MAXREL, LOSS_RTOL, build_inputs, compare_grads,
+                     make_context, maxrel, oracle_step, run_step)
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def _check_against_oracle(wl, inp, loss, grads, logits, ctx):
+    ref = oracle_step(wl, inp, schedule="streamed")
+    assert abs(loss - ref["loss"]) <= LOSS_RTOL * abs(ref["loss"]), (loss, ref["loss"])
+    if logits is not None:
+        assert maxrel(logits, ref["logits"]) <= LOGITS_MAXREL, maxrel(logits, ref["logits"])
+    worst_cos, worst_rel = 1.0, 0.0
+    for l, p, w, cs, mr in compare_grads(ctx, grads, ref["grads"]):
+        worst_cos, worst_rel = min(worst_cos, cs), max(worst_rel, mr)
+        assert cs >= GRAD_COS and mr <= GRAD_MAXREL, (l, p, w, cs, mr)
+    return worst_cos, worst_rel
+
+
+WORKLOADS = {
+    "tiny": syn.WORKLOADS["tiny"],
+    # GQA, q/k/v bias, bf16 base, ragged sequence (S=100 is not a multiple of the 64-row tiles)
+    "tiny_gqa_bias_bf16": syn.WORKLOADS["tiny"].with_(n_kv_heads=2, qkv_bias=True, base_format="bf16",
+                                                      batch=3, seq=100),
+    # one Llama-3.1-8B-shaped layer (headless), shorter sequence
+    "llama8b_layer_T256": syn.WORKLOADS["llama8b_layer"].with_(batch=1, seq=256),
+    # two Qwen2.5-3B-shaped layers with the bf16 base and the full head
+    "qwen3b_bf16_2L": syn.WORKLOADS["qwen3b_bf16"].with_(n_layers=2, batch=2, seq=128),
+}
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_step_matches_oracle_and_streamed_equals_resident(name):
+    wl = WORKLOADS[name]
+    inp = build_inputs(wl)
+    ctx_s = make_context(wl, inp, streamed=True)
+    loss_s, g_s, lg_s = run_step(ctx_s, wl, inp)
+    st = ctx_s.stats()
+    assert st["layer_reads_last_step"] == 2 * wl.n_layers
+    ctx_s.close()
+    ctx_r = make_context(wl, inp, streamed=False)
+    loss_r, g_r, lg_r = run_step(ctx_r, wl, inp)
+    ctx_r.close()
+    # streamed and resident runs are the same bytes
+    assert np.float32(loss_s).tobytes() == np.float32(loss_r).tobytes()
+    assert g_s.tobytes() == g_r.tobytes()
+    if lg_s is not None:
+        assert lg_s.tobytes() == lg_r.tobytes()
+    _check_against_oracle(wl, inp, loss_s, g_s, lg_s, ctx_s)
+
+
+def test_deterministic_and_adapters_matter():
+    wl = syn.WORKLOADS["tiny"]
+    inp = build_inputs(wl)
+    ctx = make_context(wl, inp, streamed=True)
+    a = run_step(ctx, wl, inp)
+    b = run_step(ctx, wl, inp)
+    assert a[0] == b[0] and a[1].tobytes() == b[1].tobytes()
+    # B = 0 on every projection gives a different loss (adapters are live), and then dA == 0
+    for l in range(wl.n_layers):
+        for j, p in enumerate(syn.PROJ):
+            ctx.set_lora(l, j, inp["raw"][l]["A"][p], np.zeros_like(inp["raw"][l]["B"][p]))
+    c = run_step(ctx, wl, inp)
+    assert c[0] != a[0]
+    from helpers import split_grads
+    for (l, p), (dA, dB) in split_grads(ctx, c[1]).items():
+        assert np.all(dA == 0)
+        assert np.any(dB != 0)
+    ctx.close()
+
+
+def test_errors_are_status_codes():
+    import layer_streamed_qlora_streaming_b200 as lst
+    wl = syn.WORKLOADS["tiny"]
+    inp = build_inputs(wl)
+    cfg = lst.make_config(wl, streamed=True)
+    E, gf, H = inp["head"]
+    ctx = lst.Context(cfg, E, gf, H)
+    with pytest.raises(lst.LstError) as e:          # no layer registered yet
+        ctx.step(inp["tokens"], inp["targets"], wl.batch, wl.seq)
+    assert e.value.status == 2
+    for i, r in enumerate(inp["raw"]):
+        ctx.register_layer(i, r["W"], r["A"], r["B"], r["attn_norm"], r["mlp_norm"], r["bias"])
+    with pytest.raises(lst.LstError) as e:          # sequence beyond max_seq
+        ctx.step(inp["tokens"], inp["targets"], wl.batch, wl.seq * 2)
+    assert e.value.status == 1
+    bad = inp["tokens"].copy()
+    bad[3] = wl.vocab + 5                            # token id out of range: device-side check
+    with pytest.raises(lst.LstError) as e:
+        ctx.step(bad, inp["targets"], wl.batch, wl.seq)
+    assert e.value.status == 6
+    loss = ctx.step(inp["tokens"], inp["targets"], wl.batch, wl.seq)   # context still usable
+    assert np.isfinite(loss)
+    ctx.close()
+
+
+@pytest.mark.slow
+def test_layer_above_165mb_nf4():
+    # two Qwen2.5-32B-shaped layers: 251.6 MB of NF4 per layer, above the size at which the
+    # pages report silently wrong gradients; checked directly against the oracle
+    wl = syn.WORKLOADS["qwen32b"].with_(n_layers=2, batch=1, seq=256)
+    inp = build_inputs(wl)
+    ctx = make_context(wl, inp, streamed=True)
+    assert ctx.stats()["blob_bytes"] > 165e6
+    loss, g, lg = run_step(ctx, wl, inp)
+    _check_against_oracle(wl, inp, loss, g, lg, ctx)
+    ctx.close()
+
+
+@pytest.mark.slow
+def test_full_size_llama8b_layer_against_oracle():
+    # the single-layer workload at its full size (batch 4 x seq 512), streamed and resident
+    wl = syn.WORKLOADS["llama8b_layer"]
+    inp = build_inputs(wl)
+    ctx = make_context(wl, inp, streamed=True)
+    loss, g, _ = run_step(ctx, wl, inp)
+    ctx.close()
+    ctx_r = make_context(wl, inp, streamed=False)
+    loss_r, g_r, _ = run_step(ctx_r, wl, inp)
+    ctx_r.close()
+    assert np.float32(loss).tobytes() == np.float32(loss_r).tobytes() and g.tobytes() == g_r.tobytes()
+    _check_against_oracle(wl, inp, loss, g, None, ctx)
