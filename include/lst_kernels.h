@@ -31,13 +31,13 @@ lst_status lst_k_nf4_dequant(const uint8_t* packed, const int8_t* qabs, const fl
 /* C = alpha * (A B' + A2 B2') + bias + R on the tcgen05 tensor cores (fp32 accumulate).
  * A [M, K] row stride lda; B' = B^T with B [N, K] (b_mn = 0) or B' = B with B [K, N] (b_mn = 1),
  * row stride ldb; (A2 [M, K2], B2) optional second pair of the same major-ness (NULL to skip);
- * C [M, N] fp32 (c_f32 = 1) or bf16; bias [N] fp32 or NULL; R [M, N] bf16 or NULL.
+ * C [M, N] fp32 (c_f32 = 1) or bf16; bias [N] fp32 or NULL; R [M, N] fp32 (residual) or NULL.
  * Leading dimensions must be multiples of 8 and A/B/A2/B2 16-byte aligned. */
 lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda,
                       const uint16_t* B, int64_t ldb, int32_t b_mn, const uint16_t* A2,
                       int64_t lda2, const uint16_t* B2, int64_t ldb2, int32_t K2, void* C,
                       int64_t ldc, int32_t c_f32, float alpha, const float* bias,
-                      const uint16_t* R, int64_t ldr, void* stream);
+                      const float* R, int64_t ldr, void* stream);
 
 /* Causal GQA attention forward over T = batch*S tokens: q [T, ldq], k [T, ldk], v [T, ldv]
  * (head h at column h*hd), o [T, ldo] bf16, lse [T, hq] fp32. hd in {64, 128}. */
@@ -55,11 +55,11 @@ lst_status lst_k_attention_bwd(const uint16_t* q, int64_t ldq, const uint16_t* k
                                uint16_t* dv, int64_t lddv, int64_t T, int32_t S, int32_t hq,
                                int32_t hkv, int32_t hd, void* stream);
 
-/* RMSNorm forward: y = bf16(x * rstd * g), rstd [T]. */
-lst_status lst_k_rmsnorm_fwd(const uint16_t* x, const float* g, int64_t T, int32_t d, float eps,
+/* RMSNorm forward of the fp32 residual stream x [T, d]: y = bf16(x * rstd * g), rstd [T]. */
+lst_status lst_k_rmsnorm_fwd(const float* x, const float* g, int64_t T, int32_t d, float eps,
                              uint16_t* y, float* rstd, void* stream);
 /* RMSNorm backward: dx = dres + rstd (dy g - xhat mean(dy g xhat)); dres and dx_bf16 may be NULL. */
-lst_status lst_k_rmsnorm_bwd(const float* dy, const uint16_t* x, const float* g,
+lst_status lst_k_rmsnorm_bwd(const float* dy, const float* x, const float* g,
                              const float* rstd, const float* dres, int64_t T, int32_t d,
                              float* dx, uint16_t* dx_bf16, void* stream);
 

@@ -195,9 +195,10 @@ struct lst_ctx {
   std::vector<Derived> der;  // L * NGROUP
   float* grads = nullptr;
 
-  __nv_bfloat16* xs = nullptr;
-  __nv_bfloat16 *n1 = nullptr, *qkv = nullptr, *o = nullptr, *h = nullptr, *n2 = nullptr, *gu = nullptr,
-                *m = nullptr, *wscr = nullptr;
+  float* xs = nullptr;  // residual stream: the input of every layer and the final output, fp32
+  float* h = nullptr;   // residual after attention, fp32
+  __nv_bfloat16 *n1 = nullptr, *qkv = nullptr, *o = nullptr, *n2 = nullptr, *gu = nullptr, *m = nullptr,
+                *wscr = nullptr;
   float *rstd1 = nullptr, *rstd2 = nullptr, *lse = nullptr, *Dbuf = nullptr;
   float* U[NGROUP] = {};
   __nv_bfloat16* Us[NGROUP] = {};
@@ -341,7 +342,7 @@ lst_status prep_lora(lst_ctx* c, int layer) {
 const __nv_bfloat16* group_w(lst_ctx* c, const __nv_bfloat16* W, int g) { return W + c->grp[g].woff; }
 
 lst_status group_fwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const __nv_bfloat16* X, int64_t ldx,
-                     __nv_bfloat16* Y, int64_t ldy, const float* bias, const __nv_bfloat16* resid, bool gemm) {
+                     void* Y, int64_t ldy, int y_f32, const float* bias, const float* resid, bool gemm) {
   const Group& G = c->grp[g];
   const auto& D = c->der[layer * NGROUP + g];
   const int64_t T = c->curT;
@@ -366,7 +367,7 @@ lst_status group_fwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
   a.K2 = G.KP;
   a.C = Y;
   a.ldc = ldy;
-  a.c_f32 = 0;
+  a.c_f32 = y_f32;
   a.bias = bias;
   a.R = resid;
   a.ldr = c->d;
@@ -464,12 +465,12 @@ lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
   const float* g1 = reinterpret_cast<const float*>(blob + c->lay.norms);
   const float* g2 = g1 + c->d;
   const float* bias = c->cfg.qkv_bias ? reinterpret_cast<const float*>(blob + c->lay.bias) : nullptr;
-  const __nv_bfloat16* x = c->xs + (int64_t)i * c->Tmax * c->d;
+  const float* x = c->xs + (int64_t)i * c->Tmax * c->d;
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(rmsnorm_fwd(x, g1, T, c->d, c->cfg.rms_eps, c->n1, c->rstd1, c->stream));
   }
-  TRY(group_fwd(c, i, G_QKV, W, c->n1, c->d, c->qkv, c->dqkv, bias, nullptr, true));
+  TRY(group_fwd(c, i, G_QKV, W, c->n1, c->d, c->qkv, c->dqkv, 0, bias, nullptr, true));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(rope(c->qkv, c->dqkv, T, S, 0, c->hq, c->hd, c->cos_t, c->sin_t, 0, c->stream));
@@ -493,18 +494,18 @@ lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
     ProfScope ps(c, c->stream, PC_ATTN);
     CK(attention_fwd(a, c->stream));
   }
-  TRY(group_fwd(c, i, G_O, W, c->o, c->dq, c->h, c->d, nullptr, x, true));
+  TRY(group_fwd(c, i, G_O, W, c->o, c->dq, c->h, c->d, 1, nullptr, x, true));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(rmsnorm_fwd(c->h, g2, T, c->d, c->cfg.rms_eps, c->n2, c->rstd2, c->stream));
   }
-  TRY(group_fwd(c, i, G_GU, W, c->n2, c->d, c->gu, 2 * c->F, nullptr, nullptr, true));
+  TRY(group_fwd(c, i, G_GU, W, c->n2, c->d, c->gu, 2 * c->F, 0, nullptr, nullptr, true));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(swiglu_fwd(c->gu, T, c->F, c->m, c->stream));
   }
   // the recompute pass needs only the LoRA projection of m (for dB of down), not the output
-  TRY(group_fwd(c, i, G_DOWN, W, c->m, c->F, c->xs + (int64_t)(i + 1) * c->Tmax * c->d, c->d, nullptr, c->h,
+  TRY(group_fwd(c, i, G_DOWN, W, c->m, c->F, c->xs + (int64_t)(i + 1) * c->Tmax * c->d, c->d, 1, nullptr, c->h,
                 !recompute));
   return LST_OK;
 }
@@ -515,7 +516,7 @@ lst_status layer_bwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
   const int S = (int)c->curS;
   const float* g1 = reinterpret_cast<const float*>(blob + c->lay.norms);
   const float* g2 = g1 + c->d;
-  const __nv_bfloat16* x = c->xs + (int64_t)i * c->Tmax * c->d;
+  const float* x = c->xs + (int64_t)i * c->Tmax * c->d;
   TRY(group_bwd(c, i, G_DOWN, W, c->dout_b, c->d, c->m, c->F, c->dm, 1));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
@@ -567,7 +568,7 @@ lst_status layer_bwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
 
 lst_status head_fwd_bwd(lst_ctx* c) {
   const int64_t T = c->curT;
-  const __nv_bfloat16* xL = c->xs + (int64_t)c->L * c->Tmax * c->d;
+  const float* xL = c->xs + (int64_t)c->L * c->Tmax * c->d;
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(rmsnorm_fwd(xL, c->gf, T, c->d, c->cfg.rms_eps, c->nf, c->rstdf, c->stream));
@@ -629,11 +630,6 @@ lst_status enqueue_copy(lst_ctx* c, int n) {
   return LST_OK;
 }
 
-__global__ void k_bf16_to_f32(const __nv_bfloat16* x, int64_t n, float* y) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = __bfloat162float(x[i]);
-}
-
 lst_status run_layers(lst_ctx* c, bool head) {
   const int L = c->L;
   const bool streamed = c->cfg.streamed != 0;
@@ -659,13 +655,11 @@ lst_status run_layers(lst_ctx* c, bool head) {
         TRY(head_fwd_bwd(c));
       } else {
         const int64_t T = c->curT;
-        const __nv_bfloat16* xL = c->xs + (int64_t)L * c->Tmax * c->d;
+        const float* xL = c->xs + (int64_t)L * c->Tmax * c->d;
         ProfScope ps(c, c->stream, PC_OTHER);
         CK(dot_fixed(xL, c->gbuf, T * c->d, c->dot_part, c->loss_dev, c->stream));
         CK(cudaMemcpyAsync(c->dout_b, c->gbuf, T * c->d * 2, cudaMemcpyDeviceToDevice, c->stream));
-        k_bf16_to_f32<<<(unsigned)((T * c->d + 255) / 256), 256, 0, c->stream>>>(c->gbuf, T * c->d, c->ga);
-        note_launch(1);
-        CK(cudaGetLastError());
+        CK(bf16_to_f32(c->gbuf, T * c->d, c->ga, c->stream));
       }
     }
     if (streamed && n + 2 < 2 * L) TRY(enqueue_copy(c, n + 2));
@@ -1119,7 +1113,8 @@ lst_status lst_step_hidden(lst_ctx* c, const uint16_t* x, const uint16_t* g, int
   if (!x || !g || !loss) return fail(c, LST_ERR_ARG, "null x/g/loss");
   if (c->V != 0) return fail(c, LST_ERR_STATE, "lst_step_hidden needs a headless config (vocab == 0)");
   TRY(begin_step(c, batch, seq));
-  TRY(copy_in(c, c->xs, x, c->curT * c->d * 2));
+  TRY(copy_in(c, c->dout_b, x, c->curT * c->d * 2));  // bf16 input staged, widened to fp32
+  CK(bf16_to_f32(c->dout_b, c->curT * c->d, c->xs, c->stream));
   TRY(copy_in(c, c->gbuf, g, c->curT * c->d * 2));
   TRY(run_layers(c, false));
   c->have_logits = false;

@@ -24,7 +24,7 @@ struct Epi {
   void* C;
   int64_t ldc;
   const float* bias;
-  const __nv_bfloat16* R;
+  const float* R;
   int64_t ldr;
   float alpha;
   int c_f32;
@@ -52,18 +52,19 @@ __device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const
       if (full || col0 + i < e.N) v[i] += e.bias[col0 + i];
   }
   if (e.R) {
-    const __nv_bfloat16* rp = e.R + (int64_t)row * e.ldr + col0;
+    const float* rp = e.R + (int64_t)row * e.ldr + col0;
     if (full && ((reinterpret_cast<uintptr_t>(rp) & 15) == 0)) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 u = *reinterpret_cast<const uint4*>(rp + q * 8);
-        const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&u);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[q * 8 + i] += __bfloat162float(b[i]);
+      for (int q = 0; q < 8; ++q) {
+        const float4 u = *reinterpret_cast<const float4*>(rp + q * 4);
+        v[q * 4] += u.x;
+        v[q * 4 + 1] += u.y;
+        v[q * 4 + 2] += u.z;
+        v[q * 4 + 3] += u.w;
       }
     } else {
       for (int i = 0; i < 32; ++i)
-        if (col0 + i < e.N) v[i] += __bfloat162float(rp[i]);
+        if (col0 + i < e.N) v[i] += rp[i];
     }
   }
   if (e.c_f32) {

@@ -31,7 +31,7 @@ struct GemmArgs {
   int c_f32 = 0;
   float alpha = 1.0f;
   const float* bias = nullptr;        // [N] or null
-  const __nv_bfloat16* R = nullptr;   // residual [M, N] row stride ldr, or null
+  const float* R = nullptr;           // fp32 residual [M, N] row stride ldr, or null
   int64_t ldr = 0;
 };
 

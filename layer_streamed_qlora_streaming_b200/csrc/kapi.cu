@@ -55,7 +55,7 @@ lst_status lst_k_nf4_dequant(const uint8_t* packed, const int8_t* qabs, const fl
 
 lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb,
                       int32_t b_mn, const uint16_t* A2, int64_t lda2, const uint16_t* B2, int64_t ldb2, int32_t K2,
-                      void* C, int64_t ldc, int32_t c_f32, float alpha, const float* bias, const uint16_t* R,
+                      void* C, int64_t ldc, int32_t c_f32, float alpha, const float* bias, const float* R,
                       int64_t ldr, void* stream) {
   if (M <= 0 || N <= 0 || K <= 0 || !A || !B || !C) return LST_ERR_ARG;
   if ((A2 == nullptr) != (B2 == nullptr)) return LST_ERR_ARG;
@@ -78,7 +78,7 @@ lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_
   a.c_f32 = c_f32 ? 1 : 0;
   a.alpha = alpha;
   a.bias = bias;
-  a.R = B16(R);
+  a.R = R;
   a.ldr = ldr;
   return st(gemm_bf16(a, S(stream)));
 }
@@ -126,16 +126,16 @@ lst_status lst_k_attention_bwd(const uint16_t* q, int64_t ldq, const uint16_t* k
   return st(attention_bwd(a, S(stream)));
 }
 
-lst_status lst_k_rmsnorm_fwd(const uint16_t* x, const float* g, int64_t T, int32_t d, float eps, uint16_t* y,
+lst_status lst_k_rmsnorm_fwd(const float* x, const float* g, int64_t T, int32_t d, float eps, uint16_t* y,
                              float* rstd, void* stream) {
   if (!x || !g || !y || !rstd || T <= 0 || d <= 0) return LST_ERR_ARG;
-  return st(rmsnorm_fwd(B16(x), g, T, d, eps, B16(y), rstd, S(stream)));
+  return st(rmsnorm_fwd(x, g, T, d, eps, B16(y), rstd, S(stream)));
 }
 
-lst_status lst_k_rmsnorm_bwd(const float* dy, const uint16_t* x, const float* g, const float* rstd, const float* dres,
+lst_status lst_k_rmsnorm_bwd(const float* dy, const float* x, const float* g, const float* rstd, const float* dres,
                              int64_t T, int32_t d, float* dx, uint16_t* dxb, void* stream) {
   if (!dy || !x || !g || !rstd || !dx || T <= 0 || d <= 0) return LST_ERR_ARG;
-  return st(rmsnorm_bwd(dy, B16(x), g, rstd, dres, T, d, dx, B16(dxb), S(stream)));
+  return st(rmsnorm_bwd(dy, x, g, rstd, dres, T, d, dx, B16(dxb), S(stream)));
 }
 
 lst_status lst_k_rope_tables(int32_t Sq, int32_t hd, double theta, float* ct, float* sn, void* stream) {

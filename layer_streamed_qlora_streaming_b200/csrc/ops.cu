@@ -37,50 +37,44 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 }
 
 // ------------------------------------------------------------------------------- RMSNorm
-__global__ void k_rmsnorm_fwd(const bf16* __restrict__ x, const float* __restrict__ g, int d, float eps,
+__global__ void k_rmsnorm_fwd(const float* __restrict__ x, const float* __restrict__ g, int d, float eps,
                               bf16* __restrict__ y, float* __restrict__ rstd) {
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
-  const bf16* xr = x + row * d;
+  const float* xr = x + row * d;
   float ss = 0.f;
-  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
-    uint4 u = *reinterpret_cast<const uint4*>(xr + c);
-    const bf16* h = reinterpret_cast<const bf16*>(&u);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float v = __bfloat162float(h[i]);
-      ss += v * v;
-    }
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    const float4 u = *reinterpret_cast<const float4*>(xr + c);
+    ss += u.x * u.x;
+    ss += u.y * u.y;
+    ss += u.z * u.z;
+    ss += u.w * u.w;
   }
   ss = block_sum(ss, red);
   const float r = 1.0f / sqrtf(ss / (float)d + eps);
   if (threadIdx.x == 0) rstd[row] = r;
-  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
-    uint4 u = *reinterpret_cast<const uint4*>(xr + c);
-    const bf16* h = reinterpret_cast<const bf16*>(&u);
-    uint4 o;
-    __nv_bfloat162* oh = reinterpret_cast<__nv_bfloat162*>(&o);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      oh[i] = __floats2bfloat162_rn(__bfloat162float(h[2 * i]) * r * g[c + 2 * i],
-                                    __bfloat162float(h[2 * i + 1]) * r * g[c + 2 * i + 1]);
-    *reinterpret_cast<uint4*>(y + row * d + c) = o;
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    const float4 u = *reinterpret_cast<const float4*>(xr + c);
+    __nv_bfloat162 o[2];
+    o[0] = __floats2bfloat162_rn(u.x * r * g[c], u.y * r * g[c + 1]);
+    o[1] = __floats2bfloat162_rn(u.z * r * g[c + 2], u.w * r * g[c + 3]);
+    *reinterpret_cast<uint2*>(y + row * d + c) = *reinterpret_cast<const uint2*>(o);
   }
 }
 
-__global__ void k_rmsnorm_bwd(const float* __restrict__ dy, const bf16* __restrict__ x, const float* __restrict__ g,
+__global__ void k_rmsnorm_bwd(const float* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ g,
                               const float* __restrict__ rstd, const float* __restrict__ dres, int d,
                               float* __restrict__ dx, bf16* __restrict__ dxb) {
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
   const float r = rstd[row];
   const float* dyr = dy + row * d;
-  const bf16* xr = x + row * d;
+  const float* xr = x + row * d;
   float dot = 0.f;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) dot += dyr[c] * g[c] * (__bfloat162float(xr[c]) * r);
+  for (int c = threadIdx.x; c < d; c += blockDim.x) dot += dyr[c] * g[c] * (xr[c] * r);
   dot = block_sum(dot, red) / (float)d;
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    const float xh = __bfloat162float(xr[c]) * r;
+    const float xh = xr[c] * r;
     float v = r * (dyr[c] * g[c] - xh * dot);
     if (dres) v += dres[row * d + c];
     dx[row * d + c] = v;
@@ -151,7 +145,7 @@ __global__ void k_swiglu_bwd(const float* __restrict__ dm, const bf16* __restric
 
 // ------------------------------------------------------------------------------- embedding
 __global__ void k_embed(const int32_t* __restrict__ tok, const bf16* __restrict__ E, int64_t T, int d, int V,
-                        bf16* __restrict__ x) {
+                        float* __restrict__ x) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // 8-element vector index
   const int nv = d / 8;
   if (i >= T * nv) return;
@@ -161,7 +155,10 @@ __global__ void k_embed(const int32_t* __restrict__ tok, const bf16* __restrict_
   uint4 v = make_uint4(0, 0, 0, 0);
   if (id >= 0 && id < V) v = *reinterpret_cast<const uint4*>(E + (int64_t)id * d + c);
   else if (c == 0) dev_fail(DEV_ERR_BAD_INDEX);
-  *reinterpret_cast<uint4*>(x + t * d + c) = v;
+  const bf16* h = reinterpret_cast<const bf16*>(&v);
+  float4* o = reinterpret_cast<float4*>(x + t * d + c);
+  o[0] = make_float4(__bfloat162float(h[0]), __bfloat162float(h[1]), __bfloat162float(h[2]), __bfloat162float(h[3]));
+  o[1] = make_float4(__bfloat162float(h[4]), __bfloat162float(h[5]), __bfloat162float(h[6]), __bfloat162float(h[7]));
 }
 
 // ------------------------------------------------------------------------------- cross-entropy
@@ -199,13 +196,13 @@ __global__ void k_mean(const float* __restrict__ v, int64_t n, float* __restrict
   if (threadIdx.x == 0) *out = s / (float)n;
 }
 
-__global__ void k_dot_partial(const bf16* __restrict__ a, const bf16* __restrict__ b, int64_t n,
+__global__ void k_dot_partial(const float* __restrict__ a, const bf16* __restrict__ b, int64_t n,
                               float* __restrict__ part) {
   __shared__ float red[32];
   const int64_t per = (n + gridDim.x - 1) / gridDim.x;
   const int64_t lo = blockIdx.x * per, hi = min(n, lo + per);
   float s = 0.f;
-  for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x) s += __bfloat162float(a[i]) * __bfloat162float(b[i]);
+  for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x) s += a[i] * __bfloat162float(b[i]);
   s = block_sum(s, red);
   if (threadIdx.x == 0) part[blockIdx.x] = s;
 }
@@ -220,6 +217,10 @@ __global__ void k_sum_in_order(const float* __restrict__ part, int n, float* __r
 __global__ void k_f32_to_bf16(const float* __restrict__ x, int64_t n, bf16* __restrict__ y) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) y[i] = __float2bfloat16_rn(x[i]);
+}
+__global__ void k_bf16_to_f32(const bf16* __restrict__ x, int64_t n, float* __restrict__ y) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = __bfloat162float(x[i]);
 }
 
 // ------------------------------------------------------------------------------- LoRA
@@ -353,14 +354,14 @@ inline unsigned nblk(int64_t n, int t = kThreads) { return (unsigned)((n + t - 1
 
 }  // namespace
 
-cudaError_t rmsnorm_fwd(const bf16* x, const float* g, int64_t T, int d, float eps, bf16* y, float* rstd,
+cudaError_t rmsnorm_fwd(const float* x, const float* g, int64_t T, int d, float eps, bf16* y, float* rstd,
                         cudaStream_t s) {
   if (d % 8) return cudaErrorInvalidValue;
   k_rmsnorm_fwd<<<(unsigned)T, d >= 2048 ? 256 : 128, 0, s>>>(x, g, d, eps, y, rstd);
   note_launch(1);
   return cudaGetLastError();
 }
-cudaError_t rmsnorm_bwd(const float* dy, const bf16* x, const float* g, const float* rstd, const float* dres,
+cudaError_t rmsnorm_bwd(const float* dy, const float* x, const float* g, const float* rstd, const float* dres,
                         int64_t T, int d, float* dx, bf16* dxb, cudaStream_t s) {
   k_rmsnorm_bwd<<<(unsigned)T, 256, 0, s>>>(dy, x, g, rstd, dres, d, dx, dxb);
   note_launch(1);
@@ -387,7 +388,7 @@ cudaError_t swiglu_bwd(const float* dm, const bf16* gu, int64_t T, int F, bf16* 
   note_launch(1);
   return cudaGetLastError();
 }
-cudaError_t embed(const int32_t* tok, const bf16* E, int64_t T, int d, int V, bf16* x, cudaStream_t s) {
+cudaError_t embed(const int32_t* tok, const bf16* E, int64_t T, int d, int V, float* x, cudaStream_t s) {
   if (d % 8) return cudaErrorInvalidValue;
   k_embed<<<nblk(T * (d / 8)), kThreads, 0, s>>>(tok, E, T, d, V, x);
   note_launch(1);
@@ -404,7 +405,7 @@ cudaError_t mean_fixed(const float* v, int64_t n, float* out, cudaStream_t s) {
   note_launch(1);
   return cudaGetLastError();
 }
-cudaError_t dot_fixed(const bf16* a, const bf16* b, int64_t n, float* part, float* out, cudaStream_t s) {
+cudaError_t dot_fixed(const float* a, const bf16* b, int64_t n, float* part, float* out, cudaStream_t s) {
   k_dot_partial<<<1024, 256, 0, s>>>(a, b, n, part);
   k_sum_in_order<<<1, 32, 0, s>>>(part, 1024, out);
   note_launch(2);
@@ -412,6 +413,11 @@ cudaError_t dot_fixed(const bf16* a, const bf16* b, int64_t n, float* part, floa
 }
 cudaError_t f32_to_bf16(const float* x, int64_t n, bf16* y, cudaStream_t s) {
   k_f32_to_bf16<<<nblk(n), kThreads, 0, s>>>(x, n, y);
+  note_launch(1);
+  return cudaGetLastError();
+}
+cudaError_t bf16_to_f32(const bf16* x, int64_t n, float* y, cudaStream_t s) {
+  k_bf16_to_f32<<<nblk(n), kThreads, 0, s>>>(x, n, y);
   note_launch(1);
   return cudaGetLastError();
 }

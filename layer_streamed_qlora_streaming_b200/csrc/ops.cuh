@@ -9,11 +9,12 @@ namespace lst {
 
 using bf16 = __nv_bfloat16;
 
-// y = bf16(x * rstd * g), rstd = 1/sqrt(mean(x^2) + eps) per row; rstd saved [T].
-cudaError_t rmsnorm_fwd(const bf16* x, const float* g, int64_t T, int d, float eps, bf16* y, float* rstd,
+// y = bf16(x * rstd * g), rstd = 1/sqrt(mean(x^2) + eps) per row (x fp32: the residual stream);
+// rstd saved [T].
+cudaError_t rmsnorm_fwd(const float* x, const float* g, int64_t T, int d, float eps, bf16* y, float* rstd,
                         cudaStream_t s);
 // dx = dres + rstd * (dy*g - xhat * mean(dy*g*xhat)); writes fp32 dx and (optional) bf16 copy.
-cudaError_t rmsnorm_bwd(const float* dy, const bf16* x, const float* g, const float* rstd, const float* dres,
+cudaError_t rmsnorm_bwd(const float* dy, const float* x, const float* g, const float* rstd, const float* dres,
                         int64_t T, int d, float* dx, bf16* dx_bf16, cudaStream_t s);
 
 // Rotate pairs (j, j + hd/2) of the first nh heads of each row of buf (row stride ld) by the
@@ -28,17 +29,19 @@ cudaError_t swiglu_fwd(const bf16* gu, int64_t T, int F, bf16* m, cudaStream_t s
 // dgu = [dm * u * silu'(g) | dm * silu(g)] (bf16), dm fp32 [T, F].
 cudaError_t swiglu_bwd(const float* dm, const bf16* gu, int64_t T, int F, bf16* dgu, cudaStream_t s);
 
-cudaError_t embed(const int32_t* tok, const bf16* E, int64_t T, int d, int vocab, bf16* x, cudaStream_t s);
+// x[t] = E[tok[t]] as fp32 (the residual stream); out-of-range ids set the device error word.
+cudaError_t embed(const int32_t* tok, const bf16* E, int64_t T, int d, int vocab, float* x, cudaStream_t s);
 
 // Cross-entropy rows: loss_t = lse_t - logit[t, y_t]; dlogits = (softmax - onehot) * inv_T (bf16).
 cudaError_t cross_entropy(const float* logits, int64_t T, int V, const int32_t* targets, float inv_T,
                           float* loss_rows, bf16* dlogits, cudaStream_t s);
 // out = mean of v[0..n) with a fixed summation order.
 cudaError_t mean_fixed(const float* v, int64_t n, float* out, cudaStream_t s);
-// out = sum_i a[i] * b[i] (bf16 inputs) with a fixed order; partials: scratch of 1024 floats.
-cudaError_t dot_fixed(const bf16* a, const bf16* b, int64_t n, float* partials, float* out, cudaStream_t s);
+// out = sum_i a[i] * b[i] with a fixed order; partials: scratch of 1024 floats.
+cudaError_t dot_fixed(const float* a, const bf16* b, int64_t n, float* partials, float* out, cudaStream_t s);
 
 cudaError_t f32_to_bf16(const float* x, int64_t n, bf16* y, cudaStream_t s);
+cudaError_t bf16_to_f32(const bf16* x, int64_t n, float* y, cudaStream_t s);
 
 // ------------------------------------------------------------------------ LoRA side path
 // U[t, j] = sum_i X[t, i] * A[j, i] for j < R (A fp32 [R, in] row stride lda); writes U fp32

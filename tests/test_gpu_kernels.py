@@ -92,9 +92,9 @@ def test_gemm(M, N, K, b_mn, ext, f32, bias, resid):
         ref = ref + bv
         kw["bias"] = torch_f32(bv)
     if resid:
-        Rv = _bf(r.normal(size=(M, N)))
+        Rv = r.normal(size=(M, N)).astype(np.float32)
         ref = ref + Rv
-        kw.update(R=torch_bf16(Rv), ldr=N)
+        kw.update(R=torch_f32(Rv), ldr=N)
     C = torch.zeros(M, N, dtype=torch.float32 if f32 else torch.bfloat16, device="cuda")
     lst.k_gemm(M, N, K, torch_bf16(A), K, torch_bf16(B), N if b_mn else K, b_mn, C, N, int(f32), **kw)
     torch.cuda.synchronize()
@@ -172,16 +172,16 @@ def test_attention_deterministic():
 def test_rmsnorm_fwd_bwd():
     r = _rng(6)
     T, d = 37, 4096
-    x = _bf(r.normal(size=(T, d)))
+    x = r.normal(size=(T, d)).astype(np.float32)
     g = r.uniform(0.5, 1.5, size=d).astype(np.float32)
     y_ref, rs = M.rmsnorm(x.astype(np.float64), g.astype(np.float64), 1e-5)
     y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
     rstd = torch.empty(T, dtype=torch.float32, device="cuda")
-    lst.k_rmsnorm_fwd(torch_bf16(x), torch_f32(g), T, d, 1e-5, y, rstd)
+    lst.k_rmsnorm_fwd(torch_f32(x), torch_f32(g), T, d, 1e-5, y, rstd)
     dy = r.normal(size=(T, d)).astype(np.float32)
     dres = r.normal(size=(T, d)).astype(np.float32)
     dx = torch.empty(T, d, dtype=torch.float32, device="cuda")
-    lst.k_rmsnorm_bwd(torch_f32(dy), torch_bf16(x), torch_f32(g), rstd, torch_f32(dres), T, d, dx)
+    lst.k_rmsnorm_bwd(torch_f32(dy), torch_f32(x), torch_f32(g), rstd, torch_f32(dres), T, d, dx)
     torch.cuda.synchronize()
     assert maxrel(to_np(y), y_ref) < 8e-3
     dx_ref = dres + M.rmsnorm_bwd(dy.astype(np.float64), x.astype(np.float64), g.astype(np.float64), rs)
