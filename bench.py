@@ -1,0 +1,416 @@
+"""Benchmark of the layer-streamed LoRA training step (forward + backward) on B200 GPUs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one call of the library's step through its C ABI: embedding, every decoder layer copied
+from the pinned host arena through the two-buffer device pool (2L layer reads), forward, LM head +
+cross-entropy, recompute + backward of every layer, LoRA gradients. Inputs are seeded synthetic
+weights / tokens of the workload's shape (no dataset, no trained weights).
+
+Prints ONE JSON line (rank 0). For N > 1 (torchrun, one process per GPU) every rank runs its own
+replica of the workload on its own GPU and PCIe link and the LoRA gradients are all-reduced over
+NCCL after each step (data parallel); the time is the max over ranks.
+
+--impl reference times the CPU oracle (tests' reference implementation) on this host's cores, on
+a bounded sample of the same workload, and reports the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "streamed LoRA fwd+bwd tokens/sec on 1 B200; % of PCIe/HBM/tensor roofline"
+UNIT = "tokens/s"
+
+
+# ---------------------------------------------------------------------------------------- setup
+def workload(name: str):
+    import synthetic as syn
+    return syn.WORKLOADS[name]
+
+
+def describe(wl) -> str:
+    base = "NF4 (double-quant) base" if wl.base_format == "nf4" else "bf16 base"
+    head = f", vocab {wl.vocab} head + CE" if wl.vocab else ", no head (loss = sum(x_L * G))"
+    return (f"{wl.name}: {wl.n_layers} x decoder layer d{wl.d_model} h{wl.n_heads}/{wl.n_kv_heads} "
+            f"hd{wl.head_dim} ffn{wl.ffn}, {base} streamed from pinned host, LoRA r{wl.lora_rank} "
+            f"a{int(wl.lora_alpha)} on 7 projections{head}, batch {wl.batch} x seq {wl.seq}")
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def h2d_peak_gbs(torch) -> float:
+    """Pinned host -> device copy bandwidth of this GPU's link (1 GiB, best of 5, CUDA events)."""
+    n = 1 << 30
+    h = torch.empty(n, dtype=torch.uint8).pin_memory()
+    d = torch.empty(n, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    best = 0.0
+    for i in range(7):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            d.copy_(h, non_blocking=True)
+            e1.record(s)
+        s.synchronize()
+        if i >= 2:
+            best = max(best, n / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    del h, d
+    return best
+
+
+def build_context(wl, torch, stream, seed: int = 1234):
+    """Library context with every layer registered from device-resident synthetic weights."""
+    import layer_streamed_qlora_streaming_b200 as lst
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    dev = "cuda"
+
+    def normal(shape, std):
+        return torch.randn(shape, generator=g, device=dev, dtype=torch.float32) * std
+
+    def uniform(shape, b):
+        return (torch.rand(shape, generator=g, device=dev, dtype=torch.float32) * 2 - 1) * b
+
+    cfg = lst.make_config(wl, streamed=True)
+    if wl.vocab:
+        E = normal((wl.vocab, wl.d_model), 0.02)
+        H = normal((wl.vocab, wl.d_model), 0.02)
+        gf = torch.ones(wl.d_model, device=dev)
+        ctx = lst.Context(cfg, E, gf, H, stream=stream)
+        del E, H
+    else:
+        ctx = lst.Context(cfg, stream=stream)
+    ones = torch.ones(wl.d_model, device=dev)
+    for i in range(wl.n_layers):
+        W, A, B = {}, {}, {}
+        for p in lst.PROJ:
+            out, inp = wl.proj_shape(p)
+            W[p] = normal((out, inp), 0.02)
+            A[p] = uniform((wl.lora_rank, inp), 1.0 / math.sqrt(inp))
+            B[p] = normal((out, wl.lora_rank), 0.01)
+        bias = None
+        if wl.qkv_bias:
+            bias = {p: normal((wl.proj_shape(p)[0],), 0.02) for p in ("q", "k", "v")}
+        ctx.register_layer(i, W, A, B, ones, ones, bias)
+        del W, A, B, bias
+    torch.cuda.synchronize()
+    return ctx
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.p = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.out, _ = self.p.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+                self.out, _ = self.p.communicate()
+
+    def summary(self) -> dict:
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------------- CPU oracle
+def oracle_sample(wl, seq: int = 512):
+    """Time the CPU oracle on a bounded sample of the workload: one decoder layer (forward,
+    recompute, backward; streamed schedule) and the head at batch 1 x seq tokens. Returns
+    (tokens/s extrapolated to the whole workload, seconds of CPU work, description)."""
+    import numpy as np
+    from oracle import model as M
+
+    rng = np.random.default_rng(7)
+    T = seq
+    lw = wl.with_(n_layers=1, vocab=0, batch=1, seq=seq)
+    raw = [{"W": {p: (rng.standard_normal(lw.proj_shape(p), dtype=np.float32) * 0.02) for p in M.PROJ},
+            "A": {p: rng.uniform(-1, 1, (lw.lora_rank, lw.proj_shape(p)[1])).astype(np.float32) /
+                  math.sqrt(lw.proj_shape(p)[1]) for p in M.PROJ},
+            "B": {p: (rng.standard_normal((lw.proj_shape(p)[0], lw.lora_rank), dtype=np.float32) * 0.01)
+                  for p in M.PROJ},
+            "attn_norm": np.ones(lw.d_model, np.float32), "mlp_norm": np.ones(lw.d_model, np.float32),
+            "bias": ({p: rng.standard_normal(lw.proj_shape(p)[0], dtype=np.float32) * 0.02
+                      for p in ("q", "k", "v")} if lw.qkv_bias else None)}]
+    x = rng.standard_normal((T, lw.d_model), dtype=np.float32)
+    G = rng.standard_normal((T, lw.d_model), dtype=np.float32)
+    t0 = time.perf_counter()
+    M.step(lw, raw_layers=raw, x_in=x, G=G, schedule="streamed")
+    t_layer = time.perf_counter() - t0
+    t_head = 0.0
+    if wl.vocab:
+        H = rng.standard_normal((wl.vocab, wl.d_model), dtype=np.float32) * 0.02
+        y = rng.integers(0, wl.vocab, T)
+        t0 = time.perf_counter()
+        loss, logits, hc = M.head_fwd(x.astype(np.float64), np.ones(wl.d_model), H.astype(np.float64), y,
+                                      wl.rms_eps)
+        M.head_bwd(hc, logits, np.ones(wl.d_model), H.astype(np.float64), y)
+        t_head = time.perf_counter() - t0
+    step_s = wl.n_layers * t_layer + t_head
+    desc = (f"oracle (numpy fp64) on batch 1 x seq {seq}: one decoder layer fwd+recompute+bwd "
+            f"({t_layer:.2f} s) x {wl.n_layers} layers" + (f" + head and CE ({t_head:.2f} s)" if wl.vocab else "")
+            + "; tokens/s = tokens / extrapolated step time")
+    return T / step_s, t_layer + t_head, desc
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((i.get("num_threads", 0) for i in info), default=0)
+        if n:
+            return int(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------------------- ranks
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's time (every rank calls this at the same point)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def allreduce_grads(grads, dist) -> None:
+    """Data-parallel exchange: sum the LoRA gradients of all replicas (NCCL on GPUs)."""
+    if dist is not None:
+        dist.all_reduce(grads)
+
+
+def job_throughput(world: int, tokens_per_step: int, steps: int, ms: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batch each step."""
+    return world * tokens_per_step * steps / (ms * 1e-3)
+
+
+# ---------------------------------------------------------------------------------------- arms
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(wl, seq=args.ref_seq)
+    vals, secs, desc = [], 0.0, ""
+    for _ in range(args.steps):
+        v, s, desc = oracle_sample(wl, seq=args.ref_seq)
+        vals.append(v)
+        secs += s
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.tokens / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": describe(wl), "batch": wl.batch, "seq": wl.seq},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_gpu(args, wl):
+    import torch
+    import layer_streamed_qlora_streaming_b200 as lst
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    stream = torch.cuda.Stream()
+    link_gbs = h2d_peak_gbs(torch)
+    ctx = build_context(wl, torch, stream, seed=1234 + rank)
+    n_grad = ctx.lora_numel()
+    grads = torch.zeros(n_grad, dtype=torch.float32, device="cuda")
+    g = torch.Generator(device="cpu")
+    g.manual_seed(99 + rank)
+    T = wl.tokens
+    if wl.vocab:
+        toks = torch.randint(0, wl.vocab, (T,), generator=g, dtype=torch.int32)
+        tgts = torch.randint(0, wl.vocab, (T,), generator=g, dtype=torch.int32)
+        toks_d, tgts_d = toks.cuda(), tgts.cuda()
+
+        def step(gr):
+            return ctx.step(toks_d, tgts_d, wl.batch, wl.seq, gr)
+    else:
+        xg = (torch.randn(T, wl.d_model, generator=g)).to(torch.bfloat16)
+        gg = (torch.randn(T, wl.d_model, generator=g)).to(torch.bfloat16)
+        x_d, g_d = xg.cuda().view(torch.int16), gg.cuda().view(torch.int16)
+
+        def step(gr):
+            return ctx.step_hidden(x_d, g_d, wl.batch, wl.seq, gr)
+
+    def one_step():
+        loss = step(grads)
+        with torch.cuda.stream(stream):
+            allreduce_grads(grads, dist)
+        return loss
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    ctx.set_profiling(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    agg = {k: 0.0 for k in ("gemm_ms", "attention_ms", "dequant_ms", "other_ms", "copy_ms", "gemm_flops",
+                            "gemm_launches", "launches_last_step", "h2d_bytes_last_step")}
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            loss = one_step()
+            st = ctx.stats()
+            for k in agg:
+                agg[k] += st[k]
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ctx.set_profiling(False)
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
+    value = job_throughput(world, T, args.steps, ms)
+
+    # end to end: host tokens in (pinned), host loss and gradients out, inside the timed region
+    hg = torch.zeros(n_grad, dtype=torch.float32).pin_memory()
+    if wl.vocab:
+        ht, hy = toks.pin_memory(), tgts.pin_memory()
+        host_step = lambda: ctx.step(ht, hy, wl.batch, wl.seq, hg)
+        h2d = 2 * T * 4
+    else:
+        hx, hgg = xg.view(torch.int16).pin_memory(), gg.view(torch.int16).pin_memory()
+        host_step = lambda: ctx.step_hidden(hx, hgg, wl.batch, wl.seq, hg)
+        h2d = 2 * T * wl.d_model * 2
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    f0.record(stream)
+    for _ in range(args.steps):
+        host_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    ems = max_over_ranks(f0.elapsed_time(f1), dist, "cuda")
+    e2e = {"value": job_throughput(world, T, args.steps, ems), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": n_grad * 4 + 4,
+           "path": "lst_step with pinned host inputs and host gradient buffer (copies inside the call)"}
+
+    st = ctx.stats()
+    peaks = measured_peaks()
+    K = args.steps
+    gemm_ms = agg["gemm_ms"] / K
+    gemm_tflops = agg["gemm_flops"] / K / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else 0.0
+    peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    step_ms = ms / K
+    h2d_bytes = agg["h2d_bytes_last_step"] / K
+    pcie_ms = h2d_bytes / (link_gbs * 1e9) * 1e3
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded torch.randn weights / uniform tokens)",
+        "config": {"workload": describe(wl), "batch": wl.batch, "seq": wl.seq, "layers": wl.n_layers,
+                   "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                   "l2": "not flushed: every step streams all layer blobs (GBs) through HBM, far above the 126 MB L2",
+                   "loss_last": loss},
+        "roofline": {"bound": "tensor", "kernel": "tcgen05 bf16 GEMM (all projection + LM-head GEMMs)",
+                     "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / peak_t if peak_t else None, "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
+                     "gemm_ms_per_step": gemm_ms, "gemm_launches_per_step": agg["gemm_launches"] / K},
+        "step_roofline": {"bound": "pcie", "h2d_bytes_per_step": h2d_bytes, "link_gbs": link_gbs,
+                          "link_source": "measured in this run: pinned 1 GiB host->device copy",
+                          "min_ms": pcie_ms, "frac": pcie_ms / step_ms,
+                          "achieved_h2d_gbs": h2d_bytes / (step_ms * 1e-3) / 1e9,
+                          "copy_ms_per_step": agg["copy_ms"] / K,
+                          "attention_ms_per_step": agg["attention_ms"] / K,
+                          "dequant_ms_per_step": agg["dequant_ms"] / K},
+        "gpu_launches": int(agg["launches_last_step"]),
+        "clocks": clk.summary(),
+    }
+    line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, secs, desc = oracle_sample(wl, seq=args.ref_seq)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                                "sample": desc, "cpu_seconds": secs}
+    ctx.close()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-seq", type=int, default=512)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_gpu(args, wl)
+
+
+if __name__ == "__main__":
+    main()

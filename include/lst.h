@@ -142,6 +142,18 @@ lst_status lst_step_hidden(lst_ctx* ctx, const uint16_t* x, const uint16_t* g, i
 /* Copy the last step's logits [batch * seq, V] fp32 to dst (host or device). */
 lst_status lst_get_logits(lst_ctx* ctx, float* dst);
 
+/* Inspect activations of the last step (for checking a step stage by stage). `which`:
+ *  LST_ACT_X  : the fp32 residual-stream input of decoder layer `layer` [T, d] (layer == L gives
+ *               the output of the last layer);
+ *  LST_ACT_N1, _QKV, _O, _N2, _GU, _M : bf16 intermediates [T, d], [T, dq+2dkv] (q and k after
+ *               RoPE), [T, dq], [T, d], [T, 2F], [T, F]; LST_ACT_H : fp32 [T, d];
+ *               these hold the most recently computed layer, which after a step is layer 0
+ *               (`layer` must be 0).
+ * dst: host or device memory of the stated size. */
+enum { LST_ACT_X = 0, LST_ACT_N1 = 1, LST_ACT_QKV = 2, LST_ACT_O = 3, LST_ACT_H = 4, LST_ACT_N2 = 5,
+       LST_ACT_GU = 6, LST_ACT_M = 7 };
+lst_status lst_get_activation(lst_ctx* ctx, int32_t which, int32_t layer, void* dst);
+
 /* Record per-class device times of every step (CUDA events around each launch) when on != 0. */
 lst_status lst_set_profiling(lst_ctx* ctx, int32_t on);
 lst_status lst_get_stats(const lst_ctx* ctx, lst_stats* out);

@@ -61,6 +61,7 @@ _SIGS = {
     "lst_step": (_I32, [_P, _P, _P, _I32, _I32, C.POINTER(C.c_float), _P]),
     "lst_step_hidden": (_I32, [_P, _P, _P, _I32, _I32, C.POINTER(C.c_float), _P]),
     "lst_get_logits": (_I32, [_P, _P]),
+    "lst_get_activation": (_I32, [_P, _I32, _I32, _P]),
     "lst_set_profiling": (_I32, [_P, _I32]),
     "lst_get_stats": (_I32, [_P, C.POINTER(Stats)]),
     "lst_last_error": (C.c_char_p, [_P]),
@@ -211,6 +212,12 @@ class Context:
 
     def logits(self, dst) -> None:
         _check(lib().lst_get_logits(self.h, _ptr(dst)), self.h, "lst_get_logits")
+
+    ACT = {"x": 0, "n1": 1, "qkv": 2, "o": 3, "h": 4, "n2": 5, "gu": 6, "m": 7}
+
+    def activation(self, which: str, layer: int, dst) -> None:
+        _check(lib().lst_get_activation(self.h, self.ACT[which], layer, _ptr(dst)), self.h,
+               "lst_get_activation")
 
     def set_profiling(self, on: bool) -> None:
         _check(lib().lst_set_profiling(self.h, int(on)), self.h, "lst_set_profiling")

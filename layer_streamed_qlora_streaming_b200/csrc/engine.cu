@@ -299,14 +299,15 @@ struct ProfScope {
   int cls;
   double flops;
   cudaEvent_t a = nullptr;
+  // the many small kernels of class "other" are not bracketed, to keep the event count low
   ProfScope(lst_ctx* c_, cudaStream_t s_, int cls_, double flops_ = 0) : c(c_), s(s_), cls(cls_), flops(flops_) {
-    if (c->profiling) {
+    if (c->profiling && cls != PC_OTHER) {
       a = prof_event(c);
       cudaEventRecord(a, s);
     }
   }
   ~ProfScope() {
-    if (c->profiling) {
+    if (c->profiling && cls != PC_OTHER) {
       cudaEvent_t b = prof_event(c);
       cudaEventRecord(b, s);
       c->prof_recs.push_back({a, b, cls, flops});
@@ -1127,6 +1128,36 @@ lst_status lst_get_logits(lst_ctx* c, float* dst) {
   if (!c->have_logits) return fail(c, LST_ERR_STATE, "no logits: run lst_step first");
   const bool dev = is_device_ptr(dst);
   CK(cudaMemcpyAsync(dst, c->logits, c->curT * c->V * 4, dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
+                     c->stream));
+  CK(cudaStreamSynchronize(c->stream));
+  return LST_OK;
+}
+
+lst_status lst_get_activation(lst_ctx* c, int32_t which, int32_t layer, void* dst) {
+  if (!c) return LST_ERR_ARG;
+  if (!dst) return fail(c, LST_ERR_ARG, "null dst");
+  if (c->st.steps == 0) return fail(c, LST_ERR_STATE, "no step has run");
+  const int64_t T = c->curT, d = c->d;
+  const void* src = nullptr;
+  int64_t bytes = 0;
+  if (which == LST_ACT_X) {
+    if (layer < 0 || layer > c->L) return fail(c, LST_ERR_ARG, "layer outside [0, L]");
+    src = c->xs + (int64_t)layer * c->Tmax * d;
+    bytes = T * d * 4;
+  } else {
+    if (layer != 0) return fail(c, LST_ERR_ARG, "intermediates are kept for layer 0 only");
+    switch (which) {
+      case LST_ACT_N1: src = c->n1; bytes = T * d * 2; break;
+      case LST_ACT_QKV: src = c->qkv; bytes = T * c->dqkv * 2; break;
+      case LST_ACT_O: src = c->o; bytes = T * c->dq * 2; break;
+      case LST_ACT_H: src = c->h; bytes = T * d * 4; break;
+      case LST_ACT_N2: src = c->n2; bytes = T * d * 2; break;
+      case LST_ACT_GU: src = c->gu; bytes = T * 2 * c->F * 2; break;
+      case LST_ACT_M: src = c->m; bytes = T * c->F * 2; break;
+      default: return fail(c, LST_ERR_ARG, "unknown activation");
+    }
+  }
+  CK(cudaMemcpyAsync(dst, src, bytes, is_device_ptr(dst) ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
                      c->stream));
   CK(cudaStreamSynchronize(c->stream));
   return LST_OK;

@@ -52,16 +52,41 @@ def uniform(seed: int, stream: int, n: int, lo: float = 0.0, hi: float = 1.0) ->
     return lo + (hi - lo) * u
 
 
+def _normal_chunk(args) -> np.ndarray:
+    seed, stream, s, m = args
+    z = raw_u64(seed, stream, 2 * s, 2 * m) >> np.uint64(11)
+    u = z.astype(np.float64) * (2.0 ** -53)
+    u1 = 1.0 - u[0::2]          # (0, 1]
+    u2 = u[1::2]
+    return np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+
+
+_POOL = None
+
+
+def _pool():
+    """Worker processes for large draws (spawned, so safe after CUDA is initialised)."""
+    global _POOL
+    if _POOL is None:
+        import concurrent.futures as cf
+        import multiprocessing as mp
+        import os
+        _POOL = cf.ProcessPoolExecutor(max_workers=min(16, os.cpu_count() or 1),
+                                       mp_context=mp.get_context("spawn"))
+    return _POOL
+
+
 def normal(seed: int, stream: int, n: int, std: float = 1.0, chunk: int = 1 << 24) -> np.ndarray:
-    """n standard normals x std (fp64) by Box-Muller: counters 2i, 2i+1 give one normal."""
+    """n standard normals x std (fp64) by Box-Muller: counters 2i, 2i+1 give one normal.
+    The values do not depend on the chunking (each chunk starts at its own counter)."""
     out = np.empty(n, dtype=np.float64)
-    for s in range(0, n, chunk):
-        m = min(chunk, n - s)
-        z = raw_u64(seed, stream, 2 * s, 2 * m) >> np.uint64(11)
-        u = z.astype(np.float64) * (2.0 ** -53)
-        u1 = 1.0 - u[0::2]          # (0, 1]
-        u2 = u[1::2]
-        out[s:s + m] = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+    jobs = [(seed, stream, s, min(chunk, n - s)) for s in range(0, n, chunk)]
+    if len(jobs) > 2:
+        for (_, _, s, m), part in zip(jobs, _pool().map(_normal_chunk, jobs)):
+            out[s:s + m] = part
+    else:
+        for (_, _, s, m) in jobs:
+            out[s:s + m] = _normal_chunk((seed, stream, s, m))
     return out * std
 
 
