@@ -103,6 +103,8 @@ typedef struct {
   double gemm_ms, attention_ms, dequant_ms, other_ms, copy_ms, step_ms;
   int64_t gemm_launches, attention_launches, dequant_launches, copy_count;
   double gemm_flops;           /* algorithmic FLOPs of the GEMM launches of the last step */
+  double lora_ms;              /* LoRA side path (skinny projections, dA / dB) */
+  int64_t lora_launches;
 } lst_stats;
 
 /* Create a context. embed [V, d], final_norm [d], lm_head [V, d] are fp32 (host or device; the

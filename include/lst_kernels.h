@@ -28,13 +28,14 @@ lst_status lst_k_nf4_quantize(const float* w, int64_t n, uint8_t* packed, int8_t
 lst_status lst_k_nf4_dequant(const uint8_t* packed, const int8_t* qabs, const float* gscale,
                              const float* mean, int64_t n, uint16_t* out, void* stream);
 
-/* C = alpha * (A B' + A2 B2') + bias + R on the tcgen05 tensor cores (fp32 accumulate).
- * A [M, K] row stride lda; B' = B^T with B [N, K] (b_mn = 0) or B' = B with B [K, N] (b_mn = 1),
+/* C = alpha * (A' B' + A2 B2') + bias + R on the tcgen05 tensor cores (fp32 accumulate).
+ * A' = A with A [M, K] (a_mn = 0) or A' = A^T with A [K, M] (a_mn = 1, needs b_mn = 1), row
+ * stride lda; B' = B^T with B [N, K] (b_mn = 0) or B' = B with B [K, N] (b_mn = 1),
  * row stride ldb; (A2 [M, K2], B2) optional second pair of the same major-ness (NULL to skip);
  * C [M, N] fp32 (c_f32 = 1) or bf16; bias [N] fp32 or NULL; R [M, N] fp32 (residual) or NULL.
  * Leading dimensions must be multiples of 8 and A/B/A2/B2 16-byte aligned. */
 lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda,
-                      const uint16_t* B, int64_t ldb, int32_t b_mn, const uint16_t* A2,
+                      int32_t a_mn, const uint16_t* B, int64_t ldb, int32_t b_mn, const uint16_t* A2,
                       int64_t lda2, const uint16_t* B2, int64_t ldb2, int32_t K2, void* C,
                       int64_t ldc, int32_t c_f32, float alpha, const float* bias,
                       const float* R, int64_t ldr, void* stream);
@@ -80,10 +81,14 @@ lst_status lst_k_swiglu_bwd(const float* dm, const uint16_t* gu, int64_t T, int3
 lst_status lst_k_cross_entropy(const float* logits, int64_t T, int32_t V, const int32_t* targets,
                                float inv_T, float* loss_rows, uint16_t* dlogits, void* stream);
 
-/* LoRA down-projection U = X A^T (A fp32 [R, in]); U fp32 [T, R], Us = bf16(s U) [T, ldus]. */
-lst_status lst_k_lora_project(const uint16_t* X, int64_t ldx, int64_t T, int32_t in,
-                              const float* A, int32_t R, float s, float* U, uint16_t* Us,
-                              int64_t ldus, void* stream);
+/* LoRA skinny projection Us = bf16(s * X Bop) of the side path ("Fine-Tuning an 8B Parameter
+ * Model on a 4 GB Laptop GPU", section "LoRA and QLoRA"): X bf16 [T, K] (row stride ldx); Bop bf16
+ * K-major [KP, K] (b_mn = 0: Us = s X Bop^T) or MN-major [K, KP] (b_mn = 1: Us = s X Bop);
+ * Us [T, KP] contiguous. Split-K on the tensor cores with a fixed-order reduction; scratch: fp32
+ * device buffer of scratch_floats >= 16 * T * KP. */
+lst_status lst_k_lora_skinny(const uint16_t* X, int64_t ldx, int64_t T, int32_t K,
+                             const uint16_t* Bop, int64_t ldb, int32_t b_mn, int32_t KP, float s,
+                             uint16_t* Us, float* scratch, int64_t scratch_floats, void* stream);
 
 /* Kernel launches made by this library so far in this process (all contexts). Needs no GPU. */
 int64_t lst_k_launch_count(void);

@@ -45,7 +45,8 @@ class Stats(C.Structure):
                 ("gemm_ms", C.c_double), ("attention_ms", C.c_double), ("dequant_ms", C.c_double),
                 ("other_ms", C.c_double), ("copy_ms", C.c_double), ("step_ms", C.c_double),
                 ("gemm_launches", C.c_int64), ("attention_launches", C.c_int64),
-                ("dequant_launches", C.c_int64), ("copy_count", C.c_int64), ("gemm_flops", C.c_double)]
+                ("dequant_launches", C.c_int64), ("copy_count", C.c_int64), ("gemm_flops", C.c_double),
+                ("lora_ms", C.c_double), ("lora_launches", C.c_int64)]
 
     def as_dict(self) -> dict:
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -70,7 +71,7 @@ _SIGS = {
     "lst_blob_bytes": (_I64, [C.POINTER(Config)]),
     "lst_k_nf4_quantize": (_I32, [_P, _I64, _P, _P, _P, _P, _P]),
     "lst_k_nf4_dequant": (_I32, [_P, _P, _P, _P, _I64, _P, _P]),
-    "lst_k_gemm": (_I32, [_I32, _I32, _I32, _P, _I64, _P, _I64, _I32, _P, _I64, _P, _I64, _I32,
+    "lst_k_gemm": (_I32, [_I32, _I32, _I32, _P, _I64, _I32, _P, _I64, _I32, _P, _I64, _P, _I64, _I32,
                           _P, _I64, _I32, _F32, _P, _P, _I64, _P]),
     "lst_k_attention_fwd": (_I32, [_P, _I64, _P, _I64, _P, _I64, _P, _I64, _P, _I64, _I32, _I32,
                                    _I32, _I32, _P]),
@@ -83,7 +84,7 @@ _SIGS = {
     "lst_k_swiglu_fwd": (_I32, [_P, _I64, _I32, _P, _P]),
     "lst_k_swiglu_bwd": (_I32, [_P, _P, _I64, _I32, _P, _P]),
     "lst_k_cross_entropy": (_I32, [_P, _I64, _I32, _P, _F32, _P, _P, _P]),
-    "lst_k_lora_project": (_I32, [_P, _I64, _I64, _I32, _P, _I32, _F32, _P, _P, _I64, _P]),
+    "lst_k_lora_skinny": (_I32, [_P, _I64, _I64, _I32, _P, _I64, _I32, _I32, _F32, _P, _P, _I64, _P]),
     "lst_k_launch_count": (_I64, []),
 }
 
@@ -259,9 +260,9 @@ def k_nf4_dequant(packed, qabs, gscale, mean, n, out, stream=None):
 
 
 def k_gemm(M, N, K, A, lda, B, ldb, b_mn, C_, ldc, c_f32, alpha=1.0, A2=None, lda2=0, B2=None, ldb2=0,
-           K2=0, bias=None, R=None, ldr=0, stream=None):
-    _check(lib().lst_k_gemm(M, N, K, _ptr(A), lda, _ptr(B), ldb, b_mn, _ptr(A2), lda2, _ptr(B2), ldb2, K2,
-                            _ptr(C_), ldc, c_f32, alpha, _ptr(bias), _ptr(R), ldr, _stream(stream)),
+           K2=0, bias=None, R=None, ldr=0, a_mn=0, stream=None):
+    _check(lib().lst_k_gemm(M, N, K, _ptr(A), lda, a_mn, _ptr(B), ldb, b_mn, _ptr(A2), lda2, _ptr(B2), ldb2,
+                            K2, _ptr(C_), ldc, c_f32, alpha, _ptr(bias), _ptr(R), ldr, _stream(stream)),
            what="lst_k_gemm")
 
 
@@ -311,9 +312,9 @@ def k_cross_entropy(logits, T, V, targets, inv_T, loss_rows, dlogits, stream=Non
                                      _ptr(dlogits), _stream(stream)), what="lst_k_cross_entropy")
 
 
-def k_lora_project(X, ldx, T, in_, A, R, s, U, Us, ldus, stream=None):
-    _check(lib().lst_k_lora_project(_ptr(X), ldx, T, in_, _ptr(A), R, s, _ptr(U), _ptr(Us), ldus,
-                                    _stream(stream)), what="lst_k_lora_project")
+def k_lora_skinny(X, ldx, T, K, Bop, ldb, b_mn, KP, s, Us, scratch, stream=None):
+    _check(lib().lst_k_lora_skinny(_ptr(X), ldx, T, K, _ptr(Bop), ldb, b_mn, KP, s, _ptr(Us), _ptr(scratch),
+                                   scratch.numel(), _stream(stream)), what="lst_k_lora_skinny")
 
 
 def launch_count() -> int:

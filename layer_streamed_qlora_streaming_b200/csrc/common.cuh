@@ -107,10 +107,10 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
-// Instruction descriptor of kind::f16 with bf16 A/B, fp32 accumulate, M x N, K-major A and
-// K-major (b_mn = 0) or MN-major (b_mn = 1) B.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, int b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) |
+// Instruction descriptor of kind::f16 with bf16 A/B, fp32 accumulate, M x N; A and B K-major
+// (a_mn / b_mn = 0) or MN-major (= 1).
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 

@@ -20,6 +20,7 @@
 #include "attention.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "lora.cuh"
 #include "nf4.cuh"
 #include "ops.cuh"
 
@@ -157,7 +158,7 @@ bool is_device_ptr(const void* p) {
 }
 
 // Profiling classes
-enum { PC_GEMM = 0, PC_ATTN = 1, PC_DEQ = 2, PC_OTHER = 3, PC_COPY = 4, PC_N = 5 };
+enum { PC_GEMM = 0, PC_ATTN = 1, PC_DEQ = 2, PC_OTHER = 3, PC_COPY = 4, PC_LORA = 5, PC_N = 6 };
 
 }  // namespace
 
@@ -186,11 +187,9 @@ struct lst_ctx {
   float* lora = nullptr;
   int64_t lora_numel = 0;
   std::vector<int64_t> offA, offB;
-  struct Derived {
-    float* Acat32 = nullptr;
-    __nv_bfloat16* Acat16 = nullptr;
-    float* BexpT32 = nullptr;
-    __nv_bfloat16* Bexp16 = nullptr;
+  struct Derived {                 // bf16 operands of the LoRA side path, per fused group
+    __nv_bfloat16* Acat16 = nullptr;  // [KP, in]
+    __nv_bfloat16* Bexp16 = nullptr;  // [out, KP]
   };
   std::vector<Derived> der;  // L * NGROUP
   float* grads = nullptr;
@@ -200,10 +199,8 @@ struct lst_ctx {
   __nv_bfloat16 *n1 = nullptr, *qkv = nullptr, *o = nullptr, *n2 = nullptr, *gu = nullptr, *m = nullptr,
                 *wscr = nullptr;
   float *rstd1 = nullptr, *rstd2 = nullptr, *lse = nullptr, *Dbuf = nullptr;
-  float* U[NGROUP] = {};
-  __nv_bfloat16* Us[NGROUP] = {};
-  float* Vv[NGROUP] = {};
-  __nv_bfloat16* Vs[NGROUP] = {};
+  __nv_bfloat16* Us[NGROUP] = {};  // bf16(s * x A^T) per group [T, KP]
+  __nv_bfloat16* Vs[NGROUP] = {};  // bf16(s * dy B) per group [T, KP]
   float *ga = nullptr, *gb = nullptr, *dn = nullptr, *dm = nullptr, *part = nullptr;
   __nv_bfloat16 *dout_b = nullptr, *dh_b = nullptr, *do_b = nullptr, *dqkvb = nullptr, *dgu = nullptr;
   __nv_bfloat16* nf = nullptr;
@@ -330,9 +327,7 @@ lst_status prep_lora(lst_ctx* c, int layer) {
     a.in = G.in;
     for (int k = 0; k <= G.nseg; ++k) a.bounds[k] = G.bounds[k];
     a.KP = G.KP;
-    a.Acat32 = D.Acat32;
     a.Acat16 = D.Acat16;
-    a.BexpT32 = D.BexpT32;
     a.Bexp16 = D.Bexp16;
     CK(lora_prep(a, c->stream));
   }
@@ -348,8 +343,8 @@ lst_status group_fwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
   const auto& D = c->der[layer * NGROUP + g];
   const int64_t T = c->curT;
   {
-    ProfScope ps(c, c->stream, PC_OTHER);
-    CK(lora_project(X, ldx, T, G.in, D.Acat32, G.in, G.R, c->s, c->U[g], c->Us[g], G.KP, c->stream));
+    ProfScope ps(c, c->stream, PC_LORA);  // Us = bf16(s * X Acat^T)
+    CK(lora_skinny(X, ldx, T, G.in, D.Acat16, G.in, 0, G.KP, c->s, c->part, c->Us[g], c->stream));
   }
   if (!gemm) return LST_OK;
   GemmArgs a;
@@ -383,8 +378,8 @@ lst_status group_bwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
   const auto& D = c->der[layer * NGROUP + g];
   const int64_t T = c->curT;
   {
-    ProfScope ps(c, c->stream, PC_OTHER);
-    CK(lora_project(dY, ldy, T, G.out, D.BexpT32, G.out, G.R, c->s, c->Vv[g], c->Vs[g], G.KP, c->stream));
+    ProfScope ps(c, c->stream, PC_LORA);  // Vs = bf16(s * dY Bexp)
+    CK(lora_skinny(dY, ldy, T, G.out, D.Bexp16, G.KP, 1, G.KP, c->s, c->part, c->Vs[g], c->stream));
   }
   {
     GemmArgs a;
@@ -407,35 +402,16 @@ lst_status group_bwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
     ProfScope ps(c, c->stream, PC_GEMM, 2.0 * T * G.in * (double)(G.out + G.KP));
     CK(gemm_bf16(a, c->stream));
   }
-  ProfScope ps(c, c->stream, PC_OTHER);
-  LoraGradArgs ga{};
-  ga.P = c->Vv[g];
-  ga.R = G.R;
-  ga.Q = X;
-  ga.ldq = ldx;
-  ga.C = G.in;
-  ga.T = T;
-  ga.s = c->s;
-  ga.seg_r = 0;
-  ga.nseg = G.nseg;
-  ga.rows_per_dst = c->r;
-  for (int k = 0; k < G.nseg; ++k) ga.dst[k] = c->grads + c->offA[layer * NPROJ + G.proj[k]];
-  ga.partial = c->part;
-  CK(lora_grad(ga, c->stream));
-  LoraGradArgs gb{};
-  gb.P = c->U[g];
-  gb.R = G.R;
-  gb.Q = dY;
-  gb.ldq = ldy;
-  gb.C = G.out;
-  gb.T = T;
-  gb.s = c->s;
-  gb.seg_r = c->r;
-  gb.nseg = G.nseg;
-  for (int k = 0; k <= G.nseg; ++k) gb.bounds[k] = G.bounds[k];
-  for (int k = 0; k < G.nseg; ++k) gb.dst[k] = c->grads + c->offB[layer * NPROJ + G.proj[k]];
-  gb.partial = c->part;
-  CK(lora_grad(gb, c->stream));
+  ProfScope ps(c, c->stream, PC_LORA);
+  float* dA[3] = {nullptr, nullptr, nullptr};
+  float* dB[3] = {nullptr, nullptr, nullptr};
+  for (int k = 0; k < G.nseg; ++k) {
+    dA[k] = c->grads + c->offA[layer * NPROJ + G.proj[k]];
+    dB[k] = c->grads + c->offB[layer * NPROJ + G.proj[k]];
+  }
+  // dA = s V^T X and dB = s dY^T U, with s folded into Vs and Us
+  CK(lora_grad_a(X, ldx, T, G.in, c->Vs[g], G.KP, G.nseg, c->r, dA, c->part, c->stream));
+  CK(lora_grad_b(dY, ldy, T, G.out, c->Us[g], G.KP, G.nseg, c->r, G.bounds, dB, c->part, c->stream));
   return LST_OK;
 }
 
@@ -700,8 +676,8 @@ lst_status finish_step(lst_ctx* c, float* loss, float* grads_out) {
   c->st.steps += 1;
   c->st.launches_last_step = g_launch_count.load() - c->launches_at_step_start;
   if (c->profiling) {
-    double ms[PC_N] = {0, 0, 0, 0, 0};
-    int64_t cnt[PC_N] = {0, 0, 0, 0, 0};
+    double ms[PC_N] = {};
+    int64_t cnt[PC_N] = {};
     double flops = 0;
     for (auto& r : c->prof_recs) {
       float t = 0.f;
@@ -721,6 +697,8 @@ lst_status finish_step(lst_ctx* c, float* loss, float* grads_out) {
     c->st.attention_launches = cnt[PC_ATTN];
     c->st.dequant_launches = cnt[PC_DEQ];
     c->st.copy_count = cnt[PC_COPY];
+    c->st.lora_ms = ms[PC_LORA];
+    c->st.lora_launches = cnt[PC_LORA];
     c->st.gemm_flops = flops;
     c->st.step_ms = step;
   }
@@ -838,9 +816,7 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
     for (int g = 0; g < NGROUP; ++g) {
       auto& D = c->der[l * NGROUP + g];
       const Group& G = c->grp[g];
-      TRY(dalloc(c, &D.Acat32, (int64_t)G.R * G.in, true));
       TRY(dalloc(c, &D.Acat16, (int64_t)G.KP * G.in, true));
-      TRY(dalloc(c, &D.BexpT32, (int64_t)G.R * G.out, true));
       TRY(dalloc(c, &D.Bexp16, (int64_t)G.out * G.KP, true));
     }
 
@@ -880,14 +856,12 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   int64_t part = 0;
   for (int g = 0; g < NGROUP; ++g) {
     const Group& G = c->grp[g];
-    TRY(dalloc(c, &c->U[g], T * G.R));
     TRY(dalloc(c, &c->Us[g], T * G.KP, true));
-    TRY(dalloc(c, &c->Vv[g], T * G.R));
     TRY(dalloc(c, &c->Vs[g], T * G.KP, true));
-    part = std::max(part, (int64_t)G.R * G.in);
-    part = std::max(part, (int64_t)c->r * G.out);
+    part = std::max(part, lora_skinny_scratch(T, G.KP));
+    part = std::max(part, (int64_t)G.KP * std::max(G.in, G.out));
   }
-  TRY(dalloc(c, &c->part, part * ((T + 127) / 128)));
+  TRY(dalloc(c, &c->part, part));
   TRY(dalloc(c, &c->ga, T * d));
   TRY(dalloc(c, &c->gb, T * d));
   TRY(dalloc(c, &c->dn, T * d));

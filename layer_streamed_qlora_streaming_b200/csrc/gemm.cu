@@ -95,11 +95,14 @@ __device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const
   }
 }
 
-template <int BN, int BMN>
+// AMN / BMN: A / B operand MN-major (row-major [K, M] / [K, N] in global memory), else K-major.
+// Split-K: blockIdx.z takes main k-blocks [z * kps, (z + 1) * kps) and writes its partial result
+// at C + z * split_stride (the second operand pair is only allowed without split).
+template <int BN, int AMN, int BMN>
 __global__ void __launch_bounds__(192, 1)
 k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
        const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-       const Epi ep, const int nk1, const int nk2) {
+       Epi ep, const int nk1_total, const int nk2, const int kps, const int64_t split_stride) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -114,7 +117,13 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * BM;
   const int n0 = blockIdx.x * BN;
+  const int kb0 = blockIdx.z * kps;
+  const int nk1 = min(nk1_total - kb0, kps);
   const int nk = nk1 + nk2;
+  if (blockIdx.z) {
+    ep.C = ep.c_f32 ? static_cast<void*>(static_cast<float*>(ep.C) + blockIdx.z * split_stride)
+                    : static_cast<void*>(static_cast<__nv_bfloat16*>(ep.C) + blockIdx.z * split_stride);
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -151,8 +160,14 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         const bool second = kb >= nk1;
         const CUtensorMap* ma = second ? &tmA2 : &tmA;
         const CUtensorMap* mb = second ? &tmB2 : &tmB;
-        const int kk = (second ? kb - nk1 : kb) * BK;
-        tma_load_2d(sA + s * C::A_BYTES, ma, &full[s], kk, m0);
+        const int kk = (second ? kb - nk1 : kb0 + kb) * BK;
+        if (AMN == 0) {
+          tma_load_2d(sA + s * C::A_BYTES, ma, &full[s], kk, m0);
+        } else {
+#pragma unroll
+          for (int c = 0; c < BM / 64; ++c)
+            tma_load_2d(sA + s * C::A_BYTES + c * (64 * BK * 2), ma, &full[s], m0 + c * 64, kk);
+        }
         if (BMN == 0) {
           tma_load_2d(sB + s * C::B_BYTES, mb, &full[s], kk, n0);
         } else {
@@ -164,7 +179,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16(BM, BN, BMN);
+      constexpr uint32_t idesc = umma_idesc_bf16(BM, BN, AMN, BMN);
       bool ok = true;
       for (int kb = 0; kb < nk && ok; ++kb) {
         const int s = kb % C::STAGES;
@@ -176,7 +191,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         const uint32_t b0 = smem_u32(sB + s * C::B_BYTES);
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k) {
-          const uint64_t da = umma_desc(a0 + k * 32, 16, 1024);
+          const uint64_t da = AMN ? umma_desc(a0 + k * 16 * 128, 64 * BK * 2, 1024)
+                                  : umma_desc(a0 + k * 32, 16, 1024);
           const uint64_t db = BMN ? umma_desc(b0 + k * 16 * 128, 64 * BK * 2, 1024)
                                   : umma_desc(b0 + k * 32, 16, 1024);
           umma_bf16(tmem, da, db, idesc, (kb | k) != 0);
@@ -233,12 +249,16 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int6
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int BMN>
+template <int BN, int AMN, int BMN>
 cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   using C = Cfg<BN>;
   CUtensorMap tA, tB, tA2, tB2;
   const int box_b = BMN ? BK : BN;  // K-major B: box [BN rows, 64 k]; MN-major: [64 k rows, 64 n]
-  if (!make_map(&tA, a.A, a.M, a.K, a.lda, BM)) return cudaErrorInvalidValue;
+  if (AMN) {
+    if (!make_map(&tA, a.A, a.K, a.M, a.lda, BK)) return cudaErrorInvalidValue;
+  } else {
+    if (!make_map(&tA, a.A, a.M, a.K, a.lda, BM)) return cudaErrorInvalidValue;
+  }
   if (BMN) {
     if (!make_map(&tB, a.B, a.K, a.N, a.ldb, box_b)) return cudaErrorInvalidValue;
   } else {
@@ -246,6 +266,7 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   }
   int nk2 = 0;
   if (a.A2 && a.B2 && a.K2 > 0) {
+    if (AMN || a.splits > 1) return cudaErrorInvalidValue;
     if (!make_map(&tA2, a.A2, a.M, a.K2, a.lda2, BM)) return cudaErrorInvalidValue;
     if (BMN) {
       if (!make_map(&tB2, a.B2, a.K2, a.N, a.ldb2, box_b)) return cudaErrorInvalidValue;
@@ -260,13 +281,19 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   Epi e{a.C, a.ldc, a.bias, a.R, a.ldr, a.alpha, a.c_f32, a.M, a.N};
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t err = cudaFuncSetAttribute(k_gemm<BN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t err =
+        cudaFuncSetAttribute(k_gemm<BN, AMN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (err != cudaSuccess) return err;
     attr_set = true;
   }
-  dim3 grid((a.N + BN - 1) / BN, (a.M + BM - 1) / BM);
   const int nk1 = (a.K + BK - 1) / BK;
-  k_gemm<BN, BMN><<<grid, 192, C::SMEM, s>>>(tA, tB, tA2, tB2, e, nk1, nk2);
+  int splits = a.splits < 1 ? 1 : a.splits;
+  if (splits > nk1) splits = nk1;
+  const int kps = (nk1 + splits - 1) / splits;
+  splits = (nk1 + kps - 1) / kps;  // no empty split
+  if (splits > 1 && a.split_stride < (int64_t)a.M * a.ldc) return cudaErrorInvalidValue;
+  dim3 grid((a.N + BN - 1) / BN, (a.M + BM - 1) / BM, splits);
+  k_gemm<BN, AMN, BMN><<<grid, 192, C::SMEM, s>>>(tA, tB, tA2, tB2, e, nk1, nk2, kps, a.split_stride);
   note_launch(1);
   return cudaGetLastError();
 }
@@ -275,23 +302,29 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
 
 cudaError_t gemm_bf16(const GemmArgs& a, cudaStream_t s) {
   if (a.M <= 0 || a.N <= 0 || a.K <= 0 || !a.A || !a.B || !a.C) return cudaErrorInvalidValue;
+  if (a.splits > 1 && (a.bias || a.R || a.A2)) return cudaErrorInvalidValue;  // partials are summed later
   // TMA: 16-byte aligned bases and row strides
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   if (!al16(a.A) || !al16(a.B) || (a.lda % 8) || (a.ldb % 8)) return cudaErrorInvalidValue;
   if (a.A2 && (!al16(a.A2) || !al16(a.B2) || (a.lda2 % 8) || (a.ldb2 % 8))) return cudaErrorInvalidValue;
-  const int64_t tiles256 = (int64_t)((a.M + BM - 1) / BM) * ((a.N + 255) / 256);
+  const int64_t tiles256 = (int64_t)((a.M + BM - 1) / BM) * ((a.N + 255) / 256) * (a.splits > 1 ? a.splits : 1);
   int bn;
   if (a.N <= 64) bn = 64;
   else if (a.N <= 128 || tiles256 < 120) bn = 128;
   else bn = 256;
-  if (a.b_mn) {
-    if (bn == 64) return launch<64, 1>(a, s);
-    if (bn == 128) return launch<128, 1>(a, s);
-    return launch<256, 1>(a, s);
+  const int code = bn * 4 + (a.a_mn ? 2 : 0) + (a.b_mn ? 1 : 0);
+  switch (code) {
+    case 64 * 4 + 0: return launch<64, 0, 0>(a, s);
+    case 64 * 4 + 1: return launch<64, 0, 1>(a, s);
+    case 64 * 4 + 3: return launch<64, 1, 1>(a, s);
+    case 128 * 4 + 0: return launch<128, 0, 0>(a, s);
+    case 128 * 4 + 1: return launch<128, 0, 1>(a, s);
+    case 128 * 4 + 3: return launch<128, 1, 1>(a, s);
+    case 256 * 4 + 0: return launch<256, 0, 0>(a, s);
+    case 256 * 4 + 1: return launch<256, 0, 1>(a, s);
+    case 256 * 4 + 3: return launch<256, 1, 1>(a, s);
+    default: return cudaErrorInvalidValue;  // MN-major A with K-major B is not instantiated
   }
-  if (bn == 64) return launch<64, 0>(a, s);
-  if (bn == 128) return launch<128, 0>(a, s);
-  return launch<256, 0>(a, s);
 }
 
 }  // namespace lst

@@ -2,8 +2,10 @@
 //
 //   C[m, n] = alpha * ( sum_k A[m, k] B(n, k)  +  sum_j A2[m, j] B2(n, j) ) + bias[n] + R[m, n]
 //
-// A, A2 are row-major [M, K] / [M, K2] (K-major). B is either row-major [N, K] (K-major,
-// b_mn = 0, "x W^T") or row-major [K, N] (MN-major, b_mn = 1, "x W"); B2 has the same major-ness.
+// A, A2 are row-major [M, K] / [M, K2] (K-major), or A is row-major [K, M] (a_mn = 1, "X^T ...").
+// B is either row-major [N, K] (K-major, b_mn = 0, "x W^T") or row-major [K, N] (MN-major,
+// b_mn = 1, "x W"); B2 has the same major-ness. With splits > 1 the K range is cut into slices
+// whose partial products are written side by side (fixed-order reduction left to the caller).
 // The optional (A2, B2) pair is a second contraction appended along K; the LoRA path uses it
 // to fold s (x A^T) B^T into the same accumulator as the frozen base.
 #pragma once
@@ -33,6 +35,9 @@ struct GemmArgs {
   const float* bias = nullptr;        // [N] or null
   const float* R = nullptr;           // fp32 residual [M, N] row stride ldr, or null
   int64_t ldr = 0;
+  int a_mn = 0;                       // 1: A is row-major [K, M] (MN-major); needs b_mn = 1
+  int splits = 1;                     // split-K: partial results at C + z * split_stride
+  int64_t split_stride = 0;
 };
 
 // Returns cudaSuccess or the launch / argument error. Deterministic: no split-K, no atomics.

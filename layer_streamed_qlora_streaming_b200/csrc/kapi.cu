@@ -3,6 +3,7 @@
 #include "attention.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "lora.cuh"
 #include "nf4.cuh"
 #include "ops.cuh"
 
@@ -53,7 +54,8 @@ lst_status lst_k_nf4_dequant(const uint8_t* packed, const int8_t* qabs, const fl
   return st(nf4_dequant(&s, 1, B16(out), S(stream)));
 }
 
-lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb,
+lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda, int32_t a_mn, const uint16_t* B,
+                      int64_t ldb,
                       int32_t b_mn, const uint16_t* A2, int64_t lda2, const uint16_t* B2, int64_t ldb2, int32_t K2,
                       void* C, int64_t ldc, int32_t c_f32, float alpha, const float* bias, const float* R,
                       int64_t ldr, void* stream) {
@@ -68,6 +70,7 @@ lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_
   a.B = B16(B);
   a.ldb = ldb;
   a.b_mn = b_mn ? 1 : 0;
+  a.a_mn = a_mn ? 1 : 0;
   a.A2 = B16(A2);
   a.lda2 = lda2;
   a.B2 = B16(B2);
@@ -165,10 +168,12 @@ lst_status lst_k_cross_entropy(const float* logits, int64_t T, int32_t V, const 
   return st(cross_entropy(logits, T, V, targets, inv_T, loss_rows, B16(dlogits), S(stream)));
 }
 
-lst_status lst_k_lora_project(const uint16_t* X, int64_t ldx, int64_t T, int32_t in, const float* A, int32_t R, float s,
-                              float* U, uint16_t* Us, int64_t ldus, void* stream) {
-  if (!X || !A || !U || !Us || T <= 0 || in <= 0 || R <= 0 || R > 64) return LST_ERR_ARG;
-  return st(lora_project(B16(X), ldx, T, in, A, in, R, s, U, B16(Us), ldus, S(stream)));
+lst_status lst_k_lora_skinny(const uint16_t* X, int64_t ldx, int64_t T, int32_t K, const uint16_t* Bop, int64_t ldb,
+                             int32_t b_mn, int32_t KP, float s, uint16_t* Us, float* scratch, int64_t scratch_floats,
+                             void* stream) {
+  if (!X || !Bop || !Us || !scratch || T <= 0 || K <= 0 || KP <= 0) return LST_ERR_ARG;
+  if (scratch_floats < lora_skinny_scratch(T, KP)) return LST_ERR_ARG;
+  return st(lora_skinny(B16(X), ldx, T, K, B16(Bop), ldb, b_mn ? 1 : 0, KP, s, scratch, B16(Us), S(stream)));
 }
 
 int64_t lst_k_launch_count(void) { return g_launch_count.load(); }

@@ -223,133 +223,6 @@ __global__ void k_bf16_to_f32(const bf16* __restrict__ x, int64_t n, float* __re
   if (i < n) y[i] = __bfloat162float(x[i]);
 }
 
-// ------------------------------------------------------------------------------- LoRA
-// One warp per token row; the A columns are staged 128 at a time in shared memory.
-template <int RP>
-__global__ void __launch_bounds__(256) k_lora_project(const bf16* __restrict__ X, int64_t ldx, int64_t T, int in,
-                                                      const float* __restrict__ A, int64_t lda, int R, float s,
-                                                      float* __restrict__ U, bf16* __restrict__ Us, int64_t ldus) {
-  __shared__ __align__(16) float As[RP][128];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t = (int64_t)blockIdx.x * 8 + warp;
-  float acc[RP];
-#pragma unroll
-  for (int j = 0; j < RP; ++j) acc[j] = 0.f;
-  for (int c0 = 0; c0 < in; c0 += 128) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < RP * 128; i += 256) {
-      const int j = i >> 7, c = i & 127;
-      As[j][c] = (j < R && c0 + c < in) ? A[(int64_t)j * lda + c0 + c] : 0.f;
-    }
-    __syncthreads();
-    if (t < T) {
-      const int c = c0 + lane * 4;
-      float x[4] = {0.f, 0.f, 0.f, 0.f};
-      const bf16* xr = X + t * ldx;
-      if (c + 3 < in) {
-        const uint2 u = *reinterpret_cast<const uint2*>(xr + c);
-        const bf16* h = reinterpret_cast<const bf16*>(&u);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = __bfloat162float(h[e]);
-      } else {
-        for (int e = 0; e < 4; ++e)
-          if (c + e < in) x[e] = __bfloat162float(xr[c + e]);
-      }
-#pragma unroll
-      for (int j = 0; j < RP; ++j) {
-        const float4 a = *reinterpret_cast<const float4*>(&As[j][lane * 4]);
-        float v = acc[j];
-        v = fmaf(x[0], a.x, v);
-        v = fmaf(x[1], a.y, v);
-        v = fmaf(x[2], a.z, v);
-        v = fmaf(x[3], a.w, v);
-        acc[j] = v;
-      }
-    }
-  }
-  if (t >= T) return;
-#pragma unroll
-  for (int j = 0; j < RP; ++j) {
-    const float v = warp_sum(acc[j]);
-    if (lane == 0 && j < R) {
-      U[t * R + j] = v;
-      Us[t * ldus + j] = __float2bfloat16_rn(s * v);
-    }
-  }
-}
-
-// Partial sums over a chunk of 128 tokens: thread = column.
-template <int JR>
-__global__ void __launch_bounds__(128) k_lora_grad_partial(const LoraGradArgs a) {
-  __shared__ float Ps[128][64];
-  const int c = blockIdx.x * 128 + threadIdx.x;
-  const int64_t t0 = (int64_t)blockIdx.y * 128;
-  const int nt = (int)min((int64_t)128, a.T - t0);
-  for (int i = threadIdx.x; i < nt * a.R; i += 128) Ps[i / a.R][i % a.R] = a.P[(t0 + i / a.R) * a.R + i % a.R];
-  __syncthreads();
-  if (c >= a.C) return;
-  int jb = 0;
-  if (a.seg_r) {
-    int p = 0;
-    while (p + 1 < a.nseg && c >= a.bounds[p + 1]) ++p;
-    jb = p * a.seg_r;
-  }
-  float acc[JR];
-#pragma unroll
-  for (int j = 0; j < JR; ++j) acc[j] = 0.f;
-  const bf16* q = a.Q + t0 * a.ldq + c;
-  for (int tt = 0; tt < nt; ++tt) {
-    const float qv = __bfloat162float(q[(int64_t)tt * a.ldq]);
-#pragma unroll
-    for (int j = 0; j < JR; ++j) acc[j] = fmaf(Ps[tt][jb + j], qv, acc[j]);
-  }
-  float* out = a.partial + (int64_t)blockIdx.y * JR * a.C;
-#pragma unroll
-  for (int j = 0; j < JR; ++j) out[(int64_t)j * a.C + c] = acc[j];
-}
-
-__global__ void k_lora_grad_reduce(const LoraGradArgs a, int JR, int nchunks) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (int64_t)JR * a.C) return;
-  const int j = (int)(i / a.C), c = (int)(i % a.C);
-  float s = 0.f;
-  for (int k = 0; k < nchunks; ++k) s += a.partial[((int64_t)k * JR + j) * a.C + c];
-  s *= a.s;
-  if (a.seg_r) {
-    int p = 0;
-    while (p + 1 < a.nseg && c >= a.bounds[p + 1]) ++p;
-    a.dst[p][(int64_t)(c - a.bounds[p]) * a.seg_r + j] = s;
-  } else {
-    a.dst[j / a.rows_per_dst][(int64_t)(j % a.rows_per_dst) * a.C + c] = s;
-  }
-}
-
-__global__ void k_lora_prep(const LoraPrepArgs a) {
-  const int R = a.nseg * a.r;
-  const int out = a.bounds[a.nseg];
-  const int64_t n1 = (int64_t)a.KP * a.in;      // Acat16 (covers Acat32 rows < R)
-  const int64_t n2 = (int64_t)out * a.KP;       // Bexp16 (covers BexpT32 entries j < R)
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n1; i += stride) {
-    const int j = (int)(i / a.in), c = (int)(i % a.in);
-    float v = 0.f;
-    if (j < R) {
-      v = a.A[j / a.r][(int64_t)(j % a.r) * a.in + c];
-      a.Acat32[i] = v;
-    }
-    a.Acat16[i] = __float2bfloat16_rn(v);
-  }
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += stride) {
-    const int o = (int)(i / a.KP), j = (int)(i % a.KP);
-    int p = 0;
-    while (p + 1 < a.nseg && o >= a.bounds[p + 1]) ++p;
-    float v = 0.f;
-    if (j < R && j / a.r == p) v = a.B[p][(int64_t)(o - a.bounds[p]) * a.r + (j % a.r)];
-    a.Bexp16[i] = __float2bfloat16_rn(v);
-    if (j < R) a.BexpT32[(int64_t)j * out + o] = v;
-  }
-}
-
 inline unsigned nblk(int64_t n, int t = kThreads) { return (unsigned)((n + t - 1) / t); }
 
 }  // namespace
@@ -418,44 +291,6 @@ cudaError_t f32_to_bf16(const float* x, int64_t n, bf16* y, cudaStream_t s) {
 }
 cudaError_t bf16_to_f32(const bf16* x, int64_t n, float* y, cudaStream_t s) {
   k_bf16_to_f32<<<nblk(n), kThreads, 0, s>>>(x, n, y);
-  note_launch(1);
-  return cudaGetLastError();
-}
-
-cudaError_t lora_project(const bf16* X, int64_t ldx, int64_t T, int in, const float* A, int64_t lda, int R,
-                         float s, float* U, bf16* Us, int64_t ldus, cudaStream_t st) {
-  if (R <= 0 || R > 64 || (ldx % 4)) return cudaErrorInvalidValue;
-  const unsigned g = (unsigned)((T + 7) / 8);
-  if (R <= 16) k_lora_project<16><<<g, 256, 0, st>>>(X, ldx, T, in, A, lda, R, s, U, Us, ldus);
-  else if (R <= 32) k_lora_project<32><<<g, 256, 0, st>>>(X, ldx, T, in, A, lda, R, s, U, Us, ldus);
-  else if (R <= 48) k_lora_project<48><<<g, 256, 0, st>>>(X, ldx, T, in, A, lda, R, s, U, Us, ldus);
-  else k_lora_project<64><<<g, 256, 0, st>>>(X, ldx, T, in, A, lda, R, s, U, Us, ldus);
-  note_launch(1);
-  return cudaGetLastError();
-}
-
-cudaError_t lora_grad(const LoraGradArgs& a, cudaStream_t st) {
-  const int JR = a.seg_r ? a.seg_r : a.R;
-  if (a.R <= 0 || a.R > 64 || a.C <= 0 || a.T <= 0) return cudaErrorInvalidValue;
-  const int nchunks = (int)((a.T + 127) / 128);
-  dim3 grid((a.C + 127) / 128, nchunks);
-  switch (JR) {
-    case 8: k_lora_grad_partial<8><<<grid, 128, 0, st>>>(a); break;
-    case 16: k_lora_grad_partial<16><<<grid, 128, 0, st>>>(a); break;
-    case 24: k_lora_grad_partial<24><<<grid, 128, 0, st>>>(a); break;
-    case 32: k_lora_grad_partial<32><<<grid, 128, 0, st>>>(a); break;
-    case 48: k_lora_grad_partial<48><<<grid, 128, 0, st>>>(a); break;
-    case 64: k_lora_grad_partial<64><<<grid, 128, 0, st>>>(a); break;
-    default: return cudaErrorInvalidValue;
-  }
-  k_lora_grad_reduce<<<nblk((int64_t)JR * a.C), kThreads, 0, st>>>(a, JR, nchunks);
-  note_launch(2);
-  return cudaGetLastError();
-}
-
-cudaError_t lora_prep(const LoraPrepArgs& a, cudaStream_t st) {
-  if (a.nseg < 1 || a.nseg > 3 || a.nseg * a.r > a.KP) return cudaErrorInvalidValue;
-  k_lora_prep<<<1024, kThreads, 0, st>>>(a);
   note_launch(1);
   return cudaGetLastError();
 }

@@ -43,51 +43,4 @@ cudaError_t dot_fixed(const float* a, const bf16* b, int64_t n, float* partials,
 cudaError_t f32_to_bf16(const float* x, int64_t n, bf16* y, cudaStream_t s);
 cudaError_t bf16_to_f32(const bf16* x, int64_t n, float* y, cudaStream_t s);
 
-// ------------------------------------------------------------------------ LoRA side path
-// U[t, j] = sum_i X[t, i] * A[j, i] for j < R (A fp32 [R, in] row stride lda); writes U fp32
-// [T, R] (row stride R) and Us = bf16(s * U) [T, ldus].
-cudaError_t lora_project(const bf16* X, int64_t ldx, int64_t T, int in, const float* A, int64_t lda, int R,
-                         float s, float* U, bf16* Us, int64_t ldus, cudaStream_t st);
-
-// Fixed-order reduction over tokens of out[j, c] = s * sum_t P[t, j] * Q[t, c].
-// P fp32 [T, R] (row stride R), Q bf16 [T, ldq] with C columns. If seg_r > 0 the columns are
-// split in up to 3 segments by bounds[0..nseg]; column c of segment p only pairs with
-// j in [p*seg_r, p*seg_r + seg_r) and the result goes to dst[p] + (c - bounds[p]) * seg_r + j
-// ("dB" layout [out_p, r]). If seg_r == 0, row j goes to dst[j / rows_per_dst] +
-// (j % rows_per_dst) * C + c ("dA" layout [r, in]). partial: scratch of
-// ceil(T/128) * (seg_r ? seg_r : R) * C floats.
-struct LoraGradArgs {
-  const float* P;
-  int R;
-  const bf16* Q;
-  int64_t ldq;
-  int C;
-  int64_t T;
-  float s;
-  int seg_r;
-  int nseg;
-  int bounds[4];
-  float* dst[4];
-  int rows_per_dst;
-  float* partial;
-};
-cudaError_t lora_grad(const LoraGradArgs& a, cudaStream_t st);
-
-// Build the derived LoRA operands of one fused projection group (nseg segments with own A_p
-// [r, in], B_p [out_p, r] fp32):
-//   Acat32 [R, in], Acat16 [KP, in] (rows >= R zero), BexpT32 [R, out] (segment-masked),
-//   Bexp16 [out, KP] (segment-masked, columns >= R zero), R = nseg * r.
-struct LoraPrepArgs {
-  const float* A[3];
-  const float* B[3];
-  int nseg, r, in;
-  int bounds[4];  // out-row bounds of the segments
-  int KP;
-  float* Acat32;
-  bf16* Acat16;
-  float* BexpT32;
-  bf16* Bexp16;
-};
-cudaError_t lora_prep(const LoraPrepArgs& a, cudaStream_t st);
-
 }  // namespace lst

@@ -246,16 +246,36 @@ def test_cross_entropy_rows():
     assert maxrel(to_np(dl), p / T) < 8e-3
 
 
-def test_lora_project():
-    r = _rng(10)
-    T, din, R = 300, 688, 24
-    X = _bf(r.normal(size=(T, din)))
-    A = r.uniform(-0.05, 0.05, size=(R, din)).astype(np.float32)
-    U = torch.empty(T, R, device="cuda")
+@pytest.mark.parametrize("T,K,b_mn", [(300, 688, 0), (2048, 4096, 0), (2048, 6144, 1), (128, 256, 1)])
+def test_lora_skinny(T, K, b_mn):
+    r = _rng(T + K + b_mn)
+    R = 48
+    X = _bf(r.normal(size=(T, K)))
+    if b_mn:
+        Bop = np.zeros((K, 64), np.float32)
+        Bop[:, :R] = _bf(r.normal(size=(K, R)) * 0.05)
+        ref = 2.0 * X.astype(np.float64) @ Bop.astype(np.float64)
+    else:
+        Bop = np.zeros((64, K), np.float32)
+        Bop[:R] = _bf(r.normal(size=(R, K)) * 0.05)
+        ref = 2.0 * X.astype(np.float64) @ Bop.T.astype(np.float64)
     Us = torch.zeros(T, 64, dtype=torch.bfloat16, device="cuda")
-    lst.k_lora_project(torch_bf16(X), din, T, din, torch_f32(A), R, 2.0, U, Us, 64)
+    scratch = torch.empty(16 * T * 64, dtype=torch.float32, device="cuda")
+    lst.k_lora_skinny(torch_bf16(X), K, T, K, torch_bf16(Bop), 64 if b_mn else K, b_mn, 64, 2.0, Us, scratch)
     torch.cuda.synchronize()
-    ref = X.astype(np.float64) @ A.T.astype(np.float64)
-    assert maxrel(to_np(U), ref) < 1e-5
-    assert maxrel(to_np(Us)[:, :R], 2 * ref) < 8e-3
-    assert np.all(to_np(Us)[:, R:] == 0)
+    got = to_np(Us)
+    assert maxrel(got, ref) < 8e-3
+    assert np.all(got[:, R:] == 0)
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 64, 2048), (300, 64, 200), (6144, 64, 512)])
+def test_gemm_transposed_a(M, N, K):
+    # C = A^T B with A [K, M] and B [K, N] both MN-major: the token reductions of dA / dB
+    r = _rng(M * 7 + K)
+    A = _bf(r.normal(size=(K, M)))
+    B = _bf(r.normal(size=(K, N)))
+    ref = A.T.astype(np.float64) @ B.astype(np.float64)
+    C = torch.zeros(M, N, dtype=torch.float32, device="cuda")
+    lst.k_gemm(M, N, K, torch_bf16(A), M, torch_bf16(B), N, 1, C, N, 1, a_mn=1)
+    torch.cuda.synchronize()
+    assert maxrel(to_np(C), ref) < 1e-4
