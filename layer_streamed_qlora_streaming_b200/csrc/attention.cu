@@ -83,6 +83,38 @@ __device__ __forceinline__ void ldb_trans(uint32_t (&b)[4], const __nv_bfloat16*
   ldsm4t(b, smem_u32(sm + r * Tile<HD>::LD + c));
 }
 
+// Store one accumulator row (C-fragment row r of this thread) of dq or dk scaled by `scale`; with
+// tables given, first apply the inverse rotary embedding of position pos (the transpose of the
+// forward rotation: pairs j, j + hd/2 rotated by minus the angle), so the gradient is rounded once.
+template <int HD>
+__device__ __forceinline__ void store_grad_rows(__nv_bfloat16* dst, const float (&acc)[HD / 8][4], int r, int t4,
+                                                int pos, float scale, const float* cos_t, const float* sin_t) {
+  constexpr int HALF = HD / 2;
+  if (!cos_t) {
+#pragma unroll
+    for (int i = 0; i < HD / 8; ++i) {
+      const int c = i * 8 + 2 * t4;
+      *reinterpret_cast<__nv_bfloat162*>(dst + c) =
+          __floats2bfloat162_rn(acc[i][2 * r] * scale, acc[i][2 * r + 1] * scale);
+    }
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < HD / 16; ++i) {
+    const int c = i * 8 + 2 * t4;  // first-half dimension; its partner is c + HALF (n-tile i + HD/16)
+    float y1[2], y2[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float x1 = acc[i][2 * r + u] * scale, x2 = acc[i + HD / 16][2 * r + u] * scale;
+      const float cs = cos_t[pos * HALF + c + u], sn = sin_t[pos * HALF + c + u];
+      y1[u] = x1 * cs + x2 * sn;
+      y2[u] = x2 * cs - x1 * sn;
+    }
+    *reinterpret_cast<__nv_bfloat162*>(dst + c) = __floats2bfloat162_rn(y1[0], y1[1]);
+    *reinterpret_cast<__nv_bfloat162*>(dst + c + HALF) = __floats2bfloat162_rn(y2[0], y2[1]);
+  }
+}
+
 // ------------------------------------------------------------------------------------ forward
 // grid (ceil(S/64), hq, B), 128 threads; warp w owns query rows 16w..16w+15 of the block.
 template <int HD>
@@ -335,10 +367,9 @@ __global__ void __launch_bounds__(128) k_attn_dkdv(AttnBwdArgs p) {
 #pragma unroll
     for (int i = 0; i < HD / 8; ++i) {
       const int c = i * 8 + 2 * t4;
-      *reinterpret_cast<__nv_bfloat162*>(kp + c) =
-          __floats2bfloat162_rn(dk[i][2 * r] * p.scale, dk[i][2 * r + 1] * p.scale);
       *reinterpret_cast<__nv_bfloat162*>(vp + c) = __floats2bfloat162_rn(dv[i][2 * r], dv[i][2 * r + 1]);
     }
+    store_grad_rows<HD>(kp, dk, r, t4, kr, p.scale, p.rope_cos, p.rope_sin);
   }
 }
 
@@ -430,12 +461,7 @@ __global__ void __launch_bounds__(128) k_attn_dq(AttnBwdArgs p) {
     const int qr = r ? qr1 : qr0;
     if (qr >= p.S) continue;
     __nv_bfloat16* qp = p.dq + (tok0 + qr) * p.lddq + h * HD;
-#pragma unroll
-    for (int i = 0; i < HD / 8; ++i) {
-      const int c = i * 8 + 2 * t4;
-      *reinterpret_cast<__nv_bfloat162*>(qp + c) =
-          __floats2bfloat162_rn(dq[i][2 * r] * p.scale, dq[i][2 * r + 1] * p.scale);
-    }
+    store_grad_rows<HD>(qp, dq, r, t4, qr, p.scale, p.rope_cos, p.rope_sin);
   }
 }
 

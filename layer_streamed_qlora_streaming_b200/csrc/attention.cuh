@@ -34,6 +34,9 @@ struct AttnBwdArgs {
   int64_t T;
   int S, hq, hkv, hd;
   float scale;
+  // optional: undo the rotary embedding on dq and dk before they are stored (tables [S, hd/2])
+  const float* rope_cos = nullptr;
+  const float* rope_sin = nullptr;
 };
 
 cudaError_t attention_fwd(const AttnArgs& a, cudaStream_t s);

@@ -367,6 +367,13 @@ lst_status group_fwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
   a.bias = bias;
   a.R = resid;
   a.ldr = c->d;
+  if (g == G_QKV) {  // rotary embedding of q and k applied in the epilogue (one bf16 rounding)
+    a.rope_cos = c->cos_t;
+    a.rope_sin = c->sin_t;
+    a.rope_end = (int)(c->dq + c->dkv);
+    a.rope_hd = c->hd;
+    a.rope_S = (int)c->curS;
+  }
   ProfScope ps(c, c->stream, PC_GEMM, 2.0 * T * G.out * (double)(G.in + G.KP));
   CK(gemm_bf16(a, c->stream));
   return LST_OK;
@@ -449,11 +456,6 @@ lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
   }
   TRY(group_fwd(c, i, G_QKV, W, c->n1, c->d, c->qkv, c->dqkv, 0, bias, nullptr, true));
   {
-    ProfScope ps(c, c->stream, PC_OTHER);
-    CK(rope(c->qkv, c->dqkv, T, S, 0, c->hq, c->hd, c->cos_t, c->sin_t, 0, c->stream));
-    CK(rope(c->qkv, c->dqkv, T, S, (int)c->dq, c->hkv, c->hd, c->cos_t, c->sin_t, 0, c->stream));
-  }
-  {
     AttnArgs a;
     a.q = c->qkv;
     a.k = c->qkv + c->dq;
@@ -527,13 +529,10 @@ lst_status layer_bwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
     a.hkv = c->hkv;
     a.hd = c->hd;
     a.scale = 1.0f / std::sqrt((float)c->hd);
+    a.rope_cos = c->cos_t;  // dq and dk leave the kernel with the rotary embedding undone
+    a.rope_sin = c->sin_t;
     ProfScope ps(c, c->stream, PC_ATTN);
     CK(attention_bwd(a, c->stream));
-  }
-  {
-    ProfScope ps(c, c->stream, PC_OTHER);
-    CK(rope(c->dqkvb, c->dqkv, T, S, 0, c->hq, c->hd, c->cos_t, c->sin_t, 1, c->stream));
-    CK(rope(c->dqkvb, c->dqkv, T, S, (int)c->dq, c->hkv, c->hd, c->cos_t, c->sin_t, 1, c->stream));
   }
   TRY(group_bwd(c, i, G_QKV, W, c->dqkvb, c->dqkv, c->n1, c->d, c->dn, 1));
   {

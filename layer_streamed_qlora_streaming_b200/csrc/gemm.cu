@@ -29,7 +29,51 @@ struct Epi {
   float alpha;
   int c_f32;
   int M, N;
+  // rotary embedding of output columns [0, rope_end) (whole heads of rope_hd columns)
+  const float* rope_cos;
+  const float* rope_sin;
+  int rope_end, rope_hd, rope_S;
 };
+
+// Rotate the pair of 32-column chunks (na .. na+31) and (nb .. nb+31), nb = na + hd/2, of one row
+// by the angle of position pos (pairs j, j + hd/2 with j = j0 + i), after scale and bias; store
+// bf16. Used for q and k straight out of the projection GEMM, so they are rounded once.
+__device__ __forceinline__ void epi_store_rope(const Epi& e, int row, int na, int nb, int j0,
+                                               const uint32_t (&ra)[32], const uint32_t (&rb)[32]) {
+  if (row >= e.M) return;
+  const int half = e.rope_hd / 2;
+  const int pos = row % e.rope_S;
+  const float* cs = e.rope_cos + (int64_t)pos * half + j0;
+  const float* sn = e.rope_sin + (int64_t)pos * half + j0;
+  __nv_bfloat16* ca = reinterpret_cast<__nv_bfloat16*>(e.C) + (int64_t)row * e.ldc + na;
+  __nv_bfloat16* cb = reinterpret_cast<__nv_bfloat16*>(e.C) + (int64_t)row * e.ldc + nb;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 ua, ub;
+    __nv_bfloat162* ha = reinterpret_cast<__nv_bfloat162*>(&ua);
+    __nv_bfloat162* hb = reinterpret_cast<__nv_bfloat162*>(&ub);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float ya[2], yb[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int k = q * 8 + i + u;
+        float a = __uint_as_float(ra[k]) * e.alpha, b = __uint_as_float(rb[k]) * e.alpha;
+        if (e.bias) {
+          a += e.bias[na + k];
+          b += e.bias[nb + k];
+        }
+        const float c = cs[k], s = sn[k];
+        ya[u] = a * c - b * s;
+        yb[u] = b * c + a * s;
+      }
+      ha[i / 2] = __floats2bfloat162_rn(ya[0], ya[1]);
+      hb[i / 2] = __floats2bfloat162_rn(yb[0], yb[1]);
+    }
+    *reinterpret_cast<uint4*>(ca + q * 8) = ua;
+    *reinterpret_cast<uint4*>(cb + q * 8) = ub;
+  }
+}
 
 template <int BN>
 struct Cfg {
@@ -206,12 +250,28 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     mbar_wait(accf, 0);
     tc_fence_after();
     const int row = m0 + q * 32 + lane;
+    const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+    if (n0 < ep.rope_end) {
+      const int half = ep.rope_hd / 2;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + c, r);
-      tmem_ld_wait();
-      epi_store(ep, row, n0 + c, r);
+      for (int h0 = 0; h0 < BN; h0 += ep.rope_hd) {
+#pragma unroll 1
+        for (int j0 = 0; j0 < half; j0 += 32) {
+          uint32_t ra[32], rb[32];
+          tmem_ld32(tq + h0 + j0, ra);
+          tmem_ld32(tq + h0 + half + j0, rb);
+          tmem_ld_wait();
+          epi_store_rope(ep, row, n0 + h0 + j0, n0 + h0 + half + j0, j0, ra, rb);
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tq + c, r);
+        tmem_ld_wait();
+        epi_store(ep, row, n0 + c, r);
+      }
     }
   }
   tc_fence_before();
@@ -278,7 +338,8 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
     tA2 = tA;
     tB2 = tB;
   }
-  Epi e{a.C, a.ldc, a.bias, a.R, a.ldr, a.alpha, a.c_f32, a.M, a.N};
+  Epi e{a.C, a.ldc, a.bias, a.R, a.ldr, a.alpha, a.c_f32, a.M, a.N,
+        a.rope_cos, a.rope_sin, a.rope_cos ? a.rope_end : 0, a.rope_hd, a.rope_S};
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t err =
@@ -312,6 +373,14 @@ cudaError_t gemm_bf16(const GemmArgs& a, cudaStream_t s) {
   if (a.N <= 64) bn = 64;
   else if (a.N <= 128 || tiles256 < 120) bn = 128;
   else bn = 256;
+  if (a.rope_cos) {
+    // rotated columns: whole tiles of whole heads, bf16 output, no residual / split / MN-major A
+    if (!a.rope_sin || (a.rope_hd != 64 && a.rope_hd != 128) || a.rope_S <= 0 || a.c_f32 || a.R ||
+        a.splits > 1 || a.a_mn || (a.ldc % 8) || (reinterpret_cast<uintptr_t>(a.C) & 15))
+      return cudaErrorInvalidValue;
+    if (bn == 256 && (a.rope_end % 256)) bn = 128;
+    if (bn < 128 || (a.rope_end % bn) || a.rope_end > a.N) return cudaErrorInvalidValue;
+  }
   const int code = bn * 4 + (a.a_mn ? 2 : 0) + (a.b_mn ? 1 : 0);
   switch (code) {
     case 64 * 4 + 0: return launch<64, 0, 0>(a, s);

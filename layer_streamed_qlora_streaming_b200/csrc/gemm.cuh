@@ -38,6 +38,12 @@ struct GemmArgs {
   int a_mn = 0;                       // 1: A is row-major [K, M] (MN-major); needs b_mn = 1
   int splits = 1;                     // split-K: partial results at C + z * split_stride
   int64_t split_stride = 0;
+  // Rotary embedding fused into the epilogue (q and k of a fused q/k/v projection): output
+  // columns [0, rope_end) form heads of rope_hd columns whose pairs (j, j + rope_hd/2) are rotated
+  // by the angle of position (row mod rope_S), tables rope_cos / rope_sin [rope_S, rope_hd/2].
+  const float* rope_cos = nullptr;
+  const float* rope_sin = nullptr;
+  int rope_end = 0, rope_hd = 0, rope_S = 0;
 };
 
 // Returns cudaSuccess or the launch / argument error. Deterministic: no split-K, no atomics.

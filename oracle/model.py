@@ -15,6 +15,16 @@ attention, SwiGLU MLP, residuals) is the reading of "Llama-style" / "Qwen2.5-sha
 LoRA: y = x W^T + s (x A^T) B^T (+ bias for q/k/v where present), s = alpha / r, no dropout.
 
 Every function is the plain definition in fp64. Gradients are returned only for LoRA A and B.
+
+Activation precision. The workloads state bf16 activations ("bf16 acts") with full-precision
+accumulation. ``step(..., bf16_acts=True)`` applies that rule literally: every operand of a matrix
+product that is an activation or an activation gradient is rounded to bf16 (round to nearest even)
+before the product -- the normalised inputs of the projections, q / k (after RoPE) / v, the attention
+output, the SwiGLU inputs and output, the normalised input of the LM head, and in the backward the
+upstream gradients entering a projection and the attention gradients -- while products, sums,
+norms, softmax and the residual stream stay exact (fp64). With ``bf16_acts=False`` nothing is
+rounded. The rounding points are where a bf16-activation computation must round; they are a
+reading of "bf16 acts", not taken from any implementation.
 """
 from __future__ import annotations
 
@@ -183,8 +193,17 @@ def unpack_blob(blob: dict) -> dict:
 # decoder layer
 # ------------------------------------------------------------------------------------------
 
+def _identity(x):
+    return x
+
+
+def _round_bf16(x):
+    return nf4.bf16_value(np.asarray(x, dtype=np.float32)).astype(F64)
+
+
 class Shape:
-    def __init__(self, wl):
+    def __init__(self, wl, bf16_acts: bool = False):
+        self.rb = _round_bf16 if bf16_acts else _identity
         self.batch, self.seq = wl.batch, wl.seq
         self.hq, self.hkv, self.hd = wl.n_heads, wl.n_kv_heads, wl.head_dim
         self.eps, self.theta = wl.rms_eps, wl.rope_theta
@@ -196,23 +215,27 @@ def layer_fwd(x, Wt, lora, sh: Shape):
     """One pre-norm decoder layer. Wt: unpacked weights; lora: {proj: (A, B)} fp64.
     Returns (x_out, cache) where cache holds what the backward needs."""
     T = x.shape[0]
+    rb = sh.rb
     bias = Wt["bias"] or {}
     n1, r1 = rmsnorm(x, Wt["attn_norm"], sh.eps)
+    n1 = rb(n1)
     c = {"x": x, "n1": n1, "r1": r1}
     for p in ("q", "k", "v"):
         y, u = lora_linear(n1, Wt["W"][p], *lora[p], sh.s, bias.get(p))
         c[p + "_pre"], c["u_" + p] = y, u
-    q = rope(c["q_pre"].reshape(T, sh.hq, sh.hd), sh.cos, sh.sin, sh.batch, sh.seq)
-    k = rope(c["k_pre"].reshape(T, sh.hkv, sh.hd), sh.cos, sh.sin, sh.batch, sh.seq)
-    v = c["v_pre"].reshape(T, sh.hkv, sh.hd)
+    q = rb(rope(c["q_pre"].reshape(T, sh.hq, sh.hd), sh.cos, sh.sin, sh.batch, sh.seq))
+    k = rb(rope(c["k_pre"].reshape(T, sh.hkv, sh.hd), sh.cos, sh.sin, sh.batch, sh.seq))
+    v = rb(c["v_pre"].reshape(T, sh.hkv, sh.hd))
     o, P = attention(q, k, v, sh.batch, sh.seq)
-    c.update(q=q, k=k, v=v, P=P, o=o.reshape(T, -1))
+    c.update(q=q, k=k, v=v, P=P, o=rb(o.reshape(T, -1)))
     ao, c["u_o"] = lora_linear(c["o"], Wt["W"]["o"], *lora["o"], sh.s)
     h = x + ao
     n2, r2 = rmsnorm(h, Wt["mlp_norm"], sh.eps)
+    n2 = rb(n2)
     g, c["u_gate"] = lora_linear(n2, Wt["W"]["gate"], *lora["gate"], sh.s)
     u, c["u_up"] = lora_linear(n2, Wt["W"]["up"], *lora["up"], sh.s)
-    m = silu(g) * u
+    g, u = rb(g), rb(u)
+    m = rb(silu(g) * u)
     dn, c["u_down"] = lora_linear(m, Wt["W"]["down"], *lora["down"], sh.s)
     c.update(h=h, n2=n2, r2=r2, g=g, up=u, m=m)
     return h + dn, c
@@ -221,20 +244,21 @@ def layer_fwd(x, Wt, lora, sh: Shape):
 def layer_bwd(dout, c, Wt, lora, sh: Shape):
     """Backward of ``layer_fwd``: returns (dx, {proj: (dA, dB)})."""
     T = dout.shape[0]
+    rb = sh.rb
     grads = {}
-    dm, grads["down"] = _lin_bwd(dout, c["m"], c["u_down"], Wt["W"]["down"], lora["down"], sh.s)
+    dm, grads["down"] = _lin_bwd(rb(dout), c["m"], c["u_down"], Wt["W"]["down"], lora["down"], sh.s)
     sg = 1.0 / (1.0 + np.exp(-c["g"]))
-    dg = dm * c["up"] * sg * (1.0 + c["g"] * (1.0 - sg))
-    du = dm * c["g"] * sg
+    dg = rb(dm * c["up"] * sg * (1.0 + c["g"] * (1.0 - sg)))
+    du = rb(dm * c["g"] * sg)
     dn2_g, grads["gate"] = _lin_bwd(dg, c["n2"], c["u_gate"], Wt["W"]["gate"], lora["gate"], sh.s)
     dn2_u, grads["up"] = _lin_bwd(du, c["n2"], c["u_up"], Wt["W"]["up"], lora["up"], sh.s)
     dh = dout + rmsnorm_bwd(dn2_g + dn2_u, c["h"], Wt["mlp_norm"], c["r2"])
-    do, grads["o"] = _lin_bwd(dh, c["o"], c["u_o"], Wt["W"]["o"], lora["o"], sh.s)
-    dq, dk, dv = attention_bwd(do.reshape(T, sh.hq, sh.hd), c["q"], c["k"], c["v"], c["P"],
+    do, grads["o"] = _lin_bwd(rb(dh), c["o"], c["u_o"], Wt["W"]["o"], lora["o"], sh.s)
+    dq, dk, dv = attention_bwd(rb(do).reshape(T, sh.hq, sh.hd), c["q"], c["k"], c["v"], c["P"],
                                sh.batch, sh.seq)
-    dq = rope_bwd(dq, sh.cos, sh.sin, sh.batch, sh.seq).reshape(T, -1)
-    dk = rope_bwd(dk, sh.cos, sh.sin, sh.batch, sh.seq).reshape(T, -1)
-    dv = dv.reshape(T, -1)
+    dq = rb(rope_bwd(dq, sh.cos, sh.sin, sh.batch, sh.seq).reshape(T, -1))
+    dk = rb(rope_bwd(dk, sh.cos, sh.sin, sh.batch, sh.seq).reshape(T, -1))
+    dv = rb(dv.reshape(T, -1))
     dn1 = 0.0
     for p, dy in (("q", dq), ("k", dk), ("v", dv)):
         dxp, grads[p] = _lin_bwd(dy, c["n1"], c["u_" + p], Wt["W"][p], lora[p], sh.s)
@@ -252,9 +276,10 @@ def _lin_bwd(dy, x, u, W, AB, s):
 # head: final norm, resident LM head, cross-entropy
 # ------------------------------------------------------------------------------------------
 
-def head_fwd(x, gf, H, targets, eps):
+def head_fwd(x, gf, H, targets, eps, rb=_identity):
     """logits = rmsnorm(x) H^T; loss = mean_t(logsumexp(logits_t) - logits_t[target_t])."""
     n, r = rmsnorm(x, gf, eps)
+    n = rb(n)
     logits = n @ H.T
     mx = logits.max(axis=1, keepdims=True)
     lse = (mx + np.log(np.exp(logits - mx).sum(axis=1, keepdims=True)))[:, 0]
@@ -263,14 +288,14 @@ def head_fwd(x, gf, H, targets, eps):
     return loss, logits, (x, n, r, lse)
 
 
-def head_bwd(cache, logits, gf, H, targets):
+def head_bwd(cache, logits, gf, H, targets, rb=_identity):
     """dL/dx of ``head_fwd``: dlogits = (softmax - onehot) / T, dn = dlogits H."""
     x, n, r, lse = cache
     T = x.shape[0]
     dlog = np.exp(logits - lse[:, None])
     dlog[np.arange(T), targets] -= 1.0
     dlog /= T
-    return rmsnorm_bwd(dlog @ H, x, gf, r)
+    return rmsnorm_bwd(rb(dlog) @ H, x, gf, r)
 
 
 # ------------------------------------------------------------------------------------------
@@ -282,7 +307,7 @@ def _lora64(raw):
 
 
 def step(wl, raw_layers, blobs=None, head=None, tokens=None, targets=None, x_in=None, G=None,
-         schedule="resident", lora=None):
+         schedule="resident", lora=None, bf16_acts=False):
     """Loss and LoRA gradients of one step.
 
     raw_layers: per layer the synthetic dict (only A/B are read here; base comes from ``blobs``).
@@ -291,10 +316,11 @@ def step(wl, raw_layers, blobs=None, head=None, tokens=None, targets=None, x_in=
     schedule: "resident" (all layers unpacked once, activations of every layer kept) or
       "streamed" (2L reads through two buffers: forward keeps only each layer's input, backward
       copies the layer again and recomputes it).
+    bf16_acts: round matrix-product operands that are activations to bf16 (see module doc).
     Returns dict(loss, grads[layer][proj] = (dA, dB), logits or None, reads).
     """
     L = wl.n_layers
-    sh = Shape(wl)
+    sh = Shape(wl, bf16_acts)
     if blobs is None:
         blobs = [pack_layer(raw_layers[i], wl.base_format) for i in range(L)]
     if lora is None:
@@ -325,8 +351,8 @@ def step(wl, raw_layers, blobs=None, head=None, tokens=None, targets=None, x_in=
 
     logits = None
     if head is not None:
-        loss, logits, hc = head_fwd(x, gf, H, targets, wl.rms_eps)
-        dx = head_bwd(hc, logits, gf, H, targets)
+        loss, logits, hc = head_fwd(x, gf, H, targets, wl.rms_eps, sh.rb)
+        dx = head_bwd(hc, logits, gf, H, targets, sh.rb)
     else:
         Gf = G.astype(F64)
         loss = float(np.sum(x * Gf))

@@ -5,11 +5,15 @@ import numpy as np
 
 import synthetic as syn
 
-# tolerances of the parity criteria (loss / logits relative; gradients cosine and max-rel)
+# Tolerances of the parity criteria against the oracle with bf16 activations (the workloads'
+# stated precision): loss relative, logits max|d| / max|ref|, gradients cosine and max-rel.
 LOSS_RTOL = 1e-2
 LOGITS_MAXREL = 1e-2
 GRAD_COS = 0.999
 GRAD_MAXREL = 2e-2
+# Against the exact (unrounded fp64) oracle the difference is the rounding noise of bf16 operands
+# (unit roundoff 2^-8, amplified by softmax and products); bound the logits at 3x the above.
+EXACT_LOGITS_MAXREL = 3e-2
 
 
 def cosine(a, b) -> float:
@@ -82,9 +86,9 @@ def run_step(ctx, wl, inp: dict, want_logits: bool = True):
     return loss, grads, None
 
 
-def oracle_step(wl, inp: dict, schedule: str = "streamed"):
+def oracle_step(wl, inp: dict, schedule: str = "streamed", bf16_acts: bool = True):
     from oracle import model as M
-    kw = dict(raw_layers=inp["raw"], schedule=schedule)
+    kw = dict(raw_layers=inp["raw"], schedule=schedule, bf16_acts=bf16_acts)
     if wl.vocab:
         kw.update(head=inp["head"], tokens=inp["tokens"], targets=inp["targets"])
     else:

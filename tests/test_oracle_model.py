@@ -210,3 +210,21 @@ def test_input_gradient_matches_finite_differences_headless():
             vals.append(M.step(wl, **{**inp, "x_in": x})["loss"])
         fd = (vals[0] - vals[1]) / (2 * h)
         assert abs(fd - ref["dx_in"][t, c]) <= 1e-6 * np.abs(ref["dx_in"]).max() + 1e-9
+
+
+def test_bf16_rounding_matches_torch_and_bf16_mode_is_consistent():
+    import torch
+    rng = np.random.default_rng(11)
+    x = np.concatenate([rng.normal(size=10000), rng.normal(size=1000) * 1e-30,
+                        np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -2.5, 0.0])]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()   # library routine
+    assert np.array_equal(nf4.bf16_value(x), ref)
+    # bf16 mode: streamed == resident bitwise, and close to the exact mode
+    wl = tiny(n_layers=2)
+    inp = build(wl)
+    a = M.step(wl, schedule="resident", bf16_acts=True, **inp)
+    b = M.step(wl, schedule="streamed", bf16_acts=True, **inp)
+    e = M.step(wl, schedule="resident", bf16_acts=False, **inp)
+    assert a["loss"] == b["loss"]
+    assert abs(a["loss"] - e["loss"]) < 1e-3 * abs(e["loss"])
+    assert a["loss"] != e["loss"]          # the rounding is really applied
