@@ -237,6 +237,12 @@ __global__ void __launch_bounds__(128) k_attn_fwd(AttnArgs p) {
       const int c = i * 8 + 2 * t4;
       *reinterpret_cast<__nv_bfloat162*>(op + c) = __floats2bfloat162_rn(o[i][2 * r] * inv, o[i][2 * r + 1] * inv);
     }
+    if (p.o32) {  // unrounded output for the backward's D = rowsum(dO * O)
+      float* o32 = p.o32 + (tok0 + qr) * (int64_t)p.hq * HD + h * HD;
+#pragma unroll
+      for (int i = 0; i < HD / 8; ++i)
+        *reinterpret_cast<float2*>(o32 + i * 8 + 2 * t4) = make_float2(o[i][2 * r] * inv, o[i][2 * r + 1] * inv);
+    }
     if (t4 == 0) p.lse[(tok0 + qr) * p.hq + h] = (mrow[r] + log2f(lrow[r])) / kLog2e;
   }
 }
@@ -249,9 +255,14 @@ __global__ void k_attn_D(AttnBwdArgs p) {
   const int64_t t = idx / p.hq;
   const int h = (int)(idx % p.hq);
   const __nv_bfloat16* a = p.dout + t * p.lddo + (int64_t)h * p.hd;
-  const __nv_bfloat16* o = p.o + t * p.ldo + (int64_t)h * p.hd;
   float s = 0.f;
-  for (int c = l; c < p.hd; c += 32) s += __bfloat162float(a[c]) * __bfloat162float(o[c]);
+  if (p.o32) {  // the forward's unrounded output: D then matches the normalisation of P exactly
+    const float* o = p.o32 + t * (int64_t)p.hq * p.hd + (int64_t)h * p.hd;
+    for (int c = l; c < p.hd; c += 32) s += __bfloat162float(a[c]) * o[c];
+  } else {
+    const __nv_bfloat16* o = p.o + t * p.ldo + (int64_t)h * p.hd;
+    for (int c = l; c < p.hd; c += 32) s += __bfloat162float(a[c]) * __bfloat162float(o[c]);
+  }
   s = warp_sum(s);
   if (l == 0) p.D[idx] = s;
 }

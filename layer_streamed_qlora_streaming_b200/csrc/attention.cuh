@@ -13,6 +13,7 @@ struct AttnArgs {
   const __nv_bfloat16* v;  // [T, ldv]
   __nv_bfloat16* o;        // [T, ldo]
   float* lse;              // [T, hq] natural-log sum-exp of the scaled scores
+  float* o32 = nullptr;    // optional [T, hq*hd] fp32 copy of o before rounding (for the backward)
   int64_t ldq, ldk, ldv, ldo;
   int64_t T;               // batch * S tokens
   int S, hq, hkv, hd;      // hd in {64, 128}
@@ -34,6 +35,7 @@ struct AttnBwdArgs {
   int64_t T;
   int S, hq, hkv, hd;
   float scale;
+  const float* o32 = nullptr;  // optional fp32 forward output [T, hq*hd]; D uses it when given
   // optional: undo the rotary embedding on dq and dk before they are stored (tables [S, hd/2])
   const float* rope_cos = nullptr;
   const float* rope_sin = nullptr;

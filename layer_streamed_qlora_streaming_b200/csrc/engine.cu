@@ -199,6 +199,7 @@ struct lst_ctx {
   __nv_bfloat16 *n1 = nullptr, *qkv = nullptr, *o = nullptr, *n2 = nullptr, *gu = nullptr, *m = nullptr,
                 *wscr = nullptr;
   float *rstd1 = nullptr, *rstd2 = nullptr, *lse = nullptr, *Dbuf = nullptr;
+  float* o32 = nullptr;  // attention output before rounding (recompute pass), for the backward's D
   __nv_bfloat16* Us[NGROUP] = {};  // bf16(s * x A^T) per group [T, KP]
   __nv_bfloat16* Vs[NGROUP] = {};  // bf16(s * dy B) per group [T, KP]
   float *ga = nullptr, *gb = nullptr, *dn = nullptr, *dm = nullptr, *part = nullptr;
@@ -462,6 +463,7 @@ lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
     a.v = c->qkv + c->dq + c->dkv;
     a.o = c->o;
     a.lse = c->lse;
+    a.o32 = c->o32;
     a.ldq = a.ldk = a.ldv = c->dqkv;
     a.ldo = c->dq;
     a.T = T;
@@ -515,6 +517,7 @@ lst_status layer_bwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
     a.o = c->o;
     a.dout = c->do_b;
     a.lse = c->lse;
+    a.o32 = c->o32;
     a.D = c->Dbuf;
     a.dq = c->dqkvb;
     a.dk = c->dqkvb + c->dq;
@@ -851,6 +854,7 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   TRY(dalloc(c, &c->rstd1, T));
   TRY(dalloc(c, &c->rstd2, T));
   TRY(dalloc(c, &c->lse, T * c->hq));
+  TRY(dalloc(c, &c->o32, T * c->dq));
   TRY(dalloc(c, &c->Dbuf, T * c->hq));
   int64_t part = 0;
   for (int g = 0; g < NGROUP; ++g) {

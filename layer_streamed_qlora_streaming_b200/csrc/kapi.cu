@@ -90,7 +90,7 @@ lst_status lst_k_attention_fwd(const uint16_t* q, int64_t ldq, const uint16_t* k
                                int64_t ldv, uint16_t* o, int64_t ldo, float* lse, int64_t T, int32_t Sq, int32_t hq,
                                int32_t hkv, int32_t hd, void* stream) {
   if (!q || !k || !v || !o || !lse) return LST_ERR_ARG;
-  AttnArgs a{B16(q), B16(k), B16(v), B16(o), lse, ldq, ldk, ldv, ldo, T, Sq, hq, hkv, hd, 0.f};
+  AttnArgs a{B16(q), B16(k), B16(v), B16(o), lse, nullptr, ldq, ldk, ldv, ldo, T, Sq, hq, hkv, hd, 0.f};
   a.scale = 1.0f / sqrtf((float)hd);
   return st(attention_fwd(a, S(stream)));
 }
