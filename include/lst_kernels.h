@@ -23,6 +23,23 @@ extern "C" {
 lst_status lst_k_nf4_quantize(const float* w, int64_t n, uint8_t* packed, int8_t* qabs,
                               float* gscale, float* mean, void* stream);
 
+/* Same result as lst_k_nf4_quantize, for callers that cannot allocate device memory: code whose
+ * GPU memory is all reserved by its own caching allocator, or code that must not trigger the
+ * device-wide synchronisation of cudaMalloc / cudaFree while other streams run. The pages have no
+ * counterpart of this entry point; it is an interface variant of this library.
+ *  - Scratch comes from one fixed device array inside the library (4 MiB + 32 KiB), present on
+ *    every GPU that loads the library until the process exits. It allocates nothing and calls no
+ *    allocating routine.
+ *  - n is limited to 67,108,864 elements (1 << 26); larger n returns LST_ERR_ARG and launches
+ *    nothing, as does n not a multiple of 64 or a null pointer.
+ *  - The first call on a device (which must be the current device) looks up the array's device
+ *    address once (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Asynchronous on `stream`. All calls share the one array, which keeps the last call's
+ *    contents (nothing in it needs clearing: it is fully rewritten before being read), so calls
+ *    whose work overlaps on the GPU (other streams, other threads) race on it: order them. */
+lst_status lst_k_nf4_quantize_noalloc(const float* w, int64_t n, uint8_t* packed, int8_t* qabs,
+                                      float* gscale, float* mean, void* stream);
+
 /* Dequantise one NF4 tensor into bf16 [n]: a^ = (q * s) / 127 + mean, w^ = bf16(code * a^),
  * each operation one fp32 rounding; bit-exact by construction. */
 lst_status lst_k_nf4_dequant(const uint8_t* packed, const int8_t* qabs, const float* gscale,

@@ -70,6 +70,7 @@ _SIGS = {
     "lst_nf4_codebook": (_I32, [C.POINTER(C.c_float)]),
     "lst_blob_bytes": (_I64, [C.POINTER(Config)]),
     "lst_k_nf4_quantize": (_I32, [_P, _I64, _P, _P, _P, _P, _P]),
+    "lst_k_nf4_quantize_noalloc": (_I32, [_P, _I64, _P, _P, _P, _P, _P]),
     "lst_k_nf4_dequant": (_I32, [_P, _P, _P, _P, _I64, _P, _P]),
     "lst_k_gemm": (_I32, [_I32, _I32, _I32, _P, _I64, _I32, _P, _I64, _I32, _P, _I64, _P, _I64, _I32,
                           _P, _I64, _I32, _F32, _P, _P, _I64, _P]),
@@ -252,6 +253,13 @@ class Context:
 def k_nf4_quantize(w, packed, qabs, gscale, mean, stream=None):
     _check(lib().lst_k_nf4_quantize(_ptr(w), w.numel(), _ptr(packed), _ptr(qabs), _ptr(gscale),
                                     _ptr(mean), _stream(stream)), what="lst_k_nf4_quantize")
+
+
+def k_nf4_quantize_noalloc(w, packed, qabs, gscale, mean, n=None, stream=None):
+    """NF4 quantisation with the library's fixed scratch array (no device allocation)."""
+    _check(lib().lst_k_nf4_quantize_noalloc(_ptr(w), w.numel() if n is None else n, _ptr(packed), _ptr(qabs),
+                                            _ptr(gscale), _ptr(mean), _stream(stream)),
+           what="lst_k_nf4_quantize_noalloc")
 
 
 def k_nf4_dequant(packed, qabs, gscale, mean, n, out, stream=None):
