@@ -81,7 +81,7 @@ struct Cfg {
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t SMEM = STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*bars*/;
-  static constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;
+  static constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;  // one accumulator; two are allocated
 };
 
 __device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const uint32_t (&r)[32]) {
@@ -139,14 +139,37 @@ __device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const
   }
 }
 
+// Tile order: groups of kGroupM M-tiles; inside a group the M-tile index runs fastest, so the
+// CTAs working at the same time share a few weight (B) tiles and the group's activation rows in
+// L2. Split-K slices (z) are the slowest index.
+constexpr int kGroupM = 8;
+
+struct TileSched {
+  int mt, nt, tiles_per_z;
+  __device__ __forceinline__ void get(int t, int& m, int& n, int& z) const {
+    z = t / tiles_per_z;
+    const int r = t - z * tiles_per_z;
+    const int per_group = kGroupM * nt;
+    const int g = r / per_group;
+    const int first = g * kGroupM;
+    const int gsz = min(kGroupM, mt - first);
+    const int q = r - g * per_group;
+    m = first + q % gsz;
+    n = q / gsz;
+  }
+};
+
+// Persistent tcgen05 GEMM. Each CTA loops over tiles t = blockIdx.x, + gridDim.x, ... and keeps
+// two fp32 accumulators in TMEM, so the epilogue of one tile overlaps the main loop of the next.
 // AMN / BMN: A / B operand MN-major (row-major [K, M] / [K, N] in global memory), else K-major.
-// Split-K: blockIdx.z takes main k-blocks [z * kps, (z + 1) * kps) and writes its partial result
-// at C + z * split_stride (the second operand pair is only allowed without split).
+// Split-K: slice z takes main k-blocks [z * kps, (z + 1) * kps) and writes its partial result at
+// C + z * split_stride (the second operand pair is only allowed without split).
 template <int BN, int AMN, int BMN>
 __global__ void __launch_bounds__(192, 1)
 k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
        const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-       Epi ep, const int nk1_total, const int nk2, const int kps, const int64_t split_stride) {
+       const Epi ep0, const TileSched sched, const int total_tiles, const int nk1_total, const int nk2,
+       const int kps, const int64_t split_stride) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -154,27 +177,22 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* accf = empty + C::STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* acc_full = empty + C::STAGES;   // [2] accumulator ready for the epilogue
+  uint64_t* acc_empty = acc_full + 2;       // [2] accumulator drained by the epilogue
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM;
-  const int n0 = blockIdx.x * BN;
-  const int kb0 = blockIdx.z * kps;
-  const int nk1 = min(nk1_total - kb0, kps);
-  const int nk = nk1 + nk2;
-  if (blockIdx.z) {
-    ep.C = ep.c_f32 ? static_cast<void*>(static_cast<float*>(ep.C) + blockIdx.z * split_stride)
-                    : static_cast<void*>(static_cast<__nv_bfloat16*>(ep.C) + blockIdx.z * split_stride);
-  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accf, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -186,7 +204,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_alloc(tmem_slot, 2 * C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -196,89 +214,131 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % C::STAGES;
-        const uint32_t ph = (kb / C::STAGES) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1)) break;
-        mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
-        const bool second = kb >= nk1;
-        const CUtensorMap* ma = second ? &tmA2 : &tmA;
-        const CUtensorMap* mb = second ? &tmB2 : &tmB;
-        const int kk = (second ? kb - nk1 : kb0 + kb) * BK;
-        if (AMN == 0) {
-          tma_load_2d(sA + s * C::A_BYTES, ma, &full[s], kk, m0);
-        } else {
+      uint32_t it = 0;  // stage counter across tiles
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        int mi, ni, z;
+        sched.get(t, mi, ni, z);
+        const int m0 = mi * BM, n0 = ni * BN, kb0 = z * kps;
+        const int nk1 = min(nk1_total - kb0, kps);
+        const int nk = nk1 + nk2;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
+          const bool second = kb >= nk1;
+          const CUtensorMap* ma = second ? &tmA2 : &tmA;
+          const CUtensorMap* mb = second ? &tmB2 : &tmB;
+          const int kk = (second ? kb - nk1 : kb0 + kb) * BK;
+          if (AMN == 0) {
+            tma_load_2d(sA + s * C::A_BYTES, ma, &full[s], kk, m0);
+          } else {
 #pragma unroll
-          for (int c = 0; c < BM / 64; ++c)
-            tma_load_2d(sA + s * C::A_BYTES + c * (64 * BK * 2), ma, &full[s], m0 + c * 64, kk);
-        }
-        if (BMN == 0) {
-          tma_load_2d(sB + s * C::B_BYTES, mb, &full[s], kk, n0);
-        } else {
+            for (int c = 0; c < BM / 64; ++c)
+              tma_load_2d(sA + s * C::A_BYTES + c * (64 * BK * 2), ma, &full[s], m0 + c * 64, kk);
+          }
+          if (BMN == 0) {
+            tma_load_2d(sB + s * C::B_BYTES, mb, &full[s], kk, n0);
+          } else {
 #pragma unroll
-          for (int c = 0; c < BN / 64; ++c)
-            tma_load_2d(sB + s * C::B_BYTES + c * (64 * BK * 2), mb, &full[s], n0 + c * 64, kk);
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(sB + s * C::B_BYTES + c * (64 * BK * 2), mb, &full[s], n0 + c * 64, kk);
+          }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_bf16(BM, BN, AMN, BMN);
+      uint32_t it = 0;
       bool ok = true;
-      for (int kb = 0; kb < nk && ok; ++kb) {
-        const int s = kb % C::STAGES;
-        const uint32_t ph = (kb / C::STAGES) & 1;
-        ok = mbar_wait(&full[s], ph);
-        if (!ok) break;
+      int local = 0;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++local) {
+        int mi, ni, z;
+        sched.get(t, mi, ni, z);
+        const int nk = min(nk1_total - z * kps, kps) + nk2;
+        const int buf = local & 1;
+        const uint32_t use = (uint32_t)(local >> 1);
+        // the epilogue must have drained this accumulator (its use two tiles ago)
+        if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + s * C::A_BYTES);
-        const uint32_t b0 = smem_u32(sB + s * C::B_BYTES);
+        const uint32_t dacc = tmem + (uint32_t)(buf * C::TMEM_COLS);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          if (!mbar_wait(&full[s], ph)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * C::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + s * C::B_BYTES);
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k) {
-          const uint64_t da = AMN ? umma_desc(a0 + k * 16 * 128, 64 * BK * 2, 1024)
-                                  : umma_desc(a0 + k * 32, 16, 1024);
-          const uint64_t db = BMN ? umma_desc(b0 + k * 16 * 128, 64 * BK * 2, 1024)
-                                  : umma_desc(b0 + k * 32, 16, 1024);
-          umma_bf16(tmem, da, db, idesc, (kb | k) != 0);
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t da = AMN ? umma_desc(a0 + k * 16 * 128, 64 * BK * 2, 1024)
+                                    : umma_desc(a0 + k * 32, 16, 1024);
+            const uint64_t db = BMN ? umma_desc(b0 + k * 16 * 128, 64 * BK * 2, 1024)
+                                    : umma_desc(b0 + k * 32, 16, 1024);
+            umma_bf16(dacc, da, db, idesc, (kb | k) != 0);
+          }
+          umma_commit(&empty[s]);
         }
-        umma_commit(&empty[s]);
+        umma_commit(&acc_full[buf]);
       }
-      umma_commit(accf);
     }
   } else {
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    mbar_wait(accf, 0);
-    tc_fence_after();
-    const int row = m0 + q * 32 + lane;
-    const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
-    if (n0 < ep.rope_end) {
-      const int half = ep.rope_hd / 2;
+    int local = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
+      int mi, ni, z;
+      sched.get(t, mi, ni, z);
+      const int m0 = mi * BM, n0 = ni * BN;
+      Epi ep = ep0;
+      if (z) {
+        ep.C = ep.c_f32 ? static_cast<void*>(static_cast<float*>(ep.C) + z * split_stride)
+                        : static_cast<void*>(static_cast<__nv_bfloat16*>(ep.C) + z * split_stride);
+      }
+      const int buf = local & 1;
+      const uint32_t use = (uint32_t)(local >> 1);
+      if (!mbar_wait(&acc_full[buf], use & 1)) break;
+      tc_fence_after();
+      const int row = m0 + q * 32 + lane;
+      const uint32_t tq = tmem + (uint32_t)(buf * C::TMEM_COLS) + ((uint32_t)(q * 32) << 16);
+      if (n0 < ep.rope_end) {
+        const int half = ep.rope_hd / 2;
 #pragma unroll 1
-      for (int h0 = 0; h0 < BN; h0 += ep.rope_hd) {
+        for (int h0 = 0; h0 < BN; h0 += ep.rope_hd) {
 #pragma unroll 1
-        for (int j0 = 0; j0 < half; j0 += 32) {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(tq + h0 + j0, ra);
-          tmem_ld32(tq + h0 + half + j0, rb);
+          for (int j0 = 0; j0 < half; j0 += 32) {
+            uint32_t ra[32], rb[32];
+            tmem_ld32(tq + h0 + j0, ra);
+            tmem_ld32(tq + h0 + half + j0, rb);
+            tmem_ld_wait();
+            epi_store_rope(ep, row, n0 + h0 + j0, n0 + h0 + half + j0, j0, ra, rb);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tq + c, r);
           tmem_ld_wait();
-          epi_store_rope(ep, row, n0 + h0 + j0, n0 + h0 + half + j0, j0, ra, rb);
+          epi_store(ep, row, n0 + c, r);
         }
       }
-    } else {
-#pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tq + c, r);
-        tmem_ld_wait();
-        epi_store(ep, row, n0 + c, r);
-      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);  // all 128 epilogue threads arrive once per tile
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc(tmem, 2 * C::TMEM_COLS);
   }
 }
 
@@ -353,8 +413,20 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   const int kps = (nk1 + splits - 1) / splits;
   splits = (nk1 + kps - 1) / kps;  // no empty split
   if (splits > 1 && a.split_stride < (int64_t)a.M * a.ldc) return cudaErrorInvalidValue;
-  dim3 grid((a.N + BN - 1) / BN, (a.M + BM - 1) / BM, splits);
-  k_gemm<BN, AMN, BMN><<<grid, 192, C::SMEM, s>>>(tA, tB, tA2, tB2, e, nk1, nk2, kps, a.split_stride);
+  TileSched sched;
+  sched.mt = (a.M + BM - 1) / BM;
+  sched.nt = (a.N + BN - 1) / BN;
+  sched.tiles_per_z = sched.mt * sched.nt;
+  const int total = sched.tiles_per_z * splits;
+  static int num_sms = 0;
+  if (!num_sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || num_sms <= 0)
+      num_sms = 148;
+  }
+  const int grid = total < num_sms ? total : num_sms;
+  k_gemm<BN, AMN, BMN><<<grid, 192, C::SMEM, s>>>(tA, tB, tA2, tB2, e, sched, total, nk1, nk2, kps, a.split_stride);
   note_launch(1);
   return cudaGetLastError();
 }

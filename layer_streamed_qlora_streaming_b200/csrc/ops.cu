@@ -71,14 +71,32 @@ __global__ void k_rmsnorm_bwd(const float* __restrict__ dy, const float* __restr
   const float* dyr = dy + row * d;
   const float* xr = x + row * d;
   float dot = 0.f;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) dot += dyr[c] * g[c] * (xr[c] * r);
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    const float4 a = *reinterpret_cast<const float4*>(dyr + c);
+    const float4 b = *reinterpret_cast<const float4*>(xr + c);
+    dot += a.x * g[c] * (b.x * r);
+    dot += a.y * g[c + 1] * (b.y * r);
+    dot += a.z * g[c + 2] * (b.z * r);
+    dot += a.w * g[c + 3] * (b.w * r);
+  }
   dot = block_sum(dot, red) / (float)d;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    const float xh = xr[c] * r;
-    float v = r * (dyr[c] * g[c] - xh * dot);
-    if (dres) v += dres[row * d + c];
-    dx[row * d + c] = v;
-    if (dxb) dxb[row * d + c] = __float2bfloat16_rn(v);
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    const float4 a = *reinterpret_cast<const float4*>(dyr + c);
+    const float4 b = *reinterpret_cast<const float4*>(xr + c);
+    float v[4] = {r * (a.x * g[c] - b.x * r * dot), r * (a.y * g[c + 1] - b.y * r * dot),
+                  r * (a.z * g[c + 2] - b.z * r * dot), r * (a.w * g[c + 3] - b.w * r * dot)};
+    if (dres) {
+      const float4 q = *reinterpret_cast<const float4*>(dres + row * d + c);
+      v[0] += q.x;
+      v[1] += q.y;
+      v[2] += q.z;
+      v[3] += q.w;
+    }
+    *reinterpret_cast<float4*>(dx + row * d + c) = make_float4(v[0], v[1], v[2], v[3]);
+    if (dxb) {
+      __nv_bfloat162 h[2] = {__floats2bfloat162_rn(v[0], v[1]), __floats2bfloat162_rn(v[2], v[3])};
+      *reinterpret_cast<uint2*>(dxb + row * d + c) = *reinterpret_cast<const uint2*>(h);
+    }
   }
 }
 
@@ -118,29 +136,66 @@ __global__ void k_rope_tables(int S, int hd, double theta, float* ct, float* st)
 }
 
 // ------------------------------------------------------------------------------- SwiGLU
+// 8 consecutive elements per thread (16-byte loads and stores); F is a multiple of 8.
 __global__ void k_swiglu_fwd(const bf16* __restrict__ gu, int64_t T, int F, bf16* __restrict__ m) {
+  const int f8 = F / 8;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= T * F) return;
-  const int64_t t = i / F;
-  const int j = (int)(i % F);
-  const float g = __bfloat162float(gu[t * 2 * F + j]);
-  const float u = __bfloat162float(gu[t * 2 * F + F + j]);
-  const float sg = 1.0f / (1.0f + expf(-g));
-  m[i] = __float2bfloat16_rn(g * sg * u);
+  if (i >= T * f8) return;
+  const int64_t t = i / f8;
+  const int j = (int)(i % f8) * 8;
+  const uint4 gv = *reinterpret_cast<const uint4*>(gu + t * 2 * F + j);
+  const uint4 uv = *reinterpret_cast<const uint4*>(gu + t * 2 * F + F + j);
+  const bf16* g8 = reinterpret_cast<const bf16*>(&gv);
+  const bf16* u8 = reinterpret_cast<const bf16*>(&uv);
+  uint4 o;
+  __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float r[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float g = __bfloat162float(g8[2 * e + k]), u = __bfloat162float(u8[2 * e + k]);
+      const float sg = 1.0f / (1.0f + expf(-g));
+      r[k] = g * sg * u;
+    }
+    o2[e] = __floats2bfloat162_rn(r[0], r[1]);
+  }
+  *reinterpret_cast<uint4*>(m + t * F + j) = o;
 }
 
 __global__ void k_swiglu_bwd(const float* __restrict__ dm, const bf16* __restrict__ gu, int64_t T, int F,
                              bf16* __restrict__ dgu) {
+  const int f8 = F / 8;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= T * F) return;
-  const int64_t t = i / F;
-  const int j = (int)(i % F);
-  const float g = __bfloat162float(gu[t * 2 * F + j]);
-  const float u = __bfloat162float(gu[t * 2 * F + F + j]);
-  const float sg = 1.0f / (1.0f + expf(-g));
-  const float d = dm[i];
-  dgu[t * 2 * F + j] = __float2bfloat16_rn(d * u * sg * (1.0f + g * (1.0f - sg)));
-  dgu[t * 2 * F + F + j] = __float2bfloat16_rn(d * g * sg);
+  if (i >= T * f8) return;
+  const int64_t t = i / f8;
+  const int j = (int)(i % f8) * 8;
+  const uint4 gv = *reinterpret_cast<const uint4*>(gu + t * 2 * F + j);
+  const uint4 uv = *reinterpret_cast<const uint4*>(gu + t * 2 * F + F + j);
+  const float4 d0 = *reinterpret_cast<const float4*>(dm + t * F + j);
+  const float4 d1 = *reinterpret_cast<const float4*>(dm + t * F + j + 4);
+  const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+  const bf16* g8 = reinterpret_cast<const bf16*>(&gv);
+  const bf16* u8 = reinterpret_cast<const bf16*>(&uv);
+  uint4 og, ou;
+  __nv_bfloat162* og2 = reinterpret_cast<__nv_bfloat162*>(&og);
+  __nv_bfloat162* ou2 = reinterpret_cast<__nv_bfloat162*>(&ou);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float rg[2], ru[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float g = __bfloat162float(g8[2 * e + k]), u = __bfloat162float(u8[2 * e + k]);
+      const float sg = 1.0f / (1.0f + expf(-g));
+      const float d = dd[2 * e + k];
+      rg[k] = d * u * sg * (1.0f + g * (1.0f - sg));
+      ru[k] = d * g * sg;
+    }
+    og2[e] = __floats2bfloat162_rn(rg[0], rg[1]);
+    ou2[e] = __floats2bfloat162_rn(ru[0], ru[1]);
+  }
+  *reinterpret_cast<uint4*>(dgu + t * 2 * F + j) = og;
+  *reinterpret_cast<uint4*>(dgu + t * 2 * F + F + j) = ou;
 }
 
 // ------------------------------------------------------------------------------- embedding
@@ -236,6 +291,7 @@ cudaError_t rmsnorm_fwd(const float* x, const float* g, int64_t T, int d, float 
 }
 cudaError_t rmsnorm_bwd(const float* dy, const float* x, const float* g, const float* rstd, const float* dres,
                         int64_t T, int d, float* dx, bf16* dxb, cudaStream_t s) {
+  if (d % 8) return cudaErrorInvalidValue;
   k_rmsnorm_bwd<<<(unsigned)T, 256, 0, s>>>(dy, x, g, rstd, dres, d, dx, dxb);
   note_launch(1);
   return cudaGetLastError();
@@ -252,12 +308,14 @@ cudaError_t rope_tables(int S, int hd, double theta, float* ct, float* st, cudaS
   return cudaGetLastError();
 }
 cudaError_t swiglu_fwd(const bf16* gu, int64_t T, int F, bf16* m, cudaStream_t s) {
-  k_swiglu_fwd<<<nblk(T * F), kThreads, 0, s>>>(gu, T, F, m);
+  if (F % 8) return cudaErrorInvalidValue;
+  k_swiglu_fwd<<<nblk(T * (F / 8)), kThreads, 0, s>>>(gu, T, F, m);
   note_launch(1);
   return cudaGetLastError();
 }
 cudaError_t swiglu_bwd(const float* dm, const bf16* gu, int64_t T, int F, bf16* dgu, cudaStream_t s) {
-  k_swiglu_bwd<<<nblk(T * F), kThreads, 0, s>>>(dm, gu, T, F, dgu);
+  if (F % 8) return cudaErrorInvalidValue;
+  k_swiglu_bwd<<<nblk(T * (F / 8)), kThreads, 0, s>>>(dm, gu, T, F, dgu);
   note_launch(1);
   return cudaGetLastError();
 }
