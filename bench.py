@@ -277,6 +277,8 @@ def run_gpu(args, wl):
     stream = torch.cuda.Stream()
     link_gbs = h2d_peak_gbs(torch)
     ctx = build_context(wl, torch, stream, seed=1234 + rank)
+    if not args.no_optimizer:
+        ctx.set_optimizer(lr=2e-4)   # the step includes the AdamW update of every adapter
     n_grad = ctx.lora_numel()
     grads = torch.zeros(n_grad, dtype=torch.float32, device="cuda")
     g = torch.Generator(device="cpu")
@@ -370,6 +372,7 @@ def run_gpu(args, wl):
         "dtype": "bf16", "data": "synthetic (seeded torch.randn weights / uniform tokens)",
         "config": {"workload": describe(wl), "batch": wl.batch, "seq": wl.seq, "layers": wl.n_layers,
                    "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                   "optimizer": "none" if args.no_optimizer else "AdamW lr 2e-4 on every adapter, inside the step",
                    "l2": "not flushed: every step streams all layer blobs (GBs) through HBM, far above the 126 MB L2",
                    "loss_last": loss},
         "roofline": {"bound": "tensor", "kernel": "tcgen05 bf16 GEMM (all projection + LM-head GEMMs)",
@@ -411,6 +414,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-seq", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-optimizer", action="store_true")
     args = ap.parse_args()
     wl = workload(args.workload)
     if args.impl == "reference":

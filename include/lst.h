@@ -127,6 +127,26 @@ lst_status lst_set_lora(lst_ctx* ctx, int32_t layer, int32_t proj, const float* 
  * projection in LST_PROJ order, dA [r, in] then dB [out, r]. */
 int64_t lst_lora_numel(const lst_ctx* ctx);
 
+/* AdamW on the adapters ("Fine-tune Llama 3.1 8B on a 4GB GPU with Soup", "Step 5": lr 2e-4;
+ * "Fine-Tuning an 8B Parameter Model on a 4 GB Laptop GPU": Adam keeps two extra tensors per
+ * parameter). With an optimizer set, every step ends with
+ *   m <- b1 m + (1-b1) g;  v <- b2 v + (1-b2) g^2;
+ *   p <- p (1 - lr wd) - lr / (1 - b1^t) * m / (sqrt(v) / sqrt(1 - b2^t) + eps)
+ * on every adapter element (fp32, t = 1, 2, ... counted from lst_set_optimizer), after the step's
+ * gradients are complete; the next step computes with the updated adapters. */
+typedef struct {
+  float lr;            /* learning rate */
+  float beta1, beta2;  /* moment decay rates, in [0, 1) */
+  float eps;           /* > 0 */
+  float weight_decay;  /* decoupled weight decay, >= 0 */
+} lst_adamw;
+
+/* Enable (cfg non-NULL: moments reset to zero, t reset) or disable (NULL) the update. */
+lst_status lst_set_optimizer(lst_ctx* ctx, const lst_adamw* cfg);
+
+/* Copy the current adapters (lst_lora_numel fp32 values, gradient layout) to dst (host or device). */
+lst_status lst_get_lora(lst_ctx* ctx, float* dst);
+
 /* One forward + backward step of the model with a head: tokens and targets are int32
  * [batch * seq] (host or device), the loss is the mean cross-entropy over all tokens (written to
  * *loss, host memory). grads (host or device, may be NULL) receives lst_lora_numel() fp32 values.

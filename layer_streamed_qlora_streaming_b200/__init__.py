@@ -38,6 +38,11 @@ class LayerWeights(C.Structure):
                 ("mlp_norm", C.c_void_p), ("lora_a", C.c_void_p * 7), ("lora_b", C.c_void_p * 7)]
 
 
+class AdamW(C.Structure):
+    _fields_ = [("lr", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float), ("eps", C.c_float),
+                ("weight_decay", C.c_float)]
+
+
 class Stats(C.Structure):
     _fields_ = [("steps", C.c_int64), ("launches_last_step", C.c_int64),
                 ("layer_reads_last_step", C.c_int64), ("h2d_bytes_last_step", C.c_int64),
@@ -59,6 +64,8 @@ _SIGS = {
     "lst_register_layer": (_I32, [_P, _I32, C.POINTER(LayerWeights)]),
     "lst_set_lora": (_I32, [_P, _I32, _I32, _P, _P]),
     "lst_lora_numel": (_I64, [_P]),
+    "lst_set_optimizer": (_I32, [_P, _P]),
+    "lst_get_lora": (_I32, [_P, _P]),
     "lst_step": (_I32, [_P, _P, _P, _I32, _I32, C.POINTER(C.c_float), _P]),
     "lst_step_hidden": (_I32, [_P, _P, _P, _I32, _I32, C.POINTER(C.c_float), _P]),
     "lst_get_logits": (_I32, [_P, _P]),
@@ -199,6 +206,17 @@ class Context:
 
     def lora_numel(self) -> int:
         return int(lib().lst_lora_numel(self.h))
+
+    def set_optimizer(self, lr=2e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, off=False):
+        """AdamW on the adapters at the end of every step (off=True disables it)."""
+        if off:
+            _check(lib().lst_set_optimizer(self.h, None), self.h, "lst_set_optimizer")
+            return
+        cfg = AdamW(lr, beta1, beta2, eps, weight_decay)
+        _check(lib().lst_set_optimizer(self.h, C.byref(cfg)), self.h, "lst_set_optimizer")
+
+    def get_lora(self, dst) -> None:
+        _check(lib().lst_get_lora(self.h, _ptr(dst)), self.h, "lst_get_lora")
 
     def step(self, tokens, targets, batch: int, seq: int, grads=None) -> float:
         loss = C.c_float()

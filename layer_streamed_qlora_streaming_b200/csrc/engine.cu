@@ -23,6 +23,7 @@
 #include "lora.cuh"
 #include "nf4.cuh"
 #include "ops.cuh"
+#include "optim.cuh"
 
 #include <atomic>
 #include <chrono>
@@ -226,6 +227,14 @@ struct lst_ctx {
   bool have_logits = false;
 
   lst_stats st{};
+  // AdamW on the adapters (off until lst_set_optimizer)
+  bool opt_on = false;
+  lst_adamw opt{};
+  int64_t opt_t = 0;
+  float *opt_m = nullptr, *opt_v = nullptr;
+  AdamTensor* opt_tab = nullptr;  // device table of every adapter tensor and its bf16 mirror
+  int opt_ntab = 0;
+  int64_t opt_maxn = 0;
   // profiling
   bool profiling = false;
   struct ProfRec {
@@ -821,6 +830,28 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
       TRY(dalloc(c, &D.Acat16, (int64_t)G.KP * G.in, true));
       TRY(dalloc(c, &D.Bexp16, (int64_t)G.out * G.KP, true));
     }
+  {
+    // table of every adapter tensor for the fused AdamW pass (and where its bf16 copy lives)
+    std::vector<AdamTensor> tab;
+    for (int l = 0; l < c->L; ++l)
+      for (int g = 0; g < NGROUP; ++g) {
+        const Group& G = c->grp[g];
+        const auto& D = c->der[l * NGROUP + g];
+        for (int k = 0; k < G.nseg; ++k) {
+          const int p = G.proj[k];
+          AdamTensor a{c->offA[l * NPROJ + p], (int64_t)c->r * G.in, c->r, G.in, D.Acat16, G.in, k * c->r, 0};
+          const int outp = G.bounds[k + 1] - G.bounds[k];
+          AdamTensor b{c->offB[l * NPROJ + p], (int64_t)outp * c->r, outp, c->r, D.Bexp16, G.KP, G.bounds[k],
+                       k * c->r};
+          tab.push_back(a);
+          tab.push_back(b);
+          c->opt_maxn = std::max(c->opt_maxn, std::max(a.n, b.n));
+        }
+      }
+    c->opt_ntab = (int)tab.size();
+    TRY(dalloc(c, &c->opt_tab, (int64_t)tab.size()));
+    CK(cudaMemcpy(c->opt_tab, tab.data(), tab.size() * sizeof(AdamTensor), cudaMemcpyHostToDevice));
+  }
 
   // base storage
   const int64_t blob = c->lay.total;
@@ -1068,6 +1099,23 @@ lst_status lst_set_lora(lst_ctx* c, int32_t layer, int32_t proj, const float* a,
 
 int64_t lst_lora_numel(const lst_ctx* c) { return c ? c->lora_numel : 0; }
 
+static lst_status optimizer_update(lst_ctx* c) {
+  if (!c->opt_on) return LST_OK;
+  c->opt_t += 1;
+  const double t = (double)c->opt_t;
+  AdamHyper h;
+  h.lr = c->opt.lr;
+  h.b1 = c->opt.beta1;
+  h.b2 = c->opt.beta2;
+  h.eps = c->opt.eps;
+  h.wd = c->opt.weight_decay;
+  h.step_size = (float)(c->opt.lr / (1.0 - std::pow((double)c->opt.beta1, t)));
+  h.sqrt_bc2 = (float)std::sqrt(1.0 - std::pow((double)c->opt.beta2, t));
+  ProfScope ps(c, c->stream, PC_OTHER);
+  CK(adamw_update(c->opt_tab, c->opt_ntab, c->opt_maxn, c->lora, c->grads, c->opt_m, c->opt_v, h, c->stream));
+  return LST_OK;
+}
+
 lst_status lst_step(lst_ctx* c, const int32_t* tokens, const int32_t* targets, int32_t batch, int32_t seq,
                     float* loss, float* grads) {
   if (!c) return LST_ERR_ARG;
@@ -1081,6 +1129,7 @@ lst_status lst_step(lst_ctx* c, const int32_t* tokens, const int32_t* targets, i
     CK(embed(c->tok, c->E, c->curT, c->d, c->V, c->xs, c->stream));
   }
   TRY(run_layers(c, true));
+  TRY(optimizer_update(c));
   c->have_logits = true;
   return finish_step(c, loss, grads);
 }
@@ -1095,6 +1144,7 @@ lst_status lst_step_hidden(lst_ctx* c, const uint16_t* x, const uint16_t* g, int
   CK(bf16_to_f32(c->dout_b, c->curT * c->d, c->xs, c->stream));
   TRY(copy_in(c, c->gbuf, g, c->curT * c->d * 2));
   TRY(run_layers(c, false));
+  TRY(optimizer_update(c));
   c->have_logits = false;
   return finish_step(c, loss, grads);
 }
@@ -1135,6 +1185,39 @@ lst_status lst_get_activation(lst_ctx* c, int32_t which, int32_t layer, void* ds
     }
   }
   CK(cudaMemcpyAsync(dst, src, bytes, is_device_ptr(dst) ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
+                     c->stream));
+  CK(cudaStreamSynchronize(c->stream));
+  return LST_OK;
+}
+
+lst_status lst_set_optimizer(lst_ctx* c, const lst_adamw* cfg) {
+  if (!c) return LST_ERR_ARG;
+  if (!cfg) {
+    c->opt_on = false;
+    return LST_OK;
+  }
+  if (!(cfg->lr >= 0.f) || !(cfg->beta1 >= 0.f && cfg->beta1 < 1.f) || !(cfg->beta2 >= 0.f && cfg->beta2 < 1.f) ||
+      !(cfg->eps > 0.f) || !(cfg->weight_decay >= 0.f))
+    return fail(c, LST_ERR_ARG, "bad AdamW hyper-parameters");
+  if (!c->opt_m) {
+    TRY(dalloc(c, &c->opt_m, c->lora_numel, true));
+    TRY(dalloc(c, &c->opt_v, c->lora_numel, true));
+  } else {
+    CK(cudaMemsetAsync(c->opt_m, 0, c->lora_numel * 4, c->stream));
+    CK(cudaMemsetAsync(c->opt_v, 0, c->lora_numel * 4, c->stream));
+    CK(cudaStreamSynchronize(c->stream));
+  }
+  c->opt = *cfg;
+  c->opt_t = 0;
+  c->opt_on = true;
+  return LST_OK;
+}
+
+lst_status lst_get_lora(lst_ctx* c, float* dst) {
+  if (!c) return LST_ERR_ARG;
+  if (!dst) return fail(c, LST_ERR_ARG, "null dst");
+  const bool dev = is_device_ptr(dst);
+  CK(cudaMemcpyAsync(dst, c->lora, c->lora_numel * 4, dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
                      c->stream));
   CK(cudaStreamSynchronize(c->stream));
   return LST_OK;

@@ -228,3 +228,19 @@ def test_bf16_rounding_matches_torch_and_bf16_mode_is_consistent():
     assert a["loss"] == b["loss"]
     assert abs(a["loss"] - e["loss"]) < 1e-3 * abs(e["loss"])
     assert a["loss"] != e["loss"]          # the rounding is really applied
+
+
+def test_adamw_matches_torch():
+    import torch
+    from oracle import optim
+    rng = np.random.default_rng(12)
+    p0 = rng.normal(size=500)
+    grads = [rng.normal(size=500) * s for s in (1e-3, 1e-1, 1.0)]
+    tp = torch.tensor(p0.copy(), dtype=torch.float64, requires_grad=True)
+    opt = torch.optim.AdamW([tp], lr=1e-2, betas=(0.9, 0.95), eps=1e-8, weight_decay=0.1)
+    p, m, v = p0.copy(), np.zeros(500), np.zeros(500)
+    for t, g in enumerate(grads, start=1):
+        tp.grad = torch.tensor(g)
+        opt.step()
+        p, m, v = optim.adamw_step(p, g, m, v, t, lr=1e-2, b1=0.9, b2=0.95, eps=1e-8, wd=0.1)
+        np.testing.assert_allclose(p, tp.detach().numpy(), rtol=1e-13, atol=1e-15)
