@@ -203,14 +203,14 @@ def test_adamw_step_matches_oracle_and_trains():
     loss0, g0, _ = run_step(ctx, wl, inp, want_logits=False)
     p1 = np.zeros_like(p0)
     ctx.get_lora(p1)
-    # oracle: gradients at the initial adapters, one AdamW update
+    # the update rule on the step's own gradients (identical inputs): AdamW's first update is
+    # close to lr * sign(g), so comparing it on independently computed gradients would only
+    # measure sign flips of near-zero gradient entries
+    p1_ref, _, _ = optim.adamw_step(p0, g0, np.zeros_like(g0), np.zeros_like(g0), 1, lr=lr, wd=0.01)
+    assert np.abs(p1.astype(np.float64) - p1_ref).max() <= 1e-7 + 1e-6 * np.abs(p1_ref).max()
+    # the gradients themselves are the oracle's (cosine; max-rel is covered by the other tests)
     ref = oracle_step(wl, inp, bf16_acts=True)
-    g_ref = _flat_from_oracle(ctx, ref["grads"])
-    p1_ref, _, _ = optim.adamw_step(p0, g_ref, np.zeros_like(g_ref), np.zeros_like(g_ref), 1, lr=lr,
-                                    wd=0.01)
-    d_gpu, d_ref = p1.astype(np.float64) - p0, p1_ref - p0
-    assert cosine(d_gpu, d_ref) > 0.999
-    assert np.abs(d_gpu - d_ref).max() < 0.05 * lr
+    assert cosine(g0, _flat_from_oracle(ctx, ref["grads"])) > 0.999
     # the next step computes with the updated adapters: loss matches the oracle at p1_ref
     loss1, _, _ = run_step(ctx, wl, inp, want_logits=False)
     raw1 = [dict(r) for r in inp["raw"]]
