@@ -101,8 +101,10 @@ lst_status lst_k_cross_entropy(const float* logits, int64_t T, int32_t V, const 
 /* LoRA skinny projection Us = bf16(s * X Bop) of the side path ("Fine-Tuning an 8B Parameter
  * Model on a 4 GB Laptop GPU", section "LoRA and QLoRA"): X bf16 [T, K] (row stride ldx); Bop bf16
  * K-major [KP, K] (b_mn = 0: Us = s X Bop^T) or MN-major [K, KP] (b_mn = 1: Us = s X Bop);
- * Us [T, KP] contiguous. Split-K on the tensor cores with a fixed-order reduction; scratch: fp32
- * device buffer of scratch_floats >= 16 * T * KP. */
+ * Us [T, KP] contiguous. Split-K on the tensor cores; the last split of each row tile sums the
+ * partials in split order (deterministic). scratch: fp32 device buffer of scratch_floats >=
+ * 16 * T * KP + ceil(T / 128) + 4 floats, ZERO-FILLED before the first call (its tail holds tile
+ * counters, which every call leaves at zero again). */
 lst_status lst_k_lora_skinny(const uint16_t* X, int64_t ldx, int64_t T, int32_t K,
                              const uint16_t* Bop, int64_t ldb, int32_t b_mn, int32_t KP, float s,
                              uint16_t* Us, float* scratch, int64_t scratch_floats, void* stream);

@@ -895,7 +895,7 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
     part = std::max(part, lora_skinny_scratch(T, G.KP));
     part = std::max(part, (int64_t)G.KP * std::max(G.in, G.out));
   }
-  TRY(dalloc(c, &c->part, part));
+  TRY(dalloc(c, &c->part, part, true));  // zero: its tail holds split-K tile semaphores
   TRY(dalloc(c, &c->ga, T * d));
   TRY(dalloc(c, &c->gb, T * d));
   TRY(dalloc(c, &c->dn, T * d));

@@ -33,6 +33,16 @@ struct Epi {
   const float* rope_cos;
   const float* rope_sin;
   int rope_end, rope_hd, rope_S;
+  // store mode: 0 plain; 1 / 2 scatter the [M, nseg*r] result into per-segment adapter gradients
+  int mode;
+  float* sdst[3];
+  int sr, snseg;
+  int sbounds[4];
+  // split-K: the CTA that completes a tile last sums the partials in split order into kout
+  __nv_bfloat16* kout;
+  int64_t ldk;
+  float kscale;
+  int* sem;
 };
 
 // Rotate the pair of 32-column chunks (na .. na+31) and (nb .. nb+31), nb = na + hd/2, of one row
@@ -86,6 +96,29 @@ struct Cfg {
 
 __device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const uint32_t (&r)[32]) {
   if (row >= e.M || col0 >= e.N) return;
+  if (e.mode == 1) {
+    // dA: column jj = p*r + j of row i goes to dst[p][j * M + i] (warp lanes hold consecutive i,
+    // so each column is written as one coalesced run)
+    const int R = e.snseg * e.sr;
+#pragma unroll 4
+    for (int i = 0; i < 32; ++i) {
+      const int jj = col0 + i;
+      if (jj < R) e.sdst[jj / e.sr][(int64_t)(jj % e.sr) * e.M + row] = __uint_as_float(r[i]) * e.alpha;
+    }
+    return;
+  }
+  if (e.mode == 2) {
+    // dB: row o of segment p keeps columns p*r .. p*r+r-1, stored at dst[p][(o - bounds[p]) * r + j]
+    int p = 0;
+    while (p + 1 < e.snseg && row >= e.sbounds[p + 1]) ++p;
+    float* d = e.sdst[p] + (int64_t)(row - e.sbounds[p]) * e.sr;
+#pragma unroll 4
+    for (int i = 0; i < 32; ++i) {
+      const int j = col0 + i - p * e.sr;
+      if (j >= 0 && j < e.sr) d[j] = __uint_as_float(r[i]) * e.alpha;
+    }
+    return;
+  }
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * e.alpha;
@@ -180,6 +213,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   uint64_t* acc_full = empty + C::STAGES;   // [2] accumulator ready for the epilogue
   uint64_t* acc_empty = acc_full + 2;       // [2] accumulator drained by the epilogue
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -332,6 +366,36 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);  // all 128 epilogue threads arrive once per tile
+      if (ep0.kout) {
+        // split-K: publish this partial tile; the last of the `splits` CTAs of the tile reduces
+        const int etid = threadIdx.x - 64;
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        int* sem = ep0.sem + (mi * sched.nt + ni);
+        if (etid == 0) *last_flag = (atomicAdd(sem, 1) == total_tiles / sched.tiles_per_z - 1);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (*last_flag) {
+          __threadfence();
+          const int nsplit = total_tiles / sched.tiles_per_z;
+          if (row < ep0.M) {
+            const float* base = static_cast<const float*>(ep0.C) + (int64_t)row * ep0.ldc;
+            for (int c = n0; c < n0 + BN && c < ep0.N; c += 4) {
+              float4 acc = *reinterpret_cast<const float4*>(base + c);
+              for (int zz = 1; zz < nsplit; ++zz) {
+                const float4 v = *reinterpret_cast<const float4*>(base + zz * split_stride + c);
+                acc.x += v.x;
+                acc.y += v.y;
+                acc.z += v.z;
+                acc.w += v.w;
+              }
+              __nv_bfloat162 h[2] = {__floats2bfloat162_rn(ep0.kscale * acc.x, ep0.kscale * acc.y),
+                                     __floats2bfloat162_rn(ep0.kscale * acc.z, ep0.kscale * acc.w)};
+              *reinterpret_cast<uint2*>(ep0.kout + (int64_t)row * ep0.ldk + c) = *reinterpret_cast<const uint2*>(h);
+            }
+          }
+          if (etid == 0) *sem = 0;  // ready for the next launch
+        }
+      }
     }
   }
   tc_fence_before();
@@ -399,7 +463,9 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
     tB2 = tB;
   }
   Epi e{a.C, a.ldc, a.bias, a.R, a.ldr, a.alpha, a.c_f32, a.M, a.N,
-        a.rope_cos, a.rope_sin, a.rope_cos ? a.rope_end : 0, a.rope_hd, a.rope_S};
+        a.rope_cos, a.rope_sin, a.rope_cos ? a.rope_end : 0, a.rope_hd, a.rope_S,
+        a.epi_mode, {a.sdst[0], a.sdst[1], a.sdst[2]}, a.sr, a.snseg,
+        {a.sbounds[0], a.sbounds[1], a.sbounds[2], a.sbounds[3]}, a.kout, a.ldk, a.kscale, a.sem};
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t err =
@@ -436,6 +502,9 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
 cudaError_t gemm_bf16(const GemmArgs& a, cudaStream_t s) {
   if (a.M <= 0 || a.N <= 0 || a.K <= 0 || !a.A || !a.B || !a.C) return cudaErrorInvalidValue;
   if (a.splits > 1 && (a.bias || a.R || a.A2)) return cudaErrorInvalidValue;  // partials are summed later
+  if (a.kout && (!a.sem || !a.c_f32 || a.epi_mode || (a.N % 4) || (a.ldc % 4) || (a.ldk % 4))) return cudaErrorInvalidValue;
+  if (a.epi_mode && (a.splits > 1 || a.kout || a.rope_cos || a.sr <= 0 || a.snseg < 1 || a.snseg > 3))
+    return cudaErrorInvalidValue;
   // TMA: 16-byte aligned bases and row strides
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   if (!al16(a.A) || !al16(a.B) || (a.lda % 8) || (a.ldb % 8)) return cudaErrorInvalidValue;

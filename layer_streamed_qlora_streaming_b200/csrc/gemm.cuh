@@ -44,6 +44,20 @@ struct GemmArgs {
   const float* rope_cos = nullptr;
   const float* rope_sin = nullptr;
   int rope_end = 0, rope_hd = 0, rope_S = 0;
+  // Store mode for the LoRA gradients (result [M, snseg * sr], fp32, scaled by alpha):
+  //   1: column p*sr + j of row i -> sdst[p][j * M + i]                        (dA, [r, in])
+  //   2: row o of segment p (sbounds), column p*sr + j -> sdst[p][(o - sbounds[p]) * sr + j] (dB)
+  int epi_mode = 0;
+  float* sdst[3] = {nullptr, nullptr, nullptr};
+  int sr = 0, snseg = 0;
+  int sbounds[4] = {0, 0, 0, 0};
+  // Split-K with the reduction in the kernel: C receives the fp32 partials; the last CTA of each
+  // output tile sums them in split order and writes bf16(kscale * sum) to kout [M, N] (row stride
+  // ldk). sem: one int per output tile, zero before the call and left zero after it.
+  __nv_bfloat16* kout = nullptr;
+  int64_t ldk = 0;
+  float kscale = 1.0f;
+  int* sem = nullptr;
 };
 
 // Returns cudaSuccess or the launch / argument error. Deterministic: no split-K, no atomics.

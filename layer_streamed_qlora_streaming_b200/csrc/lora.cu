@@ -30,45 +30,6 @@ int skinny_splits(int64_t T, int K) {
   return (nk + kps - 1) / kps;  // the same count the GEMM launch settles on (no empty split)
 }
 
-__global__ void k_splitk_reduce(const float* __restrict__ part, int splits, int64_t stride, int64_t n, float s,
-                                __nv_bfloat16* __restrict__ out) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  float acc = 0.f;
-  for (int z = 0; z < splits; ++z) acc += part[z * stride + i];
-  out[i] = __float2bfloat16_rn(s * acc);
-}
-
-__global__ void k_scatter_a(const float* __restrict__ C, int in, int KP, int R, int r, float* d0, float* d1,
-                            float* d2) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (int64_t)in * R) return;
-  const int i = (int)(idx / R), jj = (int)(idx % R);
-  const int p = jj / r, j = jj % r;
-  float* d = p == 0 ? d0 : (p == 1 ? d1 : d2);
-  d[(int64_t)j * in + i] = C[(int64_t)i * KP + jj];
-}
-
-__global__ void k_scatter_b(const float* __restrict__ C, int out, int KP, int nseg, int r, int b1, int b2,
-                            float* d0, float* d1, float* d2) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (int64_t)out * r) return;
-  const int o = (int)(idx / r), j = (int)(idx % r);
-  int p = 0, lo = 0;
-  float* d = d0;
-  if (nseg > 1 && o >= b1) {
-    p = 1;
-    lo = b1;
-    d = d1;
-  }
-  if (nseg > 2 && o >= b2) {
-    p = 2;
-    lo = b2;
-    d = d2;
-  }
-  d[(int64_t)(o - lo) * r + j] = C[(int64_t)o * KP + p * r + j];
-}
-
 __global__ void k_lora_prep(const LoraPrepArgs a) {
   const int R = a.nseg * a.r;
   const int out = a.bounds[a.nseg];
@@ -94,7 +55,8 @@ inline unsigned nblk(int64_t n) { return (unsigned)((n + 255) / 256); }
 
 }  // namespace
 
-int64_t lora_skinny_scratch(int64_t T, int KP) { return (int64_t)kMaxSplits * T * KP; }
+// fp32 partials of up to kMaxSplits splits, then one int semaphore per 128-row tile
+int64_t lora_skinny_scratch(int64_t T, int KP) { return (int64_t)kMaxSplits * T * KP + (T + 127) / 128 + 4; }
 
 cudaError_t lora_skinny(const __nv_bfloat16* X, int64_t ldx, int64_t T, int K, const __nv_bfloat16* Bop,
                         int64_t ldb, int b_mn, int KP, float s, float* part, __nv_bfloat16* Us, cudaStream_t st) {
@@ -114,11 +76,11 @@ cudaError_t lora_skinny(const __nv_bfloat16* X, int64_t ldx, int64_t T, int K, c
   a.c_f32 = 1;
   a.splits = splits;
   a.split_stride = T * KP;
-  cudaError_t e = gemm_bf16(a, st);
-  if (e != cudaSuccess) return e;
-  k_splitk_reduce<<<nblk(T * KP), 256, 0, st>>>(part, splits, T * KP, T * KP, s, Us);
-  note_launch(1);
-  return cudaGetLastError();
+  a.kout = Us;  // reduced in the kernel by the last split of each tile, in split order
+  a.ldk = KP;
+  a.kscale = s;
+  a.sem = reinterpret_cast<int*>(part + (int64_t)kMaxSplits * T * KP);
+  return gemm_bf16(a, st);
 }
 
 cudaError_t lora_grad_a(const __nv_bfloat16* X, int64_t ldx, int64_t T, int in, const __nv_bfloat16* Vs, int KP,
@@ -134,16 +96,15 @@ cudaError_t lora_grad_a(const __nv_bfloat16* X, int64_t ldx, int64_t T, int in, 
   a.B = Vs;
   a.ldb = KP;
   a.b_mn = 1;
-  a.C = part;
+  a.C = dst[0];  // not written: the epilogue scatters straight into the per-segment dA
   a.ldc = KP;
   a.c_f32 = 1;
-  cudaError_t e = gemm_bf16(a, st);
-  if (e != cudaSuccess) return e;
-  const int R = nseg * r;
-  k_scatter_a<<<nblk((int64_t)in * R), 256, 0, st>>>(part, in, KP, R, r, dst[0], nseg > 1 ? dst[1] : nullptr,
-                                                     nseg > 2 ? dst[2] : nullptr);
-  note_launch(1);
-  return cudaGetLastError();
+  a.epi_mode = 1;
+  for (int k = 0; k < nseg; ++k) a.sdst[k] = dst[k];
+  a.sr = r;
+  a.snseg = nseg;
+  (void)part;
+  return gemm_bf16(a, st);
 }
 
 cudaError_t lora_grad_b(const __nv_bfloat16* dY, int64_t ldy, int64_t T, int out, const __nv_bfloat16* Us, int KP,
@@ -159,16 +120,16 @@ cudaError_t lora_grad_b(const __nv_bfloat16* dY, int64_t ldy, int64_t T, int out
   a.B = Us;
   a.ldb = KP;
   a.b_mn = 1;
-  a.C = part;
+  a.C = dst[0];  // not written: the epilogue keeps each row's own segment and stores it as dB
   a.ldc = KP;
   a.c_f32 = 1;
-  cudaError_t e = gemm_bf16(a, st);
-  if (e != cudaSuccess) return e;
-  k_scatter_b<<<nblk((int64_t)out * r), 256, 0, st>>>(part, out, KP, nseg, r, nseg > 1 ? bounds[1] : out,
-                                                      nseg > 2 ? bounds[2] : out, dst[0],
-                                                      nseg > 1 ? dst[1] : nullptr, nseg > 2 ? dst[2] : nullptr);
-  note_launch(1);
-  return cudaGetLastError();
+  a.epi_mode = 2;
+  for (int k = 0; k < nseg; ++k) a.sdst[k] = dst[k];
+  for (int k = 0; k <= nseg; ++k) a.sbounds[k] = bounds[k];
+  a.sr = r;
+  a.snseg = nseg;
+  (void)part;
+  return gemm_bf16(a, st);
 }
 
 cudaError_t lora_prep(const LoraPrepArgs& a, cudaStream_t st) {

@@ -260,9 +260,14 @@ def test_lora_skinny(T, K, b_mn):
         Bop[:R] = _bf(r.normal(size=(R, K)) * 0.05)
         ref = 2.0 * X.astype(np.float64) @ Bop.T.astype(np.float64)
     Us = torch.zeros(T, 64, dtype=torch.bfloat16, device="cuda")
-    scratch = torch.empty(16 * T * 64, dtype=torch.float32, device="cuda")
-    lst.k_lora_skinny(torch_bf16(X), K, T, K, torch_bf16(Bop), 64 if b_mn else K, b_mn, 64, 2.0, Us, scratch)
-    torch.cuda.synchronize()
+    scratch = torch.zeros(16 * T * 64 + (T + 127) // 128 + 4, dtype=torch.float32, device="cuda")
+    outs = []
+    for _ in range(2):  # twice: the tile counters must come back to zero, results identical
+        lst.k_lora_skinny(torch_bf16(X), K, T, K, torch_bf16(Bop), 64 if b_mn else K, b_mn, 64, 2.0, Us, scratch)
+        torch.cuda.synchronize()
+        outs.append(Us.view(torch.int16).cpu().numpy().copy())
+    assert np.array_equal(outs[0], outs[1])
+    assert np.all(scratch[16 * T * 64:].cpu().numpy() == 0)
     got = to_np(Us)
     assert maxrel(got, ref) < 8e-3
     assert np.all(got[:, R:] == 0)
