@@ -109,6 +109,11 @@ lst_status lst_k_lora_skinny(const uint16_t* X, int64_t ldx, int64_t T, int32_t 
                              const uint16_t* Bop, int64_t ldb, int32_t b_mn, int32_t KP, float s,
                              uint16_t* Us, float* scratch, int64_t scratch_floats, void* stream);
 
+/* Read and clear the device error word of the current device: 0 when no kernel reported a
+ * problem, else the code of the first report (1: a bounded wait gave up, 2: an index was out of
+ * range). Synchronises the device. Returns -1 if the word cannot be read. */
+int32_t lst_k_device_error(void);
+
 /* Kernel launches made by this library so far in this process (all contexts). Needs no GPU. */
 int64_t lst_k_launch_count(void);
 

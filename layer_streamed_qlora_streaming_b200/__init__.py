@@ -94,6 +94,7 @@ _SIGS = {
     "lst_k_cross_entropy": (_I32, [_P, _I64, _I32, _P, _F32, _P, _P, _P]),
     "lst_k_lora_skinny": (_I32, [_P, _I64, _I64, _I32, _P, _I64, _I32, _I32, _F32, _P, _P, _I64, _P]),
     "lst_k_launch_count": (_I64, []),
+    "lst_k_device_error": (_I32, []),
 }
 
 
@@ -341,6 +342,11 @@ def k_cross_entropy(logits, T, V, targets, inv_T, loss_rows, dlogits, stream=Non
 def k_lora_skinny(X, ldx, T, K, Bop, ldb, b_mn, KP, s, Us, scratch, stream=None):
     _check(lib().lst_k_lora_skinny(_ptr(X), ldx, T, K, _ptr(Bop), ldb, b_mn, KP, s, _ptr(Us), _ptr(scratch),
                                    scratch.numel(), _stream(stream)), what="lst_k_lora_skinny")
+
+
+def device_error() -> int:
+    """Read and clear the device error word (0 = none)."""
+    return int(lib().lst_k_device_error())
 
 
 def launch_count() -> int:

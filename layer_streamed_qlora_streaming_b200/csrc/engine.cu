@@ -1257,3 +1257,20 @@ int64_t lst_blob_bytes(const lst_config* cfg) {
 }
 
 }  // extern "C"
+
+extern "C" int32_t lst_k_device_error(void) {
+  int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  if (cudaMemcpyFromSymbol(&v, lst::g_lst_dev_error, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  if (v) {
+    int zero = 0;
+    cudaMemcpyToSymbol(lst::g_lst_dev_error, &zero, sizeof(int));
+  }
+  return v;
+}

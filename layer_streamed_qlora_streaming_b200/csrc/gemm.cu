@@ -43,20 +43,21 @@ struct Epi {
   int64_t ldk;
   float kscale;
   int* sem;
+  int64_t sstride;  // elements between the partial results of consecutive K splits
 };
 
 // Rotate the pair of 32-column chunks (na .. na+31) and (nb .. nb+31), nb = na + hd/2, of one row
 // by the angle of position pos (pairs j, j + hd/2 with j = j0 + i), after scale and bias; store
 // bf16. Used for q and k straight out of the projection GEMM, so they are rounded once.
-__device__ __forceinline__ void epi_store_rope(const Epi& e, int row, int na, int nb, int j0,
+__device__ __forceinline__ void epi_store_rope(const Epi& e, void* C, int row, int na, int nb, int j0,
                                                const uint32_t (&ra)[32], const uint32_t (&rb)[32]) {
   if (row >= e.M) return;
   const int half = e.rope_hd / 2;
   const int pos = row % e.rope_S;
   const float* cs = e.rope_cos + (int64_t)pos * half + j0;
   const float* sn = e.rope_sin + (int64_t)pos * half + j0;
-  __nv_bfloat16* ca = reinterpret_cast<__nv_bfloat16*>(e.C) + (int64_t)row * e.ldc + na;
-  __nv_bfloat16* cb = reinterpret_cast<__nv_bfloat16*>(e.C) + (int64_t)row * e.ldc + nb;
+  __nv_bfloat16* ca = reinterpret_cast<__nv_bfloat16*>(C) + (int64_t)row * e.ldc + na;
+  __nv_bfloat16* cb = reinterpret_cast<__nv_bfloat16*>(C) + (int64_t)row * e.ldc + nb;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint4 ua, ub;
@@ -94,7 +95,7 @@ struct Cfg {
   static constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;  // one accumulator; two are allocated
 };
 
-__device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void epi_store(const Epi& e, void* C, int row, int col0, const uint32_t (&r)[32]) {
   if (row >= e.M || col0 >= e.N) return;
   if (e.mode == 1) {
     // dA: column jj = p*r + j of row i goes to dst[p][j * M + i] (warp lanes hold consecutive i,
@@ -145,7 +146,7 @@ __device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const
     }
   }
   if (e.c_f32) {
-    float* cp = reinterpret_cast<float*>(e.C) + (int64_t)row * e.ldc + col0;
+    float* cp = reinterpret_cast<float*>(C) + (int64_t)row * e.ldc + col0;
     if (full && ((reinterpret_cast<uintptr_t>(cp) & 15) == 0)) {
 #pragma unroll
       for (int q = 0; q < 8; ++q)
@@ -155,7 +156,7 @@ __device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const
         if (col0 + i < e.N) cp[i] = v[i];
     }
   } else {
-    __nv_bfloat16* cp = reinterpret_cast<__nv_bfloat16*>(e.C) + (int64_t)row * e.ldc + col0;
+    __nv_bfloat16* cp = reinterpret_cast<__nv_bfloat16*>(C) + (int64_t)row * e.ldc + col0;
     if (full && ((reinterpret_cast<uintptr_t>(cp) & 15) == 0)) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -196,13 +197,13 @@ struct TileSched {
 // two fp32 accumulators in TMEM, so the epilogue of one tile overlaps the main loop of the next.
 // AMN / BMN: A / B operand MN-major (row-major [K, M] / [K, N] in global memory), else K-major.
 // Split-K: slice z takes main k-blocks [z * kps, (z + 1) * kps) and writes its partial result at
-// C + z * split_stride (the second operand pair is only allowed without split).
+// C + z * ep.sstride (the second operand pair is only allowed without split).
 template <int BN, int AMN, int BMN>
 __global__ void __launch_bounds__(192, 1)
 k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
        const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
        const Epi ep0, const TileSched sched, const int total_tiles, const int nk1_total, const int nk2,
-       const int kps, const int64_t split_stride) {
+       const int kps) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -331,11 +332,9 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
       int mi, ni, z;
       sched.get(t, mi, ni, z);
       const int m0 = mi * BM, n0 = ni * BN;
-      Epi ep = ep0;
-      if (z) {
-        ep.C = ep.c_f32 ? static_cast<void*>(static_cast<float*>(ep.C) + z * split_stride)
-                        : static_cast<void*>(static_cast<__nv_bfloat16*>(ep.C) + z * split_stride);
-      }
+      const Epi& ep = ep0;
+      // this split's partial-result slot
+      void* const cz = static_cast<char*>(ep0.C) + (int64_t)z * ep0.sstride * (ep0.c_f32 ? 4 : 2);
       const int buf = local & 1;
       const uint32_t use = (uint32_t)(local >> 1);
       if (!mbar_wait(&acc_full[buf], use & 1)) break;
@@ -352,7 +351,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
             tmem_ld32(tq + h0 + j0, ra);
             tmem_ld32(tq + h0 + half + j0, rb);
             tmem_ld_wait();
-            epi_store_rope(ep, row, n0 + h0 + j0, n0 + h0 + half + j0, j0, ra, rb);
+            epi_store_rope(ep, cz, row, n0 + h0 + j0, n0 + h0 + half + j0, j0, ra, rb);
           }
         }
       } else {
@@ -361,7 +360,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           uint32_t r[32];
           tmem_ld32(tq + c, r);
           tmem_ld_wait();
-          epi_store(ep, row, n0 + c, r);
+          epi_store(ep, cz, row, n0 + c, r);
         }
       }
       tc_fence_before();
@@ -369,10 +368,15 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
       if (ep0.kout) {
         // split-K: publish this partial tile; the last of the `splits` CTAs of the tile reduces
         const int etid = threadIdx.x - 64;
-        __threadfence();
+        __threadfence();  // this thread's partial stores, then the group barrier, then one release
         asm volatile("bar.sync 1, 128;" ::: "memory");
         int* sem = ep0.sem + (mi * sched.nt + ni);
-        if (etid == 0) *last_flag = (atomicAdd(sem, 1) == total_tiles / sched.tiles_per_z - 1);
+        if (etid == 0) {
+          __threadfence();
+          const int prev = atomicAdd(sem, 1);
+          __threadfence();  // acquire side for the reducer
+          *last_flag = (prev == total_tiles / sched.tiles_per_z - 1);
+        }
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (*last_flag) {
           __threadfence();
@@ -380,9 +384,10 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           if (row < ep0.M) {
             const float* base = static_cast<const float*>(ep0.C) + (int64_t)row * ep0.ldc;
             for (int c = n0; c < n0 + BN && c < ep0.N; c += 4) {
-              float4 acc = *reinterpret_cast<const float4*>(base + c);
+              // L2-coherent loads (bypass L1): the partials were written by other SMs
+              float4 acc = __ldcg(reinterpret_cast<const float4*>(base + c));
               for (int zz = 1; zz < nsplit; ++zz) {
-                const float4 v = *reinterpret_cast<const float4*>(base + zz * split_stride + c);
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(base + (int64_t)zz * ep0.sstride + c));
                 acc.x += v.x;
                 acc.y += v.y;
                 acc.z += v.z;
@@ -465,7 +470,8 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   Epi e{a.C, a.ldc, a.bias, a.R, a.ldr, a.alpha, a.c_f32, a.M, a.N,
         a.rope_cos, a.rope_sin, a.rope_cos ? a.rope_end : 0, a.rope_hd, a.rope_S,
         a.epi_mode, {a.sdst[0], a.sdst[1], a.sdst[2]}, a.sr, a.snseg,
-        {a.sbounds[0], a.sbounds[1], a.sbounds[2], a.sbounds[3]}, a.kout, a.ldk, a.kscale, a.sem};
+        {a.sbounds[0], a.sbounds[1], a.sbounds[2], a.sbounds[3]}, a.kout, a.ldk, a.kscale, a.sem,
+        a.split_stride};
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t err =
@@ -492,7 +498,7 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
       num_sms = 148;
   }
   const int grid = total < num_sms ? total : num_sms;
-  k_gemm<BN, AMN, BMN><<<grid, 192, C::SMEM, s>>>(tA, tB, tA2, tB2, e, sched, total, nk1, nk2, kps, a.split_stride);
+  k_gemm<BN, AMN, BMN><<<grid, 192, C::SMEM, s>>>(tA, tB, tA2, tB2, e, sched, total, nk1, nk2, kps);
   note_launch(1);
   return cudaGetLastError();
 }

@@ -71,9 +71,19 @@ def _pool():
         import concurrent.futures as cf
         import multiprocessing as mp
         import os
+        import atexit
         _POOL = cf.ProcessPoolExecutor(max_workers=min(16, os.cpu_count() or 1),
                                        mp_context=mp.get_context("spawn"))
+        atexit.register(_shutdown_pool)
     return _POOL
+
+
+def _shutdown_pool():
+    """Stop the workers while the interpreter is still whole (avoids noise at exit)."""
+    global _POOL
+    if _POOL is not None:
+        _POOL.shutdown(wait=True)
+        _POOL = None
 
 
 def normal(seed: int, stream: int, n: int, std: float = 1.0, chunk: int = 1 << 24) -> np.ndarray:
