@@ -101,13 +101,26 @@ lst_status lst_k_cross_entropy(const float* logits, int64_t T, int32_t V, const 
 /* LoRA skinny projection Us = bf16(s * X Bop) of the side path ("Fine-Tuning an 8B Parameter
  * Model on a 4 GB Laptop GPU", section "LoRA and QLoRA"): X bf16 [T, K] (row stride ldx); Bop bf16
  * K-major [KP, K] (b_mn = 0: Us = s X Bop^T) or MN-major [K, KP] (b_mn = 1: Us = s X Bop);
- * Us [T, KP] contiguous. Split-K on the tensor cores; the last split of each row tile sums the
- * partials in split order (deterministic). scratch: fp32 device buffer of scratch_floats >=
- * 16 * T * KP + ceil(T / 128) + 4 floats, ZERO-FILLED before the first call (its tail holds tile
- * counters, which every call leaves at zero again). */
+ * Us [T, KP] contiguous, KP a multiple of 8; ldx, ldb multiples of 8 and X, Bop 16-byte aligned.
+ * The K range is split over a thread-block cluster whose partial tiles are summed in slice order
+ * through distributed shared memory: deterministic, no scratch. */
 lst_status lst_k_lora_skinny(const uint16_t* X, int64_t ldx, int64_t T, int32_t K,
                              const uint16_t* Bop, int64_t ldb, int32_t b_mn, int32_t KP, float s,
-                             uint16_t* Us, float* scratch, int64_t scratch_floats, void* stream);
+                             uint16_t* Us, void* stream);
+
+/* LoRA adapter gradients of one fused projection group (same section): nseg (1..3) segments of rank
+ * r sharing the input X bf16 [T, in] (row stride ldx), with output-gradient dY bf16 [T, out] (row
+ * stride ldy) whose columns [bounds[p], bounds[p+1]) belong to segment p (bounds: HOST array of
+ * nseg + 1 ints, bounds[0] = 0, bounds[nseg] = out). Us = bf16(s X A_cat^T), Vs = bf16(s dY B_exp)
+ * [T, KP] (column p*r + j = rank j of segment p). Writes, fp32:
+ *   dA[p] [r, in]:        dA_p[j][i] = sum_t Vs[t][p*r + j] X[t][i]
+ *   dB[p] [out_p, r]:     dB_p[o][j] = sum_t dY[t][bounds[p] + o] Us[t][p*r + j]
+ * dA, dB: HOST arrays of nseg device pointers. Sums over t in a fixed order (deterministic). */
+lst_status lst_k_lora_grads(const uint16_t* X, int64_t ldx, int32_t in, const uint16_t* dY,
+                            int64_t ldy, int32_t out, int64_t T, const uint16_t* Us,
+                            const uint16_t* Vs, int32_t KP, int32_t nseg, int32_t r,
+                            const int32_t* bounds, float* const* dA, float* const* dB,
+                            void* stream);
 
 /* Read and clear the device error word of the current device: 0 when no kernel reported a
  * problem, else the code of the first report (1: a bounded wait gave up, 2: an index was out of

@@ -92,7 +92,8 @@ _SIGS = {
     "lst_k_swiglu_fwd": (_I32, [_P, _I64, _I32, _P, _P]),
     "lst_k_swiglu_bwd": (_I32, [_P, _P, _I64, _I32, _P, _P]),
     "lst_k_cross_entropy": (_I32, [_P, _I64, _I32, _P, _F32, _P, _P, _P]),
-    "lst_k_lora_skinny": (_I32, [_P, _I64, _I64, _I32, _P, _I64, _I32, _I32, _F32, _P, _P, _I64, _P]),
+    "lst_k_lora_skinny": (_I32, [_P, _I64, _I64, _I32, _P, _I64, _I32, _I32, _F32, _P, _P]),
+    "lst_k_lora_grads": (_I32, [_P, _I64, _I32, _P, _I64, _I32, _I64, _P, _P, _I32, _I32, _I32, _P, _P, _P, _P]),
     "lst_k_launch_count": (_I64, []),
     "lst_k_device_error": (_I32, []),
 }
@@ -339,9 +340,20 @@ def k_cross_entropy(logits, T, V, targets, inv_T, loss_rows, dlogits, stream=Non
                                      _ptr(dlogits), _stream(stream)), what="lst_k_cross_entropy")
 
 
-def k_lora_skinny(X, ldx, T, K, Bop, ldb, b_mn, KP, s, Us, scratch, stream=None):
-    _check(lib().lst_k_lora_skinny(_ptr(X), ldx, T, K, _ptr(Bop), ldb, b_mn, KP, s, _ptr(Us), _ptr(scratch),
-                                   scratch.numel(), _stream(stream)), what="lst_k_lora_skinny")
+def k_lora_skinny(X, ldx, T, K, Bop, ldb, b_mn, KP, s, Us, stream=None):
+    _check(lib().lst_k_lora_skinny(_ptr(X), ldx, T, K, _ptr(Bop), ldb, b_mn, KP, s, _ptr(Us), _stream(stream)),
+           what="lst_k_lora_skinny")
+
+
+def k_lora_grads(X, ldx, in_f, dY, ldy, out_f, T, Us, Vs, KP, r, bounds, dA, dB, stream=None):
+    """dA[p] [r, in] and dB[p] [out_p, r] (fp32 device tensors) of one fused group; bounds: the
+    nseg + 1 column bounds of the segments in dY."""
+    nseg = len(dA)
+    b = (C.c_int32 * 4)(*([int(v) for v in bounds] + [0] * (4 - len(bounds))))
+    pa = (C.c_void_p * 3)(*([_ptr(t) for t in dA] + [None] * (3 - nseg)))
+    pb = (C.c_void_p * 3)(*([_ptr(t) for t in dB] + [None] * (3 - nseg)))
+    _check(lib().lst_k_lora_grads(_ptr(X), ldx, in_f, _ptr(dY), ldy, out_f, T, _ptr(Us), _ptr(Vs), KP, nseg, r,
+                                  b, pa, pb, _stream(stream)), what="lst_k_lora_grads")
 
 
 def device_error() -> int:

@@ -203,7 +203,7 @@ struct lst_ctx {
   float* o32 = nullptr;  // attention output before rounding (recompute pass), for the backward's D
   __nv_bfloat16* Us[NGROUP] = {};  // bf16(s * x A^T) per group [T, KP]
   __nv_bfloat16* Vs[NGROUP] = {};  // bf16(s * dy B) per group [T, KP]
-  float *ga = nullptr, *gb = nullptr, *dn = nullptr, *dm = nullptr, *part = nullptr;
+  float *ga = nullptr, *gb = nullptr, *dn = nullptr, *dm = nullptr;
   __nv_bfloat16 *dout_b = nullptr, *dh_b = nullptr, *do_b = nullptr, *dqkvb = nullptr, *dgu = nullptr;
   __nv_bfloat16* nf = nullptr;
   float *rstdf = nullptr, *logits = nullptr, *loss_rows = nullptr, *loss_dev = nullptr, *dot_part = nullptr;
@@ -354,7 +354,7 @@ lst_status group_fwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
   const int64_t T = c->curT;
   {
     ProfScope ps(c, c->stream, PC_LORA);  // Us = bf16(s * X Acat^T)
-    CK(lora_skinny(X, ldx, T, G.in, D.Acat16, G.in, 0, G.KP, c->s, c->part, c->Us[g], c->stream));
+    CK(lora_skinny(X, ldx, T, G.in, D.Acat16, G.in, 0, G.KP, c->s, c->Us[g], c->stream));
   }
   if (!gemm) return LST_OK;
   GemmArgs a;
@@ -396,7 +396,7 @@ lst_status group_bwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
   const int64_t T = c->curT;
   {
     ProfScope ps(c, c->stream, PC_LORA);  // Vs = bf16(s * dY Bexp)
-    CK(lora_skinny(dY, ldy, T, G.out, D.Bexp16, G.KP, 1, G.KP, c->s, c->part, c->Vs[g], c->stream));
+    CK(lora_skinny(dY, ldy, T, G.out, D.Bexp16, G.KP, 1, G.KP, c->s, c->Vs[g], c->stream));
   }
   {
     GemmArgs a;
@@ -427,8 +427,8 @@ lst_status group_bwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
     dB[k] = c->grads + c->offB[layer * NPROJ + G.proj[k]];
   }
   // dA = s V^T X and dB = s dY^T U, with s folded into Vs and Us
-  CK(lora_grad_a(X, ldx, T, G.in, c->Vs[g], G.KP, G.nseg, c->r, dA, c->part, c->stream));
-  CK(lora_grad_b(dY, ldy, T, G.out, c->Us[g], G.KP, G.nseg, c->r, G.bounds, dB, c->part, c->stream));
+  CK(lora_grad_a(X, ldx, T, G.in, c->Vs[g], G.KP, G.nseg, c->r, dA, c->stream));
+  CK(lora_grad_b(dY, ldy, T, G.out, c->Us[g], G.KP, G.nseg, c->r, G.bounds, dB, c->stream));
   return LST_OK;
 }
 
@@ -887,15 +887,11 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   TRY(dalloc(c, &c->lse, T * c->hq));
   TRY(dalloc(c, &c->o32, T * c->dq));
   TRY(dalloc(c, &c->Dbuf, T * c->hq));
-  int64_t part = 0;
   for (int g = 0; g < NGROUP; ++g) {
     const Group& G = c->grp[g];
     TRY(dalloc(c, &c->Us[g], T * G.KP, true));
     TRY(dalloc(c, &c->Vs[g], T * G.KP, true));
-    part = std::max(part, lora_skinny_scratch(T, G.KP));
-    part = std::max(part, (int64_t)G.KP * std::max(G.in, G.out));
   }
-  TRY(dalloc(c, &c->part, part, true));  // zero: its tail holds split-K tile semaphores
   TRY(dalloc(c, &c->ga, T * d));
   TRY(dalloc(c, &c->gb, T * d));
   TRY(dalloc(c, &c->dn, T * d));

@@ -33,31 +33,20 @@ struct Epi {
   const float* rope_cos;
   const float* rope_sin;
   int rope_end, rope_hd, rope_S;
-  // store mode: 0 plain; 1 / 2 scatter the [M, nseg*r] result into per-segment adapter gradients
-  int mode;
-  float* sdst[3];
-  int sr, snseg;
-  int sbounds[4];
-  // split-K: the CTA that completes a tile last sums the partials in split order into kout
-  __nv_bfloat16* kout;
-  int64_t ldk;
-  float kscale;
-  int* sem;
-  int64_t sstride;  // elements between the partial results of consecutive K splits
 };
 
 // Rotate the pair of 32-column chunks (na .. na+31) and (nb .. nb+31), nb = na + hd/2, of one row
 // by the angle of position pos (pairs j, j + hd/2 with j = j0 + i), after scale and bias; store
 // bf16. Used for q and k straight out of the projection GEMM, so they are rounded once.
-__device__ __forceinline__ void epi_store_rope(const Epi& e, void* C, int row, int na, int nb, int j0,
+__device__ __forceinline__ void epi_store_rope(const Epi& e, int row, int na, int nb, int j0,
                                                const uint32_t (&ra)[32], const uint32_t (&rb)[32]) {
   if (row >= e.M) return;
   const int half = e.rope_hd / 2;
   const int pos = row % e.rope_S;
   const float* cs = e.rope_cos + (int64_t)pos * half + j0;
   const float* sn = e.rope_sin + (int64_t)pos * half + j0;
-  __nv_bfloat16* ca = reinterpret_cast<__nv_bfloat16*>(C) + (int64_t)row * e.ldc + na;
-  __nv_bfloat16* cb = reinterpret_cast<__nv_bfloat16*>(C) + (int64_t)row * e.ldc + nb;
+  __nv_bfloat16* ca = reinterpret_cast<__nv_bfloat16*>(e.C) + (int64_t)row * e.ldc + na;
+  __nv_bfloat16* cb = reinterpret_cast<__nv_bfloat16*>(e.C) + (int64_t)row * e.ldc + nb;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint4 ua, ub;
@@ -95,31 +84,8 @@ struct Cfg {
   static constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;  // one accumulator; two are allocated
 };
 
-__device__ __forceinline__ void epi_store(const Epi& e, void* C, int row, int col0, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const uint32_t (&r)[32]) {
   if (row >= e.M || col0 >= e.N) return;
-  if (e.mode == 1) {
-    // dA: column jj = p*r + j of row i goes to dst[p][j * M + i] (warp lanes hold consecutive i,
-    // so each column is written as one coalesced run)
-    const int R = e.snseg * e.sr;
-#pragma unroll 4
-    for (int i = 0; i < 32; ++i) {
-      const int jj = col0 + i;
-      if (jj < R) e.sdst[jj / e.sr][(int64_t)(jj % e.sr) * e.M + row] = __uint_as_float(r[i]) * e.alpha;
-    }
-    return;
-  }
-  if (e.mode == 2) {
-    // dB: row o of segment p keeps columns p*r .. p*r+r-1, stored at dst[p][(o - bounds[p]) * r + j]
-    int p = 0;
-    while (p + 1 < e.snseg && row >= e.sbounds[p + 1]) ++p;
-    float* d = e.sdst[p] + (int64_t)(row - e.sbounds[p]) * e.sr;
-#pragma unroll 4
-    for (int i = 0; i < 32; ++i) {
-      const int j = col0 + i - p * e.sr;
-      if (j >= 0 && j < e.sr) d[j] = __uint_as_float(r[i]) * e.alpha;
-    }
-    return;
-  }
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * e.alpha;
@@ -146,7 +112,7 @@ __device__ __forceinline__ void epi_store(const Epi& e, void* C, int row, int co
     }
   }
   if (e.c_f32) {
-    float* cp = reinterpret_cast<float*>(C) + (int64_t)row * e.ldc + col0;
+    float* cp = reinterpret_cast<float*>(e.C) + (int64_t)row * e.ldc + col0;
     if (full && ((reinterpret_cast<uintptr_t>(cp) & 15) == 0)) {
 #pragma unroll
       for (int q = 0; q < 8; ++q)
@@ -156,7 +122,7 @@ __device__ __forceinline__ void epi_store(const Epi& e, void* C, int row, int co
         if (col0 + i < e.N) cp[i] = v[i];
     }
   } else {
-    __nv_bfloat16* cp = reinterpret_cast<__nv_bfloat16*>(C) + (int64_t)row * e.ldc + col0;
+    __nv_bfloat16* cp = reinterpret_cast<__nv_bfloat16*>(e.C) + (int64_t)row * e.ldc + col0;
     if (full && ((reinterpret_cast<uintptr_t>(cp) & 15) == 0)) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -175,14 +141,13 @@ __device__ __forceinline__ void epi_store(const Epi& e, void* C, int row, int co
 
 // Tile order: groups of kGroupM M-tiles; inside a group the M-tile index runs fastest, so the
 // CTAs working at the same time share a few weight (B) tiles and the group's activation rows in
-// L2. Split-K slices (z) are the slowest index.
+// L2.
 constexpr int kGroupM = 8;
 
 struct TileSched {
-  int mt, nt, tiles_per_z;
-  __device__ __forceinline__ void get(int t, int& m, int& n, int& z) const {
-    z = t / tiles_per_z;
-    const int r = t - z * tiles_per_z;
+  int mt, nt;
+  __device__ __forceinline__ void get(int t, int& m, int& n) const {
+    const int r = t;
     const int per_group = kGroupM * nt;
     const int g = r / per_group;
     const int first = g * kGroupM;
@@ -196,14 +161,11 @@ struct TileSched {
 // Persistent tcgen05 GEMM. Each CTA loops over tiles t = blockIdx.x, + gridDim.x, ... and keeps
 // two fp32 accumulators in TMEM, so the epilogue of one tile overlaps the main loop of the next.
 // AMN / BMN: A / B operand MN-major (row-major [K, M] / [K, N] in global memory), else K-major.
-// Split-K: slice z takes main k-blocks [z * kps, (z + 1) * kps) and writes its partial result at
-// C + z * ep.sstride (the second operand pair is only allowed without split).
 template <int BN, int AMN, int BMN>
 __global__ void __launch_bounds__(192, 1)
 k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
        const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-       const Epi ep0, const TileSched sched, const int total_tiles, const int nk1_total, const int nk2,
-       const int kps) {
+       const Epi ep, const TileSched sched, const int total_tiles, const int nk1, const int nk2) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -214,7 +176,6 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   uint64_t* acc_full = empty + C::STAGES;   // [2] accumulator ready for the epilogue
   uint64_t* acc_empty = acc_full + 2;       // [2] accumulator drained by the epilogue
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -252,10 +213,9 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
       uint32_t it = 0;  // stage counter across tiles
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        int mi, ni, z;
-        sched.get(t, mi, ni, z);
-        const int m0 = mi * BM, n0 = ni * BN, kb0 = z * kps;
-        const int nk1 = min(nk1_total - kb0, kps);
+        int mi, ni;
+        sched.get(t, mi, ni);
+        const int m0 = mi * BM, n0 = ni * BN;
         const int nk = nk1 + nk2;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % C::STAGES;
@@ -268,7 +228,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           const bool second = kb >= nk1;
           const CUtensorMap* ma = second ? &tmA2 : &tmA;
           const CUtensorMap* mb = second ? &tmB2 : &tmB;
-          const int kk = (second ? kb - nk1 : kb0 + kb) * BK;
+          const int kk = (second ? kb - nk1 : kb) * BK;
           if (AMN == 0) {
             tma_load_2d(sA + s * C::A_BYTES, ma, &full[s], kk, m0);
           } else {
@@ -293,9 +253,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
       bool ok = true;
       int local = 0;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++local) {
-        int mi, ni, z;
-        sched.get(t, mi, ni, z);
-        const int nk = min(nk1_total - z * kps, kps) + nk2;
+        const int nk = nk1 + nk2;
         const int buf = local & 1;
         const uint32_t use = (uint32_t)(local >> 1);
         // the epilogue must have drained this accumulator (its use two tiles ago)
@@ -329,12 +287,9 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int local = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
-      int mi, ni, z;
-      sched.get(t, mi, ni, z);
+      int mi, ni;
+      sched.get(t, mi, ni);
       const int m0 = mi * BM, n0 = ni * BN;
-      const Epi& ep = ep0;
-      // this split's partial-result slot
-      void* const cz = static_cast<char*>(ep0.C) + (int64_t)z * ep0.sstride * (ep0.c_f32 ? 4 : 2);
       const int buf = local & 1;
       const uint32_t use = (uint32_t)(local >> 1);
       if (!mbar_wait(&acc_full[buf], use & 1)) break;
@@ -351,7 +306,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
             tmem_ld32(tq + h0 + j0, ra);
             tmem_ld32(tq + h0 + half + j0, rb);
             tmem_ld_wait();
-            epi_store_rope(ep, cz, row, n0 + h0 + j0, n0 + h0 + half + j0, j0, ra, rb);
+            epi_store_rope(ep, row, n0 + h0 + j0, n0 + h0 + half + j0, j0, ra, rb);
           }
         }
       } else {
@@ -360,47 +315,11 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           uint32_t r[32];
           tmem_ld32(tq + c, r);
           tmem_ld_wait();
-          epi_store(ep, cz, row, n0 + c, r);
+          epi_store(ep, row, n0 + c, r);
         }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);  // all 128 epilogue threads arrive once per tile
-      if (ep0.kout) {
-        // split-K: publish this partial tile; the last of the `splits` CTAs of the tile reduces
-        const int etid = threadIdx.x - 64;
-        __threadfence();  // this thread's partial stores, then the group barrier, then one release
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        int* sem = ep0.sem + (mi * sched.nt + ni);
-        if (etid == 0) {
-          __threadfence();
-          const int prev = atomicAdd(sem, 1);
-          __threadfence();  // acquire side for the reducer
-          *last_flag = (prev == total_tiles / sched.tiles_per_z - 1);
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (*last_flag) {
-          __threadfence();
-          const int nsplit = total_tiles / sched.tiles_per_z;
-          if (row < ep0.M) {
-            const float* base = static_cast<const float*>(ep0.C) + (int64_t)row * ep0.ldc;
-            for (int c = n0; c < n0 + BN && c < ep0.N; c += 4) {
-              // L2-coherent loads (bypass L1): the partials were written by other SMs
-              float4 acc = __ldcg(reinterpret_cast<const float4*>(base + c));
-              for (int zz = 1; zz < nsplit; ++zz) {
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(base + (int64_t)zz * ep0.sstride + c));
-                acc.x += v.x;
-                acc.y += v.y;
-                acc.z += v.z;
-                acc.w += v.w;
-              }
-              __nv_bfloat162 h[2] = {__floats2bfloat162_rn(ep0.kscale * acc.x, ep0.kscale * acc.y),
-                                     __floats2bfloat162_rn(ep0.kscale * acc.z, ep0.kscale * acc.w)};
-              *reinterpret_cast<uint2*>(ep0.kout + (int64_t)row * ep0.ldk + c) = *reinterpret_cast<const uint2*>(h);
-            }
-          }
-          if (etid == 0) *sem = 0;  // ready for the next launch
-        }
-      }
     }
   }
   tc_fence_before();
@@ -410,6 +329,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     tmem_dealloc(tmem, 2 * C::TMEM_COLS);
   }
 }
+
+}  // namespace
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -423,8 +344,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2D bf16 tensor map over a row-major [rows, cols] matrix with row stride ld (elements),
-// box = [box_rows, 64 columns], 128-byte swizzle, zero fill out of bounds.
 bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
@@ -437,6 +356,8 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int6
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <int BN, int AMN, int BMN>
 cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
@@ -455,7 +376,7 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   }
   int nk2 = 0;
   if (a.A2 && a.B2 && a.K2 > 0) {
-    if (AMN || a.splits > 1) return cudaErrorInvalidValue;
+    if (AMN) return cudaErrorInvalidValue;
     if (!make_map(&tA2, a.A2, a.M, a.K2, a.lda2, BM)) return cudaErrorInvalidValue;
     if (BMN) {
       if (!make_map(&tB2, a.B2, a.K2, a.N, a.ldb2, box_b)) return cudaErrorInvalidValue;
@@ -468,10 +389,7 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
     tB2 = tB;
   }
   Epi e{a.C, a.ldc, a.bias, a.R, a.ldr, a.alpha, a.c_f32, a.M, a.N,
-        a.rope_cos, a.rope_sin, a.rope_cos ? a.rope_end : 0, a.rope_hd, a.rope_S,
-        a.epi_mode, {a.sdst[0], a.sdst[1], a.sdst[2]}, a.sr, a.snseg,
-        {a.sbounds[0], a.sbounds[1], a.sbounds[2], a.sbounds[3]}, a.kout, a.ldk, a.kscale, a.sem,
-        a.split_stride};
+        a.rope_cos, a.rope_sin, a.rope_cos ? a.rope_end : 0, a.rope_hd, a.rope_S};
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t err =
@@ -480,16 +398,10 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
     attr_set = true;
   }
   const int nk1 = (a.K + BK - 1) / BK;
-  int splits = a.splits < 1 ? 1 : a.splits;
-  if (splits > nk1) splits = nk1;
-  const int kps = (nk1 + splits - 1) / splits;
-  splits = (nk1 + kps - 1) / kps;  // no empty split
-  if (splits > 1 && a.split_stride < (int64_t)a.M * a.ldc) return cudaErrorInvalidValue;
   TileSched sched;
   sched.mt = (a.M + BM - 1) / BM;
   sched.nt = (a.N + BN - 1) / BN;
-  sched.tiles_per_z = sched.mt * sched.nt;
-  const int total = sched.tiles_per_z * splits;
+  const int total = sched.mt * sched.nt;
   static int num_sms = 0;
   if (!num_sms) {
     int dev = 0;
@@ -498,7 +410,7 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
       num_sms = 148;
   }
   const int grid = total < num_sms ? total : num_sms;
-  k_gemm<BN, AMN, BMN><<<grid, 192, C::SMEM, s>>>(tA, tB, tA2, tB2, e, sched, total, nk1, nk2, kps);
+  k_gemm<BN, AMN, BMN><<<grid, 192, C::SMEM, s>>>(tA, tB, tA2, tB2, e, sched, total, nk1, nk2);
   note_launch(1);
   return cudaGetLastError();
 }
@@ -507,15 +419,11 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
 
 cudaError_t gemm_bf16(const GemmArgs& a, cudaStream_t s) {
   if (a.M <= 0 || a.N <= 0 || a.K <= 0 || !a.A || !a.B || !a.C) return cudaErrorInvalidValue;
-  if (a.splits > 1 && (a.bias || a.R || a.A2)) return cudaErrorInvalidValue;  // partials are summed later
-  if (a.kout && (!a.sem || !a.c_f32 || a.epi_mode || (a.N % 4) || (a.ldc % 4) || (a.ldk % 4))) return cudaErrorInvalidValue;
-  if (a.epi_mode && (a.splits > 1 || a.kout || a.rope_cos || a.sr <= 0 || a.snseg < 1 || a.snseg > 3))
-    return cudaErrorInvalidValue;
   // TMA: 16-byte aligned bases and row strides
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   if (!al16(a.A) || !al16(a.B) || (a.lda % 8) || (a.ldb % 8)) return cudaErrorInvalidValue;
   if (a.A2 && (!al16(a.A2) || !al16(a.B2) || (a.lda2 % 8) || (a.ldb2 % 8))) return cudaErrorInvalidValue;
-  const int64_t tiles256 = (int64_t)((a.M + BM - 1) / BM) * ((a.N + 255) / 256) * (a.splits > 1 ? a.splits : 1);
+  const int64_t tiles256 = (int64_t)((a.M + BM - 1) / BM) * ((a.N + 255) / 256);
   int bn;
   if (a.N <= 64) bn = 64;
   else if (a.N <= 128 || tiles256 < 120) bn = 128;
@@ -523,7 +431,7 @@ cudaError_t gemm_bf16(const GemmArgs& a, cudaStream_t s) {
   if (a.rope_cos) {
     // rotated columns: whole tiles of whole heads, bf16 output, no residual / split / MN-major A
     if (!a.rope_sin || (a.rope_hd != 64 && a.rope_hd != 128) || a.rope_S <= 0 || a.c_f32 || a.R ||
-        a.splits > 1 || a.a_mn || (a.ldc % 8) || (reinterpret_cast<uintptr_t>(a.C) & 15))
+        a.a_mn || (a.ldc % 8) || (reinterpret_cast<uintptr_t>(a.C) & 15))
       return cudaErrorInvalidValue;
     if (bn == 256 && (a.rope_end % 256)) bn = 128;
     if (bn < 128 || (a.rope_end % bn) || a.rope_end > a.N) return cudaErrorInvalidValue;

@@ -169,11 +169,24 @@ lst_status lst_k_cross_entropy(const float* logits, int64_t T, int32_t V, const 
 }
 
 lst_status lst_k_lora_skinny(const uint16_t* X, int64_t ldx, int64_t T, int32_t K, const uint16_t* Bop, int64_t ldb,
-                             int32_t b_mn, int32_t KP, float s, uint16_t* Us, float* scratch, int64_t scratch_floats,
-                             void* stream) {
-  if (!X || !Bop || !Us || !scratch || T <= 0 || K <= 0 || KP <= 0) return LST_ERR_ARG;
-  if (scratch_floats < lora_skinny_scratch(T, KP)) return LST_ERR_ARG;
-  return st(lora_skinny(B16(X), ldx, T, K, B16(Bop), ldb, b_mn ? 1 : 0, KP, s, scratch, B16(Us), S(stream)));
+                             int32_t b_mn, int32_t KP, float s, uint16_t* Us, void* stream) {
+  if (!X || !Bop || !Us || T <= 0 || K <= 0 || KP <= 0 || (KP % 8)) return LST_ERR_ARG;
+  return st(lora_skinny(B16(X), ldx, T, K, B16(Bop), ldb, b_mn ? 1 : 0, KP, s, B16(Us), S(stream)));
+}
+
+lst_status lst_k_lora_grads(const uint16_t* X, int64_t ldx, int32_t in, const uint16_t* dY, int64_t ldy,
+                            int32_t out, int64_t T, const uint16_t* Us, const uint16_t* Vs, int32_t KP, int32_t nseg,
+                            int32_t r, const int32_t* bounds, float* const* dA, float* const* dB, void* stream) {
+  if (!X || !dY || !Us || !Vs || !bounds || !dA || !dB || T <= 0 || in <= 0 || out <= 0) return LST_ERR_ARG;
+  if (nseg < 1 || nseg > 3 || r <= 0 || nseg * r > KP || (KP % 8)) return LST_ERR_ARG;
+  int b[4] = {0, 0, 0, 0};
+  for (int p = 0; p <= nseg; ++p) b[p] = bounds[p];
+  for (int p = 0; p < nseg; ++p)
+    if (!dA[p] || !dB[p] || b[p + 1] <= b[p]) return LST_ERR_ARG;
+  if (b[0] != 0 || b[nseg] != out) return LST_ERR_ARG;
+  const lst_status sa = st(lora_grad_a(B16(X), ldx, T, in, B16(Vs), KP, nseg, r, dA, S(stream)));
+  if (sa != LST_OK) return sa;
+  return st(lora_grad_b(B16(dY), ldy, T, out, B16(Us), KP, nseg, r, b, dB, S(stream)));
 }
 
 int64_t lst_k_launch_count(void) { return g_launch_count.load(); }

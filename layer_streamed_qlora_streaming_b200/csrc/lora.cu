@@ -6,10 +6,13 @@
 //   forward   U  = x Acat^T          [T, nseg*r]   (then s*U enters the base GEMM as extra K columns)
 //   backward  V  = dy Bexp            [T, nseg*r]  (s*V enters the dX GEMM the same way)
 //             dA = s V^T x,  dB = s dy^T U          (reductions over the T tokens)
-// All four are bf16 tcgen05 GEMMs with fp32 accumulation. U and V have only nseg*r <= 64 columns,
-// so they are split along K over many CTAs and the fp32 partials are summed in a fixed order; dA and
-// dB contract over tokens, with x / dy read as MN-major operands. Nothing uses atomics, so results
-// are deterministic.
+// Each of the four has one short side (nseg*r <= 64) and a long contraction (the in / out features,
+// or the T tokens), so one output tile holds little work and a plain tiling leaves most SMs idle.
+// One kernel serves all four: a 128 x 64 output tile is computed by a thread-block cluster of cs
+// CTAs, CTA z contracting K-slice z with bf16 tcgen05 MMAs into TMEM (fp32); the cs partial tiles
+// are then parked in shared memory and summed through distributed shared memory, each CTA summing
+// 128/cs rows in slice order 0, 1, ..., cs-1, and stored by the mode's epilogue. No atomics and no
+// global scratch: the result depends only on the shapes, so it is deterministic.
 #include "common.cuh"
 #include "gemm.cuh"
 #include "lora.cuh"
@@ -17,18 +20,244 @@
 namespace lst {
 namespace {
 
-constexpr int kMaxSplits = 16;
+constexpr int kBM = 128, kBN = 64, kBK = 64, kStages = 4, kMaxCluster = 8;
+constexpr uint32_t kABytes = kBM * kBK * 2;
+constexpr uint32_t kBBytes = kBN * kBK * 2;
+constexpr int kRedLd = kBN + 4;  // fp32 row stride of a parked partial tile (conflict-free float4 rows)
+constexpr uint32_t kSmem = kStages * (kABytes + kBBytes) + 1024 /*align*/ + 256 /*barriers*/;
+static_assert(kBM * kRedLd * 4 <= kStages * kABytes, "the partial tile reuses the A stages");
 
-int skinny_splits(int64_t T, int K) {
-  const int mtiles = (int)((T + 127) / 128);
-  int splits = (148 + mtiles - 1) / mtiles;
-  if (splits > kMaxSplits) splits = kMaxSplits;
-  const int nk = (K + 63) / 64;
-  if (splits > nk) splits = nk;
-  if (splits < 1) splits = 1;
-  const int kps = (nk + splits - 1) / splits;
-  return (nk + kps - 1) / kps;  // the same count the GEMM launch settles on (no empty split)
+// Destination of the summed tile C [M, N] (times scale).
+struct SideOut {
+  // 0: out16[row * ld + col] = bf16(c)                                      (U or V, [T, KP])
+  // 1: row p*r + j (< nseg*r) -> dst[p][j * N + col]                       (dA, [r, in] each)
+  // 2: row o of segment p, column p*r + j -> dst[p][(o - bounds[p]) * r + j] (dB, [out_p, r] each)
+  int mode;
+  int M, N;
+  float scale;
+  __nv_bfloat16* out16;
+  int64_t ld;
+  float* dst[3];
+  int r, nseg;
+  int bounds[4];
+};
+
+__device__ __forceinline__ void side_store(const SideOut& o, int row, int col, float4 v) {
+  if (row >= o.M || col >= o.N) return;
+  const float a[4] = {o.scale * v.x, o.scale * v.y, o.scale * v.z, o.scale * v.w};
+  const bool full = col + 4 <= o.N;
+  if (o.mode == 0) {
+    __nv_bfloat16* p = o.out16 + (int64_t)row * o.ld + col;
+    if (full && (reinterpret_cast<uintptr_t>(p) & 7) == 0) {
+      const __nv_bfloat162 h[2] = {__floats2bfloat162_rn(a[0], a[1]), __floats2bfloat162_rn(a[2], a[3])};
+      *reinterpret_cast<uint2*>(p) = *reinterpret_cast<const uint2*>(h);
+    } else {
+      for (int i = 0; i < 4; ++i)
+        if (col + i < o.N) p[i] = __float2bfloat16_rn(a[i]);
+    }
+  } else if (o.mode == 1) {
+    if (row >= o.nseg * o.r) return;
+    const int p = row / o.r;
+    float* d = o.dst[p] + (int64_t)(row - p * o.r) * o.N + col;
+    if (full && (reinterpret_cast<uintptr_t>(d) & 15) == 0) {
+      *reinterpret_cast<float4*>(d) = make_float4(a[0], a[1], a[2], a[3]);
+    } else {
+      for (int i = 0; i < 4; ++i)
+        if (col + i < o.N) d[i] = a[i];
+    }
+  } else {
+    int p = 0;
+    while (p + 1 < o.nseg && row >= o.bounds[p + 1]) ++p;
+    float* d = o.dst[p] + (int64_t)(row - o.bounds[p]) * o.r;
+    for (int i = 0; i < 4; ++i) {
+      const int j = col + i - p * o.r;
+      if (col + i < o.N && j >= 0 && j < o.r) d[j] = a[i];
+    }
+  }
 }
+
+// grid (cs, ceil(M/128), ceil(N/64)), cluster (cs, 1, 1), 192 threads: warp 0 TMA producer, warp 1
+// TMEM owner + MMA issuer, warps 2-5 park the accumulator; then all threads sum and store.
+// AMN / BMN: A / B MN-major ([K, M] / [K, N] row-major in memory), else K-major.
+template <int AMN, int BMN>
+__global__ void __launch_bounds__(192, 2)
+k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const SideOut o,
+       const int nk, const int kps) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * kBBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  float* red = reinterpret_cast<float*>(smem);  // parked partial tile, once the last MMA has read sA
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int cs = (int)gridDim.x;  // one cluster = the K slices of one output tile
+  const int z = (int)cluster_rank();
+  const int m0 = blockIdx.y * kBM, n0 = blockIdx.z * kBN;
+  const int kb0 = z * kps;
+  const int nkb = max(0, min(nk - kb0, kps));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kBN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (kb / kStages) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1)) break;
+        mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
+        const int kk = (kb0 + kb) * kBK;
+        if (AMN == 0) {
+          tma_load_2d(sA + s * kABytes, &tmA, &full[s], kk, m0);
+        } else {
+          tma_load_2d(sA + s * kABytes, &tmA, &full[s], m0, kk);
+          tma_load_2d(sA + s * kABytes + 64 * kBK * 2, &tmA, &full[s], m0 + 64, kk);
+        }
+        if (BMN == 0) {
+          tma_load_2d(sB + s * kBBytes, &tmB, &full[s], kk, n0);
+        } else {
+          tma_load_2d(sB + s * kBBytes, &tmB, &full[s], n0, kk);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && nkb > 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(kBM, kBN, AMN, BMN);
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (kb / kStages) & 1;
+        if (!mbar_wait(&full[s], ph)) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s * kABytes);
+        const uint32_t b0 = smem_u32(sB + s * kBBytes);
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          const uint64_t da = AMN ? umma_desc(a0 + k * 16 * 128, 64 * kBK * 2, 1024) : umma_desc(a0 + k * 32, 16, 1024);
+          const uint64_t db = BMN ? umma_desc(b0 + k * 16 * 128, 64 * kBK * 2, 1024) : umma_desc(b0 + k * 32, 16, 1024);
+          umma_bf16(tmem, da, db, idesc, (kb | k) != 0);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(acc_full);  // arrives once every MMA issued above has completed
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    float* rr = red + (q * 32 + lane) * kRedLd;
+    if (nkb > 0) {
+      mbar_wait(acc_full, 0);
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < kBN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + (uint32_t)c + ((uint32_t)(q * 32) << 16), r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(rr + c + i) = make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                                                               __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+      }
+    } else {
+      for (int c = 0; c < kBN; c += 4) *reinterpret_cast<float4*>(rr + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();  // every slice's partial tile is parked
+
+  // CTA z sums rows [z * 128/cs, (z + 1) * 128/cs) over the slices in order 0 .. cs-1
+  const int rows = kBM / cs;
+  const int r0 = z * rows;
+  const uint32_t red0 = smem_u32(red);
+  for (int f = threadIdx.x; f < rows * (kBN / 4); f += blockDim.x) {
+    const int rl = r0 + f / (kBN / 4);
+    const int c = (f % (kBN / 4)) * 4;
+    const uint32_t a = red0 + (uint32_t)((rl * kRedLd + c) * 4);
+    float4 acc = ld_cluster_f4(cluster_map(a, 0));
+    for (int p = 1; p < cs; ++p) {
+      const float4 v = ld_cluster_f4(cluster_map(a, (uint32_t)p));
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    side_store(o, m0 + rl, n0 + c, acc);
+  }
+  __syncwarp();
+  cluster_sync_all();  // no CTA leaves while another still reads its shared memory
+  __syncwarp();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBN);
+  }
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int AMN, int BMN>
+cudaError_t launch_side(const CUtensorMap& tA, const CUtensorMap& tB, int M, int N, int K, const SideOut& o,
+                        cudaStream_t st) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(k_side<AMN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int mt = (M + kBM - 1) / kBM, nt = (N + kBN - 1) / kBN, nk = (K + kBK - 1) / kBK;
+  if (mt > 65535 || nt > 65535) return cudaErrorInvalidValue;
+  // widest cluster (K split) that keeps every CTA resident at two per SM
+  const int64_t slots = 2 * (int64_t)sm_count();
+  int cs = 1;
+  while (cs < kMaxCluster && (int64_t)mt * nt * cs * 2 <= slots && cs * 2 <= nk) cs *= 2;
+  const int kps = (nk + cs - 1) / cs;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)cs, (unsigned)mt, (unsigned)nt);
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)cs;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_side<AMN, BMN>, tA, tB, o, nk, kps);
+  note_launch(1);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 __global__ void k_lora_prep(const LoraPrepArgs a) {
   const int R = a.nseg * a.r;
@@ -51,85 +280,66 @@ __global__ void k_lora_prep(const LoraPrepArgs a) {
   }
 }
 
-inline unsigned nblk(int64_t n) { return (unsigned)((n + 255) / 256); }
-
 }  // namespace
 
-// fp32 partials of up to kMaxSplits splits, then one int semaphore per 128-row tile
-int64_t lora_skinny_scratch(int64_t T, int KP) { return (int64_t)kMaxSplits * T * KP + (T + 127) / 128 + 4; }
-
 cudaError_t lora_skinny(const __nv_bfloat16* X, int64_t ldx, int64_t T, int K, const __nv_bfloat16* Bop,
-                        int64_t ldb, int b_mn, int KP, float s, float* part, __nv_bfloat16* Us, cudaStream_t st) {
-  if (T <= 0 || K <= 0 || KP <= 0 || KP > 256) return cudaErrorInvalidValue;
-  const int splits = skinny_splits(T, K);
-  GemmArgs a;
-  a.M = (int)T;
-  a.N = KP;
-  a.K = K;
-  a.A = X;
-  a.lda = ldx;
-  a.B = Bop;
-  a.ldb = ldb;
-  a.b_mn = b_mn;
-  a.C = part;
-  a.ldc = KP;
-  a.c_f32 = 1;
-  a.splits = splits;
-  a.split_stride = T * KP;
-  a.kout = Us;  // reduced in the kernel by the last split of each tile, in split order
-  a.ldk = KP;
-  a.kscale = s;
-  a.sem = reinterpret_cast<int*>(part + (int64_t)kMaxSplits * T * KP);
-  return gemm_bf16(a, st);
+                        int64_t ldb, int b_mn, int KP, float s, __nv_bfloat16* Us, cudaStream_t st) {
+  if (T <= 0 || T > INT32_MAX || K <= 0 || KP <= 0 || KP % 8 || !X || !Bop || !Us) return cudaErrorInvalidValue;
+  if (!al16(X) || !al16(Bop) || (ldx % 8) || (ldb % 8)) return cudaErrorInvalidValue;
+  CUtensorMap tA, tB;
+  if (!make_map(&tA, X, T, K, ldx, kBM)) return cudaErrorInvalidValue;
+  if (b_mn) {
+    if (!make_map(&tB, Bop, K, KP, ldb, kBK)) return cudaErrorInvalidValue;
+  } else {
+    if (!make_map(&tB, Bop, KP, K, ldb, kBN)) return cudaErrorInvalidValue;
+  }
+  SideOut o{};
+  o.mode = 0;
+  o.M = (int)T;
+  o.N = KP;
+  o.scale = s;
+  o.out16 = Us;
+  o.ld = KP;
+  return b_mn ? launch_side<0, 1>(tA, tB, (int)T, KP, K, o, st) : launch_side<0, 0>(tA, tB, (int)T, KP, K, o, st);
 }
 
 cudaError_t lora_grad_a(const __nv_bfloat16* X, int64_t ldx, int64_t T, int in, const __nv_bfloat16* Vs, int KP,
-                        int nseg, int r, float* const* dst, float* part, cudaStream_t st) {
-  if (nseg < 1 || nseg > 3 || nseg * r > KP) return cudaErrorInvalidValue;
-  GemmArgs a;
-  a.M = in;
-  a.N = KP;
-  a.K = (int)T;
-  a.A = X;
-  a.lda = ldx;
-  a.a_mn = 1;
-  a.B = Vs;
-  a.ldb = KP;
-  a.b_mn = 1;
-  a.C = dst[0];  // not written: the epilogue scatters straight into the per-segment dA
-  a.ldc = KP;
-  a.c_f32 = 1;
-  a.epi_mode = 1;
-  for (int k = 0; k < nseg; ++k) a.sdst[k] = dst[k];
-  a.sr = r;
-  a.snseg = nseg;
-  (void)part;
-  return gemm_bf16(a, st);
+                        int nseg, int r, float* const* dst, cudaStream_t st) {
+  if (nseg < 1 || nseg > 3 || r <= 0 || nseg * r > KP || KP % 8 || T <= 0 || in <= 0) return cudaErrorInvalidValue;
+  if (!al16(X) || !al16(Vs) || (ldx % 8)) return cudaErrorInvalidValue;
+  // C [KP, in] = Vs^T X: A = Vs read MN-major ([T, KP]), B = X read MN-major ([T, in])
+  CUtensorMap tA, tB;
+  if (!make_map(&tA, Vs, T, KP, KP, kBK)) return cudaErrorInvalidValue;
+  if (!make_map(&tB, X, T, in, ldx, kBK)) return cudaErrorInvalidValue;
+  SideOut o{};
+  o.mode = 1;
+  o.M = KP;
+  o.N = in;
+  o.scale = 1.0f;
+  for (int k = 0; k < nseg; ++k) o.dst[k] = dst[k];
+  o.r = r;
+  o.nseg = nseg;
+  return launch_side<1, 1>(tA, tB, KP, in, (int)T, o, st);
 }
 
 cudaError_t lora_grad_b(const __nv_bfloat16* dY, int64_t ldy, int64_t T, int out, const __nv_bfloat16* Us, int KP,
-                        int nseg, int r, const int* bounds, float* const* dst, float* part, cudaStream_t st) {
-  if (nseg < 1 || nseg > 3 || nseg * r > KP) return cudaErrorInvalidValue;
-  GemmArgs a;
-  a.M = out;
-  a.N = KP;
-  a.K = (int)T;
-  a.A = dY;
-  a.lda = ldy;
-  a.a_mn = 1;
-  a.B = Us;
-  a.ldb = KP;
-  a.b_mn = 1;
-  a.C = dst[0];  // not written: the epilogue keeps each row's own segment and stores it as dB
-  a.ldc = KP;
-  a.c_f32 = 1;
-  a.epi_mode = 2;
-  for (int k = 0; k < nseg; ++k) a.sdst[k] = dst[k];
-  for (int k = 0; k <= nseg; ++k) a.sbounds[k] = bounds[k];
-  a.sr = r;
-  a.snseg = nseg;
-  (void)part;
-  return gemm_bf16(a, st);
+                        int nseg, int r, const int* bounds, float* const* dst, cudaStream_t st) {
+  if (nseg < 1 || nseg > 3 || r <= 0 || nseg * r > KP || KP % 8 || T <= 0 || out <= 0) return cudaErrorInvalidValue;
+  if (!al16(dY) || !al16(Us) || (ldy % 8) || bounds[0] != 0 || bounds[nseg] != out) return cudaErrorInvalidValue;
+  // C [out, KP] = dY^T Us: A = dY read MN-major ([T, out]), B = Us read MN-major ([T, KP])
+  CUtensorMap tA, tB;
+  if (!make_map(&tA, dY, T, out, ldy, kBK)) return cudaErrorInvalidValue;
+  if (!make_map(&tB, Us, T, KP, KP, kBK)) return cudaErrorInvalidValue;
+  SideOut o{};
+  o.mode = 2;
+  o.M = out;
+  o.N = KP;
+  o.scale = 1.0f;
+  for (int k = 0; k < nseg; ++k) o.dst[k] = dst[k];
+  for (int k = 0; k <= nseg; ++k) o.bounds[k] = bounds[k];
+  o.r = r;
+  o.nseg = nseg;
+  return launch_side<1, 1>(tA, tB, out, KP, (int)T, o, st);
 }
 
 cudaError_t lora_prep(const LoraPrepArgs& a, cudaStream_t st) {

@@ -259,19 +259,52 @@ def test_lora_skinny(T, K, b_mn):
         Bop = np.zeros((64, K), np.float32)
         Bop[:R] = _bf(r.normal(size=(R, K)) * 0.05)
         ref = 2.0 * X.astype(np.float64) @ Bop.T.astype(np.float64)
-    Us = torch.zeros(T, 64, dtype=torch.bfloat16, device="cuda")
-    scratch = torch.zeros(16 * T * 64 + (T + 127) // 128 + 4, dtype=torch.float32, device="cuda")
+    Us = torch.full((T, 64), float("nan"), dtype=torch.bfloat16, device="cuda")
     outs = []
-    for _ in range(2):  # twice: the tile counters must come back to zero, results identical
-        lst.k_lora_skinny(torch_bf16(X), K, T, K, torch_bf16(Bop), 64 if b_mn else K, b_mn, 64, 2.0, Us, scratch)
+    for _ in range(2):  # twice: identical bytes (fixed-order reduction over the K slices)
+        lst.k_lora_skinny(torch_bf16(X), K, T, K, torch_bf16(Bop), 64 if b_mn else K, b_mn, 64, 2.0, Us)
         torch.cuda.synchronize()
         outs.append(Us.view(torch.int16).cpu().numpy().copy())
         assert maxrel(to_np(Us), ref) < 8e-3, (len(outs), maxrel(to_np(Us), ref))
     assert np.array_equal(outs[0], outs[1])
-    assert np.all(scratch[16 * T * 64:].cpu().numpy() == 0)
     got = to_np(Us)
     assert maxrel(got, ref) < 8e-3
     assert np.all(got[:, R:] == 0)
+
+
+@pytest.mark.parametrize("T,in_f,bounds,r", [
+    (2048, 4096, [0, 4096, 5120, 6144], 16),   # q/k/v of an 8B layer
+    (2048, 14336, [0, 4096], 16),              # down of an 8B layer
+    (300, 688, [0, 688, 1376], 8),             # gate/up of the tiny stack, ragged token count
+    (128, 256, [0, 256], 8),
+])
+def test_lora_grads(T, in_f, bounds, r):
+    # dA_p = Vs_p^T X and dB_p = dY_p^T Us_p over the T tokens, every element written, same bytes twice
+    rng = _rng(T + in_f + r)
+    nseg, out_f, KP = len(bounds) - 1, bounds[-1], 64
+    R = nseg * r
+    X = _bf(rng.normal(size=(T, in_f)))
+    dY = _bf(rng.normal(size=(T, out_f)) * 0.1)
+    Us = np.zeros((T, KP), np.float32)
+    Us[:, :R] = _bf(rng.normal(size=(T, R)))
+    Vs = np.zeros((T, KP), np.float32)
+    Vs[:, :R] = _bf(rng.normal(size=(T, R)))
+    dA = [torch.full((r, in_f), float("nan"), device="cuda") for _ in range(nseg)]
+    dB = [torch.full((bounds[p + 1] - bounds[p], r), float("nan"), device="cuda") for p in range(nseg)]
+    outs = []
+    for _ in range(2):
+        lst.k_lora_grads(torch_bf16(X), in_f, in_f, torch_bf16(dY), out_f, out_f, T, torch_bf16(Us), torch_bf16(Vs),
+                         KP, r, bounds, dA, dB)
+        torch.cuda.synchronize()
+        outs.append([t.cpu().numpy().copy() for t in dA + dB])
+    for a, b in zip(*outs):
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    X64, dY64 = X.astype(np.float64), dY.astype(np.float64)
+    for p in range(nseg):
+        refA = Vs[:, p * r:(p + 1) * r].astype(np.float64).T @ X64
+        refB = dY64[:, bounds[p]:bounds[p + 1]].T @ Us[:, p * r:(p + 1) * r].astype(np.float64)
+        assert maxrel(to_np(dA[p]), refA) < 1e-4, (p, maxrel(to_np(dA[p]), refA))
+        assert maxrel(to_np(dB[p]), refB) < 1e-4, (p, maxrel(to_np(dB[p]), refB))
 
 
 @pytest.mark.parametrize("M,N,K", [(4096, 64, 2048), (304, 64, 200), (6144, 64, 512)])
