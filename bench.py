@@ -357,6 +357,31 @@ def run_gpu(args, wl):
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": n_grad * 4 + 4,
            "path": "lst_step with pinned host inputs and host gradient buffer (copies inside the call)"}
 
+    # the reuse schedule (layers still in the pool are not copied again): same results, fewer bytes
+    ctx.set_reuse(True)
+    for _ in range(2):
+        one_step()
+    torch.cuda.synchronize()
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    r0.record(stream)
+    for _ in range(args.steps):
+        one_step()
+    r1.record(stream)
+    torch.cuda.synchronize()
+    rms = max_over_ranks(r0.elapsed_time(r1), dist, "cuda")
+    rst = ctx.stats()
+    ctx.set_reuse(False)
+    reuse_bytes = rst["h2d_bytes_last_step"]
+    reuse = {"value": job_throughput(world, T, args.steps, rms), "unit": UNIT, "ms_per_step": rms / args.steps,
+             "layer_reads_per_step": rst["layer_reads_last_step"], "h2d_bytes_per_step": reuse_bytes,
+             "min_ms": reuse_bytes / (link_gbs * 1e9) * 1e3,
+             "frac": reuse_bytes / (link_gbs * 1e9) * 1e3 / (rms / args.steps),
+             "note": "steady state: the two layers at the forward/backward turn and layers 0, 1 from the "
+                     "previous step are not copied again (2L - 4 reads)"}
+
     st = ctx.stats()
     peaks = measured_peaks()
     K = args.steps
@@ -393,6 +418,7 @@ def run_gpu(args, wl):
         "clocks": clk.summary(),
     }
     line["e2e"] = e2e
+    line["reuse_schedule"] = reuse
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, secs, desc = oracle_sample(wl, seq=args.ref_seq)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",

@@ -80,6 +80,12 @@ typedef struct {
                            device pool on a dedicated copy stream; 0: all layers resident on the
                            device (same kernels, same results) */
   int32_t timeout_ms;   /* host-side wait limit of one step; <= 0 means 600000 */
+  int32_t head_chunk;   /* LM head + cross-entropy in passes of this many token rows, so logits
+                           [rows, V] are never resident for the whole batch; <= 0: one pass.
+                           The result does not depend on it. */
+  int32_t reuse;        /* 1: a layer still in the pool is not copied again (the two layers at the
+                           forward/backward turn, and layers 0, 1 from the end of the previous
+                           step); 0: every read copies (2L reads per step). Same results. */
 } lst_config;
 
 typedef struct {
@@ -178,6 +184,10 @@ lst_status lst_get_activation(lst_ctx* ctx, int32_t which, int32_t layer, void* 
 
 /* Record per-class device times of every step (CUDA events around each launch) when on != 0. */
 lst_status lst_set_profiling(lst_ctx* ctx, int32_t on);
+
+/* Switch the copy schedule of the next steps (the config's `reuse`): 1 keeps layers that are still
+ * in the pool instead of copying them again, 0 copies every read. Results are the same bytes. */
+lst_status lst_set_reuse(lst_ctx* ctx, int32_t reuse);
 lst_status lst_get_stats(const lst_ctx* ctx, lst_stats* out);
 
 const char* lst_last_error(const lst_ctx* ctx);

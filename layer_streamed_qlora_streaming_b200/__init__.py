@@ -30,7 +30,8 @@ class Config(C.Structure):
                 ("vocab", C.c_int32), ("rms_eps", C.c_float), ("rope_theta", C.c_float),
                 ("qkv_bias", C.c_int32), ("lora_rank", C.c_int32), ("lora_alpha", C.c_float),
                 ("base_format", C.c_int32), ("max_batch", C.c_int32), ("max_seq", C.c_int32),
-                ("streamed", C.c_int32), ("timeout_ms", C.c_int32)]
+                ("streamed", C.c_int32), ("timeout_ms", C.c_int32), ("head_chunk", C.c_int32),
+                ("reuse", C.c_int32)]
 
 
 class LayerWeights(C.Structure):
@@ -71,6 +72,7 @@ _SIGS = {
     "lst_get_logits": (_I32, [_P, _P]),
     "lst_get_activation": (_I32, [_P, _I32, _I32, _P]),
     "lst_set_profiling": (_I32, [_P, _I32]),
+    "lst_set_reuse": (_I32, [_P, _I32]),
     "lst_get_stats": (_I32, [_P, C.POINTER(Stats)]),
     "lst_last_error": (C.c_char_p, [_P]),
     "lst_destroy": (None, [_P]),
@@ -159,12 +161,14 @@ def nf4_codebook():
     return np.array(list(out), dtype=np.float32)
 
 
-def make_config(wl, streamed: bool = True, max_batch=None, max_seq=None, timeout_ms: int = 600000) -> Config:
+def make_config(wl, streamed: bool = True, max_batch=None, max_seq=None, timeout_ms: int = 600000,
+                head_chunk: int = 0, reuse: bool = False) -> Config:
     """lst_config of a synthetic.Workload-like object."""
     return Config(wl.n_layers, wl.d_model, wl.n_heads, wl.n_kv_heads, wl.head_dim, wl.ffn, wl.vocab,
                   wl.rms_eps, wl.rope_theta, int(wl.qkv_bias), wl.lora_rank, wl.lora_alpha,
                   BASE_NF4 if wl.base_format == "nf4" else BASE_BF16,
-                  max_batch or wl.batch, max_seq or wl.seq, int(streamed), timeout_ms)
+                  max_batch or wl.batch, max_seq or wl.seq, int(streamed), timeout_ms, int(head_chunk),
+                  int(bool(reuse)))
 
 
 def blob_bytes(cfg: Config) -> int:
@@ -243,6 +247,9 @@ class Context:
 
     def set_profiling(self, on: bool) -> None:
         _check(lib().lst_set_profiling(self.h, int(on)), self.h, "lst_set_profiling")
+
+    def set_reuse(self, on: bool) -> None:
+        _check(lib().lst_set_reuse(self.h, int(on)), self.h, "lst_set_reuse")
 
     def stats(self) -> dict:
         s = Stats()

@@ -163,6 +163,13 @@ enum { PC_GEMM = 0, PC_ATTN = 1, PC_DEQ = 2, PC_OTHER = 3, PC_COPY = 4, PC_LORA 
 
 }  // namespace
 
+struct ReadPlan {
+  int slot = 0;         // pool slot the read computes from
+  bool copy = true;     // the layer is copied into the slot for this read
+  int wait_free = -1;   // the copy waits for this read's compute to finish (-1: nothing to wait for)
+  int loaded_by = -1;   // read whose copy filled the slot (-1: filled by an earlier step)
+};
+
 struct lst_ctx {
   lst_config cfg{};
   int dev = 0;
@@ -208,12 +215,20 @@ struct lst_ctx {
   __nv_bfloat16* nf = nullptr;
   float *rstdf = nullptr, *logits = nullptr, *loss_rows = nullptr, *loss_dev = nullptr, *dot_part = nullptr;
   __nv_bfloat16* dlog = nullptr;
+  int64_t head_rows = 0;      // token rows per head pass (logits / dlogits buffers hold this many)
+  bool logits_whole = false;  // the last step's logits are all in `logits`
   __nv_bfloat16* gbuf = nullptr;
   int32_t *tok = nullptr, *tgt = nullptr;
   float *cos_t = nullptr, *sin_t = nullptr;
   float* host_loss = nullptr;
 
   std::vector<cudaEvent_t> ev_loaded, ev_free;
+  // pool slot use per read (see plan_reads)
+  std::vector<ReadPlan> plan;
+  int plan_held[2] = {-1, -1};   // layers the slots hold once the planned step has run
+  int slot_layer[2] = {-1, -1};  // layers the slots hold after the last completed step (-1: unknown)
+  int w_layer = -1;              // layer whose dequantised weights the scratch holds (-1: unknown)
+  int pending_w_layer = -1;
   cudaEvent_t ev_done = nullptr;
 
   float* stage_w = nullptr;
@@ -554,6 +569,9 @@ lst_status layer_bwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
   return LST_OK;
 }
 
+// Final RMSNorm, LM head, cross-entropy and the head's backward, in passes of at most head_rows
+// token rows: logits [rows, V] fp32 and dlogits [rows, V] bf16 exist for one pass at a time. Every
+// row is independent, so the result does not depend on the pass size.
 lst_status head_fwd_bwd(lst_ctx* c) {
   const int64_t T = c->curT;
   const float* xL = c->xs + (int64_t)c->L * c->Tmax * c->d;
@@ -561,56 +579,108 @@ lst_status head_fwd_bwd(lst_ctx* c) {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(rmsnorm_fwd(xL, c->gf, T, c->d, c->cfg.rms_eps, c->nf, c->rstdf, c->stream));
   }
-  {
-    GemmArgs a;
-    a.M = (int)T;
-    a.N = c->V;
-    a.K = c->d;
-    a.A = c->nf;
-    a.lda = c->d;
-    a.B = c->H;
-    a.ldb = c->d;
-    a.b_mn = 0;
-    a.C = c->logits;
-    a.ldc = c->V;
-    a.c_f32 = 1;
-    ProfScope ps(c, c->stream, PC_GEMM, 2.0 * T * c->V * (double)c->d);
-    CK(gemm_bf16(a, c->stream));
-  }
-  {
-    ProfScope ps(c, c->stream, PC_OTHER);
-    CK(cross_entropy(c->logits, T, c->V, c->tgt, 1.0f / (float)T, c->loss_rows, c->dlog, c->stream));
-    CK(mean_fixed(c->loss_rows, T, c->loss_dev, c->stream));
-  }
-  {
-    GemmArgs a;
-    a.M = (int)T;
-    a.N = c->d;
-    a.K = c->V;
-    a.A = c->dlog;
-    a.lda = c->V;
-    a.B = c->H;
-    a.ldb = c->d;
-    a.b_mn = 1;
-    a.C = c->dn;
-    a.ldc = c->d;
-    a.c_f32 = 1;
-    ProfScope ps(c, c->stream, PC_GEMM, 2.0 * T * c->V * (double)c->d);
-    CK(gemm_bf16(a, c->stream));
+  for (int64_t r0 = 0; r0 < T; r0 += c->head_rows) {
+    const int64_t rows = std::min<int64_t>(c->head_rows, T - r0);
+    {
+      GemmArgs a;
+      a.M = (int)rows;
+      a.N = c->V;
+      a.K = c->d;
+      a.A = c->nf + r0 * c->d;
+      a.lda = c->d;
+      a.B = c->H;
+      a.ldb = c->d;
+      a.b_mn = 0;
+      a.C = c->logits;
+      a.ldc = c->V;
+      a.c_f32 = 1;
+      ProfScope ps(c, c->stream, PC_GEMM, 2.0 * rows * c->V * (double)c->d);
+      CK(gemm_bf16(a, c->stream));
+    }
+    {
+      ProfScope ps(c, c->stream, PC_OTHER);
+      CK(cross_entropy(c->logits, rows, c->V, c->tgt + r0, 1.0f / (float)T, c->loss_rows + r0, c->dlog, c->stream));
+    }
+    {
+      GemmArgs a;
+      a.M = (int)rows;
+      a.N = c->d;
+      a.K = c->V;
+      a.A = c->dlog;
+      a.lda = c->V;
+      a.B = c->H;
+      a.ldb = c->d;
+      a.b_mn = 1;
+      a.C = c->dn + r0 * c->d;
+      a.ldc = c->d;
+      a.c_f32 = 1;
+      ProfScope ps(c, c->stream, PC_GEMM, 2.0 * rows * c->V * (double)c->d);
+      CK(gemm_bf16(a, c->stream));
+    }
   }
   ProfScope ps(c, c->stream, PC_OTHER);
+  CK(mean_fixed(c->loss_rows, T, c->loss_dev, c->stream));
   CK(rmsnorm_bwd(c->dn, xL, c->gf, c->rstdf, nullptr, T, c->d, c->ga, c->dout_b, c->stream));
+  c->logits_whole = T <= c->head_rows;
   return LST_OK;
+}
+
+// Reads n = 0 .. 2L-1 visit layer j(n) = n < L ? n : 2L-1-n (forward, then backward with
+// recompute). plan_reads decides, for each read, the pool slot it computes from and whether the
+// layer is copied into that slot first:
+//  - reuse off: every read copies, into slot n % 2 (2L copies per step);
+//  - reuse on: a read whose layer is still held by a slot (the two layers at the forward/backward
+//    turn; layers 0 and 1 left by the previous step's backward) uses it as it is; otherwise it copies
+//    into the slot the previous read does not use (for read 0, the slot whose layer is needed last).
+// A copy into a slot waits until the last read that computed from that slot has finished.
+void plan_reads(lst_ctx* c) {
+  const int L = c->L, R = 2 * L;
+  const bool reuse = c->cfg.reuse != 0;
+  auto layer_of = [L](int n) { return n < L ? n : 2 * L - 1 - n; };
+  int held[2] = {reuse ? c->slot_layer[0] : -1, reuse ? c->slot_layer[1] : -1};
+  int last_use[2] = {-1, -1}, loaded_by[2] = {-1, -1};
+  c->plan.assign(R, ReadPlan{});
+  for (int n = 0; n < R; ++n) {
+    const int j = layer_of(n);
+    ReadPlan& p = c->plan[n];
+    p.slot = -1;
+    if (reuse) {
+      if (held[0] == j) p.slot = 0;
+      else if (held[1] == j) p.slot = 1;
+    }
+    p.copy = p.slot < 0;
+    if (p.copy) {
+      if (n > 0) {
+        p.slot = 1 - c->plan[n - 1].slot;
+      } else {
+        int next[2] = {R, R};  // first read that needs the held layer
+        for (int s = 0; s < 2; ++s)
+          for (int m = 0; m < R; ++m)
+            if (layer_of(m) == held[s]) {
+              next[s] = m;
+              break;
+            }
+        p.slot = next[1] > next[0] ? 1 : 0;
+      }
+      p.wait_free = last_use[p.slot];
+      held[p.slot] = j;
+      loaded_by[p.slot] = n;
+    }
+    p.loaded_by = loaded_by[p.slot];
+    last_use[p.slot] = n;
+  }
+  c->plan_held[0] = held[0];
+  c->plan_held[1] = held[1];
 }
 
 lst_status enqueue_copy(lst_ctx* c, int n) {
   const int L = c->L;
   const int j = n < L ? n : 2 * L - 1 - n;
-  const int b = n & 1;
+  const ReadPlan& p = c->plan[n];
   if (c->faults.fail_memcpy()) return fail(c, LST_ERR_CUDA, "layer copy enqueue failed (injected)");
-  if (n >= 2) CK(cudaStreamWaitEvent(c->copy_stream, c->ev_free[n - 2], 0));
+  if (p.wait_free >= 0) CK(cudaStreamWaitEvent(c->copy_stream, c->ev_free[p.wait_free], 0));
   ProfScope ps(c, c->copy_stream, PC_COPY);
-  CK(cudaMemcpyAsync(c->pool[b], c->arena + (int64_t)j * c->lay.total, c->lay.total, cudaMemcpyHostToDevice,
+  CK(cudaMemcpyAsync(c->pool[p.slot], c->arena + (int64_t)j * c->lay.total, c->lay.total, cudaMemcpyHostToDevice,
                      c->copy_stream));
   CK(cudaEventRecord(c->ev_loaded[n], c->copy_stream));
   c->st.layer_reads_last_step += 1;
@@ -618,19 +688,45 @@ lst_status enqueue_copy(lst_ctx* c, int n) {
   return LST_OK;
 }
 
+// Enqueue, in read order, every planned copy whose slot is released by a read <= done.
+lst_status issue_copies(lst_ctx* c, int done, int& next) {
+  const int R = 2 * c->L;
+  while (next < R) {
+    const ReadPlan& p = c->plan[next];
+    if (p.copy) {
+      if (p.wait_free > done) break;
+      TRY(enqueue_copy(c, next));
+    }
+    ++next;
+  }
+  return LST_OK;
+}
+
 lst_status run_layers(lst_ctx* c, bool head) {
   const int L = c->L;
   const bool streamed = c->cfg.streamed != 0;
+  const bool reuse = streamed && c->cfg.reuse != 0;
+  int next_copy = 0;
   if (streamed) {
-    TRY(enqueue_copy(c, 0));
-    if (2 * L > 1) TRY(enqueue_copy(c, 1));
+    plan_reads(c);
+    // the slots' contents are only trusted again once this step has completed
+    c->slot_layer[0] = c->slot_layer[1] = -1;
+    TRY(issue_copies(c, -1, next_copy));
   }
+  const int w_held = c->w_layer;
+  c->w_layer = -1;
+  int w_now = reuse ? w_held : -1;
   for (int n = 0; n < 2 * L; ++n) {
     const int j = n < L ? n : 2 * L - 1 - n;
-    const uint8_t* blob = streamed ? c->pool[n & 1] : c->resident + (int64_t)j * c->lay.total;
-    if (streamed) CK(cudaStreamWaitEvent(c->stream, c->ev_loaded[n], 0));
+    const uint8_t* blob = streamed ? c->pool[c->plan[n].slot] : c->resident + (int64_t)j * c->lay.total;
+    if (streamed && c->plan[n].loaded_by >= 0) CK(cudaStreamWaitEvent(c->stream, c->ev_loaded[c->plan[n].loaded_by], 0));
     const __nv_bfloat16* W = nullptr;
-    TRY(layer_weights(c, blob, &W));
+    if (reuse && c->cfg.base_format != LST_BASE_BF16 && w_now == j) {
+      W = c->wscr;  // the dequantised copy of this layer is still in the scratch
+    } else {
+      TRY(layer_weights(c, blob, &W));
+      w_now = j;
+    }
     if (n < L) {
       TRY(layer_fwd(c, j, blob, W, false));
     } else {
@@ -650,8 +746,9 @@ lst_status run_layers(lst_ctx* c, bool head) {
         CK(bf16_to_f32(c->gbuf, T * c->d, c->ga, c->stream));
       }
     }
-    if (streamed && n + 2 < 2 * L) TRY(enqueue_copy(c, n + 2));
+    if (streamed) TRY(issue_copies(c, n, next_copy));
   }
+  c->pending_w_layer = w_now;
   return LST_OK;
 }
 
@@ -684,6 +781,11 @@ lst_status finish_step(lst_ctx* c, float* loss, float* grads_out) {
     return fail(c, LST_ERR_DEVICE, "device code reported error " + std::to_string(derr));
   }
   *loss = *c->host_loss;
+  if (c->cfg.streamed) {
+    c->slot_layer[0] = c->plan_held[0];
+    c->slot_layer[1] = c->plan_held[1];
+  }
+  c->w_layer = c->pending_w_layer;
   c->st.steps += 1;
   c->st.launches_last_step = g_launch_count.load() - c->launches_at_step_start;
   if (c->profiling) {
@@ -921,8 +1023,9 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
     TRY(copy_in(c, c->gf, final_norm, d * 4));
     TRY(dalloc(c, &c->nf, T * d));
     TRY(dalloc(c, &c->rstdf, T));
-    TRY(dalloc(c, &c->logits, T * c->V));
-    TRY(dalloc(c, &c->dlog, T * c->V));
+    c->head_rows = k.head_chunk > 0 ? std::min<int64_t>(k.head_chunk, T) : T;
+    TRY(dalloc(c, &c->logits, c->head_rows * c->V));
+    TRY(dalloc(c, &c->dlog, c->head_rows * c->V));
     TRY(dalloc(c, &c->loss_rows, T));
     TRY(dalloc(c, &c->tok, T));
     TRY(dalloc(c, &c->tgt, T));
@@ -1079,6 +1182,9 @@ lst_status lst_create(const lst_config* cfg, const float* embed, const float* fi
 lst_status lst_register_layer(lst_ctx* c, int32_t layer, const lst_layer_weights* w) {
   if (!c) return LST_ERR_ARG;
   if (!w || layer < 0 || layer >= c->L) return fail(c, LST_ERR_ARG, "bad layer index or null weights");
+  // the layer's bytes change: nothing kept in the pool or the weight scratch is trusted any more
+  c->slot_layer[0] = c->slot_layer[1] = -1;
+  c->w_layer = -1;
   return register_impl(c, layer, w);
 }
 
@@ -1149,6 +1255,7 @@ lst_status lst_get_logits(lst_ctx* c, float* dst) {
   if (!c) return LST_ERR_ARG;
   if (!dst) return fail(c, LST_ERR_ARG, "null dst");
   if (!c->have_logits) return fail(c, LST_ERR_STATE, "no logits: run lst_step first");
+  if (!c->logits_whole) return fail(c, LST_ERR_STATE, "the head ran in passes (head_chunk): logits are not kept whole");
   const bool dev = is_device_ptr(dst);
   CK(cudaMemcpyAsync(dst, c->logits, c->curT * c->V * 4, dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
                      c->stream));
@@ -1222,6 +1329,12 @@ lst_status lst_get_lora(lst_ctx* c, float* dst) {
 lst_status lst_set_profiling(lst_ctx* c, int32_t on) {
   if (!c) return LST_ERR_ARG;
   c->profiling = on != 0;
+  return LST_OK;
+}
+
+lst_status lst_set_reuse(lst_ctx* c, int32_t reuse) {
+  if (!c) return LST_ERR_ARG;
+  c->cfg.reuse = reuse != 0;
   return LST_OK;
 }
 

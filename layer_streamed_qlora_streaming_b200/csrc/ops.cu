@@ -217,29 +217,76 @@ __global__ void k_embed(const int32_t* __restrict__ tok, const bf16* __restrict_
 }
 
 // ------------------------------------------------------------------------------- cross-entropy
-__global__ void k_ce(const float* __restrict__ logits, int V, const int32_t* __restrict__ y, float inv_T,
-                     float* __restrict__ loss_rows, bf16* __restrict__ dlog) {
-  __shared__ float red[32];
+// One CTA per row. Pass 1 reads the row once and keeps a running (max, sum of exp) pair per thread,
+// rescaling the sum when the max grows (the online normaliser of Milakov & Gimelshein, "Online
+// normalizer calculation for softmax", 2018); the pairs are merged in a fixed tree. Pass 2 reads
+// the row again, usually from L2 (one 1024-thread CTA per SM keeps ~148 rows in flight), and writes
+// dlogits. Deterministic: the thread-to-element map and the merge order depend only on V.
+__device__ __forceinline__ void ms_merge(float& m, float& s, float m2, float s2) {
+  const float M = fmaxf(m, m2);
+  if (M == -INFINITY) return;  // both empty
+  s = s * expf(m - M) + s2 * expf(m2 - M);
+  m = M;
+}
+__device__ __forceinline__ void ms_add4(float& m, float& s, float4 v) {
+  const float M = fmaxf(fmaxf(m, fmaxf(v.x, v.y)), fmaxf(v.z, v.w));
+  s = s * expf(m - M) + (expf(v.x - M) + expf(v.y - M)) + (expf(v.z - M) + expf(v.w - M));
+  m = M;
+}
+
+__global__ void __launch_bounds__(1024, 1)
+k_ce(const float* __restrict__ logits, int V, const int32_t* __restrict__ y, float inv_T,
+     float* __restrict__ loss_rows, bf16* __restrict__ dlog) {
+  __shared__ float sm[32], ss[32];
   const int64_t row = blockIdx.x;
   const float* lr = logits + row * V;
-  float mx = -INFINITY;
-  for (int c = threadIdx.x; c < V; c += blockDim.x) mx = fmaxf(mx, lr[c]);
-  mx = block_max(mx, red);
-  float se = 0.f;
-  for (int c = threadIdx.x; c < V; c += blockDim.x) se += expf(lr[c] - mx);
-  se = block_sum(se, red);
-  const float lse = mx + logf(se);
+  bf16* dr = dlog + row * V;
+  const bool vec = (V % 4) == 0;  // rows then start 16-byte aligned
+  float m = -INFINITY, s = 0.f;
+  if (vec) {
+    const float4* l4 = reinterpret_cast<const float4*>(lr);
+    for (int c = threadIdx.x; c < V / 4; c += blockDim.x) ms_add4(m, s, __ldg(l4 + c));
+  } else {
+    for (int c = threadIdx.x; c < V; c += blockDim.x) ms_add4(m, s, make_float4(lr[c], -INFINITY, -INFINITY, -INFINITY));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    ms_merge(m, s, m2, s2);
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    sm[w] = m;
+    ss[w] = s;
+  }
+  __syncthreads();
+  m = sm[0];
+  s = ss[0];
+  for (int i = 1; i < (int)(blockDim.x >> 5); ++i) ms_merge(m, s, sm[i], ss[i]);
+  const float lse = m + logf(s);
   int tgt = y[row];
   if (tgt < 0 || tgt >= V) {
     if (threadIdx.x == 0) dev_fail(DEV_ERR_BAD_INDEX);
     tgt = 0;
   }
   if (threadIdx.x == 0) loss_rows[row] = lse - lr[tgt];
-  bf16* dr = dlog + row * V;
-  for (int c = threadIdx.x; c < V; c += blockDim.x) {
-    float p = expf(lr[c] - lse);
-    if (c == tgt) p -= 1.0f;
-    dr[c] = __float2bfloat16_rn(p * inv_T);
+  if (vec) {
+    const float4* l4 = reinterpret_cast<const float4*>(lr);
+    for (int c = threadIdx.x; c < V / 4; c += blockDim.x) {
+      const float4 v = __ldg(l4 + c);
+      float p[4] = {expf(v.x - lse), expf(v.y - lse), expf(v.z - lse), expf(v.w - lse)};
+      const int d = tgt - 4 * c;
+      if (d >= 0 && d < 4) p[d] -= 1.0f;
+      const __nv_bfloat162 h[2] = {__floats2bfloat162_rn(p[0] * inv_T, p[1] * inv_T),
+                                   __floats2bfloat162_rn(p[2] * inv_T, p[3] * inv_T)};
+      *reinterpret_cast<uint2*>(dr + 4 * c) = *reinterpret_cast<const uint2*>(h);
+    }
+  } else {
+    for (int c = threadIdx.x; c < V; c += blockDim.x) {
+      float p = expf(lr[c] - lse);
+      if (c == tgt) p -= 1.0f;
+      dr[c] = __float2bfloat16_rn(p * inv_T);
+    }
   }
 }
 
@@ -327,7 +374,7 @@ cudaError_t embed(const int32_t* tok, const bf16* E, int64_t T, int d, int V, fl
 }
 cudaError_t cross_entropy(const float* logits, int64_t T, int V, const int32_t* y, float inv_T, float* loss_rows,
                           bf16* dlog, cudaStream_t s) {
-  k_ce<<<(unsigned)T, 512, 0, s>>>(logits, V, y, inv_T, loss_rows, dlog);
+  k_ce<<<(unsigned)T, 1024, 0, s>>>(logits, V, y, inv_T, loss_rows, dlog);
   note_launch(1);
   return cudaGetLastError();
 }

@@ -10,7 +10,16 @@ Cases are the shapes of the Llama-3.1-8B-shaped layer at batch 4 x seq 512 (T = 
   dequant      NF4 -> bf16 of one 8B layer (218 M elements, 7 tensors)
   attn_fwd     causal GQA attention forward, 4 x 512, 32/8 heads, hd 128
   attn_bwd     its backward (D, dK/dV, dQ kernels)
-Prints one JSON line with the per-launch time and the achieved rate. Inputs are seeded random
+  lora_u_qkv   LoRA projection U = s X Acat^T, X [2048, 4096], Acat [64, 4096]
+  lora_u_down  the same for the down projection's input, X [2048, 14336]
+  lora_v_gu    V = s dY Bexp, dY [2048, 28672], Bexp [28672, 64] (MN-major)
+  lora_grads_qkv  dA = Vs^T X and dB = dY^T Us of the q/k/v group (dY [2048, 6144])
+  lora_grads_gu   the same for gate/up (dY [2048, 28672])
+  ce           cross-entropy rows + dlogits over fp32 logits [2048, 128256]
+The LoRA cases rotate over enough input copies to exceed the 126 MB L2, so every launch reads
+its operands from HBM.
+Prints one JSON line with the per-launch device time (launches queued back to back) and the
+achieved rate. Inputs are seeded random
 tensors on the device (values do not matter for timing). Used for the ncu captures in profiles/.
 """
 from __future__ import annotations
@@ -20,7 +29,8 @@ import json
 
 import torch
 
-from . import k_attention_bwd, k_attention_fwd, k_gemm, k_nf4_dequant, k_nf4_quantize
+from . import (k_attention_bwd, k_attention_fwd, k_cross_entropy, k_gemm, k_lora_grads, k_lora_skinny, k_nf4_dequant,
+               k_nf4_quantize)
 
 T, D, F, HQ, HKV, HD, S = 2048, 4096, 14336, 32, 8, 128, 512
 
@@ -80,7 +90,58 @@ def build(case: str):
             k_attention_bwd(q, ld, k, ld, v, ld, o, HQ * HD, do, HQ * HD, lse, Dd, dqkv, ld, dqkv[:, HQ * HD:], ld,
                             dqkv[:, (HQ + HKV) * HD:], ld, T, S, HQ, HKV, HD)
         return run, {"flop": 2.5 * flop_fwd, "bytes": None}
+    if case.startswith("lora_"):
+        return _lora_case(case, g)
+    if case == "ce":
+        V = 128256
+        logits = torch.randn(T, V, generator=g, device="cuda") * 2.0
+        tg = torch.randint(0, V, (T,), generator=g, device="cuda", dtype=torch.int32)
+        loss_rows = torch.empty(T, device="cuda")
+        dlog = torch.empty(T, V, dtype=torch.bfloat16, device="cuda")
+
+        def run():
+            k_cross_entropy(logits, T, V, tg, 1.0 / T, loss_rows, dlog)
+        return run, {"flop": None, "bytes": T * V * 4 + T * V * 2}
     raise SystemExit(f"unknown case {case}")
+
+
+def _copies(nbytes: int) -> int:
+    return max(2, -(-256 * 2**20 // max(nbytes, 1)))
+
+
+def _lora_case(case: str, g):
+    KP = 64
+    if case.startswith("lora_u") or case.startswith("lora_v"):
+        K, bmn = {"lora_u_qkv": (D, 0), "lora_u_down": (F, 0), "lora_v_gu": (2 * F, 1)}[case]
+        nb = _copies(T * K * 2)
+        Xs = [_bf((T, K), g) for _ in range(nb)]
+        Bop = _bf((K, KP) if bmn else (KP, K), g, 0.02)
+        Us = torch.empty(T, KP, dtype=torch.bfloat16, device="cuda")
+        it = [0]
+
+        def run():
+            X = Xs[it[0] % nb]
+            it[0] += 1
+            k_lora_skinny(X, K, T, K, Bop, KP if bmn else K, bmn, KP, 2.0, Us)
+        return run, {"flop": 2.0 * T * K * KP, "bytes": T * K * 2 + K * KP * 2 + T * KP * 2}
+    in_f, bounds, r = {"lora_grads_qkv": (D, [0, 4096, 5120, 6144], 16),
+                       "lora_grads_gu": (D, [0, F, 2 * F], 16)}[case]
+    out_f = bounds[-1]
+    nb = _copies(T * (in_f + out_f) * 2)
+    Xs = [_bf((T, in_f), g) for _ in range(nb)]
+    dYs = [_bf((T, out_f), g) for _ in range(nb)]
+    Us, Vs = _bf((T, KP), g), _bf((T, KP), g)
+    nseg = len(bounds) - 1
+    dA = [torch.empty(r, in_f, device="cuda") for _ in range(nseg)]
+    dB = [torch.empty(bounds[p + 1] - bounds[p], r, device="cuda") for p in range(nseg)]
+    it = [0]
+
+    def run():
+        i = it[0] % nb
+        it[0] += 1
+        k_lora_grads(Xs[i], in_f, in_f, dYs[i], out_f, out_f, T, Us, Vs, KP, r, bounds, dA, dB)
+    return run, {"flop": 2.0 * T * KP * (in_f + out_f),
+                 "bytes": T * (in_f + out_f) * 2 + 2 * T * KP * 2 + nseg * r * (in_f + out_f) * 4}
 
 
 def main():
@@ -94,6 +155,9 @@ def main():
         run()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # hold the stream with a spin kernel while the host enqueues every launch, so the timed
+    # region is back-to-back device time even for launches shorter than their host overhead
+    torch.cuda._sleep(200_000_000)
     e0.record()
     for _ in range(a.iters):
         run()

@@ -56,10 +56,11 @@ def build_inputs(wl, step: int = 0) -> dict:
     return d
 
 
-def make_context(wl, inp: dict, streamed: bool, timeout_ms: int = 600000):
-    """A library context with every layer registered from host (numpy) weights."""
+def make_context(wl, inp: dict, streamed: bool, timeout_ms: int = 600000, **cfg_kw):
+    """A library context with every layer registered from host (numpy) weights; cfg_kw go to
+    make_config (head_chunk, reuse)."""
     import layer_streamed_qlora_streaming_b200 as lst
-    cfg = lst.make_config(wl, streamed=streamed, timeout_ms=timeout_ms)
+    cfg = lst.make_config(wl, streamed=streamed, timeout_ms=timeout_ms, **cfg_kw)
     if wl.vocab:
         E, gf, H = inp["head"]
         ctx = lst.Context(cfg, E, gf, H)

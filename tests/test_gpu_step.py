@@ -89,6 +89,52 @@ def test_deterministic_and_adapters_matter():
     ctx.close()
 
 
+@pytest.mark.parametrize("name", ["tiny", "qwen3b_bf16_2L"])
+def test_reuse_schedule_same_bytes_fewer_reads(name):
+    # keeping layers resident in the pool (turnaround, and across steps) changes the copies only
+    wl = WORKLOADS[name].with_(n_layers=3) if name == "tiny" else WORKLOADS[name]
+    L = wl.n_layers
+    inp = build_inputs(wl)
+    runs = {}
+    for reuse in (False, True):
+        ctx = make_context(wl, inp, streamed=True, reuse=reuse)
+        out, reads = [], []
+        for _ in range(3):
+            out.append(run_step(ctx, wl, inp, want_logits=False)[:2])
+            reads.append(ctx.stats()["layer_reads_last_step"])
+        # a re-registered layer is copied again on the next step
+        r = inp["raw"][0]
+        ctx.register_layer(0, r["W"], r["A"], r["B"], r["attn_norm"], r["mlp_norm"], r["bias"])
+        out.append(run_step(ctx, wl, inp, want_logits=False)[:2])
+        reads.append(ctx.stats()["layer_reads_last_step"])
+        ctx.close()
+        runs[reuse] = (out, reads)
+    for (la, ga), (lb, gb) in zip(runs[False][0], runs[True][0]):
+        assert np.float32(la).tobytes() == np.float32(lb).tobytes()
+        assert ga.tobytes() == gb.tobytes()
+    assert runs[False][1] == [2 * L] * 4
+    assert runs[True][1] == [2 * L - 2, max(2 * L - 4, 0), max(2 * L - 4, 0), 2 * L - 2]
+
+
+@pytest.mark.parametrize("chunk", [48, 64])
+def test_head_in_passes_same_bytes(chunk):
+    # the LM head + CE in passes of `chunk` token rows (T = 128: ragged 48+48+32, even 64+64)
+    import layer_streamed_qlora_streaming_b200 as lst
+    wl = syn.WORKLOADS["tiny"]
+    inp = build_inputs(wl)
+    ctx = make_context(wl, inp, streamed=True)
+    loss_a, g_a, _ = run_step(ctx, wl, inp, want_logits=False)
+    ctx.close()
+    ctx = make_context(wl, inp, streamed=True, head_chunk=chunk)
+    loss_b, g_b, _ = run_step(ctx, wl, inp, want_logits=False)
+    assert np.float32(loss_a).tobytes() == np.float32(loss_b).tobytes()
+    assert g_a.tobytes() == g_b.tobytes()
+    with pytest.raises(lst.LstError) as e:   # logits are not kept whole
+        ctx.logits(np.zeros((wl.tokens, wl.vocab), dtype=np.float32))
+    assert e.value.status == 2
+    ctx.close()
+
+
 def test_errors_are_status_codes():
     import layer_streamed_qlora_streaming_b200 as lst
     wl = syn.WORKLOADS["tiny"]
