@@ -274,7 +274,8 @@ def run_gpu(args, wl):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local))
-    stream = torch.cuda.Stream()
+    # above the library's prep stream, so the next read's dequant only takes SM slots this leaves free
+    stream = torch.cuda.Stream(priority=-1)
     link_gbs = h2d_peak_gbs(torch)
     ctx = build_context(wl, torch, stream, seed=1234 + rank)
     if not args.no_optimizer:

@@ -168,12 +168,18 @@ struct ReadPlan {
   bool copy = true;     // the layer is copied into the slot for this read
   int wait_free = -1;   // the copy waits for this read's compute to finish (-1: nothing to wait for)
   int loaded_by = -1;   // read whose copy filled the slot (-1: filled by an earlier step)
+  // NF4 base: bf16 weight scratch the read computes from
+  int wslot = 0;
+  bool deq = true;      // the layer is dequantised into the scratch for this read
+  int wwait = -1;       // the dequant waits for this read's compute to finish
+  int wfilled_by = -1;  // read whose dequant filled the scratch (-1: an earlier step)
 };
 
 struct lst_ctx {
   lst_config cfg{};
   int dev = 0;
   cudaStream_t stream = nullptr, copy_stream = nullptr;
+  cudaStream_t prep_stream = nullptr;  // dequant of the next read, below the compute stream's priority
   bool own_stream = false;
   std::string err;
   Faults faults;
@@ -205,7 +211,7 @@ struct lst_ctx {
   float* xs = nullptr;  // residual stream: the input of every layer and the final output, fp32
   float* h = nullptr;   // residual after attention, fp32
   __nv_bfloat16 *n1 = nullptr, *qkv = nullptr, *o = nullptr, *n2 = nullptr, *gu = nullptr, *m = nullptr,
-                *wscr = nullptr;
+                *wscr[2] = {nullptr, nullptr};
   float *rstd1 = nullptr, *rstd2 = nullptr, *lse = nullptr, *Dbuf = nullptr;
   float* o32 = nullptr;  // attention output before rounding (recompute pass), for the backward's D
   __nv_bfloat16* Us[NGROUP] = {};  // bf16(s * x A^T) per group [T, KP]
@@ -227,9 +233,10 @@ struct lst_ctx {
   std::vector<ReadPlan> plan;
   int plan_held[2] = {-1, -1};   // layers the slots hold once the planned step has run
   int slot_layer[2] = {-1, -1};  // layers the slots hold after the last completed step (-1: unknown)
-  int w_layer = -1;              // layer whose dequantised weights the scratch holds (-1: unknown)
-  int pending_w_layer = -1;
-  cudaEvent_t ev_done = nullptr;
+  int plan_wheld[2] = {-1, -1};  // layers the weight scratches hold once the planned step has run
+  int w_layer[2] = {-1, -1};     // layers the weight scratches hold after the last completed step
+  std::vector<cudaEvent_t> ev_deq;
+  cudaEvent_t ev_done = nullptr, ev_start = nullptr;
 
   float* stage_w = nullptr;
   uint8_t* stage_blob = nullptr;
@@ -448,11 +455,9 @@ lst_status group_bwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
 }
 
 // Weights of a layer read: the bf16 [P] matrix the GEMMs consume.
-lst_status layer_weights(lst_ctx* c, const uint8_t* blob, const __nv_bfloat16** W) {
-  if (c->cfg.base_format == LST_BASE_BF16) {
-    *W = reinterpret_cast<const __nv_bfloat16*>(blob + c->lay.w16);
-    return LST_OK;
-  }
+// NF4 blob -> bf16 weights of the 7 projections in the concatenated [q;k;v], o, [gate;up], down
+// order, written to dst on stream st.
+lst_status dequant_layer(lst_ctx* c, const uint8_t* blob, __nv_bfloat16* dst, cudaStream_t st) {
   Nf4Seg segs[NPROJ];
   for (int p = 0; p < NPROJ; ++p) {
     segs[p].packed = blob + c->lay.packed[p];
@@ -462,9 +467,8 @@ lst_status layer_weights(lst_ctx* c, const uint8_t* blob, const __nv_bfloat16** 
     segs[p].n = c->lay.n[p];
     segs[p].out_offset = c->lay.woff[p];
   }
-  ProfScope ps(c, c->stream, PC_DEQ);
-  CK(nf4_dequant(segs, NPROJ, c->wscr, c->stream));
-  *W = c->wscr;
+  ProfScope ps(c, st, PC_DEQ);
+  CK(nf4_dequant(segs, NPROJ, dst, st));
   return LST_OK;
 }
 
@@ -633,12 +637,23 @@ lst_status head_fwd_bwd(lst_ctx* c) {
 //    turn; layers 0 and 1 left by the previous step's backward) uses it as it is; otherwise it copies
 //    into the slot the previous read does not use (for read 0, the slot whose layer is needed last).
 // A copy into a slot waits until the last read that computed from that slot has finished.
+// An NF4 base is dequantised into one of two bf16 weight scratches by the same rule (a read reuses
+// a scratch that still holds its layer only with reuse on), on the prep stream, one read ahead: the
+// dequant of read n+1 overlaps the compute of read n.
 void plan_reads(lst_ctx* c) {
   const int L = c->L, R = 2 * L;
   const bool reuse = c->cfg.reuse != 0;
   auto layer_of = [L](int n) { return n < L ? n : 2 * L - 1 - n; };
   int held[2] = {reuse ? c->slot_layer[0] : -1, reuse ? c->slot_layer[1] : -1};
   int last_use[2] = {-1, -1}, loaded_by[2] = {-1, -1};
+  int wheld[2] = {reuse ? c->w_layer[0] : -1, reuse ? c->w_layer[1] : -1};
+  int wlast[2] = {-1, -1}, wfill[2] = {-1, -1};
+  const bool nf4 = c->cfg.base_format != LST_BASE_BF16;
+  auto first_need = [&](int layer) {
+    for (int m = 0; m < R; ++m)
+      if (layer_of(m) == layer) return m;
+    return R;
+  };
   c->plan.assign(R, ReadPlan{});
   for (int n = 0; n < R; ++n) {
     const int j = layer_of(n);
@@ -653,14 +668,7 @@ void plan_reads(lst_ctx* c) {
       if (n > 0) {
         p.slot = 1 - c->plan[n - 1].slot;
       } else {
-        int next[2] = {R, R};  // first read that needs the held layer
-        for (int s = 0; s < 2; ++s)
-          for (int m = 0; m < R; ++m)
-            if (layer_of(m) == held[s]) {
-              next[s] = m;
-              break;
-            }
-        p.slot = next[1] > next[0] ? 1 : 0;
+        p.slot = first_need(held[1]) > first_need(held[0]) ? 1 : 0;
       }
       p.wait_free = last_use[p.slot];
       held[p.slot] = j;
@@ -668,9 +676,28 @@ void plan_reads(lst_ctx* c) {
     }
     p.loaded_by = loaded_by[p.slot];
     last_use[p.slot] = n;
+
+    p.deq = false;
+    if (!nf4) continue;
+    p.wslot = -1;
+    if (reuse) {
+      if (wheld[0] == j) p.wslot = 0;
+      else if (wheld[1] == j) p.wslot = 1;
+    }
+    if (p.wslot < 0) {
+      p.deq = true;
+      p.wslot = n > 0 ? 1 - c->plan[n - 1].wslot : (first_need(wheld[1]) > first_need(wheld[0]) ? 1 : 0);
+      p.wwait = wlast[p.wslot];
+      wheld[p.wslot] = j;
+      wfill[p.wslot] = n;
+    }
+    p.wfilled_by = wfill[p.wslot];
+    wlast[p.wslot] = n;
   }
   c->plan_held[0] = held[0];
   c->plan_held[1] = held[1];
+  c->plan_wheld[0] = wheld[0];
+  c->plan_wheld[1] = wheld[1];
 }
 
 lst_status enqueue_copy(lst_ctx* c, int n) {
@@ -703,29 +730,47 @@ lst_status issue_copies(lst_ctx* c, int done, int& next) {
 }
 
 lst_status run_layers(lst_ctx* c, bool head) {
-  const int L = c->L;
+  const int L = c->L, R = 2 * L;
   const bool streamed = c->cfg.streamed != 0;
-  const bool reuse = streamed && c->cfg.reuse != 0;
-  int next_copy = 0;
-  if (streamed) {
-    plan_reads(c);
-    // the slots' contents are only trusted again once this step has completed
-    c->slot_layer[0] = c->slot_layer[1] = -1;
-    TRY(issue_copies(c, -1, next_copy));
-  }
-  const int w_held = c->w_layer;
-  c->w_layer = -1;
-  int w_now = reuse ? w_held : -1;
-  for (int n = 0; n < 2 * L; ++n) {
+  const bool nf4 = c->cfg.base_format != LST_BASE_BF16;
+  auto blob_of = [&](int n) -> const uint8_t* {
     const int j = n < L ? n : 2 * L - 1 - n;
-    const uint8_t* blob = streamed ? c->pool[c->plan[n].slot] : c->resident + (int64_t)j * c->lay.total;
-    if (streamed && c->plan[n].loaded_by >= 0) CK(cudaStreamWaitEvent(c->stream, c->ev_loaded[c->plan[n].loaded_by], 0));
-    const __nv_bfloat16* W = nullptr;
-    if (reuse && c->cfg.base_format != LST_BASE_BF16 && w_now == j) {
-      W = c->wscr;  // the dequantised copy of this layer is still in the scratch
+    return streamed ? c->pool[c->plan[n].slot] : c->resident + (int64_t)j * c->lay.total;
+  };
+  plan_reads(c);
+  // the slots' and scratches' contents are only trusted again once this step has completed
+  c->slot_layer[0] = c->slot_layer[1] = -1;
+  c->w_layer[0] = c->w_layer[1] = -1;
+  // copies and dequants of this step start after everything already on the compute stream (e.g. a
+  // step that returned early with work in flight)
+  CK(cudaEventRecord(c->ev_start, c->stream));
+  CK(cudaStreamWaitEvent(c->copy_stream, c->ev_start, 0));
+  CK(cudaStreamWaitEvent(c->prep_stream, c->ev_start, 0));
+  int next_copy = 0;
+  if (streamed) TRY(issue_copies(c, -1, next_copy));
+  // dequant of read m on the prep stream; every event it waits on is already recorded
+  auto enqueue_deq = [&](int m) -> lst_status {
+    if (m >= R || !c->plan[m].deq) return LST_OK;
+    const ReadPlan& p = c->plan[m];
+    if (streamed && p.loaded_by >= 0) CK(cudaStreamWaitEvent(c->prep_stream, c->ev_loaded[p.loaded_by], 0));
+    if (p.wwait >= 0) CK(cudaStreamWaitEvent(c->prep_stream, c->ev_free[p.wwait], 0));
+    TRY(dequant_layer(c, blob_of(m), c->wscr[p.wslot], c->prep_stream));
+    CK(cudaEventRecord(c->ev_deq[m], c->prep_stream));
+    return LST_OK;
+  };
+  TRY(enqueue_deq(0));
+  for (int n = 0; n < R; ++n) {
+    const int j = n < L ? n : 2 * L - 1 - n;
+    const ReadPlan& p = c->plan[n];
+    TRY(enqueue_deq(n + 1));
+    const uint8_t* blob = blob_of(n);
+    if (streamed && p.loaded_by >= 0) CK(cudaStreamWaitEvent(c->stream, c->ev_loaded[p.loaded_by], 0));
+    const __nv_bfloat16* W;
+    if (nf4) {
+      if (p.wfilled_by >= 0) CK(cudaStreamWaitEvent(c->stream, c->ev_deq[p.wfilled_by], 0));
+      W = c->wscr[p.wslot];
     } else {
-      TRY(layer_weights(c, blob, &W));
-      w_now = j;
+      W = reinterpret_cast<const __nv_bfloat16*>(blob + c->lay.w16);
     }
     if (n < L) {
       TRY(layer_fwd(c, j, blob, W, false));
@@ -733,7 +778,7 @@ lst_status run_layers(lst_ctx* c, bool head) {
       TRY(layer_fwd(c, j, blob, W, true));
       TRY(layer_bwd(c, j, blob, W));
     }
-    if (streamed) CK(cudaEventRecord(c->ev_free[n], c->stream));
+    CK(cudaEventRecord(c->ev_free[n], c->stream));
     if (n == L - 1) {
       if (head) {
         TRY(head_fwd_bwd(c));
@@ -748,7 +793,6 @@ lst_status run_layers(lst_ctx* c, bool head) {
     }
     if (streamed) TRY(issue_copies(c, n, next_copy));
   }
-  c->pending_w_layer = w_now;
   return LST_OK;
 }
 
@@ -785,7 +829,8 @@ lst_status finish_step(lst_ctx* c, float* loss, float* grads_out) {
     c->slot_layer[0] = c->plan_held[0];
     c->slot_layer[1] = c->plan_held[1];
   }
-  c->w_layer = c->pending_w_layer;
+  c->w_layer[0] = c->plan_wheld[0];
+  c->w_layer[1] = c->plan_wheld[1];
   c->st.steps += 1;
   c->st.launches_last_step = g_launch_count.load() - c->launches_at_step_start;
   if (c->profiling) {
@@ -902,13 +947,17 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   setg(G_GU, 2, {4, 5}, c->d, {0, c->F, 2 * c->F});
   setg(G_DOWN, 1, {6}, c->F, {0, c->d});
 
+  int prio_low = 0, prio_high = 0;
+  CK(cudaDeviceGetStreamPriorityRange(&prio_low, &prio_high));
   if (stream) {
     c->stream = static_cast<cudaStream_t>(stream);
   } else {
-    CK(cudaStreamCreateWithFlags(&c->stream, cudaStreamNonBlocking));
+    CK(cudaStreamCreateWithPriority(&c->stream, cudaStreamNonBlocking, prio_high));
     c->own_stream = true;
   }
   CK(cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking));
+  // lowest priority: the next read's dequant takes the SM slots the compute stream leaves free
+  CK(cudaStreamCreateWithPriority(&c->prep_stream, cudaStreamNonBlocking, prio_low));
 
   // LoRA parameter / gradient layout
   c->offA.resize(c->L * NPROJ);
@@ -972,7 +1021,10 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   }
   c->st.blob_bytes = blob;
   c->registered.assign(c->L, 0);
-  if (k.base_format == LST_BASE_NF4) TRY(dalloc(c, &c->wscr, c->lay.P));
+  if (k.base_format == LST_BASE_NF4) {
+    TRY(dalloc(c, &c->wscr[0], c->lay.P));
+    TRY(dalloc(c, &c->wscr[1], c->lay.P));
+  }
 
   // activations
   const int64_t T = c->Tmax, d = c->d;
@@ -1034,11 +1086,14 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   }
   c->ev_loaded.resize(2 * c->L);
   c->ev_free.resize(2 * c->L);
+  c->ev_deq.resize(2 * c->L);
   for (int i = 0; i < 2 * c->L; ++i) {
     CK(cudaEventCreateWithFlags(&c->ev_loaded[i], cudaEventDisableTiming));
     CK(cudaEventCreateWithFlags(&c->ev_free[i], cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&c->ev_deq[i], cudaEventDisableTiming));
   }
   CK(cudaEventCreateWithFlags(&c->ev_done, cudaEventDisableTiming));
+  CK(cudaEventCreateWithFlags(&c->ev_start, cudaEventDisableTiming));
   CK(cudaEventCreate(&c->prof_step0));
   CK(cudaEventCreate(&c->prof_step1));
   CK(cudaStreamSynchronize(c->stream));
@@ -1049,6 +1104,7 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
 void free_all(lst_ctx* c) {
   if (c->stream) cudaStreamSynchronize(c->stream);
   if (c->copy_stream) cudaStreamSynchronize(c->copy_stream);
+  if (c->prep_stream) cudaStreamSynchronize(c->prep_stream);
   for (void* p : c->dev_allocs) cudaFree(p);
   c->dev_allocs.clear();
   if (c->stage_w) cudaFree(c->stage_w);
@@ -1059,11 +1115,14 @@ void free_all(lst_ctx* c) {
   if (c->host_loss) cudaFreeHost(c->host_loss);
   for (auto e : c->ev_loaded) cudaEventDestroy(e);
   for (auto e : c->ev_free) cudaEventDestroy(e);
+  for (auto e : c->ev_deq) cudaEventDestroy(e);
   for (auto e : c->prof_pool) cudaEventDestroy(e);
   if (c->ev_done) cudaEventDestroy(c->ev_done);
+  if (c->ev_start) cudaEventDestroy(c->ev_start);
   if (c->prof_step0) cudaEventDestroy(c->prof_step0);
   if (c->prof_step1) cudaEventDestroy(c->prof_step1);
   if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
+  if (c->prep_stream) cudaStreamDestroy(c->prep_stream);
   if (c->own_stream && c->stream) cudaStreamDestroy(c->stream);
   cudaGetLastError();
 }
@@ -1184,7 +1243,7 @@ lst_status lst_register_layer(lst_ctx* c, int32_t layer, const lst_layer_weights
   if (!w || layer < 0 || layer >= c->L) return fail(c, LST_ERR_ARG, "bad layer index or null weights");
   // the layer's bytes change: nothing kept in the pool or the weight scratch is trusted any more
   c->slot_layer[0] = c->slot_layer[1] = -1;
-  c->w_layer = -1;
+  c->w_layer[0] = c->w_layer[1] = -1;
   return register_impl(c, layer, w);
 }
 

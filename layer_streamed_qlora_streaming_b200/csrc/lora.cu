@@ -195,13 +195,20 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     const int rl = r0 + f / (kBN / 4);
     const int c = (f % (kBN / 4)) * 4;
     const uint32_t a = red0 + (uint32_t)((rl * kRedLd + c) * 4);
-    float4 acc = ld_cluster_f4(cluster_map(a, 0));
-    for (int p = 1; p < cs; ++p) {
-      const float4 v = ld_cluster_f4(cluster_map(a, (uint32_t)p));
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+    // all slices' loads in flight first, then the sum in slice order
+    float4 v[kMaxCluster];
+#pragma unroll
+    for (int p = 0; p < kMaxCluster; ++p)
+      if (p < cs) v[p] = ld_cluster_f4(cluster_map(a, (uint32_t)p));
+    float4 acc = v[0];
+#pragma unroll
+    for (int p = 1; p < kMaxCluster; ++p) {
+      if (p < cs) {
+        acc.x += v[p].x;
+        acc.y += v[p].y;
+        acc.z += v[p].z;
+        acc.w += v[p].w;
+      }
     }
     side_store(o, m0 + rl, n0 + c, acc);
   }
