@@ -111,7 +111,7 @@ def test_gemm_rejects_misaligned_stride():
 
 # ------------------------------------------------------------------------------------ attention
 @pytest.mark.parametrize("B,S,hq,hkv,hd", [(2, 64, 4, 4, 64), (2, 100, 4, 2, 64), (1, 200, 4, 1, 128),
-                                           (2, 128, 8, 2, 128)])
+                                           (2, 128, 8, 2, 128), (1, 160, 16, 2, 128), (2, 96, 10, 2, 64)])
 def test_attention_fwd_bwd(B, S, hq, hkv, hd):
     r = _rng(S * hq + hd)
     T = B * S
