@@ -371,3 +371,97 @@ def step(wl, raw_layers, blobs=None, head=None, tokens=None, targets=None, x_in=
             _, c = layer_fwd(saved[i], Wt, lora[i], sh)   # recompute from the saved input
             dx, grads[i] = layer_bwd(dx, c, Wt, lora[i], sh)
     return {"loss": loss, "grads": grads, "logits": logits, "reads": reads, "dx_in": dx}
+
+
+# ------------------------------------------------------------------------------------------
+# preference step: DPO against the same base with the adapters switched off
+# ------------------------------------------------------------------------------------------
+# [TESS] (the paragraph on the economics of layer streaming) names DPO among the preference
+# losses run over the streamed base and fixes its reference model: the same streamed base with
+# the adapters switched off, so the reference costs one more forward pass of reads, not weights.
+# The loss is the one of Rafailov et al., "Direct Preference Optimization: Your Language Model is
+# Secretly a Reward Model" (2023): for a pair (chosen w, rejected l)
+#     L = -log sigmoid(beta * ((pi_w - ref_w) - (pi_l - ref_l)))
+# with pi / ref the sequence log-likelihood under the policy / reference. Readings: the batch holds
+# the P chosen sequences first, then the P rejected ones (row-aligned pairs); a sequence's
+# log-likelihood sums log softmax(logits_t)[target_t] over its positions whose mask is 1 (all
+# positions when no mask is given); the step's loss is the mean over the P pairs.
+
+def seq_logp(logits, targets, mask, nseq, seq):
+    """Per-sequence sum over the masked positions of log softmax(logits_t)[target_t]."""
+    mx = logits.max(axis=1, keepdims=True)
+    lse = (mx + np.log(np.exp(logits - mx).sum(axis=1, keepdims=True)))[:, 0]
+    T = logits.shape[0]
+    lp = (logits[np.arange(T), targets] - lse) * mask
+    return lp.reshape(nseq, seq).sum(axis=1), lse
+
+
+def dpo_loss(pi, ref, beta):
+    """Mean DPO loss over pairs and dL/dpi per sequence (pi, ref: [2P], chosen first)."""
+    P = pi.shape[0] // 2
+    z = beta * ((pi[:P] - ref[:P]) - (pi[P:] - ref[P:]))
+    loss = float(np.mean(np.logaddexp(0.0, -z)))          # -log sigmoid(z)
+    g = (1.0 / (1.0 + np.exp(-z)) - 1.0) * beta / P        # dL/dz_p * dz/dpi_w
+    return loss, np.concatenate([g, -g])
+
+
+def dpo_dlogits(logits, targets, mask, nseq, seq, ref, beta):
+    """(loss, dL/dlogits, pi) of the DPO loss as a function of the policy logits [nseq*seq, V]:
+    d pi_s / d logits_t = mask_t (onehot(target_t) - softmax(logits_t)) for t in sequence s."""
+    pi, lse = seq_logp(logits, targets, mask, nseq, seq)
+    loss, g = dpo_loss(pi, ref, beta)
+    T = logits.shape[0]
+    w = -np.repeat(g, seq) * mask
+    dlog = np.exp(logits - lse[:, None])
+    dlog[np.arange(T), targets] -= 1.0
+    return loss, dlog * w[:, None], pi
+
+
+def _forward(x, Ws, lora, sh):
+    caches = []
+    for i in range(len(Ws)):
+        x, c = layer_fwd(x, Ws[i], lora[i], sh)
+        caches.append(c)
+    return x, caches
+
+
+def dpo_step(wl, raw_layers, head, tokens, targets, npairs, beta, mask=None, blobs=None, bf16_acts=False,
+             lora=None):
+    """Loss and LoRA gradients of one DPO step on 2 * npairs sequences of wl.seq tokens.
+
+    The reference pass runs every layer with the adapters off (B = 0 makes the side path exactly
+    zero); the policy pass is the ordinary forward, then the head turns the per-sequence weights
+    dL/dpi into dlogits = -w (softmax - onehot) on masked rows, and the backward is the SFT one.
+    Returns dict(loss, grads, pi, ref).
+    """
+    L = wl.n_layers
+    sh = Shape(wl, bf16_acts)
+    nseq, S = 2 * npairs, wl.seq
+    assert nseq == wl.batch
+    if blobs is None:
+        blobs = [pack_layer(raw_layers[i], wl.base_format) for i in range(L)]
+    if lora is None:
+        lora = [_lora64(raw_layers[i]) for i in range(L)]
+    off = [{p: (a, np.zeros_like(b)) for p, (a, b) in lo.items()} for lo in lora]
+    E, gf, H = (a.astype(F64) for a in head)
+    T = nseq * S
+    m = np.ones(T) if mask is None else np.asarray(mask, dtype=F64)
+    Ws = [unpack_blob(blobs[i]) for i in range(L)]
+
+    def head_logits(xL):
+        n, r = rmsnorm(xL, gf, wl.rms_eps)
+        n = sh.rb(n)
+        return n @ H.T, (n, r)
+
+    x_ref, _ = _forward(E[tokens], Ws, off, sh)
+    ref, _ = seq_logp(head_logits(x_ref)[0], targets, m, nseq, S)
+
+    x0 = E[tokens]
+    xL, caches = _forward(x0, Ws, lora, sh)
+    logits, (n, r) = head_logits(xL)
+    loss, dlog, pi = dpo_dlogits(logits, targets, m, nseq, S, ref, beta)
+    dx = rmsnorm_bwd(sh.rb(dlog) @ H, xL, gf, r)
+    grads = [None] * L
+    for i in reversed(range(L)):
+        dx, grads[i] = layer_bwd(dx, caches[i], Ws[i], lora[i], sh)
+    return {"loss": loss, "grads": grads, "pi": pi, "ref": ref}

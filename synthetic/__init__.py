@@ -129,7 +129,7 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
 PROJ = ("q", "k", "v", "o", "gate", "up", "down")
 
 # seeds
-SEED_BASE_W, SEED_LORA, SEED_TOKENS, SEED_X, SEED_HEAD, SEED_G = 1, 2, 3, 4, 5, 6
+SEED_BASE_W, SEED_LORA, SEED_TOKENS, SEED_X, SEED_HEAD, SEED_G, SEED_PREF = 1, 2, 3, 4, 5, 6, 7
 
 
 @dataclass(frozen=True)
@@ -245,6 +245,23 @@ def tokens(w: Workload, step: int = 0) -> tuple[np.ndarray, np.ndarray]:
     t = integers(SEED_TOKENS, 2 * step, w.tokens, w.vocab)
     y = integers(SEED_TOKENS, 2 * step + 1, w.tokens, w.vocab)
     return t, y
+
+
+def preference_pairs(w: Workload, step: int = 0) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """(tokens, targets, mask), int32 [batch*seq] each, for batch/2 preference pairs: sequences
+    [0, P) are the chosen ones and [P, 2P) the rejected ones (P = batch/2). Chosen p and rejected p
+    share their prompt (tokens and targets of the first seq/2 positions); the response positions
+    are drawn independently; mask is 1 on the response positions, 0 on the prompt. Uniform ids."""
+    assert w.batch % 2 == 0
+    P, S = w.batch // 2, w.seq
+    half = S // 2
+    t = integers(SEED_PREF, 4 * step, w.tokens, w.vocab).reshape(w.batch, S)
+    y = integers(SEED_PREF, 4 * step + 1, w.tokens, w.vocab).reshape(w.batch, S)
+    t[P:, :half] = t[:P, :half]
+    y[P:, :half] = y[:P, :half]
+    m = np.zeros((w.batch, S), dtype=np.int32)
+    m[:, half:] = 1
+    return t.reshape(-1), y.reshape(-1), m.reshape(-1)
 
 
 def hidden_input(w: Workload) -> np.ndarray:

@@ -244,3 +244,80 @@ def test_adamw_matches_torch():
         opt.step()
         p, m, v = optim.adamw_step(p, g, m, v, t, lr=1e-2, b1=0.9, b2=0.95, eps=1e-8, wd=0.1)
         np.testing.assert_allclose(p, tp.detach().numpy(), rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- DPO (preference step)
+def _dpo_inputs(wl):
+    raw = [syn.layer_weights(wl, i) for i in range(wl.n_layers)]
+    head = (syn.embedding(wl), syn.norm_gain(wl), syn.lm_head(wl))
+    toks, tgts, mask = syn.preference_pairs(wl)
+    return raw, head, toks, tgts, mask
+
+
+def test_dpo_loss_is_log2_when_policy_equals_reference():
+    # B = 0 on every adapter: the policy is the reference, so z = 0 and the loss is ln 2
+    wl = tiny(batch=4)
+    raw, head, toks, tgts, mask = _dpo_inputs(wl)
+    lora = [{p: (r["A"][p].astype(np.float64), np.zeros_like(r["B"][p], dtype=np.float64)) for p in M.PROJ}
+            for r in raw]
+    out = M.dpo_step(wl, raw, head, toks, tgts, 2, 0.1, mask=mask, lora=lora)
+    assert np.array_equal(out["pi"], out["ref"])
+    assert out["loss"] == math.log(2.0)
+    # the gradient is still live: dL/dz = -1/2 at z = 0
+    assert any(np.abs(dB).max() > 0 for g in out["grads"] for (_, dB) in g.values())
+
+
+def test_dpo_identical_pair_has_no_gradient():
+    # chosen == rejected: both sequences get opposite weights, so every gradient cancels
+    wl = tiny(batch=2)
+    raw, head, toks, tgts, mask = _dpo_inputs(wl)
+    S = wl.seq
+    toks[S:], tgts[S:], mask[S:] = toks[:S], tgts[:S], mask[:S]
+    out = M.dpo_step(wl, raw, head, toks, tgts, 1, 0.5, mask=mask)
+    assert abs(out["loss"] - math.log(2.0)) < 1e-15
+    for g in out["grads"]:
+        for dA, dB in g.values():
+            assert np.abs(dA).max() < 1e-14 and np.abs(dB).max() < 1e-14
+
+
+def test_dpo_logit_gradient_matches_torch_autograd():
+    # the loss as a function of the logits, differentiated by torch on CPU (fp64)
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(3)
+    nseq, S, V, beta = 4, 6, 11, 0.3
+    logits = rng.normal(size=(nseq * S, V)) * 2
+    tg = rng.integers(0, V, nseq * S)
+    mask = (rng.random(nseq * S) < 0.7).astype(np.float64)
+    ref = rng.normal(size=nseq) * 3
+    loss, dlog, pi = M.dpo_dlogits(logits, tg, mask, nseq, S, ref, beta)
+    lt = torch.tensor(logits, requires_grad=True)
+    lp = torch.log_softmax(lt, dim=1).gather(1, torch.tensor(tg)[:, None])[:, 0] * torch.tensor(mask)
+    pit = lp.reshape(nseq, S).sum(1)
+    r = torch.tensor(ref)
+    P = nseq // 2
+    z = beta * ((pit[:P] - r[:P]) - (pit[P:] - r[P:]))
+    lt_loss = -torch.nn.functional.logsigmoid(z).mean()
+    lt_loss.backward()
+    assert abs(float(lt_loss.detach()) - loss) < 1e-12
+    assert np.allclose(pit.detach().numpy(), pi, rtol=0, atol=1e-12)
+    assert np.allclose(lt.grad.numpy(), dlog, rtol=0, atol=1e-13)
+
+
+def test_dpo_backward_matches_finite_differences():
+    wl = tiny(batch=2, n_layers=1)
+    raw, head, toks, tgts, mask = _dpo_inputs(wl)
+    lora0 = [{p: (r["A"][p].astype(np.float64), r["B"][p].astype(np.float64)) for p in M.PROJ} for r in raw]
+    ref = M.dpo_step(wl, raw, head, toks, tgts, 1, 0.5, mask=mask, lora=lora0)
+    rng = np.random.default_rng(11)
+    h = 1e-4
+    for proj in M.PROJ:
+        for which in (0, 1):
+            an = ref["grads"][0][proj][which]
+            idx = tuple(rng.integers(0, s) for s in an.shape)
+            vals = []
+            for sgn in (1, -1):
+                lora = [{p: (A.copy(), B.copy()) for p, (A, B) in l.items()} for l in lora0]
+                lora[0][proj][which][idx] += sgn * h
+                vals.append(M.dpo_step(wl, raw, head, toks, tgts, 1, 0.5, mask=mask, lora=lora)["loss"])
+            fd = (vals[0] - vals[1]) / (2 * h)
+            assert abs(fd - an[idx]) <= 1e-6 * np.abs(an).max() + 1e-11, (proj, which, fd, an[idx])
