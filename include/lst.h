@@ -167,6 +167,21 @@ lst_status lst_step(lst_ctx* ctx, const int32_t* tokens, const int32_t* targets,
 lst_status lst_step_hidden(lst_ctx* ctx, const uint16_t* x, const uint16_t* g, int32_t batch,
                            int32_t seq, float* loss, float* grads);
 
+/* One DPO training step over the streamed base ("Soup CLI fine-tunes Llama-3.1-8B on a 4 GB laptop
+ * GPU, and that changes who owns AI", paragraph on the economics: preference training with the
+ * reference model being the same streamed base with its adapters switched off; loss of Rafailov et
+ * al., "Direct Preference Optimization", 2023). The batch is 2 * n_pairs sequences of `seq` tokens:
+ * the n_pairs chosen sequences, then the n_pairs rejected ones in the same pair order. tokens,
+ * targets and mask are int32 [2 * n_pairs * seq] (host or device); mask (NULL = all ones) marks the
+ * positions whose target log-likelihood counts towards a sequence's log-likelihood pi.
+ * The step runs the reference forward with the adapters off (L layer reads), then the policy
+ * forward, head and backward (2L reads): 3L reads, or fewer with reuse. *loss (host) = mean over
+ * the pairs of -log sigmoid(beta * ((pi_w - ref_w) - (pi_l - ref_l))); grads as in lst_step.
+ * Needs vocab > 0, 2 * n_pairs <= max_batch, beta > 0. */
+lst_status lst_step_dpo(lst_ctx* ctx, const int32_t* tokens, const int32_t* targets,
+                        const int32_t* mask, int32_t n_pairs, int32_t seq, float beta, float* loss,
+                        float* grads);
+
 /* Copy the last step's logits [batch * seq, V] fp32 to dst (host or device). */
 lst_status lst_get_logits(lst_ctx* ctx, float* dst);
 

@@ -72,6 +72,7 @@ _SIGS = {
     "lst_get_logits": (_I32, [_P, _P]),
     "lst_get_activation": (_I32, [_P, _I32, _I32, _P]),
     "lst_set_profiling": (_I32, [_P, _I32]),
+    "lst_step_dpo": (_I32, [_P, _P, _P, _P, _I32, _I32, _F32, C.POINTER(C.c_float), _P]),
     "lst_set_reuse": (_I32, [_P, _I32]),
     "lst_get_stats": (_I32, [_P, C.POINTER(Stats)]),
     "lst_last_error": (C.c_char_p, [_P]),
@@ -234,6 +235,13 @@ class Context:
         loss = C.c_float()
         _check(lib().lst_step_hidden(self.h, _ptr(x_bits), _ptr(g_bits), batch, seq, C.byref(loss),
                                      _ptr(grads)), self.h, "lst_step_hidden")
+        return loss.value
+
+    def step_dpo(self, tokens, targets, mask, n_pairs: int, seq: int, beta: float, grads=None) -> float:
+        """DPO step on 2 * n_pairs sequences (chosen first); mask may be None (all positions)."""
+        loss = C.c_float()
+        _check(lib().lst_step_dpo(self.h, _ptr(tokens), _ptr(targets), _ptr(mask), n_pairs, seq, beta,
+                                  C.byref(loss), _ptr(grads)), self.h, "lst_step_dpo")
         return loss.value
 
     def logits(self, dst) -> None:

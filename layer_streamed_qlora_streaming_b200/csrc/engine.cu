@@ -163,6 +163,9 @@ enum { PC_GEMM = 0, PC_ATTN = 1, PC_DEQ = 2, PC_OTHER = 3, PC_COPY = 4, PC_LORA 
 
 }  // namespace
 
+enum ReadKind { RD_REF = 0, RD_FWD = 1, RD_BWD = 2 };
+enum HeadMode { HEAD_SFT = 0, HEAD_HIDDEN = 1, HEAD_DPO = 2 };
+
 struct ReadPlan {
   int slot = 0;         // pool slot the read computes from
   bool copy = true;     // the layer is copied into the slot for this read
@@ -222,6 +225,13 @@ struct lst_ctx {
   float *rstdf = nullptr, *logits = nullptr, *loss_rows = nullptr, *loss_dev = nullptr, *dot_part = nullptr;
   __nv_bfloat16* dlog = nullptr;
   int64_t head_rows = 0;      // token rows per head pass (logits / dlogits buffers hold this many)
+  // preference (DPO) step
+  bool adapters_off = false;  // the layer GEMMs skip the LoRA term (reference pass)
+  float* lse_rows = nullptr;  // [T] row logsumexp of the logits
+  float *seq_pi = nullptr, *seq_ref = nullptr, *w_seq = nullptr;  // [max_batch] per sequence
+  int32_t* mask_dev = nullptr;  // [T] positions that count (DPO)
+  bool have_mask = false;
+  float dpo_beta = 0.f;
   bool logits_whole = false;  // the last step's logits are all in `logits`
   __nv_bfloat16* gbuf = nullptr;
   int32_t *tok = nullptr, *tgt = nullptr;
@@ -229,6 +239,8 @@ struct lst_ctx {
   float* host_loss = nullptr;
 
   std::vector<cudaEvent_t> ev_loaded, ev_free;
+  // the step's layer reads in order: layer index and kind (reference forward, forward, backward)
+  std::vector<int> rd_layer, rd_kind;
   // pool slot use per read (see plan_reads)
   std::vector<ReadPlan> plan;
   int plan_held[2] = {-1, -1};   // layers the slots hold once the planned step has run
@@ -374,7 +386,8 @@ lst_status group_fwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
   const Group& G = c->grp[g];
   const auto& D = c->der[layer * NGROUP + g];
   const int64_t T = c->curT;
-  {
+  const bool lora = !c->adapters_off;
+  if (lora) {
     ProfScope ps(c, c->stream, PC_LORA);  // Us = bf16(s * X Acat^T)
     CK(lora_skinny(X, ldx, T, G.in, D.Acat16, G.in, 0, G.KP, c->s, c->Us[g], c->stream));
   }
@@ -388,11 +401,13 @@ lst_status group_fwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
   a.B = group_w(c, W, g);
   a.ldb = G.in;
   a.b_mn = 0;
-  a.A2 = c->Us[g];
-  a.lda2 = G.KP;
-  a.B2 = D.Bexp16;
-  a.ldb2 = G.KP;
-  a.K2 = G.KP;
+  if (lora) {
+    a.A2 = c->Us[g];
+    a.lda2 = G.KP;
+    a.B2 = D.Bexp16;
+    a.ldb2 = G.KP;
+    a.K2 = G.KP;
+  }
   a.C = Y;
   a.ldc = ldy;
   a.c_f32 = y_f32;
@@ -406,7 +421,7 @@ lst_status group_fwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
     a.rope_hd = c->hd;
     a.rope_S = (int)c->curS;
   }
-  ProfScope ps(c, c->stream, PC_GEMM, 2.0 * T * G.out * (double)(G.in + G.KP));
+  ProfScope ps(c, c->stream, PC_GEMM, 2.0 * T * G.out * (double)(G.in + (lora ? G.KP : 0)));
   CK(gemm_bf16(a, c->stream));
   return LST_OK;
 }
@@ -629,9 +644,92 @@ lst_status head_fwd_bwd(lst_ctx* c) {
   return LST_OK;
 }
 
-// Reads n = 0 .. 2L-1 visit layer j(n) = n < L ? n : 2L-1-n (forward, then backward with
-// recompute). plan_reads decides, for each read, the pool slot it computes from and whether the
-// layer is copied into that slot first:
+// logits of token rows [r0, r0 + rows) into c->logits
+lst_status head_logits(lst_ctx* c, int64_t r0, int64_t rows) {
+  GemmArgs a;
+  a.M = (int)rows;
+  a.N = c->V;
+  a.K = c->d;
+  a.A = c->nf + r0 * c->d;
+  a.lda = c->d;
+  a.B = c->H;
+  a.ldb = c->d;
+  a.b_mn = 0;
+  a.C = c->logits;
+  a.ldc = c->V;
+  a.c_f32 = 1;
+  ProfScope ps(c, c->stream, PC_GEMM, 2.0 * rows * c->V * (double)c->d);
+  CK(gemm_bf16(a, c->stream));
+  return LST_OK;
+}
+
+// Final norm, logits and per-sequence log-likelihood of the targets (masked positions) into out;
+// leaves lse_rows and, when one pass covers every row, the logits.
+lst_status head_seq_logp(lst_ctx* c, float* out) {
+  const int64_t T = c->curT;
+  const float* xL = c->xs + (int64_t)c->L * c->Tmax * c->d;
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(rmsnorm_fwd(xL, c->gf, T, c->d, c->cfg.rms_eps, c->nf, c->rstdf, c->stream));
+  }
+  for (int64_t r0 = 0; r0 < T; r0 += c->head_rows) {
+    const int64_t rows = std::min<int64_t>(c->head_rows, T - r0);
+    TRY(head_logits(c, r0, rows));
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(ce_stats(c->logits, rows, c->V, c->tgt + r0, c->lse_rows + r0, c->loss_rows + r0, c->stream));
+  }
+  ProfScope ps(c, c->stream, PC_OTHER);
+  CK(seq_sum(c->loss_rows, c->have_mask ? c->mask_dev : nullptr, (int)c->curB, (int)c->curS, out, c->stream));
+  return LST_OK;
+}
+
+// Reference model of the DPO step: the adapters-off pass just ran; keep its sequence log-likelihoods.
+lst_status head_ref(lst_ctx* c) { return head_seq_logp(c, c->seq_ref); }
+
+// Policy head of the DPO step: sequence log-likelihoods, the DPO loss and per-sequence weights,
+// then dlogits = w (softmax - onehot) on masked rows and the head's backward (logits recomputed
+// per pass when the head runs in more than one pass).
+lst_status head_dpo(lst_ctx* c) {
+  const int64_t T = c->curT;
+  const float* xL = c->xs + (int64_t)c->L * c->Tmax * c->d;
+  TRY(head_seq_logp(c, c->seq_pi));
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(dpo_loss(c->seq_pi, c->seq_ref, (int)(c->curB / 2), c->dpo_beta, c->loss_dev, c->w_seq, c->stream));
+  }
+  const bool one_pass = T <= c->head_rows;
+  for (int64_t r0 = 0; r0 < T; r0 += c->head_rows) {
+    const int64_t rows = std::min<int64_t>(c->head_rows, T - r0);
+    if (!one_pass) TRY(head_logits(c, r0, rows));
+    {
+      ProfScope ps(c, c->stream, PC_OTHER);
+      CK(ce_grad(c->logits, rows, r0, c->V, c->tgt, c->lse_rows, c->w_seq, c->have_mask ? c->mask_dev : nullptr,
+                 (int)c->curS, c->dlog, c->stream));
+    }
+    GemmArgs a;
+    a.M = (int)rows;
+    a.N = c->d;
+    a.K = c->V;
+    a.A = c->dlog;
+    a.lda = c->V;
+    a.B = c->H;
+    a.ldb = c->d;
+    a.b_mn = 1;
+    a.C = c->dn + r0 * c->d;
+    a.ldc = c->d;
+    a.c_f32 = 1;
+    ProfScope ps(c, c->stream, PC_GEMM, 2.0 * rows * c->V * (double)c->d);
+    CK(gemm_bf16(a, c->stream));
+  }
+  ProfScope ps(c, c->stream, PC_OTHER);
+  CK(rmsnorm_bwd(c->dn, xL, c->gf, c->rstdf, nullptr, T, c->d, c->ga, c->dout_b, c->stream));
+  return LST_OK;
+}
+
+// An SFT step reads layers 0 .. L-1 (forward), then L-1 .. 0 (backward with recompute); a DPO step
+// first reads 0 .. L-1 once more for the reference forward (adapters off): 2L or 3L reads.
+// plan_reads decides, for each read, the pool slot it computes from and whether the layer is
+// copied into that slot first:
 //  - reuse off: every read copies, into slot n % 2 (2L copies per step);
 //  - reuse on: a read whose layer is still held by a slot (the two layers at the forward/backward
 //    turn; layers 0 and 1 left by the previous step's backward) uses it as it is; otherwise it copies
@@ -641,9 +739,9 @@ lst_status head_fwd_bwd(lst_ctx* c) {
 // a scratch that still holds its layer only with reuse on), on the prep stream, one read ahead: the
 // dequant of read n+1 overlaps the compute of read n.
 void plan_reads(lst_ctx* c) {
-  const int L = c->L, R = 2 * L;
+  const int R = (int)c->rd_layer.size();
   const bool reuse = c->cfg.reuse != 0;
-  auto layer_of = [L](int n) { return n < L ? n : 2 * L - 1 - n; };
+  auto layer_of = [c](int n) { return c->rd_layer[n]; };
   int held[2] = {reuse ? c->slot_layer[0] : -1, reuse ? c->slot_layer[1] : -1};
   int last_use[2] = {-1, -1}, loaded_by[2] = {-1, -1};
   int wheld[2] = {reuse ? c->w_layer[0] : -1, reuse ? c->w_layer[1] : -1};
@@ -701,8 +799,7 @@ void plan_reads(lst_ctx* c) {
 }
 
 lst_status enqueue_copy(lst_ctx* c, int n) {
-  const int L = c->L;
-  const int j = n < L ? n : 2 * L - 1 - n;
+  const int j = c->rd_layer[n];
   const ReadPlan& p = c->plan[n];
   if (c->faults.fail_memcpy()) return fail(c, LST_ERR_CUDA, "layer copy enqueue failed (injected)");
   if (p.wait_free >= 0) CK(cudaStreamWaitEvent(c->copy_stream, c->ev_free[p.wait_free], 0));
@@ -717,7 +814,7 @@ lst_status enqueue_copy(lst_ctx* c, int n) {
 
 // Enqueue, in read order, every planned copy whose slot is released by a read <= done.
 lst_status issue_copies(lst_ctx* c, int done, int& next) {
-  const int R = 2 * c->L;
+  const int R = (int)c->rd_layer.size();
   while (next < R) {
     const ReadPlan& p = c->plan[next];
     if (p.copy) {
@@ -729,13 +826,47 @@ lst_status issue_copies(lst_ctx* c, int done, int& next) {
   return LST_OK;
 }
 
-lst_status run_layers(lst_ctx* c, bool head) {
-  const int L = c->L, R = 2 * L;
+void build_reads(lst_ctx* c, HeadMode mode) {
+  const int L = c->L;
+  c->rd_layer.clear();
+  c->rd_kind.clear();
+  if (mode == HEAD_DPO) {
+    for (int i = 0; i < L; ++i) {
+      c->rd_layer.push_back(i);
+      c->rd_kind.push_back(RD_REF);
+    }
+  }
+  for (int i = 0; i < L; ++i) {
+    c->rd_layer.push_back(i);
+    c->rd_kind.push_back(RD_FWD);
+  }
+  for (int i = L - 1; i >= 0; --i) {
+    c->rd_layer.push_back(i);
+    c->rd_kind.push_back(RD_BWD);
+  }
+}
+
+lst_status head_after(lst_ctx* c, int kind, HeadMode mode) {
+  if (kind == RD_REF) return head_ref(c);
+  if (mode == HEAD_DPO) return head_dpo(c);
+  if (mode == HEAD_SFT) return head_fwd_bwd(c);
+  const int64_t T = c->curT;
+  const float* xL = c->xs + (int64_t)c->L * c->Tmax * c->d;
+  ProfScope ps(c, c->stream, PC_OTHER);
+  CK(dot_fixed(xL, c->gbuf, T * c->d, c->dot_part, c->loss_dev, c->stream));
+  CK(cudaMemcpyAsync(c->dout_b, c->gbuf, T * c->d * 2, cudaMemcpyDeviceToDevice, c->stream));
+  CK(bf16_to_f32(c->gbuf, T * c->d, c->ga, c->stream));
+  return LST_OK;
+}
+
+lst_status run_layers(lst_ctx* c, HeadMode mode) {
+  const int L = c->L;
   const bool streamed = c->cfg.streamed != 0;
   const bool nf4 = c->cfg.base_format != LST_BASE_BF16;
+  build_reads(c, mode);
+  const int R = (int)c->rd_layer.size();
   auto blob_of = [&](int n) -> const uint8_t* {
-    const int j = n < L ? n : 2 * L - 1 - n;
-    return streamed ? c->pool[c->plan[n].slot] : c->resident + (int64_t)j * c->lay.total;
+    return streamed ? c->pool[c->plan[n].slot] : c->resident + (int64_t)c->rd_layer[n] * c->lay.total;
   };
   plan_reads(c);
   // the slots' and scratches' contents are only trusted again once this step has completed
@@ -760,7 +891,7 @@ lst_status run_layers(lst_ctx* c, bool head) {
   };
   TRY(enqueue_deq(0));
   for (int n = 0; n < R; ++n) {
-    const int j = n < L ? n : 2 * L - 1 - n;
+    const int j = c->rd_layer[n], kind = c->rd_kind[n];
     const ReadPlan& p = c->plan[n];
     TRY(enqueue_deq(n + 1));
     const uint8_t* blob = blob_of(n);
@@ -772,27 +903,22 @@ lst_status run_layers(lst_ctx* c, bool head) {
     } else {
       W = reinterpret_cast<const __nv_bfloat16*>(blob + c->lay.w16);
     }
-    if (n < L) {
+    if (kind == RD_REF) {
+      c->adapters_off = true;
+      const lst_status st = layer_fwd(c, j, blob, W, false);
+      c->adapters_off = false;
+      TRY(st);
+    } else if (kind == RD_FWD) {
       TRY(layer_fwd(c, j, blob, W, false));
     } else {
       TRY(layer_fwd(c, j, blob, W, true));
       TRY(layer_bwd(c, j, blob, W));
     }
     CK(cudaEventRecord(c->ev_free[n], c->stream));
-    if (n == L - 1) {
-      if (head) {
-        TRY(head_fwd_bwd(c));
-      } else {
-        const int64_t T = c->curT;
-        const float* xL = c->xs + (int64_t)L * c->Tmax * c->d;
-        ProfScope ps(c, c->stream, PC_OTHER);
-        CK(dot_fixed(xL, c->gbuf, T * c->d, c->dot_part, c->loss_dev, c->stream));
-        CK(cudaMemcpyAsync(c->dout_b, c->gbuf, T * c->d * 2, cudaMemcpyDeviceToDevice, c->stream));
-        CK(bf16_to_f32(c->gbuf, T * c->d, c->ga, c->stream));
-      }
-    }
+    if (kind != RD_BWD && (n + 1 == R || c->rd_kind[n + 1] != kind)) TRY(head_after(c, kind, mode));
     if (streamed) TRY(issue_copies(c, n, next_copy));
   }
+  (void)L;
   return LST_OK;
 }
 
@@ -1079,15 +1205,20 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
     TRY(dalloc(c, &c->logits, c->head_rows * c->V));
     TRY(dalloc(c, &c->dlog, c->head_rows * c->V));
     TRY(dalloc(c, &c->loss_rows, T));
+    TRY(dalloc(c, &c->lse_rows, T));
+    TRY(dalloc(c, &c->mask_dev, T));
+    TRY(dalloc(c, &c->seq_pi, k.max_batch));
+    TRY(dalloc(c, &c->seq_ref, k.max_batch));
+    TRY(dalloc(c, &c->w_seq, k.max_batch));
     TRY(dalloc(c, &c->tok, T));
     TRY(dalloc(c, &c->tgt, T));
   } else {
     TRY(dalloc(c, &c->gbuf, T * d));
   }
-  c->ev_loaded.resize(2 * c->L);
-  c->ev_free.resize(2 * c->L);
-  c->ev_deq.resize(2 * c->L);
-  for (int i = 0; i < 2 * c->L; ++i) {
+  c->ev_loaded.resize(3 * c->L);  // up to 3L reads per step (DPO)
+  c->ev_free.resize(3 * c->L);
+  c->ev_deq.resize(3 * c->L);
+  for (int i = 0; i < 3 * c->L; ++i) {
     CK(cudaEventCreateWithFlags(&c->ev_loaded[i], cudaEventDisableTiming));
     CK(cudaEventCreateWithFlags(&c->ev_free[i], cudaEventDisableTiming));
     CK(cudaEventCreateWithFlags(&c->ev_deq[i], cudaEventDisableTiming));
@@ -1289,7 +1420,7 @@ lst_status lst_step(lst_ctx* c, const int32_t* tokens, const int32_t* targets, i
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(embed(c->tok, c->E, c->curT, c->d, c->V, c->xs, c->stream));
   }
-  TRY(run_layers(c, true));
+  TRY(run_layers(c, HEAD_SFT));
   TRY(optimizer_update(c));
   c->have_logits = true;
   return finish_step(c, loss, grads);
@@ -1304,7 +1435,30 @@ lst_status lst_step_hidden(lst_ctx* c, const uint16_t* x, const uint16_t* g, int
   TRY(copy_in(c, c->dout_b, x, c->curT * c->d * 2));  // bf16 input staged, widened to fp32
   CK(bf16_to_f32(c->dout_b, c->curT * c->d, c->xs, c->stream));
   TRY(copy_in(c, c->gbuf, g, c->curT * c->d * 2));
-  TRY(run_layers(c, false));
+  TRY(run_layers(c, HEAD_HIDDEN));
+  TRY(optimizer_update(c));
+  c->have_logits = false;
+  return finish_step(c, loss, grads);
+}
+
+lst_status lst_step_dpo(lst_ctx* c, const int32_t* tokens, const int32_t* targets, const int32_t* mask,
+                        int32_t n_pairs, int32_t seq, float beta, float* loss, float* grads) {
+  if (!c) return LST_ERR_ARG;
+  if (!tokens || !targets || !loss) return fail(c, LST_ERR_ARG, "null tokens/targets/loss");
+  if (c->V <= 0) return fail(c, LST_ERR_STATE, "lst_step_dpo needs a head (vocab > 0)");
+  if (n_pairs <= 0 || !(beta > 0.f) || !std::isfinite(beta)) return fail(c, LST_ERR_ARG, "n_pairs <= 0 or beta not > 0");
+  if ((int64_t)2 * n_pairs > c->cfg.max_batch) return fail(c, LST_ERR_ARG, "2 * n_pairs above max_batch");
+  TRY(begin_step(c, 2 * n_pairs, seq));
+  TRY(copy_in(c, c->tok, tokens, c->curT * 4));
+  TRY(copy_in(c, c->tgt, targets, c->curT * 4));
+  c->have_mask = mask != nullptr;
+  if (mask) TRY(copy_in(c, c->mask_dev, mask, c->curT * 4));
+  c->dpo_beta = beta;
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(embed(c->tok, c->E, c->curT, c->d, c->V, c->xs, c->stream));
+  }
+  TRY(run_layers(c, HEAD_DPO));
   TRY(optimizer_update(c));
   c->have_logits = false;
   return finish_step(c, loss, grads);

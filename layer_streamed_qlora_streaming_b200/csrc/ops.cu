@@ -290,6 +290,105 @@ k_ce(const float* __restrict__ logits, int V, const int32_t* __restrict__ y, flo
   }
 }
 
+// Row (max, sum of exp) of a logits row by the online rule of k_ce, merged in a fixed tree.
+__device__ __forceinline__ float row_lse(const float* __restrict__ lr, int V, float* sm, float* ss) {
+  float m = -INFINITY, s = 0.f;
+  if ((V % 4) == 0) {
+    const float4* l4 = reinterpret_cast<const float4*>(lr);
+    for (int c = threadIdx.x; c < V / 4; c += blockDim.x) ms_add4(m, s, __ldg(l4 + c));
+  } else {
+    for (int c = threadIdx.x; c < V; c += blockDim.x) ms_add4(m, s, make_float4(lr[c], -INFINITY, -INFINITY, -INFINITY));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    ms_merge(m, s, m2, s2);
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    sm[w] = m;
+    ss[w] = s;
+  }
+  __syncthreads();
+  m = sm[0];
+  s = ss[0];
+  for (int i = 1; i < (int)(blockDim.x >> 5); ++i) ms_merge(m, s, sm[i], ss[i]);
+  return m + logf(s);
+}
+
+__global__ void __launch_bounds__(1024, 1)
+k_ce_stats(const float* __restrict__ logits, int V, const int32_t* __restrict__ y, float* __restrict__ lse_out,
+           float* __restrict__ logp_out) {
+  __shared__ float sm[32], ss[32];
+  const int64_t row = blockIdx.x;
+  const float* lr = logits + row * V;
+  const float lse = row_lse(lr, V, sm, ss);
+  if (threadIdx.x == 0) {
+    int tgt = y[row];
+    if (tgt < 0 || tgt >= V) {
+      dev_fail(DEV_ERR_BAD_INDEX);
+      tgt = 0;
+    }
+    lse_out[row] = lse;
+    logp_out[row] = lr[tgt] - lse;
+  }
+}
+
+// One block per sequence; the block_sum tree fixes the order.
+__global__ void k_seq_sum(const float* __restrict__ v, const int32_t* __restrict__ mask, int S, float* __restrict__ out) {
+  __shared__ float red[32];
+  const int64_t base = (int64_t)blockIdx.x * S;
+  float acc = 0.f;
+  for (int t = threadIdx.x; t < S; t += blockDim.x) acc += mask ? (float)mask[base + t] * v[base + t] : v[base + t];
+  acc = block_sum(acc, red);
+  if (threadIdx.x == 0) out[blockIdx.x] = acc;
+}
+
+__global__ void k_dpo(const float* __restrict__ pi, const float* __restrict__ ref, int P, float beta,
+                      float* __restrict__ loss, float* __restrict__ w) {
+  __shared__ float red[32];
+  float part = 0.f;
+  for (int p = threadIdx.x; p < P; p += blockDim.x) {
+    const float z = beta * ((pi[p] - ref[p]) - (pi[P + p] - ref[P + p]));
+    part += fmaxf(-z, 0.f) + log1pf(expf(-fabsf(z)));  // -log sigmoid(z), overflow-free
+    const float g = (1.0f / (1.0f + expf(-z)) - 1.0f) * beta / (float)P;  // dloss/dpi of the chosen one
+    w[p] = -g;
+    w[P + p] = g;
+  }
+  part = block_sum(part, red);
+  if (threadIdx.x == 0) *loss = part / (float)P;
+}
+
+__global__ void __launch_bounds__(1024, 1)
+k_ce_grad(const float* __restrict__ logits, int64_t row0, int V, const int32_t* __restrict__ y,
+          const float* __restrict__ lse_rows, const float* __restrict__ wseq, const int32_t* __restrict__ mask, int S,
+          bf16* __restrict__ dlog) {
+  const int64_t lrow = blockIdx.x, row = row0 + lrow;
+  const float* lr = logits + lrow * V;
+  bf16* dr = dlog + lrow * V;
+  const float lse = lse_rows[row];
+  const float w = wseq[row / S] * (mask ? (float)mask[row] : 1.0f);
+  int tgt = y[row];
+  if (tgt < 0 || tgt >= V) tgt = 0;  // reported by k_ce_stats
+  if ((V % 4) == 0) {
+    const float4* l4 = reinterpret_cast<const float4*>(lr);
+    for (int c = threadIdx.x; c < V / 4; c += blockDim.x) {
+      const float4 v = __ldg(l4 + c);
+      float p[4] = {expf(v.x - lse), expf(v.y - lse), expf(v.z - lse), expf(v.w - lse)};
+      const int d = tgt - 4 * c;
+      if (d >= 0 && d < 4) p[d] -= 1.0f;
+      const __nv_bfloat162 h[2] = {__floats2bfloat162_rn(p[0] * w, p[1] * w), __floats2bfloat162_rn(p[2] * w, p[3] * w)};
+      *reinterpret_cast<uint2*>(dr + 4 * c) = *reinterpret_cast<const uint2*>(h);
+    }
+  } else {
+    for (int c = threadIdx.x; c < V; c += blockDim.x) {
+      float p = expf(lr[c] - lse);
+      if (c == tgt) p -= 1.0f;
+      dr[c] = __float2bfloat16_rn(p * w);
+    }
+  }
+}
+
 __global__ void k_mean(const float* __restrict__ v, int64_t n, float* __restrict__ out) {
   __shared__ float red[32];
   float s = 0.f;
@@ -375,6 +474,27 @@ cudaError_t embed(const int32_t* tok, const bf16* E, int64_t T, int d, int V, fl
 cudaError_t cross_entropy(const float* logits, int64_t T, int V, const int32_t* y, float inv_T, float* loss_rows,
                           bf16* dlog, cudaStream_t s) {
   k_ce<<<(unsigned)T, 1024, 0, s>>>(logits, V, y, inv_T, loss_rows, dlog);
+  note_launch(1);
+  return cudaGetLastError();
+}
+cudaError_t ce_stats(const float* logits, int64_t T, int V, const int32_t* y, float* lse, float* logp, cudaStream_t s) {
+  k_ce_stats<<<(unsigned)T, 1024, 0, s>>>(logits, V, y, lse, logp);
+  note_launch(1);
+  return cudaGetLastError();
+}
+cudaError_t seq_sum(const float* v, const int32_t* mask, int nseq, int S, float* out, cudaStream_t s) {
+  k_seq_sum<<<nseq, 256, 0, s>>>(v, mask, S, out);
+  note_launch(1);
+  return cudaGetLastError();
+}
+cudaError_t dpo_loss(const float* pi, const float* ref, int P, float beta, float* loss, float* w, cudaStream_t s) {
+  k_dpo<<<1, 256, 0, s>>>(pi, ref, P, beta, loss, w);
+  note_launch(1);
+  return cudaGetLastError();
+}
+cudaError_t ce_grad(const float* logits, int64_t rows, int64_t row0, int V, const int32_t* y, const float* lse,
+                    const float* w, const int32_t* mask, int S, bf16* dlog, cudaStream_t s) {
+  k_ce_grad<<<(unsigned)rows, 1024, 0, s>>>(logits, row0, V, y, lse, w, mask, S, dlog);
   note_launch(1);
   return cudaGetLastError();
 }

@@ -37,6 +37,20 @@ cudaError_t cross_entropy(const float* logits, int64_t T, int V, const int32_t* 
                           float* loss_rows, bf16* dlogits, cudaStream_t s);
 // out = mean of v[0..n) with a fixed summation order.
 cudaError_t mean_fixed(const float* v, int64_t n, float* out, cudaStream_t s);
+
+// Preference (DPO) head pieces. Row statistics of fp32 logits [T, V]: lse[t] and
+// logp[t] = logits[t][y_t] - lse[t].
+cudaError_t ce_stats(const float* logits, int64_t T, int V, const int32_t* targets, float* lse, float* logp,
+                     cudaStream_t s);
+// out[q] = sum over the S rows of sequence q of mask * v (mask NULL = all ones), fixed order.
+cudaError_t seq_sum(const float* v, const int32_t* mask, int nseq, int S, float* out, cudaStream_t s);
+// DPO over P pairs (sequences [0, P) chosen, [P, 2P) rejected): loss = mean_p -log sigmoid(z_p),
+// z_p = beta ((pi_p - ref_p) - (pi_{P+p} - ref_{P+p})); w[q] = -dloss/dpi_q.
+cudaError_t dpo_loss(const float* pi, const float* ref, int P, float beta, float* loss, float* w, cudaStream_t s);
+// dlogits of rows [row0, row0 + rows) (logits / dlog point at row row0):
+// dlog = bf16(w[row / S] * mask[row] * (softmax(logits_row) - onehot(y_row))).
+cudaError_t ce_grad(const float* logits, int64_t rows, int64_t row0, int V, const int32_t* targets, const float* lse,
+                    const float* w, const int32_t* mask, int S, __nv_bfloat16* dlog, cudaStream_t s);
 // out = sum_i a[i] * b[i] with a fixed order; partials: scratch of 1024 floats.
 cudaError_t dot_fixed(const float* a, const bf16* b, int64_t n, float* partials, float* out, cudaStream_t s);
 
