@@ -383,6 +383,44 @@ def run_gpu(args, wl):
              "note": "steady state: the two layers at the forward/backward turn and layers 0, 1 from the "
                      "previous step are not copied again (2L - 4 reads)"}
 
+    dpo = None
+    if wl.vocab and wl.batch % 2 == 0:
+        # DPO step on the same model: reference forward with the adapters off + policy step (3L reads)
+        dmask = torch.zeros(wl.batch, wl.seq, dtype=torch.int32)
+        dmask[:, wl.seq // 2:] = 1                       # response half counts, prompt half does not
+        dtoks, dtgts = toks.clone().view(wl.batch, wl.seq), tgts.clone().view(wl.batch, wl.seq)
+        P = wl.batch // 2
+        dtoks[P:, :wl.seq // 2] = dtoks[:P, :wl.seq // 2]  # pair p shares its prompt
+        dtgts[P:, :wl.seq // 2] = dtgts[:P, :wl.seq // 2]
+        dt, dy, dm = dtoks.reshape(-1).cuda(), dtgts.reshape(-1).cuda(), dmask.reshape(-1).cuda()
+
+        def dpo_step():
+            loss = ctx.step_dpo(dt, dy, dm, P, wl.seq, 0.1, grads)
+            with torch.cuda.stream(stream):
+                allreduce_grads(grads, dist)
+            return loss
+        for _ in range(2):
+            dpo_step()
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        d0.record(stream)
+        for _ in range(args.steps):
+            dloss = dpo_step()
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dms = max_over_ranks(d0.elapsed_time(d1), dist, "cuda")
+        dst = ctx.stats()
+        dbytes = dst["h2d_bytes_last_step"]
+        dpo = {"value": job_throughput(world, T, args.steps, dms), "unit": UNIT, "ms_per_step": dms / args.steps,
+               "layer_reads_per_step": dst["layer_reads_last_step"], "h2d_bytes_per_step": dbytes,
+               "min_ms": dbytes / (link_gbs * 1e9) * 1e3, "frac": dbytes / (link_gbs * 1e9) * 1e3 / (dms / args.steps),
+               "pairs": P, "beta": 0.1, "loss_last": dloss,
+               "note": "DPO: reference forward with the adapters off, then the policy forward, head and backward "
+                       "(3L reads); tokens/s counts the 2P sequences once"}
+
     st = ctx.stats()
     peaks = measured_peaks()
     K = args.steps
@@ -420,6 +458,8 @@ def run_gpu(args, wl):
     }
     line["e2e"] = e2e
     line["reuse_schedule"] = reuse
+    if dpo is not None:
+        line["dpo"] = dpo
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, secs, desc = oracle_sample(wl, seq=args.ref_seq)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
