@@ -46,6 +46,28 @@ def describe(wl) -> str:
             f"a{int(wl.lora_alpha)} on 7 projections{head}, batch {wl.batch} x seq {wl.seq}")
 
 
+# DRAM traffic (read + write) of the GEMM launches of one llama8b step, from one ncu capture of the
+# bench (dram__bytes_read.sum + dram__bytes_write.sum over the step's 354 k_gemm launches; command
+# and figures in profiles/gemm_traffic_llama8b_step.md). Valid only for the GEMM sources measured.
+GEMM_TRAFFIC = {"workload": "llama8b", "bytes_per_step": 73.988e9, "launches": 354,
+                "sources": {"gemm.cu": "e42c3dc7664d7c3c", "gemm.cuh": "4a668b6d34dc410f",
+                            "common.cuh": "c89033b9dea61163"}}
+
+
+def gemm_traffic(wl_name: str):
+    """(bytes per launch, bytes per step) of the recorded capture, or (None, None) when the
+    workload differs or the GEMM sources changed since it was taken."""
+    import hashlib
+    if wl_name != GEMM_TRAFFIC["workload"]:
+        return None, None
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "layer_streamed_qlora_streaming_b200", "csrc")
+    for f, h in GEMM_TRAFFIC["sources"].items():
+        with open(os.path.join(csrc, f), "rb") as fh:
+            if hashlib.sha256(fh.read()).hexdigest()[:16] != h:
+                return None, None
+    return GEMM_TRAFFIC["bytes_per_step"] / GEMM_TRAFFIC["launches"], GEMM_TRAFFIC["bytes_per_step"]
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -424,6 +446,7 @@ def run_gpu(args, wl):
 
     st = ctx.stats()
     peaks = measured_peaks()
+    traffic_launch, traffic_step = gemm_traffic(args.workload)
     K = args.steps
     gemm_ms = agg["gemm_ms"] / K
     gemm_tflops = agg["gemm_flops"] / K / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else 0.0
@@ -442,7 +465,10 @@ def run_gpu(args, wl):
                    "loss_last": loss},
         "roofline": {"bound": "tensor", "kernel": "tcgen05 bf16 GEMM (all projection + LM-head GEMMs)",
                      "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / peak_t if peak_t else None, "traffic": None,
+                     "frac": gemm_tflops / peak_t if peak_t else None, "traffic": traffic_launch,
+                     "traffic_per_step": traffic_step,
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum over one step's GEMM "
+                                       "launches (average per launch); null when the GEMM sources changed",
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
                      "gemm_ms_per_step": gemm_ms, "gemm_launches_per_step": agg["gemm_launches"] / K},
         "step_roofline": {"bound": "pcie", "h2d_bytes_per_step": h2d_bytes, "link_gbs": link_gbs,

@@ -83,10 +83,17 @@ struct Group {
   int64_t woff = 0;  // element offset of the group's W in the concatenated bf16 weights
 };
 
+// A layer blob is group-major: the small fp32 tensors first (NF4 means, norm gains, q/k/v bias),
+// then the projection groups in compute order (q/k/v, o, gate/up, down), each group holding its
+// packed codes, absmax codes and group scales (NF4) or its bf16 matrices. Chunk g spans
+// [chunk[g], chunk[g + 1]): chunk 0 = the small tensors + q/k/v, then o, gate/up, down, so a layer
+// can be copied (and dequantised) group by group and its compute start on the first group.
+constexpr int NCHUNK = 4;
 struct Layout {
   int64_t n[NPROJ], outd[NPROJ], ind[NPROJ], woff[NPROJ];
   int64_t P = 0;
   int64_t packed[NPROJ], qabs[NPROJ], gscale[NPROJ], means = 0, w16 = 0, norms = 0, bias = 0, total = 0;
+  int64_t chunk[NCHUNK + 1];
 };
 
 bool valid_config(const lst_config* c, std::string* why) {
@@ -127,24 +134,33 @@ Layout make_layout(const lst_config& c) {
     acc += L.n[p];
   }
   L.P = acc;
+  static const int kGroupProj[NCHUNK + 1] = {0, 3, 4, 6, 7};  // projections of each chunk
   int64_t off = 0;
   if (c.base_format == LST_BASE_NF4) {
-    for (int p = 0; p < NPROJ; ++p) { L.packed[p] = off; off = align256(off + L.n[p] / 2); }
-    for (int p = 0; p < NPROJ; ++p) { L.qabs[p] = off; off = align256(off + L.n[p] / 64); }
-    for (int p = 0; p < NPROJ; ++p) {
-      L.gscale[p] = off;
-      off = align256(off + ((L.n[p] / 64 + 255) / 256) * 4);
-    }
     L.means = off;
     off = align256(off + NPROJ * 4);
-  } else {
-    L.w16 = 0;
-    off = align256(L.P * 2);
   }
   L.norms = off;
   off = align256(off + 2 * d * 4);
   L.bias = off;
   if (c.qkv_bias) off = align256(off + (dq + 2 * dkv) * 4);
+  L.chunk[0] = 0;
+  if (c.base_format == LST_BASE_NF4) {
+    for (int g = 0; g < NCHUNK; ++g) {
+      for (int p = kGroupProj[g]; p < kGroupProj[g + 1]; ++p) { L.packed[p] = off; off = align256(off + L.n[p] / 2); }
+      for (int p = kGroupProj[g]; p < kGroupProj[g + 1]; ++p) { L.qabs[p] = off; off = align256(off + L.n[p] / 64); }
+      for (int p = kGroupProj[g]; p < kGroupProj[g + 1]; ++p) {
+        L.gscale[p] = off;
+        off = align256(off + ((L.n[p] / 64 + 255) / 256) * 4);
+      }
+      L.chunk[g + 1] = off;
+    }
+  } else {
+    L.w16 = off;  // the 7 matrices back to back, so q/k/v and gate/up are single matrices
+    for (int g = 0; g < NCHUNK; ++g) L.chunk[g + 1] = L.w16 + L.woff[kGroupProj[g + 1] - 1] * 2 + L.n[kGroupProj[g + 1] - 1] * 2;
+    off = align256(off + L.P * 2);
+    L.chunk[NCHUNK] = off;
+  }
   L.total = off;
   return L;
 }
@@ -238,7 +254,7 @@ struct lst_ctx {
   float *cos_t = nullptr, *sin_t = nullptr;
   float* host_loss = nullptr;
 
-  std::vector<cudaEvent_t> ev_loaded, ev_free;
+  std::vector<cudaEvent_t> ev_chunk, ev_free;  // ev_chunk[n * NCHUNK + g]: chunk g of read n copied
   // the step's layer reads in order: layer index and kind (reference forward, forward, backward)
   std::vector<int> rd_layer, rd_kind;
   // pool slot use per read (see plan_reads)
@@ -247,7 +263,9 @@ struct lst_ctx {
   int slot_layer[2] = {-1, -1};  // layers the slots hold after the last completed step (-1: unknown)
   int plan_wheld[2] = {-1, -1};  // layers the weight scratches hold once the planned step has run
   int w_layer[2] = {-1, -1};     // layers the weight scratches hold after the last completed step
-  std::vector<cudaEvent_t> ev_deq;
+  std::vector<cudaEvent_t> ev_deqg;  // [n * NCHUNK + g]: chunk g of read n dequantised
+  // what the compute stream still waits on for the current read, per chunk: its copy, its dequant
+  cudaEvent_t cur_wait[NCHUNK][2] = {};
   cudaEvent_t ev_done = nullptr, ev_start = nullptr;
 
   float* stage_w = nullptr;
@@ -470,20 +488,34 @@ lst_status group_bwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
 }
 
 // Weights of a layer read: the bf16 [P] matrix the GEMMs consume.
-// NF4 blob -> bf16 weights of the 7 projections in the concatenated [q;k;v], o, [gate;up], down
-// order, written to dst on stream st.
-lst_status dequant_layer(lst_ctx* c, const uint8_t* blob, __nv_bfloat16* dst, cudaStream_t st) {
+// NF4 blob -> bf16 weights of the projections of chunk g (q/k/v, o, gate/up or down), written to
+// dst in the concatenated [q;k;v], o, [gate;up], down order, on stream st.
+lst_status dequant_chunk(lst_ctx* c, const uint8_t* blob, __nv_bfloat16* dst, int g, cudaStream_t st) {
+  static const int first[NCHUNK + 1] = {0, 3, 4, 6, 7};
   Nf4Seg segs[NPROJ];
-  for (int p = 0; p < NPROJ; ++p) {
-    segs[p].packed = blob + c->lay.packed[p];
-    segs[p].qabs = reinterpret_cast<const int8_t*>(blob + c->lay.qabs[p]);
-    segs[p].gscale = reinterpret_cast<const float*>(blob + c->lay.gscale[p]);
-    segs[p].mean = reinterpret_cast<const float*>(blob + c->lay.means) + p;
-    segs[p].n = c->lay.n[p];
-    segs[p].out_offset = c->lay.woff[p];
+  int k = 0;
+  for (int p = first[g]; p < first[g + 1]; ++p, ++k) {
+    segs[k].packed = blob + c->lay.packed[p];
+    segs[k].qabs = reinterpret_cast<const int8_t*>(blob + c->lay.qabs[p]);
+    segs[k].gscale = reinterpret_cast<const float*>(blob + c->lay.gscale[p]);
+    segs[k].mean = reinterpret_cast<const float*>(blob + c->lay.means) + p;
+    segs[k].n = c->lay.n[p];
+    segs[k].out_offset = c->lay.woff[p];
   }
   ProfScope ps(c, st, PC_DEQ);
-  CK(nf4_dequant(segs, NPROJ, dst, st));
+  CK(nf4_dequant(segs, k, dst, st));
+  return LST_OK;
+}
+
+// Make the compute stream wait until chunk g of the current read (its bytes and, for an NF4 base,
+// its dequantised weights) is in place; a no-op once waited or when nothing is pending.
+lst_status wait_chunk(lst_ctx* c, int g) {
+  for (int k = 0; k < 2; ++k) {
+    if (c->cur_wait[g][k]) {
+      CK(cudaStreamWaitEvent(c->stream, c->cur_wait[g][k], 0));
+      c->cur_wait[g][k] = nullptr;
+    }
+  }
   return LST_OK;
 }
 
@@ -494,6 +526,7 @@ lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
   const float* g2 = g1 + c->d;
   const float* bias = c->cfg.qkv_bias ? reinterpret_cast<const float*>(blob + c->lay.bias) : nullptr;
   const float* x = c->xs + (int64_t)i * c->Tmax * c->d;
+  TRY(wait_chunk(c, 0));  // norm gains, bias and the q/k/v weights
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(rmsnorm_fwd(x, g1, T, c->d, c->cfg.rms_eps, c->n1, c->rstd1, c->stream));
@@ -518,16 +551,19 @@ lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
     ProfScope ps(c, c->stream, PC_ATTN);
     CK(attention_fwd(a, c->stream));
   }
+  TRY(wait_chunk(c, 1));
   TRY(group_fwd(c, i, G_O, W, c->o, c->dq, c->h, c->d, 1, nullptr, x, true));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(rmsnorm_fwd(c->h, g2, T, c->d, c->cfg.rms_eps, c->n2, c->rstd2, c->stream));
   }
+  TRY(wait_chunk(c, 2));
   TRY(group_fwd(c, i, G_GU, W, c->n2, c->d, c->gu, 2 * c->F, 0, nullptr, nullptr, true));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(swiglu_fwd(c->gu, T, c->F, c->m, c->stream));
   }
+  TRY(wait_chunk(c, 3));  // also before a recompute: the backward that follows needs W_down
   // the recompute pass needs only the LoRA projection of m (for dB of down), not the output
   TRY(group_fwd(c, i, G_DOWN, W, c->m, c->F, c->xs + (int64_t)(i + 1) * c->Tmax * c->d, c->d, 1, nullptr, c->h,
                 !recompute));
@@ -804,9 +840,12 @@ lst_status enqueue_copy(lst_ctx* c, int n) {
   if (c->faults.fail_memcpy()) return fail(c, LST_ERR_CUDA, "layer copy enqueue failed (injected)");
   if (p.wait_free >= 0) CK(cudaStreamWaitEvent(c->copy_stream, c->ev_free[p.wait_free], 0));
   ProfScope ps(c, c->copy_stream, PC_COPY);
-  CK(cudaMemcpyAsync(c->pool[p.slot], c->arena + (int64_t)j * c->lay.total, c->lay.total, cudaMemcpyHostToDevice,
-                     c->copy_stream));
-  CK(cudaEventRecord(c->ev_loaded[n], c->copy_stream));
+  const uint8_t* src = c->arena + (int64_t)j * c->lay.total;
+  for (int g = 0; g < NCHUNK; ++g) {  // group by group, so compute can start on the first group
+    CK(cudaMemcpyAsync(c->pool[p.slot] + c->lay.chunk[g], src + c->lay.chunk[g], c->lay.chunk[g + 1] - c->lay.chunk[g],
+                       cudaMemcpyHostToDevice, c->copy_stream));
+    CK(cudaEventRecord(c->ev_chunk[n * NCHUNK + g], c->copy_stream));
+  }
   c->st.layer_reads_last_step += 1;
   c->st.h2d_bytes_last_step += c->lay.total;
   return LST_OK;
@@ -879,14 +918,18 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
   CK(cudaStreamWaitEvent(c->prep_stream, c->ev_start, 0));
   int next_copy = 0;
   if (streamed) TRY(issue_copies(c, -1, next_copy));
-  // dequant of read m on the prep stream; every event it waits on is already recorded
+  // dequant of read m on the prep stream, chunk by chunk as the copy lands; every event it waits on
+  // is already recorded
   auto enqueue_deq = [&](int m) -> lst_status {
     if (m >= R || !c->plan[m].deq) return LST_OK;
     const ReadPlan& p = c->plan[m];
-    if (streamed && p.loaded_by >= 0) CK(cudaStreamWaitEvent(c->prep_stream, c->ev_loaded[p.loaded_by], 0));
     if (p.wwait >= 0) CK(cudaStreamWaitEvent(c->prep_stream, c->ev_free[p.wwait], 0));
-    TRY(dequant_layer(c, blob_of(m), c->wscr[p.wslot], c->prep_stream));
-    CK(cudaEventRecord(c->ev_deq[m], c->prep_stream));
+    for (int g = 0; g < NCHUNK; ++g) {
+      if (streamed && p.loaded_by >= 0)
+        CK(cudaStreamWaitEvent(c->prep_stream, c->ev_chunk[p.loaded_by * NCHUNK + g], 0));
+      TRY(dequant_chunk(c, blob_of(m), c->wscr[p.wslot], g, c->prep_stream));
+      CK(cudaEventRecord(c->ev_deqg[m * NCHUNK + g], c->prep_stream));
+    }
     return LST_OK;
   };
   TRY(enqueue_deq(0));
@@ -895,14 +938,15 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
     const ReadPlan& p = c->plan[n];
     TRY(enqueue_deq(n + 1));
     const uint8_t* blob = blob_of(n);
-    if (streamed && p.loaded_by >= 0) CK(cudaStreamWaitEvent(c->stream, c->ev_loaded[p.loaded_by], 0));
-    const __nv_bfloat16* W;
-    if (nf4) {
-      if (p.wfilled_by >= 0) CK(cudaStreamWaitEvent(c->stream, c->ev_deq[p.wfilled_by], 0));
-      W = c->wscr[p.wslot];
-    } else {
-      W = reinterpret_cast<const __nv_bfloat16*>(blob + c->lay.w16);
+    // the compute of chunk g waits for the copy that filled the slot and, for an NF4 base, the
+    // dequant that filled the weight scratch, when they belong to this step (the slot and the
+    // scratch may have been filled by different reads when layers are reused)
+    for (int g = 0; g < NCHUNK; ++g) {
+      c->cur_wait[g][0] = streamed && p.loaded_by >= 0 ? c->ev_chunk[p.loaded_by * NCHUNK + g] : nullptr;
+      c->cur_wait[g][1] = nf4 && p.wfilled_by >= 0 ? c->ev_deqg[p.wfilled_by * NCHUNK + g] : nullptr;
     }
+    const __nv_bfloat16* W =
+        nf4 ? c->wscr[p.wslot] : reinterpret_cast<const __nv_bfloat16*>(blob + c->lay.w16);
     if (kind == RD_REF) {
       c->adapters_off = true;
       const lst_status st = layer_fwd(c, j, blob, W, false);
@@ -1215,14 +1259,12 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   } else {
     TRY(dalloc(c, &c->gbuf, T * d));
   }
-  c->ev_loaded.resize(3 * c->L);  // up to 3L reads per step (DPO)
-  c->ev_free.resize(3 * c->L);
-  c->ev_deq.resize(3 * c->L);
-  for (int i = 0; i < 3 * c->L; ++i) {
-    CK(cudaEventCreateWithFlags(&c->ev_loaded[i], cudaEventDisableTiming));
-    CK(cudaEventCreateWithFlags(&c->ev_free[i], cudaEventDisableTiming));
-    CK(cudaEventCreateWithFlags(&c->ev_deq[i], cudaEventDisableTiming));
-  }
+  c->ev_free.resize(3 * c->L);  // up to 3L reads per step (DPO)
+  c->ev_chunk.resize(3 * c->L * NCHUNK);
+  c->ev_deqg.resize(3 * c->L * NCHUNK);
+  for (auto& e : c->ev_free) CK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+  for (auto& e : c->ev_chunk) CK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+  for (auto& e : c->ev_deqg) CK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
   CK(cudaEventCreateWithFlags(&c->ev_done, cudaEventDisableTiming));
   CK(cudaEventCreateWithFlags(&c->ev_start, cudaEventDisableTiming));
   CK(cudaEventCreate(&c->prof_step0));
@@ -1244,9 +1286,9 @@ void free_all(lst_ctx* c) {
   if (c->stage_gsum) cudaFree(c->stage_gsum);
   if (c->arena) cudaFreeHost(c->arena);
   if (c->host_loss) cudaFreeHost(c->host_loss);
-  for (auto e : c->ev_loaded) cudaEventDestroy(e);
+  for (auto e : c->ev_chunk) cudaEventDestroy(e);
   for (auto e : c->ev_free) cudaEventDestroy(e);
-  for (auto e : c->ev_deq) cudaEventDestroy(e);
+  for (auto e : c->ev_deqg) cudaEventDestroy(e);
   for (auto e : c->prof_pool) cudaEventDestroy(e);
   if (c->ev_done) cudaEventDestroy(c->ev_done);
   if (c->ev_start) cudaEventDestroy(c->ev_start);

@@ -142,7 +142,7 @@ __device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const
 // Tile order: groups of kGroupM M-tiles; inside a group the M-tile index runs fastest, so the
 // CTAs working at the same time share a few weight (B) tiles and the group's activation rows in
 // L2.
-constexpr int kGroupM = 8;
+constexpr int kGroupM = 16;
 
 struct TileSched {
   int mt, nt;
