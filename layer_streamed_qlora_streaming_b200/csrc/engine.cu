@@ -165,6 +165,15 @@ Layout make_layout(const lst_config& c) {
   return L;
 }
 
+bool is_pinned_host_ptr(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
 bool is_device_ptr(const void* p) {
   cudaPointerAttributes a;
   if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
@@ -199,6 +208,9 @@ struct lst_ctx {
   int dev = 0;
   cudaStream_t stream = nullptr, copy_stream = nullptr;
   cudaStream_t prep_stream = nullptr;  // dequant of the next read, below the compute stream's priority
+  cudaStream_t d2h_stream = nullptr;   // gradients to pinned host memory, layer by layer
+  float* grads_host = nullptr;         // pinned host destination of this step's gradients (or null)
+  cudaEvent_t ev_d2h = nullptr;
   bool own_stream = false;
   std::string err;
   Faults faults;
@@ -916,6 +928,7 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
   CK(cudaEventRecord(c->ev_start, c->stream));
   CK(cudaStreamWaitEvent(c->copy_stream, c->ev_start, 0));
   CK(cudaStreamWaitEvent(c->prep_stream, c->ev_start, 0));
+  CK(cudaStreamWaitEvent(c->d2h_stream, c->ev_start, 0));
   int next_copy = 0;
   if (streamed) TRY(issue_copies(c, -1, next_copy));
   // dequant of read m on the prep stream, chunk by chunk as the copy lands; every event it waits on
@@ -959,6 +972,12 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
       TRY(layer_bwd(c, j, blob, W));
     }
     CK(cudaEventRecord(c->ev_free[n], c->stream));
+    if (kind == RD_BWD && c->grads_host) {
+      // this layer's gradients are final: send them while the layers below compute
+      const int64_t o0 = c->offA[j * NPROJ], o1 = j + 1 < L ? c->offA[(j + 1) * NPROJ] : c->lora_numel;
+      CK(cudaStreamWaitEvent(c->d2h_stream, c->ev_free[n], 0));
+      CK(cudaMemcpyAsync(c->grads_host + o0, c->grads + o0, (o1 - o0) * 4, cudaMemcpyDeviceToHost, c->d2h_stream));
+    }
     if (kind != RD_BWD && (n + 1 == R || c->rd_kind[n + 1] != kind)) TRY(head_after(c, kind, mode));
     if (streamed) TRY(issue_copies(c, n, next_copy));
   }
@@ -967,7 +986,11 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
 }
 
 lst_status finish_step(lst_ctx* c, float* loss, float* grads_out) {
-  if (grads_out) {
+  if (c->grads_host) {
+    // sent layer by layer during the backward (run_layers); the step ends when they have arrived
+    CK(cudaEventRecord(c->ev_d2h, c->d2h_stream));
+    CK(cudaStreamWaitEvent(c->stream, c->ev_d2h, 0));
+  } else if (grads_out) {
     const bool dev = is_device_ptr(grads_out);
     CK(cudaMemcpyAsync(grads_out, c->grads, c->lora_numel * 4, dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
                        c->stream));
@@ -1032,6 +1055,10 @@ lst_status finish_step(lst_ctx* c, float* loss, float* grads_out) {
   }
   return LST_OK;
 }
+
+// Pinned host gradient buffers are filled layer by layer during the backward; any other
+// destination gets one copy at the end of the step.
+void set_grads_dest(lst_ctx* c, float* grads) { c->grads_host = grads && is_pinned_host_ptr(grads) ? grads : nullptr; }
 
 lst_status begin_step(lst_ctx* c, int32_t batch, int32_t seq) {
   for (int i = 0; i < c->L; ++i)
@@ -1128,6 +1155,7 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   CK(cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking));
   // lowest priority: the next read's dequant takes the SM slots the compute stream leaves free
   CK(cudaStreamCreateWithPriority(&c->prep_stream, cudaStreamNonBlocking, prio_low));
+  CK(cudaStreamCreateWithFlags(&c->d2h_stream, cudaStreamNonBlocking));
 
   // LoRA parameter / gradient layout
   c->offA.resize(c->L * NPROJ);
@@ -1267,6 +1295,7 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   for (auto& e : c->ev_deqg) CK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
   CK(cudaEventCreateWithFlags(&c->ev_done, cudaEventDisableTiming));
   CK(cudaEventCreateWithFlags(&c->ev_start, cudaEventDisableTiming));
+  CK(cudaEventCreateWithFlags(&c->ev_d2h, cudaEventDisableTiming));
   CK(cudaEventCreate(&c->prof_step0));
   CK(cudaEventCreate(&c->prof_step1));
   CK(cudaStreamSynchronize(c->stream));
@@ -1278,6 +1307,7 @@ void free_all(lst_ctx* c) {
   if (c->stream) cudaStreamSynchronize(c->stream);
   if (c->copy_stream) cudaStreamSynchronize(c->copy_stream);
   if (c->prep_stream) cudaStreamSynchronize(c->prep_stream);
+  if (c->d2h_stream) cudaStreamSynchronize(c->d2h_stream);
   for (void* p : c->dev_allocs) cudaFree(p);
   c->dev_allocs.clear();
   if (c->stage_w) cudaFree(c->stage_w);
@@ -1292,10 +1322,12 @@ void free_all(lst_ctx* c) {
   for (auto e : c->prof_pool) cudaEventDestroy(e);
   if (c->ev_done) cudaEventDestroy(c->ev_done);
   if (c->ev_start) cudaEventDestroy(c->ev_start);
+  if (c->ev_d2h) cudaEventDestroy(c->ev_d2h);
   if (c->prof_step0) cudaEventDestroy(c->prof_step0);
   if (c->prof_step1) cudaEventDestroy(c->prof_step1);
   if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
   if (c->prep_stream) cudaStreamDestroy(c->prep_stream);
+  if (c->d2h_stream) cudaStreamDestroy(c->d2h_stream);
   if (c->own_stream && c->stream) cudaStreamDestroy(c->stream);
   cudaGetLastError();
 }
@@ -1462,6 +1494,7 @@ lst_status lst_step(lst_ctx* c, const int32_t* tokens, const int32_t* targets, i
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(embed(c->tok, c->E, c->curT, c->d, c->V, c->xs, c->stream));
   }
+  set_grads_dest(c, grads);
   TRY(run_layers(c, HEAD_SFT));
   TRY(optimizer_update(c));
   c->have_logits = true;
@@ -1477,6 +1510,7 @@ lst_status lst_step_hidden(lst_ctx* c, const uint16_t* x, const uint16_t* g, int
   TRY(copy_in(c, c->dout_b, x, c->curT * c->d * 2));  // bf16 input staged, widened to fp32
   CK(bf16_to_f32(c->dout_b, c->curT * c->d, c->xs, c->stream));
   TRY(copy_in(c, c->gbuf, g, c->curT * c->d * 2));
+  set_grads_dest(c, grads);
   TRY(run_layers(c, HEAD_HIDDEN));
   TRY(optimizer_update(c));
   c->have_logits = false;
@@ -1500,6 +1534,7 @@ lst_status lst_step_dpo(lst_ctx* c, const int32_t* tokens, const int32_t* target
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(embed(c->tok, c->E, c->curT, c->d, c->V, c->xs, c->stream));
   }
+  set_grads_dest(c, grads);
   TRY(run_layers(c, HEAD_DPO));
   TRY(optimizer_update(c));
   c->have_logits = false;

@@ -148,6 +148,22 @@ def test_head_in_passes_same_bytes(chunk):
     ctx.close()
 
 
+def test_gradients_to_pinned_host_same_bytes():
+    # a pinned host destination is filled layer by layer during the backward; same bytes as the
+    # device and pageable-host destinations
+    wl = WORKLOADS["qwen3b_bf16_2L"]
+    inp = build_inputs(wl)
+    ctx = make_context(wl, inp, streamed=True)
+    n = ctx.lora_numel()
+    gd = torch.full((n,), float("nan"), device="cuda")
+    gp = torch.full((n,), float("nan")).pin_memory()
+    gh = np.full(n, np.nan, dtype=np.float32)
+    losses = [ctx.step(inp["tokens"], inp["targets"], wl.batch, wl.seq, g) for g in (gd, gp, gh)]
+    assert losses[0] == losses[1] == losses[2]
+    assert gd.cpu().numpy().tobytes() == gp.numpy().tobytes() == gh.tobytes()
+    ctx.close()
+
+
 def test_errors_are_status_codes():
     import layer_streamed_qlora_streaming_b200 as lst
     wl = syn.WORKLOADS["tiny"]
