@@ -48,10 +48,11 @@ def describe(wl) -> str:
 
 # DRAM traffic (read + write) of the GEMM launches of one llama8b step, from one ncu capture of the
 # bench (dram__bytes_read.sum + dram__bytes_write.sum over the step's 354 k_gemm launches; command
-# and figures in profiles/gemm_traffic_llama8b_step.md). Valid only for the GEMM sources measured.
+# and figures in profiles/gemm_traffic_llama8b_step.md). Valid only for the GEMM sources measured
+# (hashes taken after a host-side change to the launcher's per-device set-up; kernel unchanged).
 GEMM_TRAFFIC = {"workload": "llama8b", "bytes_per_step": 73.988e9, "launches": 354,
-                "sources": {"gemm.cu": "e42c3dc7664d7c3c", "gemm.cuh": "4a668b6d34dc410f",
-                            "common.cuh": "c89033b9dea61163"}}
+                "sources": {"gemm.cu": "e0a88be30295bc55", "gemm.cuh": "4a668b6d34dc410f",
+                            "common.cuh": "da32f91f59c8b4d8"}}
 
 
 def gemm_traffic(wl_name: str):

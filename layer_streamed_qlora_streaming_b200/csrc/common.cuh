@@ -4,6 +4,7 @@
 // g_lst_dev_error and gives up, so a lost arrival ends the kernel instead of hanging the GPU.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -13,6 +14,13 @@ namespace lst {
 
 // Count of kernel launches made by the library (host side); every launcher adds its launches.
 void note_launch(int n);
+
+// Host helpers for per-device set-up that launchers cache (a process may drive several GPUs):
+// the current device's SM count, and per-device done flags for up to 64 devices (a device beyond
+// that is never marked done, so its set-up simply runs on every use).
+int device_sm_count();
+bool done_on_device(const std::atomic<unsigned long long>& mask);
+void mark_done_on_device(std::atomic<unsigned long long>& mask);
 
 // Error word written by device code (bounded waits that ran out, bad indices); read by the host.
 extern __device__ int g_lst_dev_error;

@@ -1418,6 +1418,31 @@ lst_status register_impl(lst_ctx* c, int layer, const lst_layer_weights* w) {
 
 namespace lst {
 void note_launch(int n) { g_launch_count.fetch_add(n, std::memory_order_relaxed); }
+
+int device_sm_count() {
+  static std::atomic<int> cached[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cached[dev].load() > 0) return cached[dev].load();
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 148;
+  }
+  if (dev >= 0 && dev < 64) cached[dev].store(n);
+  return n;
+}
+
+static unsigned long long device_bit() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev >= 0 && dev < 64 ? 1ull << dev : 0ull;
+}
+bool done_on_device(const std::atomic<unsigned long long>& mask) {
+  const unsigned long long bit = device_bit();
+  return bit && (mask.load() & bit);
+}
+void mark_done_on_device(std::atomic<unsigned long long>& mask) { mask.fetch_or(device_bit()); }
 }  // namespace lst
 
 // =========================================================================== C ABI

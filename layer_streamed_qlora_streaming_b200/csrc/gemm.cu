@@ -390,25 +390,18 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   }
   Epi e{a.C, a.ldc, a.bias, a.R, a.ldr, a.alpha, a.c_f32, a.M, a.N,
         a.rope_cos, a.rope_sin, a.rope_cos ? a.rope_end : 0, a.rope_hd, a.rope_S};
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t err =
-        cudaFuncSetAttribute(k_gemm<BN, AMN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  static std::atomic<unsigned long long> attr_done{0};  // devices whose function attribute is set
+  if (!done_on_device(attr_done)) {
+    const cudaError_t err = cudaFuncSetAttribute(k_gemm<BN, AMN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (err != cudaSuccess) return err;
-    attr_set = true;
+    mark_done_on_device(attr_done);
   }
   const int nk1 = (a.K + BK - 1) / BK;
   TileSched sched;
   sched.mt = (a.M + BM - 1) / BM;
   sched.nt = (a.N + BN - 1) / BN;
   const int total = sched.mt * sched.nt;
-  static int num_sms = 0;
-  if (!num_sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || num_sms <= 0)
-      num_sms = 148;
-  }
+  const int num_sms = device_sm_count();
   const int grid = total < num_sms ? total : num_sms;
   k_gemm<BN, AMN, BMN><<<grid, 192, C::SMEM, s>>>(tA, tB, tA2, tB2, e, sched, total, nk1, nk2);
   note_launch(1);

@@ -221,29 +221,19 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   }
 }
 
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  }
-  return n;
-}
-
 template <int AMN, int BMN>
 cudaError_t launch_side(const CUtensorMap& tA, const CUtensorMap& tB, int M, int N, int K, const SideOut& o,
                         cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(k_side<AMN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
+  static std::atomic<unsigned long long> attr_done{0};  // devices whose function attribute is set
+  if (!done_on_device(attr_done)) {
+    const cudaError_t err = cudaFuncSetAttribute(k_side<AMN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (err != cudaSuccess) return err;
+    mark_done_on_device(attr_done);
   }
   const int mt = (M + kBM - 1) / kBM, nt = (N + kBN - 1) / kBN, nk = (K + kBK - 1) / kBK;
   if (mt > 65535 || nt > 65535) return cudaErrorInvalidValue;
   // widest cluster (K split) that keeps every CTA resident at two per SM
-  const int64_t slots = 2 * (int64_t)sm_count();
+  const int64_t slots = 2 * (int64_t)device_sm_count();
   int cs = 1;
   while (cs < kMaxCluster && (int64_t)mt * nt * cs * 2 <= slots && cs * 2 <= nk) cs *= 2;
   const int kps = (nk + cs - 1) / cs;
