@@ -26,6 +26,8 @@
 #include "optim.cuh"
 
 #include <atomic>
+#include <cstdio>
+#include <nvtx3/nvToolsExt.h>
 #include <chrono>
 #include <cmath>
 #include <cstdlib>
@@ -165,6 +167,9 @@ Layout make_layout(const lst_config& c) {
   return L;
 }
 
+constexpr int64_t kGuardBytes = 4096;
+constexpr uint8_t kGuardByte = 0xA5;
+
 bool is_pinned_host_ptr(const void* p) {
   cudaPointerAttributes a;
   if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
@@ -189,6 +194,17 @@ enum { PC_GEMM = 0, PC_ATTN = 1, PC_DEQ = 2, PC_OTHER = 3, PC_COPY = 4, PC_LORA 
 }  // namespace
 
 enum ReadKind { RD_REF = 0, RD_FWD = 1, RD_BWD = 2 };
+
+// NVTX range on the host thread for the scope (shows the enqueue of each read and copy in a
+// timeline tool; costs nothing when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* fmt, int a, int b) {
+    char name[64];
+    std::snprintf(name, sizeof(name), fmt, a, b);
+    nvtxRangePushA(name);
+  }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 enum HeadMode { HEAD_SFT = 0, HEAD_HIDDEN = 1, HEAD_DPO = 2 };
 
 struct ReadPlan {
@@ -209,6 +225,13 @@ struct lst_ctx {
   cudaStream_t stream = nullptr, copy_stream = nullptr;
   cudaStream_t prep_stream = nullptr;  // dequant of the next read, below the compute stream's priority
   cudaStream_t d2h_stream = nullptr;   // gradients to pinned host memory, layer by layer
+  // guard bytes after the pool slots and weight scratches, checked after each step when the
+  // environment sets LST_CANARY=1 (a kernel or copy writing past one of them is reported)
+  std::vector<uint8_t*> guards;
+  bool check_guards = [] {
+    const char* e = std::getenv("LST_CANARY");
+    return e && e[0] && std::strcmp(e, "0") != 0;
+  }();
   float* grads_host = nullptr;         // pinned host destination of this step's gradients (or null)
   cudaEvent_t ev_d2h = nullptr;
   bool own_stream = false;
@@ -348,6 +371,24 @@ lst_status dalloc(lst_ctx* c, T** p, int64_t n, bool zero = false) {
   *p = static_cast<T*>(q);
   return LST_OK;
 }
+
+lst_status add_guard(lst_ctx* c, uint8_t* p) {
+  CK(cudaMemset(p, kGuardByte, kGuardBytes));
+  c->guards.push_back(p);
+  return LST_OK;
+}
+
+lst_status check_guards(lst_ctx* c) {
+  std::vector<uint8_t> h(kGuardBytes);
+  for (size_t i = 0; i < c->guards.size(); ++i) {
+    CK(cudaMemcpy(h.data(), c->guards[i], kGuardBytes, cudaMemcpyDeviceToHost));
+    for (int64_t k = 0; k < kGuardBytes; ++k)
+      if (h[k] != kGuardByte)
+        return fail(c, LST_ERR_DEVICE, "guard bytes after device buffer " + std::to_string(i) + " were overwritten");
+  }
+  return LST_OK;
+}
+
 
 #define TRY(x)                        \
   do {                                \
@@ -848,6 +889,7 @@ void plan_reads(lst_ctx* c) {
 
 lst_status enqueue_copy(lst_ctx* c, int n) {
   const int j = c->rd_layer[n];
+  NvtxRange nr("copy read %d (layer %d)", n, j);
   const ReadPlan& p = c->plan[n];
   if (c->faults.fail_memcpy()) return fail(c, LST_ERR_CUDA, "layer copy enqueue failed (injected)");
   if (p.wait_free >= 0) CK(cudaStreamWaitEvent(c->copy_stream, c->ev_free[p.wait_free], 0));
@@ -946,9 +988,12 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
     return LST_OK;
   };
   TRY(enqueue_deq(0));
+  static const char* kRangeName[3] = {"reference forward read %d (layer %d)", "forward read %d (layer %d)",
+                                       "backward read %d (layer %d)"};
   for (int n = 0; n < R; ++n) {
     const int j = c->rd_layer[n], kind = c->rd_kind[n];
     const ReadPlan& p = c->plan[n];
+    NvtxRange nr(kRangeName[kind], n, j);
     TRY(enqueue_deq(n + 1));
     const uint8_t* blob = blob_of(n);
     // the compute of chunk g waits for the copy that filled the slot and, for an NF4 base, the
@@ -1018,6 +1063,7 @@ lst_status finish_step(lst_ctx* c, float* loss, float* grads_out) {
     return fail(c, LST_ERR_DEVICE, "device code reported error " + std::to_string(derr));
   }
   *loss = *c->host_loss;
+  if (c->check_guards) TRY(check_guards(c));
   if (c->cfg.streamed) {
     c->slot_layer[0] = c->plan_held[0];
     c->slot_layer[1] = c->plan_held[1];
@@ -1210,8 +1256,10 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
     cudaError_t e = cudaHostAlloc(&a, (size_t)blob * c->L, cudaHostAllocDefault);
     if (e != cudaSuccess) return cuda_fail(c, e, "cudaHostAlloc(arena)");
     c->arena = static_cast<uint8_t*>(a);
-    TRY(dalloc(c, &c->pool[0], blob));
-    TRY(dalloc(c, &c->pool[1], blob));
+    TRY(dalloc(c, &c->pool[0], blob + kGuardBytes));
+    TRY(dalloc(c, &c->pool[1], blob + kGuardBytes));
+    TRY(add_guard(c, c->pool[0] + blob));
+    TRY(add_guard(c, c->pool[1] + blob));
     c->st.arena_bytes = blob * c->L;
   } else {
     TRY(dalloc(c, &c->resident, blob * c->L));
@@ -1220,8 +1268,10 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   c->st.blob_bytes = blob;
   c->registered.assign(c->L, 0);
   if (k.base_format == LST_BASE_NF4) {
-    TRY(dalloc(c, &c->wscr[0], c->lay.P));
-    TRY(dalloc(c, &c->wscr[1], c->lay.P));
+    TRY(dalloc(c, &c->wscr[0], c->lay.P + kGuardBytes / 2));
+    TRY(dalloc(c, &c->wscr[1], c->lay.P + kGuardBytes / 2));
+    TRY(add_guard(c, reinterpret_cast<uint8_t*>(c->wscr[0] + c->lay.P)));
+    TRY(add_guard(c, reinterpret_cast<uint8_t*>(c->wscr[1] + c->lay.P)));
   }
 
   // activations

@@ -164,6 +164,19 @@ def test_gradients_to_pinned_host_same_bytes():
     ctx.close()
 
 
+def test_guard_bytes_checked_after_steps(monkeypatch):
+    # LST_CANARY=1: the guard bytes after the pool slots and weight scratches are checked after each
+    # step (a write past the end of one of them would turn the step into LST_ERR_DEVICE)
+    monkeypatch.setenv("LST_CANARY", "1")
+    wl = syn.WORKLOADS["tiny"]
+    inp = build_inputs(wl)
+    for reuse in (False, True):
+        ctx = make_context(wl, inp, streamed=True, reuse=reuse)
+        for _ in range(2):
+            assert np.isfinite(run_step(ctx, wl, inp, want_logits=False)[0])
+        ctx.close()
+
+
 def test_errors_are_status_codes():
     import layer_streamed_qlora_streaming_b200 as lst
     wl = syn.WORKLOADS["tiny"]
