@@ -449,8 +449,9 @@ def run_gpu(args, wl):
                "min_ms": dbytes / (link_gbs * 1e9) * 1e3, "frac": dbytes / (link_gbs * 1e9) * 1e3 / (dms / args.steps),
                "pairs": P, "beta": 0.1, "loss_first": dloss_first, "loss_last": dloss,
                "note": "DPO: reference forward with the adapters off, then the policy forward, head and backward "
-                       "(3L reads); tokens/s counts the 2P sequences once; starts from the initial adapters "
-                       "(loss_first near ln 2); the same pairs every step, so the loss falls fast under AdamW"}
+                       "(3L reads); tokens/s counts the 2P sequences once; starts from the initial adapters, "
+                       "whose B != 0 already separates policy and reference; the same pairs every step, so "
+                       "the loss falls fast under AdamW"}
 
     st = ctx.stats()
     peaks = measured_peaks()
