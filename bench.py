@@ -250,9 +250,11 @@ def max_over_ranks(ms: float, dist, device) -> float:
 
 
 def allreduce_grads(grads, dist) -> None:
-    """Data-parallel exchange: sum the LoRA gradients of all replicas (NCCL on GPUs)."""
+    """Data-parallel exchange: average the LoRA gradients of all replicas (NCCL on GPUs), so every
+    replica applies the same update."""
     if dist is not None:
         dist.all_reduce(grads)
+        grads.div_(dist.get_world_size())
 
 
 def job_throughput(world: int, tokens_per_step: int, steps: int, ms: float) -> float:
@@ -302,7 +304,8 @@ def run_gpu(args, wl):
     link_gbs = h2d_peak_gbs(torch)
     ctx = build_context(wl, torch, stream, seed=1234 + rank)
     if not args.no_optimizer:
-        ctx.set_optimizer(lr=2e-4)   # the step includes the AdamW update of every adapter
+        # one process: the step applies AdamW itself; replicas: after the gradient average
+        ctx.set_optimizer(lr=2e-4, deferred=world > 1)
     n_grad = ctx.lora_numel()
     lora0 = torch.empty(n_grad, dtype=torch.float32, device="cuda")
     ctx.get_lora(lora0)              # initial adapters, restored before the DPO measurement
@@ -325,10 +328,17 @@ def run_gpu(args, wl):
         def step(gr):
             return ctx.step_hidden(x_d, g_d, wl.batch, wl.seq, gr)
 
-    def one_step():
-        loss = step(grads)
+    def exchange_and_update():
+        if dist is None:
+            return
         with torch.cuda.stream(stream):
             allreduce_grads(grads, dist)
+        if not args.no_optimizer:
+            ctx.apply_optimizer(grads)   # the replicas' mean gradient, on the context's stream
+
+    def one_step():
+        loss = step(grads)
+        exchange_and_update()
         return loss
 
     for _ in range(args.warmup):
@@ -422,12 +432,11 @@ def run_gpu(args, wl):
         for (l, pname), ((oa, sa), (ob, sb)) in ctx.grad_slices().items():
             ctx.set_lora(l, lst.PROJ.index(pname), lora0[oa:oa + sa[0] * sa[1]], lora0[ob:ob + sb[0] * sb[1]])
         if not args.no_optimizer:
-            ctx.set_optimizer(lr=2e-4)
+            ctx.set_optimizer(lr=2e-4, deferred=world > 1)
 
         def dpo_step():
             loss = ctx.step_dpo(dt, dy, dm, P, wl.seq, 0.1, grads)
-            with torch.cuda.stream(stream):
-                allreduce_grads(grads, dist)
+            exchange_and_update()
             return loss
         dloss_first = dpo_step()
         dpo_step()
@@ -469,7 +478,9 @@ def run_gpu(args, wl):
         "dtype": "bf16", "data": "synthetic (seeded torch.randn weights / uniform tokens)",
         "config": {"workload": describe(wl), "batch": wl.batch, "seq": wl.seq, "layers": wl.n_layers,
                    "parallelism": f"dp{world}" if world > 1 else "single GPU",
-                   "optimizer": "none" if args.no_optimizer else "AdamW lr 2e-4 on every adapter, inside the step",
+                   "optimizer": "none" if args.no_optimizer else (
+                       "AdamW lr 2e-4 on every adapter, inside the step" if world == 1 else
+                       "AdamW lr 2e-4 on every adapter with the replicas' mean gradient (NCCL all-reduce)"),
                    "l2": "not flushed: every step streams all layer blobs (GBs) through HBM, far above the 126 MB L2",
                    "loss_last": loss},
         "roofline": {"bound": "tensor", "kernel": "tcgen05 bf16 GEMM (all projection + LM-head GEMMs)",

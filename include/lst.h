@@ -145,10 +145,20 @@ typedef struct {
   float beta1, beta2;  /* moment decay rates, in [0, 1) */
   float eps;           /* > 0 */
   float weight_decay;  /* decoupled weight decay, >= 0 */
+  int32_t deferred;    /* 0: applied by every step with its own gradients; 1: applied only by
+                          lst_apply_optimizer, with the caller's gradients */
 } lst_adamw;
 
 /* Enable (cfg non-NULL: moments reset to zero, t reset) or disable (NULL) the update. */
 lst_status lst_set_optimizer(lst_ctx* ctx, const lst_adamw* cfg);
+
+/* One AdamW update of the adapters with the gradient g (lst_lora_numel fp32 values in the gradient
+ * layout, host or device), using the moments and step count of lst_set_optimizer. For data-parallel
+ * training: each replica's step leaves its gradients, the caller averages them over the replicas
+ * (e.g. an NCCL all-reduce on the context's stream) and applies the average here, so every replica
+ * takes the same update. Needs the optimizer set with deferred = 1 (else LST_ERR_STATE).
+ * Enqueued on the context's stream; returns when the update is done. */
+lst_status lst_apply_optimizer(lst_ctx* ctx, const float* g);
 
 /* Copy the current adapters (lst_lora_numel fp32 values, gradient layout) to dst (host or device). */
 lst_status lst_get_lora(lst_ctx* ctx, float* dst);

@@ -41,7 +41,7 @@ class LayerWeights(C.Structure):
 
 class AdamW(C.Structure):
     _fields_ = [("lr", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float), ("eps", C.c_float),
-                ("weight_decay", C.c_float)]
+                ("weight_decay", C.c_float), ("deferred", C.c_int32)]
 
 
 class Stats(C.Structure):
@@ -72,6 +72,7 @@ _SIGS = {
     "lst_get_logits": (_I32, [_P, _P]),
     "lst_get_activation": (_I32, [_P, _I32, _I32, _P]),
     "lst_set_profiling": (_I32, [_P, _I32]),
+    "lst_apply_optimizer": (_I32, [_P, _P]),
     "lst_step_dpo": (_I32, [_P, _P, _P, _P, _I32, _I32, _F32, C.POINTER(C.c_float), _P]),
     "lst_set_reuse": (_I32, [_P, _I32]),
     "lst_get_stats": (_I32, [_P, C.POINTER(Stats)]),
@@ -214,13 +215,19 @@ class Context:
     def lora_numel(self) -> int:
         return int(lib().lst_lora_numel(self.h))
 
-    def set_optimizer(self, lr=2e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, off=False):
-        """AdamW on the adapters at the end of every step (off=True disables it)."""
+    def set_optimizer(self, lr=2e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, off=False,
+                      deferred=False):
+        """AdamW on the adapters at the end of every step (off=True disables it); deferred=True
+        leaves the update to apply_optimizer (data-parallel: apply the replicas' mean gradient)."""
         if off:
             _check(lib().lst_set_optimizer(self.h, None), self.h, "lst_set_optimizer")
             return
-        cfg = AdamW(lr, beta1, beta2, eps, weight_decay)
+        cfg = AdamW(lr, beta1, beta2, eps, weight_decay, int(bool(deferred)))
         _check(lib().lst_set_optimizer(self.h, C.byref(cfg)), self.h, "lst_set_optimizer")
+
+    def apply_optimizer(self, grads) -> None:
+        """One AdamW update with the given gradient (host or device, gradient layout)."""
+        _check(lib().lst_apply_optimizer(self.h, _ptr(grads)), self.h, "lst_apply_optimizer")
 
     def get_lora(self, dst) -> None:
         _check(lib().lst_get_lora(self.h, _ptr(dst)), self.h, "lst_get_lora")

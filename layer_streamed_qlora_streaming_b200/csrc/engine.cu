@@ -1540,8 +1540,8 @@ lst_status lst_set_lora(lst_ctx* c, int32_t layer, int32_t proj, const float* a,
 
 int64_t lst_lora_numel(const lst_ctx* c) { return c ? c->lora_numel : 0; }
 
-static lst_status optimizer_update(lst_ctx* c) {
-  if (!c->opt_on) return LST_OK;
+// One AdamW update of every adapter with the gradient g (device), refreshing the bf16 operands.
+static lst_status adamw_apply(lst_ctx* c, const float* g) {
   c->opt_t += 1;
   const double t = (double)c->opt_t;
   AdamHyper h;
@@ -1553,8 +1553,14 @@ static lst_status optimizer_update(lst_ctx* c) {
   h.step_size = (float)(c->opt.lr / (1.0 - std::pow((double)c->opt.beta1, t)));
   h.sqrt_bc2 = (float)std::sqrt(1.0 - std::pow((double)c->opt.beta2, t));
   ProfScope ps(c, c->stream, PC_OTHER);
-  CK(adamw_update(c->opt_tab, c->opt_ntab, c->opt_maxn, c->lora, c->grads, c->opt_m, c->opt_v, h, c->stream));
+  CK(adamw_update(c->opt_tab, c->opt_ntab, c->opt_maxn, c->lora, g, c->opt_m, c->opt_v, h, c->stream));
   return LST_OK;
+}
+
+// The in-step update (optimizer on and not deferred) with the step's own gradients.
+static lst_status optimizer_update(lst_ctx* c) {
+  if (!c->opt_on || c->opt.deferred) return LST_OK;
+  return adamw_apply(c, c->grads);
 }
 
 lst_status lst_step(lst_ctx* c, const int32_t* tokens, const int32_t* targets, int32_t batch, int32_t seq,
@@ -1678,6 +1684,20 @@ lst_status lst_set_optimizer(lst_ctx* c, const lst_adamw* cfg) {
   c->opt = *cfg;
   c->opt_t = 0;
   c->opt_on = true;
+  return LST_OK;
+}
+
+lst_status lst_apply_optimizer(lst_ctx* c, const float* g) {
+  if (!c) return LST_ERR_ARG;
+  if (!g) return fail(c, LST_ERR_ARG, "null gradient");
+  if (!c->opt_on || !c->opt.deferred) return fail(c, LST_ERR_STATE, "set the optimizer with deferred = 1 first");
+  const float* src = g;
+  if (!is_device_ptr(g)) {  // host gradient: staged through the context's gradient buffer
+    TRY(copy_in(c, c->grads, g, c->lora_numel * 4));
+    src = c->grads;
+  }
+  TRY(adamw_apply(c, src));
+  CK(cudaStreamSynchronize(c->stream));
   return LST_OK;
 }
 

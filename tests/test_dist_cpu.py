@@ -1,5 +1,6 @@
-"""The multi-rank plumbing of bench.py on CPU: two gloo ranks, gradient all-reduce (the only
-exchange of data-parallel replicas), max-over-ranks timing and the whole-job throughput."""
+"""The multi-rank plumbing of bench.py on CPU: two gloo ranks, the gradient average (the only
+exchange of data-parallel replicas, applied by every replica's deferred AdamW update), max-over-ranks
+timing and the whole-job throughput."""
 import os
 import socket
 
@@ -45,6 +46,6 @@ def test_two_ranks_gloo():
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(world))
     for rank, g0, g1, ms, thr in res:
-        assert g0 == g1 == 3.0            # 1 + 2 summed on both ranks
+        assert g0 == g1 == 1.5            # mean of 1 and 2 on both ranks
         assert ms == 150.0                # the slowest rank
         assert abs(thr - 2 * 2048 * 10 / 0.150) < 1e-6

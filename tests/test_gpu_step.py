@@ -177,6 +177,32 @@ def test_guard_bytes_checked_after_steps(monkeypatch):
         ctx.close()
 
 
+def test_deferred_optimizer_matches_in_step_update():
+    # data-parallel form: the step leaves its gradients, apply_optimizer takes the (here: own)
+    # gradient; same adapters and losses as the update inside the step, step after step
+    wl = WORKLOADS["tiny"]
+    inp = build_inputs(wl)
+    runs = []
+    for mode in ("in_step", "deferred_device", "deferred_host"):
+        ctx = make_context(wl, inp, streamed=True)
+        ctx.set_optimizer(lr=1e-3, deferred=mode != "in_step")
+        n = ctx.lora_numel()
+        g = torch.zeros(n, device="cuda") if mode != "deferred_host" else torch.zeros(n).pin_memory()
+        losses = []
+        for _ in range(3):
+            losses.append(ctx.step(inp["tokens"], inp["targets"], wl.batch, wl.seq, g))
+            if mode != "in_step":
+                ctx.apply_optimizer(g)
+        p = torch.zeros(n, device="cuda")
+        ctx.get_lora(p)
+        runs.append((losses, p.cpu().numpy()))
+        ctx.close()
+    for losses, p in runs[1:]:
+        assert np.float32(losses).tobytes() == np.float32(runs[0][0]).tobytes()
+        assert p.tobytes() == runs[0][1].tobytes()
+    assert runs[0][0][2] < runs[0][0][0]
+
+
 def test_errors_are_status_codes():
     import layer_streamed_qlora_streaming_b200 as lst
     wl = syn.WORKLOADS["tiny"]
@@ -199,6 +225,9 @@ def test_errors_are_status_codes():
     assert e.value.status == 6
     loss = ctx.step(inp["tokens"], inp["targets"], wl.batch, wl.seq)   # context still usable
     assert np.isfinite(loss)
+    with pytest.raises(lst.LstError) as e:          # apply_optimizer without a deferred optimizer
+        ctx.apply_optimizer(np.zeros(ctx.lora_numel(), dtype=np.float32))
+    assert e.value.status == 2
     ctx.close()
 
 
