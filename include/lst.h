@@ -115,7 +115,12 @@ typedef struct {
 
 /* Create a context. embed [V, d], final_norm [d], lm_head [V, d] are fp32 (host or device; the
  * library rounds E and H to bf16 and keeps them resident); all three must be NULL iff vocab == 0.
- * cuda_stream: cudaStream_t the steps run on, or NULL for a stream owned by the context.
+ * cuda_stream: cudaStream_t the steps run on, or NULL for a stream owned by the context (created
+ * at the highest priority). The context adds a copy stream, a device-to-host stream and a prep
+ * stream at the lowest priority for the dequant of the next layer read, which then only takes SM
+ * slots the step stream leaves free: give a caller stream a priority above the lowest.
+ * Environment: LST_CANARY=1 checks guard bytes after the pool and scratch buffers after each step;
+ * LST_FAULT injects host-side failures (pinned_alloc:N, device_alloc:N, memcpy:N, timeout).
  * Errors: LST_ERR_ARG (bad config), LST_ERR_OOM, LST_ERR_CUDA. On error *out is NULL. */
 lst_status lst_create(const lst_config* cfg, const float* embed, const float* final_norm,
                       const float* lm_head, void* cuda_stream, lst_ctx** out);

@@ -1,20 +1,25 @@
 // Streaming engine and the C ABI of include/lst.h.
 //
-// The frozen base of every decoder layer is one contiguous blob. In streamed mode the blobs live in
-// one pinned host arena; each step makes 2L layer reads n = 0..2L-1 (layer n for n < L, layer
-// 2L-1-n after), copied with cudaMemcpyAsync on a dedicated copy stream into a two-buffer device
-// pool (read n uses buffer n % 2). Events fence the two streams: compute of read n waits for
-// "loaded[n]"; the copy of read n+2 into the same buffer waits for "free[n]", recorded when the
-// compute of read n is done with the buffer. So layer n+1 streams in while layer n computes
-// ("Soup: Fine-Tuning an 8B Model on a 4 GB Laptop GPU, One Layer at a Time", first paragraph:
-// double buffering; tutorial "Fine-tune Llama 3.1 8B on a 4GB GPU with Soup", section "What Soup
-// layer streaming changes": two-buffer pool, forward read plus backward-recomputation read;
-// "Soup CLI fine-tunes Llama-3.1-8B on a 4 GB laptop GPU", second paragraph: a dedicated CUDA
-// stream for the copies).
+// The frozen base of every decoder layer is one contiguous, group-major blob. In streamed mode the
+// blobs live in one pinned host arena; an SFT step makes 2L layer reads (layers 0..L-1 forward,
+// then L-1..0 backward with recompute), a DPO step 3L (a reference forward with the adapters off
+// first). Each read computes from one of two device pool slots, filled with cudaMemcpyAsync on a
+// dedicated copy stream in four chunks (q/k/v with the small tensors, o, gate/up, down), and for
+// an NF4 base from one of two bf16 weight scratches, filled chunk by chunk on a low-priority prep
+// stream one read ahead. Events fence the streams: the compute of a weight group waits for its
+// chunk's copy and dequant; a copy into a slot waits for "free" of the last read that computed from
+// it. So the next layer streams in while the current one computes ("Soup: Fine-Tuning an 8B Model
+// on a 4 GB Laptop GPU, One Layer at a Time", first paragraph: double buffering; tutorial
+// "Fine-tune Llama 3.1 8B on a 4GB GPU with Soup", section "What Soup layer streaming changes":
+// two-buffer pool, forward read plus backward-recomputation read; "Soup CLI fine-tunes
+// Llama-3.1-8B on a 4 GB laptop GPU", second paragraph: a dedicated CUDA stream for the copies).
+// plan_reads fixes, before a step, every read's slot and scratch and which copies and dequants run
+// (with `reuse`, a layer still held by a slot or scratch is not fetched again).
 //
 // The forward keeps only each layer's input; the backward reads the layer again, recomputes its
-// forward (keeping the intermediates) and runs its backward. Resident mode runs the same launches
-// on blobs that stay on the device, so both modes give the same bytes.
+// forward (keeping the intermediates) and runs its backward. A pinned host gradient buffer is
+// filled layer by layer on a device-to-host stream during the backward. Resident mode runs the same
+// launches on blobs that stay on the device, so every mode and schedule gives the same bytes.
 #include "../../include/lst.h"
 #include "../../include/lst_kernels.h"
 #include "attention.cuh"
