@@ -215,6 +215,18 @@ lst_status lst_get_activation(lst_ctx* ctx, int32_t which, int32_t layer, void* 
 /* Record per-class device times of every step (CUDA events around each launch) when on != 0. */
 lst_status lst_set_profiling(lst_ctx* ctx, int32_t on);
 
+/* The copy / dequant plan of one step, host only (no context, no GPU), for inspection and tests.
+ * reads: the layer of each read in order (an SFT step reads 0..L-1 then L-1..0; a DPO step reads
+ * 0..L-1 once more first); reuse / nf4: the config's reuse and base_format == LST_BASE_NF4;
+ * held[2] / wheld[2]: the layers the two pool slots / two bf16 weight scratches hold before the step
+ * (-1 = nothing), overwritten with what they hold after it. out: n_reads rows of 8 int32:
+ * slot, copy (0/1), wait_free (the read whose compute the copy waits for, -1 none), loaded_by
+ * (the read whose copy filled the slot, -1 an earlier step), wslot, dequant (0/1), wwait,
+ * wfilled_by (the same for the weight scratch; -1 / 0 for a bf16 base). LST_ERR_ARG on a null
+ * pointer, n_reads <= 0 or a negative layer. */
+lst_status lst_plan_reads(const int32_t* reads, int32_t n_reads, int32_t reuse, int32_t nf4,
+                          int32_t* held, int32_t* wheld, int32_t* out);
+
 /* Switch the copy schedule of the next steps (the config's `reuse`): 1 keeps layers that are still
  * in the pool instead of copying them again, 0 copies every read. Results are the same bytes. */
 lst_status lst_set_reuse(lst_ctx* ctx, int32_t reuse);

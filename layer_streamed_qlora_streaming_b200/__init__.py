@@ -75,6 +75,7 @@ _SIGS = {
     "lst_apply_optimizer": (_I32, [_P, _P]),
     "lst_step_dpo": (_I32, [_P, _P, _P, _P, _I32, _I32, _F32, C.POINTER(C.c_float), _P]),
     "lst_set_reuse": (_I32, [_P, _I32]),
+    "lst_plan_reads": (_I32, [_P, _I32, _I32, _I32, _P, _P, _P]),
     "lst_get_stats": (_I32, [_P, C.POINTER(Stats)]),
     "lst_last_error": (C.c_char_p, [_P]),
     "lst_destroy": (None, [_P]),
@@ -171,6 +172,19 @@ def make_config(wl, streamed: bool = True, max_batch=None, max_seq=None, timeout
                   BASE_NF4 if wl.base_format == "nf4" else BASE_BF16,
                   max_batch or wl.batch, max_seq or wl.seq, int(streamed), timeout_ms, int(head_chunk),
                   int(bool(reuse)))
+
+
+def plan_reads(reads, reuse: bool, nf4: bool, held=(-1, -1), wheld=(-1, -1)):
+    """The step's copy / dequant plan (host only): (rows [n, 8] int32 of slot, copy, wait_free,
+    loaded_by, wslot, dequant, wwait, wfilled_by; held after; wheld after)."""
+    import numpy as np
+    r = np.ascontiguousarray(reads, dtype=np.int32)
+    h = np.array(held, dtype=np.int32)
+    w = np.array(wheld, dtype=np.int32)
+    out = np.zeros((len(r), 8), dtype=np.int32)
+    _check(lib().lst_plan_reads(_ptr(r), len(r), int(bool(reuse)), int(bool(nf4)), _ptr(h), _ptr(w), _ptr(out)),
+           what="lst_plan_reads")
+    return out, tuple(int(x) for x in h), tuple(int(x) for x in w)
 
 
 def blob_bytes(cfg: Config) -> int:

@@ -832,24 +832,24 @@ lst_status head_dpo(lst_ctx* c) {
 // An NF4 base is dequantised into one of two bf16 weight scratches by the same rule (a read reuses
 // a scratch that still holds its layer only with reuse on), on the prep stream, one read ahead: the
 // dequant of read n+1 overlaps the compute of read n.
-void plan_reads(lst_ctx* c) {
-  const int R = (int)c->rd_layer.size();
-  const bool reuse = c->cfg.reuse != 0;
-  auto layer_of = [c](int n) { return c->rd_layer[n]; };
-  int held[2] = {reuse ? c->slot_layer[0] : -1, reuse ? c->slot_layer[1] : -1};
+// The planning itself, on host data only: layers[n] is the layer of read n; held / wheld are the
+// layers the two slots / weight scratches hold before the step (-1: nothing known) and are updated
+// to what they hold after it.
+void plan_schedule(const std::vector<int>& layers, bool reuse, bool nf4, int held[2], int wheld[2],
+                   std::vector<ReadPlan>& plan) {
+  const int R = (int)layers.size();
+  if (!reuse) held[0] = held[1] = wheld[0] = wheld[1] = -1;
   int last_use[2] = {-1, -1}, loaded_by[2] = {-1, -1};
-  int wheld[2] = {reuse ? c->w_layer[0] : -1, reuse ? c->w_layer[1] : -1};
   int wlast[2] = {-1, -1}, wfill[2] = {-1, -1};
-  const bool nf4 = c->cfg.base_format != LST_BASE_BF16;
   auto first_need = [&](int layer) {
     for (int m = 0; m < R; ++m)
-      if (layer_of(m) == layer) return m;
+      if (layers[m] == layer) return m;
     return R;
   };
-  c->plan.assign(R, ReadPlan{});
+  plan.assign(R, ReadPlan{});
   for (int n = 0; n < R; ++n) {
-    const int j = layer_of(n);
-    ReadPlan& p = c->plan[n];
+    const int j = layers[n];
+    ReadPlan& p = plan[n];
     p.slot = -1;
     if (reuse) {
       if (held[0] == j) p.slot = 0;
@@ -858,7 +858,7 @@ void plan_reads(lst_ctx* c) {
     p.copy = p.slot < 0;
     if (p.copy) {
       if (n > 0) {
-        p.slot = 1 - c->plan[n - 1].slot;
+        p.slot = 1 - plan[n - 1].slot;
       } else {
         p.slot = first_need(held[1]) > first_need(held[0]) ? 1 : 0;
       }
@@ -878,7 +878,7 @@ void plan_reads(lst_ctx* c) {
     }
     if (p.wslot < 0) {
       p.deq = true;
-      p.wslot = n > 0 ? 1 - c->plan[n - 1].wslot : (first_need(wheld[1]) > first_need(wheld[0]) ? 1 : 0);
+      p.wslot = n > 0 ? 1 - plan[n - 1].wslot : (first_need(wheld[1]) > first_need(wheld[0]) ? 1 : 0);
       p.wwait = wlast[p.wslot];
       wheld[p.wslot] = j;
       wfill[p.wslot] = n;
@@ -886,6 +886,13 @@ void plan_reads(lst_ctx* c) {
     p.wfilled_by = wfill[p.wslot];
     wlast[p.wslot] = n;
   }
+}
+
+void plan_reads(lst_ctx* c) {
+  const bool reuse = c->cfg.reuse != 0;
+  int held[2] = {c->slot_layer[0], c->slot_layer[1]};
+  int wheld[2] = {c->w_layer[0], c->w_layer[1]};
+  plan_schedule(c->rd_layer, reuse, c->cfg.base_format != LST_BASE_BF16, held, wheld, c->plan);
   c->plan_held[0] = held[0];
   c->plan_held[1] = held[1];
   c->plan_wheld[0] = wheld[0];
@@ -1719,6 +1726,28 @@ lst_status lst_get_lora(lst_ctx* c, float* dst) {
 lst_status lst_set_profiling(lst_ctx* c, int32_t on) {
   if (!c) return LST_ERR_ARG;
   c->profiling = on != 0;
+  return LST_OK;
+}
+
+lst_status lst_plan_reads(const int32_t* reads, int32_t n_reads, int32_t reuse, int32_t nf4, int32_t* held,
+                          int32_t* wheld, int32_t* out) {
+  if (!reads || n_reads <= 0 || !held || !wheld || !out) return LST_ERR_ARG;
+  std::vector<int> layers(reads, reads + n_reads);
+  for (int v : layers)
+    if (v < 0) return LST_ERR_ARG;
+  int h[2] = {held[0], held[1]}, w[2] = {wheld[0], wheld[1]};
+  std::vector<ReadPlan> plan;
+  plan_schedule(layers, reuse != 0, nf4 != 0, h, w, plan);
+  for (int n = 0; n < n_reads; ++n) {
+    const ReadPlan& p = plan[n];
+    const int32_t row[8] = {p.slot, p.copy ? 1 : 0, p.wait_free, p.loaded_by,
+                            nf4 ? p.wslot : -1, p.deq ? 1 : 0, p.wwait, p.wfilled_by};
+    std::memcpy(out + 8 * (int64_t)n, row, sizeof(row));
+  }
+  held[0] = h[0];
+  held[1] = h[1];
+  wheld[0] = w[0];
+  wheld[1] = w[1];
   return LST_OK;
 }
 
