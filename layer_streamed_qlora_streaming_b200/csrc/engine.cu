@@ -1038,7 +1038,6 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
     if (kind != RD_BWD && (n + 1 == R || c->rd_kind[n + 1] != kind)) TRY(head_after(c, kind, mode));
     if (streamed) TRY(issue_copies(c, n, next_copy));
   }
-  (void)L;
   return LST_OK;
 }
 
