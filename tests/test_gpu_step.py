@@ -203,6 +203,35 @@ def test_deferred_optimizer_matches_in_step_update():
     assert runs[0][0][2] < runs[0][0][0]
 
 
+@pytest.mark.parametrize("fault,status", [("pinned_alloc:1", 3), ("device_alloc:5", 3), ("memcpy:2", 4),
+                                          ("timeout", 5)])
+def test_injected_host_faults_are_status_codes(monkeypatch, fault, status):
+    # failures made on the host (LST_FAULT): a failed pinned or device allocation at create time,
+    # a failed layer-copy enqueue in a step, a step whose wait runs out; no GPU fault involved
+    import layer_streamed_qlora_streaming_b200 as lst
+    wl = syn.WORKLOADS["tiny"]
+    inp = build_inputs(wl)
+    monkeypatch.setenv("LST_FAULT", fault)
+    if "alloc" in fault:
+        with pytest.raises(lst.LstError) as e:
+            make_context(wl, inp, streamed=True)
+        assert e.value.status == status
+        return
+    ctx = make_context(wl, inp, streamed=True)
+    with pytest.raises(lst.LstError) as e:
+        run_step(ctx, wl, inp, want_logits=False)
+    assert e.value.status == status
+    if fault.startswith("memcpy"):
+        # the copy counter has moved past the failing one: the next step runs, with the clean result
+        loss, g, _ = run_step(ctx, wl, inp, want_logits=False)
+        monkeypatch.delenv("LST_FAULT")
+        clean = make_context(wl, inp, streamed=True)
+        loss_c, g_c, _ = run_step(clean, wl, inp, want_logits=False)
+        clean.close()
+        assert np.float32(loss).tobytes() == np.float32(loss_c).tobytes() and g.tobytes() == g_c.tobytes()
+    ctx.close()
+
+
 def test_errors_are_status_codes():
     import layer_streamed_qlora_streaming_b200 as lst
     wl = syn.WORKLOADS["tiny"]
