@@ -119,6 +119,8 @@ typedef struct {
  * at the highest priority). The context adds a copy stream, a device-to-host stream and a prep
  * stream at the lowest priority for the dequant of the next layer read, which then only takes SM
  * slots the step stream leaves free: give a caller stream a priority above the lowest.
+ * The context belongs to the device current at this call; every later call on it runs there and
+ * restores the caller's current device (one thread may drive contexts on several GPUs).
  * Environment: LST_CANARY=1 checks guard bytes after the pool and scratch buffers after each step;
  * LST_FAULT injects host-side failures (pinned_alloc:N, device_alloc:N, memcpy:N, timeout).
  * Errors: LST_ERR_ARG (bad config), LST_ERR_OOM, LST_ERR_CUDA. On error *out is NULL. */

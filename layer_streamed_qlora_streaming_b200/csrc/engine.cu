@@ -1506,6 +1506,23 @@ bool done_on_device(const std::atomic<unsigned long long>& mask) {
 void mark_done_on_device(std::atomic<unsigned long long>& mask) { mask.fetch_or(device_bit()); }
 }  // namespace lst
 
+// Makes the context's device current for the duration of an API call and restores the caller's
+// device afterwards (a thread may drive contexts on several GPUs).
+struct DeviceScope {
+  int prev = -1;
+  explicit DeviceScope(const lst_ctx* c) {
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) {
+      cudaGetLastError();
+      return;
+    }
+    if (cur != c->dev && cudaSetDevice(c->dev) == cudaSuccess) prev = cur;
+  }
+  ~DeviceScope() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
 // =========================================================================== C ABI
 extern "C" {
 
@@ -1531,6 +1548,7 @@ lst_status lst_create(const lst_config* cfg, const float* embed, const float* fi
 
 lst_status lst_register_layer(lst_ctx* c, int32_t layer, const lst_layer_weights* w) {
   if (!c) return LST_ERR_ARG;
+  DeviceScope ds(c);
   if (!w || layer < 0 || layer >= c->L) return fail(c, LST_ERR_ARG, "bad layer index or null weights");
   // the layer's bytes change: nothing kept in the pool or the weight scratch is trusted any more
   c->slot_layer[0] = c->slot_layer[1] = -1;
@@ -1540,6 +1558,7 @@ lst_status lst_register_layer(lst_ctx* c, int32_t layer, const lst_layer_weights
 
 lst_status lst_set_lora(lst_ctx* c, int32_t layer, int32_t proj, const float* a, const float* b) {
   if (!c) return LST_ERR_ARG;
+  DeviceScope ds(c);
   if (layer < 0 || layer >= c->L || proj < 0 || proj >= NPROJ || !a || !b)
     return fail(c, LST_ERR_ARG, "bad layer/projection or null pointer");
   TRY(copy_in(c, c->lora + c->offA[layer * NPROJ + proj], a, (int64_t)c->r * c->lay.ind[proj] * 4));
@@ -1577,6 +1596,7 @@ static lst_status optimizer_update(lst_ctx* c) {
 lst_status lst_step(lst_ctx* c, const int32_t* tokens, const int32_t* targets, int32_t batch, int32_t seq,
                     float* loss, float* grads) {
   if (!c) return LST_ERR_ARG;
+  DeviceScope ds(c);
   if (!tokens || !targets || !loss) return fail(c, LST_ERR_ARG, "null tokens/targets/loss");
   if (c->V <= 0) return fail(c, LST_ERR_STATE, "lst_step needs a head (vocab > 0); use lst_step_hidden");
   TRY(begin_step(c, batch, seq));
@@ -1596,6 +1616,7 @@ lst_status lst_step(lst_ctx* c, const int32_t* tokens, const int32_t* targets, i
 lst_status lst_step_hidden(lst_ctx* c, const uint16_t* x, const uint16_t* g, int32_t batch, int32_t seq,
                            float* loss, float* grads) {
   if (!c) return LST_ERR_ARG;
+  DeviceScope ds(c);
   if (!x || !g || !loss) return fail(c, LST_ERR_ARG, "null x/g/loss");
   if (c->V != 0) return fail(c, LST_ERR_STATE, "lst_step_hidden needs a headless config (vocab == 0)");
   TRY(begin_step(c, batch, seq));
@@ -1612,6 +1633,7 @@ lst_status lst_step_hidden(lst_ctx* c, const uint16_t* x, const uint16_t* g, int
 lst_status lst_step_dpo(lst_ctx* c, const int32_t* tokens, const int32_t* targets, const int32_t* mask,
                         int32_t n_pairs, int32_t seq, float beta, float* loss, float* grads) {
   if (!c) return LST_ERR_ARG;
+  DeviceScope ds(c);
   if (!tokens || !targets || !loss) return fail(c, LST_ERR_ARG, "null tokens/targets/loss");
   if (c->V <= 0) return fail(c, LST_ERR_STATE, "lst_step_dpo needs a head (vocab > 0)");
   if (n_pairs <= 0 || !(beta > 0.f) || !std::isfinite(beta)) return fail(c, LST_ERR_ARG, "n_pairs <= 0 or beta not > 0");
@@ -1635,6 +1657,7 @@ lst_status lst_step_dpo(lst_ctx* c, const int32_t* tokens, const int32_t* target
 
 lst_status lst_get_logits(lst_ctx* c, float* dst) {
   if (!c) return LST_ERR_ARG;
+  DeviceScope ds(c);
   if (!dst) return fail(c, LST_ERR_ARG, "null dst");
   if (!c->have_logits) return fail(c, LST_ERR_STATE, "no logits: run lst_step first");
   if (!c->logits_whole) return fail(c, LST_ERR_STATE, "the head ran in passes (head_chunk): logits are not kept whole");
@@ -1647,6 +1670,7 @@ lst_status lst_get_logits(lst_ctx* c, float* dst) {
 
 lst_status lst_get_activation(lst_ctx* c, int32_t which, int32_t layer, void* dst) {
   if (!c) return LST_ERR_ARG;
+  DeviceScope ds(c);
   if (!dst) return fail(c, LST_ERR_ARG, "null dst");
   if (c->st.steps == 0) return fail(c, LST_ERR_STATE, "no step has run");
   const int64_t T = c->curT, d = c->d;
@@ -1677,6 +1701,7 @@ lst_status lst_get_activation(lst_ctx* c, int32_t which, int32_t layer, void* ds
 
 lst_status lst_set_optimizer(lst_ctx* c, const lst_adamw* cfg) {
   if (!c) return LST_ERR_ARG;
+  DeviceScope ds(c);
   if (!cfg) {
     c->opt_on = false;
     return LST_OK;
@@ -1700,6 +1725,7 @@ lst_status lst_set_optimizer(lst_ctx* c, const lst_adamw* cfg) {
 
 lst_status lst_apply_optimizer(lst_ctx* c, const float* g) {
   if (!c) return LST_ERR_ARG;
+  DeviceScope ds(c);
   if (!g) return fail(c, LST_ERR_ARG, "null gradient");
   if (!c->opt_on || !c->opt.deferred) return fail(c, LST_ERR_STATE, "set the optimizer with deferred = 1 first");
   const float* src = g;
@@ -1714,6 +1740,7 @@ lst_status lst_apply_optimizer(lst_ctx* c, const float* g) {
 
 lst_status lst_get_lora(lst_ctx* c, float* dst) {
   if (!c) return LST_ERR_ARG;
+  DeviceScope ds(c);
   if (!dst) return fail(c, LST_ERR_ARG, "null dst");
   const bool dev = is_device_ptr(dst);
   CK(cudaMemcpyAsync(dst, c->lora, c->lora_numel * 4, dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
@@ -1767,7 +1794,10 @@ const char* lst_last_error(const lst_ctx* c) { return c ? c->err.c_str() : "null
 
 void lst_destroy(lst_ctx* c) {
   if (!c) return;
-  free_all(c);
+  {
+    DeviceScope ds(c);
+    free_all(c);
+  }
   delete c;
 }
 
