@@ -210,6 +210,12 @@ class Context:
 
     __del__ = close
 
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
     def register_layer(self, layer: int, W: dict, A: dict, B: dict, attn_norm, mlp_norm, bias=None):
         lw = LayerWeights()
         for i, p in enumerate(PROJ):
