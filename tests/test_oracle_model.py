@@ -321,3 +321,16 @@ def test_dpo_backward_matches_finite_differences():
                 vals.append(M.dpo_step(wl, raw, head, toks, tgts, 1, 0.5, mask=mask, lora=lora)["loss"])
             fd = (vals[0] - vals[1]) / (2 * h)
             assert abs(fd - an[idx]) <= 1e-6 * np.abs(an).max() + 1e-11, (proj, which, fd, an[idx])
+
+
+def test_preference_pairs_share_prompts_and_mask_responses():
+    wl = tiny(batch=6, seq=10)
+    t, y, m = syn.preference_pairs(wl)
+    P, S = 3, 10
+    t, y, m = t.reshape(2 * P, S), y.reshape(2 * P, S), m.reshape(2 * P, S)
+    assert np.array_equal(t[:P, :S // 2], t[P:, :S // 2]) and np.array_equal(y[:P, :S // 2], y[P:, :S // 2])
+    assert not np.array_equal(t[:P, S // 2:], t[P:, S // 2:])          # responses differ
+    assert np.all(m[:, :S // 2] == 0) and np.all(m[:, S // 2:] == 1)
+    assert t.min() >= 0 and t.max() < wl.vocab and y.max() < wl.vocab
+    t2, _, _ = syn.preference_pairs(wl)
+    assert np.array_equal(t.reshape(-1), t2)                               # seeded
