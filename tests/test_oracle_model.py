@@ -334,3 +334,44 @@ def test_preference_pairs_share_prompts_and_mask_responses():
     assert t.min() >= 0 and t.max() < wl.vocab and y.max() < wl.vocab
     t2, _, _ = syn.preference_pairs(wl)
     assert np.array_equal(t.reshape(-1), t2)                               # seeded
+
+
+def _fd_discrepancy(wl, picks, h=1e-4):
+    """max over picks of |central difference - analytic| / max|analytic| of the oracle's loss."""
+    inp = build(wl)
+    ref = M.step(wl, **inp)
+    lora0 = [{p: (r["A"][p].astype(np.float64), r["B"][p].astype(np.float64)) for p in M.PROJ}
+             for r in inp["raw_layers"]]
+    rng = np.random.default_rng(5)
+    worst = 0.0
+    for layer, proj, which in picks:
+        an = ref["grads"][layer][proj][which]
+        idx = tuple(rng.integers(0, s) for s in an.shape)
+        vals = []
+        for sgn in (1, -1):
+            lora = [{p: (A.copy(), B.copy()) for p, (A, B) in l.items()} for l in lora0]
+            lora[layer][proj][which][idx] += sgn * h
+            vals.append(M.step(wl, lora=lora, **inp)["loss"])
+        fd = (vals[0] - vals[1]) / (2 * h)
+        worst = max(worst, abs(fd - an[idx]) / np.abs(an).max())
+    return worst
+
+
+@pytest.mark.parametrize("plant", ["rope_sign", "rmsnorm_term", "dv_scale"])
+def test_planted_backward_mistakes_fail_the_difference_check(monkeypatch, plant):
+    # a mistake planted in the oracle's backward (on the CPU) must show up against central
+    # differences of its own forward; the clean backward agrees to ~1e-7
+    wl = tiny(n_layers=1, n_kv_heads=2)
+    picks = [(0, p, w) for p in ("q", "k", "v") for w in (0, 1)]
+    clean = _fd_discrepancy(wl, picks)
+    assert clean < 1e-6
+    if plant == "rope_sign":
+        monkeypatch.setattr(M, "rope_bwd", lambda dy, cos, sin, b, s: M.rope(dy, cos, sin, b, s))
+    elif plant == "rmsnorm_term":
+        def no_mean_term(dy, x, g, r):
+            return dy * g[None, :] * r[:, None]
+        monkeypatch.setattr(M, "rmsnorm_bwd", no_mean_term)
+    else:
+        orig = M.attention_bwd
+        monkeypatch.setattr(M, "attention_bwd", lambda *a: (lambda dq, dk, dv: (dq, dk, dv * 1.01))(*orig(*a)))
+    assert _fd_discrepancy(wl, picks) > 100 * max(clean, 1e-9)
