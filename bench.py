@@ -251,10 +251,27 @@ def max_over_ranks(ms: float, dist, device) -> float:
 
 def allreduce_grads(grads, dist) -> None:
     """Data-parallel exchange: average the LoRA gradients of all replicas (NCCL on GPUs), so every
-    replica applies the same update."""
-    if dist is not None:
-        dist.all_reduce(grads)
-        grads.div_(dist.get_world_size())
+    replica applies the same update. The sum runs in a fixed order (rank 0, 1, ..., N-1), whatever
+    algorithm the collective library picks, so every replica and every run gets the same bytes:
+    rank q gathers shard q of every replica's gradient (all-to-all), adds the N copies in rank
+    order, and the reduced shards are then gathered by everyone (all-gather)."""
+    if dist is None:
+        return
+    import torch
+    N = dist.get_world_size()
+    n = grads.numel()
+    shard = -(-n // N)
+    g = torch.nn.functional.pad(grads, (0, shard * N - n)) if shard * N != n else grads
+    parts = torch.empty_like(g)
+    dist.all_to_all_single(parts, g)              # parts[q] = replica q's copy of my shard
+    parts = parts.view(N, shard)
+    acc = parts[0].clone()
+    for q in range(1, N):
+        acc += parts[q]
+    acc /= N
+    out = torch.empty(N * shard, dtype=grads.dtype, device=grads.device)
+    dist.all_gather_into_tensor(out, acc)
+    grads.copy_(out[:n])
 
 
 def job_throughput(world: int, tokens_per_step: int, steps: int, ms: float) -> float:

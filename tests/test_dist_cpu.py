@@ -26,6 +26,16 @@ def _worker(rank, world, port, q):
     try:
         g = torch.full((1000,), float(rank + 1))
         bench.allreduce_grads(g, dist)
+        # uneven length, values whose sum rounds: every rank gets the fixed-order mean, same bytes
+        gen = torch.Generator().manual_seed(7)
+        all_g = [torch.randn(1001, generator=gen) * 10 ** k for k in range(world)]
+        mine = all_g[rank].clone()
+        bench.allreduce_grads(mine, dist)
+        ref = all_g[0].clone()
+        for k in range(1, world):
+            ref += all_g[k]
+        ref /= world
+        q.put(("mean", rank, mine.numpy().tobytes() == ref.numpy().tobytes()))
         ms = bench.max_over_ranks(100.0 + 50.0 * rank, dist, "cpu")
         thr = bench.job_throughput(world, 2048, 10, ms)
         q.put((rank, float(g[0]), float(g[-1]), ms, thr))
@@ -44,7 +54,9 @@ def test_two_ranks_gloo():
     for p in procs:
         p.join(120)
         assert p.exitcode == 0
-    res = sorted(q.get(timeout=10) for _ in range(world))
+    got = [q.get(timeout=10) for _ in range(2 * world)]
+    assert all(ok for tag, _, ok in (x for x in got if x[0] == "mean"))
+    res = sorted(x for x in got if x[0] != "mean")
     for rank, g0, g1, ms, thr in res:
         assert g0 == g1 == 1.5            # mean of 1 and 2 on both ranks
         assert ms == 150.0                # the slowest rank
