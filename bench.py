@@ -518,6 +518,8 @@ def run_gpu(args, wl):
                           "profiled_step_ms": agg["step_ms"] / K,
                           "note": "class times from K extra steps with CUDA events around each launch"},
         "gpu_launches": int(agg["launches_last_step"] / K * K),
+        "memory": {"library_device_bytes": int(st["device_bytes"]), "pinned_host_bytes": int(st["arena_bytes"]),
+                   "layer_blob_bytes": int(st["blob_bytes"])},
         "clocks": clk.summary(),
     }
     line["e2e"] = e2e
