@@ -465,3 +465,82 @@ def dpo_step(wl, raw_layers, head, tokens, targets, npairs, beta, mask=None, blo
     for i in reversed(range(L)):
         dx, grads[i] = layer_bwd(dx, caches[i], Ws[i], lora[i], sh)
     return {"loss": loss, "grads": grads, "pi": pi, "ref": ref}
+
+
+# ------------------------------------------------------------------------------------------
+# reference-free preference losses named next to DPO (ORPO, SimPO)
+# ------------------------------------------------------------------------------------------
+# [TESS] lists ORPO and SimPO (with DPO and KTO) among the preference losses run over the streamed
+# base. Neither needs a reference model, so a step is the ordinary 2L reads. Losses as published:
+# SimPO (Meng, Xia and Chen, "SimPO: Simple Preference Optimization with a Reference-Free Reward",
+# 2024): reward r(y) = beta / |y| * log pi(y); L = -log sigmoid(r(y_w) - r(y_l) - gamma).
+# ORPO (Hong, Lee and Thorne, "ORPO: Monolithic Preference Optimization without Reference Model",
+# 2024): with l(y) = log pi(y) / |y| (length-normalised) and odds(y) = e^l / (1 - e^l),
+# L = -l(y_w) + lambda * -log sigmoid(log odds(y_w) - log odds(y_l)).
+# |y| is the number of masked positions of a sequence. Same batch layout and masks as DPO; the
+# step's loss is the mean over pairs.
+
+def simpo_loss(pi, counts, beta, gamma):
+    """Mean SimPO loss over pairs and dL/dpi per sequence (pi, counts: [2P], chosen first)."""
+    P = pi.shape[0] // 2
+    r = beta * pi / counts
+    z = r[:P] - r[P:] - gamma
+    loss = float(np.mean(np.logaddexp(0.0, -z)))
+    dz = (1.0 / (1.0 + np.exp(-z)) - 1.0) / P                # dL/dz per pair
+    return loss, np.concatenate([dz * beta / counts[:P], -dz * beta / counts[P:]])
+
+
+def orpo_loss(pi, counts, lam):
+    """Mean ORPO loss over pairs and dL/dpi per sequence (pi, counts: [2P], chosen first)."""
+    P = pi.shape[0] // 2
+    ell = pi / counts                                        # mean log-likelihood per token, < 0
+    log_odds = ell - np.log1p(-np.exp(ell))
+    z = log_odds[:P] - log_odds[P:]
+    loss = float(np.mean(-ell[:P] + lam * np.logaddexp(0.0, -z)))
+    dz = lam * (1.0 / (1.0 + np.exp(-z)) - 1.0) / P           # d(mean lam * L_OR)/dz per pair
+    dodds = 1.0 / (1.0 - np.exp(ell))                          # d log_odds / d ell
+    d_ell = np.concatenate([-1.0 / P + dz * dodds[:P], -dz * dodds[P:]])
+    return loss, d_ell / counts
+
+
+def pref_dlogits(logits, targets, mask, nseq, seq, kind, **kw):
+    """(loss, dL/dlogits, pi) of a reference-free preference loss (kind "simpo" or "orpo") as a
+    function of the policy logits, the same way as ``dpo_dlogits``."""
+    pi, lse = seq_logp(logits, targets, mask, nseq, seq)
+    counts = np.asarray(mask, dtype=F64).reshape(nseq, seq).sum(axis=1)
+    if kind == "simpo":
+        loss, g = simpo_loss(pi, counts, kw["beta"], kw["gamma"])
+    elif kind == "orpo":
+        loss, g = orpo_loss(pi, counts, kw["lam"])
+    else:
+        raise ValueError(kind)
+    T = logits.shape[0]
+    w = -np.repeat(g, seq) * mask
+    dlog = np.exp(logits - lse[:, None])
+    dlog[np.arange(T), targets] -= 1.0
+    return loss, dlog * w[:, None], pi
+
+
+def pref_step(wl, raw_layers, head, tokens, targets, npairs, kind, mask=None, blobs=None, bf16_acts=False,
+              lora=None, **kw):
+    """Loss and LoRA gradients of one SimPO or ORPO step (no reference pass)."""
+    L = wl.n_layers
+    sh = Shape(wl, bf16_acts)
+    nseq, S = 2 * npairs, wl.seq
+    assert nseq == wl.batch
+    if blobs is None:
+        blobs = [pack_layer(raw_layers[i], wl.base_format) for i in range(L)]
+    if lora is None:
+        lora = [_lora64(raw_layers[i]) for i in range(L)]
+    E, gf, H = (a.astype(F64) for a in head)
+    m = np.ones(nseq * S) if mask is None else np.asarray(mask, dtype=F64)
+    Ws = [unpack_blob(blobs[i]) for i in range(L)]
+    xL, caches = _forward(E[tokens], Ws, lora, sh)
+    n, r = rmsnorm(xL, gf, wl.rms_eps)
+    logits = sh.rb(n) @ H.T
+    loss, dlog, pi = pref_dlogits(logits, targets, m, nseq, S, kind, **kw)
+    dx = rmsnorm_bwd(sh.rb(dlog) @ H, xL, gf, r)
+    grads = [None] * L
+    for i in reversed(range(L)):
+        dx, grads[i] = layer_bwd(dx, caches[i], Ws[i], lora[i], sh)
+    return {"loss": loss, "grads": grads, "pi": pi}

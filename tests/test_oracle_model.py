@@ -375,3 +375,74 @@ def test_planted_backward_mistakes_fail_the_difference_check(monkeypatch, plant)
         orig = M.attention_bwd
         monkeypatch.setattr(M, "attention_bwd", lambda *a: (lambda dq, dk, dv: (dq, dk, dv * 1.01))(*orig(*a)))
     assert _fd_discrepancy(wl, picks) > 100 * max(clean, 1e-9)
+
+
+# ---------------------------------------------------------------- SimPO / ORPO (reference-free)
+@pytest.mark.parametrize("kind", ["simpo", "orpo"])
+def test_reference_free_losses_match_torch_autograd(kind):
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(4)
+    nseq, S, V = 4, 7, 13
+    logits = rng.normal(size=(nseq * S, V)) * 2
+    tg = rng.integers(0, V, nseq * S)
+    mask = (rng.random(nseq * S) < 0.7).astype(np.float64)
+    mask.reshape(nseq, S)[:, 0] = 1.0                        # every sequence counts a position
+    kw = {"beta": 2.0, "gamma": 0.3} if kind == "simpo" else {"lam": 0.25}
+    loss, dlog, pi = M.pref_dlogits(logits, tg, mask, nseq, S, kind, **kw)
+    lt = torch.tensor(logits, requires_grad=True)
+    lp = torch.log_softmax(lt, dim=1).gather(1, torch.tensor(tg)[:, None])[:, 0] * torch.tensor(mask)
+    pit = lp.reshape(nseq, S).sum(1)
+    cnt = torch.tensor(mask).reshape(nseq, S).sum(1)
+    P = nseq // 2
+    F = torch.nn.functional
+    if kind == "simpo":
+        r = kw["beta"] * pit / cnt
+        lt_loss = -F.logsigmoid(r[:P] - r[P:] - kw["gamma"]).mean()
+    else:
+        ell = pit / cnt
+        lo = ell - torch.log1p(-torch.exp(ell))
+        lt_loss = (-ell[:P] - kw["lam"] * F.logsigmoid(lo[:P] - lo[P:])).mean()
+    lt_loss.backward()
+    assert abs(float(lt_loss.detach()) - loss) < 1e-12
+    assert np.allclose(pit.detach().numpy(), pi, rtol=0, atol=1e-12)
+    assert np.allclose(lt.grad.numpy(), dlog, rtol=0, atol=1e-13)
+
+
+def test_reference_free_losses_closed_forms_on_identical_pairs():
+    # chosen == rejected: SimPO's margin term alone remains and its gradient cancels; ORPO keeps
+    # its SFT term on the chosen sequence
+    wl = tiny(batch=2, n_layers=1)
+    raw, head, toks, tgts, mask = _dpo_inputs(wl)
+    S = wl.seq
+    toks[S:], tgts[S:], mask[S:] = toks[:S], tgts[:S], mask[:S]
+    out = M.pref_step(wl, raw, head, toks, tgts, 1, "simpo", mask=mask, beta=2.0, gamma=0.5)
+    assert abs(out["loss"] - math.log1p(math.exp(0.5))) < 1e-14
+    for g in out["grads"]:
+        for dA, dB in g.values():
+            assert np.abs(dA).max() < 1e-14 and np.abs(dB).max() < 1e-14
+    out = M.pref_step(wl, raw, head, toks, tgts, 1, "orpo", mask=mask, lam=0.1)
+    ell = out["pi"][0] / mask[:S].sum()
+    assert abs(out["loss"] - (-ell + 0.1 * math.log(2.0))) < 1e-12
+    assert any(np.abs(dB).max() > 0 for g in out["grads"] for (_, dB) in g.values())
+
+
+@pytest.mark.parametrize("kind", ["simpo", "orpo"])
+def test_reference_free_backward_matches_finite_differences(kind):
+    wl = tiny(batch=2, n_layers=1)
+    raw, head, toks, tgts, mask = _dpo_inputs(wl)
+    kw = {"beta": 2.0, "gamma": 0.3} if kind == "simpo" else {"lam": 0.5}
+    lora0 = [{p: (r["A"][p].astype(np.float64), r["B"][p].astype(np.float64)) for p in M.PROJ} for r in raw]
+    ref = M.pref_step(wl, raw, head, toks, tgts, 1, kind, mask=mask, lora=lora0, **kw)
+    rng = np.random.default_rng(12)
+    h = 1e-4
+    for proj in ("q", "v", "up", "down"):
+        for which in (0, 1):
+            an = ref["grads"][0][proj][which]
+            idx = tuple(rng.integers(0, s) for s in an.shape)
+            vals = []
+            for sgn in (1, -1):
+                lora = [{p: (A.copy(), B.copy()) for p, (A, B) in l.items()} for l in lora0]
+                lora[0][proj][which][idx] += sgn * h
+                vals.append(M.pref_step(wl, raw, head, toks, tgts, 1, kind, mask=mask, lora=lora, **kw)["loss"])
+            fd = (vals[0] - vals[1]) / (2 * h)
+            assert abs(fd - an[idx]) <= 1e-6 * np.abs(an).max() + 1e-11, (kind, proj, which, fd, an[idx])
