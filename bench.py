@@ -46,29 +46,6 @@ def describe(wl) -> str:
             f"a{int(wl.lora_alpha)} on 7 projections{head}, batch {wl.batch} x seq {wl.seq}")
 
 
-# DRAM traffic (read + write) of the GEMM launches of one llama8b step, from one ncu capture of the
-# bench (dram__bytes_read.sum + dram__bytes_write.sum over the step's 354 k_gemm launches; command
-# and figures in profiles/gemm_traffic_llama8b_step.md). Valid only for the GEMM sources measured
-# (hashes taken after a host-side change to the launcher's per-device set-up; kernel unchanged).
-GEMM_TRAFFIC = {"workload": "llama8b", "bytes_per_step": 73.988e9, "launches": 354,
-                "sources": {"gemm.cu": "e0a88be30295bc55", "gemm.cuh": "4a668b6d34dc410f",
-                            "common.cuh": "da32f91f59c8b4d8"}}
-
-
-def gemm_traffic(wl_name: str):
-    """(bytes per launch, bytes per step) of the recorded capture, or (None, None) when the
-    workload differs or the GEMM sources changed since it was taken."""
-    import hashlib
-    if wl_name != GEMM_TRAFFIC["workload"]:
-        return None, None
-    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "layer_streamed_qlora_streaming_b200", "csrc")
-    for f, h in GEMM_TRAFFIC["sources"].items():
-        with open(os.path.join(csrc, f), "rb") as fh:
-            if hashlib.sha256(fh.read()).hexdigest()[:16] != h:
-                return None, None
-    return GEMM_TRAFFIC["bytes_per_step"] / GEMM_TRAFFIC["launches"], GEMM_TRAFFIC["bytes_per_step"]
-
-
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -99,7 +76,7 @@ def h2d_peak_gbs(torch) -> float:
     return best
 
 
-def build_context(wl, torch, stream, seed: int = 1234):
+def build_context(wl, torch, stream, seed: int = 1234, streamed: bool = True):
     """Library context with every layer registered from device-resident synthetic weights."""
     import layer_streamed_qlora_streaming_b200 as lst
     g = torch.Generator(device="cuda")
@@ -112,7 +89,7 @@ def build_context(wl, torch, stream, seed: int = 1234):
     def uniform(shape, b):
         return (torch.rand(shape, generator=g, device=dev, dtype=torch.float32) * 2 - 1) * b
 
-    cfg = lst.make_config(wl, streamed=True)
+    cfg = lst.make_config(wl, streamed=streamed)
     if wl.vocab:
         E = normal((wl.vocab, wl.d_model), 0.02)
         H = normal((wl.vocab, wl.d_model), 0.02)
@@ -136,6 +113,99 @@ def build_context(wl, torch, stream, seed: int = 1234):
         del W, A, B, bias
     torch.cuda.synchronize()
     return ctx
+
+
+def timeline_summary(tl) -> dict:
+    """Copy / compute overlap of one profiled step, from the library's per-read timeline: per read
+    kind, mean copy, dequant and compute durations; how much of each read's copy ran while the
+    compute stream was busy with an earlier read; and the compute stream's idle time waiting for
+    copies inside the step."""
+    out = {}
+    for kind in ("forward", "backward"):
+        rows = [r for r in tl if r["kind"] == kind]
+        if not rows:
+            continue
+        def mean(xs):
+            xs = [x for x in xs if x is not None]
+            return sum(xs) / len(xs) if xs else None
+        cp = [r["copy"][1] - r["copy"][0] for r in rows if r["copy"][0] is not None]
+        dq = [r["dequant"][1] - r["dequant"][0] for r in rows if r["dequant"][0] is not None]
+        cm = [r["compute"][1] - r["compute"][0] for r in rows]
+        out[kind] = {"reads": len(rows), "copy_ms": mean(cp), "dequant_ms": mean(dq), "compute_ms": mean(cm)}
+    # hidden copy time: the part of each copy interval covered by the compute intervals of the reads
+    comp = sorted(r["compute"] for r in tl)
+    hidden = total = 0.0
+    for r in tl:
+        c0, c1 = r["copy"]
+        if c0 is None:
+            continue
+        total += c1 - c0
+        for k0, k1 in comp:
+            hidden += max(0.0, min(c1, k1) - max(c0, k0))
+    # compute-stream gaps between consecutive reads (waiting for a copy or dequant, or the head)
+    gaps = [max(0.0, tl[n]["compute"][0] - tl[n - 1]["compute"][1]) for n in range(1, len(tl))]
+    out["copy_hidden_frac"] = hidden / total if total else None
+    out["compute_gap_ms_total"] = sum(gaps)
+    out["first_compute_start_ms"] = tl[0]["compute"][0]
+    out["last_compute_end_ms"] = tl[-1]["compute"][1]
+    return out
+
+
+def time_steps(torch, stream, step, steps: int, warmup: int) -> float:
+    """ms of `steps` back-to-back calls of step() after `warmup` untimed ones (CUDA events on the
+    library's stream, synchronised on both sides)."""
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def sub_workload(name: str, torch, stream, link_gbs: float, steps: int, warmup: int, modes=("streamed",)):
+    """tokens/s of one more workload on this GPU in the given modes ("streamed": base in pinned host
+    memory, 2L layer copies per step; "resident": base kept on the GPU), the streamed mode's PCIe
+    floor and the copy / compute overlap of one profiled step. AdamW inside every step, as the
+    main line."""
+    import synthetic as syn
+    wl = syn.WORKLOADS[name]
+    T = wl.tokens
+    out = {"workload": describe(wl)}
+    for streamed in (m == "streamed" for m in modes):
+        ctx = build_context(wl, torch, stream, seed=4321, streamed=streamed)
+        ctx.set_optimizer(lr=2e-4)
+        g = torch.Generator(device="cpu")
+        g.manual_seed(7)
+        if wl.vocab:
+            toks = torch.randint(0, wl.vocab, (T,), generator=g, dtype=torch.int32).cuda()
+            tgts = torch.randint(0, wl.vocab, (T,), generator=g, dtype=torch.int32).cuda()
+            step = lambda: ctx.step(toks, tgts, wl.batch, wl.seq)
+        else:
+            x = torch.randn(T, wl.d_model, generator=g).to(torch.bfloat16).cuda().view(torch.int16)
+            gg = torch.randn(T, wl.d_model, generator=g).to(torch.bfloat16).cuda().view(torch.int16)
+            step = lambda: ctx.step_hidden(x, gg, wl.batch, wl.seq)
+        ms = time_steps(torch, stream, step, steps, warmup) / steps
+        st = ctx.stats()
+        entry = {"value": T / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "steps": steps, "warmup": warmup,
+                 "layer_reads_per_step": st["layer_reads_last_step"], "h2d_bytes_per_step": st["h2d_bytes_last_step"],
+                 "layer_blob_bytes": st["blob_bytes"], "base_bytes": st["arena_bytes"]}
+        if streamed:
+            floor = st["h2d_bytes_last_step"] / (link_gbs * 1e9) * 1e3
+            entry.update({"pinned_host_bytes": st["arena_bytes"], "min_ms": floor, "frac": floor / ms})
+            ctx.set_profiling(True)
+            step()
+            torch.cuda.synchronize()
+            entry["overlap"] = timeline_summary(ctx.read_timeline())
+            ctx.set_profiling(False)
+        out["streamed" if streamed else "resident"] = entry
+        ctx.close()
+        del ctx
+        torch.cuda.empty_cache()
+    return out
 
 
 class ClockSampler:
@@ -226,6 +296,15 @@ def oracle_sample(wl, seq: int = 512):
     return T / step_s, t_layer + t_head, desc
 
 
+def oracle_sample_threads(wl, seq: int, threads: int):
+    """oracle_sample with the BLAS thread pool limited to `threads` (None: as configured)."""
+    if threads is None:
+        return oracle_sample(wl, seq=seq)
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=threads):
+        return oracle_sample(wl, seq=seq)
+
+
 def cpu_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -286,14 +365,19 @@ def run_reference(args, wl):
         return
     for _ in range(args.warmup):
         oracle_sample(wl, seq=args.ref_seq)
-    vals, secs, desc = [], 0.0, ""
+    vals, secs, desc = [], [], ""
     for _ in range(args.steps):
-        v, s, desc = oracle_sample(wl, seq=args.ref_seq)
+        v, sec, desc = oracle_sample(wl, seq=args.ref_seq)
         vals.append(v)
-        secs += s
+        secs.append(sec)
     value = statistics.median(vals)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.tokens / value * 1e3,
+            "steps": args.steps, "warmup": args.warmup,
+            # each step is a bounded sample of the workload, timed as it ran; the metric is the
+            # whole workload's tokens over the step time extrapolated from the sample
+            "ms_per_step": statistics.median(secs) * 1e3, "extrapolated": True,
+            "extrapolated_ms_per_step": wl.tokens / value * 1e3,
+            "sample_shape": {"layers": 1, "batch": 1, "seq": args.ref_seq, "head": bool(wl.vocab)},
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": describe(wl), "batch": wl.batch, "seq": wl.seq},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
@@ -320,6 +404,12 @@ def run_gpu(args, wl):
     stream = torch.cuda.Stream(priority=-1)
     link_gbs = h2d_peak_gbs(torch)
     ctx = build_context(wl, torch, stream, seed=1234 + rank)
+    split = world > 1 and args.split_copy
+    if split:
+        # every rank copies 1/N of each layer blob over its own link; NCCL all-gathers the rest
+        uid = [lst.nccl_unique_id() if rank == 0 else b""]
+        dist.broadcast_object_list(uid, src=0)
+        ctx.set_split_copy(rank, world, uid[0])
     if not args.no_optimizer:
         # one process: the step applies AdamW itself; replicas: after the gradient average
         ctx.set_optimizer(lr=2e-4, deferred=world > 1)
@@ -383,6 +473,7 @@ def run_gpu(args, wl):
         for k in agg:
             agg[k] += st[k]
     torch.cuda.synchronize()
+    overlap = timeline_summary(ctx.read_timeline())
     ctx.set_profiling(False)
     value = job_throughput(world, T, args.steps, ms)
 
@@ -481,7 +572,7 @@ def run_gpu(args, wl):
 
     st = ctx.stats()
     peaks = measured_peaks()
-    traffic_launch, traffic_step = gemm_traffic(args.workload)
+    traffic_launch, traffic_step = None, None
     K = args.steps
     gemm_ms = agg["gemm_ms"] / K
     gemm_tflops = agg["gemm_flops"] / K / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else 0.0
@@ -495,6 +586,8 @@ def run_gpu(args, wl):
         "dtype": "bf16", "data": "synthetic (seeded torch.randn weights / uniform tokens)",
         "config": {"workload": describe(wl), "batch": wl.batch, "seq": wl.seq, "layers": wl.n_layers,
                    "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                   "layer_copies": ("each rank copies 1/N of every layer blob, NCCL all-gathers the blob over "
+                                    "NVLink" if split else "every rank copies whole layer blobs over its own link"),
                    "optimizer": "none" if args.no_optimizer else (
                        "AdamW lr 2e-4 on every adapter, inside the step" if world == 1 else
                        "AdamW lr 2e-4 on every adapter with the replicas' mean gradient (NCCL all-reduce)"),
@@ -515,8 +608,9 @@ def run_gpu(args, wl):
                           "copy_ms_per_step": agg["copy_ms"] / K,
                           "attention_ms_per_step": agg["attention_ms"] / K,
                           "dequant_ms_per_step": agg["dequant_ms"] / K, "lora_ms_per_step": agg["lora_ms"] / K,
-                          "profiled_step_ms": agg["step_ms"] / K,
-                          "note": "class times from K extra steps with CUDA events around each launch"},
+                          "profiled_step_ms": agg["step_ms"] / K, "overlap": overlap,
+                          "note": "class times from K extra steps with CUDA events around each launch; "
+                                  "overlap from the per-read timeline of the last of them"},
         "gpu_launches": int(agg["launches_last_step"] / K * K),
         "memory": {"library_device_bytes": int(st["device_bytes"]), "pinned_host_bytes": int(st["arena_bytes"]),
                    "layer_blob_bytes": int(st["blob_bytes"])},
@@ -526,11 +620,30 @@ def run_gpu(args, wl):
     line["reuse_schedule"] = reuse
     if dpo is not None:
         line["dpo"] = dpo
+    ctx.close()
+    del ctx
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_extra and args.workload == "llama8b":
+        # the other configurations of the method, each its own context on this GPU in turn
+        Ke, We = min(args.steps, 5), 2
+        extra = {"note": f"{Ke} timed steps after {We} warm-up each; AdamW inside every step"}
+        extra["llama8b_resident"] = sub_workload("llama8b", torch, stream, link_gbs, Ke, We, modes=("resident",))
+        r = extra["llama8b_resident"]["resident"]
+        r["streamed_over_resident_time"] = step_ms / r["ms_per_step"]
+        extra["llama8b_layer"] = sub_workload("llama8b_layer", torch, stream, link_gbs, Ke, We,
+                                              modes=("streamed", "resident"))
+        e = extra["llama8b_layer"]
+        e["streamed_over_resident_time"] = e["streamed"]["ms_per_step"] / e["resident"]["ms_per_step"]
+        extra["qwen3b_bf16"] = sub_workload("qwen3b_bf16", torch, stream, link_gbs, Ke, We)
+        extra["qwen32b"] = sub_workload("qwen32b", torch, stream, link_gbs, Ke, We)
+        line["workloads"] = extra
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, secs, desc = oracle_sample(wl, seq=args.ref_seq)
+        v, secs, desc = oracle_sample_threads(wl, args.ref_seq, None)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                                 "sample": desc, "cpu_seconds": secs}
-    ctx.close()
+        v1, secs1, desc1 = oracle_sample_threads(wl, 64, 1)
+        line["cpu_baseline"]["one_core"] = {"value": v1, "unit": UNIT, "cores": 1, "sample": desc1,
+                                            "cpu_seconds": secs1}
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -545,9 +658,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="llama8b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-seq", type=int, default=512)
+    ap.add_argument("--ref-seq", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-optimizer", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="time only the main workload")
+    ap.add_argument("--split-copy", action="store_true",
+                    help="N > 1: each rank copies 1/N of every layer blob, NCCL all-gathers it over NVLink")
     args = ap.parse_args()
     wl = workload(args.workload)
     if args.impl == "reference":

@@ -217,6 +217,38 @@ lst_status lst_get_activation(lst_ctx* ctx, int32_t which, int32_t layer, void* 
 /* Record per-class device times of every step (CUDA events around each launch) when on != 0. */
 lst_status lst_set_profiling(lst_ctx* ctx, int32_t on);
 
+/* Per-read timeline of the last step run with profiling on (the library's own CUDA events; stands
+ * in for a trace). One row of 8 floats per layer read, in read order: layer, kind (0 reference
+ * forward, 1 forward, 2 backward with recompute), then milliseconds from the start of the step:
+ * copy start, copy end (copy stream), dequant start, dequant end (prep stream, NF4 base), compute
+ * start (compute stream, once the read's first weight group is in place), compute end. A time is
+ * -1 where the read had no copy or dequant of its own (reuse, bf16 base). *n_reads receives the
+ * number of reads; out must hold max_reads >= that many rows (else LST_ERR_ARG). LST_ERR_STATE if
+ * no profiled step has run. Host only; no synchronisation (the step has completed). */
+lst_status lst_get_read_timeline(const lst_ctx* ctx, float* out, int32_t max_reads, int32_t* n_reads);
+
+/* Split copies over several GPUs (one process per GPU, each with its own context holding the same
+ * base): each layer read copies only this rank's slice of the blob over its own host link, and an
+ * in-place NCCL all-gather on the copy stream assembles the whole blob in every rank's pool slot
+ * over NVLink / NVSwitch, so N GPUs divide the host-link bytes of every read by N. All ranks must
+ * run the same steps in the same order (the reads are collective). The library loads
+ * libnccl.so.2 on first use (LST_ERR_STATE if it cannot); the communicator is created here
+ * (ncclCommInitRank, collective over the ranks) and destroyed with the context. unique_id: the 128
+ * bytes of lst_nccl_unique_id from one rank, passed to every rank. world == 1 does nothing. Needs
+ * a streamed context; call once, before the first step. The results are the same bytes as
+ * without it (the assembled blob is the same). */
+lst_status lst_set_split_copy(lst_ctx* ctx, int32_t rank, int32_t world, const void* unique_id);
+
+/* A fresh NCCL unique id (128 bytes into out) for lst_set_split_copy. LST_ERR_STATE without NCCL. */
+lst_status lst_nccl_unique_id(void* out);
+
+/* The split-copy plan of a blob of blob_bytes (host only, no GPU): rank `rank` of `world` copies
+ * bytes [*offset, *offset + *bytes) of the blob (*bytes may be 0) and contributes *count bytes
+ * (a multiple of 256) from offset *offset of its pool slot to the all-gather of world * *count
+ * bytes, whose first blob_bytes are the blob. */
+lst_status lst_split_plan(int64_t blob_bytes, int32_t world, int32_t rank, int64_t* offset, int64_t* bytes,
+                          int64_t* count);
+
 /* The copy / dequant plan of one step, host only (no context, no GPU), for inspection and tests.
  * reads: the layer of each read in order (an SFT step reads 0..L-1 then L-1..0; a DPO step reads
  * 0..L-1 once more first); reuse / nf4: the config's reuse and base_format == LST_BASE_NF4;
@@ -228,6 +260,13 @@ lst_status lst_set_profiling(lst_ctx* ctx, int32_t on);
  * pointer, n_reads <= 0 or a negative layer. */
 lst_status lst_plan_reads(const int32_t* reads, int32_t n_reads, int32_t reuse, int32_t nf4,
                           int32_t* held, int32_t* wheld, int32_t* out);
+
+/* Where an NF4 base is dequantised in the next steps: 0 (default) in a separate pass that writes
+ * each layer read's bf16 weights to a device scratch, one read ahead on a low-priority stream;
+ * 1 inside the GEMMs, which build the bf16 operand tile by tile in shared memory from the NF4 blob
+ * (groups whose rows are not whole 64-element blocks keep the separate pass). The results are the
+ * same bytes. LST_ERR_ARG for other values. */
+lst_status lst_set_dequant_mode(lst_ctx* ctx, int32_t mode);
 
 /* Switch the copy schedule of the next steps (the config's `reuse`): 1 keeps layers that are still
  * in the pool instead of copying them again, 0 copies every read. Results are the same bytes. */

@@ -32,8 +32,9 @@ lst_status lst_k_nf4_quantize(const float* w, int64_t n, uint8_t* packed, int8_t
  *    allocating routine.
  *  - n is limited to 67,108,864 elements (1 << 26); larger n returns LST_ERR_ARG and launches
  *    nothing, as does n not a multiple of 64 or a null pointer.
- *  - The first call on a device (which must be the current device) looks up the array's device
- *    address once (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Every call looks up the array's address on the current device (cudaGetSymbolAddress, which
+ *    allocates nothing), so the entry point stays valid across a device reset. The first call on
+ *    a device may load the library's device code there; make it before any stream capture.
  *  - Asynchronous on `stream`. All calls share the one array, which keeps the last call's
  *    contents (nothing in it needs clearing: it is fully rewritten before being read), so calls
  *    whose work overlaps on the GPU (other streams, other threads) race on it: order them. */
@@ -56,6 +57,29 @@ lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_
                       int64_t lda2, const uint16_t* B2, int64_t ldb2, int32_t K2, void* C,
                       int64_t ldc, int32_t c_f32, float alpha, const float* bias,
                       const float* R, int64_t ldr, void* stream);
+
+/* One NF4 tensor (format of lst_k_nf4_quantize) of a weight matrix stacked from up to three
+ * such tensors along its rows (q/k/v, gate/up), covering `rows` consecutive rows. */
+typedef struct {
+  const uint8_t* packed;  /* [rows * cols / 2], 16-byte aligned */
+  const int8_t* qabs;     /* [rows * cols / 64] */
+  const float* gscale;    /* [ceil(rows * cols / 64 / 256)] */
+  const float* mean;      /* [1] */
+  int32_t rows;
+} lst_nf4_part;
+
+/* lst_k_gemm with the frozen base B dequantised from NF4 inside the GEMM ("Fine-Tuning an 8B
+ * Parameter Model on a 4 GB Laptop GPU", section "Quantization: Shrink the Weights": the 4-bit
+ * base is expanded to 16 bits for the matrix product): W = the nparts (1..3) tensors stacked
+ * along rows; b_mn = 0: C = A W^T with W [N, K]; b_mn = 1: C = A W with W [K, N]. W's row length
+ * (K or N) must be a multiple of 64, a_mn is 0, the parts must cover W's rows. The operand equals
+ * lst_k_nf4_dequant of the parts bit for bit, so C equals lst_k_gemm on the dequantised matrix
+ * byte for byte. parts is a HOST array. Other arguments as lst_k_gemm. */
+lst_status lst_k_gemm_nf4(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda,
+                          const lst_nf4_part* parts, int32_t nparts, int32_t b_mn,
+                          const uint16_t* A2, int64_t lda2, const uint16_t* B2, int64_t ldb2,
+                          int32_t K2, void* C, int64_t ldc, int32_t c_f32, float alpha,
+                          const float* bias, const float* R, int64_t ldr, void* stream);
 
 /* Causal GQA attention forward over T = batch*S tokens: q [T, ldq], k [T, ldk], v [T, ldv]
  * (head h at column h*hd), o [T, ldo] bf16, lse [T, hq] fp32. hd in {64, 128}. */
@@ -108,11 +132,25 @@ lst_status lst_k_lora_skinny(const uint16_t* X, int64_t ldx, int64_t T, int32_t 
                              const uint16_t* Bop, int64_t ldb, int32_t b_mn, int32_t KP, float s,
                              uint16_t* Us, void* stream);
 
+/* The same projection at fp32-level precision for adapters kept in full precision (same section):
+ * each adapter value is stored as the bf16 pair hi = bf16(a), lo = bf16(a - hi), hi in sections
+ * [0, RS) and [RS, 2 RS) and lo in [2 RS, 3 RS) of the KP-wide dimension of Bop (rows when
+ * b_mn = 0, columns when b_mn = 1). U = s X (hi + lo) is accumulated in fp32 and its columns
+ * j < R are stored as bf16 pairs too: Us[t][j] = Us[t][2 RS + j] = bf16(U), Us[t][RS + j] =
+ * bf16(U - bf16(U)); the other columns of Us [T, KP] are not written. Sections [hi | lo | hi] of
+ * Us against [hi | hi | lo] of the operand form, in one extra K block of the base GEMM, the
+ * product of U and the adapter up to the lo x lo term. R <= RS <= 64, RS a multiple of 8,
+ * 3 RS <= KP, KP a multiple of 8. Deterministic, no scratch. */
+lst_status lst_k_lora_skinny_split(const uint16_t* X, int64_t ldx, int64_t T, int32_t K,
+                                   const uint16_t* Bop, int64_t ldb, int32_t b_mn, int32_t R,
+                                   int32_t RS, int32_t KP, float s, uint16_t* Us, void* stream);
+
 /* LoRA adapter gradients of one fused projection group (same section): nseg (1..3) segments of rank
  * r sharing the input X bf16 [T, in] (row stride ldx), with output-gradient dY bf16 [T, out] (row
  * stride ldy) whose columns [bounds[p], bounds[p+1]) belong to segment p (bounds: HOST array of
  * nseg + 1 ints, bounds[0] = 0, bounds[nseg] = out). Us = bf16(s X A_cat^T), Vs = bf16(s dY B_exp)
- * [T, KP] (column p*r + j = rank j of segment p). Writes, fp32:
+ * [T, KP] (column p*r + j = rank j of segment p; only columns < nseg*r are read, so the hi section
+ * of a split Us / Vs serves as well). Writes, fp32:
  *   dA[p] [r, in]:        dA_p[j][i] = sum_t Vs[t][p*r + j] X[t][i]
  *   dB[p] [out_p, r]:     dB_p[o][j] = sum_t dY[t][bounds[p] + o] Us[t][p*r + j]
  * dA, dB: HOST arrays of nseg device pointers. Sums over t in a fixed order (deterministic). */

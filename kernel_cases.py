@@ -1,12 +1,15 @@
 """Run one kernel of the library on a fixed case and time it with CUDA events.
 
-    python -m layer_streamed_qlora_streaming_b200.kernel_cases CASE [--iters N] [--warmup W]
+    python kernel_cases.py CASE [--iters N] [--warmup W]
 
 Cases are the shapes of the Llama-3.1-8B-shaped layer at batch 4 x seq 512 (T = 2048 tokens):
   gemm_qkv     fused q/k/v projection: [2048, 4096] x [6144, 4096]^T + LoRA block (K + 64)
   gemm_gu      fused gate/up projection: [2048, 4096] x [28672, 4096]^T + LoRA block
   gemm_dx_gu   dX of gate/up: [2048, 28672] x [28672, 4096] (MN-major W) + LoRA block
   gemm_dx_down dX of down: [2048, 4096] x [4096, 14336] (MN-major W) + LoRA block
+  gemm_*_nf4   the same four GEMMs with W dequantised from NF4 inside the GEMM (3 weight copies
+               rotated so every launch reads its codes from HBM)
+  dequant_gu   NF4 -> bf16 of the gate/up group alone (2 x 14336 x 4096 elements)
   dequant      NF4 -> bf16 of one 8B layer (218 M elements, 7 tensors)
   attn_fwd     causal GQA attention forward, 4 x 512, 32/8 heads, hd 128
   attn_bwd     its backward (D, dK/dV, dQ kernels)
@@ -26,10 +29,14 @@ from __future__ import annotations
 
 import argparse
 import json
+import os
+import sys
 
 import torch
 
-from . import (k_attention_bwd, k_attention_fwd, k_cross_entropy, k_gemm, k_lora_grads, k_lora_skinny, k_nf4_dequant,
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+from layer_streamed_qlora_streaming_b200 import (k_attention_bwd, k_attention_fwd, k_cross_entropy, k_gemm, k_gemm_nf4,
+                                                 k_lora_grads, k_lora_skinny, k_nf4_dequant,
                k_nf4_quantize)
 
 T, D, F, HQ, HKV, HD, S = 2048, 4096, 14336, 32, 8, 128, 512
@@ -39,9 +46,57 @@ def _bf(shape, g, scale=1.0):
     return (torch.randn(shape, generator=g, device="cuda") * scale).to(torch.bfloat16)
 
 
+def _nf4(rows_list, cols, g):
+    """NF4 tensors [rows, cols] quantised on the device: the parts of a stacked weight matrix."""
+    parts = []
+    for rows in rows_list:
+        n = rows * cols
+        w = torch.randn(n, generator=g, device="cuda") * 0.02
+        packed = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
+        qabs = torch.empty(n // 64, dtype=torch.int8, device="cuda")
+        gs = torch.empty((n // 64 + 255) // 256, dtype=torch.float32, device="cuda")
+        mean = torch.empty(1, dtype=torch.float32, device="cuda")
+        k_nf4_quantize(w, packed, qabs, gs, mean)
+        parts.append((packed, qabs, gs, mean, rows))
+    return parts
+
+
 def build(case: str):
     g = torch.Generator(device="cuda")
     g.manual_seed(0)
+    if case.startswith("gemm") and case.endswith("_nf4"):
+        base = case[:-4]
+        M, N, K, bmn = {"gemm_qkv": (T, 6144, D, 0), "gemm_gu": (T, 2 * F, D, 0),
+                        "gemm_dx_gu": (T, D, 2 * F, 1), "gemm_dx_down": (T, F, D, 1)}[base]
+        rows = {"gemm_qkv": [4096, 1024, 1024], "gemm_gu": [F, F], "gemm_dx_gu": [F, F], "gemm_dx_down": [D]}[base]
+        cols = K if bmn == 0 else N
+        copies = [_nf4(rows, cols, g) for _ in range(3)]
+        A = _bf((M, K), g)
+        A2 = _bf((M, 64), g)
+        B2 = _bf((64, N) if bmn else (N, 64), g, 0.01)
+        C = torch.empty(M, N, dtype=torch.float32 if bmn else torch.bfloat16, device="cuda")
+        state = {"i": 0}
+
+        def run():
+            parts = copies[state["i"] % len(copies)]
+            state["i"] += 1
+            k_gemm_nf4(M, N, K, A, K, parts, bmn, C, N, int(bmn), A2=A2, lda2=64, B2=B2,
+                       ldb2=N if bmn else 64, K2=64)
+        return run, {"flop": 2.0 * M * N * (K + 64), "bytes": None}
+    if case == "dequant_gu":
+        n = 2 * F * D
+        w = torch.randn(n, generator=g, device="cuda") * 0.02
+        packed = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
+        qabs = torch.empty(n // 64, dtype=torch.int8, device="cuda")
+        gs = torch.empty((n // 64 + 255) // 256, dtype=torch.float32, device="cuda")
+        mean = torch.empty(1, dtype=torch.float32, device="cuda")
+        k_nf4_quantize(w, packed, qabs, gs, mean)
+        del w
+        out = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+
+        def run():
+            k_nf4_dequant(packed, qabs, gs, mean, n, out)
+        return run, {"flop": None, "bytes": n * (0.5 + 1 / 64 + 2)}
     if case.startswith("gemm"):
         spec = {"gemm_qkv": (T, 6144, D, 0), "gemm_gu": (T, 2 * F, D, 0),
                 "gemm_dx_gu": (T, D, 2 * F, 1), "gemm_dx_down": (T, F, D, 1)}[case]

@@ -77,6 +77,11 @@ _SIGS = {
     "lst_set_reuse": (_I32, [_P, _I32]),
     "lst_plan_reads": (_I32, [_P, _I32, _I32, _I32, _P, _P, _P]),
     "lst_get_stats": (_I32, [_P, C.POINTER(Stats)]),
+    "lst_get_read_timeline": (_I32, [_P, _P, _I32, C.POINTER(_I32)]),
+    "lst_set_split_copy": (_I32, [_P, _I32, _I32, _P]),
+    "lst_set_dequant_mode": (_I32, [_P, _I32]),
+    "lst_nccl_unique_id": (_I32, [_P]),
+    "lst_split_plan": (_I32, [_I64, _I32, _I32, C.POINTER(_I64), C.POINTER(_I64), C.POINTER(_I64)]),
     "lst_last_error": (C.c_char_p, [_P]),
     "lst_destroy": (None, [_P]),
     "lst_nf4_codebook": (_I32, [C.POINTER(C.c_float)]),
@@ -84,6 +89,8 @@ _SIGS = {
     "lst_k_nf4_quantize": (_I32, [_P, _I64, _P, _P, _P, _P, _P]),
     "lst_k_nf4_quantize_noalloc": (_I32, [_P, _I64, _P, _P, _P, _P, _P]),
     "lst_k_nf4_dequant": (_I32, [_P, _P, _P, _P, _I64, _P, _P]),
+    "lst_k_gemm_nf4": (_I32, [_I32, _I32, _I32, _P, _I64, _P, _I32, _I32, _P, _I64, _P, _I64, _I32, _P, _I64, _I32,
+                              _F32, _P, _P, _I64, _P]),
     "lst_k_gemm": (_I32, [_I32, _I32, _I32, _P, _I64, _I32, _P, _I64, _I32, _P, _I64, _P, _I64, _I32,
                           _P, _I64, _I32, _F32, _P, _P, _I64, _P]),
     "lst_k_attention_fwd": (_I32, [_P, _I64, _P, _I64, _P, _I64, _P, _I64, _P, _I64, _I32, _I32,
@@ -98,6 +105,7 @@ _SIGS = {
     "lst_k_swiglu_bwd": (_I32, [_P, _P, _I64, _I32, _P, _P]),
     "lst_k_cross_entropy": (_I32, [_P, _I64, _I32, _P, _F32, _P, _P, _P]),
     "lst_k_lora_skinny": (_I32, [_P, _I64, _I64, _I32, _P, _I64, _I32, _I32, _F32, _P, _P]),
+    "lst_k_lora_skinny_split": (_I32, [_P, _I64, _I64, _I32, _P, _I64, _I32, _I32, _I32, _I32, _F32, _P, _P]),
     "lst_k_lora_grads": (_I32, [_P, _I64, _I32, _P, _I64, _I32, _I64, _P, _P, _I32, _I32, _I32, _P, _P, _P, _P]),
     "lst_k_launch_count": (_I64, []),
     "lst_k_device_error": (_I32, []),
@@ -185,6 +193,19 @@ def plan_reads(reads, reuse: bool, nf4: bool, held=(-1, -1), wheld=(-1, -1)):
     _check(lib().lst_plan_reads(_ptr(r), len(r), int(bool(reuse)), int(bool(nf4)), _ptr(h), _ptr(w), _ptr(out)),
            what="lst_plan_reads")
     return out, tuple(int(x) for x in h), tuple(int(x) for x in w)
+
+
+def split_plan(blob: int, world: int, rank: int):
+    """(offset, bytes, count) of rank's slice in split-copy mode (host only)."""
+    o, b, c = C.c_int64(0), C.c_int64(0), C.c_int64(0)
+    _check(lib().lst_split_plan(blob, world, rank, C.byref(o), C.byref(b), C.byref(c)), what="lst_split_plan")
+    return o.value, b.value, c.value
+
+
+def nccl_unique_id() -> bytes:
+    buf = (C.c_char * 128)()
+    _check(lib().lst_nccl_unique_id(buf), what="lst_nccl_unique_id")
+    return bytes(buf)
 
 
 def blob_bytes(cfg: Config) -> int:
@@ -291,6 +312,31 @@ class Context:
         _check(lib().lst_get_stats(self.h, C.byref(s)), self.h, "lst_get_stats")
         return s.as_dict()
 
+    def set_dequant_mode(self, mode: int) -> None:
+        """0: separate NF4 dequantisation pass (default); 1: inside the GEMMs (lst_set_dequant_mode)."""
+        _check(lib().lst_set_dequant_mode(self.h, int(mode)), self.h, "lst_set_dequant_mode")
+
+    def set_split_copy(self, rank: int, world: int, unique_id: bytes) -> None:
+        """Split copies over `world` GPUs (lst_set_split_copy); unique_id from nccl_unique_id()."""
+        buf = (C.c_char * 128).from_buffer_copy(unique_id) if unique_id else None
+        _check(lib().lst_set_split_copy(self.h, rank, world, buf), self.h, "lst_set_split_copy")
+
+    def read_timeline(self) -> list:
+        """Per-read timeline of the last profiled step: dicts with layer, kind and the copy, dequant
+        and compute start / end in ms from the step's start (None where the read had none)."""
+        n = C.c_int32(0)
+        lib().lst_get_read_timeline(self.h, None, 0, C.byref(n))
+        buf = (C.c_float * (8 * max(n.value, 1)))()
+        _check(lib().lst_get_read_timeline(self.h, buf, n.value, C.byref(n)), self.h, "lst_get_read_timeline")
+        kinds = ("reference", "forward", "backward")
+        rows = []
+        for i in range(n.value):
+            r = buf[8 * i:8 * i + 8]
+            t = [None if v < 0 else float(v) for v in r[2:]]
+            rows.append({"layer": int(r[0]), "kind": kinds[int(r[1])], "copy": (t[0], t[1]), "dequant": (t[2], t[3]),
+                         "compute": (t[4], t[5])})
+        return rows
+
     def grad_slices(self) -> dict:
         """{(layer, proj): ((offA, shapeA), (offB, shapeB))} of the gradient layout."""
         c = self.cfg
@@ -334,6 +380,20 @@ def k_gemm(M, N, K, A, lda, B, ldb, b_mn, C_, ldc, c_f32, alpha=1.0, A2=None, ld
     _check(lib().lst_k_gemm(M, N, K, _ptr(A), lda, a_mn, _ptr(B), ldb, b_mn, _ptr(A2), lda2, _ptr(B2), ldb2,
                             K2, _ptr(C_), ldc, c_f32, alpha, _ptr(bias), _ptr(R), ldr, _stream(stream)),
            what="lst_k_gemm")
+
+
+class Nf4Part(C.Structure):
+    _fields_ = [("packed", C.c_void_p), ("qabs", C.c_void_p), ("gscale", C.c_void_p), ("mean", C.c_void_p),
+                ("rows", C.c_int32)]
+
+
+def k_gemm_nf4(M, N, K, A, lda, parts, b_mn, C_, ldc, c_f32, alpha=1.0, A2=None, lda2=0, B2=None, ldb2=0, K2=0,
+               bias=None, R=None, ldr=0, stream=None):
+    """parts: up to 3 (packed, qabs, gscale, mean, rows) NF4 tensors stacked along W's rows."""
+    arr = (Nf4Part * len(parts))(*[Nf4Part(_ptr(p), _ptr(q), _ptr(g), _ptr(m), int(r)) for p, q, g, m, r in parts])
+    _check(lib().lst_k_gemm_nf4(M, N, K, _ptr(A), lda, arr, len(parts), b_mn, _ptr(A2), lda2, _ptr(B2), ldb2, K2,
+                                _ptr(C_), ldc, c_f32, alpha, _ptr(bias), _ptr(R), ldr, _stream(stream)),
+           what="lst_k_gemm_nf4")
 
 
 def k_attention_fwd(q, ldq, k, ldk, v, ldv, o, ldo, lse, T, S, hq, hkv, hd, stream=None):
@@ -385,6 +445,11 @@ def k_cross_entropy(logits, T, V, targets, inv_T, loss_rows, dlogits, stream=Non
 def k_lora_skinny(X, ldx, T, K, Bop, ldb, b_mn, KP, s, Us, stream=None):
     _check(lib().lst_k_lora_skinny(_ptr(X), ldx, T, K, _ptr(Bop), ldb, b_mn, KP, s, _ptr(Us), _stream(stream)),
            what="lst_k_lora_skinny")
+
+
+def k_lora_skinny_split(X, ldx, T, K, Bop, ldb, b_mn, R, RS, KP, s, Us, stream=None):
+    _check(lib().lst_k_lora_skinny_split(_ptr(X), ldx, T, K, _ptr(Bop), ldb, b_mn, R, RS, KP, s, _ptr(Us),
+                                         _stream(stream)), what="lst_k_lora_skinny_split")
 
 
 def k_lora_grads(X, ldx, in_f, dY, ldy, out_f, T, Us, Vs, KP, r, bounds, dA, dB, stream=None):

@@ -13,6 +13,8 @@
 #include "attention.cuh"
 #include "common.cuh"
 
+#include <cuda_fp16.h>
+
 namespace lst {
 namespace {
 
@@ -22,6 +24,15 @@ constexpr int kMaxGroup = 8;  // query heads per kv head: the dK/dV cluster size
 __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// The same shape with fp16 operands: the forward's P V product, where P in [0, 1] keeps 3 more
+// mantissa bits in fp16 than in bf16 and V converts to fp16 without loss (see k_attn_fwd).
+__device__ __forceinline__ void mma16816_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -40,6 +51,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 
 // Shared tile of `rows` x HD bf16 with a 16-byte row pad (conflict-free ldmatrix).
 template <int HD>
@@ -84,6 +100,27 @@ __device__ __forceinline__ void load_tile_async(__nv_bfloat16* sm, const __nv_bf
     const int r = i / V, c = (i % V) * 8;
     const bool in = r0 + r < S;
     cp_async16(sm + r * Tile<HD>::LD + c, in ? g + (tok0 + r0 + r) * ld + col + c : g, in);
+  }
+}
+
+// Rewrite, in place, the 16-byte chunks of a shared bf16 tile that this thread loaded with
+// load_tile_async (same chunk assignment) as fp16. Every bf16 value of magnitude in
+// [2^-14, 65504] is an fp16 value, so the attention's V (|v| of order 1) converts exactly; smaller
+// ones lose at most 2^-25 in absolute terms. Call after the thread's cp_async_wait_all and before
+// the barrier that publishes the tile.
+template <int HD>
+__device__ __forceinline__ void tile_to_f16(__nv_bfloat16* sm, int nrows) {
+  constexpr int V = HD / 8;
+  for (int i = threadIdx.x; i < nrows * V; i += blockDim.x) {
+    uint4* p = reinterpret_cast<uint4*>(sm + (i / V) * Tile<HD>::LD + (i % V) * 8);
+    uint4 u = *p;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+      w[j] = pack_f16(f.x, f.y);
+    }
+    *p = u;
   }
 }
 
@@ -146,7 +183,9 @@ __device__ __forceinline__ void store_grad_rows(__nv_bfloat16* dst, const float 
 
 // ------------------------------------------------------------------------------------ forward
 // grid (hq, B, ceil(S/64)), 128 threads; the last query block (most keys) is scheduled first;
-// warp w owns query rows 16w..16w+15 of the block. K/V tiles of 64 keys, double-buffered.
+// warp w owns query rows 16w..16w+15 of the block. K/V tiles of 64 keys, double-buffered. The
+// unnormalised probabilities enter the P V product as fp16 (V tiles converted exactly to fp16 once
+// they land), which keeps the rounding of P 8x below bf16's.
 template <int HD>
 __global__ void __launch_bounds__(128) k_attn_fwd(AttnArgs p) {
   extern __shared__ __align__(16) uint8_t sm_raw[];
@@ -174,6 +213,7 @@ __global__ void __launch_bounds__(128) k_attn_fwd(AttnArgs p) {
   cp_async_commit();
   for (int kb = 0; kb < nkb; ++kb) {
     cp_async_wait_all();
+    tile_to_f16<HD>(Vbuf + (kb & 1) * TL, 64);  // this thread's chunks of V tile kb
     __syncthreads();  // tile kb is in; every warp is done with tile kb-1, whose buffer is refilled now
     if (kb + 1 < nkb) {
       const int nb = (kb + 1) & 1;
@@ -248,20 +288,20 @@ __global__ void __launch_bounds__(128) k_attn_fwd(AttnArgs p) {
       o[i][2] *= corr[1];
       o[i][3] *= corr[1];
     }
-    // o += P v
+    // o += P v (fp16 operands)
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {  // 16 keys per k-step
       uint32_t a[4];
-      a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-      a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-      a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+      a[0] = pack_f16(s[2 * kk][0], s[2 * kk][1]);
+      a[1] = pack_f16(s[2 * kk][2], s[2 * kk][3]);
+      a[2] = pack_f16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      a[3] = pack_f16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
 #pragma unroll
       for (int i = 0; i < HD / 8; i += 2) {
         uint32_t bb[4];
         ldb_trans<HD>(bb, Vs, kk * 16, i * 8);
-        mma16816(o[i], a, bb[0], bb[1]);
-        mma16816(o[i + 1], a, bb[2], bb[3]);
+        mma16816_f16(o[i], a, bb[0], bb[1]);
+        mma16816_f16(o[i + 1], a, bb[2], bb[3]);
       }
     }
   }

@@ -32,6 +32,7 @@
 
 #include <atomic>
 #include <cstdio>
+#include <dlfcn.h>
 #include <nvtx3/nvToolsExt.h>
 #include <chrono>
 #include <cmath>
@@ -86,7 +87,9 @@ struct Group {
   int proj[3] = {0, 0, 0};
   int in = 0, out = 0;
   int bounds[4] = {0, 0, 0, 0};
-  int R = 0, KP = 0;
+  // LoRA side path: R = nseg * r adapter ranks; the split operands hold sections [hi | hi | lo] of
+  // RS = round_up(R, 8) each, padded to KP = round_up(3 RS, 64) (the GEMMs' extra K block)
+  int R = 0, RS = 0, KP = 0;
   int64_t woff = 0;  // element offset of the group's W in the concatenated bf16 weights
 };
 
@@ -193,6 +196,53 @@ bool is_device_ptr(const void* p) {
   return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
 }
 
+// ------------------------------------------------------------------------- NCCL, loaded on demand
+// The split-copy mode (lst_set_split_copy) all-gathers each layer blob over NVLink with NCCL. The
+// library does not link NCCL: the few entry points it uses are looked up in libnccl.so.2 the first
+// time the mode is switched on (the copy a process already loaded, e.g. torch's, is found first).
+// Declarations follow NCCL's public API (nccl.h); ncclUniqueId is 128 opaque bytes.
+struct NcclUid {
+  char internal[128];
+};
+typedef struct NcclComm* NcclCommT;
+enum { kNcclUint8 = 1 };  // ncclUint8 in nccl.h's ncclDataType_t
+struct NcclApi {
+  bool ok = false;
+  int (*get_unique_id)(NcclUid*) = nullptr;
+  int (*comm_init_rank)(NcclCommT*, int, NcclUid, int) = nullptr;
+  int (*all_gather)(const void*, void*, size_t, int, NcclCommT, cudaStream_t) = nullptr;
+  int (*comm_destroy)(NcclCommT) = nullptr;
+  const char* (*error_string)(int) = nullptr;
+};
+const NcclApi& nccl() {
+  static NcclApi api = [] {
+    NcclApi a;
+    void* h = dlopen("libnccl.so.2", RTLD_NOW | RTLD_GLOBAL);
+    if (!h) h = dlopen("libnccl.so", RTLD_NOW | RTLD_GLOBAL);
+    if (!h) return a;
+    a.get_unique_id = reinterpret_cast<int (*)(NcclUid*)>(dlsym(h, "ncclGetUniqueId"));
+    a.comm_init_rank = reinterpret_cast<int (*)(NcclCommT*, int, NcclUid, int)>(dlsym(h, "ncclCommInitRank"));
+    a.all_gather = reinterpret_cast<int (*)(const void*, void*, size_t, int, NcclCommT, cudaStream_t)>(
+        dlsym(h, "ncclAllGather"));
+    a.comm_destroy = reinterpret_cast<int (*)(NcclCommT)>(dlsym(h, "ncclCommDestroy"));
+    a.error_string = reinterpret_cast<const char* (*)(int)>(dlsym(h, "ncclGetErrorString"));
+    a.ok = a.get_unique_id && a.comm_init_rank && a.all_gather && a.comm_destroy && a.error_string;
+    return a;
+  }();
+  return api;
+}
+
+// The slice of a blob of `blob` bytes that rank `rank` of `world` copies in split-copy mode: every
+// rank contributes `count` bytes (a multiple of 256) to an all-gather of world * count bytes;
+// rank r's part is [r * count, r * count + count) clipped to the blob (possibly empty).
+void split_plan(int64_t blob, int world, int rank, int64_t* off, int64_t* bytes, int64_t* count) {
+  const int64_t c = ((blob + (int64_t)world * 256 - 1) / ((int64_t)world * 256)) * 256;
+  const int64_t o = (int64_t)rank * c;
+  *count = c;
+  *off = o;
+  *bytes = o >= blob ? 0 : std::min(c, blob - o);
+}
+
 // Profiling classes
 enum { PC_GEMM = 0, PC_ATTN = 1, PC_DEQ = 2, PC_OTHER = 3, PC_COPY = 4, PC_LORA = 5, PC_N = 6 };
 
@@ -238,6 +288,14 @@ struct lst_ctx {
     return e && e[0] && std::strcmp(e, "0") != 0;
   }();
   float* grads_host = nullptr;         // pinned host destination of this step's gradients (or null)
+  // split-copy mode: this rank copies its slice of each blob, NCCL all-gathers the rest (world > 1)
+  int split_world = 1, split_rank = 0;
+  NcclCommT nccl_comm = nullptr;
+  int64_t pool_bytes = 0;               // bytes of each pool slot before its guard
+  // NF4 base: where the weights are dequantised -- 0: a separate pass into a bf16 scratch, one read
+  // ahead on the prep stream; 1: inside the GEMMs, for every group whose rows are whole NF4 blocks
+  int deq_mode = 0;
+  bool fuse_ok[NGROUP] = {false, false, false, false};
   cudaEvent_t ev_d2h = nullptr;
   bool own_stream = false;
   std::string err;
@@ -261,8 +319,8 @@ struct lst_ctx {
   int64_t lora_numel = 0;
   std::vector<int64_t> offA, offB;
   struct Derived {                 // bf16 operands of the LoRA side path, per fused group
-    __nv_bfloat16* Acat16 = nullptr;  // [KP, in]
-    __nv_bfloat16* Bexp16 = nullptr;  // [out, KP]
+    __nv_bfloat16* Acat16 = nullptr;  // [KP, in], split rows (hi, hi, lo)
+    __nv_bfloat16* Bexp16 = nullptr;  // [out, KP], split columns (hi, hi, lo)
   };
   std::vector<Derived> der;  // L * NGROUP
   float* grads = nullptr;
@@ -273,8 +331,8 @@ struct lst_ctx {
                 *wscr[2] = {nullptr, nullptr};
   float *rstd1 = nullptr, *rstd2 = nullptr, *lse = nullptr, *Dbuf = nullptr;
   float* o32 = nullptr;  // attention output before rounding (recompute pass), for the backward's D
-  __nv_bfloat16* Us[NGROUP] = {};  // bf16(s * x A^T) per group [T, KP]
-  __nv_bfloat16* Vs[NGROUP] = {};  // bf16(s * dy B) per group [T, KP]
+  __nv_bfloat16* Us[NGROUP] = {};  // split bf16 s * x A^T per group [T, KP] (sections hi, lo, hi)
+  __nv_bfloat16* Vs[NGROUP] = {};  // split bf16 s * dy B per group [T, KP]
   float *ga = nullptr, *gb = nullptr, *dn = nullptr, *dm = nullptr;
   __nv_bfloat16 *dout_b = nullptr, *dh_b = nullptr, *do_b = nullptr, *dqkvb = nullptr, *dgu = nullptr;
   __nv_bfloat16* nf = nullptr;
@@ -339,6 +397,13 @@ struct lst_ctx {
   std::vector<ProfRec> prof_recs;
   cudaEvent_t prof_step0 = nullptr, prof_step1 = nullptr;
   int64_t launches_at_step_start = 0;
+  // per-read timeline of the last profiled step: events [read][TL_N] and the times they gave (ms
+  // from the step's start; -1: the read had no copy / dequant of its own)
+  enum { TL_COPY0 = 0, TL_COPY1, TL_DEQ0, TL_DEQ1, TL_COMP0, TL_COMP1, TL_N };
+  std::vector<cudaEvent_t> tl_ev;
+  std::vector<char> tl_set;
+  std::vector<float> tl_ms;
+  int tl_reads = 0;
 };
 
 namespace {
@@ -432,6 +497,16 @@ struct ProfScope {
   }
 };
 
+// Timeline event `which` of read n on stream st (profiling only).
+lst_status tl_record(lst_ctx* c, int n, int which, cudaStream_t st) {
+  if (!c->profiling) return LST_OK;
+  const size_t i = (size_t)n * lst_ctx::TL_N + which;
+  if (i >= c->tl_ev.size()) return LST_OK;
+  CK(cudaEventRecord(c->tl_ev[i], st));
+  c->tl_set[i] = 1;
+  return LST_OK;
+}
+
 // ------------------------------------------------------------------------- LoRA operands
 lst_status prep_lora(lst_ctx* c, int layer) {
   for (int g = 0; g < NGROUP; ++g) {
@@ -446,6 +521,7 @@ lst_status prep_lora(lst_ctx* c, int layer) {
     a.r = c->r;
     a.in = G.in;
     for (int k = 0; k <= G.nseg; ++k) a.bounds[k] = G.bounds[k];
+    a.RS = G.RS;
     a.KP = G.KP;
     a.Acat16 = D.Acat16;
     a.Bexp16 = D.Bexp16;
@@ -454,18 +530,41 @@ lst_status prep_lora(lst_ctx* c, int layer) {
   return LST_OK;
 }
 
+// True when group g's GEMMs dequantise the NF4 blob themselves in the current mode.
+bool fused_group(const lst_ctx* c, int g) { return c->deq_mode == 1 && c->fuse_ok[g]; }
+
+// The NF4 tensors of group g in a blob, stacked along the output rows as the GEMMs see them.
+Nf4Mat group_nf4(const lst_ctx* c, const uint8_t* blob, int g) {
+  static const int first[NCHUNK + 1] = {0, 3, 4, 6, 7};
+  Nf4Mat q;
+  q.nseg = first[g + 1] - first[g];
+  q.cols = c->grp[g].in;
+  int rows = 0;
+  for (int k = 0; k < q.nseg; ++k) {
+    const int p = first[g] + k;
+    rows += (int)c->lay.outd[p];
+    q.row_end[k] = rows;
+    q.packed[k] = blob + c->lay.packed[p];
+    q.qabs[k] = reinterpret_cast<const int8_t*>(blob + c->lay.qabs[p]);
+    q.gscale[k] = reinterpret_cast<const float*>(blob + c->lay.gscale[p]);
+    q.mean[k] = reinterpret_cast<const float*>(blob + c->lay.means) + p;
+  }
+  nf4_codebook(q.cb);
+  return q;
+}
+
 // ------------------------------------------------------------------------- layer compute
 const __nv_bfloat16* group_w(lst_ctx* c, const __nv_bfloat16* W, int g) { return W + c->grp[g].woff; }
 
-lst_status group_fwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const __nv_bfloat16* X, int64_t ldx,
-                     void* Y, int64_t ldy, int y_f32, const float* bias, const float* resid, bool gemm) {
+lst_status group_fwd(lst_ctx* c, int layer, int g, const uint8_t* blob, const __nv_bfloat16* W, const __nv_bfloat16* X,
+                     int64_t ldx, void* Y, int64_t ldy, int y_f32, const float* bias, const float* resid, bool gemm) {
   const Group& G = c->grp[g];
   const auto& D = c->der[layer * NGROUP + g];
   const int64_t T = c->curT;
   const bool lora = !c->adapters_off;
   if (lora) {
-    ProfScope ps(c, c->stream, PC_LORA);  // Us = bf16(s * X Acat^T)
-    CK(lora_skinny(X, ldx, T, G.in, D.Acat16, G.in, 0, G.KP, c->s, c->Us[g], c->stream));
+    ProfScope ps(c, c->stream, PC_LORA);  // Us = split(s * X Acat^T)
+    CK(lora_skinny_split(X, ldx, T, G.in, D.Acat16, G.in, 0, G.R, G.RS, G.KP, c->s, c->Us[g], c->stream));
   }
   if (!gemm) return LST_OK;
   GemmArgs a;
@@ -477,6 +576,11 @@ lst_status group_fwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
   a.B = group_w(c, W, g);
   a.ldb = G.in;
   a.b_mn = 0;
+  Nf4Mat q;
+  if (fused_group(c, g)) {
+    q = group_nf4(c, blob, g);
+    a.Bq = &q;
+  }
   if (lora) {
     a.A2 = c->Us[g];
     a.lda2 = G.KP;
@@ -502,14 +606,14 @@ lst_status group_fwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
   return LST_OK;
 }
 
-lst_status group_bwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const __nv_bfloat16* dY, int64_t ldy,
-                     const __nv_bfloat16* X, int64_t ldx, void* dX, int dx_f32) {
+lst_status group_bwd(lst_ctx* c, int layer, int g, const uint8_t* blob, const __nv_bfloat16* W, const __nv_bfloat16* dY,
+                     int64_t ldy, const __nv_bfloat16* X, int64_t ldx, void* dX, int dx_f32) {
   const Group& G = c->grp[g];
   const auto& D = c->der[layer * NGROUP + g];
   const int64_t T = c->curT;
   {
-    ProfScope ps(c, c->stream, PC_LORA);  // Vs = bf16(s * dY Bexp)
-    CK(lora_skinny(dY, ldy, T, G.out, D.Bexp16, G.KP, 1, G.KP, c->s, c->Vs[g], c->stream));
+    ProfScope ps(c, c->stream, PC_LORA);  // Vs = split(s * dY Bexp)
+    CK(lora_skinny_split(dY, ldy, T, G.out, D.Bexp16, G.KP, 1, G.R, G.RS, G.KP, c->s, c->Vs[g], c->stream));
   }
   {
     GemmArgs a;
@@ -521,6 +625,11 @@ lst_status group_bwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
     a.B = group_w(c, W, g);
     a.ldb = G.in;
     a.b_mn = 1;
+    Nf4Mat q;
+    if (fused_group(c, g)) {
+      q = group_nf4(c, blob, g);
+      a.Bq = &q;
+    }
     a.A2 = c->Vs[g];
     a.lda2 = G.KP;
     a.B2 = D.Acat16;
@@ -539,7 +648,8 @@ lst_status group_bwd(lst_ctx* c, int layer, int g, const __nv_bfloat16* W, const
     dA[k] = c->grads + c->offA[layer * NPROJ + G.proj[k]];
     dB[k] = c->grads + c->offB[layer * NPROJ + G.proj[k]];
   }
-  // dA = s V^T X and dB = s dY^T U, with s folded into Vs and Us
+  // dA = s V^T X and dB = s dY^T U, with s folded into Vs and Us (their hi sections: the gradients are
+  // fp32 reductions of bf16 products, so the lo parts would only refine the last bits of V and U)
   CK(lora_grad_a(X, ldx, T, G.in, c->Vs[g], G.KP, G.nseg, c->r, dA, c->stream));
   CK(lora_grad_b(dY, ldy, T, G.out, c->Us[g], G.KP, G.nseg, c->r, G.bounds, dB, c->stream));
   return LST_OK;
@@ -589,7 +699,7 @@ lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(rmsnorm_fwd(x, g1, T, c->d, c->cfg.rms_eps, c->n1, c->rstd1, c->stream));
   }
-  TRY(group_fwd(c, i, G_QKV, W, c->n1, c->d, c->qkv, c->dqkv, 0, bias, nullptr, true));
+  TRY(group_fwd(c, i, G_QKV, blob, W, c->n1, c->d, c->qkv, c->dqkv, 0, bias, nullptr, true));
   {
     AttnArgs a;
     a.q = c->qkv;
@@ -610,21 +720,21 @@ lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
     CK(attention_fwd(a, c->stream));
   }
   TRY(wait_chunk(c, 1));
-  TRY(group_fwd(c, i, G_O, W, c->o, c->dq, c->h, c->d, 1, nullptr, x, true));
+  TRY(group_fwd(c, i, G_O, blob, W, c->o, c->dq, c->h, c->d, 1, nullptr, x, true));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(rmsnorm_fwd(c->h, g2, T, c->d, c->cfg.rms_eps, c->n2, c->rstd2, c->stream));
   }
   TRY(wait_chunk(c, 2));
-  TRY(group_fwd(c, i, G_GU, W, c->n2, c->d, c->gu, 2 * c->F, 0, nullptr, nullptr, true));
+  TRY(group_fwd(c, i, G_GU, blob, W, c->n2, c->d, c->gu, 2 * c->F, 0, nullptr, nullptr, true));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(swiglu_fwd(c->gu, T, c->F, c->m, c->stream));
   }
   TRY(wait_chunk(c, 3));  // also before a recompute: the backward that follows needs W_down
   // the recompute pass needs only the LoRA projection of m (for dB of down), not the output
-  TRY(group_fwd(c, i, G_DOWN, W, c->m, c->F, c->xs + (int64_t)(i + 1) * c->Tmax * c->d, c->d, 1, nullptr, c->h,
-                !recompute));
+  TRY(group_fwd(c, i, G_DOWN, blob, W, c->m, c->F, c->xs + (int64_t)(i + 1) * c->Tmax * c->d, c->d, 1, nullptr,
+                c->h, !recompute));
   return LST_OK;
 }
 
@@ -635,17 +745,17 @@ lst_status layer_bwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
   const float* g1 = reinterpret_cast<const float*>(blob + c->lay.norms);
   const float* g2 = g1 + c->d;
   const float* x = c->xs + (int64_t)i * c->Tmax * c->d;
-  TRY(group_bwd(c, i, G_DOWN, W, c->dout_b, c->d, c->m, c->F, c->dm, 1));
+  TRY(group_bwd(c, i, G_DOWN, blob, W, c->dout_b, c->d, c->m, c->F, c->dm, 1));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(swiglu_bwd(c->dm, c->gu, T, c->F, c->dgu, c->stream));
   }
-  TRY(group_bwd(c, i, G_GU, W, c->dgu, 2 * c->F, c->n2, c->d, c->dn, 1));
+  TRY(group_bwd(c, i, G_GU, blob, W, c->dgu, 2 * c->F, c->n2, c->d, c->dn, 1));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(rmsnorm_bwd(c->dn, c->h, g2, c->rstd2, c->ga, T, c->d, c->gb, c->dh_b, c->stream));
   }
-  TRY(group_bwd(c, i, G_O, W, c->dh_b, c->d, c->o, c->dq, c->do_b, 0));
+  TRY(group_bwd(c, i, G_O, blob, W, c->dh_b, c->d, c->o, c->dq, c->do_b, 0));
   {
     AttnBwdArgs a;
     a.q = c->qkv;
@@ -674,7 +784,7 @@ lst_status layer_bwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
     ProfScope ps(c, c->stream, PC_ATTN);
     CK(attention_bwd(a, c->stream));
   }
-  TRY(group_bwd(c, i, G_QKV, W, c->dqkvb, c->dqkv, c->n1, c->d, c->dn, 1));
+  TRY(group_bwd(c, i, G_QKV, blob, W, c->dqkvb, c->dqkv, c->n1, c->d, c->dn, 1));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(rmsnorm_bwd(c->dn, x, g1, c->rstd1, c->gb, T, c->d, c->ga, c->dout_b, c->stream));
@@ -906,12 +1016,30 @@ lst_status enqueue_copy(lst_ctx* c, int n) {
   if (c->faults.fail_memcpy()) return fail(c, LST_ERR_CUDA, "layer copy enqueue failed (injected)");
   if (p.wait_free >= 0) CK(cudaStreamWaitEvent(c->copy_stream, c->ev_free[p.wait_free], 0));
   ProfScope ps(c, c->copy_stream, PC_COPY);
+  TRY(tl_record(c, n, lst_ctx::TL_COPY0, c->copy_stream));
   const uint8_t* src = c->arena + (int64_t)j * c->lay.total;
+  if (c->split_world > 1) {
+    // this rank's slice over its own link, then the whole blob from every rank's slice over
+    // NVLink (in-place all-gather into the pool slot); the blob is complete for every chunk at once
+    int64_t off = 0, bytes = 0, count = 0;
+    split_plan(c->lay.total, c->split_world, c->split_rank, &off, &bytes, &count);
+    if (bytes > 0)
+      CK(cudaMemcpyAsync(c->pool[p.slot] + off, src + off, bytes, cudaMemcpyHostToDevice, c->copy_stream));
+    const int r = nccl().all_gather(c->pool[p.slot] + off, c->pool[p.slot], (size_t)count, kNcclUint8, c->nccl_comm,
+                                    c->copy_stream);
+    if (r != 0) return fail(c, LST_ERR_CUDA, std::string("ncclAllGather: ") + nccl().error_string(r));
+    for (int g = 0; g < NCHUNK; ++g) CK(cudaEventRecord(c->ev_chunk[n * NCHUNK + g], c->copy_stream));
+    TRY(tl_record(c, n, lst_ctx::TL_COPY1, c->copy_stream));
+    c->st.layer_reads_last_step += 1;
+    c->st.h2d_bytes_last_step += bytes;
+    return LST_OK;
+  }
   for (int g = 0; g < NCHUNK; ++g) {  // group by group, so compute can start on the first group
     CK(cudaMemcpyAsync(c->pool[p.slot] + c->lay.chunk[g], src + c->lay.chunk[g], c->lay.chunk[g + 1] - c->lay.chunk[g],
                        cudaMemcpyHostToDevice, c->copy_stream));
     CK(cudaEventRecord(c->ev_chunk[n * NCHUNK + g], c->copy_stream));
   }
+  TRY(tl_record(c, n, lst_ctx::TL_COPY1, c->copy_stream));
   c->st.layer_reads_last_step += 1;
   c->st.h2d_bytes_last_step += c->lay.total;
   return LST_OK;
@@ -991,12 +1119,17 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
     if (m >= R || !c->plan[m].deq) return LST_OK;
     const ReadPlan& p = c->plan[m];
     if (p.wwait >= 0) CK(cudaStreamWaitEvent(c->prep_stream, c->ev_free[p.wwait], 0));
+    bool started = false;
     for (int g = 0; g < NCHUNK; ++g) {
+      if (fused_group(c, g)) continue;  // dequantised inside the GEMMs
       if (streamed && p.loaded_by >= 0)
         CK(cudaStreamWaitEvent(c->prep_stream, c->ev_chunk[p.loaded_by * NCHUNK + g], 0));
+      if (!started) TRY(tl_record(c, m, lst_ctx::TL_DEQ0, c->prep_stream));
+      started = true;
       TRY(dequant_chunk(c, blob_of(m), c->wscr[p.wslot], g, c->prep_stream));
       CK(cudaEventRecord(c->ev_deqg[m * NCHUNK + g], c->prep_stream));
     }
+    if (started) TRY(tl_record(c, m, lst_ctx::TL_DEQ1, c->prep_stream));
     return LST_OK;
   };
   TRY(enqueue_deq(0));
@@ -1013,10 +1146,15 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
     // scratch may have been filled by different reads when layers are reused)
     for (int g = 0; g < NCHUNK; ++g) {
       c->cur_wait[g][0] = streamed && p.loaded_by >= 0 ? c->ev_chunk[p.loaded_by * NCHUNK + g] : nullptr;
-      c->cur_wait[g][1] = nf4 && p.wfilled_by >= 0 ? c->ev_deqg[p.wfilled_by * NCHUNK + g] : nullptr;
+      c->cur_wait[g][1] =
+          nf4 && p.wfilled_by >= 0 && !fused_group(c, g) ? c->ev_deqg[p.wfilled_by * NCHUNK + g] : nullptr;
     }
     const __nv_bfloat16* W =
         nf4 ? c->wscr[p.wslot] : reinterpret_cast<const __nv_bfloat16*>(blob + c->lay.w16);
+    if (c->profiling) {  // the read's compute starts once its first weight group is in place
+      TRY(wait_chunk(c, 0));
+      TRY(tl_record(c, n, lst_ctx::TL_COMP0, c->stream));
+    }
     if (kind == RD_REF) {
       c->adapters_off = true;
       const lst_status st = layer_fwd(c, j, blob, W, false);
@@ -1029,6 +1167,7 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
       TRY(layer_bwd(c, j, blob, W));
     }
     CK(cudaEventRecord(c->ev_free[n], c->stream));
+    TRY(tl_record(c, n, lst_ctx::TL_COMP1, c->stream));
     if (kind == RD_BWD && c->grads_host) {
       // this layer's gradients are final: send them while the layers below compute
       const int64_t o0 = c->offA[j * NPROJ], o1 = j + 1 < L ? c->offA[(j + 1) * NPROJ] : c->lora_numel;
@@ -1109,6 +1248,13 @@ lst_status finish_step(lst_ctx* c, float* loss, float* grads_out) {
     c->st.lora_launches = cnt[PC_LORA];
     c->st.gemm_flops = flops;
     c->st.step_ms = step;
+    c->tl_reads = (int)c->rd_layer.size();
+    c->tl_ms.assign((size_t)c->tl_reads * lst_ctx::TL_N, -1.f);
+    for (size_t i = 0; i < c->tl_ms.size(); ++i) {
+      float t = -1.f;
+      if (c->tl_set[i] && cudaEventElapsedTime(&t, c->prof_step0, c->tl_ev[i]) == cudaSuccess) c->tl_ms[i] = t;
+    }
+    cudaGetLastError();
   }
   return LST_OK;
 }
@@ -1129,6 +1275,15 @@ lst_status begin_step(lst_ctx* c, int32_t batch, int32_t seq) {
   c->st.h2d_bytes_last_step = 0;
   c->prof_used = 0;
   c->prof_recs.clear();
+  if (c->profiling) {
+    const size_t need = (size_t)3 * c->L * lst_ctx::TL_N;
+    while (c->tl_ev.size() < need) {
+      cudaEvent_t e;
+      CK(cudaEventCreate(&e));
+      c->tl_ev.push_back(e);
+    }
+    c->tl_set.assign(need, 0);
+  }
   c->launches_at_step_start = g_launch_count.load();
   if (c->profiling) CK(cudaEventRecord(c->prof_step0, c->stream));
   return LST_OK;
@@ -1181,8 +1336,6 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   c->dqkv = c->dq + 2 * c->dkv;
   c->Tmax = (int64_t)k.max_batch * k.max_seq;
   c->lay = make_layout(k);
-  const int R3 = 3 * c->r;
-  const int KP = ((R3 + 63) / 64) * 64;
   auto setg = [&](int g, int nseg, std::initializer_list<int> pr, int in, std::initializer_list<int> bnd) {
     Group& G = c->grp[g];
     G.nseg = nseg;
@@ -1193,13 +1346,15 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
     for (int b : bnd) G.bounds[i++] = b;
     G.out = G.bounds[nseg];
     G.R = nseg * c->r;
-    G.KP = KP;
+    G.RS = (G.R + 7) / 8 * 8;
+    G.KP = (3 * G.RS + 63) / 64 * 64;
     G.woff = c->lay.woff[G.proj[0]];
   };
   setg(G_QKV, 3, {0, 1, 2}, c->d, {0, (int)c->dq, (int)(c->dq + c->dkv), (int)c->dqkv});
   setg(G_O, 1, {3}, (int)c->dq, {0, c->d});
   setg(G_GU, 2, {4, 5}, c->d, {0, c->F, 2 * c->F});
   setg(G_DOWN, 1, {6}, c->F, {0, c->d});
+  for (int g = 0; g < NGROUP; ++g) c->fuse_ok[g] = k.base_format == LST_BASE_NF4 && c->grp[g].in % 64 == 0;
 
   int prio_low = 0, prio_high = 0;
   CK(cudaDeviceGetStreamPriorityRange(&prio_low, &prio_high));
@@ -1245,10 +1400,11 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
         const auto& D = c->der[l * NGROUP + g];
         for (int k = 0; k < G.nseg; ++k) {
           const int p = G.proj[k];
-          AdamTensor a{c->offA[l * NPROJ + p], (int64_t)c->r * G.in, c->r, G.in, D.Acat16, G.in, k * c->r, 0};
+          AdamTensor a{c->offA[l * NPROJ + p], (int64_t)c->r * G.in, c->r, G.in, D.Acat16, G.in, k * c->r, 0,
+                       (int64_t)G.RS * G.in};
           const int outp = G.bounds[k + 1] - G.bounds[k];
           AdamTensor b{c->offB[l * NPROJ + p], (int64_t)outp * c->r, outp, c->r, D.Bexp16, G.KP, G.bounds[k],
-                       k * c->r};
+                       k * c->r, (int64_t)G.RS};
           tab.push_back(a);
           tab.push_back(b);
           c->opt_maxn = std::max(c->opt_maxn, std::max(a.n, b.n));
@@ -1271,6 +1427,7 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
     TRY(dalloc(c, &c->pool[1], blob + kGuardBytes));
     TRY(add_guard(c, c->pool[0] + blob));
     TRY(add_guard(c, c->pool[1] + blob));
+    c->pool_bytes = blob;
     c->st.arena_bytes = blob * c->L;
   } else {
     TRY(dalloc(c, &c->resident, blob * c->L));
@@ -1366,6 +1523,11 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
 
 void free_all(lst_ctx* c) {
   if (c->stream) cudaStreamSynchronize(c->stream);
+  if (c->nccl_comm) {
+    if (c->copy_stream) cudaStreamSynchronize(c->copy_stream);
+    nccl().comm_destroy(c->nccl_comm);
+    c->nccl_comm = nullptr;
+  }
   if (c->copy_stream) cudaStreamSynchronize(c->copy_stream);
   if (c->prep_stream) cudaStreamSynchronize(c->prep_stream);
   if (c->d2h_stream) cudaStreamSynchronize(c->d2h_stream);
@@ -1381,6 +1543,7 @@ void free_all(lst_ctx* c) {
   for (auto e : c->ev_free) cudaEventDestroy(e);
   for (auto e : c->ev_deqg) cudaEventDestroy(e);
   for (auto e : c->prof_pool) cudaEventDestroy(e);
+  for (auto e : c->tl_ev) cudaEventDestroy(e);
   if (c->ev_done) cudaEventDestroy(c->ev_done);
   if (c->ev_start) cudaEventDestroy(c->ev_start);
   if (c->ev_d2h) cudaEventDestroy(c->ev_d2h);
@@ -1755,6 +1918,72 @@ lst_status lst_set_profiling(lst_ctx* c, int32_t on) {
   return LST_OK;
 }
 
+lst_status lst_split_plan(int64_t blob_bytes, int32_t world, int32_t rank, int64_t* offset, int64_t* bytes,
+                          int64_t* count) {
+  if (blob_bytes <= 0 || world < 1 || rank < 0 || rank >= world || !offset || !bytes || !count) return LST_ERR_ARG;
+  split_plan(blob_bytes, world, rank, offset, bytes, count);
+  return LST_OK;
+}
+
+lst_status lst_nccl_unique_id(void* out) {
+  if (!out) return LST_ERR_ARG;
+  if (!nccl().ok) return LST_ERR_STATE;
+  NcclUid id;
+  if (nccl().get_unique_id(&id) != 0) return LST_ERR_CUDA;
+  std::memcpy(out, &id, sizeof(id));
+  return LST_OK;
+}
+
+lst_status lst_set_split_copy(lst_ctx* c, int32_t rank, int32_t world, const void* unique_id) {
+  if (!c) return LST_ERR_ARG;
+  DeviceScope ds(c);
+  if (world < 1 || rank < 0 || rank >= world || (world > 1 && !unique_id))
+    return fail(c, LST_ERR_ARG, "bad rank / world or null unique id");
+  if (!c->cfg.streamed) return fail(c, LST_ERR_STATE, "split copies need a streamed context");
+  if (c->nccl_comm) return fail(c, LST_ERR_STATE, "split copies are already set");
+  if (world == 1) return LST_OK;
+  if (!nccl().ok) return fail(c, LST_ERR_STATE, "libnccl.so.2 could not be loaded");
+  int64_t off = 0, bytes = 0, count = 0;
+  split_plan(c->lay.total, world, rank, &off, &bytes, &count);
+  if (world * count > c->pool_bytes) {
+    // the all-gather fills world * count bytes: grow both slots (new guards after them)
+    CK(cudaStreamSynchronize(c->stream));
+    CK(cudaStreamSynchronize(c->copy_stream));
+    for (int k = 0; k < 2; ++k) {
+      uint8_t* q = nullptr;
+      TRY(dalloc(c, &q, world * count + kGuardBytes));
+      TRY(add_guard(c, q + world * count));
+      c->pool[k] = q;  // the old slot stays in dev_allocs and is freed with the context
+    }
+    c->pool_bytes = world * count;
+    c->slot_layer[0] = c->slot_layer[1] = -1;
+  }
+  NcclUid id;
+  std::memcpy(&id, unique_id, sizeof(id));
+  NcclCommT comm = nullptr;
+  const int r = nccl().comm_init_rank(&comm, world, id, rank);
+  if (r != 0) return fail(c, LST_ERR_CUDA, std::string("ncclCommInitRank: ") + nccl().error_string(r));
+  c->nccl_comm = comm;
+  c->split_world = world;
+  c->split_rank = rank;
+  return LST_OK;
+}
+
+lst_status lst_get_read_timeline(const lst_ctx* c, float* out, int32_t max_reads, int32_t* n_reads) {
+  if (!c || !n_reads) return LST_ERR_ARG;
+  *n_reads = c->tl_reads;
+  if (c->tl_reads == 0) return LST_ERR_STATE;
+  if (!out || max_reads < c->tl_reads) return LST_ERR_ARG;
+  for (int n = 0; n < c->tl_reads; ++n) {
+    const int j = c->rd_layer[n], kind = c->rd_kind[n];
+    float* row = out + (int64_t)n * 8;
+    row[0] = (float)j;
+    row[1] = (float)kind;
+    for (int k = 0; k < lst_ctx::TL_N; ++k) row[2 + k] = c->tl_ms[(size_t)n * lst_ctx::TL_N + k];
+  }
+  return LST_OK;
+}
+
 lst_status lst_plan_reads(const int32_t* reads, int32_t n_reads, int32_t reuse, int32_t nf4, int32_t* held,
                           int32_t* wheld, int32_t* out) {
   if (!reads || n_reads <= 0 || !held || !wheld || !out) return LST_ERR_ARG;
@@ -1774,6 +2003,16 @@ lst_status lst_plan_reads(const int32_t* reads, int32_t n_reads, int32_t reuse, 
   held[1] = h[1];
   wheld[0] = w[0];
   wheld[1] = w[1];
+  return LST_OK;
+}
+
+lst_status lst_set_dequant_mode(lst_ctx* c, int32_t mode) {
+  if (!c) return LST_ERR_ARG;
+  if (mode != 0 && mode != 1) return fail(c, LST_ERR_ARG, "dequant mode must be 0 or 1");
+  if (mode != c->deq_mode) {
+    c->deq_mode = mode;
+    c->w_layer[0] = c->w_layer[1] = -1;  // the scratches may lack the groups the GEMMs dequantised
+  }
   return LST_OK;
 }
 

@@ -330,6 +330,275 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// NF4-dequantising variant: the B operand is built in shared memory by dequantiser warps.
+//
+// Warp roles (320 threads): 0 TMA producer of A (and of the LoRA pair's A2 / B2), 1 MMA issuer,
+// 2-5 epilogue (as k_gemm), 6-9 dequantisers. For each K stage below nk1 the dequantisers read the
+// stage's NF4 blocks straight from global memory -- BN blocks of 64 codes, one per 128-byte row of
+// the stage's B tile -- and write bf16(code value x absmax) in the same 128-byte-swizzled layout a
+// TMA load of the bf16 matrix would produce, so the MMA descriptors are those of k_gemm. The
+// absmax is dequantised with the same fp32 operations as nf4.cu ((q * s) / 127 + mean), so the
+// operand equals the dequantised matrix bit for bit. Every generic-proxy write is fenced for the
+// async proxy before the writer arrives on the stage's bfull barrier (one arrival per thread).
+constexpr int kDqWarps = 4;
+constexpr int kDqThreads = kDqWarps * 32;
+
+template <int BN, int BMN>
+__device__ __forceinline__ void dq_stage(const Nf4Mat& q, const float* cbs, uint8_t* sBs, int n0, int kb, int N,
+                                         int K) {
+  constexpr int HPT = 2 * BN / kDqThreads;  // half blocks (32 codes) per thread and stage
+  const int dt = (int)threadIdx.x - 192;
+  const int kk = kb * 64;
+  uint4 raw[HPT];
+  float ahat[HPT];
+#pragma unroll
+  for (int j = 0; j < HPT; ++j) {
+    const int h = dt + kDqThreads * j;
+    const int bi = h >> 1, half = h & 1;
+    int wrow, wcol;  // W element (row, column) of the block's first code
+    bool ok;
+    if (BMN == 0) {  // B(n, k) = W[n][k]: tile row bi is W row n0 + bi, columns kk .. kk + 63
+      wrow = n0 + bi;
+      wcol = kk;
+      ok = wrow < N;
+    } else {         // B(k, n) = W[k][n]: sub-tile bi / 64, row bi % 64 is W row kk + bi % 64
+      wrow = kk + (bi & 63);
+      wcol = n0 + (bi >> 6) * 64;
+      ok = wrow < K && wcol < N;
+    }
+    raw[j] = make_uint4(0, 0, 0, 0);
+    ahat[j] = 0.f;
+    if (ok) {
+      int g = 0;
+      while (g + 1 < q.nseg && wrow >= q.row_end[g]) ++g;
+      const int r0 = g ? q.row_end[g - 1] : 0;
+      const int64_t b = (int64_t)(wrow - r0) * (q.cols >> 6) + (wcol >> 6);
+      raw[j] = __ldg(reinterpret_cast<const uint4*>(q.packed[g] + b * 32 + half * 16));
+      const float qs = __fmul_rn((float)q.qabs[g][b], q.gscale[g][b >> 8]);
+      ahat[j] = __fadd_rn(__fdiv_rn(qs, 127.0f), *q.mean[g]);
+    }
+  }
+  // (the caller has waited until the stage is free)
+#pragma unroll
+  for (int j = 0; j < HPT; ++j) {
+    const int h = dt + kDqThreads * j;
+    const int bi = h >> 1, half = h & 1;
+    const int row = BMN == 0 ? bi : (bi & 63);
+    uint8_t* rowp = sBs + (BMN == 0 ? bi * 128 : (bi >> 6) * (64 * 128) + (bi & 63) * 128);
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(&raw[j]);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {  // 16-byte chunk 4 * half + c of the row: codes 8c .. 8c + 7 of the half
+      uint4 o;
+      uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int by = 0; by < 4; ++by) {
+        const uint32_t v = (w[c] >> (8 * by)) & 0xffu;  // element 2 by in the high nibble
+        const float hi = __fmul_rn(cbs[v >> 4], ahat[j]);
+        const float lo = __fmul_rn(cbs[v & 15u], ahat[j]);
+        __nv_bfloat162 pr = __floats2bfloat162_rn(hi, lo);
+        op[by] = *reinterpret_cast<uint32_t*>(&pr);
+      }
+      const int chunk = (4 * half + c) ^ (row & 7);  // 128-byte swizzle
+      *reinterpret_cast<uint4*>(rowp + chunk * 16) = o;
+    }
+  }
+}
+
+template <int BN, int BMN>
+__global__ void __launch_bounds__(192 + kDqThreads, 1)
+k_gemm_nf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+           const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ Nf4Mat q, const Epi ep,
+           const TileSched sched, const int total_tiles, const int nk1, const int nk2, const int N, const int K) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* bfull = empty + C::STAGES;      // [STAGES] dequantised B tile written
+  uint64_t* acc_full = bfull + C::STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  float* cbs = reinterpret_cast<float*>(tmem_slot + 4);  // codebook [16]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&bfull[s], kDqThreads);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 16) cbs[threadIdx.x] = q.cb[threadIdx.x];
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    if (nk2) {
+      tma_prefetch_desc(&tmA2);
+      tma_prefetch_desc(&tmB2);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        int mi, ni;
+        sched.get(t, mi, ni);
+        const int m0 = mi * BM, n0 = ni * BN;
+        const int nk = nk1 + nk2;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1)) {
+            ok = false;
+            break;
+          }
+          if (kb < nk1) {  // A only; the dequantisers fill B
+            mbar_arrive_expect_tx(&full[s], C::A_BYTES);
+            tma_load_2d(sA + s * C::A_BYTES, &tmA, &full[s], kb * BK, m0);
+          } else {         // the LoRA pair, both by TMA
+            const int kk = (kb - nk1) * BK;
+            mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
+            tma_load_2d(sA + s * C::A_BYTES, &tmA2, &full[s], kk, m0);
+            if (BMN == 0) {
+              tma_load_2d(sB + s * C::B_BYTES, &tmB2, &full[s], kk, n0);
+            } else {
+#pragma unroll
+              for (int c = 0; c < BN / 64; ++c)
+                tma_load_2d(sB + s * C::B_BYTES + c * (64 * BK * 2), &tmB2, &full[s], n0 + c * 64, kk);
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(BM, BN, 0, BMN);
+      uint32_t it = 0, bph = 0;  // bph: bit s = parity of the next bfull[s] phase
+      bool ok = true;
+      int local = 0;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++local) {
+        const int nk = nk1 + nk2;
+        const int buf = local & 1;
+        const uint32_t use = (uint32_t)(local >> 1);
+        if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) break;
+        tc_fence_after();
+        const uint32_t dacc = tmem + (uint32_t)(buf * C::TMEM_COLS);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          if (!mbar_wait(&full[s], ph)) {
+            ok = false;
+            break;
+          }
+          if (kb < nk1) {
+            if (!mbar_wait(&bfull[s], (bph >> s) & 1)) {
+              ok = false;
+              break;
+            }
+            bph ^= 1u << s;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * C::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + s * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t da = umma_desc(a0 + k * 32, 16, 1024);
+            const uint64_t db = BMN ? umma_desc(b0 + k * 16 * 128, 64 * BK * 2, 1024) : umma_desc(b0 + k * 32, 16, 1024);
+            umma_bf16(dacc, da, db, idesc, (kb | k) != 0);
+          }
+          umma_commit(&empty[s]);
+        }
+        umma_commit(&acc_full[buf]);
+      }
+    }
+  } else if (warp < 6) {
+    const int qd = warp & 3;
+    int local = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
+      int mi, ni;
+      sched.get(t, mi, ni);
+      const int m0 = mi * BM, n0 = ni * BN;
+      const int buf = local & 1;
+      const uint32_t use = (uint32_t)(local >> 1);
+      if (!mbar_wait(&acc_full[buf], use & 1)) break;
+      tc_fence_after();
+      const int row = m0 + qd * 32 + lane;
+      const uint32_t tq = tmem + (uint32_t)(buf * C::TMEM_COLS) + ((uint32_t)(qd * 32) << 16);
+      if (n0 < ep.rope_end) {
+        const int half = ep.rope_hd / 2;
+#pragma unroll 1
+        for (int h0 = 0; h0 < BN; h0 += ep.rope_hd) {
+#pragma unroll 1
+          for (int j0 = 0; j0 < half; j0 += 32) {
+            uint32_t ra[32], rb[32];
+            tmem_ld32(tq + h0 + j0, ra);
+            tmem_ld32(tq + h0 + half + j0, rb);
+            tmem_ld_wait();
+            epi_store_rope(ep, row, n0 + h0 + j0, n0 + h0 + half + j0, j0, ra, rb);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tq + c, r);
+          tmem_ld_wait();
+          epi_store(ep, row, n0 + c, r);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+    }
+  } else {
+    uint32_t it = 0, bph = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      int mi, ni;
+      sched.get(t, mi, ni);
+      const int n0 = ni * BN;
+      const int nk = nk1 + nk2;
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        if (kb >= nk1) continue;
+        const int s = it % C::STAGES;
+        const uint32_t ph = (it / C::STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1)) {
+          ok = false;
+          break;
+        }
+        dq_stage<BN, BMN>(q, cbs, sB + s * C::B_BYTES, n0, kb, N, K);
+        fence_proxy_async();  // the tensor core reads this stage through the async proxy
+        mbar_arrive(&bfull[s]);
+        bph ^= 1u << s;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * C::TMEM_COLS);
+  }
+}
+
 }  // namespace
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -358,6 +627,45 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int6
 }
 
 namespace {
+
+template <int BN, int BMN>
+cudaError_t launch_nf4(const GemmArgs& a, cudaStream_t s) {
+  using C = Cfg<BN>;
+  constexpr uint32_t kSmemQ = C::STAGES * (C::A_BYTES + C::B_BYTES) + 1024 /*align*/ + 512 /*barriers, codebook*/;
+  CUtensorMap tA, tA2, tB2;
+  if (!make_map(&tA, a.A, a.M, a.K, a.lda, BM)) return cudaErrorInvalidValue;
+  int nk2 = 0;
+  if (a.A2 && a.B2 && a.K2 > 0) {
+    if (!make_map(&tA2, a.A2, a.M, a.K2, a.lda2, BM)) return cudaErrorInvalidValue;
+    if (BMN) {
+      if (!make_map(&tB2, a.B2, a.K2, a.N, a.ldb2, BK)) return cudaErrorInvalidValue;
+    } else {
+      if (!make_map(&tB2, a.B2, a.N, a.K2, a.ldb2, BN)) return cudaErrorInvalidValue;
+    }
+    nk2 = (a.K2 + BK - 1) / BK;
+  } else {
+    tA2 = tA;
+    tB2 = tA;
+  }
+  Epi e{a.C, a.ldc, a.bias, a.R, a.ldr, a.alpha, a.c_f32, a.M, a.N,
+        a.rope_cos, a.rope_sin, a.rope_cos ? a.rope_end : 0, a.rope_hd, a.rope_S};
+  static std::atomic<unsigned long long> attr_done{0};
+  if (!done_on_device(attr_done)) {
+    const cudaError_t err = cudaFuncSetAttribute(k_gemm_nf4<BN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemQ);
+    if (err != cudaSuccess) return err;
+    mark_done_on_device(attr_done);
+  }
+  const int nk1 = a.K / BK;
+  TileSched sched;
+  sched.mt = (a.M + BM - 1) / BM;
+  sched.nt = (a.N + BN - 1) / BN;
+  const int total = sched.mt * sched.nt;
+  const int num_sms = device_sm_count();
+  const int grid = total < num_sms ? total : num_sms;
+  k_gemm_nf4<BN, BMN><<<grid, 192 + kDqThreads, kSmemQ, s>>>(tA, tA2, tB2, *a.Bq, e, sched, total, nk1, nk2, a.N, a.K);
+  note_launch(1);
+  return cudaGetLastError();
+}
 
 template <int BN, int AMN, int BMN>
 cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
@@ -411,10 +719,22 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t gemm_bf16(const GemmArgs& a, cudaStream_t s) {
-  if (a.M <= 0 || a.N <= 0 || a.K <= 0 || !a.A || !a.B || !a.C) return cudaErrorInvalidValue;
+  if (a.M <= 0 || a.N <= 0 || a.K <= 0 || !a.A || (!a.B && !a.Bq) || !a.C) return cudaErrorInvalidValue;
   // TMA: 16-byte aligned bases and row strides
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
-  if (!al16(a.A) || !al16(a.B) || (a.lda % 8) || (a.ldb % 8)) return cudaErrorInvalidValue;
+  if (!al16(a.A) || (a.lda % 8)) return cudaErrorInvalidValue;
+  if (!a.Bq && (!al16(a.B) || (a.ldb % 8))) return cudaErrorInvalidValue;
+  if (a.Bq) {
+    // W's rows are whole NF4 blocks; packed tensors 16-byte aligned; rows covered by the tensors
+    const Nf4Mat& q = *a.Bq;
+    const int wrows = a.b_mn ? a.K : a.N, wcols = a.b_mn ? a.N : a.K;
+    if (a.a_mn || q.nseg < 1 || q.nseg > 3 || q.cols != wcols || (wcols % 64) || q.row_end[q.nseg - 1] < wrows)
+      return cudaErrorInvalidValue;
+    for (int g = 0; g < q.nseg; ++g)
+      if (!q.packed[g] || !q.qabs[g] || !q.gscale[g] || !q.mean[g] || !al16(q.packed[g]) ||
+          (g && q.row_end[g] <= q.row_end[g - 1]))
+        return cudaErrorInvalidValue;
+  }
   if (a.A2 && (!al16(a.A2) || !al16(a.B2) || (a.lda2 % 8) || (a.ldb2 % 8))) return cudaErrorInvalidValue;
   const int64_t tiles256 = (int64_t)((a.M + BM - 1) / BM) * ((a.N + 255) / 256);
   int bn;
@@ -428,6 +748,16 @@ cudaError_t gemm_bf16(const GemmArgs& a, cudaStream_t s) {
       return cudaErrorInvalidValue;
     if (bn == 256 && (a.rope_end % 256)) bn = 128;
     if (bn < 128 || (a.rope_end % bn) || a.rope_end > a.N) return cudaErrorInvalidValue;
+  }
+  if (a.Bq) {
+    switch (bn * 2 + (a.b_mn ? 1 : 0)) {
+      case 64 * 2 + 0: return launch_nf4<64, 0>(a, s);
+      case 64 * 2 + 1: return launch_nf4<64, 1>(a, s);
+      case 128 * 2 + 0: return launch_nf4<128, 0>(a, s);
+      case 128 * 2 + 1: return launch_nf4<128, 1>(a, s);
+      case 256 * 2 + 0: return launch_nf4<256, 0>(a, s);
+      default: return launch_nf4<256, 1>(a, s);
+    }
   }
   const int code = bn * 4 + (a.a_mn ? 2 : 0) + (a.b_mn ? 1 : 0);
   switch (code) {

@@ -16,6 +16,22 @@
 
 namespace lst {
 
+// A bf16 weight matrix W [rows, cols] (row-major, cols a multiple of 64) held as up to three NF4
+// tensors stacked along its rows (q/k/v or gate/up of a layer), each in the format of nf4.cu:
+// tensor g covers rows [row_end[g-1], row_end[g]) (row_end[-1] = 0) and its element (r, c) is
+// element (r - row_end[g-1]) * cols + c of the tensor, so that with cols % 64 == 0 every 64-wide
+// column block of a row is exactly one NF4 block.
+struct Nf4Mat {
+  int nseg = 0;
+  int cols = 0;
+  int row_end[3] = {0, 0, 0};
+  const uint8_t* packed[3] = {};
+  const int8_t* qabs[3] = {};
+  const float* gscale[3] = {};
+  const float* mean[3] = {};
+  float cb[16] = {};  // the codebook
+};
+
 struct GemmArgs {
   int M = 0, N = 0, K = 0;
   const __nv_bfloat16* A = nullptr;   // [M, K], row stride lda
@@ -42,6 +58,11 @@ struct GemmArgs {
   const float* rope_cos = nullptr;
   const float* rope_sin = nullptr;
   int rope_end = 0, rope_hd = 0, rope_S = 0;
+  // Optional: B dequantised from NF4 inside the GEMM (B and ldb are then not used). b_mn = 0:
+  // B(n, k) = W[n][k] (W [N, K], "x W^T"); b_mn = 1: B(k, n) = W[k][n] (W [K, N], "x W"). The
+  // values equal those of nf4_dequant bit for bit, so the result equals the GEMM on the
+  // dequantised matrix byte for byte. Needs a_mn = 0 and W's row length (K or N) % 64 == 0.
+  const Nf4Mat* Bq = nullptr;
 };
 
 // Returns cudaSuccess or the launch / argument error. Deterministic: no split-K, no atomics.

@@ -86,6 +86,50 @@ lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_
   return st(gemm_bf16(a, S(stream)));
 }
 
+lst_status lst_k_gemm_nf4(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda, const lst_nf4_part* parts,
+                          int32_t nparts, int32_t b_mn, const uint16_t* A2, int64_t lda2, const uint16_t* B2,
+                          int64_t ldb2, int32_t K2, void* C, int64_t ldc, int32_t c_f32, float alpha, const float* bias,
+                          const float* R, int64_t ldr, void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0 || !A || !C || !parts || nparts < 1 || nparts > 3) return LST_ERR_ARG;
+  if ((A2 == nullptr) != (B2 == nullptr)) return LST_ERR_ARG;
+  Nf4Mat q;
+  q.nseg = nparts;
+  q.cols = b_mn ? N : K;
+  int rows = 0;
+  for (int g = 0; g < nparts; ++g) {
+    if (parts[g].rows <= 0 || ((int64_t)parts[g].rows * q.cols) % 64) return LST_ERR_ARG;
+    rows += parts[g].rows;
+    q.row_end[g] = rows;
+    q.packed[g] = parts[g].packed;
+    q.qabs[g] = parts[g].qabs;
+    q.gscale[g] = parts[g].gscale;
+    q.mean[g] = parts[g].mean;
+  }
+  if (rows != (b_mn ? K : N)) return LST_ERR_ARG;
+  nf4_codebook(q.cb);
+  GemmArgs a;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.A = B16(A);
+  a.lda = lda;
+  a.b_mn = b_mn ? 1 : 0;
+  a.Bq = &q;
+  a.A2 = B16(A2);
+  a.lda2 = lda2;
+  a.B2 = B16(B2);
+  a.ldb2 = ldb2;
+  a.K2 = A2 ? K2 : 0;
+  a.C = C;
+  a.ldc = ldc;
+  a.c_f32 = c_f32 ? 1 : 0;
+  a.alpha = alpha;
+  a.bias = bias;
+  a.R = R;
+  a.ldr = ldr;
+  return st(gemm_bf16(a, S(stream)));
+}
+
 lst_status lst_k_attention_fwd(const uint16_t* q, int64_t ldq, const uint16_t* k, int64_t ldk, const uint16_t* v,
                                int64_t ldv, uint16_t* o, int64_t ldo, float* lse, int64_t T, int32_t Sq, int32_t hq,
                                int32_t hkv, int32_t hd, void* stream) {
@@ -172,6 +216,14 @@ lst_status lst_k_lora_skinny(const uint16_t* X, int64_t ldx, int64_t T, int32_t 
                              int32_t b_mn, int32_t KP, float s, uint16_t* Us, void* stream) {
   if (!X || !Bop || !Us || T <= 0 || K <= 0 || KP <= 0 || (KP % 8)) return LST_ERR_ARG;
   return st(lora_skinny(B16(X), ldx, T, K, B16(Bop), ldb, b_mn ? 1 : 0, KP, s, B16(Us), S(stream)));
+}
+
+lst_status lst_k_lora_skinny_split(const uint16_t* X, int64_t ldx, int64_t T, int32_t K, const uint16_t* Bop,
+                                   int64_t ldb, int32_t b_mn, int32_t R, int32_t RS, int32_t KP, float s, uint16_t* Us,
+                                   void* stream) {
+  if (!X || !Bop || !Us || T <= 0 || K <= 0 || R <= 0 || R > RS || RS > 64 || (RS % 8) || 3 * RS > KP || (KP % 8))
+    return LST_ERR_ARG;
+  return st(lora_skinny_split(B16(X), ldx, T, K, B16(Bop), ldb, b_mn ? 1 : 0, R, RS, KP, s, B16(Us), S(stream)));
 }
 
 lst_status lst_k_lora_grads(const uint16_t* X, int64_t ldx, int32_t in, const uint16_t* dY, int64_t ldy,

@@ -8,6 +8,9 @@
 //             dA = s V^T x,  dB = s dy^T U          (reductions over the T tokens)
 // Each of the four has one short side (nseg*r <= 64) and a long contraction (the in / out features,
 // or the T tokens), so one output tile holds little work and a plain tiling leaves most SMs idle.
+// The adapters are kept in full precision, so the projections run on a split operand: each adapter
+// value is the bf16 pair (hi, lo), both parts are contracted against the same tile of x or dy into
+// one fp32 accumulator, and U / V are stored as bf16 pairs again (lora.cuh, lora_skinny_split).
 // One kernel serves all four: a 128 x 64 output tile is computed by a thread-block cluster of cs
 // CTAs, CTA z contracting K-slice z with bf16 tcgen05 MMAs into TMEM (fp32); the cs partial tiles
 // are then parked in shared memory and summed through distributed shared memory, each CTA summing
@@ -20,18 +23,27 @@
 namespace lst {
 namespace {
 
-constexpr int kBM = 128, kBN = 64, kBK = 64, kStages = 4, kMaxCluster = 8;
+constexpr int kBM = 128, kBN = 64, kBK = 64, kMaxCluster = 8;
 constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint32_t kBBytes = kBN * kBK * 2;
 constexpr int kRedLd = kBN + 4;  // fp32 row stride of a parked partial tile (conflict-free float4 rows)
-constexpr uint32_t kSmem = kStages * (kABytes + kBBytes) + 1024 /*align*/ + 256 /*barriers*/;
-static_assert(kBM * kRedLd * 4 <= kStages * kABytes, "the partial tile reuses the A stages");
+// DUAL: two B tiles per K step (the hi and lo parts of a split operand), one stage fewer so that
+// two CTAs still fit on an SM.
+template <int DUAL>
+struct SideCfg {
+  static constexpr int kStages = DUAL ? 3 : 4;
+  static constexpr uint32_t kStageB = (1 + DUAL) * kBBytes;
+  static constexpr uint32_t kSmem = kStages * (kABytes + kStageB) + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(kBM * kRedLd * 4 <= kStages * kABytes, "the partial tile reuses the A stages");
+};
 
 // Destination of the summed tile C [M, N] (times scale).
 struct SideOut {
   // 0: out16[row * ld + col] = bf16(c)                                      (U or V, [T, KP])
   // 1: row p*r + j (< nseg*r) -> dst[p][j * N + col]                       (dA, [r, in] each)
   // 2: row o of segment p, column p*r + j -> dst[p][(o - bounds[p]) * r + j] (dB, [out_p, r] each)
+  // 3: column j < R: hi = bf16(c) to out16[row * ld + j] and [.. + 2 RS + j], lo = bf16(c - hi)
+  //    to [.. + RS + j]                                                     (split U or V, [T, KP])
   int mode;
   int M, N;
   float scale;
@@ -40,13 +52,24 @@ struct SideOut {
   float* dst[3];
   int r, nseg;
   int bounds[4];
+  int R, RS;  // mode 3
 };
 
 __device__ __forceinline__ void side_store(const SideOut& o, int row, int col, float4 v) {
   if (row >= o.M || col >= o.N) return;
   const float a[4] = {o.scale * v.x, o.scale * v.y, o.scale * v.z, o.scale * v.w};
   const bool full = col + 4 <= o.N;
-  if (o.mode == 0) {
+  if (o.mode == 3) {
+    __nv_bfloat16* p = o.out16 + (int64_t)row * o.ld;
+    for (int i = 0; i < 4; ++i) {
+      const int j = col + i;
+      if (j >= o.R) break;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(a[i]);
+      p[j] = hi;
+      p[o.RS + j] = __float2bfloat16_rn(a[i] - __bfloat162float(hi));
+      p[2 * o.RS + j] = hi;
+    }
+  } else if (o.mode == 0) {
     __nv_bfloat16* p = o.out16 + (int64_t)row * o.ld + col;
     if (full && (reinterpret_cast<uintptr_t>(p) & 7) == 0) {
       const __nv_bfloat162 h[2] = {__floats2bfloat162_rn(a[0], a[1]), __floats2bfloat162_rn(a[2], a[3])};
@@ -79,15 +102,19 @@ __device__ __forceinline__ void side_store(const SideOut& o, int row, int col, f
 // grid (cs, ceil(M/128), ceil(N/64)), cluster (cs, 1, 1), 192 threads: warp 0 TMA producer, warp 1
 // TMEM owner + MMA issuer, warps 2-5 park the accumulator; then all threads sum and store.
 // AMN / BMN: A / B MN-major ([K, M] / [K, N] row-major in memory), else K-major.
-template <int AMN, int BMN>
+// DUAL: every K step also loads the B tile b_off further along N (rows of a K-major B, columns of
+// an MN-major B) and accumulates its product with the same A tile.
+template <int AMN, int BMN, int DUAL>
 __global__ void __launch_bounds__(192, 2)
 k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const SideOut o,
-       const int nk, const int kps) {
+       const int nk, const int kps, const int b_off) {
+  constexpr int kStages = SideCfg<DUAL>::kStages;
+  constexpr uint32_t kStageB = SideCfg<DUAL>::kStageB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * kBBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * kStageB);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
@@ -128,7 +155,7 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         const int s = kb % kStages;
         const uint32_t ph = (kb / kStages) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1)) break;
-        mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
+        mbar_arrive_expect_tx(&full[s], kABytes + kStageB);
         const int kk = (kb0 + kb) * kBK;
         if (AMN == 0) {
           tma_load_2d(sA + s * kABytes, &tmA, &full[s], kk, m0);
@@ -137,9 +164,11 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           tma_load_2d(sA + s * kABytes + 64 * kBK * 2, &tmA, &full[s], m0 + 64, kk);
         }
         if (BMN == 0) {
-          tma_load_2d(sB + s * kBBytes, &tmB, &full[s], kk, n0);
+          tma_load_2d(sB + s * kStageB, &tmB, &full[s], kk, n0);
+          if (DUAL) tma_load_2d(sB + s * kStageB + kBBytes, &tmB, &full[s], kk, n0 + b_off);
         } else {
-          tma_load_2d(sB + s * kBBytes, &tmB, &full[s], n0, kk);
+          tma_load_2d(sB + s * kStageB, &tmB, &full[s], n0, kk);
+          if (DUAL) tma_load_2d(sB + s * kStageB + kBBytes, &tmB, &full[s], n0 + b_off, kk);
         }
       }
     }
@@ -152,12 +181,17 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         if (!mbar_wait(&full[s], ph)) break;
         tc_fence_after();
         const uint32_t a0 = smem_u32(sA + s * kABytes);
-        const uint32_t b0 = smem_u32(sB + s * kBBytes);
+        const uint32_t b0 = smem_u32(sB + s * kStageB);
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
           const uint64_t da = AMN ? umma_desc(a0 + k * 16 * 128, 64 * kBK * 2, 1024) : umma_desc(a0 + k * 32, 16, 1024);
           const uint64_t db = BMN ? umma_desc(b0 + k * 16 * 128, 64 * kBK * 2, 1024) : umma_desc(b0 + k * 32, 16, 1024);
           umma_bf16(tmem, da, db, idesc, (kb | k) != 0);
+          if (DUAL) {
+            const uint32_t b1 = b0 + kBBytes;
+            const uint64_t db1 = BMN ? umma_desc(b1 + k * 16 * 128, 64 * kBK * 2, 1024) : umma_desc(b1 + k * 32, 16, 1024);
+            umma_bf16(tmem, da, db1, idesc, 1);
+          }
         }
         umma_commit(&empty[s]);
       }
@@ -221,12 +255,13 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   }
 }
 
-template <int AMN, int BMN>
+template <int AMN, int BMN, int DUAL = 0>
 cudaError_t launch_side(const CUtensorMap& tA, const CUtensorMap& tB, int M, int N, int K, const SideOut& o,
-                        cudaStream_t st) {
+                        cudaStream_t st, int b_off = 0) {
+  constexpr uint32_t kSmem = SideCfg<DUAL>::kSmem;
   static std::atomic<unsigned long long> attr_done{0};  // devices whose function attribute is set
   if (!done_on_device(attr_done)) {
-    const cudaError_t err = cudaFuncSetAttribute(k_side<AMN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    const cudaError_t err = cudaFuncSetAttribute(k_side<AMN, BMN, DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (err != cudaSuccess) return err;
     mark_done_on_device(attr_done);
   }
@@ -249,12 +284,18 @@ cudaError_t launch_side(const CUtensorMap& tA, const CUtensorMap& tB, int M, int
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_side<AMN, BMN>, tA, tB, o, nk, kps);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_side<AMN, BMN, DUAL>, tA, tB, o, nk, kps, b_off);
   note_launch(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Part `sec` of the split value of v: 0 and 1 hi = bf16(v), 2 lo = bf16(v - hi).
+__device__ __forceinline__ __nv_bfloat16 split_part(float v, int sec) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+  return sec == 2 ? __float2bfloat16_rn(v - __bfloat162float(hi)) : hi;
+}
 
 __global__ void k_lora_prep(const LoraPrepArgs a) {
   const int R = a.nseg * a.r;
@@ -263,17 +304,20 @@ __global__ void k_lora_prep(const LoraPrepArgs a) {
   const int64_t n2 = (int64_t)out * a.KP;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n1; i += stride) {
-    const int j = (int)(i / a.in), c = (int)(i % a.in);
-    const float v = j < R ? a.A[j / a.r][(int64_t)(j % a.r) * a.in + c] : 0.f;
-    a.Acat16[i] = __float2bfloat16_rn(v);
+    const int row = (int)(i / a.in), c = (int)(i % a.in);
+    const int sec = row / a.RS, j = row % a.RS;  // section 3 and beyond: padding
+    float v = 0.f;
+    if (sec < 3 && j < R) v = a.A[j / a.r][(int64_t)(j % a.r) * a.in + c];
+    a.Acat16[i] = split_part(v, sec);
   }
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += stride) {
-    const int o = (int)(i / a.KP), j = (int)(i % a.KP);
+    const int o = (int)(i / a.KP), col = (int)(i % a.KP);
+    const int sec = col / a.RS, j = col % a.RS;
     int p = 0;
     while (p + 1 < a.nseg && o >= a.bounds[p + 1]) ++p;
     float v = 0.f;
-    if (j < R && j / a.r == p) v = a.B[p][(int64_t)(o - a.bounds[p]) * a.r + (j % a.r)];
-    a.Bexp16[i] = __float2bfloat16_rn(v);
+    if (sec < 3 && j < R && j / a.r == p) v = a.B[p][(int64_t)(o - a.bounds[p]) * a.r + (j % a.r)];
+    a.Bexp16[i] = split_part(v, sec);
   }
 }
 
@@ -300,6 +344,35 @@ cudaError_t lora_skinny(const __nv_bfloat16* X, int64_t ldx, int64_t T, int K, c
   return b_mn ? launch_side<0, 1>(tA, tB, (int)T, KP, K, o, st) : launch_side<0, 0>(tA, tB, (int)T, KP, K, o, st);
 }
 
+cudaError_t lora_skinny_split(const __nv_bfloat16* X, int64_t ldx, int64_t T, int K, const __nv_bfloat16* Bop,
+                              int64_t ldb, int b_mn, int R, int RS, int KP, float s, __nv_bfloat16* Us,
+                              cudaStream_t st) {
+  if (T <= 0 || T > INT32_MAX || K <= 0 || R <= 0 || R > RS || RS % 8 || RS > kBN || 3 * RS > KP || KP % 8 || !X ||
+      !Bop || !Us)
+    return cudaErrorInvalidValue;
+  if (!al16(X) || !al16(Bop) || (ldx % 8) || (ldb % 8)) return cudaErrorInvalidValue;
+  CUtensorMap tA, tB;
+  if (!make_map(&tA, X, T, K, ldx, kBM)) return cudaErrorInvalidValue;
+  if (b_mn) {
+    if (!make_map(&tB, Bop, K, KP, ldb, kBK)) return cudaErrorInvalidValue;
+  } else {
+    if (!make_map(&tB, Bop, KP, K, ldb, kBN)) return cudaErrorInvalidValue;
+  }
+  SideOut o{};
+  o.mode = 3;
+  o.M = (int)T;
+  o.N = R;
+  o.scale = s;
+  o.out16 = Us;
+  o.ld = KP;
+  o.R = R;
+  o.RS = RS;
+  // the lo part of the operand starts 2 RS further along N: a multiple of 16 elements, so the TMA
+  // x coordinate of the MN-major case stays 16-byte aligned
+  return b_mn ? launch_side<0, 1, 1>(tA, tB, (int)T, R, K, o, st, 2 * RS)
+              : launch_side<0, 0, 1>(tA, tB, (int)T, R, K, o, st, 2 * RS);
+}
+
 cudaError_t lora_grad_a(const __nv_bfloat16* X, int64_t ldx, int64_t T, int in, const __nv_bfloat16* Vs, int KP,
                         int nseg, int r, float* const* dst, cudaStream_t st) {
   if (nseg < 1 || nseg > 3 || r <= 0 || nseg * r > KP || KP % 8 || T <= 0 || in <= 0) return cudaErrorInvalidValue;
@@ -310,13 +383,13 @@ cudaError_t lora_grad_a(const __nv_bfloat16* X, int64_t ldx, int64_t T, int in, 
   if (!make_map(&tB, X, T, in, ldx, kBK)) return cudaErrorInvalidValue;
   SideOut o{};
   o.mode = 1;
-  o.M = KP;
+  o.M = nseg * r;  // rows of C past the adapters' ranks are not stored
   o.N = in;
   o.scale = 1.0f;
   for (int k = 0; k < nseg; ++k) o.dst[k] = dst[k];
   o.r = r;
   o.nseg = nseg;
-  return launch_side<1, 1>(tA, tB, KP, in, (int)T, o, st);
+  return launch_side<1, 1>(tA, tB, o.M, in, (int)T, o, st);
 }
 
 cudaError_t lora_grad_b(const __nv_bfloat16* dY, int64_t ldy, int64_t T, int out, const __nv_bfloat16* Us, int KP,
@@ -330,17 +403,17 @@ cudaError_t lora_grad_b(const __nv_bfloat16* dY, int64_t ldy, int64_t T, int out
   SideOut o{};
   o.mode = 2;
   o.M = out;
-  o.N = KP;
+  o.N = nseg * r;  // columns of C past the adapters' ranks are not stored
   o.scale = 1.0f;
   for (int k = 0; k < nseg; ++k) o.dst[k] = dst[k];
   for (int k = 0; k <= nseg; ++k) o.bounds[k] = bounds[k];
   o.r = r;
   o.nseg = nseg;
-  return launch_side<1, 1>(tA, tB, out, KP, (int)T, o, st);
+  return launch_side<1, 1>(tA, tB, out, o.N, (int)T, o, st);
 }
 
 cudaError_t lora_prep(const LoraPrepArgs& a, cudaStream_t st) {
-  if (a.nseg < 1 || a.nseg > 3 || a.nseg * a.r > a.KP) return cudaErrorInvalidValue;
+  if (a.nseg < 1 || a.nseg > 3 || a.nseg * a.r > a.RS || a.RS % 8 || 3 * a.RS > a.KP) return cudaErrorInvalidValue;
   k_lora_prep<<<1024, 256, 0, st>>>(a);
   note_launch(1);
   return cudaGetLastError();

@@ -15,6 +15,17 @@ namespace lst {
 cudaError_t lora_skinny(const __nv_bfloat16* X, int64_t ldx, int64_t T, int K, const __nv_bfloat16* Bop,
                         int64_t ldb, int b_mn, int KP, float s, __nv_bfloat16* Us, cudaStream_t st);
 
+// The same projection at fp32-level precision from a split operand, for adapters kept in full
+// precision: Bop holds the adapter as two bf16 parts, hi = bf16(a) in sections [0, RS) and
+// lo = bf16(a - hi) in [2 RS, 3 RS) of its KP-wide dimension (rows when K-major, columns when
+// MN-major), and U = s X (hi + lo) is accumulated in fp32 in one pass over X. U (columns j < R) is
+// stored split as well: Us[t][j] = Us[t][2 RS + j] = bf16(U), Us[t][RS + j] = bf16(U - bf16(U)),
+// so that the pair (Us, operand) sections [hi | lo | hi] x [hi | hi | lo] form the three products
+// whose sum is U W'^T up to the lo x lo term. RS is a multiple of 8, R <= RS, 3 RS <= KP.
+cudaError_t lora_skinny_split(const __nv_bfloat16* X, int64_t ldx, int64_t T, int K, const __nv_bfloat16* Bop,
+                              int64_t ldb, int b_mn, int R, int RS, int KP, float s, __nv_bfloat16* Us,
+                              cudaStream_t st);
+
 // dA of every segment of a fused group: dA_p[j][i] = sum_t Vs[t][p*r + j] X[t][i] with X bf16
 // [T, in] and Vs = bf16(s V) [T, KP]; dst[p] fp32 [r, in]. Computed as the [KP, in] product
 // Vs^T X, each row stored straight into its segment.
@@ -27,16 +38,20 @@ cudaError_t lora_grad_b(const __nv_bfloat16* dY, int64_t ldy, int64_t T, int out
                         int nseg, int r, const int* bounds, float* const* dst, cudaStream_t st);
 
 // Derived bf16 operands of one fused projection group from its fp32 adapters (nseg segments,
-// A_p [r, in], B_p [out_p, r]):
-//   Acat16 [KP, in]: rows p*r + j = A_p[j] (rows >= nseg*r zero);
-//   Bexp16 [out, KP]: row o of segment p holds B_p[o - bounds[p]] in columns p*r .. p*r + r - 1,
-//   zero elsewhere.
+// A_p [r, in], B_p [out_p, r]), each adapter value a stored as the pair hi = bf16(a),
+// lo = bf16(a - hi) in three sections of RS rows (Acat) or columns (Bexp):
+//   Acat16 [KP, in]: row p*r + j holds hi(A_p[j]), row RS + p*r + j hi(A_p[j]) again and row
+//   2 RS + p*r + j lo(A_p[j]);
+//   Bexp16 [out, KP]: row o of segment p holds hi(B_p[o - bounds[p]]) in columns p*r .. p*r + r - 1
+//   and RS + p*r .., and lo(...) in columns 2 RS + p*r ..;
+// every other element zero. With the split Us / Vs of the projections this keeps the side path at
+// fp32-level precision on the bf16 tensor cores.
 struct LoraPrepArgs {
   const float* A[3];
   const float* B[3];
   int nseg, r, in;
   int bounds[4];  // out-row bounds of the segments
-  int KP;
+  int RS, KP;
   __nv_bfloat16* Acat16;
   __nv_bfloat16* Bexp16;
 };

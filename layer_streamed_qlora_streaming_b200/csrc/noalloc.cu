@@ -12,8 +12,6 @@
 #include "common.cuh"
 #include "nf4.cuh"
 
-#include <mutex>
-
 namespace {
 
 constexpr int64_t kNoAllocMaxElems = int64_t(1) << 26;           // 67,108,864 elements per call
@@ -25,34 +23,19 @@ constexpr size_t kScratchBytes = (size_t)kAbsmaxFloats * 4 + (size_t)kGsumDouble
 // a device comes from cudaGetSymbolAddress below and is what the kernels receive.
 static __device__ __align__(256) unsigned char g_nf4_noalloc_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};  // device address of the array, per device ordinal
-
 }  // namespace
 
 extern "C" lst_status lst_k_nf4_quantize_noalloc(const float* w, int64_t n, uint8_t* packed, int8_t* qabs,
                                                  float* gscale, float* mean, void* stream) {
   if (!w || !packed || !qabs || !gscale || !mean || n <= 0 || n % 64) return LST_ERR_ARG;
   if (n > kNoAllocMaxElems) return LST_ERR_ARG;  // beyond the fixed scratch: rejected, nothing launched
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  // The array's address on the current device, looked up on every call (cheap, allocates
+  // nothing): a cached address would go stale if the device's primary context were recreated
+  // (cudaDeviceReset), which may place the module's arrays elsewhere.
+  void* base = nullptr;
+  if (cudaGetSymbolAddress(&base, g_nf4_noalloc_scratch) != cudaSuccess || !base) {
     cudaGetLastError();
     return LST_ERR_CUDA;
-  }
-  void* base = nullptr;
-  {
-    // first call on this device (which must be the current device): look the array up once
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
-      void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_nf4_noalloc_scratch) != cudaSuccess || !p) {
-        cudaGetLastError();
-        return LST_ERR_CUDA;
-      }
-      g_scratch_ptr[dev] = p;
-    }
-    base = g_scratch_ptr[dev];
   }
   // Both scratch arrays are fully written by the quantiser before they are read, so nothing has
   // to be cleared between calls.

@@ -7,8 +7,9 @@
 // The update is the decoupled-weight-decay Adam of Loshchilov & Hutter:
 //   m <- b1 m + (1 - b1) g ;  v <- b2 v + (1 - b2) g^2
 //   p <- p (1 - lr wd) - (lr / (1 - b1^t)) m / (sqrt(v) / sqrt(1 - b2^t) + eps)
-// in fp32, element by element (deterministic). The same pass writes bf16(p) to the place the
-// element occupies in the group operands (Acat [KP, in] or Bexp [out, KP]) the GEMMs read.
+// in fp32, element by element (deterministic). The same pass writes the split bf16 pair
+// (bf16(p), bf16(p - bf16(p))) to the places the element occupies in the group operands
+// (Acat [KP, in] or Bexp [out, KP]) the GEMMs read.
 #include "common.cuh"
 #include "optim.cuh"
 
@@ -29,7 +30,11 @@ __global__ void k_adamw(const AdamTensor* __restrict__ tab, float* __restrict__ 
     const float pi = p[i] * (1.0f - h.lr * h.wd) - h.step_size * (mi / denom);
     p[i] = pi;
     const int row = (int)(e / t.cols), col = (int)(e % t.cols);
-    t.dst[(int64_t)(t.dst_row0 + row) * t.dst_ld + t.dst_col0 + col] = __float2bfloat16_rn(pi);
+    __nv_bfloat16* e0 = t.dst + (int64_t)(t.dst_row0 + row) * t.dst_ld + t.dst_col0 + col;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(pi);
+    e0[0] = hi;
+    e0[t.sec] = hi;
+    e0[2 * t.sec] = __float2bfloat16_rn(pi - __bfloat162float(hi));
   }
 }
 

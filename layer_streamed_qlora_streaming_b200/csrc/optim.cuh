@@ -8,14 +8,16 @@
 namespace lst {
 
 // One adapter tensor [rows, cols] at `off` in the parameter / gradient / moment buffers, and the
-// bf16 operand it is mirrored into: element (row, col) goes to
-// dst[(dst_row0 + row) * dst_ld + dst_col0 + col].
+// split bf16 operand it is mirrored into: element (row, col) = p goes to
+// e = dst + (dst_row0 + row) * dst_ld + dst_col0 + col as e[0] = e[sec] = bf16(p) and
+// e[2 sec] = bf16(p - bf16(p)), sec being the section stride (elements) of the operand.
 struct AdamTensor {
   int64_t off, n;
   int rows, cols;
   __nv_bfloat16* dst;
   int64_t dst_ld;
   int dst_row0, dst_col0;
+  int64_t sec;
 };
 
 struct AdamHyper {

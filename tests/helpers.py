@@ -14,6 +14,13 @@ GRAD_MAXREL = 2e-2
 # Against the exact (unrounded fp64) oracle the difference is the rounding noise of bf16 operands
 # (unit roundoff 2^-8, amplified by softmax and products); bound the logits at 3x the above.
 EXACT_LOGITS_MAXREL = 3e-2
+# Gradients against the exact oracle: the workloads compute with bf16 activations, and on two
+# Qwen2.5-32B-shaped layers (batch 1 x 256) the oracle's own bf16-activation mode is already 2.48%
+# (q dA) and 2.66% (k dA) max-rel from its exact mode -- the rounding of layer 0's forward
+# activations moves the top layer's q/k adapter gradients that much. No bf16-activation
+# computation can be held closer to exact arithmetic than that, so the exact-oracle bound is 3e-2
+# (cosine unchanged); the benchmark spec's 2e-2 applies against the bf16-activation oracle.
+EXACT_GRAD_MAXREL = 3e-2
 
 
 def cosine(a, b) -> float:

@@ -1,22 +1,29 @@
-"""Host-side pieces of bench.py that need no GPU: the recorded GEMM traffic is reported only for
-the workload and GEMM sources it was measured on; throughput and workload descriptions."""
-import copy
-
+"""Host-side pieces of bench.py that need no GPU: the copy / compute overlap summary of a read
+timeline, throughput and workload descriptions."""
 import pytest
 
 bench = pytest.importorskip("bench")
 
 
-def test_gemm_traffic_only_for_the_measured_sources(monkeypatch):
-    per_launch, per_step = bench.gemm_traffic("llama8b")
-    if per_launch is not None:          # the GEMM sources are the measured ones
-        assert per_step == bench.GEMM_TRAFFIC["bytes_per_step"]
-        assert per_launch == per_step / bench.GEMM_TRAFFIC["launches"]
-    assert bench.gemm_traffic("qwen3b_bf16") == (None, None)      # another workload
-    changed = copy.deepcopy(bench.GEMM_TRAFFIC)
-    changed["sources"]["gemm.cu"] = "0" * 16
-    monkeypatch.setattr(bench, "GEMM_TRAFFIC", changed)
-    assert bench.gemm_traffic("llama8b") == (None, None)          # sources changed since
+def _row(kind, copy, deq, comp):
+    return {"layer": 0, "kind": kind, "copy": copy, "dequant": deq, "compute": comp}
+
+
+def test_timeline_summary_overlap_and_gaps():
+    # read 0 copies alone (0-2); read 1's copy (2-4) runs under read 0's compute (2-5); read 2's
+    # copy (5-7) is half under read 1's compute (5-6); read 2 computes 7-8, after a 1 ms wait
+    tl = [_row("forward", (0.0, 2.0), (1.0, 2.0), (2.0, 5.0)),
+          _row("forward", (2.0, 4.0), (4.0, 4.5), (5.0, 6.0)),
+          _row("backward", (5.0, 7.0), (None, None), (7.0, 8.0))]
+    s = bench.timeline_summary(tl)
+    assert s["forward"]["reads"] == 2 and s["backward"]["reads"] == 1
+    assert s["forward"]["copy_ms"] == pytest.approx(2.0)
+    assert s["forward"]["compute_ms"] == pytest.approx(2.0)
+    assert s["backward"]["dequant_ms"] is None
+    # hidden copy: read 0 none, read 1 2 ms (under read 0), read 2 1 ms (under read 1) of 6 ms
+    assert s["copy_hidden_frac"] == pytest.approx(3.0 / 6.0)
+    assert s["compute_gap_ms_total"] == pytest.approx(0.0 + 1.0)
+    assert s["first_compute_start_ms"] == 2.0 and s["last_compute_end_ms"] == 8.0
 
 
 def test_job_throughput_counts_every_rank():

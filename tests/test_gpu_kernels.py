@@ -103,6 +103,97 @@ def test_gemm(M, N, K, b_mn, ext, f32, bias, resid):
     assert maxrel(got, ref) < tol, maxrel(got, ref)
 
 
+def _nf4_parts(rows_list, cols, seed):
+    """Quantise len(rows_list) random tensors [rows, cols] on the GPU; returns (parts for
+    lst_k_gemm_nf4, the stacked dequantised bf16 matrix on the GPU, keep-alive list)."""
+    parts, deq, keep = [], [], []
+    for i, rows in enumerate(rows_list):
+        n = rows * cols
+        w = syn.normal(seed, i, n, 0.02).astype(np.float32)
+        packed = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
+        qabs = torch.empty(n // 64, dtype=torch.int8, device="cuda")
+        gsc = torch.empty((n // 64 + 255) // 256, dtype=torch.float32, device="cuda")
+        mean = torch.empty(1, dtype=torch.float32, device="cuda")
+        lst.k_nf4_quantize(torch_f32(w), packed, qabs, gsc, mean)
+        out = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        lst.k_nf4_dequant(packed, qabs, gsc, mean, n, out)
+        parts.append((packed, qabs, gsc, mean, rows))
+        deq.append(out.view(rows, cols))
+        keep += [packed, qabs, gsc, mean]
+    return parts, torch.cat(deq, 0).contiguous(), keep
+
+
+NF4_GEMM_CASES = [
+    # M, parts (rows of W), cols of W, b_mn, LoRA pair, out_f32, bias, resid
+    (256, [256, 64, 64], 256, 0, False, False, True, False),   # q/k/v-like, BN=128 K-major, bias
+    (300, [384, 384], 128, 0, True, True, False, False),       # gate/up-like, ragged M, LoRA pair
+    (128, [64], 512, 0, False, True, False, True),             # BN = 64, residual
+    (256, [256, 128, 128], 320, 1, True, True, False, False),  # dX of q/k/v: W [K, N] MN-major
+    (384, [1024, 1024], 256, 1, False, True, False, False),    # dX of gate/up
+    (2048, [4096, 1024, 1024], 4096, 0, True, False, False, False),  # 8B q/k/v forward
+    (2048, [14336, 14336], 4096, 1, True, True, False, False),       # 8B gate/up dX
+]
+
+
+@pytest.mark.parametrize("M,rows,cols,b_mn,ext,f32,bias,resid", NF4_GEMM_CASES)
+def test_gemm_nf4_equals_dequant_then_gemm(M, rows, cols, b_mn, ext, f32, bias, resid):
+    # the GEMM that dequantises its NF4 operand in shared memory gives the same bytes as the
+    # separate dequantisation followed by the bf16 GEMM (same operand bits, same K order)
+    r = _rng(M + sum(rows) + cols + b_mn)
+    parts, Wd, keep = _nf4_parts(rows, cols, 900 + len(rows) + b_mn)
+    W_rows = sum(rows)
+    if b_mn:
+        K, N = W_rows, cols
+    else:
+        N, K = W_rows, cols
+    A = torch_bf16(r.normal(size=(M, K)))
+    kw = {}
+    if ext:
+        A2 = np.zeros((M, 64), np.float32)
+        A2[:, :48] = _bf(r.normal(size=(M, 48)))
+        B2 = np.zeros((64, N) if b_mn else (N, 64), np.float32)
+        if b_mn:
+            B2[:48] = _bf(r.normal(size=(48, N)) * 0.1)
+        else:
+            B2[:, :48] = _bf(r.normal(size=(N, 48)) * 0.1)
+        kw.update(A2=torch_bf16(A2), lda2=64, B2=torch_bf16(B2), ldb2=N if b_mn else 64, K2=64)
+    if bias:
+        kw["bias"] = torch_f32(r.normal(size=N).astype(np.float32))
+    if resid:
+        kw.update(R=torch_f32(r.normal(size=(M, N)).astype(np.float32)), ldr=N)
+    dt = torch.float32 if f32 else torch.bfloat16
+    C1 = torch.full((M, N), float("nan"), dtype=dt, device="cuda")
+    C2 = torch.full((M, N), float("nan"), dtype=dt, device="cuda")
+    lst.k_gemm(M, N, K, A, K, Wd, cols, b_mn, C1, N, int(f32), **kw)
+    for _ in range(2):  # twice: the same bytes again
+        lst.k_gemm_nf4(M, N, K, A, K, parts, b_mn, C2, N, int(f32), **kw)
+        torch.cuda.synchronize()
+        assert torch.equal(C1.view(torch.int16 if not f32 else torch.int32),
+                           C2.view(torch.int16 if not f32 else torch.int32))
+    # and against the oracle's arithmetic on the same operand values
+    Wn = to_np(Wd).astype(np.float64)
+    ref = to_np(A).astype(np.float64) @ (Wn if b_mn else Wn.T)
+    if ext:
+        ref = ref + to_np(kw["A2"]).astype(np.float64) @ (to_np(kw["B2"]) if b_mn else to_np(kw["B2"]).T)
+    if bias:
+        ref = ref + to_np(kw["bias"])
+    if resid:
+        ref = ref + to_np(kw["R"])
+    assert maxrel(to_np(C2), ref) < (1e-4 if f32 else 8e-3)
+    del keep
+
+
+def test_gemm_nf4_rejects_rows_not_whole_blocks():
+    # a W row length that is not a multiple of 64 cannot be dequantised block by block in the tile
+    parts, _, keep = _nf4_parts([64], 64, 5)
+    A = torch.zeros(128, 688, dtype=torch.bfloat16, device="cuda")
+    p = list(parts[0])
+    p[4] = 64
+    with pytest.raises(lst.LstError):
+        lst.k_gemm_nf4(128, 64, 688, A, 688, [tuple(p)], 0, torch.zeros(128, 64, device="cuda"), 64, 1)
+    del keep
+
+
 def test_gemm_rejects_misaligned_stride():
     A = torch.zeros(128, 100, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(lst.LstError):
@@ -270,6 +361,55 @@ def test_lora_skinny(T, K, b_mn):
     got = to_np(Us)
     assert maxrel(got, ref) < 8e-3
     assert np.all(got[:, R:] == 0)
+
+
+def _split_pair(a):
+    """(hi, lo) bf16 parts of fp32 values: hi = bf16(a), lo = bf16(a - hi)."""
+    hi = _bf(a)
+    return hi, _bf(a.astype(np.float32) - hi)
+
+
+@pytest.mark.parametrize("T,K,R,b_mn", [(300, 688, 24, 0), (2048, 4096, 48, 0), (2048, 6144, 48, 1),
+                                        (128, 256, 8, 1), (256, 5120, 16, 0)])
+def test_lora_skinny_split(T, K, R, b_mn):
+    # U = s X (hi + lo) for an fp32 adapter held as bf16 pairs: fp32-level accuracy, stored as pairs
+    rng = _rng(T * 3 + K + R + b_mn)
+    RS = (R + 7) // 8 * 8
+    KP = (3 * RS + 63) // 64 * 64
+    X = _bf(rng.normal(size=(T, K)))
+    A = (rng.uniform(-1, 1, size=(R, K)) / np.sqrt(K)).astype(np.float32)   # fp32 adapter [R, K]
+    hi, lo = _split_pair(A)
+    if b_mn:                                   # operand [K, KP]: sections along columns
+        Bop = np.zeros((K, KP), np.float32)
+        Bop[:, :R], Bop[:, RS:RS + R], Bop[:, 2 * RS:2 * RS + R] = hi.T, hi.T, lo.T
+        ldb = KP
+    else:                                      # operand [KP, K]: sections along rows
+        Bop = np.zeros((KP, K), np.float32)
+        Bop[:R], Bop[RS:RS + R], Bop[2 * RS:2 * RS + R] = hi, hi, lo
+        ldb = K
+    ref = 2.0 * X.astype(np.float64) @ A.astype(np.float64).T           # [T, R], exact fp32 adapter
+    Us = torch.full((T, KP), float("nan"), dtype=torch.bfloat16, device="cuda")
+    outs = []
+    for _ in range(2):
+        lst.k_lora_skinny_split(torch_bf16(X), K, T, K, torch_bf16(Bop), ldb, b_mn, R, RS, KP, 2.0, Us)
+        torch.cuda.synchronize()
+        outs.append(Us.view(torch.int16).cpu().numpy().copy())
+    assert np.array_equal(outs[0], outs[1])
+    got = to_np(Us)
+    u_hi, u_lo, u_hi2 = got[:, :R], got[:, RS:RS + R], got[:, 2 * RS:2 * RS + R]
+    assert np.array_equal(u_hi, u_hi2)
+    assert np.array_equal(u_hi, _bf(u_hi))                             # hi is a bf16 value
+    u = u_hi.astype(np.float64) + u_lo.astype(np.float64)
+    # fp32 accumulation of exact bf16 products: far below bf16's 2^-8 (the lo part is live)
+    assert maxrel(u, ref) < 2e-5, maxrel(u, ref)
+    assert maxrel(u_hi, ref) > 1e-4 or np.allclose(u_lo, 0)
+    # lo is the bf16 rounding of the remainder of the fp32 sum: |lo| <= half an ulp of hi
+    assert np.all(np.abs(u_lo) <= np.abs(u_hi) * 2.0 ** -8 + 1e-30)
+    # columns outside the three sections are not written
+    untouched = np.ones(KP, bool)
+    for s0 in (0, RS, 2 * RS):
+        untouched[s0:s0 + R] = False
+    assert np.all(np.isnan(got[:, untouched]))
 
 
 @pytest.mark.parametrize("T,in_f,bounds,r", [

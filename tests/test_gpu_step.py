@@ -4,8 +4,8 @@ import numpy as np
 import pytest
 
 import synthetic as syn
-from helpers import (EXACT_LOGITS_MAXREL, GRAD_COS, GRAD_MAXREL, LOGITS_MAXREL, LOSS_RTOL, build_inputs,
-                     compare_grads, make_context, maxrel, oracle_step, run_step)
+from helpers import (EXACT_GRAD_MAXREL, EXACT_LOGITS_MAXREL, GRAD_COS, GRAD_MAXREL, LOGITS_MAXREL, LOSS_RTOL,
+                     build_inputs, compare_grads, make_context, maxrel, oracle_step, run_step)
 
 pytestmark = pytest.mark.gpu
 
@@ -18,36 +18,30 @@ def _gpu():
         pytest.skip("needs a CUDA device")
 
 
-def _check_against_oracle(wl, inp, loss, grads, logits, ctx, exact_too=True, noise_floor=False):
-    """primary: the oracle with the workload's bf16 activations, at the parity tolerances.
-
-    noise_floor: a gradient tensor's max-rel bound is raised to the distance between the oracle's
-    own bf16-activation mode and its exact mode for that tensor, when that distance is larger: two
-    computations at the workload's precision cannot be expected to agree more closely than bf16
-    agrees with exact arithmetic (the cosine bound is unchanged)."""
+def _check_against_oracle(wl, inp, loss, grads, logits, ctx, exact_too=True):
+    """primary: the oracle with the workload's bf16 activations, at the parity tolerances (loss and
+    logits 1e-2, every gradient tensor cosine >= 0.999 and max-rel <= 2e-2); secondary: the exact
+    oracle, at the bounds of bf16 noise (helpers.py). Returns the worst (tensor, cosine, max-rel)
+    of each comparison."""
     ref = oracle_step(wl, inp, schedule="streamed", bf16_acts=True)
     assert abs(loss - ref["loss"]) <= LOSS_RTOL * abs(ref["loss"]), (loss, ref["loss"])
     if logits is not None:
         assert maxrel(logits, ref["logits"]) <= LOGITS_MAXREL, maxrel(logits, ref["logits"])
-    floor = {}
-    if noise_floor:
-        ex = oracle_step(wl, inp, schedule="streamed", bf16_acts=False)
-        for l, g in enumerate(ref["grads"]):
-            for p, (dA, dB) in g.items():
-                floor[(l, p, "A")] = maxrel(dA, ex["grads"][l][p][0])
-                floor[(l, p, "B")] = maxrel(dB, ex["grads"][l][p][1])
-    for l, p, w, cs, mr in compare_grads(ctx, grads, ref["grads"]):
-        bound = max(GRAD_MAXREL, floor.get((l, p, w), 0.0))
-        assert cs >= GRAD_COS and mr <= bound, (l, p, w, cs, mr, bound)
+    res = compare_grads(ctx, grads, ref["grads"])
+    for l, p, w, cs, mr in res:
+        assert cs >= GRAD_COS and mr <= GRAD_MAXREL, (l, p, w, cs, mr)
+    worst = {"bf16": max(res, key=lambda t: t[4])}
     if not exact_too:
-        return
-    # secondary: the exact oracle (no rounding at all), bounded by bf16 rounding noise
+        return worst
     ex = oracle_step(wl, inp, schedule="streamed", bf16_acts=False)
     assert abs(loss - ex["loss"]) <= LOSS_RTOL * abs(ex["loss"]), (loss, ex["loss"])
     if logits is not None:
         assert maxrel(logits, ex["logits"]) <= EXACT_LOGITS_MAXREL, maxrel(logits, ex["logits"])
-    for l, p, w, cs, mr in compare_grads(ctx, grads, ex["grads"]):
-        assert cs >= GRAD_COS and mr <= GRAD_MAXREL, ("exact", l, p, w, cs, mr)
+    res = compare_grads(ctx, grads, ex["grads"])
+    for l, p, w, cs, mr in res:
+        assert cs >= GRAD_COS and mr <= EXACT_GRAD_MAXREL, ("exact", l, p, w, cs, mr)
+    worst["exact"] = max(res, key=lambda t: t[4])
+    return worst
 
 
 WORKLOADS = {
@@ -269,9 +263,8 @@ def test_layer_above_165mb_nf4():
     ctx = make_context(wl, inp, streamed=True)
     assert ctx.stats()["blob_bytes"] > 165e6
     loss, g, lg = run_step(ctx, wl, inp)
-    # the top layer's q/k gradients sit at the bf16 noise floor here (the oracle's bf16 mode is
-    # ~2.5% max-rel from its exact mode on them): bounded by that floor where it exceeds 2e-2
-    _check_against_oracle(wl, inp, loss, g, lg, ctx, exact_too=False, noise_floor=True)
+    worst = _check_against_oracle(wl, inp, loss, g, lg, ctx)
+    print("layer above 165 MB: worst gradient tensors (layer, proj, A/B, cosine, max-rel):", worst)
     ctx.close()
 
 
@@ -287,7 +280,8 @@ def test_full_size_llama8b_layer_against_oracle():
     loss_r, g_r, _ = run_step(ctx_r, wl, inp)
     ctx_r.close()
     assert np.float32(loss).tobytes() == np.float32(loss_r).tobytes() and g.tobytes() == g_r.tobytes()
-    _check_against_oracle(wl, inp, loss, g, None, ctx, exact_too=False)
+    worst = _check_against_oracle(wl, inp, loss, g, None, ctx)
+    print("full-size 8B layer: worst gradient tensors (layer, proj, A/B, cosine, max-rel):", worst)
 
 
 @pytest.mark.parametrize("name", ["tiny", "tiny_gqa_bias_bf16"])
@@ -372,3 +366,49 @@ def test_adamw_step_matches_oracle_and_trains():
     assert losses[-1] < losses[0]
     assert all(b < a for a, b in zip(losses, losses[1:]))
     ctx.close()
+
+
+def test_read_timeline_orders_copies_before_compute():
+    # the per-read timeline of a profiled step: 2L reads in order, every read's compute starts after
+    # its copy (and dequant) started and ends after they ended; a copy into a slot starts only once
+    # the read two earlier, which computed from that slot, has finished
+    wl = syn.WORKLOADS["tiny"].with_(n_layers=3)
+    inp = build_inputs(wl)
+    ctx = make_context(wl, inp, streamed=True)
+    ctx.set_profiling(True)
+    run_step(ctx, wl, inp, want_logits=False)
+    tl = ctx.read_timeline()
+    ctx.close()
+    L = wl.n_layers
+    assert [r["layer"] for r in tl] == list(range(L)) + list(range(L - 1, -1, -1))
+    assert [r["kind"] for r in tl] == ["forward"] * L + ["backward"] * L
+    eps = 1e-3
+    for n, r in enumerate(tl):
+        c0, c1 = r["copy"]
+        d0, d1 = r["dequant"]
+        k0, k1 = r["compute"]
+        assert None not in (c0, c1, d0, d1, k0, k1)
+        assert 0 <= c0 <= c1 and c0 <= d0 + eps and d0 <= d1 and c0 <= k0 + eps and k0 <= k1
+        assert c1 <= k1 + eps and d1 <= k1 + eps
+        if n >= 2:
+            assert tl[n - 2]["compute"][1] <= c0 + eps
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama8b_layer_T256"])
+def test_dequant_inside_gemm_same_bytes(name):
+    # NF4 dequantised inside the GEMMs (mode 1) instead of a separate pass into a bf16 scratch: the
+    # same operand bits and the same GEMM order, so the same loss and gradient bytes; the tiny stack
+    # mixes both (its down projection has 688-wide rows, not whole NF4 blocks, and keeps the pass)
+    wl = WORKLOADS[name]
+    inp = build_inputs(wl)
+    out = []
+    for mode in (0, 1, 0):
+        ctx = make_context(wl, inp, streamed=True, reuse=True)
+        ctx.set_dequant_mode(mode)
+        res = [run_step(ctx, wl, inp, want_logits=False)[:2] for _ in range(2)]
+        ctx.close()
+        out.append(res)
+    for res in out[1:]:
+        for (la, ga), (lb, gb) in zip(out[0], res):
+            assert np.float32(la).tobytes() == np.float32(lb).tobytes()
+            assert ga.tobytes() == gb.tobytes()
