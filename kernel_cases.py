@@ -3,12 +3,11 @@
     python kernel_cases.py CASE [--iters N] [--warmup W]
 
 Cases are the shapes of the Llama-3.1-8B-shaped layer at batch 4 x seq 512 (T = 2048 tokens):
-  gemm_qkv     fused q/k/v projection: [2048, 4096] x [6144, 4096]^T + LoRA block (K + 64)
-  gemm_gu      fused gate/up projection: [2048, 4096] x [28672, 4096]^T + LoRA block
-  gemm_dx_gu   dX of gate/up: [2048, 28672] x [28672, 4096] (MN-major W) + LoRA block
-  gemm_dx_down dX of down: [2048, 4096] x [4096, 14336] (MN-major W) + LoRA block
-  gemm_*_nf4   the same four GEMMs with W dequantised from NF4 inside the GEMM (3 weight copies
-               rotated so every launch reads its codes from HBM)
+  gemm_*       every GEMM shape of a step (GEMM_SHAPES): the q/k/v, o, gate/up and down
+               projections with their LoRA block, their dX, and the LM head's two GEMMs
+  gemm_{qkv,gu,dx_gu,dx_down}_nf4
+               four of them with W dequantised from NF4 inside the GEMM (3 weight copies rotated
+               so every launch reads its codes from HBM)
   dequant_gu   NF4 -> bf16 of the gate/up group alone (2 x 14336 x 4096 elements)
   dequant      NF4 -> bf16 of one 8B layer (218 M elements, 7 tensors)
   attn_fwd     causal GQA attention forward, 4 x 512, 32/8 heads, hd 128
@@ -40,6 +39,26 @@ from layer_streamed_qlora_streaming_b200 import (k_attention_bwd, k_attention_fw
                k_nf4_quantize)
 
 T, D, F, HQ, HKV, HD, S = 2048, 4096, 14336, 32, 8, 128, 512
+VOCAB = 128256
+
+# Every GEMM of a training step of the 8B-shaped stack: (M, N, K, B MN-major, extra K of the LoRA
+# block, fp32 output, fp32 residual added), and how many times one step launches it.
+GEMM_SHAPES = {
+    "gemm_qkv": (T, 6144, D, 0, 192, 0, 0),        # q/k/v forward (bias, RoPE in the step)
+    "gemm_o": (T, D, D, 0, 64, 1, 1),              # o forward + residual
+    "gemm_gu": (T, 2 * F, D, 0, 128, 0, 0),        # gate/up forward
+    "gemm_down": (T, D, F, 0, 64, 1, 1),           # down forward + residual
+    "gemm_dx_down": (T, F, D, 1, 64, 1, 0),        # dX of down
+    "gemm_dx_gu": (T, D, 2 * F, 1, 128, 1, 0),     # dX of gate/up
+    "gemm_dx_o": (T, D, D, 1, 64, 0, 0),           # dX of o (bf16 output)
+    "gemm_dx_qkv": (T, D, 6144, 1, 192, 1, 0),     # dX of q/k/v
+    "gemm_head": (T, VOCAB, D, 0, 0, 1, 0),        # logits
+    "gemm_dx_head": (T, D, VOCAB, 1, 0, 1, 0),     # dlogits H
+}
+# per step of the 32-layer stack: forward reads run 4 projection GEMMs, backward reads recompute 3
+# (the down projection's output is not needed) and run 4 dX GEMMs, and the head runs 2
+GEMM_LAUNCHES_PER_STEP = {"gemm_qkv": 64, "gemm_o": 64, "gemm_gu": 64, "gemm_down": 32, "gemm_dx_down": 32,
+                          "gemm_dx_gu": 32, "gemm_dx_o": 32, "gemm_dx_qkv": 32, "gemm_head": 1, "gemm_dx_head": 1}
 
 
 def _bf(shape, g, scale=1.0):
@@ -66,23 +85,22 @@ def build(case: str):
     g.manual_seed(0)
     if case.startswith("gemm") and case.endswith("_nf4"):
         base = case[:-4]
-        M, N, K, bmn = {"gemm_qkv": (T, 6144, D, 0), "gemm_gu": (T, 2 * F, D, 0),
-                        "gemm_dx_gu": (T, D, 2 * F, 1), "gemm_dx_down": (T, F, D, 1)}[base]
+        M, N, K, bmn, K2, f32, _ = GEMM_SHAPES[base]
         rows = {"gemm_qkv": [4096, 1024, 1024], "gemm_gu": [F, F], "gemm_dx_gu": [F, F], "gemm_dx_down": [D]}[base]
         cols = K if bmn == 0 else N
         copies = [_nf4(rows, cols, g) for _ in range(3)]
         A = _bf((M, K), g)
-        A2 = _bf((M, 64), g)
-        B2 = _bf((64, N) if bmn else (N, 64), g, 0.01)
-        C = torch.empty(M, N, dtype=torch.float32 if bmn else torch.bfloat16, device="cuda")
+        A2 = _bf((M, K2), g)
+        B2 = _bf((K2, N) if bmn else (N, K2), g, 0.01)
+        C = torch.empty(M, N, dtype=torch.float32 if f32 else torch.bfloat16, device="cuda")
         state = {"i": 0}
 
         def run():
             parts = copies[state["i"] % len(copies)]
             state["i"] += 1
-            k_gemm_nf4(M, N, K, A, K, parts, bmn, C, N, int(bmn), A2=A2, lda2=64, B2=B2,
-                       ldb2=N if bmn else 64, K2=64)
-        return run, {"flop": 2.0 * M * N * (K + 64), "bytes": None}
+            k_gemm_nf4(M, N, K, A, K, parts, bmn, C, N, int(f32), A2=A2, lda2=K2, B2=B2,
+                       ldb2=N if bmn else K2, K2=K2)
+        return run, {"flop": 2.0 * M * N * (K + K2), "bytes": None}
     if case == "dequant_gu":
         n = 2 * F * D
         w = torch.randn(n, generator=g, device="cuda") * 0.02
@@ -98,19 +116,18 @@ def build(case: str):
             k_nf4_dequant(packed, qabs, gs, mean, n, out)
         return run, {"flop": None, "bytes": n * (0.5 + 1 / 64 + 2)}
     if case.startswith("gemm"):
-        spec = {"gemm_qkv": (T, 6144, D, 0), "gemm_gu": (T, 2 * F, D, 0),
-                "gemm_dx_gu": (T, D, 2 * F, 1), "gemm_dx_down": (T, F, D, 1)}[case]
-        M, N, K, bmn = spec
+        M, N, K, bmn, K2, f32, resid = GEMM_SHAPES[case]
         A = _bf((M, K), g)
         B = _bf((K, N) if bmn else (N, K), g, 0.02)
-        A2 = _bf((M, 64), g)
-        B2 = _bf((64, N) if bmn else (N, 64), g, 0.01)
-        C = torch.empty(M, N, dtype=torch.float32 if bmn else torch.bfloat16, device="cuda")
+        A2 = _bf((M, K2), g) if K2 else None
+        B2 = (_bf((K2, N) if bmn else (N, K2), g, 0.01)) if K2 else None
+        C = torch.empty(M, N, dtype=torch.float32 if f32 else torch.bfloat16, device="cuda")
+        R = torch.randn(M, N, generator=g, device="cuda") if resid else None
 
         def run():
-            k_gemm(M, N, K, A, K, B, N if bmn else K, bmn, C, N, int(bmn), A2=A2, lda2=64, B2=B2,
-                   ldb2=N if bmn else 64, K2=64)
-        return run, {"flop": 2.0 * M * N * (K + 64), "bytes": None}
+            k_gemm(M, N, K, A, K, B, N if bmn else K, bmn, C, N, int(f32), A2=A2, lda2=K2, B2=B2,
+                   ldb2=(N if bmn else K2), K2=K2, R=R, ldr=N if resid else 0)
+        return run, {"flop": 2.0 * M * N * (K + K2), "bytes": None}
     if case == "dequant":
         n = 4096 * 4096 * 2 + 1024 * 4096 * 2 + 14336 * 4096 * 3
         w = torch.randn(n, generator=g, device="cuda") * 0.02

@@ -12,8 +12,13 @@
 // blocks with the most work are scheduled first.
 #include "attention.cuh"
 #include "common.cuh"
+#include "gemm.cuh"
 
 #include <cuda_fp16.h>
+
+#include <atomic>
+#include <cstdlib>
+#include <cstring>
 
 namespace lst {
 namespace {
@@ -324,6 +329,801 @@ __global__ void __launch_bounds__(128) k_attn_fwd(AttnArgs p) {
         *reinterpret_cast<float2*>(o32 + i * 8 + 2 * t4) = make_float2(o[i][2 * r] * inv, o[i][2 * r + 1] * inv);
     }
     if (t4 == 0) p.lse[(tok0 + qr) * p.hq + h] = (mrow[r] + log2f(lrow[r])) / kLog2e;
+  }
+}
+
+// ------------------------------------------------------------------------------------ forward, tcgen05
+// One CTA per 128 queries of one head (the last query blocks, with the most keys, first); 192
+// threads: warp 0 TMA producer (Q once; K and V tiles of 128 keys, double-buffered), warp 1 MMA
+// issuer, warps 2-5 softmax (one thread per query row, TMEM lane = row).
+//   S = Q K^T           tcgen05, bf16 operands, fp32 in one of two TMEM buffers (so the next block's
+//                       Q K^T runs while this block's softmax reads its scores);
+//   P = exp2(S' - m)    softmax threads, written as fp16 to a 128-byte-swizzled shared tile (the
+//                       MMA's A operand) -- the V tile is converted to fp16 in place meanwhile;
+//   O += P V            tcgen05, fp16 operands (V MN-major), fp32 accumulator in TMEM.
+// The reference max m of a row only moves when the block's max exceeds it by more than 2^8 (then O
+// is rescaled in TMEM), so P <= 256 and every value of P is exact to fp16's precision; the final
+// O / l and lse use the same m and l. Every wait is bounded.
+template <int HD>
+struct AttnTc {
+  static constexpr int QB = 128, KB = 128;
+  static constexpr uint32_t CH = 128 * 128;               // bytes of one [128 rows x 64] bf16 chunk
+  static constexpr uint32_t Q_BYTES = (HD / 64) * CH;
+  static constexpr uint32_t KV_BYTES = 2 * (HD / 64) * CH; // K then V of one stage
+  static constexpr uint32_t P_BYTES = 2 * CH;              // 128 queries x 128 keys fp16
+  static constexpr uint32_t SMEM = Q_BYTES + 2 * KV_BYTES + P_BYTES + 1024 + 256;
+  static constexpr uint32_t TMEM_COLS = 512;              // S[2] at columns 0 / 128, O at 256
+};
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const AttnArgs p) {
+  using C = AttnTc<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + C::Q_BYTES;        // [2] stages: K chunks, then V chunks
+  uint8_t* sP = sKV + 2 * C::KV_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + C::P_BYTES);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_free = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* pv_done = bars + 10;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+
+  const int h = blockIdx.x, b = blockIdx.y, qb = (int)gridDim.z - 1 - (int)blockIdx.z;
+  const int kvh = h / (p.hq / p.hkv);
+  const int64_t tok0 = (int64_t)b * p.S;
+  const int q0 = qb * C::QB;
+  const int nkb = qb + 1;  // key blocks 0 .. qb (the causal mask ends inside block qb)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < HD / 64; ++c)
+        tma_load_2d(sQ + c * C::CH, &tmQ, q_full, h * HD + c * 64, (int32_t)(tok0 + q0));
+      for (int j = 0; j < nkb; ++j) {
+        const int st = j & 1;
+        if (j >= 2 && !mbar_wait(&kv_empty[st], ((j - 2) >> 1) & 1)) break;
+        uint8_t* sk = sKV + st * C::KV_BYTES;
+        mbar_arrive_expect_tx(&kv_full[st], C::KV_BYTES);
+        const int32_t y = (int32_t)(tok0 + j * C::KB);
+#pragma unroll
+        for (int c = 0; c < HD / 64; ++c) {
+          tma_load_2d(sk + c * C::CH, &tmK, &kv_full[st], kvh * HD + c * 64, y);
+          tma_load_2d(sk + (HD / 64 + c) * C::CH, &tmV, &kv_full[st], kvh * HD + c * 64, y);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idS = umma_idesc_bf16(128, C::KB, 0, 0);
+      constexpr uint32_t idO = umma_idesc_f16(128, HD, 0, 1);
+      bool ok = mbar_wait(q_full, 0);
+      for (int j = 0; j <= nkb && ok; ++j) {
+        if (j < nkb) {  // S_j = Q K_j^T into buffer j & 1
+          const int st = j & 1;
+          if (!mbar_wait(&kv_full[st], (j >> 1) & 1)) break;
+          if (j >= 2 && !mbar_wait(&s_free[st], ((j - 2) >> 1) & 1)) break;
+          tc_fence_after();
+          const uint32_t q = smem_u32(sQ), k = smem_u32(sKV + st * C::KV_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::CH + (kk & 3) * 32;
+            umma_bf16(tmem + st * C::KB, umma_desc(q + off, 16, 1024), umma_desc(k + off, 16, 1024), idS, kk != 0);
+          }
+          umma_commit(&s_full[st]);
+        }
+        if (j >= 1) {  // O += P_{j-1} V_{j-1}
+          const int i = j - 1, st = i & 1;
+          if (!mbar_wait(p_full, i & 1)) break;
+          tc_fence_after();
+          const uint32_t pa = smem_u32(sP), v = smem_u32(sKV + st * C::KV_BYTES + (HD / 64) * C::CH);
+#pragma unroll
+          for (int kk = 0; kk < C::KB / 16; ++kk) {
+            const uint64_t da = umma_desc(pa + (kk >> 2) * C::CH + (kk & 3) * 32, 16, 1024);
+            const uint64_t db = umma_desc(v + kk * 16 * 128, C::CH, 1024);  // 16 key rows per step
+            umma_bf16(tmem + 256, da, db, idO, (i | kk) != 0);
+          }
+          umma_commit(&kv_empty[st]);
+          umma_commit(pv_done);
+        }
+      }
+    }
+  } else {
+    const int r = (warp & 3) * 32 + lane;  // query row of this thread = its TMEM lane
+    const int qrow = q0 + r;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const float sl2 = p.scale * kLog2e;
+    float mref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkb && ok; ++j) {
+      const int st = j & 1;
+      // V_j to fp16 in place (this thread's 16-byte pieces), once its TMA has landed
+      if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[st], (j >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      {
+        uint4* vt = reinterpret_cast<uint4*>(sKV + st * C::KV_BYTES + (HD / 64) * C::CH);
+        for (int i = r; i < (int)((HD / 64) * C::CH / 16); i += 128) {
+          uint4 u = vt[i];
+          uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+            w[e] = pack_f16(f.x, f.y);
+          }
+          vt[i] = u;
+        }
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float x[C::KB];
+#pragma unroll
+      for (int c = 0; c < C::KB; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(tmem + st * C::KB + c + lane_off, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[c + e] = __uint_as_float(u[e]) * sl2;
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[st]);
+      const bool diag = j == nkb - 1;
+      float bm = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < C::KB; ++e) {
+        const int key = j * C::KB + e;
+        if (diag && (key > qrow || key >= p.S)) x[e] = -INFINITY;
+        bm = fmaxf(bm, x[e]);
+      }
+      float corr = 1.f;
+      if (j == 0) {
+        mref = bm;
+      } else if (bm > mref + 8.f) {
+        corr = exp2f(mref - bm);
+        mref = bm;
+      }
+      float rs = 0.f;
+#pragma unroll
+      for (int e = 0; e < C::KB; ++e) {
+        x[e] = exp2f(x[e] - mref);
+        rs += x[e];
+      }
+      l = l * corr + rs;
+      if (j >= 1) {  // P_{j-1} V_{j-1} done: the P tile is free and O holds the blocks so far
+        if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, corr != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < HD; c += 32) {
+            uint32_t u[32];
+            tmem_ld32(tmem + 256 + c + lane_off, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * corr);
+            tmem_st32(tmem + 256 + c + lane_off, u);
+          }
+          tmem_st_wait();
+        }
+      }
+      // P row r: keys 0-63 in chunk 0, 64-127 in chunk 1; 16-byte piece i of a row at i ^ (r & 7)
+#pragma unroll
+      for (int kc = 0; kc < 2; ++kc) {
+        uint8_t* row = sP + kc * C::CH + r * 128;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float* v = x + kc * 64 + i * 8;
+          uint4 u = make_uint4(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]), pack_f16(v[4], v[5]),
+                               pack_f16(v[6], v[7]));
+          *reinterpret_cast<uint4*>(row + ((i ^ (r & 7)) * 16)) = u;
+        }
+      }
+      fence_proxy_async();  // P and the converted V are read by the tensor core
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    // O / l, lse
+    if (ok && __all_sync(0xffffffffu, mbar_wait(pv_done, (nkb - 1) & 1))) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      const bool live = qrow < p.S;
+      __nv_bfloat16* op = p.o + (tok0 + qrow) * p.ldo + h * HD;
+      float* o32 = p.o32 ? p.o32 + (tok0 + qrow) * (int64_t)p.hq * HD + h * HD : nullptr;
+#pragma unroll
+      for (int c = 0; c < HD; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(tmem + 256 + c + lane_off, u);
+        tmem_ld_wait();
+        if (live) {
+          float v[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(u[e]) * inv;
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w = make_uint4(pack_bf16(v[e], v[e + 1]), pack_bf16(v[e + 2], v[e + 3]),
+                                 pack_bf16(v[e + 4], v[e + 5]), pack_bf16(v[e + 6], v[e + 7]));
+            *reinterpret_cast<uint4*>(op + c + e) = w;
+            if (o32) {
+              *reinterpret_cast<float4*>(o32 + c + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+              *reinterpret_cast<float4*>(o32 + c + e + 4) = make_float4(v[e + 4], v[e + 5], v[e + 6], v[e + 7]);
+            }
+          }
+        }
+      }
+      if (live) p.lse[(tok0 + qrow) * p.hq + h] = (mref + log2f(l)) / kLog2e;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// --------------------------------------------------------------------------- backward: dQ, tcgen05
+// One CTA per 128 queries of one head (heaviest first), 192 threads: warp 0 TMA (Q and dO once; K
+// and V tiles of 64 keys, double-buffered), warp 1 MMA issuer, warps 2-5 one thread per query row.
+//   S = Q K^T, dP = dO V^T   tcgen05 (bf16), into one of two TMEM buffer pairs;
+//   dS = P (dP - D)          the row's threads, P = exp2(S' - lse'), written bf16 to a swizzled tile;
+//   dQ += dS K               tcgen05 (K read MN-major from the same tile), fp32 in TMEM;
+// then dQ * scale with the rotary embedding undone is stored once as bf16.
+template <int HD>
+struct DqTc {
+  static constexpr int QB = 128, KB = 64;
+  static constexpr uint32_t CH = 128 * 128;                  // [128 rows x 64] bf16 chunk
+  static constexpr uint32_t KCH = 64 * 128;                  // [64 rows x 64] bf16 chunk
+  static constexpr uint32_t Q_BYTES = (HD / 64) * CH;
+  static constexpr uint32_t KV_BYTES = 2 * (HD / 64) * KCH;  // K then V of one stage
+  static constexpr uint32_t DS_BYTES = CH;                   // 128 queries x 64 keys bf16
+  static constexpr uint32_t SMEM = 2 * Q_BYTES + 2 * KV_BYTES + DS_BYTES + 1024 + 256;
+  static constexpr uint32_t TMEM_COLS = 512;                 // S[2] at 0/64, dP[2] at 128/192, dQ at 256
+};
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+             const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const AttnBwdArgs p) {
+  using C = DqTc<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sO = sQ + C::Q_BYTES;          // dO
+  uint8_t* sKV = sO + C::Q_BYTES;         // [2] stages: K chunks, then V chunks
+  uint8_t* sDS = sKV + 2 * C::KV_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + C::DS_BYTES);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_free = bars + 7;    // [2]
+  uint64_t* ds_full = bars + 9;
+  uint64_t* dq_done = bars + 10;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+
+  const int h = blockIdx.x, b = blockIdx.y, qb = (int)gridDim.z - 1 - (int)blockIdx.z;
+  const int kvh = h / (p.hq / p.hkv);
+  const int64_t tok0 = (int64_t)b * p.S;
+  const int q0 = qb * C::QB;
+  const int nkb = min((q0 + C::QB + C::KB - 1) / C::KB, (p.S + C::KB - 1) / C::KB);  // keys < q0 + 128 and < S
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+    }
+    mbar_init(ds_full, 128);
+    mbar_init(dq_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmO);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * C::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < HD / 64; ++c) {
+        tma_load_2d(sQ + c * C::CH, &tmQ, q_full, h * HD + c * 64, (int32_t)(tok0 + q0));
+        tma_load_2d(sO + c * C::CH, &tmO, q_full, h * HD + c * 64, (int32_t)(tok0 + q0));
+      }
+      for (int j = 0; j < nkb; ++j) {
+        const int st = j & 1;
+        if (j >= 2 && !mbar_wait(&kv_empty[st], ((j - 2) >> 1) & 1)) break;
+        uint8_t* sk = sKV + st * C::KV_BYTES;
+        mbar_arrive_expect_tx(&kv_full[st], C::KV_BYTES);
+        const int32_t y = (int32_t)(tok0 + j * C::KB);
+#pragma unroll
+        for (int c = 0; c < HD / 64; ++c) {
+          tma_load_2d(sk + c * C::KCH, &tmK, &kv_full[st], kvh * HD + c * 64, y);
+          tma_load_2d(sk + (HD / 64 + c) * C::KCH, &tmV, &kv_full[st], kvh * HD + c * 64, y);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idS = umma_idesc_bf16(128, C::KB, 0, 0);
+      constexpr uint32_t idQ = umma_idesc_bf16(128, HD, 0, 1);
+      bool ok = mbar_wait(q_full, 0);
+      for (int j = 0; j <= nkb && ok; ++j) {
+        if (j < nkb) {  // S_j = Q K_j^T and dP_j = dO V_j^T into buffer pair j & 1
+          const int st = j & 1;
+          if (!mbar_wait(&kv_full[st], (j >> 1) & 1)) break;
+          if (j >= 2 && !mbar_wait(&s_free[st], ((j - 2) >> 1) & 1)) break;
+          tc_fence_after();
+          const uint32_t q = smem_u32(sQ), o = smem_u32(sO);
+          const uint32_t k = smem_u32(sKV + st * C::KV_BYTES), v = k + (HD / 64) * C::KCH;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t offq = (kk >> 2) * C::CH + (kk & 3) * 32, offk = (kk >> 2) * C::KCH + (kk & 3) * 32;
+            umma_bf16(tmem + st * C::KB, umma_desc(q + offq, 16, 1024), umma_desc(k + offk, 16, 1024), idS, kk != 0);
+            umma_bf16(tmem + 128 + st * C::KB, umma_desc(o + offq, 16, 1024), umma_desc(v + offk, 16, 1024), idS,
+                      kk != 0);
+          }
+          umma_commit(&s_full[st]);
+        }
+        if (j >= 1) {  // dQ += dS_{j-1} K_{j-1}
+          const int i = j - 1, st = i & 1;
+          if (!mbar_wait(ds_full, i & 1)) break;
+          tc_fence_after();
+          const uint32_t ds = smem_u32(sDS), k = smem_u32(sKV + st * C::KV_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < C::KB / 16; ++kk) {
+            const uint64_t da = umma_desc(ds + kk * 32, 16, 1024);
+            const uint64_t db = umma_desc(k + kk * 16 * 128, C::KCH, 1024);  // K rows = keys: MN-major
+            umma_bf16(tmem + 256, da, db, idQ, (i | kk) != 0);
+          }
+          umma_commit(&kv_empty[st]);
+          umma_commit(dq_done);
+        }
+      }
+    }
+  } else {
+    const int r = (warp & 3) * 32 + lane;
+    const int qrow = q0 + r;
+    const bool live = qrow < p.S;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const float sl2 = p.scale * kLog2e;
+    const float lse2 = live ? p.lse[(tok0 + qrow) * p.hq + h] * kLog2e : 0.f;
+    const float dd = live ? p.D[(tok0 + qrow) * p.hq + h] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkb && ok; ++j) {
+      const int st = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float ds[C::KB];
+      {
+        uint32_t us[32], ud[32];
+#pragma unroll
+        for (int c = 0; c < C::KB; c += 32) {
+          tmem_ld32(tmem + st * C::KB + c + lane_off, us);
+          tmem_ld32(tmem + 128 + st * C::KB + c + lane_off, ud);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int key = j * C::KB + c + e;
+            float pv = exp2f(__uint_as_float(us[e]) * sl2 - lse2);
+            if (!live || key > qrow || key >= p.S) pv = 0.f;
+            ds[c + e] = pv * (__uint_as_float(ud[e]) - dd);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[st]);
+      if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(dq_done, (j - 1) & 1))) {  // the dS tile is free
+        ok = false;
+        break;
+      }
+      uint8_t* row = sDS + r * 128;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float* v = ds + i * 8;
+        uint4 u = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+        *reinterpret_cast<uint4*>(row + ((i ^ (r & 7)) * 16)) = u;
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(dq_done, (nkb - 1) & 1))) {
+      tc_fence_after();
+      // the whole dQ row (HD fp32), scaled, with the rotation of position qrow undone
+      float acc[HD];
+#pragma unroll
+      for (int c = 0; c < HD; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(tmem + 256 + c + lane_off, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[c + e] = __uint_as_float(u[e]) * p.scale;
+      }
+      if (live) {  // pairs (c, c + hd/2) rotated by minus the angle of position qrow, 8 columns at a time
+        constexpr int HALF = HD / 2;
+        __nv_bfloat16* dst = p.dq + (tok0 + qrow) * p.lddq + h * HD;
+#pragma unroll
+        for (int c0 = 0; c0 < HALF; c0 += 8) {
+          float y1[8], y2[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float x1 = acc[c0 + e], x2 = acc[c0 + e + HALF];
+            if (p.rope_cos) {
+              const float cs = p.rope_cos[qrow * HALF + c0 + e], sn = p.rope_sin[qrow * HALF + c0 + e];
+              y1[e] = x1 * cs + x2 * sn;
+              y2[e] = x2 * cs - x1 * sn;
+            } else {
+              y1[e] = x1;
+              y2[e] = x2;
+            }
+          }
+          *reinterpret_cast<uint4*>(dst + c0) = make_uint4(pack_bf16(y1[0], y1[1]), pack_bf16(y1[2], y1[3]),
+                                                           pack_bf16(y1[4], y1[5]), pack_bf16(y1[6], y1[7]));
+          *reinterpret_cast<uint4*>(dst + c0 + HALF) = make_uint4(pack_bf16(y2[0], y2[1]), pack_bf16(y2[2], y2[3]),
+                                                                  pack_bf16(y2[4], y2[5]), pack_bf16(y2[6], y2[7]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// --------------------------------------------------------------------------- backward: dK, dV, tcgen05
+// grid (grp, B * hkv, ceil(S/128)), cluster (grp, 1, 1), 192 threads. The cluster owns 128 keys of
+// kv head kvh; its CTA of rank hh sums the contributions of query head kvh * grp + hh over query
+// blocks of 64 (double-buffered Q / dO tiles): warp 0 TMA, warp 1 MMA issuer, warps 2-5 one thread
+// per key row.
+//   S^T = K Q^T, dP^T = V dO^T      tcgen05 (bf16), into one of two TMEM buffer pairs;
+//   P^T, dS^T = P^T (dP^T - D)      the key row's thread (lse and D of the block's queries from
+//                                    shared memory), written bf16 to swizzled tiles;
+//   dV += P^T dO, dK += dS^T Q       tcgen05, with Q / dO read MN-major from the tiles used K-major above.
+// The grp partial dK / dV tiles are then parked in shared memory and CTA hh adds rows
+// [hh * 128/grp, ...) over the heads in order 0 .. grp-1 (distributed shared memory), scales dK,
+// undoes the rotary embedding and stores both. Deterministic, no atomics.
+template <int HD>
+struct DkvTc {
+  static constexpr int KB = 128, QB = 64;
+  static constexpr uint32_t CH = 128 * 128;                  // [128 rows x 64] bf16
+  static constexpr uint32_t QCH = 64 * 128;                  // [64 rows x 64] bf16
+  static constexpr uint32_t K_BYTES = (HD / 64) * CH;
+  static constexpr uint32_t QO_BYTES = 2 * (HD / 64) * QCH;  // Q then dO of one stage
+  static constexpr uint32_t T_BYTES = 128 * 128;             // one [128 keys x 64 queries] bf16 tile
+  static constexpr int RLD = HD + 4;                         // fp32 row stride of a parked tile
+  static constexpr uint32_t MAIN = 2 * K_BYTES + 2 * QO_BYTES + 2 * T_BYTES + 2 * 2 * QB * 4;
+  static constexpr uint32_t PARK = 2 * 128 * RLD * 4;
+  static constexpr uint32_t SMEM = (MAIN > PARK ? MAIN : PARK) + 1024 + 256;
+  static constexpr uint32_t TMEM_COLS = 2 * 128 + 2 * HD <= 256 ? 256 : 512;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const AttnBwdArgs p) {
+  using C = DkvTc<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + C::K_BYTES;
+  uint8_t* sQO = sV + C::K_BYTES;               // [2] stages: Q chunks, then dO chunks
+  uint8_t* sP = sQO + 2 * C::QO_BYTES;          // P^T tile
+  uint8_t* sS = sP + C::T_BYTES;                // dS^T tile
+  float* sLse = reinterpret_cast<float*>(sS + C::T_BYTES);  // [2][64]
+  float* sD = sLse + 2 * C::QB;                             // [2][64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (C::MAIN > C::PARK ? C::MAIN : C::PARK));
+  uint64_t* kv_full = bars;
+  uint64_t* qo_full = bars + 1;   // [2]
+  uint64_t* qo_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_free = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* kv_done = bars + 10;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  float* redK = reinterpret_cast<float*>(smem);  // after the main loop: [128][RLD] each
+  float* redV = redK + 128 * C::RLD;
+
+  const int grp = (int)gridDim.x;
+  const int hh = (int)cluster_rank();
+  const int kvh = (int)blockIdx.y % p.hkv, b = (int)blockIdx.y / p.hkv, kb = (int)blockIdx.z;
+  const int h = kvh * grp + hh;
+  const int64_t tok0 = (int64_t)b * p.S;
+  const int k0 = kb * C::KB;
+  const int i0 = k0 / C::QB;                        // first query block with a query >= k0
+  const int nqb = (p.S + C::QB - 1) / C::QB - i0;   // query blocks of this CTA
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qo_full[i], 1);
+      mbar_init(&qo_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(kv_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmO);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tV = tmem + 256, tK = tmem + 256 + HD;  // dV, dK accumulators
+
+  bool ok = true;
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * C::K_BYTES);
+#pragma unroll
+      for (int c = 0; c < HD / 64; ++c) {
+        tma_load_2d(sK + c * C::CH, &tmK, kv_full, kvh * HD + c * 64, (int32_t)(tok0 + k0));
+        tma_load_2d(sV + c * C::CH, &tmV, kv_full, kvh * HD + c * 64, (int32_t)(tok0 + k0));
+      }
+      for (int j = 0; j < nqb; ++j) {
+        const int st = j & 1;
+        if (j >= 2 && !mbar_wait(&qo_empty[st], ((j - 2) >> 1) & 1)) break;
+        uint8_t* sq = sQO + st * C::QO_BYTES;
+        mbar_arrive_expect_tx(&qo_full[st], C::QO_BYTES);
+        const int32_t y = (int32_t)(tok0 + (i0 + j) * C::QB);
+#pragma unroll
+        for (int c = 0; c < HD / 64; ++c) {
+          tma_load_2d(sq + c * C::QCH, &tmQ, &qo_full[st], h * HD + c * 64, y);
+          tma_load_2d(sq + (HD / 64 + c) * C::QCH, &tmO, &qo_full[st], h * HD + c * 64, y);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idS = umma_idesc_bf16(128, C::QB, 0, 0);
+      constexpr uint32_t idG = umma_idesc_bf16(128, HD, 0, 1);
+      bool okm = mbar_wait(kv_full, 0);
+      for (int j = 0; j <= nqb && okm; ++j) {
+        if (j < nqb) {  // S^T_j = K Q_j^T, dP^T_j = V dO_j^T into buffer pair j & 1
+          const int st = j & 1;
+          if (!mbar_wait(&qo_full[st], (j >> 1) & 1)) break;
+          if (j >= 2 && !mbar_wait(&s_free[st], ((j - 2) >> 1) & 1)) break;
+          tc_fence_after();
+          const uint32_t k = smem_u32(sK), v = smem_u32(sV);
+          const uint32_t q = smem_u32(sQO + st * C::QO_BYTES), o = q + (HD / 64) * C::QCH;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t offk = (kk >> 2) * C::CH + (kk & 3) * 32, offq = (kk >> 2) * C::QCH + (kk & 3) * 32;
+            umma_bf16(tmem + st * C::QB, umma_desc(k + offk, 16, 1024), umma_desc(q + offq, 16, 1024), idS, kk != 0);
+            umma_bf16(tmem + 128 + st * C::QB, umma_desc(v + offk, 16, 1024), umma_desc(o + offq, 16, 1024), idS,
+                      kk != 0);
+          }
+          umma_commit(&s_full[st]);
+        }
+        if (j >= 1) {  // dV += P^T dO, dK += dS^T Q of block j-1
+          const int i = j - 1, st = i & 1;
+          if (!mbar_wait(p_full, i & 1)) break;
+          tc_fence_after();
+          const uint32_t pt = smem_u32(sP), ds = smem_u32(sS);
+          const uint32_t q = smem_u32(sQO + st * C::QO_BYTES), o = q + (HD / 64) * C::QCH;
+#pragma unroll
+          for (int kk = 0; kk < C::QB / 16; ++kk) {
+            umma_bf16(tV, umma_desc(pt + kk * 32, 16, 1024), umma_desc(o + kk * 16 * 128, C::QCH, 1024), idG,
+                      (i | kk) != 0);
+            umma_bf16(tK, umma_desc(ds + kk * 32, 16, 1024), umma_desc(q + kk * 16 * 128, C::QCH, 1024), idG,
+                      (i | kk) != 0);
+          }
+          umma_commit(&qo_empty[st]);
+          umma_commit(kv_done);
+        }
+      }
+    }
+  } else {
+    const int t = (int)threadIdx.x - 64;   // 0 .. 127
+    const int r = (warp & 3) * 32 + lane;  // key row = TMEM lane
+    const int kr = k0 + r;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const float sl2 = p.scale * kLog2e;
+    // every iteration reaches the named barrier (the four warps together), also after a failed wait
+    for (int j = 0; j < nqb; ++j) {
+      const int st = j & 1;
+      const int q0 = (i0 + j) * C::QB;
+      if (t < C::QB) {  // the block's lse (log2 domain) and D, shared by every key row
+        const int qr = q0 + t;
+        const bool in = qr < p.S;
+        sLse[st * C::QB + t] = in ? p.lse[(tok0 + qr) * p.hq + h] * kLog2e : 0.f;
+        sD[st * C::QB + t] = in ? p.D[(tok0 + qr) * p.hq + h] : 0.f;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!ok) continue;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1))) {
+        ok = false;
+        continue;
+      }
+      tc_fence_after();
+      float pv[C::QB], dv[C::QB];
+      {
+        uint32_t us[32], ud[32];
+#pragma unroll
+        for (int c = 0; c < C::QB; c += 32) {
+          tmem_ld32(tmem + st * C::QB + c + lane_off, us);
+          tmem_ld32(tmem + 128 + st * C::QB + c + lane_off, ud);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int q = q0 + c + e;
+            float pe = exp2f(__uint_as_float(us[e]) * sl2 - sLse[st * C::QB + c + e]);
+            if (q < kr || q >= p.S || kr >= p.S) pe = 0.f;
+            pv[c + e] = pe;
+            dv[c + e] = pe * (__uint_as_float(ud[e]) - sD[st * C::QB + c + e]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[st]);
+      if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(kv_done, (j - 1) & 1))) {  // P^T / dS^T tiles free
+        ok = false;
+        continue;
+      }
+      uint8_t* prow = sP + r * 128;
+      uint8_t* srow = sS + r * 128;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float* a = pv + i * 8;
+        const float* d = dv + i * 8;
+        const int pos = (i ^ (r & 7)) * 16;
+        *reinterpret_cast<uint4*>(prow + pos) =
+            make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
+        *reinterpret_cast<uint4*>(srow + pos) =
+            make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]), pack_bf16(d[4], d[5]), pack_bf16(d[6], d[7]));
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    // park this head's dK, dV rows (fp32) once the last block's MMAs are done
+    if (ok && __all_sync(0xffffffffu, mbar_wait(kv_done, (nqb - 1) & 1))) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < HD; c += 32) {
+        uint32_t uk[32], uv[32];
+        tmem_ld32(tK + c + lane_off, uk);
+        tmem_ld32(tV + c + lane_off, uv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          *reinterpret_cast<float4*>(redK + r * C::RLD + c + e) =
+              make_float4(__uint_as_float(uk[e]), __uint_as_float(uk[e + 1]), __uint_as_float(uk[e + 2]),
+                          __uint_as_float(uk[e + 3]));
+          *reinterpret_cast<float4*>(redV + r * C::RLD + c + e) =
+              make_float4(__uint_as_float(uv[e]), __uint_as_float(uv[e + 1]), __uint_as_float(uv[e + 2]),
+                          __uint_as_float(uv[e + 3]));
+        }
+      }
+    } else {
+      ok = false;
+    }
+  }
+  // (the tiles the parked rows overwrite are no longer read: every MMA completed before kv_done)
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();  // every head's partial tile is parked
+
+  constexpr int HALF = HD / 2;
+  const int rows = (C::KB + grp - 1) / grp;
+  const int rbeg = hh * rows, rend = min(C::KB, rbeg + rows);
+  const uint32_t rk0 = smem_u32(redK), rv0 = smem_u32(redV);
+  for (int item = threadIdx.x; item < (rend - rbeg) * (HALF / 2); item += blockDim.x) {
+    const int row = rbeg + item / (HALF / 2);
+    const int c = (item % (HALF / 2)) * 2;  // columns c, c+1 and their rotary partners c+HALF, c+HALF+1
+    const int kr = k0 + row;
+    const uint32_t o1 = (uint32_t)((row * C::RLD + c) * 4), o2 = (uint32_t)((row * C::RLD + c + HALF) * 4);
+    float2 a1[kMaxGroup], a2[kMaxGroup], b1[kMaxGroup], b2[kMaxGroup];
+#pragma unroll
+    for (int q = 0; q < kMaxGroup; ++q) {
+      if (q < grp) {
+        a1[q] = ld_cluster_f2(cluster_map(rk0 + o1, (uint32_t)q));
+        a2[q] = ld_cluster_f2(cluster_map(rk0 + o2, (uint32_t)q));
+        b1[q] = ld_cluster_f2(cluster_map(rv0 + o1, (uint32_t)q));
+        b2[q] = ld_cluster_f2(cluster_map(rv0 + o2, (uint32_t)q));
+      }
+    }
+    float2 k1 = a1[0], k2 = a2[0], v1 = b1[0], v2 = b2[0];
+#pragma unroll
+    for (int q = 1; q < kMaxGroup; ++q) {
+      if (q < grp) {
+        k1.x += a1[q].x; k1.y += a1[q].y; k2.x += a2[q].x; k2.y += a2[q].y;
+        v1.x += b1[q].x; v1.y += b1[q].y; v2.x += b2[q].x; v2.y += b2[q].y;
+      }
+    }
+    if (kr >= p.S) continue;
+    __nv_bfloat16* vp = p.dv + (tok0 + kr) * p.lddv + kvh * HD;
+    *reinterpret_cast<__nv_bfloat162*>(vp + c) = __floats2bfloat162_rn(v1.x, v1.y);
+    *reinterpret_cast<__nv_bfloat162*>(vp + c + HALF) = __floats2bfloat162_rn(v2.x, v2.y);
+    float y1[2] = {k1.x * p.scale, k1.y * p.scale}, y2[2] = {k2.x * p.scale, k2.y * p.scale};
+    if (p.rope_cos) {  // inverse rotation of key position kr: pairs (c + u, c + u + HALF)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float x1 = y1[u], x2 = y2[u];
+        const float cs = p.rope_cos[kr * HALF + c + u], sn = p.rope_sin[kr * HALF + c + u];
+        y1[u] = x1 * cs + x2 * sn;
+        y2[u] = x2 * cs - x1 * sn;
+      }
+    }
+    __nv_bfloat16* kp = p.dk + (tok0 + kr) * p.lddk + kvh * HD;
+    *reinterpret_cast<__nv_bfloat162*>(kp + c) = __floats2bfloat162_rn(y1[0], y1[1]);
+    *reinterpret_cast<__nv_bfloat162*>(kp + c + HALF) = __floats2bfloat162_rn(y2[0], y2[1]);
+  }
+  __syncwarp();
+  cluster_sync_all();  // no CTA leaves while another still reads its shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -654,11 +1454,46 @@ bool check_common(int hd, int hq, int hkv, int S, int64_t T) {
   return true;
 }
 
+template <int HD>
+cudaError_t launch_fwd_tc(const AttnArgs& a, int B, cudaStream_t s) {
+  using C = AttnTc<HD>;
+  CUtensorMap tQ, tK, tV;
+  if ((a.ldq % 8) || (a.ldk % 8) || (a.ldv % 8)) return cudaErrorInvalidValue;
+  if (!make_map(&tQ, a.q, a.T, (int64_t)a.hq * HD, a.ldq, C::QB)) return cudaErrorInvalidValue;
+  if (!make_map(&tK, a.k, a.T, (int64_t)a.hkv * HD, a.ldk, C::KB)) return cudaErrorInvalidValue;
+  if (!make_map(&tV, a.v, a.T, (int64_t)a.hkv * HD, a.ldv, C::KB)) return cudaErrorInvalidValue;
+  static std::atomic<unsigned long long> attr_done{0};
+  if (!done_on_device(attr_done)) {
+    const cudaError_t e = set_smem(k_attn_fwd_tc<HD>, C::SMEM);
+    if (e != cudaSuccess) return e;
+    mark_done_on_device(attr_done);
+  }
+  dim3 grid(a.hq, B, (a.S + C::QB - 1) / C::QB);
+  k_attn_fwd_tc<HD><<<grid, 192, C::SMEM, s>>>(tQ, tK, tV, a);
+  return cudaSuccess;
+}
+
+// LST_ATTN_FWD=mma selects the warp-level mma.sync forward (for comparing the two); the tcgen05
+// kernel is the default.
+bool use_mma_fwd() {
+  static const bool v = [] {
+    const char* e = std::getenv("LST_ATTN_FWD");
+    return e && std::strcmp(e, "mma") == 0;
+  }();
+  return v;
+}
+
 }  // namespace
 
 cudaError_t attention_fwd(const AttnArgs& a, cudaStream_t s) {
   if (!check_common(a.hd, a.hq, a.hkv, a.S, a.T)) return cudaErrorInvalidValue;
   const int B = (int)(a.T / a.S);
+  if (!use_mma_fwd()) {
+    const cudaError_t e = a.hd == 128 ? launch_fwd_tc<128>(a, B, s) : launch_fwd_tc<64>(a, B, s);
+    note_launch(1);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   dim3 grid(a.hq, B, (a.S + 63) / 64);
   if (a.hd == 128) {
     const int sm = 5 * 64 * Tile<128>::LD * 2;
@@ -697,6 +1532,58 @@ cudaError_t launch_dkdv(const AttnBwdArgs& a, int B, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, k_attn_dkdv<HD>, a);
 }
 
+namespace {
+
+template <int HD>
+cudaError_t launch_bwd_tc(const AttnBwdArgs& a, int B, cudaStream_t s) {
+  using Q = DqTc<HD>;
+  using K = DkvTc<HD>;
+  if ((a.ldq % 8) || (a.ldk % 8) || (a.ldv % 8) || (a.lddo % 8)) return cudaErrorInvalidValue;
+  CUtensorMap q64, o64, k128, v128, q128, o128, k64, v64;
+  const int64_t cq = (int64_t)a.hq * HD, ck = (int64_t)a.hkv * HD;
+  if (!make_map(&q64, a.q, a.T, cq, a.ldq, 64) || !make_map(&o64, a.dout, a.T, cq, a.lddo, 64) ||
+      !make_map(&k128, a.k, a.T, ck, a.ldk, 128) || !make_map(&v128, a.v, a.T, ck, a.ldv, 128) ||
+      !make_map(&q128, a.q, a.T, cq, a.ldq, 128) || !make_map(&o128, a.dout, a.T, cq, a.lddo, 128) ||
+      !make_map(&k64, a.k, a.T, ck, a.ldk, 64) || !make_map(&v64, a.v, a.T, ck, a.ldv, 64))
+    return cudaErrorInvalidValue;
+  static std::atomic<unsigned long long> attr_done{0};
+  if (!done_on_device(attr_done)) {
+    cudaError_t e = set_smem(k_attn_dkdv_tc<HD>, K::SMEM);
+    if (e == cudaSuccess) e = set_smem(k_attn_dq_tc<HD>, Q::SMEM);
+    if (e != cudaSuccess) return e;
+    mark_done_on_device(attr_done);
+  }
+  const int grp = a.hq / a.hkv;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grp, (unsigned)(B * a.hkv), (unsigned)((a.S + K::KB - 1) / K::KB));
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = K::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)grp;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_attn_dkdv_tc<HD>, q64, o64, k128, v128, a);
+  if (e != cudaSuccess) return e;
+  dim3 gq(a.hq, B, (a.S + Q::QB - 1) / Q::QB);
+  k_attn_dq_tc<HD><<<gq, 192, Q::SMEM, s>>>(q128, o128, k64, v64, a);
+  return cudaGetLastError();
+}
+
+// LST_ATTN_BWD=mma selects the warp-level mma.sync backward (for comparing the two).
+bool use_mma_bwd() {
+  static const bool v = [] {
+    const char* e = std::getenv("LST_ATTN_BWD");
+    return e && std::strcmp(e, "mma") == 0;
+  }();
+  return v;
+}
+
+}  // namespace
+
 cudaError_t attention_bwd(const AttnBwdArgs& a, cudaStream_t s) {
   if (!check_common(a.hd, a.hq, a.hkv, a.S, a.T)) return cudaErrorInvalidValue;
   if (a.hq / a.hkv > kMaxGroup) return cudaErrorInvalidValue;
@@ -704,6 +1591,11 @@ cudaError_t attention_bwd(const AttnBwdArgs& a, cudaStream_t s) {
   {
     const int64_t n = a.T * (int64_t)a.hq;
     k_attn_D<<<(unsigned)((n + 7) / 8), 256, 0, s>>>(a);
+  }
+  if (!use_mma_bwd()) {
+    const cudaError_t e = a.hd == 128 ? launch_bwd_tc<128>(a, B, s) : launch_bwd_tc<64>(a, B, s);
+    note_launch(3);
+    return e;
   }
   dim3 gq(a.hq, B, (a.S + 63) / 64);
   cudaError_t e;
