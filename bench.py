@@ -46,6 +46,31 @@ def describe(wl) -> str:
             f"a{int(wl.lora_alpha)} on 7 projections{head}, batch {wl.batch} x seq {wl.seq}")
 
 
+# DRAM traffic of the GEMMs of one llama8b step, from small ncu captures: for each GEMM shape of
+# the step, one launch of `kernel_cases.py <shape>` (dram__bytes_read.sum + dram__bytes_write.sum),
+# times the launches of that shape in a step (kernel_cases.GEMM_LAUNCHES_PER_STEP). The figures
+# belong to the GEMM sources whose hashes are recorded with them; with other sources bench.py
+# reports the traffic as null. Commands and values: profiles/gemm_traffic_llama8b_shapes.md.
+GEMM_TRAFFIC = {"workload": "llama8b", "bytes_per_launch": {}, "sources": {}}
+
+
+def gemm_traffic(wl_name: str):
+    """(average DRAM bytes per GEMM launch, bytes per step) of the recorded per-shape captures, or
+    (None, None) when the workload differs, nothing is recorded or the GEMM sources changed."""
+    import hashlib
+    from kernel_cases import GEMM_LAUNCHES_PER_STEP
+    rec = GEMM_TRAFFIC
+    if wl_name != rec["workload"] or not rec["bytes_per_launch"] or not rec["sources"]:
+        return None, None
+    csrc = os.path.join(ROOT, "layer_streamed_qlora_streaming_b200", "csrc")
+    for f, h in rec["sources"].items():
+        with open(os.path.join(csrc, f), "rb") as fh:
+            if hashlib.sha256(fh.read()).hexdigest()[:16] != h:
+                return None, None
+    per_step = sum(rec["bytes_per_launch"][c] * n for c, n in GEMM_LAUNCHES_PER_STEP.items())
+    return per_step / sum(GEMM_LAUNCHES_PER_STEP.values()), per_step
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -572,7 +597,7 @@ def run_gpu(args, wl):
 
     st = ctx.stats()
     peaks = measured_peaks()
-    traffic_launch, traffic_step = None, None
+    traffic_launch, traffic_step = gemm_traffic(args.workload)
     K = args.steps
     gemm_ms = agg["gemm_ms"] / K
     gemm_tflops = agg["gemm_flops"] / K / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else 0.0
@@ -597,8 +622,9 @@ def run_gpu(args, wl):
                      "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": gemm_tflops / peak_t if peak_t else None, "traffic": traffic_launch,
                      "traffic_per_step": traffic_step,
-                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum over one step's GEMM "
-                                       "launches (average per launch); null when the GEMM sources changed",
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of each "
+                                       "GEMM shape, times its launches per step (average per launch); null when "
+                                       "the GEMM sources differ from those captured",
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
                      "gemm_ms_per_step": gemm_ms, "gemm_launches_per_step": agg["gemm_launches"] / K},
         "step_roofline": {"bound": "pcie", "h2d_bytes_per_step": h2d_bytes, "link_gbs": link_gbs,

@@ -650,8 +650,7 @@ lst_status group_bwd(lst_ctx* c, int layer, int g, const uint8_t* blob, const __
   }
   // dA = s V^T X and dB = s dY^T U, with s folded into Vs and Us (their hi sections: the gradients are
   // fp32 reductions of bf16 products, so the lo parts would only refine the last bits of V and U)
-  CK(lora_grad_a(X, ldx, T, G.in, c->Vs[g], G.KP, G.nseg, c->r, dA, c->stream));
-  CK(lora_grad_b(dY, ldy, T, G.out, c->Us[g], G.KP, G.nseg, c->r, G.bounds, dB, c->stream));
+  CK(lora_grads(X, ldx, G.in, dY, ldy, G.out, T, c->Us[g], c->Vs[g], G.KP, G.nseg, c->r, G.bounds, dA, dB, c->stream));
   return LST_OK;
 }
 

@@ -236,9 +236,7 @@ lst_status lst_k_lora_grads(const uint16_t* X, int64_t ldx, int32_t in, const ui
   for (int p = 0; p < nseg; ++p)
     if (!dA[p] || !dB[p] || b[p + 1] <= b[p]) return LST_ERR_ARG;
   if (b[0] != 0 || b[nseg] != out) return LST_ERR_ARG;
-  const lst_status sa = st(lora_grad_a(B16(X), ldx, T, in, B16(Vs), KP, nseg, r, dA, S(stream)));
-  if (sa != LST_OK) return sa;
-  return st(lora_grad_b(B16(dY), ldy, T, out, B16(Us), KP, nseg, r, b, dB, S(stream)));
+  return st(lora_grads(B16(X), ldx, in, B16(dY), ldy, out, T, B16(Us), B16(Vs), KP, nseg, r, b, dA, dB, S(stream)));
 }
 
 int64_t lst_k_launch_count(void) { return g_launch_count.load(); }

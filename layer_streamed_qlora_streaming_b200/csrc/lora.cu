@@ -104,10 +104,14 @@ __device__ __forceinline__ void side_store(const SideOut& o, int row, int col, f
 // AMN / BMN: A / B MN-major ([K, M] / [K, N] row-major in memory), else K-major.
 // DUAL: every K step also loads the B tile b_off further along N (rows of a K-major B, columns of
 // an MN-major B) and accumulates its product with the same A tile.
+// A launch may carry two problems of the same K (the dA and dB reductions of a group): clusters
+// blockIdx.y < tiles1 take tiles of (tmA, tmB, o) in M-fastest order over mt1 M-tiles, the rest
+// tiles of (tmA2, tmB2, o2) over mt2.
 template <int AMN, int BMN, int DUAL>
 __global__ void __launch_bounds__(192, 2)
 k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const SideOut o,
-       const int nk, const int kps, const int b_off) {
+       const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, const SideOut o2,
+       const int tiles1, const int mt1, const int mt2, const int nk, const int kps, const int b_off) {
   constexpr int kStages = SideCfg<DUAL>::kStages;
   constexpr uint32_t kStageB = SideCfg<DUAL>::kStageB;
   extern __shared__ uint8_t smem_raw[];
@@ -124,7 +128,13 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   const int lane = threadIdx.x & 31;
   const int cs = (int)gridDim.x;  // one cluster = the K slices of one output tile
   const int z = (int)cluster_rank();
-  const int m0 = blockIdx.y * kBM, n0 = blockIdx.z * kBN;
+  const bool second = (int)blockIdx.y >= tiles1;
+  const int tt = second ? (int)blockIdx.y - tiles1 : (int)blockIdx.y;
+  const int mtp = second ? mt2 : mt1;
+  const int m0 = (tt % mtp) * kBM, n0 = (tt / mtp) * kBN;
+  const CUtensorMap* ma = second ? &tmA2 : &tmA;
+  const CUtensorMap* mb = second ? &tmB2 : &tmB;
+  const SideOut& oo = second ? o2 : o;
   const int kb0 = z * kps;
   const int nkb = max(0, min(nk - kb0, kps));
 
@@ -137,8 +147,8 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(ma);
+    tma_prefetch_desc(mb);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kBN);
@@ -158,17 +168,17 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         mbar_arrive_expect_tx(&full[s], kABytes + kStageB);
         const int kk = (kb0 + kb) * kBK;
         if (AMN == 0) {
-          tma_load_2d(sA + s * kABytes, &tmA, &full[s], kk, m0);
+          tma_load_2d(sA + s * kABytes, ma, &full[s], kk, m0);
         } else {
-          tma_load_2d(sA + s * kABytes, &tmA, &full[s], m0, kk);
-          tma_load_2d(sA + s * kABytes + 64 * kBK * 2, &tmA, &full[s], m0 + 64, kk);
+          tma_load_2d(sA + s * kABytes, ma, &full[s], m0, kk);
+          tma_load_2d(sA + s * kABytes + 64 * kBK * 2, ma, &full[s], m0 + 64, kk);
         }
         if (BMN == 0) {
-          tma_load_2d(sB + s * kStageB, &tmB, &full[s], kk, n0);
-          if (DUAL) tma_load_2d(sB + s * kStageB + kBBytes, &tmB, &full[s], kk, n0 + b_off);
+          tma_load_2d(sB + s * kStageB, mb, &full[s], kk, n0);
+          if (DUAL) tma_load_2d(sB + s * kStageB + kBBytes, mb, &full[s], kk, n0 + b_off);
         } else {
-          tma_load_2d(sB + s * kStageB, &tmB, &full[s], n0, kk);
-          if (DUAL) tma_load_2d(sB + s * kStageB + kBBytes, &tmB, &full[s], n0 + b_off, kk);
+          tma_load_2d(sB + s * kStageB, mb, &full[s], n0, kk);
+          if (DUAL) tma_load_2d(sB + s * kStageB + kBBytes, mb, &full[s], n0 + b_off, kk);
         }
       }
     }
@@ -244,7 +254,7 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         acc.w += v[p].w;
       }
     }
-    side_store(o, m0 + rl, n0 + c, acc);
+    side_store(oo, m0 + rl, n0 + c, acc);
   }
   __syncwarp();
   cluster_sync_all();  // no CTA leaves while another still reads its shared memory
@@ -255,9 +265,12 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   }
 }
 
+// One problem [M, N] (or, with tA2 given, two problems [M, N] and [M2, N2] of the same K in one
+// launch: the clusters of the second follow those of the first).
 template <int AMN, int BMN, int DUAL = 0>
 cudaError_t launch_side(const CUtensorMap& tA, const CUtensorMap& tB, int M, int N, int K, const SideOut& o,
-                        cudaStream_t st, int b_off = 0) {
+                        cudaStream_t st, int b_off = 0, const CUtensorMap* tA2 = nullptr,
+                        const CUtensorMap* tB2 = nullptr, int M2 = 0, int N2 = 0, const SideOut* o2 = nullptr) {
   constexpr uint32_t kSmem = SideCfg<DUAL>::kSmem;
   static std::atomic<unsigned long long> attr_done{0};  // devices whose function attribute is set
   if (!done_on_device(attr_done)) {
@@ -266,14 +279,16 @@ cudaError_t launch_side(const CUtensorMap& tA, const CUtensorMap& tB, int M, int
     mark_done_on_device(attr_done);
   }
   const int mt = (M + kBM - 1) / kBM, nt = (N + kBN - 1) / kBN, nk = (K + kBK - 1) / kBK;
-  if (mt > 65535 || nt > 65535) return cudaErrorInvalidValue;
+  const int mt2 = tA2 ? (M2 + kBM - 1) / kBM : 1, nt2 = tA2 ? (N2 + kBN - 1) / kBN : 0;
+  const int64_t tiles = (int64_t)mt * nt + (int64_t)mt2 * nt2;
+  if (tiles > 65535) return cudaErrorInvalidValue;
   // widest cluster (K split) that keeps every CTA resident at two per SM
   const int64_t slots = 2 * (int64_t)device_sm_count();
   int cs = 1;
-  while (cs < kMaxCluster && (int64_t)mt * nt * cs * 2 <= slots && cs * 2 <= nk) cs *= 2;
+  while (cs < kMaxCluster && tiles * cs * 2 <= slots && cs * 2 <= nk) cs *= 2;
   const int kps = (nk + cs - 1) / cs;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)cs, (unsigned)mt, (unsigned)nt);
+  cfg.gridDim = dim3((unsigned)cs, (unsigned)tiles, 1);
   cfg.blockDim = dim3(192, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = st;
@@ -284,7 +299,8 @@ cudaError_t launch_side(const CUtensorMap& tA, const CUtensorMap& tB, int M, int
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_side<AMN, BMN, DUAL>, tA, tB, o, nk, kps, b_off);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_side<AMN, BMN, DUAL>, tA, tB, o, tA2 ? *tA2 : tA, tB2 ? *tB2 : tB,
+                                           o2 ? *o2 : o, mt * nt, mt, mt2, nk, kps, b_off);
   note_launch(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -373,43 +389,36 @@ cudaError_t lora_skinny_split(const __nv_bfloat16* X, int64_t ldx, int64_t T, in
               : launch_side<0, 0, 1>(tA, tB, (int)T, R, K, o, st, 2 * RS);
 }
 
-cudaError_t lora_grad_a(const __nv_bfloat16* X, int64_t ldx, int64_t T, int in, const __nv_bfloat16* Vs, int KP,
-                        int nseg, int r, float* const* dst, cudaStream_t st) {
-  if (nseg < 1 || nseg > 3 || r <= 0 || nseg * r > KP || KP % 8 || T <= 0 || in <= 0) return cudaErrorInvalidValue;
-  if (!al16(X) || !al16(Vs) || (ldx % 8)) return cudaErrorInvalidValue;
-  // C [KP, in] = Vs^T X: A = Vs read MN-major ([T, KP]), B = X read MN-major ([T, in])
-  CUtensorMap tA, tB;
-  if (!make_map(&tA, Vs, T, KP, KP, kBK)) return cudaErrorInvalidValue;
-  if (!make_map(&tB, X, T, in, ldx, kBK)) return cudaErrorInvalidValue;
-  SideOut o{};
-  o.mode = 1;
-  o.M = nseg * r;  // rows of C past the adapters' ranks are not stored
-  o.N = in;
-  o.scale = 1.0f;
-  for (int k = 0; k < nseg; ++k) o.dst[k] = dst[k];
-  o.r = r;
-  o.nseg = nseg;
-  return launch_side<1, 1>(tA, tB, o.M, in, (int)T, o, st);
-}
-
-cudaError_t lora_grad_b(const __nv_bfloat16* dY, int64_t ldy, int64_t T, int out, const __nv_bfloat16* Us, int KP,
-                        int nseg, int r, const int* bounds, float* const* dst, cudaStream_t st) {
-  if (nseg < 1 || nseg > 3 || r <= 0 || nseg * r > KP || KP % 8 || T <= 0 || out <= 0) return cudaErrorInvalidValue;
-  if (!al16(dY) || !al16(Us) || (ldy % 8) || bounds[0] != 0 || bounds[nseg] != out) return cudaErrorInvalidValue;
-  // C [out, KP] = dY^T Us: A = dY read MN-major ([T, out]), B = Us read MN-major ([T, KP])
-  CUtensorMap tA, tB;
-  if (!make_map(&tA, dY, T, out, ldy, kBK)) return cudaErrorInvalidValue;
-  if (!make_map(&tB, Us, T, KP, KP, kBK)) return cudaErrorInvalidValue;
-  SideOut o{};
-  o.mode = 2;
-  o.M = out;
-  o.N = nseg * r;  // columns of C past the adapters' ranks are not stored
-  o.scale = 1.0f;
-  for (int k = 0; k < nseg; ++k) o.dst[k] = dst[k];
-  for (int k = 0; k <= nseg; ++k) o.bounds[k] = bounds[k];
-  o.r = r;
-  o.nseg = nseg;
-  return launch_side<1, 1>(tA, tB, out, o.N, (int)T, o, st);
+cudaError_t lora_grads(const __nv_bfloat16* X, int64_t ldx, int in, const __nv_bfloat16* dY, int64_t ldy, int out,
+                       int64_t T, const __nv_bfloat16* Us, const __nv_bfloat16* Vs, int KP, int nseg, int r,
+                       const int* bounds, float* const* dA, float* const* dB, cudaStream_t st) {
+  if (nseg < 1 || nseg > 3 || r <= 0 || nseg * r > KP || KP % 8 || T <= 0 || in <= 0 || out <= 0)
+    return cudaErrorInvalidValue;
+  if (!al16(X) || !al16(Vs) || !al16(dY) || !al16(Us) || (ldx % 8) || (ldy % 8) || bounds[0] != 0 ||
+      bounds[nseg] != out)
+    return cudaErrorInvalidValue;
+  // dA: C [nseg*r, in] = Vs^T X; dB: C [out, nseg*r] = dY^T Us (both contract the T tokens)
+  CUtensorMap tVa, tX, tdY, tU;
+  if (!make_map(&tVa, Vs, T, KP, KP, kBK) || !make_map(&tX, X, T, in, ldx, kBK) ||
+      !make_map(&tdY, dY, T, out, ldy, kBK) || !make_map(&tU, Us, T, KP, KP, kBK))
+    return cudaErrorInvalidValue;
+  SideOut oa{}, ob{};
+  oa.mode = 1;
+  oa.M = nseg * r;
+  oa.N = in;
+  oa.scale = 1.0f;
+  ob.mode = 2;
+  ob.M = out;
+  ob.N = nseg * r;
+  ob.scale = 1.0f;
+  for (int k = 0; k < nseg; ++k) {
+    oa.dst[k] = dA[k];
+    ob.dst[k] = dB[k];
+  }
+  for (int k = 0; k <= nseg; ++k) ob.bounds[k] = bounds[k];
+  oa.r = ob.r = r;
+  oa.nseg = ob.nseg = nseg;
+  return launch_side<1, 1>(tVa, tX, oa.M, in, (int)T, oa, st, 0, &tdY, &tU, out, ob.N, &ob);
 }
 
 cudaError_t lora_prep(const LoraPrepArgs& a, cudaStream_t st) {

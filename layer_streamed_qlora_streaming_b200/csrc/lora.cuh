@@ -26,16 +26,16 @@ cudaError_t lora_skinny_split(const __nv_bfloat16* X, int64_t ldx, int64_t T, in
                               int64_t ldb, int b_mn, int R, int RS, int KP, float s, __nv_bfloat16* Us,
                               cudaStream_t st);
 
-// dA of every segment of a fused group: dA_p[j][i] = sum_t Vs[t][p*r + j] X[t][i] with X bf16
-// [T, in] and Vs = bf16(s V) [T, KP]; dst[p] fp32 [r, in]. Computed as the [KP, in] product
-// Vs^T X, each row stored straight into its segment.
-cudaError_t lora_grad_a(const __nv_bfloat16* X, int64_t ldx, int64_t T, int in, const __nv_bfloat16* Vs, int KP,
-                        int nseg, int r, float* const* dst, cudaStream_t st);
-
-// dB of every segment: C = dY^T Us (dY bf16 [T, out], Us = bf16(s U) [T, KP]), then
-// dB_p[o - bounds[p]][j] = C[o][p*r + j] for o in segment p (dst[p] fp32 [out_p, r]).
-cudaError_t lora_grad_b(const __nv_bfloat16* dY, int64_t ldy, int64_t T, int out, const __nv_bfloat16* Us, int KP,
-                        int nseg, int r, const int* bounds, float* const* dst, cudaStream_t st);
+// The adapter gradients of one fused group, in one launch (the clusters of dB follow those of dA),
+// both reductions over the T tokens:
+//   dA_p[j][i] = sum_t Vs[t][p*r + j] X[t][i]        with X bf16 [T, in] and Vs [T, KP]; dA[p] fp32 [r, in],
+//                computed as the rows of Vs^T X that belong to the adapters;
+//   dB_p[o][j] = sum_t dY[t][bounds[p] + o] Us[t][p*r + j]   with dY bf16 [T, out] and Us [T, KP];
+//                dB[p] fp32 [out_p, r], the adapter columns of dY^T Us.
+// Only columns < nseg * r of Us / Vs are read (the hi section of the split operands).
+cudaError_t lora_grads(const __nv_bfloat16* X, int64_t ldx, int in, const __nv_bfloat16* dY, int64_t ldy, int out,
+                       int64_t T, const __nv_bfloat16* Us, const __nv_bfloat16* Vs, int KP, int nseg, int r,
+                       const int* bounds, float* const* dA, float* const* dB, cudaStream_t st);
 
 // Derived bf16 operands of one fused projection group from its fp32 adapters (nseg segments,
 // A_p [r, in], B_p [out_p, r]), each adapter value a stored as the pair hi = bf16(a),

@@ -35,3 +35,24 @@ def test_workloads_are_described():
     for name in ("llama8b", "qwen3b_bf16", "qwen32b", "tiny", "llama8b_layer"):
         wl = bench.workload(name)
         assert name in bench.describe(wl)
+
+
+def test_gemm_traffic_only_for_the_captured_sources(monkeypatch):
+    import copy
+    from kernel_cases import GEMM_LAUNCHES_PER_STEP
+    rec = {"workload": "llama8b", "bytes_per_launch": {c: 1000.0 * (i + 1) for i, c in enumerate(GEMM_LAUNCHES_PER_STEP)},
+           "sources": {}}
+    monkeypatch.setattr(bench, "GEMM_TRAFFIC", rec)
+    assert bench.gemm_traffic("llama8b") == (None, None)            # no hashes recorded
+    import hashlib, os
+    csrc = os.path.join(bench.ROOT, "layer_streamed_qlora_streaming_b200", "csrc")
+    rec2 = copy.deepcopy(rec)
+    rec2["sources"] = {f: hashlib.sha256(open(os.path.join(csrc, f), "rb").read()).hexdigest()[:16]
+                       for f in ("gemm.cu", "gemm.cuh", "common.cuh")}
+    monkeypatch.setattr(bench, "GEMM_TRAFFIC", rec2)
+    per_launch, per_step = bench.gemm_traffic("llama8b")
+    want = sum(rec["bytes_per_launch"][c] * n for c, n in GEMM_LAUNCHES_PER_STEP.items())
+    assert per_step == want and per_launch == want / sum(GEMM_LAUNCHES_PER_STEP.values())
+    assert bench.gemm_traffic("qwen3b_bf16") == (None, None)        # another workload
+    rec2["sources"]["gemm.cu"] = "0" * 16
+    assert bench.gemm_traffic("llama8b") == (None, None)            # sources changed since
