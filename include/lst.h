@@ -234,7 +234,8 @@ lst_status lst_get_read_timeline(const lst_ctx* ctx, float* out, int32_t max_rea
  * run the same steps in the same order (the reads are collective). The library loads
  * libnccl.so.2 on first use (LST_ERR_STATE if it cannot); the communicator is created here
  * (ncclCommInitRank, collective over the ranks) and destroyed with the context. unique_id: the 128
- * bytes of lst_nccl_unique_id from one rank, passed to every rank. world == 1 does nothing. Needs
+ * bytes of lst_nccl_unique_id from one rank, passed to every rank. world == 1 runs the same path
+ * on one GPU (the whole blob is this rank's slice; the all-gather is a one-rank collective). Needs
  * a streamed context; call once, before the first step. The results are the same bytes as
  * without it (the assembled blob is the same). */
 lst_status lst_set_split_copy(lst_ctx* ctx, int32_t rank, int32_t world, const void* unique_id);

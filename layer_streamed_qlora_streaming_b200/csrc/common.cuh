@@ -202,6 +202,11 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
+__device__ __forceinline__ uint32_t cluster_size_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctaid.x;" : "=r"(r));
+  return r;
+}
 // Every thread of every CTA of the cluster arrives (release) and waits (acquire): shared-memory
 // writes made before it are visible to the cluster's other CTAs after it.
 __device__ __forceinline__ void cluster_sync_all() {

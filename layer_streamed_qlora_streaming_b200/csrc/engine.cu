@@ -1017,7 +1017,7 @@ lst_status enqueue_copy(lst_ctx* c, int n) {
   ProfScope ps(c, c->copy_stream, PC_COPY);
   TRY(tl_record(c, n, lst_ctx::TL_COPY0, c->copy_stream));
   const uint8_t* src = c->arena + (int64_t)j * c->lay.total;
-  if (c->split_world > 1) {
+  if (c->nccl_comm) {
     // this rank's slice over its own link, then the whole blob from every rank's slice over
     // NVLink (in-place all-gather into the pool slot); the blob is complete for every chunk at once
     int64_t off = 0, bytes = 0, count = 0;
@@ -1936,11 +1936,9 @@ lst_status lst_nccl_unique_id(void* out) {
 lst_status lst_set_split_copy(lst_ctx* c, int32_t rank, int32_t world, const void* unique_id) {
   if (!c) return LST_ERR_ARG;
   DeviceScope ds(c);
-  if (world < 1 || rank < 0 || rank >= world || (world > 1 && !unique_id))
-    return fail(c, LST_ERR_ARG, "bad rank / world or null unique id");
+  if (world < 1 || rank < 0 || rank >= world || !unique_id) return fail(c, LST_ERR_ARG, "bad rank / world or null unique id");
   if (!c->cfg.streamed) return fail(c, LST_ERR_STATE, "split copies need a streamed context");
   if (c->nccl_comm) return fail(c, LST_ERR_STATE, "split copies are already set");
-  if (world == 1) return LST_OK;
   if (!nccl().ok) return fail(c, LST_ERR_STATE, "libnccl.so.2 could not be loaded");
   int64_t off = 0, bytes = 0, count = 0;
   split_plan(c->lay.total, world, rank, &off, &bytes, &count);

@@ -290,6 +290,92 @@ k_ce(const float* __restrict__ logits, int V, const int32_t* __restrict__ y, flo
   }
 }
 
+// Cross-entropy rows that read each logit once: a thread-block cluster of cs CTAs holds one row
+// in shared memory, CTA z the slice [z * slice, (z + 1) * slice). Each CTA reduces its slice to
+// (max, sum of exp) in a fixed tree; the cs pairs are merged in rank order through distributed
+// shared memory (every CTA gets the same lse); then each CTA writes dlogits of its slice from
+// shared memory, and the CTA holding the target writes the row's loss.
+constexpr int kCeThreads = 512;
+__global__ void __launch_bounds__(kCeThreads, 1)
+k_ce_cluster(const float* __restrict__ logits, int V, int slice, const int32_t* __restrict__ y, float inv_T,
+             float* __restrict__ loss_rows, bf16* __restrict__ dlog) {
+  extern __shared__ __align__(16) float row_s[];  // [slice], then the CTA's (max, sum) pair
+  __shared__ float sm[32], ss[32];
+  const int cs = (int)cluster_size_x();
+  const int z = (int)cluster_rank();
+  const int64_t row = blockIdx.x / cs;
+  const int c0 = z * slice, n = max(0, min(V - c0, slice));
+  const float* lr = logits + row * V + c0;
+  float m = -INFINITY, sum = 0.f;
+  if ((V % 4) == 0) {  // slices start on 16-byte boundaries (slice % 4 == 0)
+    const float4* l4 = reinterpret_cast<const float4*>(lr);
+    float4* r4 = reinterpret_cast<float4*>(row_s);
+    for (int c = threadIdx.x; c < n / 4; c += blockDim.x) {
+      const float4 v = __ldg(l4 + c);
+      r4[c] = v;
+      ms_add4(m, sum, v);
+    }
+  } else {
+    for (int c = threadIdx.x; c < n; c += blockDim.x) {
+      const float v = lr[c];
+      row_s[c] = v;
+      ms_add4(m, sum, make_float4(v, -INFINITY, -INFINITY, -INFINITY));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, sum, o);
+    ms_merge(m, sum, m2, s2);
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    sm[w] = m;
+    ss[w] = sum;
+  }
+  __syncthreads();
+  float* pair = row_s + slice;
+  if (threadIdx.x == 0) {
+    float mm = sm[0], s2 = ss[0];
+    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) ms_merge(mm, s2, sm[i], ss[i]);
+    pair[0] = mm;
+    pair[1] = s2;
+  }
+  cluster_sync_all();  // every CTA's pair is in place
+  float M = -INFINITY, Ssum = 0.f;
+  const uint32_t pa = smem_u32(pair);
+  for (int q = 0; q < cs; ++q) {
+    const float2 v = ld_cluster_f2(cluster_map(pa, (uint32_t)q));
+    ms_merge(M, Ssum, v.x, v.y);
+  }
+  cluster_sync_all();  // no CTA leaves while another still reads its pair
+  const float lse = M + logf(Ssum);
+  int tgt = y[row];
+  if (tgt < 0 || tgt >= V) {
+    if (threadIdx.x == 0 && z == 0) dev_fail(DEV_ERR_BAD_INDEX);
+    tgt = 0;
+  }
+  if (threadIdx.x == 0 && tgt >= c0 && tgt < c0 + n) loss_rows[row] = lse - row_s[tgt - c0];
+  bf16* dr = dlog + row * V + c0;
+  if ((V % 4) == 0) {
+    const float4* r4 = reinterpret_cast<const float4*>(row_s);
+    for (int c = threadIdx.x; c < n / 4; c += blockDim.x) {
+      const float4 v = r4[c];
+      float p[4] = {expf(v.x - lse), expf(v.y - lse), expf(v.z - lse), expf(v.w - lse)};
+      const int d = tgt - c0 - 4 * c;
+      if (d >= 0 && d < 4) p[d] -= 1.0f;
+      const __nv_bfloat162 h[2] = {__floats2bfloat162_rn(p[0] * inv_T, p[1] * inv_T),
+                                   __floats2bfloat162_rn(p[2] * inv_T, p[3] * inv_T)};
+      *reinterpret_cast<uint2*>(dr + 4 * c) = *reinterpret_cast<const uint2*>(h);
+    }
+  } else {
+    for (int c = threadIdx.x; c < n; c += blockDim.x) {
+      float p = expf(row_s[c] - lse);
+      if (c0 + c == tgt) p -= 1.0f;
+      dr[c] = __float2bfloat16_rn(p * inv_T);
+    }
+  }
+}
+
 // Row (max, sum of exp) of a logits row by the online rule of k_ce, merged in a fixed tree.
 __device__ __forceinline__ float row_lse(const float* __restrict__ lr, int V, float* sm, float* ss) {
   float m = -INFINITY, s = 0.f;
@@ -473,9 +559,39 @@ cudaError_t embed(const int32_t* tok, const bf16* E, int64_t T, int d, int V, fl
 }
 cudaError_t cross_entropy(const float* logits, int64_t T, int V, const int32_t* y, float inv_T, float* loss_rows,
                           bf16* dlog, cudaStream_t s) {
-  k_ce<<<(unsigned)T, 1024, 0, s>>>(logits, V, y, inv_T, loss_rows, dlog);
+  // the smallest power-of-two cluster (<= 8) whose slices fit in 200 KB of shared memory each
+  constexpr int64_t kMaxSliceBytes = 200 * 1024;
+  int cs = 1;
+  while (cs < 8 && (((int64_t)V + cs - 1) / cs + 3) / 4 * 16 > kMaxSliceBytes) cs *= 2;
+  const int slice = (int)((((int64_t)V + cs - 1) / cs + 3) / 4 * 4);
+  if ((int64_t)slice * 4 > kMaxSliceBytes || T * cs > INT32_MAX) {
+    k_ce<<<(unsigned)T, 1024, 0, s>>>(logits, V, y, inv_T, loss_rows, dlog);  // rows too long for a cluster
+    note_launch(1);
+    return cudaGetLastError();
+  }
+  const int smem = slice * 4 + 16;
+  static std::atomic<unsigned long long> attr_done{0};
+  if (!done_on_device(attr_done)) {
+    const cudaError_t e = cudaFuncSetAttribute(k_ce_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)(kMaxSliceBytes + 16));
+    if (e != cudaSuccess) return e;
+    mark_done_on_device(attr_done);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(T * cs), 1, 1);
+  cfg.blockDim = dim3(kCeThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)cs;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_ce_cluster, logits, V, slice, y, inv_T, loss_rows, dlog);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t ce_stats(const float* logits, int64_t T, int V, const int32_t* y, float* lse, float* logp, cudaStream_t s) {
   k_ce_stats<<<(unsigned)T, 1024, 0, s>>>(logits, V, y, lse, logp);

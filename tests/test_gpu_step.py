@@ -412,3 +412,32 @@ def test_dequant_inside_gemm_same_bytes(name):
         for (la, ga), (lb, gb) in zip(out[0], res):
             assert np.float32(la).tobytes() == np.float32(lb).tobytes()
             assert ga.tobytes() == gb.tobytes()
+
+
+def test_split_copy_one_rank_same_bytes():
+    # the split-copy path with a one-rank NCCL communicator: the rank's slice is the whole blob and
+    # the all-gather runs on the copy stream; every step gives the bytes of plain copies
+    import layer_streamed_qlora_streaming_b200 as lst
+    try:
+        uid = lst.nccl_unique_id()
+    except lst.LstError:
+        pytest.skip("NCCL is not available")
+    wl = WORKLOADS["tiny_gqa_bias_bf16"]
+    inp = build_inputs(wl)
+    out = []
+    for split in (False, True):
+        ctx = make_context(wl, inp, streamed=True)
+        if split:
+            ctx.set_split_copy(0, 1, uid)
+            with pytest.raises(lst.LstError):      # once per context
+                ctx.set_split_copy(0, 1, uid)
+        out.append([run_step(ctx, wl, inp, want_logits=False)[:2] for _ in range(2)])
+        assert ctx.stats()["h2d_bytes_last_step"] == 2 * wl.n_layers * ctx.stats()["blob_bytes"]
+        ctx.close()
+    for (la, ga), (lb, gb) in zip(*out):
+        assert np.float32(la).tobytes() == np.float32(lb).tobytes() and ga.tobytes() == gb.tobytes()
+    ctx = make_context(wl, inp, streamed=False)
+    with pytest.raises(lst.LstError) as e:        # resident contexts copy nothing
+        ctx.set_split_copy(0, 1, uid)
+    assert e.value.status == 2
+    ctx.close()
