@@ -496,23 +496,34 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tc_fence_after();
       float x[C::KB];
 #pragma unroll
-      for (int c = 0; c < C::KB; c += 32) {
-        uint32_t u[32];
+      for (int c = 0; c < C::KB; c += 64) {  // two TMEM loads in flight per wait
+        uint32_t u[32], w[32];
         tmem_ld32(tmem + st * C::KB + c + lane_off, u);
+        tmem_ld32(tmem + st * C::KB + c + 32 + lane_off, w);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[c + e] = __uint_as_float(u[e]) * sl2;
+        for (int e = 0; e < 32; ++e) {
+          x[c + e] = __uint_as_float(u[e]) * sl2;
+          x[c + 32 + e] = __uint_as_float(w[e]) * sl2;
+        }
       }
       tc_fence_before();
       mbar_arrive(&s_free[st]);
       const bool diag = j == nkb - 1;
-      float bm = -INFINITY;
+      if (diag) {
 #pragma unroll
-      for (int e = 0; e < C::KB; ++e) {
-        const int key = j * C::KB + e;
-        if (diag && (key > qrow || key >= p.S)) x[e] = -INFINITY;
-        bm = fmaxf(bm, x[e]);
+        for (int e = 0; e < C::KB; ++e) {
+          const int key = j * C::KB + e;
+          if (key > qrow || key >= p.S) x[e] = -INFINITY;
+        }
       }
+      // row max through 8 independent partial maxima (short dependency chains)
+      float pm[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pm[i] = x[i];
+#pragma unroll
+      for (int e = 8; e < C::KB; ++e) pm[e & 7] = fmaxf(pm[e & 7], x[e]);
+      const float bm = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       float corr = 1.f;
       if (j == 0) {
         mref = bm;
@@ -520,12 +531,13 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         corr = exp2f(mref - bm);
         mref = bm;
       }
-      float rs = 0.f;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < C::KB; ++e) {
         x[e] = exp2f(x[e] - mref);
-        rs += x[e];
+        ps[e & 7] += x[e];
       }
+      const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       l = l * corr + rs;
       if (j >= 1) {  // P_{j-1} V_{j-1} done: the P tile is free and O holds the blocks so far
         if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1))) {
@@ -989,16 +1001,24 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int kr = k0 + r;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = p.scale * kLog2e;
+    // the lse (log2 domain) and D of a block's queries, loaded by threads t < 64 one block ahead
+    auto load_ld = [&](int jb, float& lv, float& dvv) {
+      const int qr = (i0 + jb) * C::QB + t;
+      const bool in = t < C::QB && jb < nqb && qr < p.S;
+      lv = in ? p.lse[(tok0 + qr) * p.hq + h] * kLog2e : 0.f;
+      dvv = in ? p.D[(tok0 + qr) * p.hq + h] : 0.f;
+    };
+    float nl = 0.f, nd = 0.f;
+    load_ld(0, nl, nd);
     // every iteration reaches the named barrier (the four warps together), also after a failed wait
     for (int j = 0; j < nqb; ++j) {
       const int st = j & 1;
       const int q0 = (i0 + j) * C::QB;
-      if (t < C::QB) {  // the block's lse (log2 domain) and D, shared by every key row
-        const int qr = q0 + t;
-        const bool in = qr < p.S;
-        sLse[st * C::QB + t] = in ? p.lse[(tok0 + qr) * p.hq + h] * kLog2e : 0.f;
-        sD[st * C::QB + t] = in ? p.D[(tok0 + qr) * p.hq + h] : 0.f;
+      if (t < C::QB) {  // the block's values, shared by every key row
+        sLse[st * C::QB + t] = nl;
+        sD[st * C::QB + t] = nd;
       }
+      load_ld(j + 1, nl, nd);
       asm volatile("bar.sync 1, 128;" ::: "memory");
       if (!ok) continue;
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1))) {

@@ -706,7 +706,7 @@ lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
     a.v = c->qkv + c->dq + c->dkv;
     a.o = c->o;
     a.lse = c->lse;
-    a.o32 = c->o32;
+    a.o32 = recompute ? c->o32 : nullptr;  // only the backward of a recomputed layer reads it
     a.ldq = a.ldk = a.ldv = c->dqkv;
     a.ldo = c->dq;
     a.T = T;

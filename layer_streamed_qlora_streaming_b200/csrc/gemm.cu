@@ -655,7 +655,7 @@ cudaError_t launch_nf4(const GemmArgs& a, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     mark_done_on_device(attr_done);
   }
-  const int nk1 = a.K / BK;
+  const int nk1 = (a.K + BK - 1) / BK;  // MN-major W: K = W's rows, any count (the tail rows are zero)
   TileSched sched;
   sched.mt = (a.M + BM - 1) / BM;
   sched.nt = (a.N + BN - 1) / BN;

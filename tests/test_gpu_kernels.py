@@ -130,6 +130,7 @@ NF4_GEMM_CASES = [
     (128, [64], 512, 0, False, True, False, True),             # BN = 64, residual
     (256, [256, 128, 128], 320, 1, True, True, False, False),  # dX of q/k/v: W [K, N] MN-major
     (384, [1024, 1024], 256, 1, False, True, False, False),    # dX of gate/up
+    (128, [688, 688], 256, 1, True, True, False, False),       # dX of the tiny gate/up: K = 1376 rows, ragged
     (2048, [4096, 1024, 1024], 4096, 0, True, False, False, False),  # 8B q/k/v forward
     (2048, [14336, 14336], 4096, 1, True, True, False, False),       # 8B gate/up dX
 ]
