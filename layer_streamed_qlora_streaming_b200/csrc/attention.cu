@@ -333,9 +333,9 @@ __global__ void __launch_bounds__(128) k_attn_fwd(AttnArgs p) {
 }
 
 // ------------------------------------------------------------------------------------ forward, tcgen05
-// One CTA per 128 queries of one head (the last query blocks, with the most keys, first); 192
+// One CTA per 128 queries of one head (the last query blocks, with the most keys, first); 320
 // threads: warp 0 TMA producer (Q once; K and V tiles of 128 keys, double-buffered), warp 1 MMA
-// issuer, warps 2-5 softmax (one thread per query row, TMEM lane = row).
+// issuer, warps 2-9 softmax (two threads per query row, TMEM lane = row, each half of the keys).
 //   S = Q K^T           tcgen05, bf16 operands, fp32 in one of two TMEM buffers (so the next block's
 //                       Q K^T runs while this block's softmax reads its scores);
 //   P = exp2(S' - m)    softmax threads, written as fp16 to a 128-byte-swizzled shared tile (the
@@ -351,12 +351,13 @@ struct AttnTc {
   static constexpr uint32_t Q_BYTES = (HD / 64) * CH;
   static constexpr uint32_t KV_BYTES = 2 * (HD / 64) * CH; // K then V of one stage
   static constexpr uint32_t P_BYTES = 2 * CH;              // 128 queries x 128 keys fp16
-  static constexpr uint32_t SMEM = Q_BYTES + 2 * KV_BYTES + P_BYTES + 1024 + 256;
+  // + barriers (128 B) and the row threads' max / sum exchange (3 KB)
+  static constexpr uint32_t SMEM = Q_BYTES + 2 * KV_BYTES + P_BYTES + 1024 + 128 + 3 * 1024;
   static constexpr uint32_t TMEM_COLS = 512;              // S[2] at columns 0 / 128, O at 256
 };
 
 template <int HD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const AttnArgs p) {
   using C = AttnTc<HD>;
@@ -388,9 +389,9 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
+      mbar_init(&s_free[i], 256);
     }
-    mbar_init(p_full, 128);
+    mbar_init(p_full, 256);
     mbar_init(pv_done, 1);
     fence_mbar_init();
   }
@@ -463,22 +464,27 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
     }
   } else {
-    const int r = (warp & 3) * 32 + lane;  // query row of this thread = its TMEM lane
+    // Two threads per query row (warps 2-5: half 0, warps 6-9: half 1, the same TMEM lanes): half
+    // h takes keys [64h, 64h + 64) of each block and O columns [h HD/2, (h + 1) HD/2). The block
+    // max is exchanged through shared memory (double-buffered over blocks); the row sums are kept
+    // per half and added once at the end.
+    const int ts = (int)threadIdx.x - 64;  // 0 .. 255
+    const int half = ts >> 7;
+    const int r = (warp & 3) * 32 + lane;  // query row = TMEM lane
     const int qrow = q0 + r;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = p.scale * kLog2e;
+    constexpr int NK = C::KB / 2, NO = HD / 2;
+    float* smax = reinterpret_cast<float*>(bars + 12);  // [2 blocks][2 halves][128 rows]
+    float* ssum = smax + 512;                            // [2 halves][128 rows]
     float mref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkb && ok; ++j) {
+    for (int j = 0; j < nkb; ++j) {  // every iteration reaches the named barrier, also after a failed wait
       const int st = j & 1;
-      // V_j to fp16 in place (this thread's 16-byte pieces), once its TMA has landed
-      if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[st], (j >> 1) & 1))) {
-        ok = false;
-        break;
-      }
-      {
+      if (ok && !__all_sync(0xffffffffu, mbar_wait(&kv_full[st], (j >> 1) & 1))) ok = false;
+      if (ok) {  // V_j to fp16 in place, once its TMA has landed
         uint4* vt = reinterpret_cast<uint4*>(sKV + st * C::KV_BYTES + (HD / 64) * C::CH);
-        for (int i = r; i < (int)((HD / 64) * C::CH / 16); i += 128) {
+        for (int i = ts; i < (int)((HD / 64) * C::CH / 16); i += 256) {
           uint4 u = vt[i];
           uint32_t* w = reinterpret_cast<uint32_t*>(&u);
 #pragma unroll
@@ -489,102 +495,101 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           vt[i] = u;
         }
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float x[C::KB];
+      if (ok && !__all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1))) ok = false;
+      float x[NK];
+      float pmax = -INFINITY;
+      if (ok) {
+        tc_fence_after();
+        {
+          uint32_t u[32], w[32];
+          tmem_ld32(tmem + st * C::KB + half * NK + lane_off, u);
+          tmem_ld32(tmem + st * C::KB + half * NK + 32 + lane_off, w);
+          tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < C::KB; c += 64) {  // two TMEM loads in flight per wait
-        uint32_t u[32], w[32];
-        tmem_ld32(tmem + st * C::KB + c + lane_off, u);
-        tmem_ld32(tmem + st * C::KB + c + 32 + lane_off, w);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          x[c + e] = __uint_as_float(u[e]) * sl2;
-          x[c + 32 + e] = __uint_as_float(w[e]) * sl2;
+          for (int e = 0; e < 32; ++e) {
+            x[e] = __uint_as_float(u[e]) * sl2;
+            x[32 + e] = __uint_as_float(w[e]) * sl2;
+          }
         }
-      }
-      tc_fence_before();
-      mbar_arrive(&s_free[st]);
-      const bool diag = j == nkb - 1;
-      if (diag) {
+        tc_fence_before();
+        mbar_arrive(&s_free[st]);
+        if (j == nkb - 1) {  // only the diagonal block holds keys past a query or past S
 #pragma unroll
-        for (int e = 0; e < C::KB; ++e) {
-          const int key = j * C::KB + e;
-          if (key > qrow || key >= p.S) x[e] = -INFINITY;
+          for (int e = 0; e < NK; ++e) {
+            const int key = j * C::KB + half * NK + e;
+            if (key > qrow || key >= p.S) x[e] = -INFINITY;
+          }
         }
+        float pm[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pm[i] = x[i];
+#pragma unroll
+        for (int e = 8; e < NK; ++e) pm[e & 7] = fmaxf(pm[e & 7], x[e]);
+        pmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       }
-      // row max through 8 independent partial maxima (short dependency chains)
-      float pm[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) pm[i] = x[i];
-#pragma unroll
-      for (int e = 8; e < C::KB; ++e) pm[e & 7] = fmaxf(pm[e & 7], x[e]);
-      const float bm = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      smax[(j & 1) * 256 + half * 128 + r] = pmax;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (!ok) continue;
+      const float bm = fmaxf(pmax, smax[(j & 1) * 256 + (1 - half) * 128 + r]);
       float corr = 1.f;
       if (j == 0) {
-        mref = bm;
+        mref = bm;  // block 0 always holds key 0 <= query
       } else if (bm > mref + 8.f) {
         corr = exp2f(mref - bm);
         mref = bm;
       }
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int e = 0; e < C::KB; ++e) {
+      for (int e = 0; e < NK; ++e) {
         x[e] = exp2f(x[e] - mref);
         ps[e & 7] += x[e];
       }
-      const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      l = l * corr + rs;
+      l = l * corr + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
       if (j >= 1) {  // P_{j-1} V_{j-1} done: the P tile is free and O holds the blocks so far
         if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1))) {
           ok = false;
-          break;
+          continue;
         }
         tc_fence_after();
         if (__any_sync(0xffffffffu, corr != 1.f)) {
 #pragma unroll
-          for (int c = 0; c < HD; c += 32) {
+          for (int c = 0; c < NO; c += 32) {
             uint32_t u[32];
-            tmem_ld32(tmem + 256 + c + lane_off, u);
+            tmem_ld32(tmem + 256 + half * NO + c + lane_off, u);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * corr);
-            tmem_st32(tmem + 256 + c + lane_off, u);
+            tmem_st32(tmem + 256 + half * NO + c + lane_off, u);
           }
           tmem_st_wait();
         }
       }
-      // P row r: keys 0-63 in chunk 0, 64-127 in chunk 1; 16-byte piece i of a row at i ^ (r & 7)
+      // this half's 64 keys are chunk `half` of P row r; 16-byte piece i at i ^ (r & 7)
+      uint8_t* prow = sP + half * C::CH + r * 128;
 #pragma unroll
-      for (int kc = 0; kc < 2; ++kc) {
-        uint8_t* row = sP + kc * C::CH + r * 128;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float* v = x + kc * 64 + i * 8;
-          uint4 u = make_uint4(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]), pack_f16(v[4], v[5]),
-                               pack_f16(v[6], v[7]));
-          *reinterpret_cast<uint4*>(row + ((i ^ (r & 7)) * 16)) = u;
-        }
+      for (int i = 0; i < 8; ++i) {
+        const float* v = x + i * 8;
+        *reinterpret_cast<uint4*>(prow + ((i ^ (r & 7)) * 16)) =
+            make_uint4(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]), pack_f16(v[4], v[5]), pack_f16(v[6], v[7]));
       }
       fence_proxy_async();  // P and the converted V are read by the tensor core
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    // O / l, lse
+    ssum[half * 128 + r] = l;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    const float lt = l + ssum[(1 - half) * 128 + r];
+    // O / l (this half's columns), lse
     if (ok && __all_sync(0xffffffffu, mbar_wait(pv_done, (nkb - 1) & 1))) {
       tc_fence_after();
-      const float inv = 1.f / l;
+      const float inv = 1.f / lt;
       const bool live = qrow < p.S;
-      __nv_bfloat16* op = p.o + (tok0 + qrow) * p.ldo + h * HD;
-      float* o32 = p.o32 ? p.o32 + (tok0 + qrow) * (int64_t)p.hq * HD + h * HD : nullptr;
+      __nv_bfloat16* op = p.o + (tok0 + qrow) * p.ldo + h * HD + half * NO;
+      float* o32 = p.o32 ? p.o32 + (tok0 + qrow) * (int64_t)p.hq * HD + h * HD + half * NO : nullptr;
 #pragma unroll
-      for (int c = 0; c < HD; c += 32) {
+      for (int c = 0; c < NO; c += 32) {
         uint32_t u[32];
-        tmem_ld32(tmem + 256 + c + lane_off, u);
+        tmem_ld32(tmem + 256 + half * NO + c + lane_off, u);
         tmem_ld_wait();
         if (live) {
           float v[32];
@@ -602,7 +607,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           }
         }
       }
-      if (live) p.lse[(tok0 + qrow) * p.hq + h] = (mref + log2f(l)) / kLog2e;
+      if (live && half == 0) p.lse[(tok0 + qrow) * p.hq + h] = (mref + log2f(lt)) / kLog2e;
     }
   }
   tc_fence_before();
@@ -614,8 +619,8 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 }
 
 // --------------------------------------------------------------------------- backward: dQ, tcgen05
-// One CTA per 128 queries of one head (heaviest first), 192 threads: warp 0 TMA (Q and dO once; K
-// and V tiles of 64 keys, double-buffered), warp 1 MMA issuer, warps 2-5 one thread per query row.
+// One CTA per 128 queries of one head (heaviest first), 320 threads: warp 0 TMA (Q and dO once; K
+// and V tiles of 64 keys, double-buffered), warp 1 MMA issuer, warps 2-9 two threads per query row.
 //   S = Q K^T, dP = dO V^T   tcgen05 (bf16), into one of two TMEM buffer pairs;
 //   dS = P (dP - D)          the row's threads, P = exp2(S' - lse'), written bf16 to a swizzled tile;
 //   dQ += dS K               tcgen05 (K read MN-major from the same tile), fp32 in TMEM;
@@ -633,7 +638,7 @@ struct DqTc {
 };
 
 template <int HD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
              const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const AttnBwdArgs p) {
   using C = DqTc<HD>;
@@ -666,9 +671,9 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
+      mbar_init(&s_free[i], 256);
     }
-    mbar_init(ds_full, 128);
+    mbar_init(ds_full, 256);
     mbar_init(dq_done, 1);
     fence_mbar_init();
   }
@@ -747,6 +752,10 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       }
     }
   } else {
+    // two threads per query row (warps 2-5 and 6-9, the same TMEM lanes): half h takes keys
+    // [32h, 32h + 32) of each block, and a quarter of the rotation pairs of the dQ row at the end
+    const int ts = (int)threadIdx.x - 64;
+    const int half = ts >> 7;
     const int r = (warp & 3) * 32 + lane;
     const int qrow = q0 + r;
     const bool live = qrow < p.S;
@@ -762,21 +771,18 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         break;
       }
       tc_fence_after();
-      float ds[C::KB];
+      float ds[32];
       {
         uint32_t us[32], ud[32];
+        tmem_ld32(tmem + st * C::KB + half * 32 + lane_off, us);
+        tmem_ld32(tmem + 128 + st * C::KB + half * 32 + lane_off, ud);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < C::KB; c += 32) {
-          tmem_ld32(tmem + st * C::KB + c + lane_off, us);
-          tmem_ld32(tmem + 128 + st * C::KB + c + lane_off, ud);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int key = j * C::KB + c + e;
-            float pv = exp2f(__uint_as_float(us[e]) * sl2 - lse2);
-            if (!live || key > qrow || key >= p.S) pv = 0.f;
-            ds[c + e] = pv * (__uint_as_float(ud[e]) - dd);
-          }
+        for (int e = 0; e < 32; ++e) {
+          const int key = j * C::KB + half * 32 + e;
+          float pv = exp2f(__uint_as_float(us[e]) * sl2 - lse2);
+          if (!live || key > qrow || key >= p.S) pv = 0.f;
+          ds[e] = pv * (__uint_as_float(ud[e]) - dd);
         }
       }
       tc_fence_before();
@@ -787,10 +793,11 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       }
       uint8_t* row = sDS + r * 128;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 4; ++i) {  // pieces 4 half .. 4 half + 3 of the row
         const float* v = ds + i * 8;
-        uint4 u = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-        *reinterpret_cast<uint4*>(row + ((i ^ (r & 7)) * 16)) = u;
+        const int piece = half * 4 + i;
+        *reinterpret_cast<uint4*>(row + ((piece ^ (r & 7)) * 16)) =
+            make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
       }
       fence_proxy_async();
       tc_fence_before();
@@ -798,8 +805,7 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(dq_done, (nkb - 1) & 1))) {
       tc_fence_after();
-      // the whole dQ row (HD fp32), scaled, with the rotation of position qrow undone
-      float acc[HD];
+      float acc[HD];  // the whole dQ row, scaled
 #pragma unroll
       for (int c = 0; c < HD; c += 32) {
         uint32_t u[32];
@@ -808,17 +814,19 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 #pragma unroll
         for (int e = 0; e < 32; ++e) acc[c + e] = __uint_as_float(u[e]) * p.scale;
       }
-      if (live) {  // pairs (c, c + hd/2) rotated by minus the angle of position qrow, 8 columns at a time
-        constexpr int HALF = HD / 2;
+      if (live) {  // this half's rotation pairs (c, c + hd/2), c in [half hd/4, (half + 1) hd/4)
+        constexpr int HALF = HD / 2, Q4 = HD / 4;
         __nv_bfloat16* dst = p.dq + (tok0 + qrow) * p.lddq + h * HD;
 #pragma unroll
-        for (int c0 = 0; c0 < HALF; c0 += 8) {
+        for (int c0 = 0; c0 < Q4; c0 += 8) {
+          const int c = half * Q4 + c0;
           float y1[8], y2[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float x1 = acc[c0 + e], x2 = acc[c0 + e + HALF];
+            const float x1 = half ? acc[Q4 + c0 + e] : acc[c0 + e];
+            const float x2 = half ? acc[Q4 + c0 + e + HALF] : acc[c0 + e + HALF];
             if (p.rope_cos) {
-              const float cs = p.rope_cos[qrow * HALF + c0 + e], sn = p.rope_sin[qrow * HALF + c0 + e];
+              const float cs = p.rope_cos[qrow * HALF + c + e], sn = p.rope_sin[qrow * HALF + c + e];
               y1[e] = x1 * cs + x2 * sn;
               y2[e] = x2 * cs - x1 * sn;
             } else {
@@ -826,10 +834,10 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
               y2[e] = x2;
             }
           }
-          *reinterpret_cast<uint4*>(dst + c0) = make_uint4(pack_bf16(y1[0], y1[1]), pack_bf16(y1[2], y1[3]),
-                                                           pack_bf16(y1[4], y1[5]), pack_bf16(y1[6], y1[7]));
-          *reinterpret_cast<uint4*>(dst + c0 + HALF) = make_uint4(pack_bf16(y2[0], y2[1]), pack_bf16(y2[2], y2[3]),
-                                                                  pack_bf16(y2[4], y2[5]), pack_bf16(y2[6], y2[7]));
+          *reinterpret_cast<uint4*>(dst + c) = make_uint4(pack_bf16(y1[0], y1[1]), pack_bf16(y1[2], y1[3]),
+                                                          pack_bf16(y1[4], y1[5]), pack_bf16(y1[6], y1[7]));
+          *reinterpret_cast<uint4*>(dst + c + HALF) = make_uint4(pack_bf16(y2[0], y2[1]), pack_bf16(y2[2], y2[3]),
+                                                                 pack_bf16(y2[4], y2[5]), pack_bf16(y2[6], y2[7]));
         }
       }
     }
@@ -843,9 +851,9 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 }
 
 // --------------------------------------------------------------------------- backward: dK, dV, tcgen05
-// grid (grp, B * hkv, ceil(S/128)), cluster (grp, 1, 1), 192 threads. The cluster owns 128 keys of
+// grid (grp, B * hkv, ceil(S/128)), cluster (grp, 1, 1), 320 threads. The cluster owns 128 keys of
 // kv head kvh; its CTA of rank hh sums the contributions of query head kvh * grp + hh over query
-// blocks of 64 (double-buffered Q / dO tiles): warp 0 TMA, warp 1 MMA issuer, warps 2-5 one thread
+// blocks of 64 (double-buffered Q / dO tiles): warp 0 TMA, warp 1 MMA issuer, warps 2-9 two threads
 // per key row.
 //   S^T = K Q^T, dP^T = V dO^T      tcgen05 (bf16), into one of two TMEM buffer pairs;
 //   P^T, dS^T = P^T (dP^T - D)      the key row's thread (lse and D of the block's queries from
@@ -870,7 +878,7 @@ struct DkvTc {
 };
 
 template <int HD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const AttnBwdArgs p) {
   using C = DkvTc<HD>;
@@ -911,9 +919,9 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(&qo_full[i], 1);
       mbar_init(&qo_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
+      mbar_init(&s_free[i], 256);
     }
-    mbar_init(p_full, 128);
+    mbar_init(p_full, 256);
     mbar_init(kv_done, 1);
     fence_mbar_init();
   }
@@ -996,7 +1004,10 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
     }
   } else {
-    const int t = (int)threadIdx.x - 64;   // 0 .. 127
+    // two threads per key row (warps 2-5 and 6-9, the same TMEM lanes): half h takes queries
+    // [32h, 32h + 32) of each block and parks columns [h hd/2, (h + 1) hd/2) of the row at the end
+    const int t = (int)threadIdx.x - 64;   // 0 .. 255
+    const int half = t >> 7;
     const int r = (warp & 3) * 32 + lane;  // key row = TMEM lane
     const int kr = k0 + r;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -1010,7 +1021,7 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     };
     float nl = 0.f, nd = 0.f;
     load_ld(0, nl, nd);
-    // every iteration reaches the named barrier (the four warps together), also after a failed wait
+    // every iteration reaches the named barrier (the eight warps together), also after a failed wait
     for (int j = 0; j < nqb; ++j) {
       const int st = j & 1;
       const int q0 = (i0 + j) * C::QB;
@@ -1019,29 +1030,27 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         sD[st * C::QB + t] = nd;
       }
       load_ld(j + 1, nl, nd);
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 1, 256;" ::: "memory");
       if (!ok) continue;
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1))) {
         ok = false;
         continue;
       }
       tc_fence_after();
-      float pv[C::QB], dv[C::QB];
+      float pv[32], dv[32];
       {
         uint32_t us[32], ud[32];
+        tmem_ld32(tmem + st * C::QB + half * 32 + lane_off, us);
+        tmem_ld32(tmem + 128 + st * C::QB + half * 32 + lane_off, ud);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < C::QB; c += 32) {
-          tmem_ld32(tmem + st * C::QB + c + lane_off, us);
-          tmem_ld32(tmem + 128 + st * C::QB + c + lane_off, ud);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int q = q0 + c + e;
-            float pe = exp2f(__uint_as_float(us[e]) * sl2 - sLse[st * C::QB + c + e]);
-            if (q < kr || q >= p.S || kr >= p.S) pe = 0.f;
-            pv[c + e] = pe;
-            dv[c + e] = pe * (__uint_as_float(ud[e]) - sD[st * C::QB + c + e]);
-          }
+        for (int e = 0; e < 32; ++e) {
+          const int qi = half * 32 + e;
+          const int q = q0 + qi;
+          float pe = exp2f(__uint_as_float(us[e]) * sl2 - sLse[st * C::QB + qi]);
+          if (q < kr || q >= p.S || kr >= p.S) pe = 0.f;
+          pv[e] = pe;
+          dv[e] = pe * (__uint_as_float(ud[e]) - sD[st * C::QB + qi]);
         }
       }
       tc_fence_before();
@@ -1053,10 +1062,10 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       uint8_t* prow = sP + r * 128;
       uint8_t* srow = sS + r * 128;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 4; ++i) {
         const float* a = pv + i * 8;
         const float* d = dv + i * 8;
-        const int pos = (i ^ (r & 7)) * 16;
+        const int pos = ((half * 4 + i) ^ (r & 7)) * 16;
         *reinterpret_cast<uint4*>(prow + pos) =
             make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
         *reinterpret_cast<uint4*>(srow + pos) =
@@ -1066,11 +1075,11 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    // park this head's dK, dV rows (fp32) once the last block's MMAs are done
+    // park this head's dK, dV rows (fp32, this half's columns) once the last block's MMAs are done
     if (ok && __all_sync(0xffffffffu, mbar_wait(kv_done, (nqb - 1) & 1))) {
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < HD; c += 32) {
+      for (int c = half * (HD / 2); c < (half + 1) * (HD / 2); c += 32) {
         uint32_t uk[32], uv[32];
         tmem_ld32(tK + c + lane_off, uk);
         tmem_ld32(tV + c + lane_off, uv);
@@ -1489,7 +1498,7 @@ cudaError_t launch_fwd_tc(const AttnArgs& a, int B, cudaStream_t s) {
     mark_done_on_device(attr_done);
   }
   dim3 grid(a.hq, B, (a.S + C::QB - 1) / C::QB);
-  k_attn_fwd_tc<HD><<<grid, 192, C::SMEM, s>>>(tQ, tK, tV, a);
+  k_attn_fwd_tc<HD><<<grid, 320, C::SMEM, s>>>(tQ, tK, tV, a);
   return cudaSuccess;
 }
 
@@ -1576,7 +1585,7 @@ cudaError_t launch_bwd_tc(const AttnBwdArgs& a, int B, cudaStream_t s) {
   const int grp = a.hq / a.hkv;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grp, (unsigned)(B * a.hkv), (unsigned)((a.S + K::KB - 1) / K::KB));
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(320, 1, 1);
   cfg.dynamicSmemBytes = K::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute at[1];
@@ -1589,7 +1598,7 @@ cudaError_t launch_bwd_tc(const AttnBwdArgs& a, int B, cudaStream_t s) {
   cudaError_t e = cudaLaunchKernelEx(&cfg, k_attn_dkdv_tc<HD>, q64, o64, k128, v128, a);
   if (e != cudaSuccess) return e;
   dim3 gq(a.hq, B, (a.S + Q::QB - 1) / Q::QB);
-  k_attn_dq_tc<HD><<<gq, 192, Q::SMEM, s>>>(q128, o128, k64, v64, a);
+  k_attn_dq_tc<HD><<<gq, 320, Q::SMEM, s>>>(q128, o128, k64, v64, a);
   return cudaGetLastError();
 }
 

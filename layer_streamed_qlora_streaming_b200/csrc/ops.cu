@@ -291,37 +291,44 @@ k_ce(const float* __restrict__ logits, int V, const int32_t* __restrict__ y, flo
 }
 
 // Cross-entropy rows that read each logit once: a thread-block cluster of cs CTAs holds one row
-// in shared memory, CTA z the slice [z * slice, (z + 1) * slice). Each CTA reduces its slice to
-// (max, sum of exp) in a fixed tree; the cs pairs are merged in rank order through distributed
+// in shared memory, CTA z the slice [z * slice, (z + 1) * slice), brought in by one bulk
+// asynchronous copy (the copy engine keeps the whole slice in flight). Each CTA reduces its slice
+// to (max, sum of exp) in a fixed tree; the cs pairs are merged in rank order through distributed
 // shared memory (every CTA gets the same lse); then each CTA writes dlogits of its slice from
-// shared memory, and the CTA holding the target writes the row's loss.
-constexpr int kCeThreads = 512;
-__global__ void __launch_bounds__(kCeThreads, 1)
+// shared memory, and the CTA holding the target writes the row's loss. Needs V % 4 == 0 (16-byte
+// aligned slices).
+constexpr int kCeThreads = 256;
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kCeThreads)
 k_ce_cluster(const float* __restrict__ logits, int V, int slice, const int32_t* __restrict__ y, float inv_T,
              float* __restrict__ loss_rows, bf16* __restrict__ dlog) {
-  extern __shared__ __align__(16) float row_s[];  // [slice], then the CTA's (max, sum) pair
+  extern __shared__ __align__(16) float row_s[];  // [slice], the CTA's (max, sum) pair, an mbarrier
   __shared__ float sm[32], ss[32];
   const int cs = (int)cluster_size_x();
   const int z = (int)cluster_rank();
   const int64_t row = blockIdx.x / cs;
   const int c0 = z * slice, n = max(0, min(V - c0, slice));
-  const float* lr = logits + row * V + c0;
-  float m = -INFINITY, sum = 0.f;
-  if ((V % 4) == 0) {  // slices start on 16-byte boundaries (slice % 4 == 0)
-    const float4* l4 = reinterpret_cast<const float4*>(lr);
-    float4* r4 = reinterpret_cast<float4*>(row_s);
-    for (int c = threadIdx.x; c < n / 4; c += blockDim.x) {
-      const float4 v = __ldg(l4 + c);
-      r4[c] = v;
-      ms_add4(m, sum, v);
-    }
-  } else {
-    for (int c = threadIdx.x; c < n; c += blockDim.x) {
-      const float v = lr[c];
-      row_s[c] = v;
-      ms_add4(m, sum, make_float4(v, -INFINITY, -INFINITY, -INFINITY));
-    }
+  float* pair = row_s + slice;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(pair + 2);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
   }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar, (uint32_t)n * 4);
+    if (n > 0) bulk_load(row_s, logits + row * V + c0, (uint32_t)n * 4, bar);
+  }
+  mbar_wait(bar, 0);
+  float m = -INFINITY, sum = 0.f;
+  const float4* r4 = reinterpret_cast<const float4*>(row_s);
+  for (int c = threadIdx.x; c < n / 4; c += blockDim.x) ms_add4(m, sum, r4[c]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, sum, o);
@@ -333,7 +340,6 @@ k_ce_cluster(const float* __restrict__ logits, int V, int slice, const int32_t* 
     ss[w] = sum;
   }
   __syncthreads();
-  float* pair = row_s + slice;
   if (threadIdx.x == 0) {
     float mm = sm[0], s2 = ss[0];
     for (int i = 1; i < (int)(blockDim.x >> 5); ++i) ms_merge(mm, s2, sm[i], ss[i]);
@@ -356,23 +362,14 @@ k_ce_cluster(const float* __restrict__ logits, int V, int slice, const int32_t* 
   }
   if (threadIdx.x == 0 && tgt >= c0 && tgt < c0 + n) loss_rows[row] = lse - row_s[tgt - c0];
   bf16* dr = dlog + row * V + c0;
-  if ((V % 4) == 0) {
-    const float4* r4 = reinterpret_cast<const float4*>(row_s);
-    for (int c = threadIdx.x; c < n / 4; c += blockDim.x) {
-      const float4 v = r4[c];
-      float p[4] = {expf(v.x - lse), expf(v.y - lse), expf(v.z - lse), expf(v.w - lse)};
-      const int d = tgt - c0 - 4 * c;
-      if (d >= 0 && d < 4) p[d] -= 1.0f;
-      const __nv_bfloat162 h[2] = {__floats2bfloat162_rn(p[0] * inv_T, p[1] * inv_T),
-                                   __floats2bfloat162_rn(p[2] * inv_T, p[3] * inv_T)};
-      *reinterpret_cast<uint2*>(dr + 4 * c) = *reinterpret_cast<const uint2*>(h);
-    }
-  } else {
-    for (int c = threadIdx.x; c < n; c += blockDim.x) {
-      float p = expf(row_s[c] - lse);
-      if (c0 + c == tgt) p -= 1.0f;
-      dr[c] = __float2bfloat16_rn(p * inv_T);
-    }
+  for (int c = threadIdx.x; c < n / 4; c += blockDim.x) {
+    const float4 v = r4[c];
+    float p[4] = {expf(v.x - lse), expf(v.y - lse), expf(v.z - lse), expf(v.w - lse)};
+    const int d = tgt - c0 - 4 * c;
+    if (d >= 0 && d < 4) p[d] -= 1.0f;
+    const __nv_bfloat162 h[2] = {__floats2bfloat162_rn(p[0] * inv_T, p[1] * inv_T),
+                                 __floats2bfloat162_rn(p[2] * inv_T, p[3] * inv_T)};
+    *reinterpret_cast<uint2*>(dr + 4 * c) = *reinterpret_cast<const uint2*>(h);
   }
 }
 
@@ -559,17 +556,18 @@ cudaError_t embed(const int32_t* tok, const bf16* E, int64_t T, int d, int V, fl
 }
 cudaError_t cross_entropy(const float* logits, int64_t T, int V, const int32_t* y, float inv_T, float* loss_rows,
                           bf16* dlog, cudaStream_t s) {
-  // the smallest power-of-two cluster (<= 8) whose slices fit in 200 KB of shared memory each
-  constexpr int64_t kMaxSliceBytes = 200 * 1024;
+  // cluster of 1-8 CTAs with slices of about 64 KB (two or three CTAs an SM); 16-byte slices need
+  // V % 4 == 0, and a slice must fit one CTA's shared memory
+  constexpr int64_t kTargetBytes = 64 * 1024, kMaxSliceBytes = 200 * 1024;
   int cs = 1;
-  while (cs < 8 && (((int64_t)V + cs - 1) / cs + 3) / 4 * 16 > kMaxSliceBytes) cs *= 2;
+  while (cs < 8 && (((int64_t)V + cs - 1) / cs) * 4 > kTargetBytes) cs *= 2;
   const int slice = (int)((((int64_t)V + cs - 1) / cs + 3) / 4 * 4);
-  if ((int64_t)slice * 4 > kMaxSliceBytes || T * cs > INT32_MAX) {
-    k_ce<<<(unsigned)T, 1024, 0, s>>>(logits, V, y, inv_T, loss_rows, dlog);  // rows too long for a cluster
+  if ((V % 4) || (int64_t)slice * 4 > kMaxSliceBytes || T * cs > INT32_MAX) {
+    k_ce<<<(unsigned)T, 1024, 0, s>>>(logits, V, y, inv_T, loss_rows, dlog);  // the two-pass form
     note_launch(1);
     return cudaGetLastError();
   }
-  const int smem = slice * 4 + 16;
+  const int smem = slice * 4 + 16;  // the slice, the (max, sum) pair and the mbarrier
   static std::atomic<unsigned long long> attr_done{0};
   if (!done_on_device(attr_done)) {
     const cudaError_t e = cudaFuncSetAttribute(k_ce_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,

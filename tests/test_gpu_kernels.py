@@ -321,8 +321,8 @@ def test_swiglu_fwd_bwd():
 
 @pytest.mark.parametrize("T,V", [(40, 50000), (24, 128256), (16, 152064), (12, 60001), (20, 1001)])
 def test_cross_entropy_rows(T, V):
-    # one CTA per row up to 200 KB of logits, else a cluster of 2 / 4 holding the row in shared
-    # memory (128256 and 152064: 4 slices; 60001, odd: 2 slices, scalar path)
+    # V % 4 == 0: a cluster of 1-8 CTAs holds the row in shared memory (50000: 4 slices, 128256 and
+    # 152064: 8); otherwise (60001, 1001) the two-pass kernel
     r = _rng(9 + V)
     logits = r.normal(size=(T, V)).astype(np.float32) * 2
     y = r.integers(0, V, size=T).astype(np.int32)
