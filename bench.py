@@ -557,6 +557,29 @@ def run_gpu(args, wl):
              "note": "steady state: the two layers at the forward/backward turn and layers 0, 1 from the "
                      "previous step are not copied again (2L - 4 reads)"}
 
+    # the same 2L copies without copying the next step's first read ahead (A/B of that overlap)
+    ctx.set_prefetch(False)
+    for _ in range(2):
+        one_step()
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    p0.record(stream)
+    for _ in range(args.steps):
+        one_step()
+    p1.record(stream)
+    torch.cuda.synchronize()
+    pms = max_over_ranks(p0.elapsed_time(p1), dist, "cuda")
+    pst = ctx.stats()
+    ctx.set_prefetch(True)
+    no_prefetch = {"value": job_throughput(world, T, args.steps, pms), "unit": UNIT, "ms_per_step": pms / args.steps,
+                   "layer_reads_per_step": pst["layer_reads_last_step"],
+                   "frac": pst["h2d_bytes_last_step"] / (link_gbs * 1e9) * 1e3 / (pms / args.steps),
+                   "note": "every step copies its own first read at its start instead of the step before copying "
+                           "it during its last layer and the optimizer"}
+
     dpo = None
     if wl.vocab and wl.batch % 2 == 0:
         # DPO step on the same model: reference forward with the adapters off + policy step (3L reads)
@@ -650,6 +673,7 @@ def run_gpu(args, wl):
     }
     line["e2e"] = e2e
     line["reuse_schedule"] = reuse
+    line["no_prefetch"] = no_prefetch
     if dpo is not None:
         line["dpo"] = dpo
     ctx.close()

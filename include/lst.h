@@ -255,12 +255,19 @@ lst_status lst_split_plan(int64_t blob_bytes, int32_t world, int32_t rank, int64
  * 0..L-1 once more first); reuse / nf4: the config's reuse and base_format == LST_BASE_NF4;
  * held[2] / wheld[2]: the layers the two pool slots / two bf16 weight scratches hold before the step
  * (-1 = nothing), overwritten with what they hold after it. out: n_reads rows of 8 int32:
- * slot, copy (0/1), wait_free (the read whose compute the copy waits for, -1 none), loaded_by
+ * slot, copy (0/1), wait_free (the read the copy waits for, -1 none: until its compute has finished,
+ * or, in a step whose NF4 base is dequantised in a separate pass with reuse off, until its dequant
+ * has -- the compute then reads only the bf16 scratch and a copy of the blob's header), loaded_by
  * (the read whose copy filled the slot, -1 an earlier step), wslot, dequant (0/1), wwait,
- * wfilled_by (the same for the weight scratch; -1 / 0 for a bf16 base). LST_ERR_ARG on a null
- * pointer, n_reads <= 0 or a negative layer. */
+ * wfilled_by (the same for the weight scratch; -1 / 0 for a bf16 base).
+ * prefetch (may be NULL: no prefetch, as with lst_set_prefetch(ctx, 0)): in, prefetch[0] = the slot
+ * a previous step already copied this step's first read into (-1 none; used with reuse off only);
+ * out, prefetch[0] / prefetch[1] = the slot this step copies the next step's first read into and the
+ * read that copy waits for, as wait_free (-1 / -1 with reuse on). A prefetched first read has
+ * copy 0 and loaded_by -1. LST_ERR_ARG on a null pointer (other than prefetch), n_reads <= 0, a
+ * negative layer or prefetch[0] outside -1..1. */
 lst_status lst_plan_reads(const int32_t* reads, int32_t n_reads, int32_t reuse, int32_t nf4,
-                          int32_t* held, int32_t* wheld, int32_t* out);
+                          int32_t* held, int32_t* wheld, int32_t* prefetch, int32_t* out);
 
 /* Where an NF4 base is dequantised in the next steps: 0 (default) in a separate pass that writes
  * each layer read's bf16 weights to a device scratch, one read ahead on a low-priority stream;
@@ -272,6 +279,13 @@ lst_status lst_set_dequant_mode(lst_ctx* ctx, int32_t mode);
 /* Switch the copy schedule of the next steps (the config's `reuse`): 1 keeps layers that are still
  * in the pool instead of copying them again, 0 copies every read. Results are the same bytes. */
 lst_status lst_set_reuse(lst_ctx* ctx, int32_t reuse);
+
+/* Copy ahead, at the end of each step with reuse off, the next step's first read (layer 0) into the
+ * pool slot that the step's last read does not use, as soon as the read before it has finished: that
+ * copy overlaps the step's last layer and the optimizer instead of starting the next step. Every step
+ * still copies 2L (3L for DPO) layer blobs -- one of them issued by the step before -- and returns
+ * only once that copy has landed. On (1) by default; 0 switches it off. Results are the same bytes. */
+lst_status lst_set_prefetch(lst_ctx* ctx, int32_t on);
 lst_status lst_get_stats(const lst_ctx* ctx, lst_stats* out);
 
 const char* lst_last_error(const lst_ctx* ctx);

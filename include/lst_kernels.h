@@ -82,7 +82,10 @@ lst_status lst_k_gemm_nf4(int32_t M, int32_t N, int32_t K, const uint16_t* A, in
                           const float* bias, const float* R, int64_t ldr, void* stream);
 
 /* Causal GQA attention forward over T = batch*S tokens: q [T, ldq], k [T, ldk], v [T, ldv]
- * (head h at column h*hd), o [T, ldo] bf16, lse [T, hq] fp32. hd in {64, 128}. */
+ * (head h at column h*hd), o [T, ldo] bf16, lse [T, hq] fp32. hd in {64, 128}; row strides
+ * multiples of 8 and bases 16-byte aligned (the tiles are loaded by TMA). The probabilities enter
+ * the P V product as fp16 with V converted to fp16, exact for |v| in [2^-14, 65504]: entries of v
+ * must stay below 65504 in magnitude (larger ones would overflow to infinity). */
 lst_status lst_k_attention_fwd(const uint16_t* q, int64_t ldq, const uint16_t* k, int64_t ldk,
                                const uint16_t* v, int64_t ldv, uint16_t* o, int64_t ldo,
                                float* lse, int64_t T, int32_t S, int32_t hq, int32_t hkv,
@@ -159,6 +162,30 @@ lst_status lst_k_lora_grads(const uint16_t* X, int64_t ldx, int32_t in, const ui
                             const uint16_t* Vs, int32_t KP, int32_t nseg, int32_t r,
                             const int32_t* bounds, float* const* dA, float* const* dB,
                             void* stream);
+
+/* One fused group of lst_k_lora_grads_multi: the arguments of lst_k_lora_grads, with bounds, dA and
+ * dB held in the struct (dA / dB: nseg device pointers; unused entries ignored). */
+typedef struct {
+  const uint16_t* X;
+  int64_t ldx;
+  int32_t in;
+  const uint16_t* dY;
+  int64_t ldy;
+  int32_t out;
+  const uint16_t* Us;
+  const uint16_t* Vs;
+  int32_t KP, nseg, r;
+  int32_t bounds[4];
+  float* dA[3];
+  float* dB[3];
+} lst_lora_grad_group;
+
+/* The adapter gradients of n (1..4) fused groups of the same T in one launch -- what a layer's
+ * backward issues for its four groups -- each group's results as lst_k_lora_grads defines them.
+ * How far the T sums are split over a thread-block cluster follows the launch's total number of
+ * output tiles, so a group's fp32 sums may round differently alone and in company (the bytes are
+ * fixed for a given set of groups). groups: HOST array of n structs. */
+lst_status lst_k_lora_grads_multi(const lst_lora_grad_group* groups, int32_t n, int64_t T, void* stream);
 
 /* Read and clear the device error word of the current device: 0 when no kernel reported a
  * problem, else the code of the first report (1: a bounded wait gave up, 2: an index was out of

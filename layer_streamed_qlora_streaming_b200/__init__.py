@@ -75,7 +75,8 @@ _SIGS = {
     "lst_apply_optimizer": (_I32, [_P, _P]),
     "lst_step_dpo": (_I32, [_P, _P, _P, _P, _I32, _I32, _F32, C.POINTER(C.c_float), _P]),
     "lst_set_reuse": (_I32, [_P, _I32]),
-    "lst_plan_reads": (_I32, [_P, _I32, _I32, _I32, _P, _P, _P]),
+    "lst_set_prefetch": (_I32, [_P, _I32]),
+    "lst_plan_reads": (_I32, [_P, _I32, _I32, _I32, _P, _P, _P, _P]),
     "lst_get_stats": (_I32, [_P, C.POINTER(Stats)]),
     "lst_get_read_timeline": (_I32, [_P, _P, _I32, C.POINTER(_I32)]),
     "lst_set_split_copy": (_I32, [_P, _I32, _I32, _P]),
@@ -88,6 +89,7 @@ _SIGS = {
     "lst_blob_bytes": (_I64, [C.POINTER(Config)]),
     "lst_k_nf4_quantize": (_I32, [_P, _I64, _P, _P, _P, _P, _P]),
     "lst_k_nf4_quantize_noalloc": (_I32, [_P, _I64, _P, _P, _P, _P, _P]),
+    "lst_k_lora_grads_multi": (_I32, [_P, _I32, _I64, _P]),
     "lst_k_nf4_dequant": (_I32, [_P, _P, _P, _P, _I64, _P, _P]),
     "lst_k_gemm_nf4": (_I32, [_I32, _I32, _I32, _P, _I64, _P, _I32, _I32, _P, _I64, _P, _I64, _I32, _P, _I64, _I32,
                               _F32, _P, _P, _I64, _P]),
@@ -182,17 +184,22 @@ def make_config(wl, streamed: bool = True, max_batch=None, max_seq=None, timeout
                   int(bool(reuse)))
 
 
-def plan_reads(reads, reuse: bool, nf4: bool, held=(-1, -1), wheld=(-1, -1)):
+def plan_reads(reads, reuse: bool, nf4: bool, held=(-1, -1), wheld=(-1, -1), prefetch=None):
     """The step's copy / dequant plan (host only): (rows [n, 8] int32 of slot, copy, wait_free,
-    loaded_by, wslot, dequant, wwait, wfilled_by; held after; wheld after)."""
+    loaded_by, wslot, dequant, wwait, wfilled_by; held after; wheld after). With prefetch given (the
+    slot a previous step copied this step's first read into, -1 none) the plan copies the next
+    step's first read ahead, and a fourth item (slot, read it waits for) describes that copy."""
     import numpy as np
     r = np.ascontiguousarray(reads, dtype=np.int32)
     h = np.array(held, dtype=np.int32)
     w = np.array(wheld, dtype=np.int32)
+    pre = None if prefetch is None else np.array([prefetch, -1], dtype=np.int32)
     out = np.zeros((len(r), 8), dtype=np.int32)
-    _check(lib().lst_plan_reads(_ptr(r), len(r), int(bool(reuse)), int(bool(nf4)), _ptr(h), _ptr(w), _ptr(out)),
+    _check(lib().lst_plan_reads(_ptr(r), len(r), int(bool(reuse)), int(bool(nf4)), _ptr(h), _ptr(w),
+                                None if pre is None else _ptr(pre), _ptr(out)),
            what="lst_plan_reads")
-    return out, tuple(int(x) for x in h), tuple(int(x) for x in w)
+    res = (out, tuple(int(x) for x in h), tuple(int(x) for x in w))
+    return res if pre is None else res + ((int(pre[0]), int(pre[1])),)
 
 
 def split_plan(blob: int, world: int, rank: int):
@@ -306,6 +313,9 @@ class Context:
 
     def set_reuse(self, on: bool) -> None:
         _check(lib().lst_set_reuse(self.h, int(on)), self.h, "lst_set_reuse")
+
+    def set_prefetch(self, on: bool) -> None:
+        _check(lib().lst_set_prefetch(self.h, int(on)), self.h, "lst_set_prefetch")
 
     def stats(self) -> dict:
         s = Stats()
@@ -461,6 +471,30 @@ def k_lora_grads(X, ldx, in_f, dY, ldy, out_f, T, Us, Vs, KP, r, bounds, dA, dB,
     pb = (C.c_void_p * 3)(*([_ptr(t) for t in dB] + [None] * (3 - nseg)))
     _check(lib().lst_k_lora_grads(_ptr(X), ldx, in_f, _ptr(dY), ldy, out_f, T, _ptr(Us), _ptr(Vs), KP, nseg, r,
                                   b, pa, pb, _stream(stream)), what="lst_k_lora_grads")
+
+
+class LoraGradGroup(C.Structure):
+    _fields_ = [("X", _P), ("ldx", _I64), ("in_f", _I32), ("dY", _P), ("ldy", _I64), ("out_f", _I32),
+                ("Us", _P), ("Vs", _P), ("KP", _I32), ("nseg", _I32), ("r", _I32), ("bounds", _I32 * 4),
+                ("dA", _P * 3), ("dB", _P * 3)]
+
+
+def k_lora_grads_multi(groups, T, stream=None):
+    """The adapter gradients of up to four fused groups in one launch; groups: dicts with the
+    arguments of k_lora_grads (X, ldx, in_f, dY, ldy, out_f, Us, Vs, KP, r, bounds, dA, dB)."""
+    arr = (LoraGradGroup * len(groups))()
+    for g, a in zip(groups, arr):
+        nseg = len(g["dA"])
+        a.X, a.ldx, a.in_f = _ptr(g["X"]), g["ldx"], g["in_f"]
+        a.dY, a.ldy, a.out_f = _ptr(g["dY"]), g["ldy"], g["out_f"]
+        a.Us, a.Vs, a.KP, a.nseg, a.r = _ptr(g["Us"]), _ptr(g["Vs"]), g["KP"], nseg, g["r"]
+        for k, v in enumerate(g["bounds"]):
+            a.bounds[k] = int(v)
+        for k in range(nseg):
+            a.dA[k] = _ptr(g["dA"][k])
+            a.dB[k] = _ptr(g["dB"][k])
+    _check(lib().lst_k_lora_grads_multi(C.cast(arr, C.c_void_p), len(groups), T, _stream(stream)),
+           what="lst_k_lora_grads_multi")
 
 
 def device_error() -> int:

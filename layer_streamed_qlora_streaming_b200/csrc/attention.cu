@@ -12,6 +12,7 @@
 // blocks with the most work are scheduled first.
 #include "attention.cuh"
 #include "common.cuh"
+#include "ex2.cuh"
 #include "gemm.cuh"
 
 #include <cuda_fp16.h>
@@ -535,13 +536,13 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       if (j == 0) {
         mref = bm;  // block 0 always holds key 0 <= query
       } else if (bm > mref + 8.f) {
-        corr = exp2f(mref - bm);
+        corr = ex2_approx(mref - bm);
         mref = bm;
       }
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < NK; ++e) {
-        x[e] = exp2f(x[e] - mref);
+        x[e] = ex2_approx(x[e] - mref);
         ps[e & 7] += x[e];
       }
       l = l * corr + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
@@ -780,7 +781,7 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int key = j * C::KB + half * 32 + e;
-          float pv = exp2f(__uint_as_float(us[e]) * sl2 - lse2);
+          float pv = ex2_approx(__uint_as_float(us[e]) * sl2 - lse2);
           if (!live || key > qrow || key >= p.S) pv = 0.f;
           ds[e] = pv * (__uint_as_float(ud[e]) - dd);
         }
@@ -1047,7 +1048,7 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int e = 0; e < 32; ++e) {
           const int qi = half * 32 + e;
           const int q = q0 + qi;
-          float pe = exp2f(__uint_as_float(us[e]) * sl2 - sLse[st * C::QB + qi]);
+          float pe = ex2_approx(__uint_as_float(us[e]) * sl2 - sLse[st * C::QB + qi]);
           if (q < kr || q >= p.S || kr >= p.S) pe = 0.f;
           pv[e] = pe;
           dv[e] = pe * (__uint_as_float(ud[e]) - sD[st * C::QB + qi]);

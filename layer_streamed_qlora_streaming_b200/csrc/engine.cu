@@ -329,8 +329,17 @@ struct lst_ctx {
   float* h = nullptr;   // residual after attention, fp32
   __nv_bfloat16 *n1 = nullptr, *qkv = nullptr, *o = nullptr, *n2 = nullptr, *gu = nullptr, *m = nullptr,
                 *wscr[2] = {nullptr, nullptr};
+  // NF4 base: the blob's header (means, norm gains, bias) of the layer each weight scratch holds,
+  // copied by the dequant pass, so that a read's compute needs nothing from its pool slot
+  uint8_t* whdr[2] = {nullptr, nullptr};
+  int64_t hdr_bytes = 0;
+  // this step's pool slots are released by the dequant that read them, not by the compute (NF4
+  // base dequantised in a separate pass, reuse off): a copy waits for that dequant only
+  bool release_at_deq = false;
   float *rstd1 = nullptr, *rstd2 = nullptr, *lse = nullptr, *Dbuf = nullptr;
   float* o32 = nullptr;  // attention output before rounding (recompute pass), for the backward's D
+  LoraGradProb gq[NGROUP];  // adapter-gradient reductions queued by the layer's group backwards
+  int n_gq = 0;
   __nv_bfloat16* Us[NGROUP] = {};  // split bf16 s * x A^T per group [T, KP] (sections hi, lo, hi)
   __nv_bfloat16* Vs[NGROUP] = {};  // split bf16 s * dy B per group [T, KP]
   float *ga = nullptr, *gb = nullptr, *dn = nullptr, *dm = nullptr;
@@ -361,6 +370,13 @@ struct lst_ctx {
   int slot_layer[2] = {-1, -1};  // layers the slots hold after the last completed step (-1: unknown)
   int plan_wheld[2] = {-1, -1};  // layers the weight scratches hold once the planned step has run
   int w_layer[2] = {-1, -1};     // layers the weight scratches hold after the last completed step
+  // prefetch of the next step's first read (reuse off): on between steps unless switched off
+  bool prefetch_on = true;
+  int pre_slot = -1, pre_layer = -1;  // slot holding the next step's first read, copied by the last step
+  int64_t pre_bytes = 0;              // bytes that copy moved over this rank's link
+  int plan_pre[2] = {-1, -1};         // this step's prefetch: slot, read whose compute it waits for
+  bool pre_issued = false;            // the prefetch is enqueued; the step ends when ev_pre has fired
+  cudaEvent_t ev_pre = nullptr;
   std::vector<cudaEvent_t> ev_deqg;  // [n * NCHUNK + g]: chunk g of read n dequantised
   // what the compute stream still waits on for the current read, per chunk: its copy, its dequant
   cudaEvent_t cur_wait[NCHUNK][2] = {};
@@ -641,16 +657,40 @@ lst_status group_bwd(lst_ctx* c, int layer, int g, const uint8_t* blob, const __
     ProfScope ps(c, c->stream, PC_GEMM, 2.0 * T * G.in * (double)(G.out + G.KP));
     CK(gemm_bf16(a, c->stream));
   }
-  ProfScope ps(c, c->stream, PC_LORA);
-  float* dA[3] = {nullptr, nullptr, nullptr};
-  float* dB[3] = {nullptr, nullptr, nullptr};
-  for (int k = 0; k < G.nseg; ++k) {
-    dA[k] = c->grads + c->offA[layer * NPROJ + G.proj[k]];
-    dB[k] = c->grads + c->offB[layer * NPROJ + G.proj[k]];
-  }
   // dA = s V^T X and dB = s dY^T U, with s folded into Vs and Us (their hi sections: the gradients are
-  // fp32 reductions of bf16 products, so the lo parts would only refine the last bits of V and U)
-  CK(lora_grads(X, ldx, G.in, dY, ldy, G.out, T, c->Us[g], c->Vs[g], G.KP, G.nseg, c->r, G.bounds, dA, dB, c->stream));
+  // fp32 reductions of bf16 products, so the lo parts would only refine the last bits of V and U);
+  // queued here, launched for all four groups of the layer at once (flush_grads)
+  if (c->n_gq >= NGROUP) return fail(c, LST_ERR_STATE, "adapter-gradient queue full");
+  LoraGradProb& q = c->gq[c->n_gq++];
+  q = LoraGradProb{};
+  q.X = X;
+  q.ldx = ldx;
+  q.in = G.in;
+  q.dY = dY;
+  q.ldy = ldy;
+  q.out = G.out;
+  q.Us = c->Us[g];
+  q.Vs = c->Vs[g];
+  q.KP = G.KP;
+  q.nseg = G.nseg;
+  q.r = c->r;
+  for (int k = 0; k <= G.nseg; ++k) q.bounds[k] = G.bounds[k];
+  for (int k = 0; k < G.nseg; ++k) {
+    q.dA[k] = c->grads + c->offA[layer * NPROJ + G.proj[k]];
+    q.dB[k] = c->grads + c->offB[layer * NPROJ + G.proj[k]];
+  }
+  return LST_OK;
+}
+
+// The queued adapter-gradient reductions of the layer's groups in one launch. Their inputs (each
+// group's X, dY, Us and Vs) are all still in place: the layer's backward writes none of them after
+// they are made, and the launch comes before the last RMSNorm backward overwrites dL/dx_{i+1}.
+lst_status flush_grads(lst_ctx* c) {
+  if (c->n_gq == 0) return LST_OK;
+  ProfScope ps(c, c->stream, PC_LORA);
+  const int n = c->n_gq;
+  c->n_gq = 0;
+  CK(lora_grads_multi(c->gq, n, c->curT, c->stream));
   return LST_OK;
 }
 
@@ -686,12 +726,15 @@ lst_status wait_chunk(lst_ctx* c, int g) {
   return LST_OK;
 }
 
-lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16* W, bool recompute) {
+// blob: the layer's pool slot (or resident copy); hdr: where its header (norm gains, bias) is read
+// from -- the blob itself, or the copy the dequant pass made next to the weight scratch.
+lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const uint8_t* hdr, const __nv_bfloat16* W,
+                     bool recompute) {
   const int64_t T = c->curT;
   const int S = (int)c->curS;
-  const float* g1 = reinterpret_cast<const float*>(blob + c->lay.norms);
+  const float* g1 = reinterpret_cast<const float*>(hdr + c->lay.norms);
   const float* g2 = g1 + c->d;
-  const float* bias = c->cfg.qkv_bias ? reinterpret_cast<const float*>(blob + c->lay.bias) : nullptr;
+  const float* bias = c->cfg.qkv_bias ? reinterpret_cast<const float*>(hdr + c->lay.bias) : nullptr;
   const float* x = c->xs + (int64_t)i * c->Tmax * c->d;
   TRY(wait_chunk(c, 0));  // norm gains, bias and the q/k/v weights
   {
@@ -738,12 +781,13 @@ lst_status layer_fwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
 }
 
 // dL/dx_{i+1} is in c->ga (fp32) and c->dout_b (bf16); leaves dL/dx_i there.
-lst_status layer_bwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16* W) {
+lst_status layer_bwd(lst_ctx* c, int i, const uint8_t* blob, const uint8_t* hdr, const __nv_bfloat16* W) {
   const int64_t T = c->curT;
   const int S = (int)c->curS;
-  const float* g1 = reinterpret_cast<const float*>(blob + c->lay.norms);
+  const float* g1 = reinterpret_cast<const float*>(hdr + c->lay.norms);
   const float* g2 = g1 + c->d;
   const float* x = c->xs + (int64_t)i * c->Tmax * c->d;
+  c->n_gq = 0;
   TRY(group_bwd(c, i, G_DOWN, blob, W, c->dout_b, c->d, c->m, c->F, c->dm, 1));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
@@ -784,6 +828,7 @@ lst_status layer_bwd(lst_ctx* c, int i, const uint8_t* blob, const __nv_bfloat16
     CK(attention_bwd(a, c->stream));
   }
   TRY(group_bwd(c, i, G_QKV, blob, W, c->dqkvb, c->dqkv, c->n1, c->d, c->dn, 1));
+  TRY(flush_grads(c));  // before dout_b (the down group's dY) is overwritten below
   {
     ProfScope ps(c, c->stream, PC_OTHER);
     CK(rmsnorm_bwd(c->dn, x, g1, c->rstd1, c->gb, T, c->d, c->ga, c->dout_b, c->stream));
@@ -937,17 +982,32 @@ lst_status head_dpo(lst_ctx* c) {
 //  - reuse on: a read whose layer is still held by a slot (the two layers at the forward/backward
 //    turn; layers 0 and 1 left by the previous step's backward) uses it as it is; otherwise it copies
 //    into the slot the previous read does not use (for read 0, the slot whose layer is needed last).
-// A copy into a slot waits until the last read that computed from that slot has finished.
+// A copy into a slot waits until the last read that used that slot no longer needs it: until its
+// compute has finished, or -- in a step whose NF4 base is dequantised in a separate pass, with reuse
+// off -- until its dequant has (that pass also copies the blob's header, the norm gains and bias,
+// next to the bf16 scratch, so the compute reads nothing from the slot). The copies can then run
+// up to four reads ahead of the compute: two in the slots, two in the scratches.
 // An NF4 base is dequantised into one of two bf16 weight scratches by the same rule (a read reuses
 // a scratch that still holds its layer only with reuse on), on the prep stream, one read ahead: the
 // dequant of read n+1 overlaps the compute of read n.
+// With reuse off a step can also copy the next step's first read ahead (pre != null): into the slot
+// the step's last read does not use, once the last read that computed from that slot has finished,
+// so the copy overlaps the step's last read and the optimizer; the step ends when it has landed.
+// The next step then computes its first read from that slot without copying it (its copy was that
+// prefetch): 2L copies per step all the same, one of them issued by the step before.
 // The planning itself, on host data only: layers[n] is the layer of read n; held / wheld are the
 // layers the two slots / weight scratches hold before the step (-1: nothing known) and are updated
-// to what they hold after it.
+// to what they hold after it. pre[0] is the slot a previous step prefetched this step's first read
+// into (-1: none); on return pre[0] / pre[1] are the slot this step prefetches the next step's first
+// read into and the read whose compute that copy waits for (-1 / -1 with reuse on).
 void plan_schedule(const std::vector<int>& layers, bool reuse, bool nf4, int held[2], int wheld[2],
-                   std::vector<ReadPlan>& plan) {
+                   std::vector<ReadPlan>& plan, int* pre = nullptr) {
   const int R = (int)layers.size();
-  if (!reuse) held[0] = held[1] = wheld[0] = wheld[1] = -1;
+  const int pre_in = pre && !reuse && pre[0] >= 0 && pre[0] < 2 ? pre[0] : -1;
+  if (!reuse) {
+    held[0] = held[1] = wheld[0] = wheld[1] = -1;
+    if (pre_in >= 0) held[pre_in] = layers[0];
+  }
   int last_use[2] = {-1, -1}, loaded_by[2] = {-1, -1};
   int wlast[2] = {-1, -1}, wfill[2] = {-1, -1};
   auto first_need = [&](int layer) {
@@ -963,6 +1023,8 @@ void plan_schedule(const std::vector<int>& layers, bool reuse, bool nf4, int hel
     if (reuse) {
       if (held[0] == j) p.slot = 0;
       else if (held[1] == j) p.slot = 1;
+    } else if (n == 0 && pre_in >= 0) {
+      p.slot = pre_in;  // copied by the previous step's prefetch
     }
     p.copy = p.slot < 0;
     if (p.copy) {
@@ -995,27 +1057,37 @@ void plan_schedule(const std::vector<int>& layers, bool reuse, bool nf4, int hel
     p.wfilled_by = wfill[p.wslot];
     wlast[p.wslot] = n;
   }
+  if (pre) {
+    pre[0] = pre[1] = -1;
+    if (!reuse) {
+      const int s = 1 - plan[R - 1].slot;
+      pre[0] = s;
+      pre[1] = last_use[s];
+      held[s] = layers[0];
+    }
+  }
 }
 
 void plan_reads(lst_ctx* c) {
   const bool reuse = c->cfg.reuse != 0;
   int held[2] = {c->slot_layer[0], c->slot_layer[1]};
   int wheld[2] = {c->w_layer[0], c->w_layer[1]};
-  plan_schedule(c->rd_layer, reuse, c->cfg.base_format != LST_BASE_BF16, held, wheld, c->plan);
+  const bool pre = c->cfg.streamed && c->prefetch_on;
+  c->plan_pre[0] = pre && c->pre_layer == c->rd_layer[0] ? c->pre_slot : -1;
+  c->plan_pre[1] = -1;
+  plan_schedule(c->rd_layer, reuse, c->cfg.base_format != LST_BASE_BF16, held, wheld, c->plan,
+                pre ? c->plan_pre : nullptr);
   c->plan_held[0] = held[0];
   c->plan_held[1] = held[1];
   c->plan_wheld[0] = wheld[0];
   c->plan_wheld[1] = wheld[1];
 }
 
-lst_status enqueue_copy(lst_ctx* c, int n) {
-  const int j = c->rd_layer[n];
-  NvtxRange nr("copy read %d (layer %d)", n, j);
-  const ReadPlan& p = c->plan[n];
+// Copy layer j's blob from the pinned arena into pool slot `slot` on the copy stream. chunk_ev
+// (NCHUNK events, or null) is recorded after each weight group has landed; *bytes is what crossed
+// this rank's link.
+lst_status copy_layer(lst_ctx* c, int slot, int j, cudaEvent_t* chunk_ev, int64_t* bytes_out) {
   if (c->faults.fail_memcpy()) return fail(c, LST_ERR_CUDA, "layer copy enqueue failed (injected)");
-  if (p.wait_free >= 0) CK(cudaStreamWaitEvent(c->copy_stream, c->ev_free[p.wait_free], 0));
-  ProfScope ps(c, c->copy_stream, PC_COPY);
-  TRY(tl_record(c, n, lst_ctx::TL_COPY0, c->copy_stream));
   const uint8_t* src = c->arena + (int64_t)j * c->lay.total;
   if (c->nccl_comm) {
     // this rank's slice over its own link, then the whole blob from every rank's slice over
@@ -1023,24 +1095,57 @@ lst_status enqueue_copy(lst_ctx* c, int n) {
     int64_t off = 0, bytes = 0, count = 0;
     split_plan(c->lay.total, c->split_world, c->split_rank, &off, &bytes, &count);
     if (bytes > 0)
-      CK(cudaMemcpyAsync(c->pool[p.slot] + off, src + off, bytes, cudaMemcpyHostToDevice, c->copy_stream));
-    const int r = nccl().all_gather(c->pool[p.slot] + off, c->pool[p.slot], (size_t)count, kNcclUint8, c->nccl_comm,
+      CK(cudaMemcpyAsync(c->pool[slot] + off, src + off, bytes, cudaMemcpyHostToDevice, c->copy_stream));
+    const int r = nccl().all_gather(c->pool[slot] + off, c->pool[slot], (size_t)count, kNcclUint8, c->nccl_comm,
                                     c->copy_stream);
     if (r != 0) return fail(c, LST_ERR_CUDA, std::string("ncclAllGather: ") + nccl().error_string(r));
-    for (int g = 0; g < NCHUNK; ++g) CK(cudaEventRecord(c->ev_chunk[n * NCHUNK + g], c->copy_stream));
-    TRY(tl_record(c, n, lst_ctx::TL_COPY1, c->copy_stream));
-    c->st.layer_reads_last_step += 1;
-    c->st.h2d_bytes_last_step += bytes;
+    if (chunk_ev)
+      for (int g = 0; g < NCHUNK; ++g) CK(cudaEventRecord(chunk_ev[g], c->copy_stream));
+    *bytes_out = bytes;
     return LST_OK;
   }
   for (int g = 0; g < NCHUNK; ++g) {  // group by group, so compute can start on the first group
-    CK(cudaMemcpyAsync(c->pool[p.slot] + c->lay.chunk[g], src + c->lay.chunk[g], c->lay.chunk[g + 1] - c->lay.chunk[g],
+    CK(cudaMemcpyAsync(c->pool[slot] + c->lay.chunk[g], src + c->lay.chunk[g], c->lay.chunk[g + 1] - c->lay.chunk[g],
                        cudaMemcpyHostToDevice, c->copy_stream));
-    CK(cudaEventRecord(c->ev_chunk[n * NCHUNK + g], c->copy_stream));
+    if (chunk_ev) CK(cudaEventRecord(chunk_ev[g], c->copy_stream));
   }
+  *bytes_out = c->lay.total;
+  return LST_OK;
+}
+
+// The event after which read n no longer needs its pool slot: its dequant when the slots are
+// released there, else the end of its compute.
+cudaEvent_t slot_release(lst_ctx* c, int n) {
+  return c->release_at_deq ? c->ev_deqg[(size_t)n * NCHUNK + NCHUNK - 1] : c->ev_free[n];
+}
+
+lst_status enqueue_copy(lst_ctx* c, int n) {
+  const int j = c->rd_layer[n];
+  NvtxRange nr("copy read %d (layer %d)", n, j);
+  const ReadPlan& p = c->plan[n];
+  if (p.wait_free >= 0) CK(cudaStreamWaitEvent(c->copy_stream, slot_release(c, p.wait_free), 0));
+  ProfScope ps(c, c->copy_stream, PC_COPY);
+  TRY(tl_record(c, n, lst_ctx::TL_COPY0, c->copy_stream));
+  int64_t bytes = 0;
+  TRY(copy_layer(c, p.slot, j, &c->ev_chunk[(size_t)n * NCHUNK], &bytes));
   TRY(tl_record(c, n, lst_ctx::TL_COPY1, c->copy_stream));
   c->st.layer_reads_last_step += 1;
-  c->st.h2d_bytes_last_step += c->lay.total;
+  c->st.h2d_bytes_last_step += bytes;
+  return LST_OK;
+}
+
+// The next step's first read, copied ahead into the slot plan_pre names once the read that last
+// computes from it has finished; counted as a read of the next step, which finds it in place.
+lst_status enqueue_prefetch(lst_ctx* c) {
+  const int slot = c->plan_pre[0], wait = c->plan_pre[1], j = c->rd_layer[0];
+  NvtxRange nr("prefetch into slot %d (layer %d)", slot, j);
+  if (wait >= 0) CK(cudaStreamWaitEvent(c->copy_stream, slot_release(c, wait), 0));
+  ProfScope ps(c, c->copy_stream, PC_COPY);
+  int64_t bytes = 0;
+  TRY(copy_layer(c, slot, j, nullptr, &bytes));
+  CK(cudaEventRecord(c->ev_pre, c->copy_stream));
+  c->pre_issued = true;
+  c->pre_bytes = bytes;
   return LST_OK;
 }
 
@@ -1101,9 +1206,17 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
     return streamed ? c->pool[c->plan[n].slot] : c->resident + (int64_t)c->rd_layer[n] * c->lay.total;
   };
   plan_reads(c);
+  c->release_at_deq = streamed && nf4 && !c->cfg.reuse && c->whdr[0] != nullptr;
+  for (int g = 0; g < NCHUNK; ++g) c->release_at_deq = c->release_at_deq && !fused_group(c, g);
   // the slots' and scratches' contents are only trusted again once this step has completed
   c->slot_layer[0] = c->slot_layer[1] = -1;
   c->w_layer[0] = c->w_layer[1] = -1;
+  if (streamed && !c->cfg.reuse && !c->plan[0].copy) {  // the last step copied this first read
+    c->st.layer_reads_last_step += 1;
+    c->st.h2d_bytes_last_step += c->pre_bytes;
+  }
+  c->pre_slot = c->pre_layer = -1;
+  c->pre_issued = false;
   // copies and dequants of this step start after everything already on the compute stream (e.g. a
   // step that returned early with work in flight)
   CK(cudaEventRecord(c->ev_start, c->stream));
@@ -1124,6 +1237,8 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
       if (streamed && p.loaded_by >= 0)
         CK(cudaStreamWaitEvent(c->prep_stream, c->ev_chunk[p.loaded_by * NCHUNK + g], 0));
       if (!started) TRY(tl_record(c, m, lst_ctx::TL_DEQ0, c->prep_stream));
+      if (g == 0 && c->release_at_deq)  // the header lies in chunk 0
+        CK(copy16(blob_of(m), c->whdr[p.wslot], c->hdr_bytes, c->prep_stream));
       started = true;
       TRY(dequant_chunk(c, blob_of(m), c->wscr[p.wslot], g, c->prep_stream));
       CK(cudaEventRecord(c->ev_deqg[m * NCHUNK + g], c->prep_stream));
@@ -1150,20 +1265,21 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
     }
     const __nv_bfloat16* W =
         nf4 ? c->wscr[p.wslot] : reinterpret_cast<const __nv_bfloat16*>(blob + c->lay.w16);
+    const uint8_t* hdr = c->release_at_deq ? c->whdr[p.wslot] : blob;
     if (c->profiling) {  // the read's compute starts once its first weight group is in place
       TRY(wait_chunk(c, 0));
       TRY(tl_record(c, n, lst_ctx::TL_COMP0, c->stream));
     }
     if (kind == RD_REF) {
       c->adapters_off = true;
-      const lst_status st = layer_fwd(c, j, blob, W, false);
+      const lst_status st = layer_fwd(c, j, blob, hdr, W, false);
       c->adapters_off = false;
       TRY(st);
     } else if (kind == RD_FWD) {
-      TRY(layer_fwd(c, j, blob, W, false));
+      TRY(layer_fwd(c, j, blob, hdr, W, false));
     } else {
-      TRY(layer_fwd(c, j, blob, W, true));
-      TRY(layer_bwd(c, j, blob, W));
+      TRY(layer_fwd(c, j, blob, hdr, W, true));
+      TRY(layer_bwd(c, j, blob, hdr, W));
     }
     CK(cudaEventRecord(c->ev_free[n], c->stream));
     TRY(tl_record(c, n, lst_ctx::TL_COMP1, c->stream));
@@ -1176,6 +1292,7 @@ lst_status run_layers(lst_ctx* c, HeadMode mode) {
     if (kind != RD_BWD && (n + 1 == R || c->rd_kind[n + 1] != kind)) TRY(head_after(c, kind, mode));
     if (streamed) TRY(issue_copies(c, n, next_copy));
   }
+  if (streamed && c->plan_pre[0] >= 0) TRY(enqueue_prefetch(c));
   return LST_OK;
 }
 
@@ -1189,6 +1306,7 @@ lst_status finish_step(lst_ctx* c, float* loss, float* grads_out) {
     CK(cudaMemcpyAsync(grads_out, c->grads, c->lora_numel * 4, dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
                        c->stream));
   }
+  if (c->pre_issued) CK(cudaStreamWaitEvent(c->stream, c->ev_pre, 0));  // the next step's first read landed
   CK(cudaMemcpyAsync(c->host_loss, c->loss_dev, 4, cudaMemcpyDeviceToHost, c->stream));
   if (c->profiling) CK(cudaEventRecord(c->prof_step1, c->stream));
   CK(cudaEventRecord(c->ev_done, c->stream));
@@ -1216,6 +1334,10 @@ lst_status finish_step(lst_ctx* c, float* loss, float* grads_out) {
   if (c->cfg.streamed) {
     c->slot_layer[0] = c->plan_held[0];
     c->slot_layer[1] = c->plan_held[1];
+    if (c->pre_issued) {
+      c->pre_slot = c->plan_pre[0];
+      c->pre_layer = c->rd_layer[0];
+    }
   }
   c->w_layer[0] = c->plan_wheld[0];
   c->w_layer[1] = c->plan_wheld[1];
@@ -1439,6 +1561,11 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
     TRY(dalloc(c, &c->wscr[1], c->lay.P + kGuardBytes / 2));
     TRY(add_guard(c, reinterpret_cast<uint8_t*>(c->wscr[0] + c->lay.P)));
     TRY(add_guard(c, reinterpret_cast<uint8_t*>(c->wscr[1] + c->lay.P)));
+    c->hdr_bytes = c->lay.packed[0];  // means, norm gains and bias come first
+    if (k.streamed) {
+      TRY(dalloc(c, &c->whdr[0], c->hdr_bytes));
+      TRY(dalloc(c, &c->whdr[1], c->hdr_bytes));
+    }
   }
 
   // activations
@@ -1513,6 +1640,7 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   CK(cudaEventCreateWithFlags(&c->ev_done, cudaEventDisableTiming));
   CK(cudaEventCreateWithFlags(&c->ev_start, cudaEventDisableTiming));
   CK(cudaEventCreateWithFlags(&c->ev_d2h, cudaEventDisableTiming));
+  CK(cudaEventCreateWithFlags(&c->ev_pre, cudaEventDisableTiming));
   CK(cudaEventCreate(&c->prof_step0));
   CK(cudaEventCreate(&c->prof_step1));
   CK(cudaStreamSynchronize(c->stream));
@@ -1546,6 +1674,7 @@ void free_all(lst_ctx* c) {
   if (c->ev_done) cudaEventDestroy(c->ev_done);
   if (c->ev_start) cudaEventDestroy(c->ev_start);
   if (c->ev_d2h) cudaEventDestroy(c->ev_d2h);
+  if (c->ev_pre) cudaEventDestroy(c->ev_pre);
   if (c->prof_step0) cudaEventDestroy(c->prof_step0);
   if (c->prof_step1) cudaEventDestroy(c->prof_step1);
   if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
@@ -1712,9 +1841,12 @@ lst_status lst_register_layer(lst_ctx* c, int32_t layer, const lst_layer_weights
   if (!c) return LST_ERR_ARG;
   DeviceScope ds(c);
   if (!w || layer < 0 || layer >= c->L) return fail(c, LST_ERR_ARG, "bad layer index or null weights");
-  // the layer's bytes change: nothing kept in the pool or the weight scratch is trusted any more
+  // the layer's bytes change: nothing kept in the pool or the weight scratch is trusted any more,
+  // and no copy from the arena may still be running (a prefetch of the next step's first read)
+  CK(cudaStreamSynchronize(c->copy_stream));
   c->slot_layer[0] = c->slot_layer[1] = -1;
   c->w_layer[0] = c->w_layer[1] = -1;
+  c->pre_slot = c->pre_layer = -1;
   return register_impl(c, layer, w);
 }
 
@@ -1954,6 +2086,7 @@ lst_status lst_set_split_copy(lst_ctx* c, int32_t rank, int32_t world, const voi
     }
     c->pool_bytes = world * count;
     c->slot_layer[0] = c->slot_layer[1] = -1;
+    c->pre_slot = c->pre_layer = -1;
   }
   NcclUid id;
   std::memcpy(&id, unique_id, sizeof(id));
@@ -1982,14 +2115,20 @@ lst_status lst_get_read_timeline(const lst_ctx* c, float* out, int32_t max_reads
 }
 
 lst_status lst_plan_reads(const int32_t* reads, int32_t n_reads, int32_t reuse, int32_t nf4, int32_t* held,
-                          int32_t* wheld, int32_t* out) {
+                          int32_t* wheld, int32_t* prefetch, int32_t* out) {
   if (!reads || n_reads <= 0 || !held || !wheld || !out) return LST_ERR_ARG;
   std::vector<int> layers(reads, reads + n_reads);
   for (int v : layers)
     if (v < 0) return LST_ERR_ARG;
+  if (prefetch && (prefetch[0] < -1 || prefetch[0] > 1)) return LST_ERR_ARG;
   int h[2] = {held[0], held[1]}, w[2] = {wheld[0], wheld[1]};
+  int pre[2] = {prefetch ? prefetch[0] : -1, -1};
   std::vector<ReadPlan> plan;
-  plan_schedule(layers, reuse != 0, nf4 != 0, h, w, plan);
+  plan_schedule(layers, reuse != 0, nf4 != 0, h, w, plan, prefetch ? pre : nullptr);
+  if (prefetch) {
+    prefetch[0] = pre[0];
+    prefetch[1] = pre[1];
+  }
   for (int n = 0; n < n_reads; ++n) {
     const ReadPlan& p = plan[n];
     const int32_t row[8] = {p.slot, p.copy ? 1 : 0, p.wait_free, p.loaded_by,
@@ -2016,6 +2155,13 @@ lst_status lst_set_dequant_mode(lst_ctx* c, int32_t mode) {
 lst_status lst_set_reuse(lst_ctx* c, int32_t reuse) {
   if (!c) return LST_ERR_ARG;
   c->cfg.reuse = reuse != 0;
+  return LST_OK;
+}
+
+lst_status lst_set_prefetch(lst_ctx* c, int32_t on) {
+  if (!c) return LST_ERR_ARG;
+  c->prefetch_on = on != 0;
+  if (!c->prefetch_on) c->pre_slot = c->pre_layer = -1;
   return LST_OK;
 }
 

@@ -239,6 +239,36 @@ lst_status lst_k_lora_grads(const uint16_t* X, int64_t ldx, int32_t in, const ui
   return st(lora_grads(B16(X), ldx, in, B16(dY), ldy, out, T, B16(Us), B16(Vs), KP, nseg, r, b, dA, dB, S(stream)));
 }
 
+lst_status lst_k_lora_grads_multi(const lst_lora_grad_group* groups, int32_t n, int64_t T, void* stream) {
+  if (!groups || n < 1 || n > 4 || T <= 0) return LST_ERR_ARG;
+  LoraGradProb q[4];
+  for (int i = 0; i < n; ++i) {
+    const lst_lora_grad_group& g = groups[i];
+    if (!g.X || !g.dY || !g.Us || !g.Vs || g.in <= 0 || g.out <= 0) return LST_ERR_ARG;
+    if (g.nseg < 1 || g.nseg > 3 || g.r <= 0 || g.nseg * g.r > g.KP || (g.KP % 8)) return LST_ERR_ARG;
+    if (g.bounds[0] != 0 || g.bounds[g.nseg] != g.out) return LST_ERR_ARG;
+    q[i] = LoraGradProb{};
+    q[i].X = B16(g.X);
+    q[i].ldx = g.ldx;
+    q[i].in = g.in;
+    q[i].dY = B16(g.dY);
+    q[i].ldy = g.ldy;
+    q[i].out = g.out;
+    q[i].Us = B16(g.Us);
+    q[i].Vs = B16(g.Vs);
+    q[i].KP = g.KP;
+    q[i].nseg = g.nseg;
+    q[i].r = g.r;
+    for (int p = 0; p <= g.nseg; ++p) q[i].bounds[p] = g.bounds[p];
+    for (int p = 0; p < g.nseg; ++p) {
+      if (!g.dA[p] || !g.dB[p] || g.bounds[p + 1] <= g.bounds[p]) return LST_ERR_ARG;
+      q[i].dA[p] = g.dA[p];
+      q[i].dB[p] = g.dB[p];
+    }
+  }
+  return st(lora_grads_multi(q, n, T, S(stream)));
+}
+
 int64_t lst_k_launch_count(void) { return g_launch_count.load(); }
 
 }  // extern "C"

@@ -99,19 +99,30 @@ __device__ __forceinline__ void side_store(const SideOut& o, int row, int col, f
   }
 }
 
-// grid (cs, ceil(M/128), ceil(N/64)), cluster (cs, 1, 1), 192 threads: warp 0 TMA producer, warp 1
-// TMEM owner + MMA issuer, warps 2-5 park the accumulator; then all threads sum and store.
+// One problem of a launch: C [M, N] = A B^T over the launch's K, its operands' tensor maps, its
+// destination, the first output tile (cluster row) it owns and its number of M-tiles.
+constexpr int kMaxProbs = 8;
+struct SideProb {
+  CUtensorMap tA, tB;
+  SideOut o;
+  int tile0, mt;
+};
+struct SideProbs {
+  SideProb p[kMaxProbs];
+  int np;
+};
+
+// grid (cs, tiles), cluster (cs, 1, 1), 192 threads: warp 0 TMA producer, warp 1 TMEM owner + MMA
+// issuer, warps 2-5 park the accumulator; then all threads sum and store.
 // AMN / BMN: A / B MN-major ([K, M] / [K, N] row-major in memory), else K-major.
 // DUAL: every K step also loads the B tile b_off further along N (rows of a K-major B, columns of
 // an MN-major B) and accumulates its product with the same A tile.
-// A launch may carry two problems of the same K (the dA and dB reductions of a group): clusters
-// blockIdx.y < tiles1 take tiles of (tmA, tmB, o) in M-fastest order over mt1 M-tiles, the rest
-// tiles of (tmA2, tmB2, o2) over mt2.
+// A launch carries up to kMaxProbs problems of the same K (e.g. the dA and dB reductions of every
+// group of a layer): cluster row y belongs to the last problem whose tile0 <= y and takes that
+// problem's tile y - tile0, in M-fastest order over its M-tiles.
 template <int AMN, int BMN, int DUAL>
 __global__ void __launch_bounds__(192, 2)
-k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const SideOut o,
-       const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, const SideOut o2,
-       const int tiles1, const int mt1, const int mt2, const int nk, const int kps, const int b_off) {
+k_side(const __grid_constant__ SideProbs P, const int nk, const int kps, const int b_off) {
   constexpr int kStages = SideCfg<DUAL>::kStages;
   constexpr uint32_t kStageB = SideCfg<DUAL>::kStageB;
   extern __shared__ uint8_t smem_raw[];
@@ -128,13 +139,14 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   const int lane = threadIdx.x & 31;
   const int cs = (int)gridDim.x;  // one cluster = the K slices of one output tile
   const int z = (int)cluster_rank();
-  const bool second = (int)blockIdx.y >= tiles1;
-  const int tt = second ? (int)blockIdx.y - tiles1 : (int)blockIdx.y;
-  const int mtp = second ? mt2 : mt1;
-  const int m0 = (tt % mtp) * kBM, n0 = (tt / mtp) * kBN;
-  const CUtensorMap* ma = second ? &tmA2 : &tmA;
-  const CUtensorMap* mb = second ? &tmB2 : &tmB;
-  const SideOut& oo = second ? o2 : o;
+  int pi = 0;
+  while (pi + 1 < P.np && (int)blockIdx.y >= P.p[pi + 1].tile0) ++pi;
+  const SideProb& pr = P.p[pi];
+  const int tt = (int)blockIdx.y - pr.tile0;
+  const int m0 = (tt % pr.mt) * kBM, n0 = (tt / pr.mt) * kBN;
+  const CUtensorMap* ma = &pr.tA;
+  const CUtensorMap* mb = &pr.tB;
+  const SideOut& oo = pr.o;
   const int kb0 = z * kps;
   const int nkb = max(0, min(nk - kb0, kps));
 
@@ -265,12 +277,10 @@ k_side(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   }
 }
 
-// One problem [M, N] (or, with tA2 given, two problems [M, N] and [M2, N2] of the same K in one
-// launch: the clusters of the second follow those of the first).
+// The problems of P (np >= 1, each with tA, tB, o set and o.M, o.N its output size) in one launch
+// over the common K; fills in their tile0 / mt.
 template <int AMN, int BMN, int DUAL = 0>
-cudaError_t launch_side(const CUtensorMap& tA, const CUtensorMap& tB, int M, int N, int K, const SideOut& o,
-                        cudaStream_t st, int b_off = 0, const CUtensorMap* tA2 = nullptr,
-                        const CUtensorMap* tB2 = nullptr, int M2 = 0, int N2 = 0, const SideOut* o2 = nullptr) {
+cudaError_t launch_side(SideProbs& P, int K, cudaStream_t st, int b_off = 0) {
   constexpr uint32_t kSmem = SideCfg<DUAL>::kSmem;
   static std::atomic<unsigned long long> attr_done{0};  // devices whose function attribute is set
   if (!done_on_device(attr_done)) {
@@ -278,10 +288,17 @@ cudaError_t launch_side(const CUtensorMap& tA, const CUtensorMap& tB, int M, int
     if (err != cudaSuccess) return err;
     mark_done_on_device(attr_done);
   }
-  const int mt = (M + kBM - 1) / kBM, nt = (N + kBN - 1) / kBN, nk = (K + kBK - 1) / kBK;
-  const int mt2 = tA2 ? (M2 + kBM - 1) / kBM : 1, nt2 = tA2 ? (N2 + kBN - 1) / kBN : 0;
-  const int64_t tiles = (int64_t)mt * nt + (int64_t)mt2 * nt2;
-  if (tiles > 65535) return cudaErrorInvalidValue;
+  if (P.np < 1 || P.np > kMaxProbs || K <= 0) return cudaErrorInvalidValue;
+  int64_t tiles = 0;
+  for (int i = 0; i < P.np; ++i) {
+    SideProb& q = P.p[i];
+    if (q.o.M <= 0 || q.o.N <= 0) return cudaErrorInvalidValue;
+    q.mt = (q.o.M + kBM - 1) / kBM;
+    q.tile0 = (int)tiles;
+    tiles += (int64_t)q.mt * ((q.o.N + kBN - 1) / kBN);
+    if (tiles > 65535) return cudaErrorInvalidValue;
+  }
+  const int nk = (K + kBK - 1) / kBK;
   // widest cluster (K split) that keeps every CTA resident at two per SM
   const int64_t slots = 2 * (int64_t)device_sm_count();
   int cs = 1;
@@ -299,8 +316,7 @@ cudaError_t launch_side(const CUtensorMap& tA, const CUtensorMap& tB, int M, int
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_side<AMN, BMN, DUAL>, tA, tB, o, tA2 ? *tA2 : tA, tB2 ? *tB2 : tB,
-                                           o2 ? *o2 : o, mt * nt, mt, mt2, nk, kps, b_off);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_side<AMN, BMN, DUAL>, P, nk, kps, b_off);
   note_launch(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -343,21 +359,23 @@ cudaError_t lora_skinny(const __nv_bfloat16* X, int64_t ldx, int64_t T, int K, c
                         int64_t ldb, int b_mn, int KP, float s, __nv_bfloat16* Us, cudaStream_t st) {
   if (T <= 0 || T > INT32_MAX || K <= 0 || KP <= 0 || KP % 8 || !X || !Bop || !Us) return cudaErrorInvalidValue;
   if (!al16(X) || !al16(Bop) || (ldx % 8) || (ldb % 8)) return cudaErrorInvalidValue;
-  CUtensorMap tA, tB;
-  if (!make_map(&tA, X, T, K, ldx, kBM)) return cudaErrorInvalidValue;
+  SideProbs P{};
+  P.np = 1;
+  SideProb& q = P.p[0];
+  if (!make_map(&q.tA, X, T, K, ldx, kBM)) return cudaErrorInvalidValue;
   if (b_mn) {
-    if (!make_map(&tB, Bop, K, KP, ldb, kBK)) return cudaErrorInvalidValue;
+    if (!make_map(&q.tB, Bop, K, KP, ldb, kBK)) return cudaErrorInvalidValue;
   } else {
-    if (!make_map(&tB, Bop, KP, K, ldb, kBN)) return cudaErrorInvalidValue;
+    if (!make_map(&q.tB, Bop, KP, K, ldb, kBN)) return cudaErrorInvalidValue;
   }
-  SideOut o{};
+  SideOut& o = q.o;
   o.mode = 0;
   o.M = (int)T;
   o.N = KP;
   o.scale = s;
   o.out16 = Us;
   o.ld = KP;
-  return b_mn ? launch_side<0, 1>(tA, tB, (int)T, KP, K, o, st) : launch_side<0, 0>(tA, tB, (int)T, KP, K, o, st);
+  return b_mn ? launch_side<0, 1>(P, K, st) : launch_side<0, 0>(P, K, st);
 }
 
 cudaError_t lora_skinny_split(const __nv_bfloat16* X, int64_t ldx, int64_t T, int K, const __nv_bfloat16* Bop,
@@ -367,14 +385,16 @@ cudaError_t lora_skinny_split(const __nv_bfloat16* X, int64_t ldx, int64_t T, in
       !Bop || !Us)
     return cudaErrorInvalidValue;
   if (!al16(X) || !al16(Bop) || (ldx % 8) || (ldb % 8)) return cudaErrorInvalidValue;
-  CUtensorMap tA, tB;
-  if (!make_map(&tA, X, T, K, ldx, kBM)) return cudaErrorInvalidValue;
+  SideProbs P{};
+  P.np = 1;
+  SideProb& q = P.p[0];
+  if (!make_map(&q.tA, X, T, K, ldx, kBM)) return cudaErrorInvalidValue;
   if (b_mn) {
-    if (!make_map(&tB, Bop, K, KP, ldb, kBK)) return cudaErrorInvalidValue;
+    if (!make_map(&q.tB, Bop, K, KP, ldb, kBK)) return cudaErrorInvalidValue;
   } else {
-    if (!make_map(&tB, Bop, KP, K, ldb, kBN)) return cudaErrorInvalidValue;
+    if (!make_map(&q.tB, Bop, KP, K, ldb, kBN)) return cudaErrorInvalidValue;
   }
-  SideOut o{};
+  SideOut& o = q.o;
   o.mode = 3;
   o.M = (int)T;
   o.N = R;
@@ -385,40 +405,69 @@ cudaError_t lora_skinny_split(const __nv_bfloat16* X, int64_t ldx, int64_t T, in
   o.RS = RS;
   // the lo part of the operand starts 2 RS further along N: a multiple of 16 elements, so the TMA
   // x coordinate of the MN-major case stays 16-byte aligned
-  return b_mn ? launch_side<0, 1, 1>(tA, tB, (int)T, R, K, o, st, 2 * RS)
-              : launch_side<0, 0, 1>(tA, tB, (int)T, R, K, o, st, 2 * RS);
+  return b_mn ? launch_side<0, 1, 1>(P, K, st, 2 * RS) : launch_side<0, 0, 1>(P, K, st, 2 * RS);
+}
+
+cudaError_t lora_grads_multi(const LoraGradProb* g, int n, int64_t T, cudaStream_t st) {
+  if (!g || n < 1 || 2 * n > kMaxProbs || T <= 0 || T > INT32_MAX) return cudaErrorInvalidValue;
+  SideProbs P{};
+  P.np = 2 * n;
+  for (int i = 0; i < n; ++i) {
+    const LoraGradProb& q = g[i];
+    if (q.nseg < 1 || q.nseg > 3 || q.r <= 0 || q.nseg * q.r > q.KP || q.KP % 8 || q.in <= 0 || q.out <= 0)
+      return cudaErrorInvalidValue;
+    if (!al16(q.X) || !al16(q.Vs) || !al16(q.dY) || !al16(q.Us) || (q.ldx % 8) || (q.ldy % 8) || q.bounds[0] != 0 ||
+        q.bounds[q.nseg] != q.out)
+      return cudaErrorInvalidValue;
+    // dA: C [nseg*r, in] = Vs^T X; dB: C [out, nseg*r] = dY^T Us (both contract the T tokens)
+    SideProb& pa = P.p[2 * i];
+    SideProb& pb = P.p[2 * i + 1];
+    if (!make_map(&pa.tA, q.Vs, T, q.KP, q.KP, kBK) || !make_map(&pa.tB, q.X, T, q.in, q.ldx, kBK) ||
+        !make_map(&pb.tA, q.dY, T, q.out, q.ldy, kBK) || !make_map(&pb.tB, q.Us, T, q.KP, q.KP, kBK))
+      return cudaErrorInvalidValue;
+    SideOut& oa = pa.o;
+    SideOut& ob = pb.o;
+    oa.mode = 1;
+    oa.M = q.nseg * q.r;
+    oa.N = q.in;
+    oa.scale = 1.0f;
+    ob.mode = 2;
+    ob.M = q.out;
+    ob.N = q.nseg * q.r;
+    ob.scale = 1.0f;
+    for (int k = 0; k < q.nseg; ++k) {
+      oa.dst[k] = q.dA[k];
+      ob.dst[k] = q.dB[k];
+    }
+    for (int k = 0; k <= q.nseg; ++k) ob.bounds[k] = q.bounds[k];
+    oa.r = ob.r = q.r;
+    oa.nseg = ob.nseg = q.nseg;
+  }
+  return launch_side<1, 1>(P, (int)T, st);
 }
 
 cudaError_t lora_grads(const __nv_bfloat16* X, int64_t ldx, int in, const __nv_bfloat16* dY, int64_t ldy, int out,
                        int64_t T, const __nv_bfloat16* Us, const __nv_bfloat16* Vs, int KP, int nseg, int r,
                        const int* bounds, float* const* dA, float* const* dB, cudaStream_t st) {
-  if (nseg < 1 || nseg > 3 || r <= 0 || nseg * r > KP || KP % 8 || T <= 0 || in <= 0 || out <= 0)
-    return cudaErrorInvalidValue;
-  if (!al16(X) || !al16(Vs) || !al16(dY) || !al16(Us) || (ldx % 8) || (ldy % 8) || bounds[0] != 0 ||
-      bounds[nseg] != out)
-    return cudaErrorInvalidValue;
-  // dA: C [nseg*r, in] = Vs^T X; dB: C [out, nseg*r] = dY^T Us (both contract the T tokens)
-  CUtensorMap tVa, tX, tdY, tU;
-  if (!make_map(&tVa, Vs, T, KP, KP, kBK) || !make_map(&tX, X, T, in, ldx, kBK) ||
-      !make_map(&tdY, dY, T, out, ldy, kBK) || !make_map(&tU, Us, T, KP, KP, kBK))
-    return cudaErrorInvalidValue;
-  SideOut oa{}, ob{};
-  oa.mode = 1;
-  oa.M = nseg * r;
-  oa.N = in;
-  oa.scale = 1.0f;
-  ob.mode = 2;
-  ob.M = out;
-  ob.N = nseg * r;
-  ob.scale = 1.0f;
+  if (nseg < 1 || nseg > 3 || !bounds || !dA || !dB) return cudaErrorInvalidValue;
+  LoraGradProb q{};
+  q.X = X;
+  q.ldx = ldx;
+  q.in = in;
+  q.dY = dY;
+  q.ldy = ldy;
+  q.out = out;
+  q.Us = Us;
+  q.Vs = Vs;
+  q.KP = KP;
+  q.nseg = nseg;
+  q.r = r;
+  for (int k = 0; k <= nseg; ++k) q.bounds[k] = bounds[k];
   for (int k = 0; k < nseg; ++k) {
-    oa.dst[k] = dA[k];
-    ob.dst[k] = dB[k];
+    q.dA[k] = dA[k];
+    q.dB[k] = dB[k];
   }
-  for (int k = 0; k <= nseg; ++k) ob.bounds[k] = bounds[k];
-  oa.r = ob.r = r;
-  oa.nseg = ob.nseg = nseg;
-  return launch_side<1, 1>(tVa, tX, oa.M, in, (int)T, oa, st, 0, &tdY, &tU, out, ob.N, &ob);
+  return lora_grads_multi(&q, 1, T, st);
 }
 
 cudaError_t lora_prep(const LoraPrepArgs& a, cudaStream_t st) {

@@ -37,6 +37,26 @@ cudaError_t lora_grads(const __nv_bfloat16* X, int64_t ldx, int in, const __nv_b
                        int64_t T, const __nv_bfloat16* Us, const __nv_bfloat16* Vs, int KP, int nseg, int r,
                        const int* bounds, float* const* dA, float* const* dB, cudaStream_t st);
 
+// The adapter gradients of n <= 4 fused groups (the same T), in one launch: group i's dA and dB
+// reductions as above, with its own operands. How far the T contraction is split over a cluster
+// follows the launch's total number of output tiles, so the fp32 sums of one group can round
+// differently alone and in company; a given set of groups always gives the same bytes.
+struct LoraGradProb {
+  const __nv_bfloat16* X;
+  int64_t ldx;
+  int in;
+  const __nv_bfloat16* dY;
+  int64_t ldy;
+  int out;
+  const __nv_bfloat16* Us;
+  const __nv_bfloat16* Vs;
+  int KP, nseg, r;
+  int bounds[4];
+  float* dA[3];
+  float* dB[3];
+};
+cudaError_t lora_grads_multi(const LoraGradProb* g, int n, int64_t T, cudaStream_t st);
+
 // Derived bf16 operands of one fused projection group from its fp32 adapters (nseg segments,
 // A_p [r, in], B_p [out_p, r]), each adapter value a stored as the pair hi = bf16(a),
 // lo = bf16(a - hi) in three sections of RS rows (Acat) or columns (Bexp):

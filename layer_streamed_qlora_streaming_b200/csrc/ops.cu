@@ -5,6 +5,7 @@
 // partials summed in index order), so results do not depend on scheduling: the streamed and the
 // resident schedule run the same launches and give the same bytes.
 #include "common.cuh"
+#include "ex2.cuh"
 #include "ops.cuh"
 
 namespace lst {
@@ -291,80 +292,117 @@ k_ce(const float* __restrict__ logits, int V, const int32_t* __restrict__ y, flo
 }
 
 // Cross-entropy rows that read each logit once: a thread-block cluster of cs CTAs holds one row
-// in shared memory, CTA z the slice [z * slice, (z + 1) * slice), brought in by one bulk
-// asynchronous copy (the copy engine keeps the whole slice in flight). Each CTA reduces its slice
-// to (max, sum of exp) in a fixed tree; the cs pairs are merged in rank order through distributed
-// shared memory (every CTA gets the same lse); then each CTA writes dlogits of its slice from
-// shared memory, and the CTA holding the target writes the row's loss. Needs V % 4 == 0 (16-byte
+// in shared memory, CTA z the slice [z * slice, (z + 1) * slice), brought in by kCeChunks bulk
+// asynchronous copies issued at once (the copy engine keeps the whole slice in flight, and the
+// first pass starts on a chunk as soon as it has landed). On the slice in shared memory: its max,
+// then its sum of exp(x - max) in a fixed order; the cs (max, sum) pairs are merged in rank order
+// through distributed shared memory (every CTA gets the same lse); then each CTA writes dlogits of
+// its slice, and the CTA holding the target writes the row's loss. exp(t) is taken as 2^(t log2 e)
+// (the SFU's approximate exp2 on the product, formed with one fma). Needs V % 4 == 0 (16-byte
 // aligned slices).
-constexpr int kCeThreads = 256;
+constexpr int kCeThreads = 256, kCeChunks = 4;
+constexpr float kLog2e = 1.4426950408889634f;
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(dst)),
                "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+// block-wide max / sum of one value per thread (kCeThreads), fixed tree; every thread gets it
+__device__ __forceinline__ float ce_block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  v = red[0];
+#pragma unroll
+  for (int i = 1; i < kCeThreads / 32; ++i) v = fmaxf(v, red[i]);
+  return v;
+}
+__device__ __forceinline__ float ce_block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  v = red[0];
+#pragma unroll
+  for (int i = 1; i < kCeThreads / 32; ++i) v += red[i];
+  return v;
+}
 
 __global__ void __launch_bounds__(kCeThreads)
 k_ce_cluster(const float* __restrict__ logits, int V, int slice, const int32_t* __restrict__ y, float inv_T,
              float* __restrict__ loss_rows, bf16* __restrict__ dlog) {
-  extern __shared__ __align__(16) float row_s[];  // [slice], the CTA's (max, sum) pair, an mbarrier
-  __shared__ float sm[32], ss[32];
+  // [slice] floats, the CTA's (max, sum) pair, kCeChunks mbarriers
+  extern __shared__ __align__(128) float row_s[];
+  __shared__ float red_m[kCeThreads / 32], red_s[kCeThreads / 32];
   const int cs = (int)cluster_size_x();
   const int z = (int)cluster_rank();
   const int64_t row = blockIdx.x / cs;
   const int c0 = z * slice, n = max(0, min(V - c0, slice));
+  const int n4 = n / 4, q4 = (n4 + kCeChunks - 1) / kCeChunks;  // float4s in the slice, in a chunk
   float* pair = row_s + slice;
   uint64_t* bar = reinterpret_cast<uint64_t*>(pair + 2);
   if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
+    for (int k = 0; k < kCeChunks; ++k) mbar_init(bar + k, 1);
     fence_mbar_init();
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bar, (uint32_t)n * 4);
-    if (n > 0) bulk_load(row_s, logits + row * V + c0, (uint32_t)n * 4, bar);
+    for (int k = 0; k < kCeChunks; ++k) {
+      const int a = min(n4, k * q4), b = min(n4, a + q4);
+      mbar_arrive_expect_tx(bar + k, (uint32_t)(b - a) * 16);
+      if (b > a) bulk_load(row_s + 4 * a, logits + row * V + c0 + 4 * a, (uint32_t)(b - a) * 16, bar + k);
+    }
   }
-  mbar_wait(bar, 0);
-  float m = -INFINITY, sum = 0.f;
+  int tgt = y[row];
   const float4* r4 = reinterpret_cast<const float4*>(row_s);
-  for (int c = threadIdx.x; c < n / 4; c += blockDim.x) ms_add4(m, sum, r4[c]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, sum, o);
-    ms_merge(m, sum, m2, s2);
+  float m = -INFINITY;
+  for (int k = 0; k < kCeChunks; ++k) {
+    const int a = min(n4, k * q4), b = min(n4, a + q4);
+    mbar_wait(bar + k, 0);
+    for (int c = a + threadIdx.x; c < b; c += kCeThreads) {
+      const float4 v = r4[c];
+      m = fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+    }
   }
-  const int w = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) {
-    sm[w] = m;
-    ss[w] = sum;
+  m = ce_block_max(m, red_m);
+  float sum = 0.f;
+  if (m != -INFINITY) {
+    const float ml = m * kLog2e;
+    for (int c = threadIdx.x; c < n4; c += kCeThreads) {
+      const float4 v = r4[c];
+      sum += (ex2_approx(fmaf(v.x, kLog2e, -ml)) + ex2_approx(fmaf(v.y, kLog2e, -ml))) +
+             (ex2_approx(fmaf(v.z, kLog2e, -ml)) + ex2_approx(fmaf(v.w, kLog2e, -ml)));
+    }
   }
-  __syncthreads();
+  sum = ce_block_sum(sum, red_s);
   if (threadIdx.x == 0) {
-    float mm = sm[0], s2 = ss[0];
-    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) ms_merge(mm, s2, sm[i], ss[i]);
-    pair[0] = mm;
-    pair[1] = s2;
+    pair[0] = m;
+    pair[1] = sum;
   }
   cluster_sync_all();  // every CTA's pair is in place
-  float M = -INFINITY, Ssum = 0.f;
   const uint32_t pa = smem_u32(pair);
+  float M = -INFINITY;
+  for (int q = 0; q < cs; ++q) M = fmaxf(M, ld_cluster_f2(cluster_map(pa, (uint32_t)q)).x);
+  float S = 0.f;
   for (int q = 0; q < cs; ++q) {
     const float2 v = ld_cluster_f2(cluster_map(pa, (uint32_t)q));
-    ms_merge(M, Ssum, v.x, v.y);
+    if (v.x != -INFINITY) S += v.y * ex2_approx((v.x - M) * kLog2e);
   }
   cluster_sync_all();  // no CTA leaves while another still reads its pair
-  const float lse = M + logf(Ssum);
-  int tgt = y[row];
+  const float lse = M + logf(S);
   if (tgt < 0 || tgt >= V) {
     if (threadIdx.x == 0 && z == 0) dev_fail(DEV_ERR_BAD_INDEX);
     tgt = 0;
   }
   if (threadIdx.x == 0 && tgt >= c0 && tgt < c0 + n) loss_rows[row] = lse - row_s[tgt - c0];
   bf16* dr = dlog + row * V + c0;
-  for (int c = threadIdx.x; c < n / 4; c += blockDim.x) {
+  const float ll = lse * kLog2e;
+  for (int c = threadIdx.x; c < n4; c += kCeThreads) {
     const float4 v = r4[c];
-    float p[4] = {expf(v.x - lse), expf(v.y - lse), expf(v.z - lse), expf(v.w - lse)};
+    float p[4] = {ex2_approx(fmaf(v.x, kLog2e, -ll)), ex2_approx(fmaf(v.y, kLog2e, -ll)),
+                  ex2_approx(fmaf(v.z, kLog2e, -ll)), ex2_approx(fmaf(v.w, kLog2e, -ll))};
     const int d = tgt - c0 - 4 * c;
     if (d >= 0 && d < 4) p[d] -= 1.0f;
     const __nv_bfloat162 h[2] = {__floats2bfloat162_rn(p[0] * inv_T, p[1] * inv_T),
@@ -502,6 +540,12 @@ __global__ void k_f32_to_bf16(const float* __restrict__ x, int64_t n, bf16* __re
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) y[i] = __float2bfloat16_rn(x[i]);
 }
+// 16-byte words src -> dst (n words), grid-stride
+__global__ void k_copy16(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = src[i];
+}
+
 __global__ void k_bf16_to_f32(const bf16* __restrict__ x, int64_t n, float* __restrict__ y) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) y[i] = __bfloat162float(x[i]);
@@ -567,11 +611,11 @@ cudaError_t cross_entropy(const float* logits, int64_t T, int V, const int32_t* 
     note_launch(1);
     return cudaGetLastError();
   }
-  const int smem = slice * 4 + 16;  // the slice, the (max, sum) pair and the mbarrier
+  const int smem = slice * 4 + 8 + 8 * kCeChunks;  // the slice, the (max, sum) pair and the mbarriers
   static std::atomic<unsigned long long> attr_done{0};
   if (!done_on_device(attr_done)) {
     const cudaError_t e = cudaFuncSetAttribute(k_ce_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)(kMaxSliceBytes + 16));
+                                               (int)(kMaxSliceBytes + 8 + 8 * kCeChunks));
     if (e != cudaSuccess) return e;
     mark_done_on_device(attr_done);
   }
@@ -630,6 +674,16 @@ cudaError_t f32_to_bf16(const float* x, int64_t n, bf16* y, cudaStream_t s) {
 }
 cudaError_t bf16_to_f32(const bf16* x, int64_t n, float* y, cudaStream_t s) {
   k_bf16_to_f32<<<nblk(n), kThreads, 0, s>>>(x, n, y);
+  note_launch(1);
+  return cudaGetLastError();
+}
+cudaError_t copy16(const void* src, void* dst, int64_t bytes, cudaStream_t s) {
+  if (bytes <= 0) return cudaSuccess;
+  if (bytes % 16 || (reinterpret_cast<uintptr_t>(src) & 15) || (reinterpret_cast<uintptr_t>(dst) & 15))
+    return cudaErrorInvalidValue;
+  const int64_t n = bytes / 16;
+  k_copy16<<<(unsigned)std::min<int64_t>((n + kThreads - 1) / kThreads, 1024), kThreads, 0, s>>>(
+      reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst), n);
   note_launch(1);
   return cudaGetLastError();
 }

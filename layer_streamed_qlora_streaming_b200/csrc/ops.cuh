@@ -55,6 +55,8 @@ cudaError_t ce_grad(const float* logits, int64_t rows, int64_t row0, int V, cons
 cudaError_t dot_fixed(const float* a, const bf16* b, int64_t n, float* partials, float* out, cudaStream_t s);
 
 cudaError_t f32_to_bf16(const float* x, int64_t n, bf16* y, cudaStream_t s);
+// bytes (a multiple of 16, both pointers 16-byte aligned) from src to dst on stream s
+cudaError_t copy16(const void* src, void* dst, int64_t bytes, cudaStream_t s);
 cudaError_t bf16_to_f32(const bf16* x, int64_t n, float* y, cudaStream_t s);
 
 }  // namespace lst

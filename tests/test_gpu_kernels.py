@@ -319,13 +319,19 @@ def test_swiglu_fwd_bwd():
     assert maxrel(to_np(dgu), ref) < 8e-3
 
 
-@pytest.mark.parametrize("T,V", [(40, 50000), (24, 128256), (16, 152064), (12, 60001), (20, 1001)])
+@pytest.mark.parametrize("T,V", [(40, 50000), (24, 128256), (16, 152064), (12, 60001), (20, 1001), (10, 1000),
+                                 (6, 262144)])
 def test_cross_entropy_rows(T, V):
-    # V % 4 == 0: a cluster of 1-8 CTAs holds the row in shared memory (50000: 4 slices, 128256 and
-    # 152064: 8); otherwise (60001, 1001) the two-pass kernel
+    # V % 4 == 0: a cluster of 1-8 CTAs holds the row in shared memory (1000: one CTA, its four
+    # copies 63/63/63/61 float4s; 50000: 4 slices; 128256 and 152064: 8; 262144: 8 slices of 128 KB);
+    # otherwise (60001, 1001) the two-pass kernel. Row 0 has one logit far above the rest, row 1
+    # only large negative logits, row 2 its maximum in the last slice.
     r = _rng(9 + V)
     logits = r.normal(size=(T, V)).astype(np.float32) * 2
     y = r.integers(0, V, size=T).astype(np.int32)
+    logits[0, y[0]] += 60.0
+    logits[1] -= 120.0
+    logits[2, V - 3] = 30.0
     loss = torch.empty(T, device="cuda")
     dl = torch.empty(T, V, dtype=torch.bfloat16, device="cuda")
     lst.k_cross_entropy(torch_f32(logits), T, V, torch.from_numpy(y).cuda(), 1.0 / T, loss, dl)
@@ -448,6 +454,51 @@ def test_lora_grads(T, in_f, bounds, r):
         refB = dY64[:, bounds[p]:bounds[p + 1]].T @ Us[:, p * r:(p + 1) * r].astype(np.float64)
         assert maxrel(to_np(dA[p]), refA) < 1e-4, (p, maxrel(to_np(dA[p]), refA))
         assert maxrel(to_np(dB[p]), refB) < 1e-4, (p, maxrel(to_np(dB[p]), refB))
+
+
+@pytest.mark.parametrize("T", [384, 200])
+def test_lora_grads_of_four_groups_in_one_launch(T):
+    # the four groups of a layer (q/k/v with three segments, o, gate/up with two, down) in one launch:
+    # every dA / dB against fp64, and against the same group launched alone (the K split may differ,
+    # so equal up to fp32 rounding); the same bytes twice
+    rng = _rng(T + 11)
+    r, KP = 8, 64
+    specs = [(256, [0, 256, 320, 384]), (256, [0, 256]), (256, [0, 688, 1376]), (688, [0, 256])]
+    groups, refs, alone = [], [], []
+    for in_f, bounds in specs:
+        nseg, out_f = len(bounds) - 1, bounds[-1]
+        R = nseg * r
+        X = _bf(rng.normal(size=(T, in_f)))
+        dY = _bf(rng.normal(size=(T, out_f)) * 0.1)
+        Us = np.zeros((T, KP), np.float32)
+        Us[:, :R] = _bf(rng.normal(size=(T, R)))
+        Vs = np.zeros((T, KP), np.float32)
+        Vs[:, :R] = _bf(rng.normal(size=(T, R)))
+        mk = lambda: ([torch.full((r, in_f), float("nan"), device="cuda") for _ in range(nseg)],
+                      [torch.full((bounds[p + 1] - bounds[p], r), float("nan"), device="cuda") for p in range(nseg)])
+        dA, dB = mk()
+        g = dict(X=torch_bf16(X), ldx=in_f, in_f=in_f, dY=torch_bf16(dY), ldy=out_f, out_f=out_f, Us=torch_bf16(Us),
+                 Vs=torch_bf16(Vs), KP=KP, r=r, bounds=bounds, dA=dA, dB=dB)
+        groups.append(g)
+        X64, dY64 = X.astype(np.float64), dY.astype(np.float64)
+        refs.append([Vs[:, p * r:(p + 1) * r].astype(np.float64).T @ X64 for p in range(nseg)] +
+                    [dY64[:, bounds[p]:bounds[p + 1]].T @ Us[:, p * r:(p + 1) * r].astype(np.float64)
+                     for p in range(nseg)])
+        aA, aB = mk()
+        lst.k_lora_grads(g["X"], in_f, in_f, g["dY"], out_f, out_f, T, g["Us"], g["Vs"], KP, r, bounds, aA, aB)
+        alone.append(aA + aB)
+    outs = []
+    for _ in range(2):
+        lst.k_lora_grads_multi(groups, T)
+        torch.cuda.synchronize()
+        outs.append([[t.cpu().numpy().copy() for t in g["dA"] + g["dB"]] for g in groups])
+    for ga, gb in zip(*outs):
+        for a, b in zip(ga, gb):
+            assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    for got, ref, al in zip(outs[0], refs, alone):
+        for a, rf, b in zip(got, ref, al):
+            assert maxrel(a, rf) < 1e-4
+            assert maxrel(a, to_np(b)) < 1e-6
 
 
 @pytest.mark.parametrize("M,N,K", [(4096, 64, 2048), (304, 64, 200), (6144, 64, 512)])

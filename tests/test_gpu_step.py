@@ -368,11 +368,15 @@ def test_adamw_step_matches_oracle_and_trains():
     ctx.close()
 
 
-def test_read_timeline_orders_copies_before_compute():
+@pytest.mark.parametrize("base", ["nf4", "bf16"])
+def test_read_timeline_orders_copies_before_compute(base):
     # the per-read timeline of a profiled step: 2L reads in order, every read's compute starts after
     # its copy (and dequant) started and ends after they ended; a copy into a slot starts only once
-    # the read two earlier, which computed from that slot, has finished
-    wl = syn.WORKLOADS["tiny"].with_(n_layers=3)
+    # the read two earlier, which used that slot, no longer needs it: with an NF4 base dequantised
+    # in a separate pass, once that read's dequant has finished (its compute reads the bf16 scratch
+    # and the header copied next to it, and may still be running); with a bf16 base, once its
+    # compute has finished
+    wl = syn.WORKLOADS["tiny"].with_(n_layers=3, base_format=base)
     inp = build_inputs(wl)
     ctx = make_context(wl, inp, streamed=True)
     ctx.set_profiling(True)
@@ -387,11 +391,55 @@ def test_read_timeline_orders_copies_before_compute():
         c0, c1 = r["copy"]
         d0, d1 = r["dequant"]
         k0, k1 = r["compute"]
-        assert None not in (c0, c1, d0, d1, k0, k1)
-        assert 0 <= c0 <= c1 and c0 <= d0 + eps and d0 <= d1 and c0 <= k0 + eps and k0 <= k1
-        assert c1 <= k1 + eps and d1 <= k1 + eps
-        if n >= 2:
-            assert tl[n - 2]["compute"][1] <= c0 + eps
+        assert None not in (c0, c1, k0, k1)
+        assert 0 <= c0 <= c1 and c0 <= k0 + eps and k0 <= k1 and c1 <= k1 + eps
+        if base == "nf4":
+            assert None not in (d0, d1)
+            assert c0 <= d0 + eps and d0 <= d1 and d1 <= k1 + eps
+            if n >= 2:
+                assert tl[n - 2]["dequant"][1] <= c0 + eps
+        else:
+            assert (d0, d1) == (None, None)
+            if n >= 2:
+                assert tl[n - 2]["compute"][1] <= c0 + eps
+
+
+@pytest.mark.parametrize("L", [1, 3])
+def test_prefetch_of_next_first_read_same_bytes(L):
+    # copying the next step's first read ahead (at the end of each step) changes when layer 0 is
+    # copied, not what is computed: the same loss and gradient bytes as without it, 2L reads counted
+    # per step; a step after switching reuse on, and one after re-registering layer 0 (which drops
+    # the prefetched copy), give the same bytes too
+    wl = syn.WORKLOADS["tiny"].with_(n_layers=L)
+    inp = build_inputs(wl)
+    runs = {}
+    for pre in (False, True):
+        ctx = make_context(wl, inp, streamed=True)
+        ctx.set_prefetch(pre)
+        out, reads = [], []
+        for _ in range(3):
+            out.append(run_step(ctx, wl, inp, want_logits=False)[:2])
+            reads.append(ctx.stats()["layer_reads_last_step"])
+        r = inp["raw"][0]
+        ctx.register_layer(0, r["W"], r["A"], r["B"], r["attn_norm"], r["mlp_norm"], r["bias"])
+        out.append(run_step(ctx, wl, inp, want_logits=False)[:2])
+        ctx.set_reuse(True)
+        out.append(run_step(ctx, wl, inp, want_logits=False)[:2])
+        ctx.set_reuse(False)
+        out.append(run_step(ctx, wl, inp, want_logits=False)[:2])
+        if pre:
+            ctx.set_profiling(True)
+            out.append(run_step(ctx, wl, inp, want_logits=False)[:2])
+            tl = ctx.read_timeline()
+            # the reuse-on step left nothing prefetched, the step after it did: read 0 of this
+            # profiled step was copied by the previous step and starts computing without a copy
+            assert tl[0]["copy"] == (None, None) and all(None not in r["copy"] for r in tl[1:])
+        ctx.close()
+        runs[pre] = (out, reads)
+    assert runs[False][1] == runs[True][1] == [2 * L] * 3
+    for (la, ga), (lb, gb) in zip(runs[False][0], runs[True][0]):
+        assert np.float32(la).tobytes() == np.float32(lb).tobytes()
+        assert ga.tobytes() == gb.tobytes()
 
 
 @pytest.mark.parametrize("name", ["tiny", "llama8b_layer_T256"])

@@ -13,11 +13,13 @@ def reads(L, dpo):
     return (list(range(L)) if dpo else []) + list(range(L)) + list(range(L - 1, -1, -1))
 
 
-def check_step(layers, rows, held0, wheld0, reuse, nf4):
+def check_step(layers, rows, held0, wheld0, reuse, nf4, pre_slot=-1):
     """Replay the plan on two slots / two scratches and check every invariant; returns the number
-    of copies and dequants."""
+    of copies and dequants. pre_slot: the slot a previous step copied this step's first read into."""
     held = list(held0) if reuse else [-1, -1]
     wheld = list(wheld0) if reuse else [-1, -1]
+    if not reuse and pre_slot >= 0:
+        held[pre_slot] = layers[0]
     last_use, loaded, wlast, wfill = [-1, -1], [-1, -1], [-1, -1], [-1, -1]
     copies = deqs = 0
     for n, (j, row) in enumerate(zip(layers, rows)):
@@ -31,7 +33,8 @@ def check_step(layers, rows, held0, wheld0, reuse, nf4):
             held[s] = j
             loaded[s] = n
         else:
-            assert reuse and held[s] == j, "a read without a copy must find its layer in the slot"
+            assert (reuse or (n == 0 and s == pre_slot)) and held[s] == j, \
+                "a read without a copy must find its layer in the slot"
         assert held[s] == j
         assert row[LOADED] == loaded[s]
         last_use[s] = n
@@ -94,3 +97,32 @@ def test_plan_rejects_bad_arguments():
         lst.plan_reads([], True, True)
     with pytest.raises(lst.LstError):
         lst.plan_reads([0, -1], True, True)
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 32])
+@pytest.mark.parametrize("dpo", [False, True])
+@pytest.mark.parametrize("nf4", [False, True])
+def test_prefetch_copies_the_next_first_read_after_the_last_read_of_its_slot(L, dpo, nf4):
+    """Reuse off with prefetch: every step still copies R blobs (R - 1 of its own reads plus the next
+    step's first read); that copy goes into the slot the step's last read does not use and waits
+    only for the read before it; the next step computes its first read from that slot uncopied."""
+    layers = reads(L, dpo)
+    R = len(layers)
+    held, wheld, pre = (-1, -1), (-1, -1), -1
+    for step in range(3):
+        rows, h2, w2, (pslot, pwait) = lst.plan_reads(layers, False, nf4, held, wheld, prefetch=pre)
+        rows = rows.tolist()
+        copies, deqs, h3, _ = check_step(layers, rows, held, wheld, False, nf4, pre_slot=pre)
+        assert copies == (R if pre < 0 else R - 1)
+        assert deqs == (R if nf4 else 0)                           # dequant is not carried over
+        if pre >= 0:
+            assert rows[0][SLOT] == pre and rows[0][COPY] == 0 and rows[0][LOADED] == -1
+        assert pslot == 1 - rows[-1][SLOT]
+        assert pwait == max(n for n in range(R) if rows[n][SLOT] == pslot) == R - 2
+        assert h2[pslot] == layers[0] and h2[1 - pslot] == h3[1 - pslot]
+        held, wheld, pre = h2, w2, pslot
+    # with reuse on there is nothing to prefetch
+    _, _, _, p = lst.plan_reads(layers, True, nf4, (-1, -1), (-1, -1), prefetch=-1)
+    assert p == (-1, -1)
+    with pytest.raises(lst.LstError):
+        lst.plan_reads(layers, False, nf4, prefetch=2)
