@@ -17,6 +17,9 @@ Cases are the shapes of the Llama-3.1-8B-shaped layer at batch 4 x seq 512 (T = 
   lora_v_gu    V = s dY Bexp, dY [2048, 28672], Bexp [28672, 64] (MN-major)
   lora_grads_qkv  dA = Vs^T X and dB = dY^T Us of the q/k/v group (dY [2048, 6144])
   lora_grads_gu   the same for gate/up (dY [2048, 28672])
+  lora_grads_layer      dA and dB of the four groups of a layer (q/k/v, o, gate/up, down) in one
+                        launch, as a backward read issues them
+  lora_grads_layer_sep  the same four groups as four launches
   ce           cross-entropy rows + dlogits over fp32 logits [2048, 128256]
 The LoRA cases rotate over enough input copies to exceed the 126 MB L2, so every launch reads
 its operands from HBM.
@@ -35,7 +38,7 @@ import torch
 
 sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 from layer_streamed_qlora_streaming_b200 import (k_attention_bwd, k_attention_fwd, k_cross_entropy, k_gemm, k_gemm_nf4,
-                                                 k_lora_grads, k_lora_skinny, k_nf4_dequant,
+                                                 k_lora_grads, k_lora_grads_multi, k_lora_skinny, k_nf4_dequant,
                k_nf4_quantize)
 
 T, D, F, HQ, HKV, HD, S = 2048, 4096, 14336, 32, 8, 128, 512
@@ -196,6 +199,8 @@ def _lora_case(case: str, g):
             it[0] += 1
             k_lora_skinny(X, K, T, K, Bop, KP if bmn else K, bmn, KP, 2.0, Us)
         return run, {"flop": 2.0 * T * K * KP, "bytes": T * K * 2 + K * KP * 2 + T * KP * 2}
+    if case.startswith("lora_grads_layer"):
+        return _lora_layer_case(case, g)
     in_f, bounds, r = {"lora_grads_qkv": (D, [0, 4096, 5120, 6144], 16),
                        "lora_grads_gu": (D, [0, F, 2 * F], 16)}[case]
     out_f = bounds[-1]
@@ -214,6 +219,38 @@ def _lora_case(case: str, g):
         k_lora_grads(Xs[i], in_f, in_f, dYs[i], out_f, out_f, T, Us, Vs, KP, r, bounds, dA, dB)
     return run, {"flop": 2.0 * T * KP * (in_f + out_f),
                  "bytes": T * (in_f + out_f) * 2 + 2 * T * KP * 2 + nseg * r * (in_f + out_f) * 4}
+
+
+def _lora_layer_case(case: str, g):
+    # (in, segment bounds of dY, KP) of the q/k/v, o, gate/up and down groups at r = 16
+    r = 16
+    specs = [(D, [0, 4096, 5120, 6144], 192), (D, [0, D], 64), (D, [0, F, 2 * F], 128), (F, [0, D], 64)]
+    per_copy = sum(T * (i + b[-1]) * 2 for i, b, _ in specs)
+    nb = _copies(per_copy)
+    sets = []
+    for _ in range(nb):
+        groups = []
+        for in_f, bounds, KP in specs:
+            nseg, out_f = len(bounds) - 1, bounds[-1]
+            groups.append(dict(X=_bf((T, in_f), g), ldx=in_f, in_f=in_f, dY=_bf((T, out_f), g), ldy=out_f,
+                               out_f=out_f, Us=_bf((T, KP), g), Vs=_bf((T, KP), g), KP=KP, r=r, bounds=bounds,
+                               dA=[torch.empty(r, in_f, device="cuda") for _ in range(nseg)],
+                               dB=[torch.empty(bounds[p + 1] - bounds[p], r, device="cuda") for p in range(nseg)]))
+        sets.append(groups)
+    it = [0]
+
+    def run():
+        groups = sets[it[0] % nb]
+        it[0] += 1
+        if case == "lora_grads_layer":
+            k_lora_grads_multi(groups, T)
+        else:
+            for q in groups:
+                k_lora_grads(q["X"], q["ldx"], q["in_f"], q["dY"], q["ldy"], q["out_f"], T, q["Us"], q["Vs"], q["KP"],
+                             q["r"], q["bounds"], q["dA"], q["dB"])
+    nbytes = sum(T * (i + b[-1]) * 2 + 2 * T * kp * 2 + (len(b) - 1) * r * (i + b[-1]) * 4 for i, b, kp in specs)
+    flop = sum(2.0 * T * (len(b) - 1) * r * (i + b[-1]) for i, b, _ in specs)
+    return run, {"flop": flop, "bytes": nbytes}
 
 
 def main():
