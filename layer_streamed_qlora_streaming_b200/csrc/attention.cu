@@ -12,6 +12,7 @@
 // blocks with the most work are scheduled first.
 #include "attention.cuh"
 #include "common.cuh"
+#include "pdl.cuh"
 #include "ex2.cuh"
 #include "gemm.cuh"
 
@@ -409,6 +410,8 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // inputs of the previous kernel in the stream are complete from here on
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -623,7 +626,8 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 // One CTA per 128 queries of one head (heaviest first), 320 threads: warp 0 TMA (Q and dO once; K
 // and V tiles of 64 keys, double-buffered), warp 1 MMA issuer, warps 2-9 two threads per query row.
 //   S = Q K^T, dP = dO V^T   tcgen05 (bf16), into one of two TMEM buffer pairs;
-//   dS = P (dP - D)          the row's threads, P = exp2(S' - lse'), written bf16 to a swizzled tile;
+//   dS = P (dP - D)          the row's threads, P = exp2(S' - lse'), written bf16 to one of two
+//                            swizzled tiles (so block j+1's dS is written while dQ reads block j's);
 //   dQ += dS K               tcgen05 (K read MN-major from the same tile), fp32 in TMEM;
 // then dQ * scale with the rotary embedding undone is stored once as bf16.
 template <int HD>
@@ -634,7 +638,7 @@ struct DqTc {
   static constexpr uint32_t Q_BYTES = (HD / 64) * CH;
   static constexpr uint32_t KV_BYTES = 2 * (HD / 64) * KCH;  // K then V of one stage
   static constexpr uint32_t DS_BYTES = CH;                   // 128 queries x 64 keys bf16
-  static constexpr uint32_t SMEM = 2 * Q_BYTES + 2 * KV_BYTES + DS_BYTES + 1024 + 256;
+  static constexpr uint32_t SMEM = 2 * Q_BYTES + 2 * KV_BYTES + 2 * DS_BYTES + 1024 + 256;
   static constexpr uint32_t TMEM_COLS = 512;                 // S[2] at 0/64, dP[2] at 128/192, dQ at 256
 };
 
@@ -648,16 +652,16 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
   uint8_t* sQ = smem;
   uint8_t* sO = sQ + C::Q_BYTES;          // dO
   uint8_t* sKV = sO + C::Q_BYTES;         // [2] stages: K chunks, then V chunks
-  uint8_t* sDS = sKV + 2 * C::KV_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + C::DS_BYTES);
+  uint8_t* sDS = sKV + 2 * C::KV_BYTES;  // [2] dS tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + 2 * C::DS_BYTES);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;   // [2]
   uint64_t* kv_empty = bars + 3;  // [2]
   uint64_t* s_full = bars + 5;    // [2]
   uint64_t* s_free = bars + 7;    // [2]
-  uint64_t* ds_full = bars + 9;
-  uint64_t* dq_done = bars + 10;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* ds_full = bars + 9;   // [2]
+  uint64_t* ds_free = bars + 11;  // [2] the dQ MMAs of the tile's block are done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
 
   const int h = blockIdx.x, b = blockIdx.y, qb = (int)gridDim.z - 1 - (int)blockIdx.z;
   const int kvh = h / (p.hq / p.hkv);
@@ -673,9 +677,9 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 256);
+      mbar_init(&ds_full[i], 256);
+      mbar_init(&ds_free[i], 1);
     }
-    mbar_init(ds_full, 256);
-    mbar_init(dq_done, 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -692,6 +696,8 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // inputs of the previous kernel in the stream are complete from here on
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -738,9 +744,9 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         }
         if (j >= 1) {  // dQ += dS_{j-1} K_{j-1}
           const int i = j - 1, st = i & 1;
-          if (!mbar_wait(ds_full, i & 1)) break;
+          if (!mbar_wait(&ds_full[st], (i >> 1) & 1)) break;
           tc_fence_after();
-          const uint32_t ds = smem_u32(sDS), k = smem_u32(sKV + st * C::KV_BYTES);
+          const uint32_t ds = smem_u32(sDS + st * C::DS_BYTES), k = smem_u32(sKV + st * C::KV_BYTES);
 #pragma unroll
           for (int kk = 0; kk < C::KB / 16; ++kk) {
             const uint64_t da = umma_desc(ds + kk * 32, 16, 1024);
@@ -748,7 +754,7 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             umma_bf16(tmem + 256, da, db, idQ, (i | kk) != 0);
           }
           umma_commit(&kv_empty[st]);
-          umma_commit(dq_done);
+          umma_commit(&ds_free[st]);
         }
       }
     }
@@ -788,11 +794,12 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       }
       tc_fence_before();
       mbar_arrive(&s_free[st]);
-      if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(dq_done, (j - 1) & 1))) {  // the dS tile is free
+      // dS tile st is free once the dQ MMAs of block j - 2 are done
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&ds_free[st], ((j - 2) >> 1) & 1))) {
         ok = false;
         break;
       }
-      uint8_t* row = sDS + r * 128;
+      uint8_t* row = sDS + st * C::DS_BYTES + r * 128;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {  // pieces 4 half .. 4 half + 3 of the row
         const float* v = ds + i * 8;
@@ -802,9 +809,10 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       }
       fence_proxy_async();
       tc_fence_before();
-      mbar_arrive(ds_full);
+      mbar_arrive(&ds_full[st]);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(dq_done, (nkb - 1) & 1))) {
+    // the commit after the last block's dQ MMAs: every MMA of this CTA is done
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&ds_free[(nkb - 1) & 1], ((nkb - 1) >> 1) & 1))) {
       tc_fence_after();
       float acc[HD];  // the whole dQ row, scaled
 #pragma unroll
@@ -857,8 +865,9 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 // blocks of 64 (double-buffered Q / dO tiles): warp 0 TMA, warp 1 MMA issuer, warps 2-9 two threads
 // per key row.
 //   S^T = K Q^T, dP^T = V dO^T      tcgen05 (bf16), into one of two TMEM buffer pairs;
-//   P^T, dS^T = P^T (dP^T - D)      the key row's thread (lse and D of the block's queries from
-//                                    shared memory), written bf16 to swizzled tiles;
+//   P^T, dS^T = P^T (dP^T - D)      the key row's threads (lse and D of the block's queries from
+//                                    shared memory), written bf16 to one of two pairs of swizzled
+//                                    tiles (block j+1's while the MMAs read block j's);
 //   dV += P^T dO, dK += dS^T Q       tcgen05, with Q / dO read MN-major from the tiles used K-major above.
 // The grp partial dK / dV tiles are then parked in shared memory and CTA hh adds rows
 // [hh * 128/grp, ...) over the heads in order 0 .. grp-1 (distributed shared memory), scales dK,
@@ -872,7 +881,7 @@ struct DkvTc {
   static constexpr uint32_t QO_BYTES = 2 * (HD / 64) * QCH;  // Q then dO of one stage
   static constexpr uint32_t T_BYTES = 128 * 128;             // one [128 keys x 64 queries] bf16 tile
   static constexpr int RLD = HD + 4;                         // fp32 row stride of a parked tile
-  static constexpr uint32_t MAIN = 2 * K_BYTES + 2 * QO_BYTES + 2 * T_BYTES + 2 * 2 * QB * 4;
+  static constexpr uint32_t MAIN = 2 * K_BYTES + 2 * QO_BYTES + 4 * T_BYTES + 2 * 2 * QB * 4;
   static constexpr uint32_t PARK = 2 * 128 * RLD * 4;
   static constexpr uint32_t SMEM = (MAIN > PARK ? MAIN : PARK) + 1024 + 256;
   static constexpr uint32_t TMEM_COLS = 2 * 128 + 2 * HD <= 256 ? 256 : 512;
@@ -888,9 +897,9 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint8_t* sK = smem;
   uint8_t* sV = sK + C::K_BYTES;
   uint8_t* sQO = sV + C::K_BYTES;               // [2] stages: Q chunks, then dO chunks
-  uint8_t* sP = sQO + 2 * C::QO_BYTES;          // P^T tile
-  uint8_t* sS = sP + C::T_BYTES;                // dS^T tile
-  float* sLse = reinterpret_cast<float*>(sS + C::T_BYTES);  // [2][64]
+  uint8_t* sP = sQO + 2 * C::QO_BYTES;          // [2] P^T tiles
+  uint8_t* sS = sP + 2 * C::T_BYTES;            // [2] dS^T tiles
+  float* sLse = reinterpret_cast<float*>(sS + 2 * C::T_BYTES);  // [2][64]
   float* sD = sLse + 2 * C::QB;                             // [2][64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (C::MAIN > C::PARK ? C::MAIN : C::PARK));
   uint64_t* kv_full = bars;
@@ -898,9 +907,9 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* qo_empty = bars + 3;  // [2]
   uint64_t* s_full = bars + 5;    // [2]
   uint64_t* s_free = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* kv_done = bars + 10;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* p_full = bars + 9;    // [2] P^T / dS^T tile pair written
+  uint64_t* t_free = bars + 11;   // [2] the dV / dK MMAs of the pair's block are done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   float* redK = reinterpret_cast<float*>(smem);  // after the main loop: [128][RLD] each
   float* redV = redK + 128 * C::RLD;
 
@@ -921,9 +930,9 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(&qo_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 256);
+      mbar_init(&p_full[i], 256);
+      mbar_init(&t_free[i], 1);
     }
-    mbar_init(p_full, 256);
-    mbar_init(kv_done, 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -940,6 +949,8 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // inputs of the previous kernel in the stream are complete from here on
+  pdl_trigger();
   const uint32_t tV = tmem + 256, tK = tmem + 256 + HD;  // dV, dK accumulators
 
   bool ok = true;
@@ -988,9 +999,9 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         if (j >= 1) {  // dV += P^T dO, dK += dS^T Q of block j-1
           const int i = j - 1, st = i & 1;
-          if (!mbar_wait(p_full, i & 1)) break;
+          if (!mbar_wait(&p_full[st], (i >> 1) & 1)) break;
           tc_fence_after();
-          const uint32_t pt = smem_u32(sP), ds = smem_u32(sS);
+          const uint32_t pt = smem_u32(sP + st * C::T_BYTES), ds = smem_u32(sS + st * C::T_BYTES);
           const uint32_t q = smem_u32(sQO + st * C::QO_BYTES), o = q + (HD / 64) * C::QCH;
 #pragma unroll
           for (int kk = 0; kk < C::QB / 16; ++kk) {
@@ -1000,7 +1011,7 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                       (i | kk) != 0);
           }
           umma_commit(&qo_empty[st]);
-          umma_commit(kv_done);
+          umma_commit(&t_free[st]);
         }
       }
     }
@@ -1056,12 +1067,13 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       tc_fence_before();
       mbar_arrive(&s_free[st]);
-      if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(kv_done, (j - 1) & 1))) {  // P^T / dS^T tiles free
+      // tile pair st is free once the dV / dK MMAs of block j - 2 are done
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&t_free[st], ((j - 2) >> 1) & 1))) {
         ok = false;
         continue;
       }
-      uint8_t* prow = sP + r * 128;
-      uint8_t* srow = sS + r * 128;
+      uint8_t* prow = sP + st * C::T_BYTES + r * 128;
+      uint8_t* srow = sS + st * C::T_BYTES + r * 128;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float* a = pv + i * 8;
@@ -1074,10 +1086,11 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       fence_proxy_async();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[st]);
     }
     // park this head's dK, dV rows (fp32, this half's columns) once the last block's MMAs are done
-    if (ok && __all_sync(0xffffffffu, mbar_wait(kv_done, (nqb - 1) & 1))) {
+    // (the commit after them covers every earlier MMA of this CTA)
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&t_free[(nqb - 1) & 1], ((nqb - 1) >> 1) & 1))) {
       tc_fence_after();
 #pragma unroll 1
       for (int c = half * (HD / 2); c < (half + 1) * (HD / 2); c += 32) {
@@ -1099,7 +1112,7 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       ok = false;
     }
   }
-  // (the tiles the parked rows overwrite are no longer read: every MMA completed before kv_done)
+  // (the tiles the parked rows overwrite are no longer read: every MMA completed before that commit)
   tc_fence_before();
   __syncwarp();
   cluster_sync_all();  // every head's partial tile is parked
@@ -1159,6 +1172,8 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
 // --------------------------------------------------------------------------- backward: D = rowsum(dO o)
 __global__ void k_attn_D(AttnBwdArgs p) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t idx = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // (t, h)
   const int l = threadIdx.x & 31;
   if (idx >= p.T * (int64_t)p.hq) return;
@@ -1499,8 +1514,7 @@ cudaError_t launch_fwd_tc(const AttnArgs& a, int B, cudaStream_t s) {
     mark_done_on_device(attr_done);
   }
   dim3 grid(a.hq, B, (a.S + C::QB - 1) / C::QB);
-  k_attn_fwd_tc<HD><<<grid, 320, C::SMEM, s>>>(tQ, tK, tV, a);
-  return cudaSuccess;
+  return launch_k(k_attn_fwd_tc<HD>, grid, dim3(320), C::SMEM, s, 0, tQ, tK, tV, a);
 }
 
 // LST_ATTN_FWD=mma selects the warp-level mma.sync forward (for comparing the two); the tcgen05
@@ -1584,23 +1598,11 @@ cudaError_t launch_bwd_tc(const AttnBwdArgs& a, int B, cudaStream_t s) {
     mark_done_on_device(attr_done);
   }
   const int grp = a.hq / a.hkv;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grp, (unsigned)(B * a.hkv), (unsigned)((a.S + K::KB - 1) / K::KB));
-  cfg.blockDim = dim3(320, 1, 1);
-  cfg.dynamicSmemBytes = K::SMEM;
-  cfg.stream = s;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = (unsigned)grp;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, k_attn_dkdv_tc<HD>, q64, o64, k128, v128, a);
-  if (e != cudaSuccess) return e;
   dim3 gq(a.hq, B, (a.S + Q::QB - 1) / Q::QB);
-  k_attn_dq_tc<HD><<<gq, 320, Q::SMEM, s>>>(q128, o128, k64, v64, a);
-  return cudaGetLastError();
+  cudaError_t e = launch_k(k_attn_dq_tc<HD>, gq, dim3(320), Q::SMEM, s, 0, q128, o128, k64, v64, a);
+  if (e != cudaSuccess) return e;
+  const dim3 gkv((unsigned)grp, (unsigned)(B * a.hkv), (unsigned)((a.S + K::KB - 1) / K::KB));
+  return launch_k(k_attn_dkdv_tc<HD>, gkv, dim3(320), K::SMEM, s, (unsigned)grp, q64, o64, k128, v128, a);
 }
 
 // LST_ATTN_BWD=mma selects the warp-level mma.sync backward (for comparing the two).
@@ -1618,14 +1620,15 @@ cudaError_t attention_bwd(const AttnBwdArgs& a, cudaStream_t s) {
   if (!check_common(a.hd, a.hq, a.hkv, a.S, a.T)) return cudaErrorInvalidValue;
   if (a.hq / a.hkv > kMaxGroup) return cudaErrorInvalidValue;
   const int B = (int)(a.T / a.S);
+  if (!use_mma_bwd()) {  // dQ (which forms D) then dK / dV
+    const cudaError_t e = a.hd == 128 ? launch_bwd_tc<128>(a, B, s) : launch_bwd_tc<64>(a, B, s);
+    note_launch(2);
+    return e;
+  }
   {
     const int64_t n = a.T * (int64_t)a.hq;
-    k_attn_D<<<(unsigned)((n + 7) / 8), 256, 0, s>>>(a);
-  }
-  if (!use_mma_bwd()) {
-    const cudaError_t e = a.hd == 128 ? launch_bwd_tc<128>(a, B, s) : launch_bwd_tc<64>(a, B, s);
-    note_launch(3);
-    return e;
+    const cudaError_t e = launch_k(k_attn_D, dim3((unsigned)((n + 7) / 8)), dim3(256), 0, s, 0, a);
+    if (e != cudaSuccess) return e;
   }
   dim3 gq(a.hq, B, (a.S + 63) / 64);
   cudaError_t e;

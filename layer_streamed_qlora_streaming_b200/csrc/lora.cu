@@ -17,6 +17,7 @@
 // 128/cs rows in slice order 0, 1, ..., cs-1, and stored by the mode's epilogue. No atomics and no
 // global scratch: the result depends only on the shapes, so it is deterministic.
 #include "common.cuh"
+#include "pdl.cuh"
 #include "gemm.cuh"
 #include "lora.cuh"
 
@@ -170,6 +171,8 @@ k_side(const __grid_constant__ SideProbs P, const int nk, const int kps, const i
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // inputs of the previous kernel in the stream are complete from here on
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -304,19 +307,8 @@ cudaError_t launch_side(SideProbs& P, int K, cudaStream_t st, int b_off = 0) {
   int cs = 1;
   while (cs < kMaxCluster && tiles * cs * 2 <= slots && cs * 2 <= nk) cs *= 2;
   const int kps = (nk + cs - 1) / cs;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)cs, (unsigned)tiles, 1);
-  cfg.blockDim = dim3(192, 1, 1);
-  cfg.dynamicSmemBytes = kSmem;
-  cfg.stream = st;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = (unsigned)cs;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_side<AMN, BMN, DUAL>, P, nk, kps, b_off);
+  const cudaError_t e = launch_k(k_side<AMN, BMN, DUAL>, dim3((unsigned)cs, (unsigned)tiles, 1), dim3(192), kSmem, st,
+                                 (unsigned)cs, P, nk, kps, b_off);
   note_launch(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -330,6 +322,8 @@ __device__ __forceinline__ __nv_bfloat16 split_part(float v, int sec) {
 }
 
 __global__ void k_lora_prep(const LoraPrepArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int R = a.nseg * a.r;
   const int out = a.bounds[a.nseg];
   const int64_t n1 = (int64_t)a.KP * a.in;
@@ -472,9 +466,9 @@ cudaError_t lora_grads(const __nv_bfloat16* X, int64_t ldx, int in, const __nv_b
 
 cudaError_t lora_prep(const LoraPrepArgs& a, cudaStream_t st) {
   if (a.nseg < 1 || a.nseg > 3 || a.nseg * a.r > a.RS || a.RS % 8 || 3 * a.RS > a.KP) return cudaErrorInvalidValue;
-  k_lora_prep<<<1024, 256, 0, st>>>(a);
+  const cudaError_t e = launch_k(k_lora_prep, dim3(1024), dim3(256), 0, st, 0, a);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace lst

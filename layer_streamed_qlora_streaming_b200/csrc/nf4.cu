@@ -12,6 +12,7 @@
 //   * dequant: a^ = (q * s) / 127 + mean and w^ = bf16_rne(code_value * a^), every operation a
 //     single fp32 rounding (explicit _rn intrinsics, so no multiply-add contraction).
 #include "common.cuh"
+#include "pdl.cuh"
 #include "nf4.cuh"
 
 #include <algorithm>
@@ -156,6 +157,8 @@ struct DequantJob {
 
 // Each thread expands 16 codes (8 packed bytes) into 16 bf16 values (two 16-byte stores).
 __global__ void __launch_bounds__(256) k_dequant(const DequantJob job, __nv_bfloat16* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float cb[16];
   if (threadIdx.x < 16) cb[threadIdx.x] = job.tab.cb[threadIdx.x];
   __syncthreads();
@@ -202,9 +205,9 @@ cudaError_t nf4_dequant(const Nf4Seg* segs, int nseg, __nv_bfloat16* out, cudaSt
   job.nseg = nseg;
   job.tab = nf4_table();
   const int64_t chunks = total / 16;
-  k_dequant<<<(unsigned)((chunks + 255) / 256), 256, 0, s>>>(job, out);
+  const cudaError_t e = launch_k(k_dequant, dim3((unsigned)((chunks + 255) / 256)), dim3(256), 0, s, 0, job, out);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace lst

@@ -5,6 +5,7 @@
 // partials summed in index order), so results do not depend on scheduling: the streamed and the
 // resident schedule run the same launches and give the same bytes.
 #include "common.cuh"
+#include "pdl.cuh"
 #include "ex2.cuh"
 #include "ops.cuh"
 
@@ -40,6 +41,8 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 // ------------------------------------------------------------------------------- RMSNorm
 __global__ void k_rmsnorm_fwd(const float* __restrict__ x, const float* __restrict__ g, int d, float eps,
                               bf16* __restrict__ y, float* __restrict__ rstd) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
   const float* xr = x + row * d;
@@ -66,6 +69,8 @@ __global__ void k_rmsnorm_fwd(const float* __restrict__ x, const float* __restri
 __global__ void k_rmsnorm_bwd(const float* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ g,
                               const float* __restrict__ rstd, const float* __restrict__ dres, int d,
                               float* __restrict__ dx, bf16* __restrict__ dxb) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
   const float r = rstd[row];
@@ -139,6 +144,8 @@ __global__ void k_rope_tables(int S, int hd, double theta, float* ct, float* st)
 // ------------------------------------------------------------------------------- SwiGLU
 // 8 consecutive elements per thread (16-byte loads and stores); F is a multiple of 8.
 __global__ void k_swiglu_fwd(const bf16* __restrict__ gu, int64_t T, int F, bf16* __restrict__ m) {
+  pdl_wait();
+  pdl_trigger();
   const int f8 = F / 8;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= T * f8) return;
@@ -166,6 +173,8 @@ __global__ void k_swiglu_fwd(const bf16* __restrict__ gu, int64_t T, int F, bf16
 
 __global__ void k_swiglu_bwd(const float* __restrict__ dm, const bf16* __restrict__ gu, int64_t T, int F,
                              bf16* __restrict__ dgu) {
+  pdl_wait();
+  pdl_trigger();
   const int f8 = F / 8;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= T * f8) return;
@@ -202,6 +211,8 @@ __global__ void k_swiglu_bwd(const float* __restrict__ dm, const bf16* __restric
 // ------------------------------------------------------------------------------- embedding
 __global__ void k_embed(const int32_t* __restrict__ tok, const bf16* __restrict__ E, int64_t T, int d, int V,
                         float* __restrict__ x) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // 8-element vector index
   const int nv = d / 8;
   if (i >= T * nv) return;
@@ -238,6 +249,8 @@ __device__ __forceinline__ void ms_add4(float& m, float& s, float4 v) {
 __global__ void __launch_bounds__(1024, 1)
 k_ce(const float* __restrict__ logits, int V, const int32_t* __restrict__ y, float inv_T,
      float* __restrict__ loss_rows, bf16* __restrict__ dlog) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float sm[32], ss[32];
   const int64_t row = blockIdx.x;
   const float* lr = logits + row * V;
@@ -348,6 +361,8 @@ k_ce_cluster(const float* __restrict__ logits, int V, int slice, const int32_t* 
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait();  // the logits of the previous kernel are complete from here on
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int k = 0; k < kCeChunks; ++k) {
       const int a = min(n4, k * q4), b = min(n4, a + q4);
@@ -440,6 +455,8 @@ __device__ __forceinline__ float row_lse(const float* __restrict__ lr, int V, fl
 __global__ void __launch_bounds__(1024, 1)
 k_ce_stats(const float* __restrict__ logits, int V, const int32_t* __restrict__ y, float* __restrict__ lse_out,
            float* __restrict__ logp_out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float sm[32], ss[32];
   const int64_t row = blockIdx.x;
   const float* lr = logits + row * V;
@@ -457,6 +474,8 @@ k_ce_stats(const float* __restrict__ logits, int V, const int32_t* __restrict__ 
 
 // One block per sequence; the block_sum tree fixes the order.
 __global__ void k_seq_sum(const float* __restrict__ v, const int32_t* __restrict__ mask, int S, float* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[32];
   const int64_t base = (int64_t)blockIdx.x * S;
   float acc = 0.f;
@@ -467,6 +486,8 @@ __global__ void k_seq_sum(const float* __restrict__ v, const int32_t* __restrict
 
 __global__ void k_dpo(const float* __restrict__ pi, const float* __restrict__ ref, int P, float beta,
                       float* __restrict__ loss, float* __restrict__ w) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[32];
   float part = 0.f;
   for (int p = threadIdx.x; p < P; p += blockDim.x) {
@@ -484,6 +505,8 @@ __global__ void __launch_bounds__(1024, 1)
 k_ce_grad(const float* __restrict__ logits, int64_t row0, int V, const int32_t* __restrict__ y,
           const float* __restrict__ lse_rows, const float* __restrict__ wseq, const int32_t* __restrict__ mask, int S,
           bf16* __restrict__ dlog) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t lrow = blockIdx.x, row = row0 + lrow;
   const float* lr = logits + lrow * V;
   bf16* dr = dlog + lrow * V;
@@ -511,6 +534,8 @@ k_ce_grad(const float* __restrict__ logits, int64_t row0, int V, const int32_t* 
 }
 
 __global__ void k_mean(const float* __restrict__ v, int64_t n, float* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[32];
   float s = 0.f;
   for (int64_t i = threadIdx.x; i < n; i += blockDim.x) s += v[i];
@@ -520,6 +545,8 @@ __global__ void k_mean(const float* __restrict__ v, int64_t n, float* __restrict
 
 __global__ void k_dot_partial(const float* __restrict__ a, const bf16* __restrict__ b, int64_t n,
                               float* __restrict__ part) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[32];
   const int64_t per = (n + gridDim.x - 1) / gridDim.x;
   const int64_t lo = blockIdx.x * per, hi = min(n, lo + per);
@@ -529,6 +556,8 @@ __global__ void k_dot_partial(const float* __restrict__ a, const bf16* __restric
   if (threadIdx.x == 0) part[blockIdx.x] = s;
 }
 __global__ void k_sum_in_order(const float* __restrict__ part, int n, float* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x == 0 && blockIdx.x == 0) {
     float s = 0.f;
     for (int i = 0; i < n; ++i) s += part[i];
@@ -537,16 +566,22 @@ __global__ void k_sum_in_order(const float* __restrict__ part, int n, float* __r
 }
 
 __global__ void k_f32_to_bf16(const float* __restrict__ x, int64_t n, bf16* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) y[i] = __float2bfloat16_rn(x[i]);
 }
 // 16-byte words src -> dst (n words), grid-stride
 __global__ void k_copy16(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
     dst[i] = src[i];
 }
 
 __global__ void k_bf16_to_f32(const bf16* __restrict__ x, int64_t n, float* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) y[i] = __bfloat162float(x[i]);
 }
@@ -558,16 +593,16 @@ inline unsigned nblk(int64_t n, int t = kThreads) { return (unsigned)((n + t - 1
 cudaError_t rmsnorm_fwd(const float* x, const float* g, int64_t T, int d, float eps, bf16* y, float* rstd,
                         cudaStream_t s) {
   if (d % 8) return cudaErrorInvalidValue;
-  k_rmsnorm_fwd<<<(unsigned)T, d >= 2048 ? 256 : 128, 0, s>>>(x, g, d, eps, y, rstd);
+  const cudaError_t e = launch_k(k_rmsnorm_fwd, dim3((unsigned)T), dim3(d >= 2048 ? 256 : 128), 0, s, 0, x, g, d, eps, y, rstd);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t rmsnorm_bwd(const float* dy, const float* x, const float* g, const float* rstd, const float* dres,
                         int64_t T, int d, float* dx, bf16* dxb, cudaStream_t s) {
   if (d % 8) return cudaErrorInvalidValue;
-  k_rmsnorm_bwd<<<(unsigned)T, 256, 0, s>>>(dy, x, g, rstd, dres, d, dx, dxb);
+  const cudaError_t e = launch_k(k_rmsnorm_bwd, dim3((unsigned)T), dim3(256), 0, s, 0, dy, x, g, rstd, dres, d, dx, dxb);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t rope(bf16* buf, int64_t ld, int64_t T, int S, int col0, int nh, int hd, const float* ct,
                  const float* st, int inverse, cudaStream_t s) {
@@ -582,21 +617,21 @@ cudaError_t rope_tables(int S, int hd, double theta, float* ct, float* st, cudaS
 }
 cudaError_t swiglu_fwd(const bf16* gu, int64_t T, int F, bf16* m, cudaStream_t s) {
   if (F % 8) return cudaErrorInvalidValue;
-  k_swiglu_fwd<<<nblk(T * (F / 8)), kThreads, 0, s>>>(gu, T, F, m);
+  const cudaError_t e = launch_k(k_swiglu_fwd, dim3(nblk(T * (F / 8))), dim3(kThreads), 0, s, 0, gu, T, F, m);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t swiglu_bwd(const float* dm, const bf16* gu, int64_t T, int F, bf16* dgu, cudaStream_t s) {
   if (F % 8) return cudaErrorInvalidValue;
-  k_swiglu_bwd<<<nblk(T * (F / 8)), kThreads, 0, s>>>(dm, gu, T, F, dgu);
+  const cudaError_t e = launch_k(k_swiglu_bwd, dim3(nblk(T * (F / 8))), dim3(kThreads), 0, s, 0, dm, gu, T, F, dgu);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t embed(const int32_t* tok, const bf16* E, int64_t T, int d, int V, float* x, cudaStream_t s) {
   if (d % 8) return cudaErrorInvalidValue;
-  k_embed<<<nblk(T * (d / 8)), kThreads, 0, s>>>(tok, E, T, d, V, x);
+  const cudaError_t e = launch_k(k_embed, dim3(nblk(T * (d / 8))), dim3(kThreads), 0, s, 0, tok, E, T, d, V, x);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t cross_entropy(const float* logits, int64_t T, int V, const int32_t* y, float inv_T, float* loss_rows,
                           bf16* dlog, cudaStream_t s) {
@@ -607,9 +642,10 @@ cudaError_t cross_entropy(const float* logits, int64_t T, int V, const int32_t* 
   while (cs < 8 && (((int64_t)V + cs - 1) / cs) * 4 > kTargetBytes) cs *= 2;
   const int slice = (int)((((int64_t)V + cs - 1) / cs + 3) / 4 * 4);
   if ((V % 4) || (int64_t)slice * 4 > kMaxSliceBytes || T * cs > INT32_MAX) {
-    k_ce<<<(unsigned)T, 1024, 0, s>>>(logits, V, y, inv_T, loss_rows, dlog);  // the two-pass form
+    const cudaError_t e = launch_k(k_ce, dim3((unsigned)T), dim3(1024), 0, s, 0, logits, V, y, inv_T, loss_rows,
+                                   dlog);  // the two-pass form
     note_launch(1);
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
   }
   const int smem = slice * 4 + 8 + 8 * kCeChunks;  // the slice, the (max, sum) pair and the mbarriers
   static std::atomic<unsigned long long> attr_done{0};
@@ -619,73 +655,63 @@ cudaError_t cross_entropy(const float* logits, int64_t T, int V, const int32_t* 
     if (e != cudaSuccess) return e;
     mark_done_on_device(attr_done);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(T * cs), 1, 1);
-  cfg.blockDim = dim3(kCeThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = (unsigned)cs;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_ce_cluster, logits, V, slice, y, inv_T, loss_rows, dlog);
+  const cudaError_t e = launch_k(k_ce_cluster, dim3((unsigned)(T * cs)), dim3(kCeThreads), (size_t)smem, s,
+                                 (unsigned)cs, logits, V, slice, y, inv_T, loss_rows, dlog);
   note_launch(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t ce_stats(const float* logits, int64_t T, int V, const int32_t* y, float* lse, float* logp, cudaStream_t s) {
-  k_ce_stats<<<(unsigned)T, 1024, 0, s>>>(logits, V, y, lse, logp);
+  const cudaError_t e = launch_k(k_ce_stats, dim3((unsigned)T), dim3(1024), 0, s, 0, logits, V, y, lse, logp);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t seq_sum(const float* v, const int32_t* mask, int nseq, int S, float* out, cudaStream_t s) {
-  k_seq_sum<<<nseq, 256, 0, s>>>(v, mask, S, out);
+  const cudaError_t e = launch_k(k_seq_sum, dim3(nseq), dim3(256), 0, s, 0, v, mask, S, out);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t dpo_loss(const float* pi, const float* ref, int P, float beta, float* loss, float* w, cudaStream_t s) {
-  k_dpo<<<1, 256, 0, s>>>(pi, ref, P, beta, loss, w);
+  const cudaError_t e = launch_k(k_dpo, dim3(1), dim3(256), 0, s, 0, pi, ref, P, beta, loss, w);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t ce_grad(const float* logits, int64_t rows, int64_t row0, int V, const int32_t* y, const float* lse,
                     const float* w, const int32_t* mask, int S, bf16* dlog, cudaStream_t s) {
-  k_ce_grad<<<(unsigned)rows, 1024, 0, s>>>(logits, row0, V, y, lse, w, mask, S, dlog);
+  const cudaError_t e = launch_k(k_ce_grad, dim3((unsigned)rows), dim3(1024), 0, s, 0, logits, row0, V, y, lse, w, mask, S, dlog);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t mean_fixed(const float* v, int64_t n, float* out, cudaStream_t s) {
-  k_mean<<<1, 1024, 0, s>>>(v, n, out);
+  const cudaError_t e = launch_k(k_mean, dim3(1), dim3(1024), 0, s, 0, v, n, out);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t dot_fixed(const float* a, const bf16* b, int64_t n, float* part, float* out, cudaStream_t s) {
-  k_dot_partial<<<1024, 256, 0, s>>>(a, b, n, part);
-  k_sum_in_order<<<1, 32, 0, s>>>(part, 1024, out);
+  cudaError_t e = launch_k(k_dot_partial, dim3(1024), dim3(256), 0, s, 0, a, b, n, part);
+  if (e == cudaSuccess) e = launch_k(k_sum_in_order, dim3(1), dim3(32), 0, s, 0, part, 1024, out);
   note_launch(2);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t f32_to_bf16(const float* x, int64_t n, bf16* y, cudaStream_t s) {
-  k_f32_to_bf16<<<nblk(n), kThreads, 0, s>>>(x, n, y);
+  const cudaError_t e = launch_k(k_f32_to_bf16, dim3(nblk(n)), dim3(kThreads), 0, s, 0, x, n, y);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t bf16_to_f32(const bf16* x, int64_t n, float* y, cudaStream_t s) {
-  k_bf16_to_f32<<<nblk(n), kThreads, 0, s>>>(x, n, y);
+  const cudaError_t e = launch_k(k_bf16_to_f32, dim3(nblk(n)), dim3(kThreads), 0, s, 0, x, n, y);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t copy16(const void* src, void* dst, int64_t bytes, cudaStream_t s) {
   if (bytes <= 0) return cudaSuccess;
   if (bytes % 16 || (reinterpret_cast<uintptr_t>(src) & 15) || (reinterpret_cast<uintptr_t>(dst) & 15))
     return cudaErrorInvalidValue;
   const int64_t n = bytes / 16;
-  k_copy16<<<(unsigned)std::min<int64_t>((n + kThreads - 1) / kThreads, 1024), kThreads, 0, s>>>(
-      reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst), n);
+  const cudaError_t e = launch_k(k_copy16, dim3((unsigned)std::min<int64_t>((n + kThreads - 1) / kThreads, 1024)),
+                                 dim3(kThreads), 0, s, 0, reinterpret_cast<const uint4*>(src),
+                                 reinterpret_cast<uint4*>(dst), n);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace lst

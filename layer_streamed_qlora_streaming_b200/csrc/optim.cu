@@ -11,6 +11,7 @@
 // (bf16(p), bf16(p - bf16(p))) to the places the element occupies in the group operands
 // (Acat [KP, in] or Bexp [out, KP]) the GEMMs read.
 #include "common.cuh"
+#include "pdl.cuh"
 #include "optim.cuh"
 
 namespace lst {
@@ -18,6 +19,8 @@ namespace {
 
 __global__ void k_adamw(const AdamTensor* __restrict__ tab, float* __restrict__ p, const float* __restrict__ g,
                         float* __restrict__ m, float* __restrict__ v, const AdamHyper h) {
+  pdl_wait();
+  pdl_trigger();
   const AdamTensor t = tab[blockIdx.y];
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < t.n; e += (int64_t)gridDim.x * blockDim.x) {
     const int64_t i = t.off + e;
@@ -46,9 +49,9 @@ cudaError_t adamw_update(const AdamTensor* tab_dev, int ntensors, int64_t max_nu
   int64_t bx = (max_numel + 255) / 256;
   if (bx > 64) bx = 64;  // grid-stride inside each tensor
   dim3 grid((unsigned)bx, (unsigned)ntensors);
-  k_adamw<<<grid, 256, 0, s>>>(tab_dev, params, grads, m, v, h);
+  const cudaError_t e = launch_k(k_adamw, grid, dim3(256), 0, s, 0, tab_dev, params, grads, m, v, h);
   note_launch(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace lst
