@@ -624,7 +624,9 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
 // --------------------------------------------------------------------------- backward: dQ, tcgen05
 // One CTA per 128 queries of one head (heaviest first), 320 threads: warp 0 TMA (Q and dO once; K
-// and V tiles of 64 keys, double-buffered), warp 1 MMA issuer, warps 2-9 two threads per query row.
+// and V tiles of 64 keys, three in flight), warp 1 MMA issuer, warps 2-9 two threads per query row.
+// The row's threads first form D = rowsum(dO o O) and store it: this kernel runs before the dK / dV
+// kernel, which reads D.
 //   S = Q K^T, dP = dO V^T   tcgen05 (bf16), into one of two TMEM buffer pairs;
 //   dS = P (dP - D)          the row's threads, P = exp2(S' - lse'), written bf16 to one of two
 //                            swizzled tiles (so block j+1's dS is written while dQ reads block j's);
@@ -638,7 +640,8 @@ struct DqTc {
   static constexpr uint32_t Q_BYTES = (HD / 64) * CH;
   static constexpr uint32_t KV_BYTES = 2 * (HD / 64) * KCH;  // K then V of one stage
   static constexpr uint32_t DS_BYTES = CH;                   // 128 queries x 64 keys bf16
-  static constexpr uint32_t SMEM = 2 * Q_BYTES + 2 * KV_BYTES + 2 * DS_BYTES + 1024 + 256;
+  static constexpr int KV_STAGES = 3;                        // K / V tiles in flight
+  static constexpr uint32_t SMEM = 2 * Q_BYTES + KV_STAGES * KV_BYTES + 2 * DS_BYTES + 1024 + 256;
   static constexpr uint32_t TMEM_COLS = 512;                 // S[2] at 0/64, dP[2] at 128/192, dQ at 256
 };
 
@@ -651,17 +654,18 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sO = sQ + C::Q_BYTES;          // dO
-  uint8_t* sKV = sO + C::Q_BYTES;         // [2] stages: K chunks, then V chunks
-  uint8_t* sDS = sKV + 2 * C::KV_BYTES;  // [2] dS tiles
+  constexpr int NS = C::KV_STAGES;
+  uint8_t* sKV = sO + C::Q_BYTES;          // [NS] stages: K chunks, then V chunks
+  uint8_t* sDS = sKV + NS * C::KV_BYTES;  // [2] dS tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + 2 * C::DS_BYTES);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_free = bars + 7;    // [2]
-  uint64_t* ds_full = bars + 9;   // [2]
-  uint64_t* ds_free = bars + 11;  // [2] the dQ MMAs of the tile's block are done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* kv_full = bars + 1;        // [NS]
+  uint64_t* kv_empty = bars + 1 + NS;  // [NS]
+  uint64_t* s_full = bars + 1 + 2 * NS;   // [2]
+  uint64_t* s_free = s_full + 2;          // [2]
+  uint64_t* ds_full = s_full + 4;         // [2]
+  uint64_t* ds_free = s_full + 6;         // [2] the dQ MMAs of the tile's block are done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 8);
 
   const int h = blockIdx.x, b = blockIdx.y, qb = (int)gridDim.z - 1 - (int)blockIdx.z;
   const int kvh = h / (p.hq / p.hkv);
@@ -672,9 +676,11 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 256);
       mbar_init(&ds_full[i], 256);
@@ -708,15 +714,15 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         tma_load_2d(sO + c * C::CH, &tmO, q_full, h * HD + c * 64, (int32_t)(tok0 + q0));
       }
       for (int j = 0; j < nkb; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait(&kv_empty[st], ((j - 2) >> 1) & 1)) break;
-        uint8_t* sk = sKV + st * C::KV_BYTES;
-        mbar_arrive_expect_tx(&kv_full[st], C::KV_BYTES);
+        const int ks = j % NS;
+        if (j >= NS && !mbar_wait(&kv_empty[ks], ((j - NS) / NS) & 1)) break;
+        uint8_t* sk = sKV + ks * C::KV_BYTES;
+        mbar_arrive_expect_tx(&kv_full[ks], C::KV_BYTES);
         const int32_t y = (int32_t)(tok0 + j * C::KB);
 #pragma unroll
         for (int c = 0; c < HD / 64; ++c) {
-          tma_load_2d(sk + c * C::KCH, &tmK, &kv_full[st], kvh * HD + c * 64, y);
-          tma_load_2d(sk + (HD / 64 + c) * C::KCH, &tmV, &kv_full[st], kvh * HD + c * 64, y);
+          tma_load_2d(sk + c * C::KCH, &tmK, &kv_full[ks], kvh * HD + c * 64, y);
+          tma_load_2d(sk + (HD / 64 + c) * C::KCH, &tmV, &kv_full[ks], kvh * HD + c * 64, y);
         }
       }
     }
@@ -727,12 +733,12 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       bool ok = mbar_wait(q_full, 0);
       for (int j = 0; j <= nkb && ok; ++j) {
         if (j < nkb) {  // S_j = Q K_j^T and dP_j = dO V_j^T into buffer pair j & 1
-          const int st = j & 1;
-          if (!mbar_wait(&kv_full[st], (j >> 1) & 1)) break;
+          const int st = j & 1, ks = j % NS;
+          if (!mbar_wait(&kv_full[ks], (j / NS) & 1)) break;
           if (j >= 2 && !mbar_wait(&s_free[st], ((j - 2) >> 1) & 1)) break;
           tc_fence_after();
           const uint32_t q = smem_u32(sQ), o = smem_u32(sO);
-          const uint32_t k = smem_u32(sKV + st * C::KV_BYTES), v = k + (HD / 64) * C::KCH;
+          const uint32_t k = smem_u32(sKV + ks * C::KV_BYTES), v = k + (HD / 64) * C::KCH;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             const uint32_t offq = (kk >> 2) * C::CH + (kk & 3) * 32, offk = (kk >> 2) * C::KCH + (kk & 3) * 32;
@@ -743,17 +749,17 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
           umma_commit(&s_full[st]);
         }
         if (j >= 1) {  // dQ += dS_{j-1} K_{j-1}
-          const int i = j - 1, st = i & 1;
+          const int i = j - 1, st = i & 1, ks = i % NS;
           if (!mbar_wait(&ds_full[st], (i >> 1) & 1)) break;
           tc_fence_after();
-          const uint32_t ds = smem_u32(sDS + st * C::DS_BYTES), k = smem_u32(sKV + st * C::KV_BYTES);
+          const uint32_t ds = smem_u32(sDS + st * C::DS_BYTES), k = smem_u32(sKV + ks * C::KV_BYTES);
 #pragma unroll
           for (int kk = 0; kk < C::KB / 16; ++kk) {
             const uint64_t da = umma_desc(ds + kk * 32, 16, 1024);
             const uint64_t db = umma_desc(k + kk * 16 * 128, C::KCH, 1024);  // K rows = keys: MN-major
             umma_bf16(tmem + 256, da, db, idQ, (i | kk) != 0);
           }
-          umma_commit(&kv_empty[st]);
+          umma_commit(&kv_empty[ks]);
           umma_commit(&ds_free[st]);
         }
       }
@@ -769,7 +775,38 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = p.scale * kLog2e;
     const float lse2 = live ? p.lse[(tok0 + qrow) * p.hq + h] * kLog2e : 0.f;
-    const float dd = live ? p.D[(tok0 + qrow) * p.hq + h] : 0.f;
+    // D = rowsum(dO o O) of this row, with the forward's unrounded O when it was kept; both threads
+    // of the row add the same products in the same order, and half 0 stores it for the dK / dV kernel
+    float dd = 0.f;
+    if (live) {
+      const __nv_bfloat16* ap = p.dout + (tok0 + qrow) * p.lddo + (int64_t)h * HD;
+#pragma unroll 4
+      for (int c = 0; c < HD; c += 8) {
+        const uint4 au = *reinterpret_cast<const uint4*>(ap + c);
+        const __nv_bfloat16* a8 = reinterpret_cast<const __nv_bfloat16*>(&au);
+        float o8[8];
+        if (p.o32) {
+          const float* op = p.o32 + (tok0 + qrow) * (int64_t)p.hq * HD + (int64_t)h * HD + c;
+          const float4 u0 = *reinterpret_cast<const float4*>(op), u1 = *reinterpret_cast<const float4*>(op + 4);
+          o8[0] = u0.x;
+          o8[1] = u0.y;
+          o8[2] = u0.z;
+          o8[3] = u0.w;
+          o8[4] = u1.x;
+          o8[5] = u1.y;
+          o8[6] = u1.z;
+          o8[7] = u1.w;
+        } else {
+          const uint4 ou = *reinterpret_cast<const uint4*>(p.o + (tok0 + qrow) * p.ldo + (int64_t)h * HD + c);
+          const __nv_bfloat16* b8 = reinterpret_cast<const __nv_bfloat16*>(&ou);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o8[e] = __bfloat162float(b8[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dd += __bfloat162float(a8[e]) * o8[e];
+      }
+      if (half == 0) p.D[(tok0 + qrow) * p.hq + h] = dd;
+    }
     bool ok = true;
     for (int j = 0; j < nkb && ok; ++j) {
       const int st = j & 1;
@@ -862,7 +899,7 @@ k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 // --------------------------------------------------------------------------- backward: dK, dV, tcgen05
 // grid (grp, B * hkv, ceil(S/128)), cluster (grp, 1, 1), 320 threads. The cluster owns 128 keys of
 // kv head kvh; its CTA of rank hh sums the contributions of query head kvh * grp + hh over query
-// blocks of 64 (double-buffered Q / dO tiles): warp 0 TMA, warp 1 MMA issuer, warps 2-9 two threads
+// blocks of 64 (three Q / dO tiles in flight): warp 0 TMA, warp 1 MMA issuer, warps 2-9 two threads
 // per key row.
 //   S^T = K Q^T, dP^T = V dO^T      tcgen05 (bf16), into one of two TMEM buffer pairs;
 //   P^T, dS^T = P^T (dP^T - D)      the key row's threads (lse and D of the block's queries from
@@ -881,7 +918,8 @@ struct DkvTc {
   static constexpr uint32_t QO_BYTES = 2 * (HD / 64) * QCH;  // Q then dO of one stage
   static constexpr uint32_t T_BYTES = 128 * 128;             // one [128 keys x 64 queries] bf16 tile
   static constexpr int RLD = HD + 4;                         // fp32 row stride of a parked tile
-  static constexpr uint32_t MAIN = 2 * K_BYTES + 2 * QO_BYTES + 4 * T_BYTES + 2 * 2 * QB * 4;
+  static constexpr int QO_STAGES = 3;                        // Q / dO tiles in flight
+  static constexpr uint32_t MAIN = 2 * K_BYTES + QO_STAGES * QO_BYTES + 4 * T_BYTES + 2 * 2 * QB * 4;
   static constexpr uint32_t PARK = 2 * 128 * RLD * 4;
   static constexpr uint32_t SMEM = (MAIN > PARK ? MAIN : PARK) + 1024 + 256;
   static constexpr uint32_t TMEM_COLS = 2 * 128 + 2 * HD <= 256 ? 256 : 512;
@@ -896,20 +934,21 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
   uint8_t* sV = sK + C::K_BYTES;
-  uint8_t* sQO = sV + C::K_BYTES;               // [2] stages: Q chunks, then dO chunks
-  uint8_t* sP = sQO + 2 * C::QO_BYTES;          // [2] P^T tiles
+  constexpr int NS = C::QO_STAGES;
+  uint8_t* sQO = sV + C::K_BYTES;               // [NS] stages: Q chunks, then dO chunks
+  uint8_t* sP = sQO + NS * C::QO_BYTES;         // [2] P^T tiles
   uint8_t* sS = sP + 2 * C::T_BYTES;            // [2] dS^T tiles
   float* sLse = reinterpret_cast<float*>(sS + 2 * C::T_BYTES);  // [2][64]
   float* sD = sLse + 2 * C::QB;                             // [2][64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (C::MAIN > C::PARK ? C::MAIN : C::PARK));
   uint64_t* kv_full = bars;
-  uint64_t* qo_full = bars + 1;   // [2]
-  uint64_t* qo_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_free = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;    // [2] P^T / dS^T tile pair written
-  uint64_t* t_free = bars + 11;   // [2] the dV / dK MMAs of the pair's block are done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* qo_full = bars + 1;        // [NS]
+  uint64_t* qo_empty = bars + 1 + NS;  // [NS]
+  uint64_t* s_full = bars + 1 + 2 * NS;  // [2]
+  uint64_t* s_free = s_full + 2;         // [2]
+  uint64_t* p_full = s_full + 4;         // [2] P^T / dS^T tile pair written
+  uint64_t* t_free = s_full + 6;         // [2] the dV / dK MMAs of the pair's block are done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 8);
   float* redK = reinterpret_cast<float*>(smem);  // after the main loop: [128][RLD] each
   float* redV = redK + 128 * C::RLD;
 
@@ -925,9 +964,11 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(&qo_full[i], 1);
       mbar_init(&qo_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 256);
       mbar_init(&p_full[i], 256);
@@ -963,15 +1004,15 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tma_load_2d(sV + c * C::CH, &tmV, kv_full, kvh * HD + c * 64, (int32_t)(tok0 + k0));
       }
       for (int j = 0; j < nqb; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait(&qo_empty[st], ((j - 2) >> 1) & 1)) break;
-        uint8_t* sq = sQO + st * C::QO_BYTES;
-        mbar_arrive_expect_tx(&qo_full[st], C::QO_BYTES);
+        const int qs = j % NS;
+        if (j >= NS && !mbar_wait(&qo_empty[qs], ((j - NS) / NS) & 1)) break;
+        uint8_t* sq = sQO + qs * C::QO_BYTES;
+        mbar_arrive_expect_tx(&qo_full[qs], C::QO_BYTES);
         const int32_t y = (int32_t)(tok0 + (i0 + j) * C::QB);
 #pragma unroll
         for (int c = 0; c < HD / 64; ++c) {
-          tma_load_2d(sq + c * C::QCH, &tmQ, &qo_full[st], h * HD + c * 64, y);
-          tma_load_2d(sq + (HD / 64 + c) * C::QCH, &tmO, &qo_full[st], h * HD + c * 64, y);
+          tma_load_2d(sq + c * C::QCH, &tmQ, &qo_full[qs], h * HD + c * 64, y);
+          tma_load_2d(sq + (HD / 64 + c) * C::QCH, &tmO, &qo_full[qs], h * HD + c * 64, y);
         }
       }
     }
@@ -982,12 +1023,12 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool okm = mbar_wait(kv_full, 0);
       for (int j = 0; j <= nqb && okm; ++j) {
         if (j < nqb) {  // S^T_j = K Q_j^T, dP^T_j = V dO_j^T into buffer pair j & 1
-          const int st = j & 1;
-          if (!mbar_wait(&qo_full[st], (j >> 1) & 1)) break;
+          const int st = j & 1, qs = j % NS;
+          if (!mbar_wait(&qo_full[qs], (j / NS) & 1)) break;
           if (j >= 2 && !mbar_wait(&s_free[st], ((j - 2) >> 1) & 1)) break;
           tc_fence_after();
           const uint32_t k = smem_u32(sK), v = smem_u32(sV);
-          const uint32_t q = smem_u32(sQO + st * C::QO_BYTES), o = q + (HD / 64) * C::QCH;
+          const uint32_t q = smem_u32(sQO + qs * C::QO_BYTES), o = q + (HD / 64) * C::QCH;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             const uint32_t offk = (kk >> 2) * C::CH + (kk & 3) * 32, offq = (kk >> 2) * C::QCH + (kk & 3) * 32;
@@ -998,11 +1039,11 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           umma_commit(&s_full[st]);
         }
         if (j >= 1) {  // dV += P^T dO, dK += dS^T Q of block j-1
-          const int i = j - 1, st = i & 1;
+          const int i = j - 1, st = i & 1, qs = i % NS;
           if (!mbar_wait(&p_full[st], (i >> 1) & 1)) break;
           tc_fence_after();
           const uint32_t pt = smem_u32(sP + st * C::T_BYTES), ds = smem_u32(sS + st * C::T_BYTES);
-          const uint32_t q = smem_u32(sQO + st * C::QO_BYTES), o = q + (HD / 64) * C::QCH;
+          const uint32_t q = smem_u32(sQO + qs * C::QO_BYTES), o = q + (HD / 64) * C::QCH;
 #pragma unroll
           for (int kk = 0; kk < C::QB / 16; ++kk) {
             umma_bf16(tV, umma_desc(pt + kk * 32, 16, 1024), umma_desc(o + kk * 16 * 128, C::QCH, 1024), idG,
@@ -1010,7 +1051,7 @@ k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             umma_bf16(tK, umma_desc(ds + kk * 32, 16, 1024), umma_desc(q + kk * 16 * 128, C::QCH, 1024), idG,
                       (i | kk) != 0);
           }
-          umma_commit(&qo_empty[st]);
+          umma_commit(&qo_empty[qs]);
           umma_commit(&t_free[st]);
         }
       }
