@@ -58,17 +58,6 @@ lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_
                       int64_t ldc, int32_t c_f32, float alpha, const float* bias,
                       const float* R, int64_t ldr, void* stream);
 
-/* The same GEMM with the SwiGLU backward as its epilogue (the dX GEMM of the down projection):
- * with d = alpha * (A' B' + A2 B2') [M, F] in fp32 (never stored), g = gu[t][j], u = gu[t][F + j]
- * (gu bf16 [M, 2F], row stride 2F) and s = 1 / (1 + exp(-g)), writes dgu bf16 [M, 2F]:
- * dgu[t][j] = d u s (1 + g (1 - s)), dgu[t][F + j] = d g s, computed in fp32 like
- * lst_k_swiglu_bwd on the fp32 output of lst_k_gemm. F % 8 == 0, gu and dgu 16-byte aligned;
- * the other arguments as lst_k_gemm. */
-lst_status lst_k_gemm_swiglu_bwd(int32_t M, int32_t F, int32_t K, const uint16_t* A, int64_t lda,
-                                 const uint16_t* B, int64_t ldb, int32_t b_mn, const uint16_t* A2,
-                                 int64_t lda2, const uint16_t* B2, int64_t ldb2, int32_t K2, float alpha,
-                                 const uint16_t* gu, uint16_t* dgu, void* stream);
-
 /* One NF4 tensor (format of lst_k_nf4_quantize) of a weight matrix stacked from up to three
  * such tensors along its rows (q/k/v, gate/up), covering `rows` consecutive rows. */
 typedef struct {

@@ -38,7 +38,6 @@ import torch
 
 sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 from layer_streamed_qlora_streaming_b200 import (k_attention_bwd, k_attention_fwd, k_cross_entropy, k_gemm, k_gemm_nf4,
-                                                 k_gemm_swiglu_bwd,
                                                  k_lora_grads, k_lora_grads_multi, k_lora_skinny, k_nf4_dequant,
                k_nf4_quantize)
 
@@ -52,7 +51,7 @@ GEMM_SHAPES = {
     "gemm_o": (T, D, D, 0, 64, 1, 1),              # o forward + residual
     "gemm_gu": (T, 2 * F, D, 0, 128, 0, 0),        # gate/up forward
     "gemm_down": (T, D, F, 0, 64, 1, 1),           # down forward + residual
-    "gemm_dx_down": (T, F, D, 1, 64, 1, 0),        # dX of down, with the SwiGLU backward as its epilogue
+    "gemm_dx_down": (T, F, D, 1, 64, 1, 0),        # dX of down
     "gemm_dx_gu": (T, D, 2 * F, 1, 128, 1, 0),     # dX of gate/up
     "gemm_dx_o": (T, D, D, 1, 64, 0, 0),           # dX of o (bf16 output)
     "gemm_dx_qkv": (T, D, 6144, 1, 192, 1, 0),     # dX of q/k/v
@@ -61,8 +60,6 @@ GEMM_SHAPES = {
 }
 # per step of the 32-layer stack: forward reads run 4 projection GEMMs, backward reads recompute 3
 # (the down projection's output is not needed) and run 4 dX GEMMs, and the head runs 2
-# the GEMMs whose epilogue is the SwiGLU backward (they write dL/d(gate, up), not their own output)
-SWIGLU_EPILOGUE = {"gemm_dx_down"}
 GEMM_LAUNCHES_PER_STEP = {"gemm_qkv": 64, "gemm_o": 64, "gemm_gu": 64, "gemm_down": 32, "gemm_dx_down": 32,
                           "gemm_dx_gu": 32, "gemm_dx_o": 32, "gemm_dx_qkv": 32, "gemm_head": 1, "gemm_dx_head": 1}
 
@@ -127,14 +124,6 @@ def build(case: str):
         B = _bf((K, N) if bmn else (N, K), g, 0.02)
         A2 = _bf((M, K2), g) if K2 else None
         B2 = (_bf((K2, N) if bmn else (N, K2), g, 0.01)) if K2 else None
-        if case in SWIGLU_EPILOGUE:
-            gu = _bf((M, 2 * N), g)
-            dgu = torch.empty(M, 2 * N, dtype=torch.bfloat16, device="cuda")
-
-            def run():
-                k_gemm_swiglu_bwd(M, N, K, A, K, B, N if bmn else K, bmn, gu, dgu, A2=A2, lda2=K2, B2=B2,
-                                  ldb2=(N if bmn else K2), K2=K2)
-            return run, {"flop": 2.0 * M * N * (K + K2), "bytes": None}
         C = torch.empty(M, N, dtype=torch.float32 if f32 else torch.bfloat16, device="cuda")
         R = torch.randn(M, N, generator=g, device="cuda") if resid else None
 

@@ -95,8 +95,6 @@ _SIGS = {
                               _F32, _P, _P, _I64, _P]),
     "lst_k_gemm": (_I32, [_I32, _I32, _I32, _P, _I64, _I32, _P, _I64, _I32, _P, _I64, _P, _I64, _I32,
                           _P, _I64, _I32, _F32, _P, _P, _I64, _P]),
-    "lst_k_gemm_swiglu_bwd": (_I32, [_I32, _I32, _I32, _P, _I64, _P, _I64, _I32, _P, _I64, _P, _I64, _I32, _F32, _P,
-                                     _P, _P]),
     "lst_k_attention_fwd": (_I32, [_P, _I64, _P, _I64, _P, _I64, _P, _I64, _P, _I64, _I32, _I32,
                                    _I32, _I32, _P]),
     "lst_k_attention_bwd": (_I32, [_P, _I64, _P, _I64, _P, _I64, _P, _I64, _P, _I64, _P, _P, _P,
@@ -392,13 +390,6 @@ def k_gemm(M, N, K, A, lda, B, ldb, b_mn, C_, ldc, c_f32, alpha=1.0, A2=None, ld
     _check(lib().lst_k_gemm(M, N, K, _ptr(A), lda, a_mn, _ptr(B), ldb, b_mn, _ptr(A2), lda2, _ptr(B2), ldb2,
                             K2, _ptr(C_), ldc, c_f32, alpha, _ptr(bias), _ptr(R), ldr, _stream(stream)),
            what="lst_k_gemm")
-
-
-def k_gemm_swiglu_bwd(M, F, K, A, lda, B, ldb, b_mn, gu, dgu, alpha=1.0, A2=None, lda2=0, B2=None, ldb2=0, K2=0,
-                      stream=None):
-    """dgu [M, 2F] bf16 = SwiGLU backward of d = alpha (A B' + A2 B2') at gu [M, 2F] (d not stored)."""
-    _check(lib().lst_k_gemm_swiglu_bwd(M, F, K, _ptr(A), lda, _ptr(B), ldb, b_mn, _ptr(A2), lda2, _ptr(B2), ldb2, K2,
-                                       alpha, _ptr(gu), _ptr(dgu), _stream(stream)), what="lst_k_gemm_swiglu_bwd")
 
 
 class Nf4Part(C.Structure):

@@ -342,7 +342,7 @@ struct lst_ctx {
   int n_gq = 0;
   __nv_bfloat16* Us[NGROUP] = {};  // split bf16 s * x A^T per group [T, KP] (sections hi, lo, hi)
   __nv_bfloat16* Vs[NGROUP] = {};  // split bf16 s * dy B per group [T, KP]
-  float *ga = nullptr, *gb = nullptr, *dn = nullptr;
+  float *ga = nullptr, *gb = nullptr, *dn = nullptr, *dm = nullptr;
   __nv_bfloat16 *dout_b = nullptr, *dh_b = nullptr, *do_b = nullptr, *dqkvb = nullptr, *dgu = nullptr;
   __nv_bfloat16* nf = nullptr;
   float *rstdf = nullptr, *logits = nullptr, *loss_rows = nullptr, *loss_dev = nullptr, *dot_part = nullptr;
@@ -622,11 +622,8 @@ lst_status group_fwd(lst_ctx* c, int layer, int g, const uint8_t* blob, const __
   return LST_OK;
 }
 
-// dX = dY W (+ the LoRA term) into dX; or, with sw_gu given (the down group), the SwiGLU backward of
-// that dX at gu into sw_dgu, done by the GEMM's epilogue (dX itself is not stored).
 lst_status group_bwd(lst_ctx* c, int layer, int g, const uint8_t* blob, const __nv_bfloat16* W, const __nv_bfloat16* dY,
-                     int64_t ldy, const __nv_bfloat16* X, int64_t ldx, void* dX, int dx_f32,
-                     const __nv_bfloat16* sw_gu = nullptr, __nv_bfloat16* sw_dgu = nullptr) {
+                     int64_t ldy, const __nv_bfloat16* X, int64_t ldx, void* dX, int dx_f32) {
   const Group& G = c->grp[g];
   const auto& D = c->der[layer * NGROUP + g];
   const int64_t T = c->curT;
@@ -654,14 +651,9 @@ lst_status group_bwd(lst_ctx* c, int layer, int g, const uint8_t* blob, const __
     a.B2 = D.Acat16;
     a.ldb2 = G.in;
     a.K2 = G.KP;
-    if (sw_gu) {
-      a.swiglu_gu = sw_gu;
-      a.swiglu_dgu = sw_dgu;
-    } else {
-      a.C = dX;
-      a.ldc = G.in;
-      a.c_f32 = dx_f32;
-    }
+    a.C = dX;
+    a.ldc = G.in;
+    a.c_f32 = dx_f32;
     ProfScope ps(c, c->stream, PC_GEMM, 2.0 * T * G.in * (double)(G.out + G.KP));
     CK(gemm_bf16(a, c->stream));
   }
@@ -796,8 +788,11 @@ lst_status layer_bwd(lst_ctx* c, int i, const uint8_t* blob, const uint8_t* hdr,
   const float* g2 = g1 + c->d;
   const float* x = c->xs + (int64_t)i * c->Tmax * c->d;
   c->n_gq = 0;
-  // dL/dm and the SwiGLU backward in one GEMM: its epilogue turns each fp32 dL/dm into dL/d(gate, up)
-  TRY(group_bwd(c, i, G_DOWN, blob, W, c->dout_b, c->d, c->m, c->F, nullptr, 1, c->gu, c->dgu));
+  TRY(group_bwd(c, i, G_DOWN, blob, W, c->dout_b, c->d, c->m, c->F, c->dm, 1));
+  {
+    ProfScope ps(c, c->stream, PC_OTHER);
+    CK(swiglu_bwd(c->dm, c->gu, T, c->F, c->dgu, c->stream));
+  }
   TRY(group_bwd(c, i, G_GU, blob, W, c->dgu, 2 * c->F, c->n2, c->d, c->dn, 1));
   {
     ProfScope ps(c, c->stream, PC_OTHER);
@@ -1596,6 +1591,7 @@ lst_status create_impl(lst_ctx* c, const float* embed, const float* final_norm, 
   TRY(dalloc(c, &c->ga, T * d));
   TRY(dalloc(c, &c->gb, T * d));
   TRY(dalloc(c, &c->dn, T * d));
+  TRY(dalloc(c, &c->dm, T * c->F));
   TRY(dalloc(c, &c->dout_b, T * d));
   TRY(dalloc(c, &c->dh_b, T * d));
   TRY(dalloc(c, &c->do_b, T * c->dq));

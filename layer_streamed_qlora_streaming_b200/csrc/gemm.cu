@@ -34,9 +34,6 @@ struct Epi {
   const float* rope_cos;
   const float* rope_sin;
   int rope_end, rope_hd, rope_S;
-  // SwiGLU backward instead of the store of C (N = F): gu / dgu [M, 2F]
-  const __nv_bfloat16* sw_gu;
-  __nv_bfloat16* sw_dgu;
 };
 
 // Rotate the pair of 32-column chunks (na .. na+31) and (nb .. nb+31), nb = na + hd/2, of one row
@@ -81,14 +78,11 @@ __device__ __forceinline__ void epi_store_rope(const Epi& e, int row, int na, in
 
 template <int BN>
 struct Cfg {
-  static constexpr int STAGES = BN == 256 ? 4 : (BN >= 192 ? 5 : 6);
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t SMEM = STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*bars*/;
   static constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;  // one accumulator; two are allocated
-  // the allocation: a power of two >= the two accumulators
-  static constexpr uint32_t TMEM_ALLOC = 2 * TMEM_COLS <= 128 ? 128 : (2 * TMEM_COLS <= 256 ? 256 : 512);
-  static constexpr uint32_t ACC_STRIDE = TMEM_ALLOC / 2;  // column of the second accumulator
 };
 
 __device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const uint32_t (&r)[32]) {
@@ -142,62 +136,6 @@ __device__ __forceinline__ void epi_store(const Epi& e, int row, int col0, const
     } else {
       for (int i = 0; i < 32; ++i)
         if (col0 + i < e.N) cp[i] = __float2bfloat16_rn(v[i]);
-    }
-  }
-}
-
-// SwiGLU backward of 32 columns col0 .. col0 + 31 of one row: d = alpha * acc is dL/dm there.
-__device__ __forceinline__ void epi_store_swiglu(const Epi& e, int row, int col0, const uint32_t (&r)[32]) {
-  if (row >= e.M || col0 >= e.N) return;
-  const int F = e.N;
-  const __nv_bfloat16* gp = e.sw_gu + (int64_t)row * 2 * F + col0;
-  __nv_bfloat16* dp = e.sw_dgu + (int64_t)row * 2 * F + col0;
-  const bool full = col0 + 32 <= F;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    if (!full && col0 + q * 8 >= F) break;
-    uint4 gv, uv;
-    if (full || col0 + q * 8 + 8 <= F) {
-      gv = *reinterpret_cast<const uint4*>(gp + q * 8);
-      uv = *reinterpret_cast<const uint4*>(gp + F + q * 8);
-    } else {
-      gv = uv = make_uint4(0, 0, 0, 0);
-      __nv_bfloat16* g8 = reinterpret_cast<__nv_bfloat16*>(&gv);
-      __nv_bfloat16* u8 = reinterpret_cast<__nv_bfloat16*>(&uv);
-      for (int i = 0; i < 8 && col0 + q * 8 + i < F; ++i) {
-        g8[i] = gp[q * 8 + i];
-        u8[i] = gp[F + q * 8 + i];
-      }
-    }
-    const __nv_bfloat16* g8 = reinterpret_cast<const __nv_bfloat16*>(&gv);
-    const __nv_bfloat16* u8 = reinterpret_cast<const __nv_bfloat16*>(&uv);
-    uint4 og, ou;
-    __nv_bfloat162* og2 = reinterpret_cast<__nv_bfloat162*>(&og);
-    __nv_bfloat162* ou2 = reinterpret_cast<__nv_bfloat162*>(&ou);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float rg[2], ru[2];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const float d = __uint_as_float(r[q * 8 + 2 * i + k]) * e.alpha;
-        const float g = __bfloat162float(g8[2 * i + k]), u = __bfloat162float(u8[2 * i + k]);
-        const float sg = 1.0f / (1.0f + expf(-g));
-        rg[k] = d * u * sg * (1.0f + g * (1.0f - sg));
-        ru[k] = d * g * sg;
-      }
-      og2[i] = __floats2bfloat162_rn(rg[0], rg[1]);
-      ou2[i] = __floats2bfloat162_rn(ru[0], ru[1]);
-    }
-    if (full || col0 + q * 8 + 8 <= F) {
-      *reinterpret_cast<uint4*>(dp + q * 8) = og;
-      *reinterpret_cast<uint4*>(dp + F + q * 8) = ou;
-    } else {
-      const __nv_bfloat16* a8 = reinterpret_cast<const __nv_bfloat16*>(&og);
-      const __nv_bfloat16* b8 = reinterpret_cast<const __nv_bfloat16*>(&ou);
-      for (int i = 0; i < 8 && col0 + q * 8 + i < F; ++i) {
-        dp[q * 8 + i] = a8[i];
-        dp[F + q * 8 + i] = b8[i];
-      }
     }
   }
 }
@@ -263,7 +201,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_ALLOC);
+    tmem_alloc(tmem_slot, 2 * C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -324,7 +262,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         // the epilogue must have drained this accumulator (its use two tiles ago)
         if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) break;
         tc_fence_after();
-        const uint32_t dacc = tmem + (uint32_t)(buf * C::ACC_STRIDE);
+        const uint32_t dacc = tmem + (uint32_t)(buf * C::TMEM_COLS);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1;
@@ -360,7 +298,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
       if (!mbar_wait(&acc_full[buf], use & 1)) break;
       tc_fence_after();
       const int row = m0 + q * 32 + lane;
-      const uint32_t tq = tmem + (uint32_t)(buf * C::ACC_STRIDE) + ((uint32_t)(q * 32) << 16);
+      const uint32_t tq = tmem + (uint32_t)(buf * C::TMEM_COLS) + ((uint32_t)(q * 32) << 16);
       if (n0 < ep.rope_end) {
         const int half = ep.rope_hd / 2;
 #pragma unroll 1
@@ -380,11 +318,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           uint32_t r[32];
           tmem_ld32(tq + c, r);
           tmem_ld_wait();
-          if (ep.sw_gu) {
-            epi_store_swiglu(ep, row, n0 + c, r);
-          } else {
-            epi_store(ep, row, n0 + c, r);
-          }
+          epi_store(ep, row, n0 + c, r);
         }
       }
       tc_fence_before();
@@ -395,7 +329,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_ALLOC);
+    tmem_dealloc(tmem, 2 * C::TMEM_COLS);
   }
 }
 
@@ -516,7 +450,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_ALLOC);
+    tmem_alloc(tmem_slot, 2 * C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -572,7 +506,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         const uint32_t use = (uint32_t)(local >> 1);
         if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) break;
         tc_fence_after();
-        const uint32_t dacc = tmem + (uint32_t)(buf * C::ACC_STRIDE);
+        const uint32_t dacc = tmem + (uint32_t)(buf * C::TMEM_COLS);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1;
@@ -613,7 +547,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       if (!mbar_wait(&acc_full[buf], use & 1)) break;
       tc_fence_after();
       const int row = m0 + qd * 32 + lane;
-      const uint32_t tq = tmem + (uint32_t)(buf * C::ACC_STRIDE) + ((uint32_t)(qd * 32) << 16);
+      const uint32_t tq = tmem + (uint32_t)(buf * C::TMEM_COLS) + ((uint32_t)(qd * 32) << 16);
       if (n0 < ep.rope_end) {
         const int half = ep.rope_hd / 2;
 #pragma unroll 1
@@ -633,11 +567,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
           uint32_t r[32];
           tmem_ld32(tq + c, r);
           tmem_ld_wait();
-          if (ep.sw_gu) {
-            epi_store_swiglu(ep, row, n0 + c, r);
-          } else {
-            epi_store(ep, row, n0 + c, r);
-          }
+          epi_store(ep, row, n0 + c, r);
         }
       }
       tc_fence_before();
@@ -670,7 +600,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_ALLOC);
+    tmem_dealloc(tmem, 2 * C::TMEM_COLS);
   }
 }
 
@@ -723,7 +653,7 @@ cudaError_t launch_nf4(const GemmArgs& a, cudaStream_t s) {
     tB2 = tA;
   }
   Epi e{a.C, a.ldc, a.bias, a.R, a.ldr, a.alpha, a.c_f32, a.M, a.N,
-        a.rope_cos, a.rope_sin, a.rope_cos ? a.rope_end : 0, a.rope_hd, a.rope_S, a.swiglu_gu, a.swiglu_dgu};
+        a.rope_cos, a.rope_sin, a.rope_cos ? a.rope_end : 0, a.rope_hd, a.rope_S};
   static std::atomic<unsigned long long> attr_done{0};
   if (!done_on_device(attr_done)) {
     const cudaError_t err = cudaFuncSetAttribute(k_gemm_nf4<BN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemQ);
@@ -773,7 +703,7 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
     tB2 = tB;
   }
   Epi e{a.C, a.ldc, a.bias, a.R, a.ldr, a.alpha, a.c_f32, a.M, a.N,
-        a.rope_cos, a.rope_sin, a.rope_cos ? a.rope_end : 0, a.rope_hd, a.rope_S, a.swiglu_gu, a.swiglu_dgu};
+        a.rope_cos, a.rope_sin, a.rope_cos ? a.rope_end : 0, a.rope_hd, a.rope_S};
   static std::atomic<unsigned long long> attr_done{0};  // devices whose function attribute is set
   if (!done_on_device(attr_done)) {
     const cudaError_t err = cudaFuncSetAttribute(k_gemm<BN, AMN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -793,43 +723,10 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 
-// Tile width. The persistent grid runs ceil(tiles / SMs) rounds of tiles whose time grows with the
-// width, so the width with the smallest rounds x width (narrower widths weighted for their lower
-// efficiency per FLOP, and 3% of margin against 256) wins: a 2048 x 4096 output takes 1.7 rounds of 128 x 256 tiles (the second
-// one 73% full) but 2.8 rounds of 128 x 160 tiles. The 160 / 224 widths exist for the plain K-major
-// form (x W^T without rotary, NF4 or MN-major operands).
-int pick_bn(const GemmArgs& a) {
-  if (a.N <= 64) return 64;
-  if (a.N <= 128) return 128;
-  static const int kWide[] = {256, 224, 160, 128};
-  static const double kWeight[] = {1.0, 1.01, 1.03, 1.06};
-  const bool wide = !a.Bq && !a.a_mn && !a.b_mn && !a.rope_cos;
-  const int64_t mt = (a.M + BM - 1) / BM;
-  const int64_t sms = device_sm_count();
-  auto cost = [&](int i) {
-    const int w = kWide[i];
-    const int64_t tiles = mt * ((a.N + w - 1) / w);
-    return (double)((tiles + sms - 1) / sms) * w * kWeight[i];
-  };
-  // a narrower width has to win by 3% to replace the 256-wide tile
-  int bn = 256;
-  double best = 0.97 * cost(0);
-  for (int i = 1; i < 4; ++i) {
-    if (!wide && kWide[i] != 128) continue;
-    const double c = cost(i);
-    if (c < best) {
-      best = c;
-      bn = kWide[i];
-    }
-  }
-  return bn;
-}
-
 }  // namespace
 
 cudaError_t gemm_bf16(const GemmArgs& a, cudaStream_t s) {
-  if (a.M <= 0 || a.N <= 0 || a.K <= 0 || !a.A || (!a.B && !a.Bq) || (!a.C && !a.swiglu_gu))
-    return cudaErrorInvalidValue;
+  if (a.M <= 0 || a.N <= 0 || a.K <= 0 || !a.A || (!a.B && !a.Bq) || !a.C) return cudaErrorInvalidValue;
   // TMA: 16-byte aligned bases and row strides
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   if (!al16(a.A) || (a.lda % 8)) return cudaErrorInvalidValue;
@@ -846,13 +743,11 @@ cudaError_t gemm_bf16(const GemmArgs& a, cudaStream_t s) {
         return cudaErrorInvalidValue;
   }
   if (a.A2 && (!al16(a.A2) || !al16(a.B2) || (a.lda2 % 8) || (a.ldb2 % 8))) return cudaErrorInvalidValue;
-  if (a.swiglu_gu) {
-    // the SwiGLU backward replaces the store of C: no C, bias, residual or rotation; 16-byte rows
-    if (!a.swiglu_dgu || a.C || a.bias || a.R || a.rope_cos || (a.N % 8) ||
-        (reinterpret_cast<uintptr_t>(a.swiglu_gu) & 15) || (reinterpret_cast<uintptr_t>(a.swiglu_dgu) & 15))
-      return cudaErrorInvalidValue;
-  }
-  int bn = pick_bn(a);
+  const int64_t tiles256 = (int64_t)((a.M + BM - 1) / BM) * ((a.N + 255) / 256);
+  int bn;
+  if (a.N <= 64) bn = 64;
+  else if (a.N <= 128 || tiles256 < 120) bn = 128;
+  else bn = 256;
   if (a.rope_cos) {
     // rotated columns: whole tiles of whole heads, bf16 output, no residual / split / MN-major A
     if (!a.rope_sin || (a.rope_hd != 64 && a.rope_hd != 128) || a.rope_S <= 0 || a.c_f32 || a.R ||
@@ -879,8 +774,6 @@ cudaError_t gemm_bf16(const GemmArgs& a, cudaStream_t s) {
     case 128 * 4 + 0: return launch<128, 0, 0>(a, s);
     case 128 * 4 + 1: return launch<128, 0, 1>(a, s);
     case 128 * 4 + 3: return launch<128, 1, 1>(a, s);
-    case 160 * 4 + 0: return launch<160, 0, 0>(a, s);
-    case 224 * 4 + 0: return launch<224, 0, 0>(a, s);
     case 256 * 4 + 0: return launch<256, 0, 0>(a, s);
     case 256 * 4 + 1: return launch<256, 0, 1>(a, s);
     case 256 * 4 + 3: return launch<256, 1, 1>(a, s);

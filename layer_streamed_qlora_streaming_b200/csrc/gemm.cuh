@@ -63,13 +63,6 @@ struct GemmArgs {
   // values equal those of nf4_dequant bit for bit, so the result equals the GEMM on the
   // dequantised matrix byte for byte. Needs a_mn = 0 and W's row length (K or N) % 64 == 0.
   const Nf4Mat* Bq = nullptr;
-  // SwiGLU backward fused into the epilogue (the dX GEMM of the down projection, whose output is
-  // dL/dm, N = F): instead of C, element (t, j) of the fp32 accumulator d = alpha * acc (plus the
-  // LoRA term) gives, with g = gu[t][j], u = gu[t][F + j] (bf16 [M, 2F], row stride 2F) and
-  // s = 1 / (1 + exp(-g)): dgu[t][j] = bf16(d u s (1 + g (1 - s))), dgu[t][F + j] = bf16(d g s), the
-  // operations of swiglu_bwd in the same order. C, bias and R must be null.
-  const __nv_bfloat16* swiglu_gu = nullptr;
-  __nv_bfloat16* swiglu_dgu = nullptr;
 };
 
 // Returns cudaSuccess or the launch / argument error. Deterministic: no split-K, no atomics.

@@ -86,32 +86,6 @@ lst_status lst_k_gemm(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_
   return st(gemm_bf16(a, S(stream)));
 }
 
-lst_status lst_k_gemm_swiglu_bwd(int32_t M, int32_t F, int32_t K, const uint16_t* A, int64_t lda, const uint16_t* B,
-                                 int64_t ldb, int32_t b_mn, const uint16_t* A2, int64_t lda2, const uint16_t* B2,
-                                 int64_t ldb2, int32_t K2, float alpha, const uint16_t* gu, uint16_t* dgu,
-                                 void* stream) {
-  if (M <= 0 || F <= 0 || K <= 0 || !A || !B || !gu || !dgu || (F % 8)) return LST_ERR_ARG;
-  if ((A2 == nullptr) != (B2 == nullptr)) return LST_ERR_ARG;
-  GemmArgs a;
-  a.M = M;
-  a.N = F;
-  a.K = K;
-  a.A = B16(A);
-  a.lda = lda;
-  a.B = B16(B);
-  a.ldb = ldb;
-  a.b_mn = b_mn ? 1 : 0;
-  a.A2 = B16(A2);
-  a.lda2 = lda2;
-  a.B2 = B16(B2);
-  a.ldb2 = ldb2;
-  a.K2 = A2 ? K2 : 0;
-  a.alpha = alpha;
-  a.swiglu_gu = B16(gu);
-  a.swiglu_dgu = B16(dgu);
-  return st(gemm_bf16(a, S(stream)));
-}
-
 lst_status lst_k_gemm_nf4(int32_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda, const lst_nf4_part* parts,
                           int32_t nparts, int32_t b_mn, const uint16_t* A2, int64_t lda2, const uint16_t* B2,
                           int64_t ldb2, int32_t K2, void* C, int64_t ldc, int32_t c_f32, float alpha, const float* bias,

@@ -67,9 +67,8 @@ GEMM_CASES = [
     (256, 1536, 512, 1, True, True, False, False),      # MN-major with extension
     (2048, 6144, 4096, 0, True, False, False, False),   # fused q/k/v of an 8B layer
     (2048, 4096, 14336, 1, True, True, False, False),   # dX of the 8B down projection
-    (2048, 4096, 512, 0, True, True, False, True),      # o-like output: 128 x 160 tiles (2.8 rounds)
-    (2048, 28672, 256, 0, True, False, False, False),   # gate/up-like output: 128 x 224 tiles
-    (1024, 4000, 256, 0, False, True, True, False),     # 128 x 224 tiles, ragged last tile
+    (2048, 4096, 512, 0, True, True, False, True),      # o-like output with residual (1.7 rounds)
+    (1024, 4000, 256, 0, False, True, True, False),     # ragged last N-tile, bias
 ]
 
 
@@ -104,35 +103,6 @@ def test_gemm(M, N, K, b_mn, ext, f32, bias, resid):
     got = to_np(C)
     tol = 1e-4 if f32 else 8e-3
     assert maxrel(got, ref) < tol, maxrel(got, ref)
-
-
-@pytest.mark.parametrize("M,F,K,ext", [(300, 688, 256, True), (256, 1000, 128, False), (2048, 14336, 4096, True)])
-def test_gemm_swiglu_bwd_epilogue(M, F, K, ext):
-    # the down projection's dX GEMM with the SwiGLU backward in its epilogue against the fp32 GEMM
-    # followed by the SwiGLU backward kernel: the same fp32 operations on the same accumulator
-    r = _rng(M + F + K)
-    A = _bf(r.normal(size=(M, K)))
-    W = _bf(r.normal(size=(K, F)) * 0.05)                 # MN-major: dX = dY W
-    gu = _bf(r.normal(size=(M, 2 * F)))
-    kw = {}
-    if ext:
-        A2 = np.zeros((M, 64), np.float32)
-        A2[:, :48] = _bf(r.normal(size=(M, 48)))
-        B2 = np.zeros((64, F), np.float32)
-        B2[:48] = _bf(r.normal(size=(48, F)) * 0.1)
-        kw = dict(A2=torch_bf16(A2), lda2=64, B2=torch_bf16(B2), ldb2=F, K2=64)
-    dm = torch.zeros(M, F, dtype=torch.float32, device="cuda")
-    lst.k_gemm(M, F, K, torch_bf16(A), K, torch_bf16(W), F, 1, dm, F, 1, **kw)
-    ref = torch.empty(M, 2 * F, dtype=torch.bfloat16, device="cuda")
-    lst.k_swiglu_bwd(dm, torch_bf16(gu), M, F, ref)
-    got = torch.full((M, 2 * F), float("nan"), dtype=torch.bfloat16, device="cuda")
-    lst.k_gemm_swiglu_bwd(M, F, K, torch_bf16(A), K, torch_bf16(W), F, 1, torch_bf16(gu), got, **kw)
-    torch.cuda.synchronize()
-    a = got.view(torch.int16).cpu().numpy()
-    b = ref.view(torch.int16).cpu().numpy()
-    assert np.isfinite(to_np(got)).all()
-    assert (a == b).mean() > 0.999, (a == b).mean()      # the same value bits, up to fma contraction
-    assert maxrel(to_np(got), to_np(ref)) < 8e-3
 
 
 def _nf4_parts(rows_list, cols, seed):
