@@ -52,12 +52,12 @@ def describe(wl) -> str:
 # belong to the GEMM sources whose hashes are recorded with them; with other sources bench.py
 # reports the traffic as null. Commands and values: profiles/gemm_traffic_llama8b_shapes.md.
 GEMM_TRAFFIC = {"workload": "llama8b",
-                "bytes_per_launch": {"gemm_qkv": 75194624, "gemm_o": 92458752, "gemm_gu": 356543744,
-                                     "gemm_down": 298611968, "gemm_dx_down": 217623552, "gemm_dx_gu": 509555712,
-                                     "gemm_dx_o": 52230912, "gemm_dx_qkv": 92554496, "gemm_head": 2089809920,
-                                     "gemm_dx_head": 2349693184},
-                "sources": {"gemm.cu": "681b07e792c02958", "gemm.cuh": "bfa9880e2fabba28",
-                            "common.cuh": "704b7549d8511a32"}}
+                "bytes_per_launch": {"gemm_qkv": 74810624, "gemm_o": 92734208, "gemm_gu": 356411136,
+                                     "gemm_down": 298519808, "gemm_dx_down": 217685504, "gemm_dx_gu": 509340416,
+                                     "gemm_dx_o": 52140032, "gemm_dx_qkv": 92449536, "gemm_head": 2111525120,
+                                     "gemm_dx_head": 2577441536},
+                "sources": {"gemm.cu": "25fb8f9c5e07d9da", "gemm.cuh": "bfa9880e2fabba28",
+                            "common.cuh": "704b7549d8511a32", "pdl.cuh": "9d27364b6fccf4eb"}}
 
 
 def gemm_traffic(wl_name: str):

@@ -21,6 +21,9 @@ Cases are the shapes of the Llama-3.1-8B-shaped layer at batch 4 x seq 512 (T = 
                         launch, as a backward read issues them
   lora_grads_layer_sep  the same four groups as four launches
   ce           cross-entropy rows + dlogits over fp32 logits [2048, 128256]
+  rmsnorm_fwd / rmsnorm_bwd   RMSNorm of the fp32 residual stream [2048, 4096] (bf16 output; the
+               backward with the residual gradient added and a bf16 copy, as a layer uses it)
+  swiglu_fwd / swiglu_bwd     SwiGLU of gate/up [2048, 2 x 14336] (the backward from fp32 dL/dm)
 The LoRA cases rotate over enough input copies to exceed the 126 MB L2, so every launch reads
 its operands from HBM.
 Prints one JSON line with the per-launch device time (launches queued back to back) and the
@@ -38,6 +41,7 @@ import torch
 
 sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 from layer_streamed_qlora_streaming_b200 import (k_attention_bwd, k_attention_fwd, k_cross_entropy, k_gemm, k_gemm_nf4,
+                                                 k_rmsnorm_bwd, k_rmsnorm_fwd, k_swiglu_bwd, k_swiglu_fwd,
                                                  k_lora_grads, k_lora_grads_multi, k_lora_skinny, k_nf4_dequant,
                k_nf4_quantize)
 
@@ -167,6 +171,38 @@ def build(case: str):
         return run, {"flop": 2.5 * flop_fwd, "bytes": None}
     if case.startswith("lora_"):
         return _lora_case(case, g)
+    if case.startswith("rmsnorm"):
+        x = torch.randn(T, D, generator=g, device="cuda")
+        gam = torch.rand(D, generator=g, device="cuda") + 0.5
+        rstd = torch.empty(T, device="cuda")
+        if case == "rmsnorm_fwd":
+            y = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
+
+            def run():
+                k_rmsnorm_fwd(x, gam, T, D, 1e-5, y, rstd)
+            return run, {"flop": None, "bytes": T * D * (4 + 2)}
+        k_rmsnorm_fwd(x, gam, T, D, 1e-5, torch.empty(T, D, dtype=torch.bfloat16, device="cuda"), rstd)
+        dy, dres = torch.randn(T, D, generator=g, device="cuda"), torch.randn(T, D, generator=g, device="cuda")
+        dx = torch.empty(T, D, device="cuda")
+        dxb = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
+
+        def run():
+            k_rmsnorm_bwd(dy, x, gam, rstd, dres, T, D, dx, dxb)
+        return run, {"flop": None, "bytes": T * D * (4 * 4 + 2)}
+    if case.startswith("swiglu"):
+        gu = _bf((T, 2 * F), g)
+        if case == "swiglu_fwd":
+            m = torch.empty(T, F, dtype=torch.bfloat16, device="cuda")
+
+            def run():
+                k_swiglu_fwd(gu, T, F, m)
+            return run, {"flop": None, "bytes": T * F * (4 + 2)}
+        dm = torch.randn(T, F, generator=g, device="cuda")
+        dgu = torch.empty(T, 2 * F, dtype=torch.bfloat16, device="cuda")
+
+        def run():
+            k_swiglu_bwd(dm, gu, T, F, dgu)
+        return run, {"flop": None, "bytes": T * F * (4 + 4 + 4)}
     if case == "ce":
         V = 128256
         logits = torch.randn(T, V, generator=g, device="cuda") * 2.0

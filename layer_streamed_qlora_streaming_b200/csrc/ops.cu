@@ -39,30 +39,47 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 }
 
 // ------------------------------------------------------------------------------- RMSNorm
+// One CTA per row, the row held in registers: thread t owns the float4 columns t, t + blockDim,
+// ..., t + (kRnV - 1) blockDim (coalesced), so the row crosses HBM once and the normalisation
+// reads it from registers after the block reduction. blockDim = rn_threads(d).
+constexpr int kRnV = 8;  // float4 per thread: rows of up to 32 * blockDim elements
+__host__ __device__ inline int rn_threads(int d) {
+  const int n = (d / 4 + kRnV - 1) / kRnV;
+  return n <= 32 ? 32 : ((n + 31) / 32) * 32;
+}
+
 __global__ void k_rmsnorm_fwd(const float* __restrict__ x, const float* __restrict__ g, int d, float eps,
                               bf16* __restrict__ y, float* __restrict__ rstd) {
   pdl_wait();
   pdl_trigger();
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
-  const float* xr = x + row * d;
+  const int n4 = d / 4;
+  const float4* xr = reinterpret_cast<const float4*>(x + row * d);
+  float4 v[kRnV];
   float ss = 0.f;
-  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
-    const float4 u = *reinterpret_cast<const float4*>(xr + c);
-    ss += u.x * u.x;
-    ss += u.y * u.y;
-    ss += u.z * u.z;
-    ss += u.w * u.w;
+#pragma unroll
+  for (int i = 0; i < kRnV; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    v[i] = c < n4 ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    ss += v[i].x * v[i].x;
+    ss += v[i].y * v[i].y;
+    ss += v[i].z * v[i].z;
+    ss += v[i].w * v[i].w;
   }
   ss = block_sum(ss, red);
   const float r = 1.0f / sqrtf(ss / (float)d + eps);
   if (threadIdx.x == 0) rstd[row] = r;
-  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
-    const float4 u = *reinterpret_cast<const float4*>(xr + c);
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+#pragma unroll
+  for (int i = 0; i < kRnV; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    if (c >= n4) break;
+    const float4 gg = g4[c];
     __nv_bfloat162 o[2];
-    o[0] = __floats2bfloat162_rn(u.x * r * g[c], u.y * r * g[c + 1]);
-    o[1] = __floats2bfloat162_rn(u.z * r * g[c + 2], u.w * r * g[c + 3]);
-    *reinterpret_cast<uint2*>(y + row * d + c) = *reinterpret_cast<const uint2*>(o);
+    o[0] = __floats2bfloat162_rn(v[i].x * r * gg.x, v[i].y * r * gg.y);
+    o[1] = __floats2bfloat162_rn(v[i].z * r * gg.z, v[i].w * r * gg.w);
+    *reinterpret_cast<uint2*>(y + row * d + 4 * c) = *reinterpret_cast<const uint2*>(o);
   }
 }
 
@@ -74,34 +91,43 @@ __global__ void k_rmsnorm_bwd(const float* __restrict__ dy, const float* __restr
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
   const float r = rstd[row];
-  const float* dyr = dy + row * d;
-  const float* xr = x + row * d;
+  const int n4 = d / 4;
+  const float4* dyr = reinterpret_cast<const float4*>(dy + row * d);
+  const float4* xr = reinterpret_cast<const float4*>(x + row * d);
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  float4 a[kRnV], b[kRnV];
   float dot = 0.f;
-  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
-    const float4 a = *reinterpret_cast<const float4*>(dyr + c);
-    const float4 b = *reinterpret_cast<const float4*>(xr + c);
-    dot += a.x * g[c] * (b.x * r);
-    dot += a.y * g[c + 1] * (b.y * r);
-    dot += a.z * g[c + 2] * (b.z * r);
-    dot += a.w * g[c + 3] * (b.w * r);
+#pragma unroll
+  for (int i = 0; i < kRnV; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    const bool in = c < n4;
+    a[i] = in ? dyr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    b[i] = in ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 gg = in ? g4[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    dot += a[i].x * gg.x * (b[i].x * r);
+    dot += a[i].y * gg.y * (b[i].y * r);
+    dot += a[i].z * gg.z * (b[i].z * r);
+    dot += a[i].w * gg.w * (b[i].w * r);
   }
   dot = block_sum(dot, red) / (float)d;
-  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
-    const float4 a = *reinterpret_cast<const float4*>(dyr + c);
-    const float4 b = *reinterpret_cast<const float4*>(xr + c);
-    float v[4] = {r * (a.x * g[c] - b.x * r * dot), r * (a.y * g[c + 1] - b.y * r * dot),
-                  r * (a.z * g[c + 2] - b.z * r * dot), r * (a.w * g[c + 3] - b.w * r * dot)};
+#pragma unroll
+  for (int i = 0; i < kRnV; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    if (c >= n4) break;
+    const float4 gg = g4[c];
+    float v[4] = {r * (a[i].x * gg.x - b[i].x * r * dot), r * (a[i].y * gg.y - b[i].y * r * dot),
+                  r * (a[i].z * gg.z - b[i].z * r * dot), r * (a[i].w * gg.w - b[i].w * r * dot)};
     if (dres) {
-      const float4 q = *reinterpret_cast<const float4*>(dres + row * d + c);
+      const float4 q = reinterpret_cast<const float4*>(dres + row * d)[c];
       v[0] += q.x;
       v[1] += q.y;
       v[2] += q.z;
       v[3] += q.w;
     }
-    *reinterpret_cast<float4*>(dx + row * d + c) = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(dx + row * d)[c] = make_float4(v[0], v[1], v[2], v[3]);
     if (dxb) {
       __nv_bfloat162 h[2] = {__floats2bfloat162_rn(v[0], v[1]), __floats2bfloat162_rn(v[2], v[3])};
-      *reinterpret_cast<uint2*>(dxb + row * d + c) = *reinterpret_cast<const uint2*>(h);
+      *reinterpret_cast<uint2*>(dxb + row * d + 4 * c) = *reinterpret_cast<const uint2*>(h);
     }
   }
 }
@@ -143,6 +169,10 @@ __global__ void k_rope_tables(int S, int hd, double theta, float* ct, float* st)
 
 // ------------------------------------------------------------------------------- SwiGLU
 // 8 consecutive elements per thread (16-byte loads and stores); F is a multiple of 8.
+// sigmoid(g) = 1 / (1 + 2^(-g log2 e)) with the SFU's approximate exp2 (about 2 ulp) and a correctly
+// rounded reciprocal; the results are rounded to bf16.
+constexpr float kLog2e = 1.4426950408889634f;
+__device__ __forceinline__ float sigmoid_fast(float g) { return __frcp_rn(1.0f + ex2_approx(-g * kLog2e)); }
 __global__ void k_swiglu_fwd(const bf16* __restrict__ gu, int64_t T, int F, bf16* __restrict__ m) {
   pdl_wait();
   pdl_trigger();
@@ -163,7 +193,7 @@ __global__ void k_swiglu_fwd(const bf16* __restrict__ gu, int64_t T, int F, bf16
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const float g = __bfloat162float(g8[2 * e + k]), u = __bfloat162float(u8[2 * e + k]);
-      const float sg = 1.0f / (1.0f + expf(-g));
+      const float sg = sigmoid_fast(g);
       r[k] = g * sg * u;
     }
     o2[e] = __floats2bfloat162_rn(r[0], r[1]);
@@ -196,7 +226,7 @@ __global__ void k_swiglu_bwd(const float* __restrict__ dm, const bf16* __restric
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const float g = __bfloat162float(g8[2 * e + k]), u = __bfloat162float(u8[2 * e + k]);
-      const float sg = 1.0f / (1.0f + expf(-g));
+      const float sg = sigmoid_fast(g);
       const float d = dd[2 * e + k];
       rg[k] = d * u * sg * (1.0f + g * (1.0f - sg));
       ru[k] = d * g * sg;
@@ -314,7 +344,6 @@ k_ce(const float* __restrict__ logits, int V, const int32_t* __restrict__ y, flo
 // (the SFU's approximate exp2 on the product, formed with one fma). Needs V % 4 == 0 (16-byte
 // aligned slices).
 constexpr int kCeThreads = 256, kCeChunks = 4;
-constexpr float kLog2e = 1.4426950408889634f;
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(dst)),
@@ -592,15 +621,16 @@ inline unsigned nblk(int64_t n, int t = kThreads) { return (unsigned)((n + t - 1
 
 cudaError_t rmsnorm_fwd(const float* x, const float* g, int64_t T, int d, float eps, bf16* y, float* rstd,
                         cudaStream_t s) {
-  if (d % 8) return cudaErrorInvalidValue;
-  const cudaError_t e = launch_k(k_rmsnorm_fwd, dim3((unsigned)T), dim3(d >= 2048 ? 256 : 128), 0, s, 0, x, g, d, eps, y, rstd);
+  if (d % 8 || rn_threads(d) > 1024) return cudaErrorInvalidValue;
+  const cudaError_t e = launch_k(k_rmsnorm_fwd, dim3((unsigned)T), dim3(rn_threads(d)), 0, s, 0, x, g, d, eps, y, rstd);
   note_launch(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 cudaError_t rmsnorm_bwd(const float* dy, const float* x, const float* g, const float* rstd, const float* dres,
                         int64_t T, int d, float* dx, bf16* dxb, cudaStream_t s) {
-  if (d % 8) return cudaErrorInvalidValue;
-  const cudaError_t e = launch_k(k_rmsnorm_bwd, dim3((unsigned)T), dim3(256), 0, s, 0, dy, x, g, rstd, dres, d, dx, dxb);
+  if (d % 8 || rn_threads(d) > 1024) return cudaErrorInvalidValue;
+  const cudaError_t e = launch_k(k_rmsnorm_bwd, dim3((unsigned)T), dim3(rn_threads(d)), 0, s, 0, dy, x, g, rstd, dres,
+                                 d, dx, dxb);
   note_launch(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
