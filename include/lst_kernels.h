@@ -42,8 +42,7 @@ lst_status lst_k_nf4_quantize_noalloc(const float* w, int64_t n, uint8_t* packed
                                       float* gscale, float* mean, void* stream);
 
 /* Dequantise one NF4 tensor into bf16 [n]: a^ = (q * s) / 127 + mean, w^ = bf16(code * a^),
- * each operation one fp32 rounding; bit-exact by construction. n a multiple of 64; packed and out
- * 16-byte aligned (LST_ERR_ARG otherwise). */
+ * each operation one fp32 rounding; bit-exact by construction. */
 lst_status lst_k_nf4_dequant(const uint8_t* packed, const int8_t* qabs, const float* gscale,
                              const float* mean, int64_t n, uint16_t* out, void* stream);
 

@@ -155,16 +155,15 @@ struct DequantJob {
   Nf4Table tab;
 };
 
-// Each thread expands 32 codes (one 16-byte load, half an NF4 block) into 32 bf16 values (four
-// 16-byte stores); the two threads of a block form its absmax the same way.
+// Each thread expands 16 codes (8 packed bytes) into 16 bf16 values (two 16-byte stores).
 __global__ void __launch_bounds__(256) k_dequant(const DequantJob job, __nv_bfloat16* __restrict__ out) {
   pdl_wait();
   pdl_trigger();
   __shared__ float cb[16];
   if (threadIdx.x < 16) cb[threadIdx.x] = job.tab.cb[threadIdx.x];
   __syncthreads();
-  const int64_t chunk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // 32-element chunk index
-  int64_t e0 = chunk * 32;
+  const int64_t chunk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // 16-element chunk index
+  int64_t e0 = chunk * 16;
   int si = 0;
   int64_t base = 0;
   for (; si < job.nseg; ++si) {
@@ -175,24 +174,21 @@ __global__ void __launch_bounds__(256) k_dequant(const DequantJob job, __nv_bflo
   const Nf4Seg& sg = job.seg[si];
   const int64_t le = e0 - base;               // element index inside the tensor
   const int64_t blk = le >> 6;
-  const uint4 pk = *reinterpret_cast<const uint4*>(sg.packed + (le >> 1));
   const float qs = __fmul_rn((float)sg.qabs[blk], sg.gscale[blk >> 8]);
   const float ahat = __fadd_rn(__fdiv_rn(qs, 127.0f), *sg.mean);
+  const uint2 pk = *reinterpret_cast<const uint2*>(sg.packed + (le >> 1));
   const uint8_t* bytes = reinterpret_cast<const uint8_t*>(&pk);
-  uint4* dst = reinterpret_cast<uint4*>(out + sg.out_offset + le);
+  uint4 o[2];
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(o);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 o;
-    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint8_t by = bytes[q * 4 + i];
-      const float hi = __fmul_rn(cb[by >> 4], ahat);
-      const float lo = __fmul_rn(cb[by & 15], ahat);
-      h[i] = __halves2bfloat162(__float2bfloat16_rn(hi), __float2bfloat16_rn(lo));
-    }
-    dst[q] = o;
+  for (int i = 0; i < 8; ++i) {
+    const float hi = __fmul_rn(cb[bytes[i] >> 4], ahat);
+    const float lo = __fmul_rn(cb[bytes[i] & 15], ahat);
+    h[i] = __halves2bfloat162(__float2bfloat16_rn(hi), __float2bfloat16_rn(lo));
   }
+  uint4* dst = reinterpret_cast<uint4*>(out + sg.out_offset + le);
+  dst[0] = o[0];
+  dst[1] = o[1];
 }
 
 }  // namespace
@@ -203,15 +199,12 @@ cudaError_t nf4_dequant(const Nf4Seg* segs, int nseg, __nv_bfloat16* out, cudaSt
   int64_t total = 0;
   for (int i = 0; i < nseg; ++i) {
     job.seg[i] = segs[i];
-    // whole blocks; 16-byte loads of the codes and 16-byte stores of the values
-    if (segs[i].n % 64 || (reinterpret_cast<uintptr_t>(segs[i].packed) & 15) ||
-        (reinterpret_cast<uintptr_t>(out + segs[i].out_offset) & 15))
-      return cudaErrorInvalidValue;
+    if (segs[i].n % 64) return cudaErrorInvalidValue;
     total += segs[i].n;
   }
   job.nseg = nseg;
   job.tab = nf4_table();
-  const int64_t chunks = total / 32;
+  const int64_t chunks = total / 16;
   const cudaError_t e = launch_k(k_dequant, dim3((unsigned)((chunks + 255) / 256)), dim3(256), 0, s, 0, job, out);
   note_launch(1);
   return e != cudaSuccess ? e : cudaGetLastError();

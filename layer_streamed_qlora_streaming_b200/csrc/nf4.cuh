@@ -40,8 +40,7 @@ struct Nf4Seg {
 };
 constexpr int kMaxNf4Segs = 8;
 
-// Dequantise up to 8 tensors into one bf16 buffer (each at its out_offset). Each tensor's packed codes
-// and its place in out must be 16-byte aligned, and its length a multiple of 64.
+// Dequantise up to 8 tensors into one bf16 buffer (each at its out_offset).
 cudaError_t nf4_dequant(const Nf4Seg* segs, int nseg, __nv_bfloat16* out, cudaStream_t s);
 
 }  // namespace lst

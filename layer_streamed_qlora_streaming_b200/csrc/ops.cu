@@ -39,9 +39,10 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 }
 
 // ------------------------------------------------------------------------------- RMSNorm
-// One CTA per row, the row held in registers: thread t owns the float4 columns t, t + blockDim,
-// ..., t + (kRnV - 1) blockDim (coalesced), so the row crosses HBM once and the normalisation
-// reads it from registers after the block reduction. blockDim = rn_threads(d).
+// Forward: one CTA per row, the row held in registers: thread t owns the float4 columns t,
+// t + blockDim, ..., t + (kRnV - 1) blockDim (coalesced), so the row crosses HBM once and the
+// normalisation reads it from registers after the block reduction; blockDim = rn_threads(d).
+// Backward: one CTA of 256 threads per row, two passes over dy and x (the second from cache).
 constexpr int kRnV = 8;  // float4 per thread: rows of up to 32 * blockDim elements
 __host__ __device__ inline int rn_threads(int d) {
   const int n = (d / 4 + kRnV - 1) / kRnV;
@@ -91,43 +92,34 @@ __global__ void k_rmsnorm_bwd(const float* __restrict__ dy, const float* __restr
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
   const float r = rstd[row];
-  const int n4 = d / 4;
-  const float4* dyr = reinterpret_cast<const float4*>(dy + row * d);
-  const float4* xr = reinterpret_cast<const float4*>(x + row * d);
-  const float4* g4 = reinterpret_cast<const float4*>(g);
-  float4 a[kRnV], b[kRnV];
+  const float* dyr = dy + row * d;
+  const float* xr = x + row * d;
   float dot = 0.f;
-#pragma unroll
-  for (int i = 0; i < kRnV; ++i) {
-    const int c = threadIdx.x + i * blockDim.x;
-    const bool in = c < n4;
-    a[i] = in ? dyr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
-    b[i] = in ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 gg = in ? g4[c] : make_float4(0.f, 0.f, 0.f, 0.f);
-    dot += a[i].x * gg.x * (b[i].x * r);
-    dot += a[i].y * gg.y * (b[i].y * r);
-    dot += a[i].z * gg.z * (b[i].z * r);
-    dot += a[i].w * gg.w * (b[i].w * r);
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    const float4 a = *reinterpret_cast<const float4*>(dyr + c);
+    const float4 b = *reinterpret_cast<const float4*>(xr + c);
+    dot += a.x * g[c] * (b.x * r);
+    dot += a.y * g[c + 1] * (b.y * r);
+    dot += a.z * g[c + 2] * (b.z * r);
+    dot += a.w * g[c + 3] * (b.w * r);
   }
   dot = block_sum(dot, red) / (float)d;
-#pragma unroll
-  for (int i = 0; i < kRnV; ++i) {
-    const int c = threadIdx.x + i * blockDim.x;
-    if (c >= n4) break;
-    const float4 gg = g4[c];
-    float v[4] = {r * (a[i].x * gg.x - b[i].x * r * dot), r * (a[i].y * gg.y - b[i].y * r * dot),
-                  r * (a[i].z * gg.z - b[i].z * r * dot), r * (a[i].w * gg.w - b[i].w * r * dot)};
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    const float4 a = *reinterpret_cast<const float4*>(dyr + c);
+    const float4 b = *reinterpret_cast<const float4*>(xr + c);
+    float v[4] = {r * (a.x * g[c] - b.x * r * dot), r * (a.y * g[c + 1] - b.y * r * dot),
+                  r * (a.z * g[c + 2] - b.z * r * dot), r * (a.w * g[c + 3] - b.w * r * dot)};
     if (dres) {
-      const float4 q = reinterpret_cast<const float4*>(dres + row * d)[c];
+      const float4 q = *reinterpret_cast<const float4*>(dres + row * d + c);
       v[0] += q.x;
       v[1] += q.y;
       v[2] += q.z;
       v[3] += q.w;
     }
-    reinterpret_cast<float4*>(dx + row * d)[c] = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(dx + row * d + c) = make_float4(v[0], v[1], v[2], v[3]);
     if (dxb) {
       __nv_bfloat162 h[2] = {__floats2bfloat162_rn(v[0], v[1]), __floats2bfloat162_rn(v[2], v[3])};
-      *reinterpret_cast<uint2*>(dxb + row * d + 4 * c) = *reinterpret_cast<const uint2*>(h);
+      *reinterpret_cast<uint2*>(dxb + row * d + c) = *reinterpret_cast<const uint2*>(h);
     }
   }
 }
@@ -628,9 +620,8 @@ cudaError_t rmsnorm_fwd(const float* x, const float* g, int64_t T, int d, float 
 }
 cudaError_t rmsnorm_bwd(const float* dy, const float* x, const float* g, const float* rstd, const float* dres,
                         int64_t T, int d, float* dx, bf16* dxb, cudaStream_t s) {
-  if (d % 8 || rn_threads(d) > 1024) return cudaErrorInvalidValue;
-  const cudaError_t e = launch_k(k_rmsnorm_bwd, dim3((unsigned)T), dim3(rn_threads(d)), 0, s, 0, dy, x, g, rstd, dres,
-                                 d, dx, dxb);
+  if (d % 8) return cudaErrorInvalidValue;
+  const cudaError_t e = launch_k(k_rmsnorm_bwd, dim3((unsigned)T), dim3(256), 0, s, 0, dy, x, g, rstd, dres, d, dx, dxb);
   note_launch(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
