@@ -19,7 +19,7 @@ EXACT_LOGITS_MAXREL = 3e-2
 # (q dA) and 2.66% (k dA) max-rel from its exact mode -- the rounding of layer 0's forward
 # activations moves the top layer's q/k adapter gradients that much. No bf16-activation
 # computation can be held closer to exact arithmetic than that, so the exact-oracle bound is 3e-2
-# (cosine unchanged); the benchmark spec's 2e-2 applies against the bf16-activation oracle.
+# (cosine unchanged); the parity bound of 2e-2 applies against the bf16-activation oracle.
 EXACT_GRAD_MAXREL = 3e-2
 
 
