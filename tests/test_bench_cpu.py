@@ -56,3 +56,16 @@ def test_gemm_traffic_only_for_the_captured_sources(monkeypatch):
     assert bench.gemm_traffic("qwen3b_bf16") == (None, None)        # another workload
     rec2["sources"]["gemm.cu"] = "0" * 16
     assert bench.gemm_traffic("llama8b") == (None, None)            # sources changed since
+
+
+def test_recorded_gemm_traffic_covers_the_gemm_sources():
+    # the recorded per-shape traffic belongs to the sources in this tree (so the bench line carries
+    # it), and its hash gate covers gemm.cu and every local header gemm.cu includes
+    import os
+    import re
+    per_launch, per_step = bench.gemm_traffic("llama8b")
+    assert per_launch is not None and per_step > 0
+    csrc = os.path.join(bench.ROOT, "layer_streamed_qlora_streaming_b200", "csrc")
+    src = open(os.path.join(csrc, "gemm.cu")).read()
+    local = set(re.findall(r'#include "([^"]+)"', src))
+    assert local <= set(bench.GEMM_TRAFFIC["sources"]), local - set(bench.GEMM_TRAFFIC["sources"])
