@@ -69,3 +69,25 @@ def test_recorded_gemm_traffic_covers_the_gemm_sources():
     src = open(os.path.join(csrc, "gemm.cu")).read()
     local = set(re.findall(r'#include "([^"]+)"', src))
     assert local <= set(bench.GEMM_TRAFFIC["sources"]), local - set(bench.GEMM_TRAFFIC["sources"])
+
+
+def test_reference_arm_prints_the_contract_line():
+    # `bench.py --impl reference` times the oracle on the host cores and prints one JSON line with
+    # the main line's metric and unit, impl "reference", its cpu_baseline and a zero-copy e2e
+    import json
+    import os
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "1", "--warmup", "0", "--ref-seq", "16"],
+                         capture_output=True, text=True, timeout=600, cwd=bench.ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["steps"] == 1 and d["warmup"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["extrapolated"] is True and d["sample_shape"]["seq"] == 16
