@@ -1083,6 +1083,16 @@ void plan_reads(lst_ctx* c) {
   c->plan_wheld[1] = wheld[1];
 }
 
+// LST_COPY_WHOLE=1 copies each blob with one cudaMemcpyAsync instead of one per weight group (for
+// measuring what the group copies cost; the compute of a read then starts only once all of it landed).
+bool whole_blob_copies() {
+  static const bool v = [] {
+    const char* e = std::getenv("LST_COPY_WHOLE");
+    return e && std::strcmp(e, "1") == 0;
+  }();
+  return v;
+}
+
 // Copy layer j's blob from the pinned arena into pool slot `slot` on the copy stream. chunk_ev
 // (NCHUNK events, or null) is recorded after each weight group has landed; *bytes is what crossed
 // this rank's link.
@@ -1102,6 +1112,13 @@ lst_status copy_layer(lst_ctx* c, int slot, int j, cudaEvent_t* chunk_ev, int64_
     if (chunk_ev)
       for (int g = 0; g < NCHUNK; ++g) CK(cudaEventRecord(chunk_ev[g], c->copy_stream));
     *bytes_out = bytes;
+    return LST_OK;
+  }
+  if (whole_blob_copies()) {  // one copy per read; every group's event after it
+    CK(cudaMemcpyAsync(c->pool[slot], src, c->lay.total, cudaMemcpyHostToDevice, c->copy_stream));
+    if (chunk_ev)
+      for (int g = 0; g < NCHUNK; ++g) CK(cudaEventRecord(chunk_ev[g], c->copy_stream));
+    *bytes_out = c->lay.total;
     return LST_OK;
   }
   for (int g = 0; g < NCHUNK; ++g) {  // group by group, so compute can start on the first group
